@@ -1,0 +1,469 @@
+#!/usr/bin/env python
+"""Benchmark of the Lizard hybrid attention layer on B200.
+
+One step = one training pass of the layer (forward + backward through
+lizard_attn_fwd / lizard_attn_bwd) over the B=8, H=32, L=2048, d=128 bf16
+batch (window 128, 4 meta tokens, chunk 64).  The same run times 1000
+consecutive single-token decode steps (B=64, H=32, d=128) and reports their
+HBM bandwidth in the same JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU: one process per GPU (torchrun); every rank processes its own batch
+(independent replicas, no collective on the data path: weak scaling); the
+step time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "hybrid attn fwd+bwd tokens/s & TFLOP/s (% bf16 peak); decode GB/s (% HBM)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+SM_COUNT = 148
+FP32_LANES_PER_SM = 128
+
+
+# ------------------------------------------------------------ counting ----
+def flops_per_token_head(d, C, w, M):
+    """Algorithmic FLOPs per (token, head), causal half of the intra tiles,
+    feature map excluded: GLA fwd (C+1)(dk+dv) + 4 dk dv, anchor fwd
+    2 (dk+dv)(w+M); a training step counts 3x GLA and 3.5x anchor."""
+    gla = (C + 1) * (2 * d) + 4 * d * d
+    swa = 2 * (2 * d) * (w + M)
+    return {"fwd": gla + swa, "train": 3 * gla + 3.5 * swa, "gla_fwd": gla, "swa_fwd": swa}
+
+
+def bytes_per_token_head(d, esz=2):
+    """Minimal HBM bytes per (token, head): forward reads q, k, v, g and
+    writes o; the training step adds dout in, dq, dk, dv out (activation
+    dtype) and dg out (fp32), and reads q, k, v, g again."""
+    fwd = 4 * d * esz + d * esz
+    bwd = 5 * d * esz + 3 * d * esz + d * 4
+    return {"fwd": fwd, "bwd": bwd, "train": fwd + bwd}
+
+
+def kernel_model(name, w, N, BH):
+    """(algorithmic bytes, algorithmic flops) of one launch of a kernel of the
+    library over N token-heads (BH sequences).  Workspace arrays are fp32."""
+    d, esz = w.d, 2 if w.dtype == "bf16" else 4
+    Nd = N * d
+    fl = flops_per_token_head(d, w.chunk, w.window, w.M)
+    phi = 2 * d * d   # two feature maps: x W for q and k, d x d/2 each
+    nch32 = math.ceil(w.L / 32)
+    table = {
+        # portable kernels
+        "prep_kernel": (3 * Nd * esz + 3 * Nd * 4, N * phi),
+        "gla_fwd_simt": (3 * Nd * 4 + Nd * esz + Nd * 4, N * fl["gla_fwd"]),
+        "swa_mix_simt": (3 * Nd * esz + Nd * 4 + Nd * esz, N * fl["swa_fwd"]),
+        "gla_states_simt": (2 * Nd * 4 + Nd * esz + BH * nch32 * d * d * 4, N * 2 * d * d),
+        "gla_bwd_simt": (3 * Nd * 4 + 2 * Nd * esz + BH * nch32 * d * d * 4 + 4 * Nd * 4,
+                         N * 2 * fl["gla_fwd"]),
+        "swa_bwd_q": (4 * Nd * esz + Nd * 4 + 2 * N * 4, N * 1.5 * fl["swa_fwd"]),
+        "swa_bwd_kv": (4 * Nd * esz + 2 * N * 4 + 2 * Nd * 4, N * 1.0 * fl["swa_fwd"]),
+        "finish_bwd": (3 * Nd * esz + 7 * Nd * 4 + 3 * Nd * esz + Nd * 4, N * 2 * phi),
+    }
+    return table.get(name, (0, 0))
+
+
+# ------------------------------------------------------------- clocks -----
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.path = None
+        try:
+            self.uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+        except Exception:
+            self.uuid = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            if self.uuid and self.uuid not in parts[1] and parts[1] not in self.uuid:
+                continue
+            rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        mx = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# -------------------------------------------------------------- helpers ----
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    d = dict(FALLBACK_PEAKS)
+    d["source"] = "fallback"
+    return d
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def max_over_ranks(x, world, device):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------ our arm -----
+def run_ours(args, rank, world, local):
+    from gated_linear_sliding_chunkwise_b200 import lizard as lz
+    from gated_linear_sliding_chunkwise_b200.synth import WORKLOADS, make_inputs
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    impl = {"auto": lz.IMPL_AUTO, "simt": lz.IMPL_SIMT, "tc": lz.IMPL_TC}[args.kernels]
+    w = WORKLOADS["train_step"]
+    inp = make_inputs(w, seed=w.seed + rank)
+    x = {k: v.to(dev).contiguous() for k, v in inp.items()}
+    kw = dict(window=w.window, chunk=w.chunk, gate_temp=w.gate_temp, fmap_wq=x["fmap_wq"],
+              fmap_wk=x["fmap_wk"], meta_k=x["meta_k"], meta_v=x["meta_v"], alpha=x["alpha"],
+              impl=impl)
+    fwd_names = lz.attn_fwd(x["q"], x["k"], x["v"], x["g"], plan_only=True, **kw)
+    bwd_names = lz.attn_bwd(x["q"], x["k"], x["v"], x["g"], x["dout"], plan_only=True, **kw)
+    # persistent outputs/workspaces so the timed loop allocates nothing
+    o = torch.empty_like(x["q"])
+    r0 = lz.attn_fwd(x["q"], x["k"], x["v"], x["g"], out=o, **kw)
+    fws = r0["workspace"]
+    g0 = lz.attn_bwd(x["q"], x["k"], x["v"], x["g"], x["dout"], **kw)
+    bws = g0["workspace"]
+    del g0
+    torch.cuda.synchronize()
+
+    def step(evf=None, evb=None):
+        lz.attn_fwd(x["q"], x["k"], x["v"], x["g"], out=o, workspace=fws, events=evf, **kw)
+        return lz.attn_bwd(x["q"], x["k"], x["v"], x["g"], x["dout"], workspace=bws,
+                           events=evb, **kw)
+
+    for _ in range(args.warmup):
+        step()
+    K = args.steps
+    evf = [lz.make_events(len(fwd_names) + 1) for _ in range(K)]
+    evb = [lz.make_events(len(bwd_names) + 1) for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    start.record()
+    for i in range(K):
+        step(evf[i], evb[i])
+    end.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier(world)
+    ms = start.elapsed_time(end) / K
+    ms_max = max_over_ranks(ms, world, dev)
+
+    N = w.B * w.H * w.L
+    BH = w.B * w.H
+    tokens = w.B * w.L
+    fl = flops_per_token_head(w.d, w.chunk, w.window, w.M)
+    by = bytes_per_token_head(w.d)
+    value = world * tokens / (ms_max / 1e3)
+    tflops = world * N * fl["train"] / (ms_max / 1e3) / 1e12
+    peaks = load_peaks()
+
+    # per-kernel device times from the library's launch events
+    per = {}
+    for names, evs in ((fwd_names, evf), (bwd_names, evb)):
+        for j, n in enumerate(names):
+            t = statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
+            per[n] = per.get(n, 0.0) + t
+    dom = max(per, key=per.get)
+    dbytes, dflops = kernel_model(dom, w, N, BH)
+    dt = per[dom] / 1e3
+    ai = dflops / max(dbytes, 1)
+    if dom.endswith("_simt") or dom in ("prep_kernel", "swa_bwd_q", "swa_bwd_kv", "finish_bwd"):
+        # CUDA-core kernels: fp32 FMA peak from unit counts and clock
+        alu_peak = SM_COUNT * FP32_LANES_PER_SM * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+        ridge = alu_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
+        if ai >= ridge:
+            roof = {"bound": "alu", "achieved": dflops / dt / 1e12, "peak": alu_peak,
+                    "unit": "TFLOP/s"}
+        else:
+            roof = {"bound": "hbm", "achieved": dbytes / dt / 1e9, "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s"}
+    else:
+        ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+        if ai >= ridge:
+            roof = {"bound": "tensor", "achieved": dflops / dt / 1e12,
+                    "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+        else:
+            roof = {"bound": "hbm", "achieved": dbytes / dt / 1e9, "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["kernel"] = dom
+    roof["ms_per_launch"] = per[dom]
+    roof["peak_source"] = peaks["source"]
+    kernels = {n: round(t, 4) for n, t in per.items()}
+
+    # end to end: pinned host inputs in, gradients out, every step
+    e2e = None
+    if not args.no_e2e:
+        hin = {n: x[n].cpu().pin_memory() for n in ("q", "k", "v", "g", "dout")}
+        hout = {n: torch.empty(x["q"].shape,
+                               dtype=torch.float32 if n == "dg" else x["q"].dtype).pin_memory()
+                for n in ("dq", "dk", "dv", "dg")}
+        h2d = sum(t.numel() * t.element_size() for t in hin.values())
+        d2h = sum(t.numel() * t.element_size() for t in hout.values())
+        Ke = max(1, min(K, 5))
+
+        def e2e_step():
+            for n, t in hin.items():
+                x[n].copy_(t, non_blocking=True)
+            gr = step()
+            for n, t in hout.items():
+                t.copy_(gr[n], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record()
+        for _ in range(Ke):
+            e2e_step()
+        e2.record()
+        torch.cuda.synchronize()
+        ems = max_over_ranks(s2.elapsed_time(e2) / Ke, world, dev)
+        e2e = {"value": world * tokens / (ems / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ems}
+
+    decode = None if args.no_decode else run_decode(args, lz, dev, rank, world, peaks)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1)/8 q,k,v; N(0,1) gate logits and dout)",
+        "config": {"workload": "train_step: lizard_attn_fwd + lizard_attn_bwd",
+                   "B": w.B, "H": w.H, "L": w.L, "d": w.d, "chunk": w.chunk,
+                   "window": w.window, "M": w.M, "global_batch": w.B * world,
+                   "seq_len": w.L, "parallelism": f"dp{world} (independent replicas)",
+                   "kernels": args.kernels,
+                   "l2": "inputs larger than L2 (q,k,v,g,dout = 5 x 134 MB per step)"},
+        "tflops": tflops, "tflops_frac_of_bf16_peak": tflops / peaks["bf16_tflops"],
+        "hbm_floor_ms": (N * by["train"]) / (peaks["hbm_gbs"] * 1e9) * 1e3,
+        "roofline": roof, "kernel_ms": kernels,
+        "gpu_launches": K * (len(fwd_names) + len(bwd_names)),
+        "clocks": clk, "e2e": e2e, "decode": decode,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(inp, w, budget_s=args.cpu_budget)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_decode(args, lz, dev, rank, world, peaks):
+    from gated_linear_sliding_chunkwise_b200.synth import WORKLOADS, make_inputs
+
+    w = WORKLOADS["decode_b64"]
+    inp = make_inputs(w, seed=w.seed + rank)
+    x = {k: v.to(dev).contiguous() for k, v in inp.items()}
+    o = torch.empty(w.B, w.H, w.d, dtype=x["q"].dtype, device=dev)
+
+    def st():
+        lz.decode_step(x["q"], x["k"], x["v"], x["g"], x["state"], x["k_cache"], x["v_cache"],
+                       x["pos"], gate_temp=w.gate_temp, fmap_wq=x["fmap_wq"],
+                       fmap_wk=x["fmap_wk"], meta_k=x["meta_k"], meta_v=x["meta_v"],
+                       alpha=x["alpha"], out=o)
+
+    for _ in range(10):
+        st()
+    n = args.decode_steps
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    s.record()
+    for _ in range(n):
+        st()
+    e.record()
+    torch.cuda.synchronize()
+    us = max_over_ranks(s.elapsed_time(e) * 1e3 / n, world, dev)
+    d, W, esz = w.d, w.window, 2
+    per_bh = 2 * d * d * 4 + 2 * W * d * esz + 4 * d * esz + 2 * d * esz + d * esz
+    step_bytes = w.B * w.H * per_bh + w.H * 2 * d * (d // 2) * 4
+    gbs = world * step_bytes / (us * 1e-6) / 1e9
+    return {"value": gbs, "unit": "GB/s", "frac_of_hbm": gbs / (world * peaks["hbm_gbs"]),
+            "us_per_step": us, "steps": n, "bytes_per_step": step_bytes,
+            "workload": "decode_b64: B=64 H=32 d=128 window 128 M=4, pos 65536",
+            "launches_per_step": 2}
+
+
+# ---------------------------------------------------------- CPU oracle ----
+def cpu_baseline(inp, w, budget_s=15.0, pairs=None):
+    """Time the fp64 oracle's forward + backward on whole sampled sequences
+    of the same workload, on this host; report layer tokens/s."""
+    import numpy as np
+    from oracle import lizard_ref as ref
+
+    pairs = pairs or [(0, 0), (1, 1), (2, 2), (3, 3), (4, 4), (5, 5), (6, 6), (7, 7)]
+    done = 0
+    t0 = time.perf_counter()
+    for (b, h) in pairs:
+        f = {k: inp[k][b:b + 1, h:h + 1].double().numpy() for k in ("q", "k", "v", "g", "dout")}
+        p = {k: inp[k][h:h + 1].double().numpy() for k in ("fmap_wq", "fmap_wk", "meta_k", "meta_v", "alpha")}
+        kw = dict(window=w.window, tau=w.gate_temp, **p)
+        ref.lizard_forward(f["q"], f["k"], f["v"], f["g"], **kw)
+        ref.lizard_backward(f["q"], f["k"], f["v"], f["g"], f["dout"], **kw)
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    token_heads = done * w.L
+    return {"value": token_heads / w.H / dt, "unit": "tokens/s", "cores": 1,
+            "host_cores_available": len(os.sched_getaffinity(0)), "kind": "oracle",
+            "sample": f"{done} whole (batch, head) sequences of L={w.L} (fp64 NumPy "
+                      f"forward + backward), {dt:.1f} s; tokens/s counts a token of all "
+                      f"H={w.H} heads, i.e. token-heads / {w.H}"}
+
+
+# ------------------------------------------------------ reference arm -----
+def run_reference(args, rank, world):
+    """The oracle as it stands, timed on the host cores over bounded samples
+    of the same workload (rank 0 only)."""
+    if rank != 0:
+        return
+    from gated_linear_sliding_chunkwise_b200.synth import WORKLOADS, make_inputs
+    from oracle import lizard_ref as ref
+
+    w = WORKLOADS["train_step"]
+    inp = make_inputs(w, B=1, H=1)            # one whole sequence per step
+    L = 256                                   # bounded sample: the first 256 tokens
+    f = {k: inp[k][:, :, :L].double().numpy() for k in ("q", "k", "v", "g", "dout")}
+    p = {k: inp[k].double().numpy() for k in ("fmap_wq", "fmap_wk", "meta_k", "meta_v", "alpha")}
+    kw = dict(window=w.window, tau=w.gate_temp, **p)
+
+    def step():
+        ref.lizard_forward(f["q"], f["k"], f["v"], f["g"], **kw)
+        ref.lizard_backward(f["q"], f["k"], f["v"], f["g"], f["dout"], **kw)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    value = L / w.H / dt
+    sample = (f"one (batch, head) sequence, first {L} tokens of the train_step workload, "
+              f"fp64 NumPy forward + backward per step; tokens/s counts a token of all "
+              f"H={w.H} heads")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "train_step (oracle sample)", "B": w.B, "H": w.H,
+                       "L": w.L, "d": w.d, "chunk": w.chunk, "window": w.window, "M": w.M},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--kernels", choices=["auto", "simt", "tc"], default="auto",
+                    help="kernel family inside the library")
+    ap.add_argument("--decode-steps", type=int, default=1000)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        print("note: --warmup below 3 is not a valid measurement", file=sys.stderr)
+    rank, world, local = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

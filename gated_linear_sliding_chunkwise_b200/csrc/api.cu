@@ -1,0 +1,376 @@
+// Host side of the C ABI declared in include/lizard.h: argument checks,
+// workspace layout and kernel dispatch.  Nothing here allocates device
+// memory; every buffer comes from the caller.
+#include <math.h>
+#include <string.h>
+
+#include <functional>
+
+#include "../../include/lizard.h"
+#include "lizard_internal.h"
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr size_t kHeader = 256;   // status word region at the workspace start
+
+size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool ok_ptr(const void *p) { return p == nullptr || aligned16(p); }
+
+lizard_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LIZARD_OK : LIZARD_ERR_CUDA; }
+
+// Shape and pointer checks shared by the forward and the backward.
+lizard_status check_fwd(const lizard_fwd_args *a) {
+  if (!a) return LIZARD_ERR_INVALID_ARG;
+  if (a->B < 0 || a->H < 0 || a->L < 0 || a->dk <= 0 || a->dv <= 0 || a->M < 0 || a->window < 1)
+    return LIZARD_ERR_INVALID_ARG;
+  if (a->B == 0 || a->H == 0) return LIZARD_ERR_INVALID_ARG;
+  if (a->dtype != LIZARD_BF16 && a->dtype != LIZARD_FP32) return LIZARD_ERR_INVALID_ARG;
+  if (a->branch < LIZARD_BRANCH_BOTH || a->branch > LIZARD_BRANCH_SWA_ONLY) return LIZARD_ERR_INVALID_ARG;
+  if (a->impl < LIZARD_IMPL_AUTO || a->impl > LIZARD_IMPL_TC) return LIZARD_ERR_INVALID_ARG;
+  if (!(a->gate_temp > 0.f) || !isfinite(a->gate_temp)) return LIZARD_ERR_INVALID_ARG;
+  if (!(a->softmax_scale >= 0.f) || !isfinite(a->softmax_scale)) return LIZARD_ERR_INVALID_ARG;
+  if (a->dk != a->dv || (a->dk != 64 && a->dk != 128)) return LIZARD_ERR_UNSUPPORTED;
+  if (a->chunk != 64) return LIZARD_ERR_UNSUPPORTED;
+  if (a->M > 16) return LIZARD_ERR_UNSUPPORTED;
+  if ((a->M > 0) != (a->meta_k != nullptr)) return LIZARD_ERR_INVALID_ARG;
+  if (a->meta_v && !a->meta_k) return LIZARD_ERR_INVALID_ARG;
+  if (a->L > 0) {
+    if (!a->q || !a->k || !a->v || !a->o) return LIZARD_ERR_INVALID_ARG;
+    if (a->branch != LIZARD_BRANCH_SWA_ONLY && !a->g) return LIZARD_ERR_INVALID_ARG;
+  }
+  const void *ptrs[] = {a->q, a->k, a->v, a->g, a->fmap_wq, a->fmap_wk, a->meta_k, a->meta_v,
+                        a->alpha, a->state_in, a->o, a->state_out, a->lse, a->workspace};
+  for (const void *p : ptrs)
+    if (!ok_ptr(p)) return LIZARD_ERR_INVALID_ARG;
+  return LIZARD_OK;
+}
+
+bool gla_on(const lizard_fwd_args *a) { return a->branch != LIZARD_BRANCH_SWA_ONLY; }
+bool swa_on(const lizard_fwd_args *a) { return a->branch != LIZARD_BRANCH_GLA_ONLY; }
+
+// Forward workspace (portable path).
+struct FwdLayout {
+  size_t phq, phk, a, o_gla, total;
+};
+FwdLayout fwd_layout(const lizard_fwd_args *a) {
+  const size_t N = (size_t)a->B * a->H * a->L;
+  const size_t nd = up(N * a->dk * sizeof(float));
+  FwdLayout l{};
+  size_t off = kHeader;
+  if (gla_on(a)) {
+    l.phq = off; off += nd;
+    l.phk = off; off += nd;
+    l.a = off; off += nd;
+    l.o_gla = off; off += up(N * a->dv * sizeof(float));
+  }
+  l.total = off;
+  return l;
+}
+
+struct BwdLayout {
+  size_t phq, phk, a, sprev, dphq, dphk, da, dv_gla, dq_swa, dk_swa, dv_swa, lse, Dterm, total;
+};
+BwdLayout bwd_layout(const lizard_fwd_args *a) {
+  const size_t BH = (size_t)a->B * a->H;
+  const size_t N = BH * a->L;
+  const size_t nd = up(N * a->dk * sizeof(float));
+  const size_t nv = up(N * a->dv * sizeof(float));
+  const size_t nch = (a->L + lz::kBwdC - 1) / lz::kBwdC;
+  BwdLayout l{};
+  size_t off = kHeader;
+  if (gla_on(a)) {
+    l.phq = off; off += nd;
+    l.phk = off; off += nd;
+    l.a = off; off += nd;
+    l.sprev = off; off += up(BH * nch * a->dk * a->dv * sizeof(float));
+    l.dphq = off; off += nd;
+    l.dphk = off; off += nd;
+    l.da = off; off += nd;
+    l.dv_gla = off; off += nv;
+  }
+  if (swa_on(a)) {
+    l.dq_swa = off; off += nd;
+    l.dk_swa = off; off += nd;
+    l.dv_swa = off; off += nv;
+    l.lse = off; off += up(N * sizeof(float));
+    l.Dterm = off; off += up(N * sizeof(float));
+  }
+  l.total = off;
+  return l;
+}
+
+template <typename P> P *at(void *base, size_t off) {
+  return reinterpret_cast<P *>(static_cast<char *>(base) + off);
+}
+
+float scale_of(const lizard_fwd_args *a) {
+  return a->softmax_scale > 0.f ? a->softmax_scale : 1.f / sqrtf((float)a->dk);
+}
+
+// A call's kernels in launch order.  The same list serves the launch and the
+// host-only plan query, so the names always match what runs.
+struct Plan {
+  static constexpr int kMax = 16;
+  const char *names[kMax];
+  std::function<cudaError_t()> fns[kMax];
+  int n = 0;
+  void add(const char *name, std::function<cudaError_t()> f) {
+    names[n] = name;
+    fns[n] = std::move(f);
+    ++n;
+  }
+  lizard_status run(cudaStream_t s, void *const *events, int nev) const {
+    if (events && nev > 0 && cudaEventRecord(static_cast<cudaEvent_t>(events[0]), s) != cudaSuccess)
+      return LIZARD_ERR_CUDA;
+    for (int i = 0; i < n; ++i) {
+      if (fns[i]() != cudaSuccess) return LIZARD_ERR_CUDA;
+      if (events && i + 1 < nev && cudaEventRecord(static_cast<cudaEvent_t>(events[i + 1]), s) != cudaSuccess)
+        return LIZARD_ERR_CUDA;
+    }
+    return LIZARD_OK;
+  }
+  int32_t names_out(const char **out, int32_t cap) const {
+    for (int i = 0; i < n && i < cap; ++i) out[i] = names[i];
+    return n;
+  }
+};
+
+void fwd_plan(const lizard_fwd_args *a, void *ws, cudaStream_t s, Plan &plan) {
+  const FwdLayout lay = fwd_layout(a);
+  const int BH = a->B * a->H, D = a->dk;
+  const bool bf16 = a->dtype == LIZARD_BF16;
+  float *o_gla = nullptr;
+  if (gla_on(a)) {
+    lz::PrepArgs pa{a->q, a->k, a->g, a->fmap_wq, a->fmap_wk, at<float>(ws, lay.phq), at<float>(ws, lay.phk),
+                    at<float>(ws, lay.a), a->H, a->L, 1.f / a->gate_temp};
+    plan.add("prep_kernel", [=] { return lz::launch_prep(pa, BH, D, bf16, s); });
+    o_gla = at<float>(ws, lay.o_gla);
+    lz::GlaFwdArgs ga{at<float>(ws, lay.phq), at<float>(ws, lay.phk), at<float>(ws, lay.a), a->v, a->state_in,
+                      o_gla, a->state_out, a->L};
+    plan.add("gla_fwd_simt", [=] { return lz::launch_gla_fwd_simt(ga, BH, D, bf16, s); });
+  }
+  lz::SwaMixArgs sa{a->q, a->k, a->v, a->meta_k, a->meta_v, a->alpha, o_gla, a->o,
+                    swa_on(a) ? a->lse : nullptr, a->H, a->L, a->window, a->M, a->branch, scale_of(a)};
+  plan.add("swa_mix_simt", [=] { return lz::launch_swa_mix_simt(sa, BH, D, bf16, s); });
+}
+
+void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan) {
+  const lizard_fwd_args *a = &b->fwd;
+  const BwdLayout lay = bwd_layout(a);
+  const int BH = a->B * a->H, D = a->dk;
+  const bool bf16 = a->dtype == LIZARD_BF16;
+  const float inv_tau = 1.f / a->gate_temp;
+  const bool g = gla_on(a), w = swa_on(a);
+  if (g) {
+    lz::PrepArgs pa{a->q, a->k, a->g, a->fmap_wq, a->fmap_wk, at<float>(ws, lay.phq), at<float>(ws, lay.phk),
+                    at<float>(ws, lay.a), a->H, a->L, inv_tau};
+    plan.add("prep_kernel", [=] { return lz::launch_prep(pa, BH, D, bf16, s); });
+    lz::GlaStatesArgs sa{at<float>(ws, lay.phk), at<float>(ws, lay.a), a->v, a->state_in, at<float>(ws, lay.sprev), a->L};
+    plan.add("gla_states_simt", [=] { return lz::launch_gla_states(sa, BH, D, bf16, s); });
+    lz::GlaBwdArgs ga{at<float>(ws, lay.phq), at<float>(ws, lay.phk), at<float>(ws, lay.a), a->v, b->dout,
+                      at<float>(ws, lay.sprev), at<float>(ws, lay.dphq), at<float>(ws, lay.dphk),
+                      at<float>(ws, lay.da), at<float>(ws, lay.dv_gla), b->dstate_in, a->L};
+    plan.add("gla_bwd_simt", [=] { return lz::launch_gla_bwd_simt(ga, BH, D, bf16, s); });
+  }
+  if (w) {
+    lz::SwaBwdQArgs qa{a->q, a->k, a->v, b->dout, a->meta_k, a->meta_v, a->alpha,
+                       at<float>(ws, lay.dq_swa), at<float>(ws, lay.lse), at<float>(ws, lay.Dterm),
+                       b->dmeta_k, b->dmeta_v, b->dalpha, a->H, a->L, a->window, a->M, scale_of(a)};
+    plan.add("swa_bwd_q", [=] { return lz::launch_swa_bwd_q(qa, BH, D, bf16, s); });
+    lz::SwaBwdKVArgs ka{a->q, a->k, a->v, b->dout, a->alpha, at<float>(ws, lay.lse), at<float>(ws, lay.Dterm),
+                        at<float>(ws, lay.dk_swa), at<float>(ws, lay.dv_swa), a->H, a->L, a->window, scale_of(a)};
+    plan.add("swa_bwd_kv", [=] { return lz::launch_swa_bwd_kv(ka, BH, D, bf16, s); });
+  }
+  lz::FinishBwdArgs fa{a->q, a->k, a->g,
+                       a->fmap_wq, a->fmap_wk,
+                       g ? at<float>(ws, lay.dphq) : nullptr, g ? at<float>(ws, lay.dphk) : nullptr,
+                       g ? at<float>(ws, lay.da) : nullptr, g ? at<float>(ws, lay.dv_gla) : nullptr,
+                       w ? at<float>(ws, lay.dq_swa) : nullptr, w ? at<float>(ws, lay.dk_swa) : nullptr,
+                       w ? at<float>(ws, lay.dv_swa) : nullptr,
+                       b->dq, b->dk, b->dv, b->dg, b->dfmap_wq, b->dfmap_wk, a->H, a->L, inv_tau};
+  plan.add("finish_bwd", [=] { return lz::launch_finish_bwd(fa, BH, D, bf16, s); });
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t lizard_fwd_workspace_size(const lizard_fwd_args *args) {
+  lizard_fwd_args a;
+  if (!args) return 0;
+  a = *args;
+  a.q = a.k = a.v = a.g = nullptr;
+  a.o = nullptr;
+  a.workspace = nullptr;
+  a.fmap_wq = a.fmap_wk = a.alpha = a.state_in = nullptr;
+  a.state_out = a.lse = nullptr;
+  const bool meta = a.M > 0;
+  a.meta_k = meta ? reinterpret_cast<const float *>(16) : nullptr;
+  a.meta_v = nullptr;
+  if (a.L > 0) {
+    // the pointer checks require non-null activations; use a stand-in
+    a.q = a.k = a.v = a.g = reinterpret_cast<const void *>(16);
+    a.o = reinterpret_cast<void *>(16);
+  }
+  if (check_fwd(&a) != LIZARD_OK) return 0;
+  return fwd_layout(&a).total;
+}
+
+lizard_status lizard_attn_fwd(const lizard_fwd_args *a, lizard_stream_t stream) {
+  lizard_status st = check_fwd(a);
+  if (st != LIZARD_OK) return st;
+  if (a->impl == LIZARD_IMPL_TC) return LIZARD_ERR_UNSUPPORTED;
+  const FwdLayout lay = fwd_layout(a);
+  if (!a->workspace || a->workspace_bytes < lay.total) return LIZARD_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int BH = a->B * a->H;
+  const size_t BHdd = (size_t)BH * a->dk * a->dv * sizeof(float);
+  if (a->L == 0) {
+    if (a->state_out) {
+      cudaError_t e = a->state_in ? cudaMemcpyAsync(a->state_out, a->state_in, BHdd, cudaMemcpyDeviceToDevice, s)
+                                  : cudaMemsetAsync(a->state_out, 0, BHdd, s);
+      return cuda_status(e);
+    }
+    return LIZARD_OK;
+  }
+  Plan plan;
+  fwd_plan(a, a->workspace, s, plan);
+  return plan.run(s, a->launch_events, a->n_launch_events);
+}
+
+static lizard_status check_bwd(const lizard_bwd_args *b) {
+  if (!b) return LIZARD_ERR_INVALID_ARG;
+  lizard_fwd_args f = b->fwd;
+  f.o = b->dq;  // the forward output is not used; dq stands in for the pointer check
+  f.state_out = nullptr;
+  f.lse = nullptr;
+  f.workspace = b->workspace;
+  f.impl = b->impl;
+  lizard_status st = check_fwd(&f);
+  if (st != LIZARD_OK) return st;
+  if (f.L > 0 && (!b->dout || !b->dq || !b->dk || !b->dv || !b->dg)) return LIZARD_ERR_INVALID_ARG;
+  if ((b->dmeta_k && !f.meta_k) || (b->dmeta_v && !f.meta_v) || (b->dfmap_wq && !f.fmap_wq) ||
+      (b->dfmap_wk && !f.fmap_wk))
+    return LIZARD_ERR_INVALID_ARG;
+  const void *ptrs[] = {b->dout, b->dq, b->dk, b->dv, b->dg, b->dmeta_k, b->dmeta_v,
+                        b->dfmap_wq, b->dfmap_wk, b->dalpha, b->dstate_in};
+  for (const void *p : ptrs)
+    if (!ok_ptr(p)) return LIZARD_ERR_INVALID_ARG;
+  return LIZARD_OK;
+}
+
+size_t lizard_bwd_workspace_size(const lizard_bwd_args *args) {
+  if (!args) return 0;
+  lizard_fwd_args a = args->fwd;
+  a.impl = args->impl;
+  a.q = a.k = a.v = a.g = nullptr;
+  a.o = nullptr;
+  a.workspace = nullptr;
+  a.fmap_wq = a.fmap_wk = a.alpha = a.state_in = nullptr;
+  a.state_out = a.lse = nullptr;
+  a.meta_k = a.M > 0 ? reinterpret_cast<const float *>(16) : nullptr;
+  a.meta_v = nullptr;
+  if (a.L > 0) {
+    a.q = a.k = a.v = a.g = reinterpret_cast<const void *>(16);
+    a.o = reinterpret_cast<void *>(16);
+  }
+  if (check_fwd(&a) != LIZARD_OK) return 0;
+  return bwd_layout(&a).total;
+}
+
+lizard_status lizard_attn_bwd(const lizard_bwd_args *b, lizard_stream_t stream) {
+  lizard_status st = check_bwd(b);
+  if (st != LIZARD_OK) return st;
+  if (b->impl == LIZARD_IMPL_TC) return LIZARD_ERR_UNSUPPORTED;
+  const lizard_fwd_args *a = &b->fwd;
+  const BwdLayout lay = bwd_layout(a);
+  if (!b->workspace || b->workspace_bytes < lay.total) return LIZARD_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int BH = a->B * a->H, D = a->dk, F = D / 2;
+  void *ws = b->workspace;
+  cudaError_t e = cudaSuccess;
+  // outputs that are accumulated atomically start at zero
+  struct Z { void *p; size_t n; } zs[] = {
+      {b->dmeta_k, (size_t)a->H * a->M * a->dk * 4}, {b->dmeta_v, (size_t)a->H * a->M * a->dv * 4},
+      {b->dfmap_wq, (size_t)a->H * D * F * 4},       {b->dfmap_wk, (size_t)a->H * D * F * 4},
+      {b->dalpha, (size_t)a->H * 4}};
+  for (const Z &z : zs)
+    if (z.p && z.n && (e = cudaMemsetAsync(z.p, 0, z.n, s)) != cudaSuccess) return LIZARD_ERR_CUDA;
+  const size_t BHdd = (size_t)BH * a->dk * a->dv * sizeof(float);
+  if (a->L == 0 || !gla_on(a)) {
+    if (b->dstate_in && (e = cudaMemsetAsync(b->dstate_in, 0, BHdd, s)) != cudaSuccess) return LIZARD_ERR_CUDA;
+  }
+  if (a->L == 0) return LIZARD_OK;
+  Plan plan;
+  bwd_plan(b, ws, s, plan);
+  return plan.run(s, b->launch_events, b->n_launch_events);
+}
+
+int32_t lizard_fwd_launch_plan(const lizard_fwd_args *a, const char **names, int32_t cap) {
+  if (check_fwd(a) != LIZARD_OK) return -1;
+  if (a->L == 0) return 0;
+  Plan plan;
+  fwd_plan(a, a->workspace, nullptr, plan);
+  return plan.names_out(names, cap);
+}
+
+int32_t lizard_bwd_launch_plan(const lizard_bwd_args *b, const char **names, int32_t cap) {
+  if (check_bwd(b) != LIZARD_OK) return -1;
+  if (b->fwd.L == 0) return 0;
+  Plan plan;
+  bwd_plan(b, b->workspace, nullptr, plan);
+  return plan.names_out(names, cap);
+}
+
+lizard_status lizard_decode_step(const lizard_decode_args *a, lizard_stream_t stream) {
+  if (!a) return LIZARD_ERR_INVALID_ARG;
+  if (a->B < 1 || a->H < 1 || a->dk <= 0 || a->dv <= 0 || a->window < 1 || a->M < 0) return LIZARD_ERR_INVALID_ARG;
+  if (a->dtype != LIZARD_BF16 && a->dtype != LIZARD_FP32) return LIZARD_ERR_INVALID_ARG;
+  if (!(a->gate_temp > 0.f) || !isfinite(a->gate_temp)) return LIZARD_ERR_INVALID_ARG;
+  if (!(a->softmax_scale >= 0.f) || !isfinite(a->softmax_scale)) return LIZARD_ERR_INVALID_ARG;
+  if (a->dk != a->dv || (a->dk != 64 && a->dk != 128)) return LIZARD_ERR_UNSUPPORTED;
+  if (a->M > 16 || a->window > 16384) return LIZARD_ERR_UNSUPPORTED;
+  if ((a->M > 0) != (a->meta_k != nullptr)) return LIZARD_ERR_INVALID_ARG;
+  if (a->meta_v && !a->meta_k) return LIZARD_ERR_INVALID_ARG;
+  if (!a->q || !a->k || !a->v || !a->g || !a->state || !a->k_cache || !a->v_cache || !a->pos || !a->o)
+    return LIZARD_ERR_INVALID_ARG;
+  const void *ptrs[] = {a->q, a->k, a->v, a->g, a->state, a->k_cache, a->v_cache, a->pos,
+                        a->fmap_wq, a->fmap_wk, a->meta_k, a->meta_v, a->alpha, a->o};
+  for (const void *p : ptrs)
+    if (!ok_ptr(p)) return LIZARD_ERR_INVALID_ARG;
+  lz::DecodeArgs d{a->q, a->k, a->v, a->g, a->state, a->k_cache, a->v_cache, a->pos,
+                   a->fmap_wq, a->fmap_wk, a->meta_k, a->meta_v, a->alpha, a->o,
+                   a->H, a->window, a->M, 1.f / a->gate_temp,
+                   a->softmax_scale > 0.f ? a->softmax_scale : 1.f / sqrtf((float)a->dk)};
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return cuda_status(lz::launch_decode(d, a->B, a->dk, a->dtype == LIZARD_BF16, a->pos, s));
+}
+
+lizard_status lizard_workspace_status(void *workspace, lizard_stream_t stream) {
+  if (!workspace) return LIZARD_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return LIZARD_ERR_CUDA;
+  uint32_t word = 0;
+  if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return LIZARD_ERR_CUDA;
+  if (word != 0 && cudaMemset(workspace, 0, sizeof(word)) != cudaSuccess) return LIZARD_ERR_CUDA;
+  return word == 0 ? LIZARD_OK : LIZARD_ERR_TIMEOUT;
+}
+
+const char *lizard_status_string(lizard_status s) {
+  switch (s) {
+    case LIZARD_OK: return "ok";
+    case LIZARD_ERR_INVALID_ARG: return "invalid argument";
+    case LIZARD_ERR_UNSUPPORTED: return "unsupported size or option";
+    case LIZARD_ERR_CUDA: return "CUDA launch or runtime error";
+    case LIZARD_ERR_TIMEOUT: return "a kernel gave up on a bounded wait";
+    case LIZARD_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+const char *lizard_version(void) { return "0.1.0"; }
+
+}  // extern "C"

@@ -1,0 +1,107 @@
+// Internal launch interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace lz {
+
+struct PrepArgs {
+  const void *q, *k, *g;
+  const float *wq, *wk;
+  float *phq, *phk, *a;
+  int H, L;
+  float inv_tau;
+};
+
+struct GlaFwdArgs {
+  const float *phq, *phk, *a;
+  const void *v;
+  const float *state_in;
+  float *o_gla;
+  float *state_out;
+  int L;
+};
+
+struct SwaMixArgs {
+  const void *q, *k, *v;
+  const float *meta_k, *meta_v, *alpha;
+  const float *o_gla;
+  void *o;
+  float *lse;
+  int H, L, window, M, branch;
+  float scale;
+};
+
+struct DecodeArgs {
+  const void *q, *k, *v, *g;
+  float *state;
+  void *k_cache, *v_cache;
+  const int64_t *pos;
+  const float *wq, *wk, *meta_k, *meta_v, *alpha;
+  void *o;
+  int H, window, M;
+  float inv_tau, scale;
+};
+
+// Backward (portable fp32 kernels).
+struct GlaStatesArgs {
+  const float *phk, *a;
+  const void *v;
+  const float *state_in;
+  float *sprev;     // [BH][nchunk][D][D] state at the start of each chunk
+  int L;
+};
+
+struct GlaBwdArgs {
+  const float *phq, *phk, *a;
+  const void *v, *dout;
+  const float *sprev;
+  float *dphq, *dphk, *da, *dv_gla;
+  float *dstate_in;  // may be null
+  int L;
+};
+
+struct SwaBwdQArgs {
+  const void *q, *k, *v, *dout;
+  const float *meta_k, *meta_v, *alpha;
+  float *dq_swa, *lse, *Dterm;
+  float *dmeta_k, *dmeta_v, *dalpha;   // accumulated atomically; may be null
+  int H, L, window, M;
+  float scale;
+};
+
+struct SwaBwdKVArgs {
+  const void *q, *k, *v, *dout;
+  const float *alpha, *lse, *Dterm;
+  float *dk_swa, *dv_swa;
+  int H, L, window;
+  float scale;
+};
+
+struct FinishBwdArgs {
+  const void *q, *k, *g;
+  const float *wq, *wk;
+  const float *dphq, *dphk, *da, *dv_gla;   // null when the GLA branch is off
+  const float *dq_swa, *dk_swa, *dv_swa;    // null when the anchor branch is off
+  void *dq, *dk, *dv;
+  float *dg, *dwq, *dwk;                    // dwq/dwk accumulated atomically; may be null
+  int H, L;
+  float inv_tau;
+};
+
+constexpr int kBwdC = 32;   // GLA chunk used by the portable backward
+
+cudaError_t launch_prep(const PrepArgs &a, int BH, int D, bool bf16, cudaStream_t s);
+cudaError_t launch_gla_fwd_simt(const GlaFwdArgs &a, int BH, int D, bool bf16, cudaStream_t s);
+cudaError_t launch_swa_mix_simt(const SwaMixArgs &a, int BH, int D, bool bf16, cudaStream_t s);
+cudaError_t launch_decode(const DecodeArgs &a, int B, int D, bool bf16, int64_t *pos, cudaStream_t s);
+
+cudaError_t launch_gla_states(const GlaStatesArgs &a, int BH, int D, bool bf16, cudaStream_t s);
+cudaError_t launch_gla_bwd_simt(const GlaBwdArgs &a, int BH, int D, bool bf16, cudaStream_t s);
+cudaError_t launch_swa_bwd_q(const SwaBwdQArgs &a, int BH, int D, bool bf16, cudaStream_t s);
+cudaError_t launch_swa_bwd_kv(const SwaBwdKVArgs &a, int BH, int D, bool bf16, cudaStream_t s);
+cudaError_t launch_finish_bwd(const FinishBwdArgs &a, int BH, int D, bool bf16, cudaStream_t s);
+
+}  // namespace lz

@@ -1,0 +1,224 @@
+/*
+ * lizard.h -- C ABI of liblizard.so: Lizard hybrid attention on NVIDIA B200.
+ *
+ * The layer (arXiv 2507.09025, "Lizard: An Efficient Linearization Framework
+ * for Large Language Models"; the gist.science technical summaries in
+ * English, French, Spanish and Chinese describe it) mixes two branches:
+ *
+ *   GLA branch (English summary, section 2.A "State Update"):
+ *     a_t   = logsigmoid(g_t) / gate_temp                   (per key dim)
+ *     S_t   = diag(exp a_t) S_{t-1} + phi_k(k_t) v_t^T      (fp32 state)
+ *     o^gla = S_t^T phi_q(q_t)
+ *   with phi(x) = [softmax(x W), softmax(-x W)], W in R^{dk x dk/2} per head
+ *   (the non-negative Hedgehog map of the Chinese summary, section 2.3), or
+ *   the identity when W is NULL.
+ *
+ *   Anchor branch (English summary, section 2.A "Anchor Window Attention"):
+ *     softmax over the keys j in [t - window + 1, t] and the M meta tokens,
+ *     logits softmax_scale * q_t . key; o^swa = sum p * value, where a meta
+ *     token's value is meta_v[m] (or nothing when meta_v is NULL: a pure
+ *     sink in the softmax denominator).
+ *
+ *   Mix (French summary, section 2.A last line):  o = o^gla + alpha_h o^swa.
+ *
+ * Conventions shared by every entry point
+ *   - All pointers are DEVICE pointers unless stated otherwise; the caller
+ *     owns all memory, including the workspace.  The library allocates and
+ *     frees nothing and keeps no state between calls.
+ *   - Activations (q, k, v, g, o, caches, their gradients) use `dtype`
+ *     (bf16 or fp32), contiguous row-major with the innermost dimension last
+ *     (the shapes below).  Parameters (feature-map weights, meta tokens,
+ *     alpha) and the recurrent state are fp32.  Gradients of parameters, of
+ *     the gate logits and of the state are fp32.
+ *   - Work is enqueued on `stream` and runs asynchronously.  Arguments are
+ *     checked on the host before anything is launched: a call that returns
+ *     an error status launched nothing.
+ *   - Every pointer must be 16-byte aligned.
+ *   - Supported: dk = dv in {64, 128}; chunk = 64; window >= 1; 0 <= M <= 16;
+ *     L >= 0 (L = 0 is a no-op); B * H >= 1.  Other sizes return
+ *     LIZARD_ERR_UNSUPPORTED.
+ *   - Launch errors return LIZARD_ERR_CUDA.  A kernel that gives up on a
+ *     bounded wait records LIZARD_ERR_TIMEOUT in the workspace status word,
+ *     which lizard_workspace_status() reads back.
+ */
+#ifndef LIZARD_H_
+#define LIZARD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *lizard_stream_t; /* == cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  LIZARD_OK = 0,
+  LIZARD_ERR_INVALID_ARG = 1, /* NULL required pointer, negative size, misaligned pointer */
+  LIZARD_ERR_UNSUPPORTED = 2, /* well-formed but outside the supported sizes */
+  LIZARD_ERR_CUDA = 3,        /* a launch or CUDA runtime call failed */
+  LIZARD_ERR_TIMEOUT = 4,     /* a kernel gave up on a bounded wait */
+  LIZARD_ERR_WORKSPACE = 5    /* workspace NULL or smaller than the queried size */
+} lizard_status;
+
+typedef enum { LIZARD_BF16 = 0, LIZARD_FP32 = 1 } lizard_dtype;
+
+/* Which terms of o = o^gla + alpha_h o^swa to compute (test hook). */
+enum { LIZARD_BRANCH_BOTH = 0, LIZARD_BRANCH_GLA_ONLY = 1, LIZARD_BRANCH_SWA_ONLY = 2 };
+
+/* Kernel family selection (lizard_fwd_args.impl / lizard_bwd_args.impl). */
+enum {
+  LIZARD_IMPL_AUTO = 0,  /* tensor-core path where it applies, else portable */
+  LIZARD_IMPL_SIMT = 1,  /* portable fp32 CUDA-core kernels (exact fp32 math) */
+  LIZARD_IMPL_TC = 2     /* tcgen05/TMEM tensor-core kernels (bf16, dk = 128) */
+};
+
+/*
+ * Forward of the hybrid layer over whole sequences.
+ *
+ * Shapes (B batch, H heads, L tokens, dk = dv = d):
+ *   q, k, g    [B, H, L, dk] dtype   (g: gate logits; the gate projection
+ *                                      W_gamma x itself is the caller's)
+ *   v          [B, H, L, dv] dtype
+ *   fmap_wq/wk [H, dk, dk/2] fp32, or NULL for the identity map
+ *   meta_k     [H, M, dk] fp32 (NULL iff M == 0)
+ *   meta_v     [H, M, dv] fp32, or NULL for sink-only meta tokens
+ *   alpha      [H] fp32 mixing weights (NULL = all ones)
+ *   state_in   [B, H, dk, dv] fp32 initial state S_{-1}, or NULL for zeros
+ *   o          [B, H, L, dv] dtype, written
+ *   state_out  [B, H, dk, dv] fp32 final state S_{L-1}, or NULL (written
+ *              only when the GLA branch runs)
+ *   lse        [B, H, L] fp32 natural-log softmax normaliser of the anchor
+ *              branch (window + meta logits), or NULL (written only when the
+ *              anchor branch runs)
+ * gate_temp is tau (> 0); softmax_scale 0 means 1/sqrt(dk).
+ * chunk is the GLA chunk length (64); it changes the schedule, not the result.
+ */
+typedef struct {
+  int32_t B, H, L, dk, dv, chunk, window, M;
+  int32_t dtype;   /* lizard_dtype */
+  int32_t branch;  /* LIZARD_BRANCH_* */
+  int32_t impl;    /* LIZARD_IMPL_* */
+  float gate_temp;
+  float softmax_scale;
+  const void *q, *k, *v, *g;
+  const float *fmap_wq, *fmap_wk;
+  const float *meta_k, *meta_v;
+  const float *alpha;
+  const float *state_in;
+  void *o;
+  float *state_out;
+  float *lse;
+  void *workspace;        /* device scratch, >= lizard_fwd_workspace_size() bytes */
+  size_t workspace_bytes;
+  /* Optional kernel timing: cudaEvent_t handles created by the caller.  When
+   * non-NULL, the call records launch_events[0] before its first kernel and
+   * launch_events[i] after its i-th kernel, for i < n_launch_events, all on
+   * `stream`.  lizard_fwd_launch_plan() names the kernels in order. */
+  void *const *launch_events;
+  int32_t n_launch_events;
+} lizard_fwd_args;
+
+/* Bytes of device workspace the forward needs for these arguments (pointer
+ * fields are ignored).  Returns 0 when the sizes are invalid. */
+size_t lizard_fwd_workspace_size(const lizard_fwd_args *args);
+
+/* Enqueue the forward.  See the conventions above for errors. */
+lizard_status lizard_attn_fwd(const lizard_fwd_args *args, lizard_stream_t stream);
+
+/*
+ * Backward of the hybrid layer: gradients of sum(dout * o) with respect to
+ * every input of lizard_attn_fwd.
+ *
+ *   fwd      the forward's inputs (fwd.o, fwd.state_out, fwd.lse and the
+ *            forward workspace are ignored)
+ *   dout     [B, H, L, dv] dtype
+ *   dq, dk   [B, H, L, dk] dtype, written
+ *   dv       [B, H, L, dv] dtype, written
+ *   dg       [B, H, L, dk] fp32 gradient of the gate logits, written
+ *   dmeta_k, dmeta_v, dfmap_wq, dfmap_wk, dalpha, dstate_in   fp32, same
+ *            shapes as the inputs, written (overwritten, not accumulated);
+ *            each may be NULL when not wanted (and must be NULL when the
+ *            matching input is NULL).
+ * The final state S_{L-1} is treated as unused (zero incoming gradient).
+ */
+typedef struct {
+  lizard_fwd_args fwd;
+  const void *dout;
+  void *dq, *dk, *dv;
+  float *dg;
+  float *dmeta_k, *dmeta_v;
+  float *dfmap_wq, *dfmap_wk;
+  float *dalpha;
+  float *dstate_in;
+  int32_t impl;           /* LIZARD_IMPL_* */
+  void *workspace;        /* >= lizard_bwd_workspace_size() bytes */
+  size_t workspace_bytes;
+  void *const *launch_events;   /* as in lizard_fwd_args */
+  int32_t n_launch_events;
+} lizard_bwd_args;
+
+size_t lizard_bwd_workspace_size(const lizard_bwd_args *args);
+lizard_status lizard_attn_bwd(const lizard_bwd_args *args, lizard_stream_t stream);
+
+/* Kernels lizard_attn_fwd / lizard_attn_bwd launch for these arguments, in
+ * launch order: fills names[0 .. min(count, cap)) with static strings and
+ * returns count (-1 when the arguments are invalid).  Host only. */
+int32_t lizard_fwd_launch_plan(const lizard_fwd_args *args, const char **names, int32_t cap);
+int32_t lizard_bwd_launch_plan(const lizard_bwd_args *args, const char **names, int32_t cap);
+
+/*
+ * One decode step for every sequence: the constant-memory generation of the
+ * English summary (section 2.A "State Update") with the fixed-size window
+ * cache of the Chinese summary (section 2.1).
+ *
+ *   q, k, g    [B, H, dk] dtype;  v [B, H, dv] dtype: the new token
+ *   state      [B, H, dk, dv] fp32, updated in place:
+ *              S <- diag(exp a) S + phi_k(k) v^T
+ *   k_cache    [B, H, window, dk] dtype, v_cache [B, H, window, dv] dtype:
+ *              ring buffers; the new (k, v) is written to slot pos[b] mod
+ *              window, in place
+ *   pos        [B] int64 tokens already seen per sequence; incremented in
+ *              place after the step
+ *   o          [B, H, dv] dtype, written: o = S^T phi_q(q) + alpha_h o^swa,
+ *              the softmax covering the min(pos+1, window) filled slots and
+ *              the M meta tokens
+ * Parameters as in lizard_fwd_args.  Needs no workspace.  Two kernels are
+ * enqueued (the step, then the pos increment), so concurrent heads of one
+ * sequence all see the same pos.
+ */
+typedef struct {
+  int32_t B, H, dk, dv, window, M;
+  int32_t dtype;
+  float gate_temp;
+  float softmax_scale;
+  const void *q, *k, *v, *g;
+  float *state;
+  void *k_cache, *v_cache;
+  int64_t *pos;
+  const float *fmap_wq, *fmap_wk;
+  const float *meta_k, *meta_v;
+  const float *alpha;
+  void *o;
+} lizard_decode_args;
+
+lizard_status lizard_decode_step(const lizard_decode_args *args, lizard_stream_t stream);
+
+/* Waits for `stream`, then reads and clears the status word that kernels
+ * with bounded waits leave at the start of a forward or backward workspace.
+ * Returns LIZARD_OK or LIZARD_ERR_TIMEOUT (LIZARD_ERR_CUDA if the copy
+ * fails).  `workspace` is a device pointer. */
+lizard_status lizard_workspace_status(void *workspace, lizard_stream_t stream);
+
+/* Static description of a status code; never NULL. */
+const char *lizard_status_string(lizard_status s);
+
+/* Library version, "major.minor.patch". */
+const char *lizard_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIZARD_H_ */

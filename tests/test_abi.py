@@ -1,0 +1,168 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/lizard.h declares, the ctypes structs match the C layout, and the
+host-side argument checks reject bad calls before anything is launched."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lizard.h")
+
+
+@pytest.fixture(scope="module")
+def lz():
+    from gated_linear_sliding_chunkwise_b200 import build
+    build.build()
+    from gated_linear_sliding_chunkwise_b200 import lizard
+    return lizard
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lizard_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = _declared_functions()
+    for required in ("lizard_attn_fwd", "lizard_attn_bwd", "lizard_decode_step"):
+        assert required in names
+
+
+def test_library_exports_every_declared_function(lz):
+    out = subprocess.run(["nm", "-D", "--defined-only", lz.LIB_PATH],
+                         capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (lizard_\w+)", out))
+    missing = [n for n in _declared_functions() if n not in exported]
+    assert not missing, f"not exported: {missing}"
+    for n in _declared_functions():
+        assert hasattr(lz.lib(), n)
+
+
+def test_struct_layouts_match_c(lz, tmp_path):
+    """Compile a C program against the header and compare sizeof/offsetof."""
+    fields = {
+        "lizard_fwd_args": lz.FwdArgs, "lizard_bwd_args": lz.BwdArgs,
+        "lizard_decode_args": lz.DecodeArgs,
+    }
+    lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "lizard.h"',
+             "int main(void) {"]
+    for cname, py in fields.items():
+        lines.append(f'printf("{cname} size %zu\\n", sizeof({cname}));')
+        for fname, _ in py._fields_:
+            lines.append(f'printf("{cname} {fname} %zu\\n", offsetof({cname}, {fname}));')
+    lines.append("return 0; }")
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), str(src),
+                    "-o", str(exe)], check=True)
+    got = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout
+    for line in got.strip().splitlines():
+        cname, what, val = line.split()
+        py = fields[cname]
+        want = ctypes.sizeof(py) if what == "size" else getattr(py, what).offset
+        assert int(val) == want, f"{cname}.{what}: C {val} vs ctypes {want}"
+
+
+def test_status_strings_and_version(lz):
+    for code in range(6):
+        assert lz.status_string(code)
+    assert lz.status_string(99) == "unknown status"
+    assert re.match(r"\d+\.\d+\.\d+$", lz.version())
+
+
+def _fwd(lz, **over):
+    a = lz.FwdArgs()
+    a.B, a.H, a.L, a.dk, a.dv, a.chunk, a.window, a.M = 1, 2, 128, 64, 64, 64, 16, 4
+    a.dtype, a.branch, a.impl = lz.BF16, 0, 0
+    a.gate_temp, a.softmax_scale = 16.0, 0.0
+    fake = 0x10000   # never dereferenced: every case fails on the host first
+    a.q = a.k = a.v = a.g = a.o = fake
+    a.meta_k = fake
+    for k_, v_ in over.items():
+        setattr(a, k_, v_)
+    return a
+
+
+@pytest.mark.parametrize("over,code", [
+    ({"dk": 96, "dv": 96}, 2),
+    ({"dk": 64, "dv": 128}, 2),
+    ({"chunk": 32}, 2),
+    ({"M": 17}, 2),
+    ({"window": 0}, 1),
+    ({"L": -1}, 1),
+    ({"B": 0}, 1),
+    ({"dtype": 7}, 1),
+    ({"branch": 3}, 1),
+    ({"gate_temp": 0.0}, 1),
+    ({"gate_temp": float("nan")}, 1),
+    ({"softmax_scale": -1.0}, 1),
+    ({"q": None}, 1),
+    ({"g": None}, 1),
+    ({"meta_k": None}, 1),            # M > 0 needs meta keys
+    ({"M": 0}, 1),                    # meta keys given but M == 0
+    ({"q": 0x10004}, 1),              # not 16-byte aligned
+])
+def test_forward_rejects_bad_arguments_on_host(lz, over, code):
+    a = _fwd(lz, **over)
+    assert lz.lib().lizard_attn_fwd(ctypes.byref(a), None) == code
+
+
+def test_forward_checks_workspace_before_launch(lz):
+    a = _fwd(lz)
+    need = lz.fwd_workspace_bytes(a)
+    assert need > 0
+    a.workspace, a.workspace_bytes = 0x20000, need - 1
+    assert lz.lib().lizard_attn_fwd(ctypes.byref(a), None) == lz.ERR_WORKSPACE
+    a.workspace, a.workspace_bytes = None, 0
+    assert lz.lib().lizard_attn_fwd(ctypes.byref(a), None) == lz.ERR_WORKSPACE
+    # the anchor-only test hook needs no GLA scratch
+    b = _fwd(lz, branch=lz.BRANCH_SWA_ONLY)
+    assert lz.fwd_workspace_bytes(b) < need
+
+
+def test_workspace_size_rejects_bad_sizes(lz):
+    assert lz.fwd_workspace_bytes(_fwd(lz, dk=96, dv=96)) == 0
+    assert lz.lib().lizard_fwd_workspace_size(None) == 0
+
+
+def test_backward_rejects_bad_arguments_on_host(lz):
+    b = lz.BwdArgs()
+    b.fwd = _fwd(lz)
+    fake = 0x10000
+    b.dout = b.dq = b.dk = b.dv = b.dg = fake
+    need = lz.bwd_workspace_bytes(b)
+    assert need > lz.fwd_workspace_bytes(b.fwd)
+    b.workspace, b.workspace_bytes = 0x20000, need - 1
+    assert lz.lib().lizard_attn_bwd(ctypes.byref(b), None) == lz.ERR_WORKSPACE
+    b.dg = None
+    assert lz.lib().lizard_attn_bwd(ctypes.byref(b), None) == lz.ERR_INVALID_ARG
+    b.dg = fake
+    b.dfmap_wq = fake          # gradient asked for an absent input
+    assert lz.lib().lizard_attn_bwd(ctypes.byref(b), None) == lz.ERR_INVALID_ARG
+    assert lz.lib().lizard_attn_bwd(None, None) == lz.ERR_INVALID_ARG
+
+
+def test_decode_rejects_bad_arguments_on_host(lz):
+    d = lz.DecodeArgs()
+    d.B, d.H, d.dk, d.dv, d.window, d.M, d.dtype = 2, 2, 128, 128, 128, 0, lz.BF16
+    d.gate_temp = 16.0
+    fake = 0x10000
+    for n in ("q", "k", "v", "g", "state", "k_cache", "v_cache", "pos", "o"):
+        setattr(d, n, fake)
+    d.dk = d.dv = 80
+    assert lz.lib().lizard_decode_step(ctypes.byref(d), None) == lz.ERR_UNSUPPORTED
+    d.dk = d.dv = 128
+    d.window = 20000
+    assert lz.lib().lizard_decode_step(ctypes.byref(d), None) == lz.ERR_UNSUPPORTED
+    d.window = 128
+    d.pos = None
+    assert lz.lib().lizard_decode_step(ctypes.byref(d), None) == lz.ERR_INVALID_ARG
+    d.pos = fake
+    d.M = 2                    # meta tokens without meta keys
+    assert lz.lib().lizard_decode_step(ctypes.byref(d), None) == lz.ERR_INVALID_ARG

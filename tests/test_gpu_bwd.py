@@ -1,0 +1,131 @@
+"""GPU parity of lizard_attn_bwd against the oracle's hand-derived backward
+(itself pinned by central differences and autograd on the CPU)."""
+
+import pytest
+import torch
+
+from gated_linear_sliding_chunkwise_b200.synth import WORKLOADS, Workload, make_inputs, random_alpha
+from lizard_testutil import check, oracle_backward, to_device
+from oracle import lizard_ref as ref
+
+pytestmark = pytest.mark.gpu
+
+GRADS = ["dq", "dk", "dv", "dg", "dmeta_k", "dmeta_v", "dfmap_wq", "dfmap_wk", "dalpha",
+         "dstate_in"]
+IMPLS = ["simt"]
+
+
+@pytest.fixture(scope="module")
+def lz():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from gated_linear_sliding_chunkwise_b200 import lizard
+    return lizard
+
+
+def _impl(lz, name):
+    return {"simt": lz.IMPL_SIMT, "tc": lz.IMPL_TC, "auto": lz.IMPL_AUTO}[name]
+
+
+def _run(lz, x, w, impl, **kw):
+    return lz.attn_bwd(x["q"], x["k"], x["v"], x["g"], x["dout"], window=w.window,
+                       chunk=w.chunk, gate_temp=w.gate_temp, fmap_wq=x.get("fmap_wq"),
+                       fmap_wk=x.get("fmap_wk"), meta_k=x.get("meta_k"),
+                       meta_v=x.get("meta_v"), alpha=x.get("alpha"),
+                       state_in=x.get("state_in"), impl=impl, **kw)
+
+
+def _grad_dtype(name, act_dtype):
+    # dq, dk, dv are stored in the activation dtype; the rest in fp32 but
+    # computed from bf16-rounded inputs, so they take the same bar.
+    return act_dtype
+
+
+SWEEP = [
+    # dtype, d, L, window, M, meta_v, state_in, random alpha
+    ("fp32", 64, 1, 4, 2, True, True, False),
+    ("fp32", 64, 97, 16, 4, True, True, True),
+    ("fp32", 128, 70, 100, 4, False, False, True),
+    ("fp32", 64, 150, 1, 0, False, True, False),
+    ("bf16", 128, 260, 128, 4, True, True, True),
+    ("bf16", 64, 129, 33, 16, True, False, True),
+]
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("dtype,d,L,window,M,with_mv,with_state,rand_alpha", SWEEP)
+def test_backward_sweep(lz, impl, dtype, d, L, window, M, with_mv, with_state, rand_alpha):
+    w = Workload("bsweep", B=2, H=2, L=L, d=d, window=window, M=M, dtype=dtype,
+                 seed=100 + L, kind="train")
+    inp = make_inputs(w)
+    if not with_mv:
+        inp["meta_v"] = None
+    if M == 0:
+        inp["meta_k"] = inp["meta_v"] = None
+    if with_state:
+        inp["state_in"] = torch.randn(2, 2, d, d, generator=torch.Generator().manual_seed(8)) * 0.1
+    if rand_alpha:
+        inp["alpha"] = random_alpha(2, seed=L)
+    got = _run(lz, to_device(inp), w, _impl(lz, impl))
+    want = oracle_backward(inp, window=window, tau=w.gate_temp)
+    for name in GRADS:
+        if want[name] is None:
+            assert got[name] is None
+            continue
+        check(name, got[name], want[name], _grad_dtype(name, dtype))
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("branch", [ref.BRANCH_GLA_ONLY, ref.BRANCH_SWA_ONLY])
+def test_backward_branch_hooks(lz, impl, branch):
+    w = Workload("bbranch", B=1, H=2, L=90, d=64, window=10, M=4, dtype="fp32", seed=5,
+                 kind="train")
+    inp = make_inputs(w)
+    inp["alpha"] = random_alpha(2, seed=1)
+    got = _run(lz, to_device(inp), w, _impl(lz, impl), branch=branch)
+    want = oracle_backward(inp, window=w.window, tau=w.gate_temp, branch=branch)
+    for name in GRADS:
+        check(name, got[name], want[name], "fp32")
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_backward_extreme_decay(lz, impl):
+    w = Workload("bextreme", B=1, H=2, L=100, d=64, window=6, M=2, dtype="fp32", seed=6,
+                 kind="train")
+    inp = make_inputs(w)
+    g = inp["g"].clone()
+    g[:, :, 5:40, :9] = -300.0
+    inp["g"] = g
+    got = _run(lz, to_device(inp), w, _impl(lz, impl))
+    want = oracle_backward(inp, window=w.window, tau=w.gate_temp)
+    for name in GRADS:
+        check(name, got[name], want[name], "fp32")
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_parameter_grads_bf16_full_reduction(lz, impl):
+    """Gradients of the per-head parameters reduce over batch and tokens:
+    check them against the oracle over every (b, h) of a mid-size case."""
+    w = Workload("params", B=2, H=2, L=512, d=128, dtype="bf16", seed=13, kind="train")
+    inp = make_inputs(w)
+    got = _run(lz, to_device(inp), w, _impl(lz, impl))
+    want = oracle_backward(inp, window=w.window, tau=w.gate_temp)
+    for name in GRADS:
+        check(name, got[name], want[name], "bf16")
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_train_step_full_size_sampled_heads(lz, impl):
+    """The full training-step workload (B=8, H=32, L=2048) as the benchmark
+    launches it; per-sequence gradients of sampled (b, h) pairs vs the oracle."""
+    w = WORKLOADS["train_step"]
+    inp = make_inputs(w)
+    got = _run(lz, to_device(inp), w, _impl(lz, impl))
+    torch.cuda.synchronize()
+    for name in ("dq", "dk", "dv", "dg", "dalpha", "dfmap_wq", "dmeta_k"):
+        assert torch.isfinite(got[name]).all(), name
+    pairs = [(0, 0), (7, 21)]
+    want = oracle_backward(inp, window=w.window, tau=w.gate_temp, pairs=pairs)
+    for (b, h), r in want.items():
+        for name in ("dq", "dk", "dv", "dg", "dstate_in"):
+            check(f"{name}[{b},{h}]", got[name][b:b + 1, h:h + 1], r[name], "bf16")

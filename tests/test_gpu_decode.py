@@ -1,0 +1,107 @@
+"""GPU parity of lizard_decode_step against the oracle, and decode replay
+against the GPU forward."""
+
+import numpy as np
+import pytest
+import torch
+
+from gated_linear_sliding_chunkwise_b200.synth import WORKLOADS, Workload, make_inputs, random_alpha
+from lizard_testutil import check, oracle_forward, to_device, to64
+from oracle import lizard_ref as ref
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def lz():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from gated_linear_sliding_chunkwise_b200 import lizard
+    return lizard
+
+
+def _oracle_step(inp, w):
+    x = {k_: (to64(v_) if k_ != "pos" else v_.numpy()) for k_, v_ in inp.items() if v_ is not None}
+    return ref.lizard_decode_step(x["q"], x["k"], x["v"], x["g"], x["state"], x["k_cache"],
+                                  x["v_cache"], x["pos"], window=w.window, tau=w.gate_temp,
+                                  fmap_wq=x.get("fmap_wq"), fmap_wk=x.get("fmap_wk"),
+                                  meta_k=x.get("meta_k"), meta_v=x.get("meta_v"),
+                                  alpha=x.get("alpha"))
+
+
+def _gpu_step(lz, x, w):
+    return lz.decode_step(x["q"], x["k"], x["v"], x["g"], x["state"], x["k_cache"],
+                          x["v_cache"], x["pos"], gate_temp=w.gate_temp,
+                          fmap_wq=x.get("fmap_wq"), fmap_wk=x.get("fmap_wk"),
+                          meta_k=x.get("meta_k"), meta_v=x.get("meta_v"), alpha=x.get("alpha"))
+
+
+def test_decode_full_batch_one_step(lz):
+    """The full decode workload (B=64, H=32, d=128, window 128, 65536 tokens
+    seen): every output of one step against the oracle."""
+    w = WORKLOADS["decode_b64"]
+    inp = make_inputs(w)
+    x = to_device(inp)
+    o = _gpu_step(lz, x, w)
+    torch.cuda.synchronize()
+    want_o, want_S, want_kc, want_vc, want_pos = _oracle_step(inp, w)
+    check("o", o, want_o, "bf16")
+    check("state", x["state"], want_S, "fp32")
+    # the ring slot write is a copy: bit-exact
+    assert torch.equal(x["k_cache"].cpu(), torch.from_numpy(want_kc).to(x["k_cache"].dtype))
+    assert torch.equal(x["v_cache"].cpu(), torch.from_numpy(want_vc).to(x["v_cache"].dtype))
+    assert torch.equal(x["pos"].cpu(), torch.from_numpy(want_pos))
+
+
+@pytest.mark.parametrize("dtype,d,window,M,pos0", [
+    ("fp32", 64, 16, 4, 0), ("fp32", 128, 128, 0, 3), ("fp32", 64, 5, 16, 1000),
+    ("bf16", 128, 128, 4, 127), ("bf16", 64, 33, 2, 32),
+])
+def test_decode_small_cases(lz, dtype, d, window, M, pos0):
+    w = Workload("dec", B=3, H=2, L=1, d=d, window=window, M=M, dtype=dtype, seed=pos0 + d,
+                 kind="decode", decode_pos=pos0)
+    inp = make_inputs(w)
+    if M == 0:
+        inp["meta_k"] = inp["meta_v"] = None
+    inp["alpha"] = random_alpha(2, seed=window)
+    inp["pos"] = torch.tensor([pos0, pos0 + 1, max(0, pos0 - 1)], dtype=torch.int64)
+    x = to_device(inp)
+    for step in range(3):
+        want = _oracle_step({k_: (v_.cpu() if v_ is not None else None) for k_, v_ in x.items()}, w)
+        o = _gpu_step(lz, x, w)
+        torch.cuda.synchronize()
+        check(f"o@{step}", o, want[0], dtype)
+        check(f"S@{step}", x["state"], want[1], "fp32")
+        assert torch.equal(x["pos"].cpu(), torch.from_numpy(want[4]))
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_decode_replay_equals_forward(lz, dtype):
+    """Prefill nothing, decode L tokens one by one: every output equals the
+    parallel forward at the same position (GPU vs GPU and vs the oracle)."""
+    B, H, L, d, window, M = 2, 2, 40, 64, 12, 4
+    w = Workload("replay", B=B, H=H, L=L, d=d, window=window, M=M, dtype=dtype, seed=77)
+    inp = make_inputs(w)
+    x = to_device(inp)
+    fwd = lz.attn_fwd(x["q"], x["k"], x["v"], x["g"], window=window, gate_temp=w.gate_temp,
+                      fmap_wq=x["fmap_wq"], fmap_wk=x["fmap_wk"], meta_k=x["meta_k"],
+                      meta_v=x["meta_v"], alpha=x["alpha"], want_state=True)
+    dt = x["q"].dtype
+    st = {"state": torch.zeros(B, H, d, d, device="cuda"),
+          "k_cache": torch.zeros(B, H, window, d, dtype=dt, device="cuda"),
+          "v_cache": torch.zeros(B, H, window, d, dtype=dt, device="cuda"),
+          "pos": torch.zeros(B, dtype=torch.int64, device="cuda")}
+    outs = []
+    for t in range(L):
+        step = {"q": x["q"][:, :, t].contiguous(), "k": x["k"][:, :, t].contiguous(),
+                "v": x["v"][:, :, t].contiguous(), "g": x["g"][:, :, t].contiguous(),
+                "fmap_wq": x["fmap_wq"], "fmap_wk": x["fmap_wk"], "meta_k": x["meta_k"],
+                "meta_v": x["meta_v"], "alpha": x["alpha"], **st}
+        outs.append(_gpu_step(lz, step, w))
+    dec = torch.stack(outs, 2)
+    torch.cuda.synchronize()
+    want = oracle_forward(inp, window=window, tau=w.gate_temp)
+    check("decode vs oracle", dec, want["o"], dtype)
+    check("forward vs oracle", fwd["o"], want["o"], dtype)
+    check("decode state", st["state"], want["state_out"], "fp32" if dtype == "fp32" else dtype)
+    assert torch.equal(st["pos"].cpu(), torch.full((B,), L, dtype=torch.int64))
