@@ -1,0 +1,55 @@
+// Forward with its scratch in a static device array, for callers that
+// cannot allocate device memory (see lizard_attn_fwd_noalloc in lizard.h).
+#include <mutex>
+
+#include "../../include/lizard.h"
+
+namespace {
+
+// The scratch every call of lizard_attn_fwd_noalloc uses.  A host-side use
+// of this name is only a stand-in for the symbol, never a device address:
+// the device address comes from cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[LIZARD_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+void *g_addr[kMaxDevices] = {};
+
+// Device address of the scratch on the current device, looked up once per
+// device with that device current.  Null on failure.
+void *scratch_address() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_addr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_addr[dev] = p;
+  }
+  return g_addr[dev];
+}
+
+}  // namespace
+
+extern "C" lizard_status lizard_attn_fwd_noalloc(const lizard_fwd_args *args, lizard_stream_t stream) {
+  if (!args) return LIZARD_ERR_INVALID_ARG;
+  const size_t need = lizard_fwd_workspace_size(args);
+  if (need == 0) {
+    // invalid arguments: let the regular checks name the error (nothing runs)
+    lizard_fwd_args a = *args;
+    a.workspace = nullptr;
+    a.workspace_bytes = 0;
+    return lizard_attn_fwd(&a, stream);
+  }
+  if (need > LIZARD_NOALLOC_SCRATCH_BYTES) return LIZARD_ERR_UNSUPPORTED;
+  void *scratch = scratch_address();
+  if (!scratch) return LIZARD_ERR_CUDA;
+  // The status word at the start of a workspace must start at zero; the
+  // rest of the scratch is written before it is read by every kernel.
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(scratch, 0, 256, s) != cudaSuccess) return LIZARD_ERR_CUDA;
+  lizard_fwd_args a = *args;
+  a.workspace = scratch;
+  a.workspace_bytes = LIZARD_NOALLOC_SCRATCH_BYTES;
+  return lizard_attn_fwd(&a, stream);
+}

@@ -205,6 +205,37 @@ typedef struct {
 
 lizard_status lizard_decode_step(const lizard_decode_args *args, lizard_stream_t stream);
 
+/*
+ * Forward for callers that cannot allocate device memory.
+ *
+ * Some callers have no way to obtain a device workspace: a plug-in living
+ * inside a host application that owns every device allocation and hands out
+ * only the tensors it already has, or a C client with a fixed device-memory
+ * budget that may not grow after start-up.  This entry point computes
+ * exactly what lizard_attn_fwd computes, but ignores args->workspace and
+ * args->workspace_bytes and uses a scratch array built into the library
+ * instead.  The paper has no counterpart to it: it only changes where the
+ * scratch lives.
+ *
+ *   - The scratch is a static device array of LIZARD_NOALLOC_SCRATCH_BYTES
+ *     bytes (32 MiB).  Every GPU that loads it keeps it until the process
+ *     exits.
+ *   - Calls whose forward needs more scratch than that (see
+ *     lizard_fwd_workspace_size) return LIZARD_ERR_UNSUPPORTED and launch
+ *     nothing.  With dk = dv = 128 that is above roughly 16K token-heads
+ *     (B * H * L) for the portable kernels.
+ *   - The first call on each device looks up the array's device address
+ *     (with that device current).  Make that first call before any stream
+ *     capture.
+ *   - No cudaMalloc, cudaFree or other allocating routine is called.
+ *   - All calls share the one array and it keeps the last call's contents.
+ *     Calls that overlap on the GPU (different streams, or different host
+ *     threads, without ordering between them) race on it.  Serialise them.
+ *   - Inputs and outputs are still the caller's, as in lizard_attn_fwd.
+ */
+#define LIZARD_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+lizard_status lizard_attn_fwd_noalloc(const lizard_fwd_args *args, lizard_stream_t stream);
+
 /* Waits for `stream`, then reads and clears the status word that kernels
  * with bounded waits leave at the start of a forward or backward workspace.
  * Returns LIZARD_OK or LIZARD_ERR_TIMEOUT (LIZARD_ERR_CUDA if the copy
