@@ -51,7 +51,14 @@ lizard_status check_fwd(const lizard_fwd_args *a) {
 bool gla_on(const lizard_fwd_args *a) { return a->branch != LIZARD_BRANCH_SWA_ONLY; }
 bool swa_on(const lizard_fwd_args *a) { return a->branch != LIZARD_BRANCH_GLA_ONLY; }
 
-// Forward workspace (portable path).
+// Kernel family the forward runs for these arguments.
+bool fwd_uses_tc(const lizard_fwd_args *a) {
+  const bool ok = lz::tc_fwd_supported(a->dk, a->dv, a->window, a->M, a->dtype == LIZARD_BF16);
+  if (a->impl == LIZARD_IMPL_TC) return ok;
+  return a->impl == LIZARD_IMPL_AUTO && ok;
+}
+
+// Forward workspace: the status header, plus fp32 scratch for the portable path.
 struct FwdLayout {
   size_t phq, phk, a, o_gla, total;
 };
@@ -60,7 +67,7 @@ FwdLayout fwd_layout(const lizard_fwd_args *a) {
   const size_t nd = up(N * a->dk * sizeof(float));
   FwdLayout l{};
   size_t off = kHeader;
-  if (gla_on(a)) {
+  if (gla_on(a) && !fwd_uses_tc(a)) {
     l.phq = off; off += nd;
     l.phk = off; off += nd;
     l.a = off; off += nd;
@@ -142,6 +149,14 @@ void fwd_plan(const lizard_fwd_args *a, void *ws, cudaStream_t s, Plan &plan) {
   const FwdLayout lay = fwd_layout(a);
   const int BH = a->B * a->H, D = a->dk;
   const bool bf16 = a->dtype == LIZARD_BF16;
+  if (fwd_uses_tc(a)) {
+    lz::TcFwdArgs t{a->q, a->k, a->v, a->g, a->fmap_wq, a->fmap_wk, a->meta_k, a->meta_v, a->alpha,
+                    a->state_in, a->o, gla_on(a) ? a->state_out : nullptr, swa_on(a) ? a->lse : nullptr,
+                    static_cast<uint32_t *>(ws), BH, a->H, a->L, a->M, a->window, a->branch,
+                    1.f / a->gate_temp, scale_of(a)};
+    plan.add("tc_fwd_kernel", [=] { return lz::launch_tc_fwd(t, s); });
+    return;
+  }
   float *o_gla = nullptr;
   if (gla_on(a)) {
     lz::PrepArgs pa{a->q, a->k, a->g, a->fmap_wq, a->fmap_wk, at<float>(ws, lay.phq), at<float>(ws, lay.phk),
@@ -222,7 +237,7 @@ size_t lizard_fwd_workspace_size(const lizard_fwd_args *args) {
 lizard_status lizard_attn_fwd(const lizard_fwd_args *a, lizard_stream_t stream) {
   lizard_status st = check_fwd(a);
   if (st != LIZARD_OK) return st;
-  if (a->impl == LIZARD_IMPL_TC) return LIZARD_ERR_UNSUPPORTED;
+  if (a->impl == LIZARD_IMPL_TC && !fwd_uses_tc(a)) return LIZARD_ERR_UNSUPPORTED;
   const FwdLayout lay = fwd_layout(a);
   if (!a->workspace || a->workspace_bytes < lay.total) return LIZARD_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -236,6 +251,7 @@ lizard_status lizard_attn_fwd(const lizard_fwd_args *a, lizard_stream_t stream) 
     }
     return LIZARD_OK;
   }
+  if (cudaMemsetAsync(a->workspace, 0, sizeof(uint32_t), s) != cudaSuccess) return LIZARD_ERR_CUDA;
   Plan plan;
   fwd_plan(a, a->workspace, s, plan);
   return plan.run(s, a->launch_events, a->n_launch_events);
@@ -304,6 +320,7 @@ lizard_status lizard_attn_bwd(const lizard_bwd_args *b, lizard_stream_t stream) 
     if (b->dstate_in && (e = cudaMemsetAsync(b->dstate_in, 0, BHdd, s)) != cudaSuccess) return LIZARD_ERR_CUDA;
   }
   if (a->L == 0) return LIZARD_OK;
+  if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), s) != cudaSuccess) return LIZARD_ERR_CUDA;
   Plan plan;
   bwd_plan(b, ws, s, plan);
   return plan.run(s, b->launch_events, b->n_launch_events);
@@ -356,7 +373,9 @@ lizard_status lizard_workspace_status(void *workspace, lizard_stream_t stream) {
   uint32_t word = 0;
   if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return LIZARD_ERR_CUDA;
   if (word != 0 && cudaMemset(workspace, 0, sizeof(word)) != cudaSuccess) return LIZARD_ERR_CUDA;
-  return word == 0 ? LIZARD_OK : LIZARD_ERR_TIMEOUT;
+  if (word & 1u) return LIZARD_ERR_TIMEOUT;
+  if (word & 2u) return LIZARD_ERR_RANGE;
+  return LIZARD_OK;
 }
 
 const char *lizard_status_string(lizard_status s) {
@@ -367,6 +386,7 @@ const char *lizard_status_string(lizard_status s) {
     case LIZARD_ERR_CUDA: return "CUDA launch or runtime error";
     case LIZARD_ERR_TIMEOUT: return "a kernel gave up on a bounded wait";
     case LIZARD_ERR_WORKSPACE: return "workspace missing or too small";
+    case LIZARD_ERR_RANGE: return "gate decay outside the tensor-core forward's range (use the portable kernels)";
   }
   return "unknown status";
 }

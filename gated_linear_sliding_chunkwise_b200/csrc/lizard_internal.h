@@ -91,11 +91,23 @@ struct FinishBwdArgs {
   float inv_tau;
 };
 
+struct TcFwdArgs {
+  const void *q, *k, *v, *g;
+  const float *wq, *wk, *meta_k, *meta_v, *alpha, *state_in;
+  void *o;
+  float *state_out, *lse;
+  uint32_t *status;   // workspace status word (bit 0 timeout, bit 1 range)
+  int BH, H, L, M, window, branch;
+  float inv_tau, scale;
+};
+
 constexpr int kBwdC = 32;   // GLA chunk used by the portable backward
 
 cudaError_t launch_prep(const PrepArgs &a, int BH, int D, bool bf16, cudaStream_t s);
 cudaError_t launch_gla_fwd_simt(const GlaFwdArgs &a, int BH, int D, bool bf16, cudaStream_t s);
 cudaError_t launch_swa_mix_simt(const SwaMixArgs &a, int BH, int D, bool bf16, cudaStream_t s);
+bool tc_fwd_supported(int dk, int dv, int window, int M, bool bf16);
+cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs &a, int B, int D, bool bf16, int64_t *pos, cudaStream_t s);
 
 cudaError_t launch_gla_states(const GlaStatesArgs &a, int BH, int D, bool bf16, cudaStream_t s);

@@ -1,0 +1,551 @@
+// Tensor-core (tcgen05 / TMEM / TMA) forward of the Lizard hybrid layer,
+// bf16 activations, dk = dv = 128, window <= 128, M <= 16.
+//
+// One CTA (128 threads, one TMEM lane per thread) walks one (batch, head)
+// sequence in tiles of T = 128 tokens, i.e. two 64-token chunks per tile with
+// the cumulative gate absorbed once per tile.  Per tile:
+//
+//   TMA     X_q, X_k, V, G (gate logits) of the tile and K of the previous
+//           tile, 128-byte swizzled; later V of the previous tile.
+//   MMA 1   L  = X_q [K_prev ; X_k]^T            (window logits, 128 x 256)
+//           Zq = X_q W_q, Zk = X_k W_k           (feature-map projections)
+//   gates   thread = key dimension i, tokens in reverse:
+//             acc_t = sum_{s>t} -a_s,  E_t = exp(acc_t) = exp(b_t - r)
+//           written as bf16 over G; exp(r) = exp(-acc_{-1}) decays the state.
+//   rows    thread = token t:
+//             anchor softmax over the 256 logits (band mask) and the M meta
+//             logits -> P^ = exp(l - max), unnormalised, into TMEM;
+//             phi_q, phi_k from Zq, Zk; Qt = phi_q E l/alpha (TMEM),
+//             Kt = phi_k / E (shared memory);
+//           thread = key dimension i: S' = diag(exp r) S in TMEM, and its
+//           bf16 copy in shared memory.
+//   MMA 2   A  = Qt Kt^T
+//   rows    A^ = tril(A) (TMEM; l/alpha comes in through Qt)
+//   MMA 3   O  = Qt S' + A^ V + P^ [V_prev ; V];   S = S' + Kt^T V
+//   store   o = O alpha/l + (alpha/l) sum_m p_m mv_m
+//
+// Scaling the GLA operands by l/alpha lets one accumulator hold both
+// branches: o = o_gla + alpha o_swa = (alpha/l) (o_gla l/alpha + P^ V).
+// (English gist.science summary, section 2.A: state update, anchor window
+// attention with meta tokens, final mix; Chinese summary, section 2.3: gate
+// absorbed into q and k in log space so the core runs as bf16 GEMMs.)
+//
+// A tile whose in-tile log-decay spread exceeds kMaxSpread in some key
+// dimension sets the RANGE bit of the workspace status word (the portable
+// path computes such inputs exactly).  Every mbarrier wait is bounded; a
+// wait that gives up sets the TIMEOUT bit and the CTA stops, frees its TMEM
+// and returns.
+#include "common.cuh"
+#include "lizard_internal.h"
+#include "tc_common.cuh"
+#include "tc_host.h"
+
+namespace lz {
+namespace {
+
+using namespace tc;
+
+constexpr int T = 128;             // tokens per tile
+constexpr int D = 128;             // dk = dv
+constexpr int F = D / 2;           // feature-map width per half
+constexpr uint32_t REG = 16384;    // one 64-column swizzled region of a 128-row tile
+constexpr uint32_t TILE = 2 * REG; // a 128 x 128 bf16 tile
+constexpr int MAXM = 16;
+
+// shared-memory regions (offsets from the 1024-aligned base)
+constexpr uint32_t R_XQ = 0;            // X_q, then S' (bf16, MN-major)
+constexpr uint32_t R_XK = 1 * TILE;     // X_k, then Kt
+constexpr uint32_t R_KP = 2 * TILE;     // K of the previous tile
+constexpr uint32_t R_V = 3 * TILE;      // V
+constexpr uint32_t R_G = 4 * TILE;      // G, then E, then V of the previous tile
+constexpr uint32_t R_WQ = 5 * TILE;     // W_q bf16, [dk rows][64 features], MN-major
+constexpr uint32_t R_WK = 5 * TILE + REG;
+constexpr uint32_t SMEM_TILES = 5 * TILE + 2 * REG;
+constexpr size_t SMEM_BYTES = SMEM_TILES + 1024;   // + alignment slack
+
+// TMEM columns
+constexpr uint32_t C_S = 0, C_O = 128, C_ZQ = 128, C_ZK = 192, C_A = 128;
+constexpr uint32_t C_L = 256, C_P = 256, C_QT = 384, C_AH = 448;
+
+constexpr uint32_t ST_TIMEOUT = 1u, ST_RANGE = 2u;
+
+struct Params {
+  CUtensorMap mq, mk, mv, mg;
+  const float *wq, *wk, *meta_k, *meta_v, *alpha, *state_in;
+  __nv_bfloat16 *o;
+  float *state_out, *lse;
+  uint32_t *status;
+  int H, L, M, window, branch;
+  float inv_tau, scale;
+};
+
+// 16-byte chunk c (8 consecutive columns 8c..8c+7) of row `row`
+__device__ __forceinline__ uint4 *chunk_ptr(unsigned char *base, uint32_t region_off, int row, int c) {
+  return reinterpret_cast<uint4 *>(base + region_off + (c >> 3) * REG + sw128_offset(row, (c & 7) * 8));
+}
+
+__device__ __forceinline__ void unpack8(const uint4 &u, float *f) {
+  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 v = __bfloat1622float2(h[i]);
+    f[2 * i] = v.x;
+    f[2 * i + 1] = v.y;
+  }
+}
+__device__ __forceinline__ uint4 pack8(const float *f) {
+  uint4 u;
+  u.x = pack_bf16(f[0], f[1]);
+  u.y = pack_bf16(f[2], f[3]);
+  u.z = pack_bf16(f[4], f[5]);
+  u.w = pack_bf16(f[6], f[7]);
+  return u;
+}
+
+// K-major operand descriptor, k-step s (16 columns) of a 128-row tile
+__device__ __forceinline__ uint64_t desc_k(uint32_t tile_addr, int s) {
+  return sdesc_sw128(tile_addr + (s >> 2) * REG + (s & 3) * 32, 0, 1024);
+}
+// MN-major operand descriptor, k-step s (16 rows) of a tile whose rows are K
+// and whose two 64-column regions are M/N blocks
+__device__ __forceinline__ uint64_t desc_mn(uint32_t tile_addr, int s) {
+  return sdesc_sw128(tile_addr + s * 2048, REG, 1024);
+}
+
+__device__ __forceinline__ void issue_tile_loads(const Params &p, unsigned char *sm, uint64_t *bar, int bh,
+                                                 int t0) {
+  mbar_expect_tx(bar, 5 * TILE);
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    tma_load_3d(sm + R_XQ + r * REG, &p.mq, bar, 64 * r, t0, bh);
+    tma_load_3d(sm + R_XK + r * REG, &p.mk, bar, 64 * r, t0, bh);
+    tma_load_3d(sm + R_KP + r * REG, &p.mk, bar, 64 * r, t0 - T, bh);
+    tma_load_3d(sm + R_V + r * REG, &p.mv, bar, 64 * r, t0, bh);
+    tma_load_3d(sm + R_G + r * REG, &p.mg, bar, 64 * r, t0, bh);
+  }
+}
+
+// phi(x) = [softmax(z), softmax(-z)] of the 64 projections z of this
+// thread's row: z is overwritten with the first half, neg gets the second.
+__device__ __forceinline__ void feature_map_row(float *z, float *neg) {
+  float mx = z[0], mn = z[0];
+#pragma unroll
+  for (int f = 1; f < F; ++f) { mx = fmaxf(mx, z[f]); mn = fminf(mn, z[f]); }
+  float sp = 0.f, sn = 0.f;
+#pragma unroll
+  for (int f = 0; f < F; ++f) {
+    neg[f] = __expf(mn - z[f]);
+    z[f] = __expf(z[f] - mx);
+    sp += z[f];
+    sn += neg[f];
+  }
+  const float ip = 1.f / sp, in_ = 1.f / sn;
+#pragma unroll
+  for (int f = 0; f < F; ++f) { z[f] *= ip; neg[f] *= in_; }
+}
+
+__global__ void __launch_bounds__(128, 1) tc_fwd_kernel(const __grid_constant__ Params p) {
+  extern __shared__ unsigned char smraw[];
+  unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
+  __shared__ float s_mk[MAXM][D], s_mv[MAXM][D];
+  __shared__ float s_dec[D];
+  __shared__ uint64_t bar_tma, bar_vp, bar_m1, bar_m2, bar_m3;
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_fail;
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int row = tid;                                 // TMEM lane == tile row
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const int bh = blockIdx.x, h = bh % p.H;
+  const float alpha = p.alpha ? p.alpha[h] : 1.f;
+  const bool gla = p.branch != 2, swa = p.branch != 1;
+  const uint32_t sbase = smem_u32(sm);
+
+  if (warp == 0) {
+    tmem_alloc(&s_tmem, 512);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(&bar_tma, 1);
+    mbar_init(&bar_vp, 1);
+    mbar_init(&bar_m1, 1);
+    mbar_init(&bar_m2, 1);
+    mbar_init(&bar_m3, 1);
+    fence_barrier_init();
+    s_fail = 0;
+  }
+  // feature-map weights -> bf16, MN-major [dk row][feature]
+  {
+    const int i = row;
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      const float *W = m == 0 ? p.wq : p.wk;
+      const uint32_t reg = m == 0 ? R_WQ : R_WK;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        float f[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) f[u] = W ? W[((size_t)h * D + i) * F + c * 8 + u] : 0.f;
+        *reinterpret_cast<uint4 *>(sm + reg + sw128_offset(i, c * 8)) = pack8(f);
+      }
+    }
+  }
+  for (int e = tid; e < p.M * D; e += 128) {
+    s_mk[e / D][e % D] = p.meta_k[(size_t)h * p.M * D + e];
+    s_mv[e / D][e % D] = p.meta_v ? p.meta_v[(size_t)h * p.M * D + e] : 0.f;
+  }
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = s_tmem;
+
+  // initial state -> TMEM columns [0, 128), lane = key dimension
+  {
+    const float *src = p.state_in ? p.state_in + ((size_t)bh * D + row) * D : nullptr;
+#pragma unroll
+    for (int c = 0; c < D; c += 8) {
+      uint32_t r[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(src ? src[c + u] : 0.f);
+      tmem_st8(tb + lane_off + C_S + c, r);
+    }
+    tmem_st_wait();
+  }
+
+  const int ntiles = (p.L + T - 1) / T;
+  uint32_t *err = p.status;
+  if (tid == 0 && ntiles > 0) issue_tile_loads(p, sm, &bar_tma, bh, 0);
+  const uint32_t id_128 = idesc_bf16(128, 128, 0, 0);
+  const uint32_t id_z = idesc_bf16(128, 64, 0, 1);
+  const uint32_t id_mn = idesc_bf16(128, 128, 0, 1);
+  const uint32_t id_st = idesc_bf16(128, 128, 1, 1);
+
+  for (int c = 0; c < ntiles; ++c) {
+    const uint32_t par = c & 1;
+    const int t0 = c * T;
+    const int tq = t0 + row;                  // this thread's query token
+    const bool qvalid = tq < p.L;
+
+    // ---------------------------------------------------------- MMA 1 ---
+    bool ok = mbar_wait(&bar_tma, par, err, ST_TIMEOUT);
+    if (__syncthreads_or(!ok)) { s_fail = 1; break; }
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t xq = sbase + R_XQ, xk = sbase + R_XK, kp = sbase + R_KP;
+      if (swa) {
+        for (int s = 0; s < 8; ++s) mma_ss(tb + C_L, desc_k(xq, s), desc_k(kp, s), id_128, s > 0);
+        for (int s = 0; s < 8; ++s) mma_ss(tb + C_L + 128, desc_k(xq, s), desc_k(xk, s), id_128, s > 0);
+      }
+      for (int s = 0; s < 8; ++s) mma_ss(tb + C_ZQ, desc_k(xq, s), desc_mn(sbase + R_WQ, s), id_z, s > 0);
+      for (int s = 0; s < 8; ++s) mma_ss(tb + C_ZK, desc_k(xk, s), desc_mn(sbase + R_WK, s), id_z, s > 0);
+      mma_commit(&bar_m1);
+    }
+
+    // ---------------------------------------------- gates (thread = dim) ---
+    {
+      const int i = row;
+      float acc = 0.f, spread = 0.f;
+      for (int t = T - 1; t >= 0; --t) {
+        __nv_bfloat16 *gp = reinterpret_cast<__nv_bfloat16 *>(sm + R_G + (i >> 6) * REG + sw128_offset(t, i & 63));
+        const float a = (t0 + t < p.L) ? log_decay(__bfloat162float(*gp), p.inv_tau) : 0.f;
+        *gp = __float2bfloat16_rn(__expf(acc));   // E_t = exp(b_t - r)
+        if (t == 0) spread = acc;
+        acc -= a;
+      }
+      s_dec[i] = __expf(-acc);                     // exp(r): the tile's total decay
+      if (spread > kMaxSpread && gla) atomicOr(err, ST_RANGE);
+    }
+
+    ok = mbar_wait(&bar_m1, par, err, ST_TIMEOUT);
+    if (__syncthreads_or(!ok)) { s_fail = 1; break; }
+    tc_fence_after();
+
+    // ------------------------------------------- rows: anchor softmax ---
+    float lsum = 1.f, mx = 0.f;           // row normaliser and max (scaled logits)
+    float em[MAXM];                       // exp(meta logit - max)
+#pragma unroll
+    for (int m = 0; m < MAXM; ++m) em[m] = 0.f;
+    if (swa) {
+      float ml[MAXM];
+      mx = kNegBig;
+#pragma unroll
+      for (int m = 0; m < MAXM; ++m) ml[m] = 0.f;
+      for (int ch = 0; ch < 16; ++ch) {
+        float q8[8];
+        unpack8(*chunk_ptr(sm, R_XQ, row, ch), q8);
+#pragma unroll
+        for (int m = 0; m < MAXM; ++m) {
+          if (m < p.M) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) ml[m] = fmaf(q8[u], s_mk[m][ch * 8 + u], ml[m]);
+          }
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < MAXM; ++m) {
+        if (m < p.M) {
+          ml[m] *= p.scale;
+          mx = fmaxf(mx, ml[m]);
+        }
+      }
+      const int jlo = max(tq - p.window + 1, 0);     // valid keys j in [jlo, tq]
+      for (int ch = 0; ch < 16; ++ch) {
+        float v[16];
+        tmem_ld16(tb + lane_off + C_L + ch * 16, v);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int j = t0 - T + ch * 16 + u;
+          if (j >= jlo && j <= tq) mx = fmaxf(mx, v[u] * p.scale);
+        }
+      }
+      lsum = 0.f;
+      for (int ch = 0; ch < 16; ++ch) {
+        float v[16];
+        tmem_ld16(tb + lane_off + C_L + ch * 16, v);
+        uint32_t pk[8];
+#pragma unroll
+        for (int u = 0; u < 16; u += 2) {
+          const int j = t0 - T + ch * 16 + u;
+          const float e0 = (j >= jlo && j <= tq) ? __expf(v[u] * p.scale - mx) : 0.f;
+          const float e1 = (j + 1 >= jlo && j + 1 <= tq) ? __expf(v[u + 1] * p.scale - mx) : 0.f;
+          lsum += e0 + e1;
+          pk[u / 2] = alpha != 0.f ? pack_bf16(e0, e1) : 0u;
+        }
+        tmem_st8(tb + lane_off + C_P + ch * 8, pk);
+      }
+#pragma unroll
+      for (int m = 0; m < MAXM; ++m) {
+        if (m < p.M) {
+          em[m] = __expf(ml[m] - mx);
+          lsum += em[m];
+        }
+      }
+      if (!qvalid) lsum = 1.f;
+    }
+    // GLA operands carry l/alpha so that one accumulator holds both terms
+    const bool mixed = swa && alpha != 0.f;
+    const float gscale = mixed ? lsum / alpha : 1.f;
+    const float oscale = mixed ? alpha / lsum : 1.f;
+    const float mscale = mixed ? alpha / lsum : 0.f;   // meta-value weight per em
+
+    // -------------------------------------------- rows: feature maps ---
+    {
+      float z[F], neg[F];
+      // phi_q -> Qt = phi_q E gscale, packed bf16 pairs into TMEM
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) tmem_ld16(tb + lane_off + C_ZQ + ch * 16, z + ch * 16);
+      feature_map_row(z, neg);
+#pragma unroll
+      for (int c16 = 0; c16 < 8; ++c16) {     // 16 dims = 8 TMEM columns
+        float e16[16];
+        unpack8(*chunk_ptr(sm, R_G, row, 2 * c16), e16);
+        unpack8(*chunk_ptr(sm, R_G, row, 2 * c16 + 1), e16 + 8);
+        uint32_t r8[8];
+#pragma unroll
+        for (int u = 0; u < 16; u += 2) {
+          const int i = c16 * 16 + u;
+          const float ph0 = i < F ? z[i] : neg[i - F];
+          const float ph1 = i + 1 < F ? z[i + 1] : neg[i + 1 - F];
+          r8[u / 2] = pack_bf16(ph0 * e16[u] * gscale, ph1 * e16[u + 1] * gscale);
+        }
+        tmem_st8(tb + lane_off + C_QT + c16 * 8, r8);
+      }
+      // phi_k -> Kt = phi_k / E, bf16 into shared memory over X_k
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) tmem_ld16(tb + lane_off + C_ZK + ch * 16, z + ch * 16);
+      feature_map_row(z, neg);
+#pragma unroll
+      for (int c8 = 0; c8 < 16; ++c8) {
+        float e8[8], k8[8];
+        unpack8(*chunk_ptr(sm, R_G, row, c8), e8);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = c8 * 8 + u;
+          const float ph = i < F ? z[i] : neg[i - F];
+          k8[u] = ph * __frcp_rn(e8[u]);
+        }
+        *chunk_ptr(sm, R_XK, row, c8) = pack8(k8);
+      }
+    }
+
+    // ------------------------------- state rescale (thread = dimension) ---
+    if (gla) {
+      const int i = row;
+      const float dec = s_dec[i];
+      for (int c16 = 0; c16 < 8; ++c16) {
+        float v[16];
+        tmem_ld16(tb + lane_off + C_S + c16 * 16, v);
+        uint32_t r[8];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) v[u] *= dec;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(v[u]);
+        tmem_st8(tb + lane_off + C_S + c16 * 16, r);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(v[8 + u]);
+        tmem_st8(tb + lane_off + C_S + c16 * 16 + 8, r);
+        // bf16 copy S'[i][v], MN-major: rows = i (K of the O = Qt S' product)
+        *chunk_ptr(sm, R_XQ, i, 2 * c16) = pack8(v);
+        *chunk_ptr(sm, R_XQ, i, 2 * c16 + 1) = pack8(v + 8);
+      }
+    }
+    tmem_st_wait();
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+
+    // ---------------------------------------------------------- MMA 2 ---
+    if (tid == 0) {
+      tc_fence_after();
+      if (gla)
+        for (int s = 0; s < 8; ++s) mma_ts(tb + C_A, tb + C_QT + s * 8, desc_k(sbase + R_XK, s), id_128, s > 0);
+      mma_commit(&bar_m2);
+      // V of the previous tile into the G region (E has been consumed)
+      mbar_expect_tx(&bar_vp, TILE);
+      tma_load_3d(sm + R_G, &p.mv, &bar_vp, 0, t0 - T, bh);
+      tma_load_3d(sm + R_G + REG, &p.mv, &bar_vp, 64, t0 - T, bh);
+    }
+    ok = mbar_wait(&bar_m2, par, err, ST_TIMEOUT);
+    if (__syncthreads_or(!ok)) { s_fail = 1; break; }
+    tc_fence_after();
+
+    // ------------------------------------------ rows: masked intra A ---
+    if (gla) {
+      for (int c16 = 0; c16 < 8; ++c16) {
+        float v[16];
+        tmem_ld16(tb + lane_off + C_A + c16 * 16, v);
+        uint32_t r[8];
+#pragma unroll
+        for (int u = 0; u < 16; u += 2) {
+          const int j = c16 * 16 + u;        // tile-local key index
+          // A = Qt Kt^T already carries l/alpha through Qt
+          const float a0 = (j <= row) ? v[u] : 0.f;
+          const float a1 = (j + 1 <= row) ? v[u + 1] : 0.f;
+          r[u / 2] = pack_bf16(a0, a1);
+        }
+        tmem_st8(tb + lane_off + C_AH + c16 * 8, r);
+      }
+    }
+    tmem_st_wait();
+    tc_fence_before();
+    ok = mbar_wait(&bar_vp, par, err, ST_TIMEOUT);
+    if (__syncthreads_or(!ok)) { s_fail = 1; break; }
+
+    // ---------------------------------------------------------- MMA 3 ---
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t sp = sbase + R_XQ, v = sbase + R_V, vp = sbase + R_G, kt = sbase + R_XK;
+      uint32_t accum = 0;
+      if (gla) {
+        for (int s = 0; s < 8; ++s) { mma_ts(tb + C_O, tb + C_QT + s * 8, desc_mn(sp, s), id_mn, accum); accum = 1; }
+        for (int s = 0; s < 8; ++s) mma_ts(tb + C_O, tb + C_AH + s * 8, desc_mn(v, s), id_mn, 1);
+      }
+      if (swa) {
+        for (int s = 0; s < 8; ++s) { mma_ts(tb + C_O, tb + C_P + s * 8, desc_mn(vp, s), id_mn, accum); accum = 1; }
+        for (int s = 0; s < 8; ++s) mma_ts(tb + C_O, tb + C_P + 64 + s * 8, desc_mn(v, s), id_mn, 1);
+      }
+      if (gla)
+        for (int s = 0; s < 8; ++s) mma_ss(tb + C_S, desc_mn(kt, s), desc_mn(v, s), id_st, 1);
+      mma_commit(&bar_m3);
+    }
+    ok = mbar_wait(&bar_m3, par, err, ST_TIMEOUT);
+    if (__syncthreads_or(!ok)) { s_fail = 1; break; }
+    tc_fence_after();
+    if (tid == 0 && c + 1 < ntiles) issue_tile_loads(p, sm, &bar_tma, bh, t0 + T);
+
+    // -------------------------------------------------------- epilogue ---
+    {
+      // tcgen05.ld is warp-collective: every lane loads, valid rows store
+      __nv_bfloat16 *orow = p.o + ((size_t)bh * p.L + (qvalid ? tq : 0)) * D;
+      for (int c16 = 0; c16 < 8; ++c16) {
+        float v[16];
+        tmem_ld16(tb + lane_off + C_O + c16 * 16, v);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) v[u] *= oscale;
+        if (swa && p.meta_v) {
+#pragma unroll
+          for (int m = 0; m < MAXM; ++m) {
+            if (m < p.M) {
+              const float w = mscale * em[m];
+#pragma unroll
+              for (int u = 0; u < 16; ++u) v[u] = fmaf(w, s_mv[m][c16 * 16 + u], v[u]);
+            }
+          }
+        }
+        if (qvalid) {
+          uint4 *dst = reinterpret_cast<uint4 *>(orow + c16 * 16);
+          dst[0] = pack8(v);
+          dst[1] = pack8(v + 8);
+        }
+      }
+      if (qvalid && p.lse && swa) p.lse[(size_t)bh * p.L + tq] = mx + logf(lsum);
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
+
+  if (!s_fail && p.state_out && gla) {
+    tc_fence_after();
+    float *dst = p.state_out + ((size_t)bh * D + row) * D;
+    for (int c16 = 0; c16 < 8; ++c16) {
+      float v[16];
+      tmem_ld16(tb + lane_off + C_S + c16 * 16, v);
+#pragma unroll
+      for (int u = 0; u < 16; u += 4) *reinterpret_cast<float4 *>(dst + c16 * 16 + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
+    }
+  }
+  if (s_fail && tid == 0) {
+    // let whatever was issued drain before the shared memory is released
+    mbar_wait(&bar_tma, 0, nullptr, 0, 1u << 16);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tb, 512);
+}
+
+}  // namespace
+
+bool tc_fwd_supported(int dk, int dv, int window, int M, bool bf16) {
+  return bf16 && dk == D && dv == D && window <= T && M <= MAXM;
+}
+
+cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t s) {
+  Params p;
+  memset(&p, 0, sizeof(p));
+  const uint64_t rows = (uint64_t)a.L;
+  if (!make_map_bf16_3d(&p.mq, a.q, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mk, a.k, D, rows, a.BH, T) ||
+      !make_map_bf16_3d(&p.mv, a.v, D, rows, a.BH, T) ||
+      !make_map_bf16_3d(&p.mg, a.g ? a.g : a.q, D, rows, a.BH, T))   // g unused without the GLA branch
+    return cudaErrorInvalidValue;
+  p.wq = a.wq;
+  p.wk = a.wk;
+  p.meta_k = a.meta_k;
+  p.meta_v = a.meta_v;
+  p.alpha = a.alpha;
+  p.state_in = a.state_in;
+  p.o = static_cast<__nv_bfloat16 *>(a.o);
+  p.state_out = a.state_out;
+  p.lse = a.lse;
+  p.status = a.status;
+  p.H = a.H;
+  p.L = a.L;
+  p.M = a.M;
+  p.window = a.window;
+  p.branch = a.branch;
+  p.inv_tau = a.inv_tau;
+  p.scale = a.scale;
+  static size_t configured[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || configured[dev] < SMEM_BYTES) {
+    e = cudaFuncSetAttribute(tc_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) configured[dev] = SMEM_BYTES;
+  }
+  tc_fwd_kernel<<<a.BH, 128, SMEM_BYTES, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace lz

@@ -37,9 +37,15 @@
  *   - Supported: dk = dv in {64, 128}; chunk = 64; window >= 1; 0 <= M <= 16;
  *     L >= 0 (L = 0 is a no-op); B * H >= 1.  Other sizes return
  *     LIZARD_ERR_UNSUPPORTED.
- *   - Launch errors return LIZARD_ERR_CUDA.  A kernel that gives up on a
- *     bounded wait records LIZARD_ERR_TIMEOUT in the workspace status word,
- *     which lizard_workspace_status() reads back.
+ *   - Launch errors return LIZARD_ERR_CUDA.  Errors found on the device are
+ *     recorded in a status word at the start of the workspace, cleared at the
+ *     start of every forward or backward call and read back by
+ *     lizard_workspace_status(): a kernel that gives up on a bounded wait
+ *     records LIZARD_ERR_TIMEOUT; the tensor-core forward records
+ *     LIZARD_ERR_RANGE when, inside one 128-token tile, the cumulative
+ *     log-decay of some key dimension spans more than 64 (gate logits below
+ *     about -8 per token at gate_temp 16); such inputs need LIZARD_IMPL_SIMT,
+ *     which computes them exactly.
  */
 #ifndef LIZARD_H_
 #define LIZARD_H_
@@ -59,7 +65,8 @@ typedef enum {
   LIZARD_ERR_UNSUPPORTED = 2, /* well-formed but outside the supported sizes */
   LIZARD_ERR_CUDA = 3,        /* a launch or CUDA runtime call failed */
   LIZARD_ERR_TIMEOUT = 4,     /* a kernel gave up on a bounded wait */
-  LIZARD_ERR_WORKSPACE = 5    /* workspace NULL or smaller than the queried size */
+  LIZARD_ERR_WORKSPACE = 5,   /* workspace NULL or smaller than the queried size */
+  LIZARD_ERR_RANGE = 6        /* the tensor-core forward met a gate decay outside its range */
 } lizard_status;
 
 typedef enum { LIZARD_BF16 = 0, LIZARD_FP32 = 1 } lizard_dtype;
@@ -71,7 +78,8 @@ enum { LIZARD_BRANCH_BOTH = 0, LIZARD_BRANCH_GLA_ONLY = 1, LIZARD_BRANCH_SWA_ONL
 enum {
   LIZARD_IMPL_AUTO = 0,  /* tensor-core path where it applies, else portable */
   LIZARD_IMPL_SIMT = 1,  /* portable fp32 CUDA-core kernels (exact fp32 math) */
-  LIZARD_IMPL_TC = 2     /* tcgen05/TMEM tensor-core kernels (bf16, dk = 128) */
+  LIZARD_IMPL_TC = 2     /* tcgen05/TMEM tensor-core kernels: forward only,
+                            bf16, dk = dv = 128, window <= 128, M <= 16 */
 };
 
 /*
@@ -236,10 +244,10 @@ lizard_status lizard_decode_step(const lizard_decode_args *args, lizard_stream_t
 #define LIZARD_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
 lizard_status lizard_attn_fwd_noalloc(const lizard_fwd_args *args, lizard_stream_t stream);
 
-/* Waits for `stream`, then reads and clears the status word that kernels
- * with bounded waits leave at the start of a forward or backward workspace.
- * Returns LIZARD_OK or LIZARD_ERR_TIMEOUT (LIZARD_ERR_CUDA if the copy
- * fails).  `workspace` is a device pointer. */
+/* Waits for `stream`, then reads and clears the status word that the last
+ * forward or backward call left at the start of `workspace` (a device
+ * pointer).  Returns LIZARD_OK, LIZARD_ERR_TIMEOUT or LIZARD_ERR_RANGE
+ * (LIZARD_ERR_CUDA if the copy fails). */
 lizard_status lizard_workspace_status(void *workspace, lizard_stream_t stream);
 
 /* Static description of a status code; never NULL. */

@@ -70,7 +70,7 @@ def test_struct_layouts_match_c(lz, tmp_path):
 
 
 def test_status_strings_and_version(lz):
-    for code in range(6):
+    for code in range(7):
         assert lz.status_string(code)
     assert lz.status_string(99) == "unknown status"
     assert re.match(r"\d+\.\d+\.\d+$", lz.version())

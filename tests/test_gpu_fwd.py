@@ -26,17 +26,24 @@ def _run(lz, x, w, impl, **kw):
                        state_in=x.get("state_in"), impl=impl, **kw)
 
 
-IMPLS = ["simt"]
+IMPLS = ["simt", "tc"]
 
 
 def _impl(lz, name):
     return {"simt": lz.IMPL_SIMT, "tc": lz.IMPL_TC, "auto": lz.IMPL_AUTO}[name]
 
 
+def _skip_unsupported(impl, dtype, d, window, M):
+    """The tensor-core forward covers bf16, d = 128, window <= 128, M <= 16."""
+    if impl == "tc" and not (dtype == "bf16" and d == 128 and window <= 128 and M <= 16):
+        pytest.skip("shape outside the tensor-core forward")
+
+
 @pytest.mark.parametrize("impl", IMPLS)
 def test_tiny_fp32_full(lz, impl):
     """The tiny fp32 workload, every output, max abs error <= 1e-4."""
     w = WORKLOADS["tiny_fp32"]
+    _skip_unsupported(impl, w.dtype, w.d, w.window, w.M)
     inp = make_inputs(w)
     x = to_device(inp)
     got = _run(lz, x, w, _impl(lz, impl), want_state=True, want_lse=True)
@@ -64,6 +71,7 @@ SWEEP = [
 def test_forward_sweep(lz, impl, dtype, d, L, window, M, with_mv, with_state, rand_alpha):
     """Ragged lengths, windows shorter/longer than a chunk, with and without
     meta tokens, sink-only meta tokens, an initial state and random alpha."""
+    _skip_unsupported(impl, dtype, d, window, M)
     w = Workload("sweep", B=2, H=3, L=L, d=d, window=window, M=M, dtype=dtype, seed=11 + L)
     inp = make_inputs(w)
     if not with_mv:
@@ -75,6 +83,7 @@ def test_forward_sweep(lz, impl, dtype, d, L, window, M, with_mv, with_state, ra
     if rand_alpha:
         inp["alpha"] = random_alpha(3, seed=L)
     got = _run(lz, to_device(inp), w, _impl(lz, impl), want_state=True, want_lse=True)
+    assert lz.workspace_status(got["workspace"]) == lz.OK
     want = oracle_forward(inp, window=window, tau=w.gate_temp)
     check("o", got["o"], want["o"], dtype)
     check("state_out", got["state_out"], want["state_out"], "fp32" if dtype == "fp32" else dtype)
@@ -84,15 +93,41 @@ def test_forward_sweep(lz, impl, dtype, d, L, window, M, with_mv, with_state, ra
 @pytest.mark.parametrize("impl", IMPLS)
 @pytest.mark.parametrize("branch", [ref.BRANCH_GLA_ONLY, ref.BRANCH_SWA_ONLY])
 def test_branch_hooks(lz, impl, branch):
-    w = Workload("branch", B=1, H=2, L=150, d=64, window=20, M=4, dtype="fp32", seed=3)
+    dtype, d = ("fp32", 64) if impl == "simt" else ("bf16", 128)
+    w = Workload("branch", B=1, H=2, L=150, d=d, window=20, M=4, dtype=dtype, seed=3)
     inp = make_inputs(w)
     inp["alpha"] = random_alpha(2, seed=9)
     got = _run(lz, to_device(inp), w, _impl(lz, impl), branch=branch)
     want = oracle_forward(inp, window=w.window, tau=w.gate_temp, branch=branch)
-    check("o", got["o"], want["o"], "fp32")
+    check("o", got["o"], want["o"], dtype)
 
 
 @pytest.mark.parametrize("impl", IMPLS)
+def test_alpha_zero_drops_anchor_branch(lz, impl):
+    dtype, d = ("fp32", 64) if impl == "simt" else ("bf16", 128)
+    w = Workload("alpha0", B=1, H=2, L=200, d=d, window=64, M=4, dtype=dtype, seed=31)
+    inp = make_inputs(w)
+    inp["alpha"] = torch.tensor([0.0, 0.7])
+    got = _run(lz, to_device(inp), w, _impl(lz, impl))
+    want = oracle_forward(inp, window=w.window, tau=w.gate_temp)
+    check("o", got["o"], want["o"], dtype)
+
+
+def test_tc_flags_decay_outside_its_range(lz):
+    """Gate logits of -300 make one tile's cumulative decay span far more than
+    the tensor-core forward's range: it must say so in the status word."""
+    w = Workload("range", B=1, H=1, L=256, d=128, window=128, M=4, dtype="bf16", seed=2)
+    inp = make_inputs(w)
+    g = inp["g"].clone()
+    g[:, :, 130:200, :3] = -300.0
+    inp["g"] = g
+    got = _run(lz, to_device(inp), w, lz.IMPL_TC)
+    assert lz.workspace_status(got["workspace"]) == lz.ERR_RANGE
+    ok = _run(lz, to_device(make_inputs(w)), w, lz.IMPL_TC)
+    assert lz.workspace_status(ok["workspace"]) == lz.OK
+
+
+@pytest.mark.parametrize("impl", ["simt"])
 def test_extreme_decay_takes_exact_path(lz, impl):
     """Gate logits near -300 make the in-chunk decay spread exceed the
     log-space absorption's range; the result must still match."""
@@ -113,19 +148,20 @@ def test_extreme_decay_takes_exact_path(lz, impl):
 def test_segmented_equals_one_shot(lz, impl):
     """state_out of one segment fed as state_in of the next reproduces the
     one-shot forward (prefill handed over in pieces)."""
-    w = Workload("seg", B=2, H=2, L=300, d=128, window=50, M=4, dtype="fp32", seed=4)
+    dtype = "fp32" if impl == "simt" else "bf16"
+    w = Workload("seg", B=2, H=2, L=300, d=128, window=50, M=4, dtype=dtype, seed=4)
     inp = to_device(make_inputs(w))
     full = _run(lz, inp, w, _impl(lz, impl), want_state=True)
     cut = 137
     a = {k_: (v_[:, :, :cut].contiguous() if k_ in ("q", "k", "v", "g") else v_) for k_, v_ in inp.items()}
     b = {k_: (v_[:, :, cut:].contiguous() if k_ in ("q", "k", "v", "g") else v_) for k_, v_ in inp.items()}
-    wa = Workload("seg", B=2, H=2, L=cut, d=128, window=50, M=4, dtype="fp32")
+    wa = Workload("seg", B=2, H=2, L=cut, d=128, window=50, M=4, dtype=dtype)
     r1 = _run(lz, a, wa, _impl(lz, impl), branch=ref.BRANCH_GLA_ONLY, want_state=True)
     b["state_in"] = r1["state_out"]
     r2 = _run(lz, b, wa, _impl(lz, impl), branch=ref.BRANCH_GLA_ONLY, want_state=True)
     gla = _run(lz, inp, w, _impl(lz, impl), branch=ref.BRANCH_GLA_ONLY, want_state=True)
-    check("o", torch.cat([r1["o"], r2["o"]], 2), to64(gla["o"]), "fp32")
-    check("S", r2["state_out"], to64(full["state_out"]), "fp32")
+    check("o", torch.cat([r1["o"], r2["o"]], 2), to64(gla["o"]), dtype)
+    check("S", r2["state_out"], to64(full["state_out"]), dtype)
 
 
 def test_empty_sequence_passes_state_through(lz):

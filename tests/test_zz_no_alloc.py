@@ -47,6 +47,7 @@ def test_noalloc_rejects_sizes_beyond_its_scratch(lz):
     a = lz.FwdArgs()
     a.B, a.H, a.L, a.dk, a.dv, a.chunk, a.window, a.M = 8, 32, 2048, 128, 128, 64, 128, 0
     a.dtype, a.gate_temp = lz.BF16, 16.0
+    a.impl = lz.IMPL_SIMT     # the portable kernels keep fp32 scratch per token
     fake = 0x10000
     a.q = a.k = a.v = a.g = a.o = fake
     assert lz.fwd_workspace_bytes(a) > 32 << 20
