@@ -300,6 +300,8 @@ def run_ours(args, rank, world, local):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ems}
 
     decode = None if args.no_decode else run_decode(args, lz, dev, rank, world, peaks)
+    fwd_long = None if args.no_fwd_long else run_forward(args, lz, dev, rank, world, peaks,
+                                                         "long_fwd_16k", max(K, 5))
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
@@ -316,12 +318,57 @@ def run_ours(args, rank, world, local):
         "hbm_floor_ms": (N * by["train"]) / (peaks["hbm_gbs"] * 1e9) * 1e3,
         "roofline": roof, "kernel_ms": kernels,
         "gpu_launches": K * (len(fwd_names) + len(bwd_names)),
-        "clocks": clk, "e2e": e2e, "decode": decode,
+        "clocks": clk, "e2e": e2e, "decode": decode, "fwd_long_16k": fwd_long,
     }
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(inp, w, budget_s=args.cpu_budget)
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def run_forward(args, lz, dev, rank, world, peaks, name, steps):
+    """Time lizard_attn_fwd alone on one workload (inputs resident)."""
+    from gated_linear_sliding_chunkwise_b200.synth import WORKLOADS, make_inputs
+
+    w = WORKLOADS[name]
+    impl = {"auto": lz.IMPL_AUTO, "simt": lz.IMPL_SIMT, "tc": lz.IMPL_TC}[args.kernels]
+    inp = make_inputs(w, seed=w.seed + rank)
+    x = {k: v.to(dev).contiguous() for k, v in inp.items()}
+    kw = dict(window=w.window, chunk=w.chunk, gate_temp=w.gate_temp, fmap_wq=x["fmap_wq"],
+              fmap_wk=x["fmap_wk"], meta_k=x["meta_k"], meta_v=x["meta_v"], alpha=x["alpha"],
+              impl=impl)
+    names = lz.attn_fwd(x["q"], x["k"], x["v"], x["g"], plan_only=True, **kw)
+    o = torch.empty_like(x["q"])
+    ws = lz.attn_fwd(x["q"], x["k"], x["v"], x["g"], out=o, **kw)["workspace"]
+    for _ in range(max(args.warmup, 1)):
+        lz.attn_fwd(x["q"], x["k"], x["v"], x["g"], out=o, workspace=ws, **kw)
+    evs = [lz.make_events(len(names) + 1) for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for i in range(steps):
+        lz.attn_fwd(x["q"], x["k"], x["v"], x["g"], out=o, workspace=ws, events=evs[i], **kw)
+    e.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(s.elapsed_time(e) / steps, world, dev)
+    per = {n: statistics.mean(ev[j].elapsed_time(ev[j + 1]) for ev in evs) for j, n in enumerate(names)}
+    N = w.B * w.H * w.L
+    fl = flops_per_token_head(w.d, w.chunk, w.window, w.M)["fwd"] * N
+    by = bytes_per_token_head(w.d)["fwd"] * N
+    tfl = world * fl / (ms / 1e3) / 1e12
+    gbs = world * by / (ms / 1e3) / 1e9
+    out = {"workload": f"{name}: B={w.B} H={w.H} L={w.L} d={w.d}", "ms": ms,
+           "tokens_per_s": world * w.B * w.L / (ms / 1e3), "tflops": tfl,
+           "tflops_frac_of_bf16_peak": tfl / peaks["bf16_tflops"],
+           "hbm_gbs": gbs, "hbm_frac": gbs / (world * peaks["hbm_gbs"]),
+           "kernel_ms": {n: round(t, 4) for n, t in per.items()}, "launches": len(names)}
+    if len(names) == 1:
+        out["roofline"] = {"bound": "hbm", "achieved": by / (per[names[0]] / 1e3) / 1e9,
+                           "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                           "frac": by / (per[names[0]] / 1e3) / 1e9 / peaks["hbm_gbs"],
+                           "kernel": names[0]}
+    return out
 
 
 def run_decode(args, lz, dev, rank, world, peaks):
@@ -444,10 +491,21 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-fwd-long", action="store_true")
+    ap.add_argument("--only", choices=["train", "fwd"], default="train",
+                    help="fwd: time lizard_attn_fwd alone on --workload (profiling aid)")
+    ap.add_argument("--workload", default="llama8b_layer_fwd")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         print("note: --warmup below 3 is not a valid measurement", file=sys.stderr)
     rank, world, local = dist_env()
+    if args.only == "fwd":
+        # forward-only timing of one workload (used for kernel profiles)
+        from gated_linear_sliding_chunkwise_b200 import lizard as lz
+        dev = torch.device("cuda", local)
+        torch.cuda.set_device(dev)
+        print(json.dumps(run_forward(args, lz, dev, rank, 1, load_peaks(), args.workload, args.steps)))
+        return
     if world > 1:
         import torch.distributed as dist
         backend = "nccl" if torch.cuda.is_available() else "gloo"

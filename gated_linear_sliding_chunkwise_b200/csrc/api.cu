@@ -67,7 +67,10 @@ FwdLayout fwd_layout(const lizard_fwd_args *a) {
   const size_t nd = up(N * a->dk * sizeof(float));
   FwdLayout l{};
   size_t off = kHeader;
-  if (gla_on(a) && !fwd_uses_tc(a)) {
+  if (fwd_uses_tc(a)) {
+    l.phq = off;   // segment states of the tensor-core path
+    off += up(lz::tc_fwd_workspace_bytes(a->B * a->H, a->L));
+  } else if (gla_on(a)) {
     l.phq = off; off += nd;
     l.phk = off; off += nd;
     l.a = off; off += nd;
@@ -152,9 +155,13 @@ void fwd_plan(const lizard_fwd_args *a, void *ws, cudaStream_t s, Plan &plan) {
   if (fwd_uses_tc(a)) {
     lz::TcFwdArgs t{a->q, a->k, a->v, a->g, a->fmap_wq, a->fmap_wk, a->meta_k, a->meta_v, a->alpha,
                     a->state_in, a->o, gla_on(a) ? a->state_out : nullptr, swa_on(a) ? a->lse : nullptr,
-                    static_cast<uint32_t *>(ws), BH, a->H, a->L, a->M, a->window, a->branch,
-                    1.f / a->gate_temp, scale_of(a)};
-    plan.add("tc_fwd_kernel", [=] { return lz::launch_tc_fwd(t, s); });
+                    static_cast<uint32_t *>(ws), at<void>(ws, lay.phq), BH, a->H, a->L, a->M, a->window,
+                    a->branch, 1.f / a->gate_temp, scale_of(a)};
+    if (lz::tc_fwd_stage_count(BH, a->L) > 1) {
+      plan.add("tc_fwd_kernel(state pass)", [=] { return lz::launch_tc_fwd(t, 0, s); });
+      plan.add("seg_combine_kernel", [=] { return lz::launch_tc_fwd(t, 1, s); });
+    }
+    plan.add("tc_fwd_kernel", [=] { return lz::launch_tc_fwd(t, 2, s); });
     return;
   }
   float *o_gla = nullptr;

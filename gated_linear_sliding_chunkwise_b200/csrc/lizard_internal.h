@@ -97,6 +97,7 @@ struct TcFwdArgs {
   void *o;
   float *state_out, *lse;
   uint32_t *status;   // workspace status word (bit 0 timeout, bit 1 range)
+  void *seg_ws;       // segment states, tc_fwd_workspace_bytes() bytes (may be null when 0)
   int BH, H, L, M, window, branch;
   float inv_tau, scale;
 };
@@ -107,7 +108,10 @@ cudaError_t launch_prep(const PrepArgs &a, int BH, int D, bool bf16, cudaStream_
 cudaError_t launch_gla_fwd_simt(const GlaFwdArgs &a, int BH, int D, bool bf16, cudaStream_t s);
 cudaError_t launch_swa_mix_simt(const SwaMixArgs &a, int BH, int D, bool bf16, cudaStream_t s);
 bool tc_fwd_supported(int dk, int dv, int window, int M, bool bf16);
-cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t s);
+size_t tc_fwd_workspace_bytes(int BH, int L);
+int tc_fwd_stage_count(int BH, int L);
+// stage 0: state pass, 1: combine (both only when the sequence is split), 2: full pass
+cudaError_t launch_tc_fwd(const TcFwdArgs &a, int stage, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs &a, int B, int D, bool bf16, int64_t *pos, cudaStream_t s);
 
 cudaError_t launch_gla_states(const GlaStatesArgs &a, int BH, int D, bool bf16, cudaStream_t s);

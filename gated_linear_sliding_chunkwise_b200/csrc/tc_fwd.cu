@@ -30,6 +30,12 @@
 // attention with meta tokens, final mix; Chinese summary, section 2.3: gate
 // absorbed into q and k in log space so the core runs as bf16 GEMMs.)
 //
+// Long sequences with few (batch, head) pairs are split into segments so
+// that every SM has a sequence slice: a state pass (the same kernel in
+// mode 1: gates, phi_k, state update only) gives each segment's local end
+// state and total log-decay, a combine kernel chains them into each
+// segment's start state, and the full pass runs all segments in parallel.
+//
 // A tile whose in-tile log-decay spread exceeds kMaxSpread in some key
 // dimension sets the RANGE bit of the workspace status word (the portable
 // path computes such inputs exactly).  Every mbarrier wait is bounded; a
@@ -75,9 +81,19 @@ struct Params {
   __nv_bfloat16 *o;
   float *state_out, *lse;
   uint32_t *status;
+  const float *seg_start;   // [BH][nseg][D][D] start state of each segment (nseg > 1)
+  float *seg_state;         // mode 1: [BH][nseg][D][D] local end state (zero start)
+  float *seg_decay;         // mode 1: [BH][nseg][D] summed log-decay of the segment
   int H, L, M, window, branch;
+  int mode;                 // 0: full forward, 1: state pass
+  int nseg, tiles_per_seg;
   float inv_tau, scale;
 };
+
+// logsigmoid(g) / tau with the fast exp/log: bf16 inputs make the last ulps moot
+__device__ __forceinline__ float log_decay_fast(float g, float inv_tau) {
+  return (fminf(g, 0.f) - __logf(1.f + __expf(-fabsf(g)))) * inv_tau;
+}
 
 // 16-byte chunk c (8 consecutive columns 8c..8c+7) of row `row`
 __device__ __forceinline__ uint4 *chunk_ptr(unsigned char *base, uint32_t region_off, int row, int c) {
@@ -113,13 +129,15 @@ __device__ __forceinline__ uint64_t desc_mn(uint32_t tile_addr, int s) {
 }
 
 __device__ __forceinline__ void issue_tile_loads(const Params &p, unsigned char *sm, uint64_t *bar, int bh,
-                                                 int t0) {
-  mbar_expect_tx(bar, 5 * TILE);
+                                                 int t0, bool full) {
+  mbar_expect_tx(bar, (full ? 5 : 3) * TILE);
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
-    tma_load_3d(sm + R_XQ + r * REG, &p.mq, bar, 64 * r, t0, bh);
+    if (full) {
+      tma_load_3d(sm + R_XQ + r * REG, &p.mq, bar, 64 * r, t0, bh);
+      tma_load_3d(sm + R_KP + r * REG, &p.mk, bar, 64 * r, t0 - T, bh);
+    }
     tma_load_3d(sm + R_XK + r * REG, &p.mk, bar, 64 * r, t0, bh);
-    tma_load_3d(sm + R_KP + r * REG, &p.mk, bar, 64 * r, t0 - T, bh);
     tma_load_3d(sm + R_V + r * REG, &p.mv, bar, 64 * r, t0, bh);
     tma_load_3d(sm + R_G + r * REG, &p.mg, bar, 64 * r, t0, bh);
   }
@@ -156,9 +174,10 @@ __global__ void __launch_bounds__(128, 1) tc_fwd_kernel(const __grid_constant__ 
   const int tid = threadIdx.x, warp = tid >> 5;
   const int row = tid;                                 // TMEM lane == tile row
   const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-  const int bh = blockIdx.x, h = bh % p.H;
+  const int bh = blockIdx.x, h = bh % p.H, seg = blockIdx.y;
   const float alpha = p.alpha ? p.alpha[h] : 1.f;
-  const bool gla = p.branch != 2, swa = p.branch != 1;
+  const bool full = p.mode == 0;
+  const bool gla = p.branch != 2, swa = full && p.branch != 1;
   const uint32_t sbase = smem_u32(sm);
 
   if (warp == 0) {
@@ -202,7 +221,9 @@ __global__ void __launch_bounds__(128, 1) tc_fwd_kernel(const __grid_constant__ 
 
   // initial state -> TMEM columns [0, 128), lane = key dimension
   {
-    const float *src = p.state_in ? p.state_in + ((size_t)bh * D + row) * D : nullptr;
+    const float *src = nullptr;
+    if (full && p.nseg > 1) src = p.seg_start + (((size_t)bh * p.nseg + seg) * D + row) * D;
+    else if (full && p.state_in) src = p.state_in + ((size_t)bh * D + row) * D;
 #pragma unroll
     for (int c = 0; c < D; c += 8) {
       uint32_t r[8];
@@ -213,16 +234,19 @@ __global__ void __launch_bounds__(128, 1) tc_fwd_kernel(const __grid_constant__ 
     tmem_st_wait();
   }
 
-  const int ntiles = (p.L + T - 1) / T;
+  const int ntiles_all = (p.L + T - 1) / T;
+  const int cbeg = seg * p.tiles_per_seg;
+  const int cend = min(ntiles_all, cbeg + p.tiles_per_seg);
   uint32_t *err = p.status;
-  if (tid == 0 && ntiles > 0) issue_tile_loads(p, sm, &bar_tma, bh, 0);
+  float tot_decay = 0.f;                      // mode 1: summed log-decay of this dimension
+  if (tid == 0 && cbeg < cend) issue_tile_loads(p, sm, &bar_tma, bh, cbeg * T, full);
   const uint32_t id_128 = idesc_bf16(128, 128, 0, 0);
   const uint32_t id_z = idesc_bf16(128, 64, 0, 1);
   const uint32_t id_mn = idesc_bf16(128, 128, 0, 1);
   const uint32_t id_st = idesc_bf16(128, 128, 1, 1);
 
-  for (int c = 0; c < ntiles; ++c) {
-    const uint32_t par = c & 1;
+  for (int c = cbeg; c < cend; ++c) {
+    const uint32_t par = (c - cbeg) & 1;
     const int t0 = c * T;
     const int tq = t0 + row;                  // this thread's query token
     const bool qvalid = tq < p.L;
@@ -237,23 +261,36 @@ __global__ void __launch_bounds__(128, 1) tc_fwd_kernel(const __grid_constant__ 
         for (int s = 0; s < 8; ++s) mma_ss(tb + C_L, desc_k(xq, s), desc_k(kp, s), id_128, s > 0);
         for (int s = 0; s < 8; ++s) mma_ss(tb + C_L + 128, desc_k(xq, s), desc_k(xk, s), id_128, s > 0);
       }
-      for (int s = 0; s < 8; ++s) mma_ss(tb + C_ZQ, desc_k(xq, s), desc_mn(sbase + R_WQ, s), id_z, s > 0);
+      if (full)
+        for (int s = 0; s < 8; ++s) mma_ss(tb + C_ZQ, desc_k(xq, s), desc_mn(sbase + R_WQ, s), id_z, s > 0);
       for (int s = 0; s < 8; ++s) mma_ss(tb + C_ZK, desc_k(xk, s), desc_mn(sbase + R_WK, s), id_z, s > 0);
       mma_commit(&bar_m1);
     }
 
     // ---------------------------------------------- gates (thread = dim) ---
     {
+      // 8 tokens per step: the logsigmoids and exps are independent, only
+      // the running suffix sum is a chain
       const int i = row;
+      unsigned char *gcol = sm + R_G + (i >> 6) * REG;
       float acc = 0.f, spread = 0.f;
-      for (int t = T - 1; t >= 0; --t) {
-        __nv_bfloat16 *gp = reinterpret_cast<__nv_bfloat16 *>(sm + R_G + (i >> 6) * REG + sw128_offset(t, i & 63));
-        const float a = (t0 + t < p.L) ? log_decay(__bfloat162float(*gp), p.inv_tau) : 0.f;
-        *gp = __float2bfloat16_rn(__expf(acc));   // E_t = exp(b_t - r)
-        if (t == 0) spread = acc;
-        acc -= a;
+      for (int tb8 = T - 8; tb8 >= 0; tb8 -= 8) {
+        float a[8], pre[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int t = tb8 + u;
+          const __nv_bfloat16 g = *reinterpret_cast<const __nv_bfloat16 *>(gcol + sw128_offset(t, i & 63));
+          a[u] = (t0 + t < p.L) ? log_decay_fast(__bfloat162float(g), p.inv_tau) : 0.f;
+        }
+#pragma unroll
+        for (int u = 7; u >= 0; --u) { pre[u] = acc; acc -= a[u]; }
+#pragma unroll
+        for (int u = 0; u < 8; ++u)      // E_t = exp(b_t - r) = exp(sum_{s>t} -a_s)
+          *reinterpret_cast<__nv_bfloat16 *>(gcol + sw128_offset(tb8 + u, i & 63)) = __float2bfloat16_rn(__expf(pre[u]));
+        if (tb8 == 0) spread = pre[0];
       }
       s_dec[i] = __expf(-acc);                     // exp(r): the tile's total decay
+      tot_decay -= acc;
       if (spread > kMaxSpread && gla) atomicOr(err, ST_RANGE);
     }
 
@@ -290,29 +327,32 @@ __global__ void __launch_bounds__(128, 1) tc_fwd_kernel(const __grid_constant__ 
         }
       }
       const int jlo = max(tq - p.window + 1, 0);     // valid keys j in [jlo, tq]
-      for (int ch = 0; ch < 16; ++ch) {
-        float v[16];
-        tmem_ld16(tb + lane_off + C_L + ch * 16, v);
+      for (int ch = 0; ch < 8; ++ch) {
+        float v[32];
+        tmem_ld32(tb + lane_off + C_L + ch * 32, v);
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int j = t0 - T + ch * 16 + u;
+        for (int u = 0; u < 32; ++u) {
+          const int j = t0 - T + ch * 32 + u;
           if (j >= jlo && j <= tq) mx = fmaxf(mx, v[u] * p.scale);
         }
       }
       lsum = 0.f;
-      for (int ch = 0; ch < 16; ++ch) {
-        float v[16];
-        tmem_ld16(tb + lane_off + C_L + ch * 16, v);
-        uint32_t pk[8];
+      for (int ch = 0; ch < 8; ++ch) {
+        float v[32];
+        tmem_ld32(tb + lane_off + C_L + ch * 32, v);
+        uint32_t pk[16];
+        float part = 0.f;
 #pragma unroll
-        for (int u = 0; u < 16; u += 2) {
-          const int j = t0 - T + ch * 16 + u;
+        for (int u = 0; u < 32; u += 2) {
+          const int j = t0 - T + ch * 32 + u;
           const float e0 = (j >= jlo && j <= tq) ? __expf(v[u] * p.scale - mx) : 0.f;
           const float e1 = (j + 1 >= jlo && j + 1 <= tq) ? __expf(v[u + 1] * p.scale - mx) : 0.f;
-          lsum += e0 + e1;
+          part += e0 + e1;
           pk[u / 2] = alpha != 0.f ? pack_bf16(e0, e1) : 0u;
         }
-        tmem_st8(tb + lane_off + C_P + ch * 8, pk);
+        lsum += part;
+        tmem_st8(tb + lane_off + C_P + ch * 16, pk);
+        tmem_st8(tb + lane_off + C_P + ch * 16 + 8, pk + 8);
       }
 #pragma unroll
       for (int m = 0; m < MAXM; ++m) {
@@ -333,8 +373,9 @@ __global__ void __launch_bounds__(128, 1) tc_fwd_kernel(const __grid_constant__ 
     {
       float z[F], neg[F];
       // phi_q -> Qt = phi_q E gscale, packed bf16 pairs into TMEM
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) tmem_ld16(tb + lane_off + C_ZQ + ch * 16, z + ch * 16);
+      if (full) {
+      tmem_ld32(tb + lane_off + C_ZQ, z);
+      tmem_ld32(tb + lane_off + C_ZQ + 32, z + 32);
       feature_map_row(z, neg);
 #pragma unroll
       for (int c16 = 0; c16 < 8; ++c16) {     // 16 dims = 8 TMEM columns
@@ -351,9 +392,10 @@ __global__ void __launch_bounds__(128, 1) tc_fwd_kernel(const __grid_constant__ 
         }
         tmem_st8(tb + lane_off + C_QT + c16 * 8, r8);
       }
+      }
       // phi_k -> Kt = phi_k / E, bf16 into shared memory over X_k
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) tmem_ld16(tb + lane_off + C_ZK + ch * 16, z + ch * 16);
+      tmem_ld32(tb + lane_off + C_ZK, z);
+      tmem_ld32(tb + lane_off + C_ZK + 32, z + 32);
       feature_map_row(z, neg);
 #pragma unroll
       for (int c8 = 0; c8 < 16; ++c8) {
@@ -363,7 +405,7 @@ __global__ void __launch_bounds__(128, 1) tc_fwd_kernel(const __grid_constant__ 
         for (int u = 0; u < 8; ++u) {
           const int i = c8 * 8 + u;
           const float ph = i < F ? z[i] : neg[i - F];
-          k8[u] = ph * __frcp_rn(e8[u]);
+          k8[u] = ph * __fdividef(1.f, e8[u]);
         }
         *chunk_ptr(sm, R_XK, row, c8) = pack8(k8);
       }
@@ -385,9 +427,10 @@ __global__ void __launch_bounds__(128, 1) tc_fwd_kernel(const __grid_constant__ 
 #pragma unroll
         for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(v[8 + u]);
         tmem_st8(tb + lane_off + C_S + c16 * 16 + 8, r);
-        // bf16 copy S'[i][v], MN-major: rows = i (K of the O = Qt S' product)
-        *chunk_ptr(sm, R_XQ, i, 2 * c16) = pack8(v);
-        *chunk_ptr(sm, R_XQ, i, 2 * c16 + 1) = pack8(v + 8);
+        if (full) {   // bf16 copy S'[i][v], MN-major: rows = i (K of the O = Qt S' product)
+          *chunk_ptr(sm, R_XQ, i, 2 * c16) = pack8(v);
+          *chunk_ptr(sm, R_XQ, i, 2 * c16 + 1) = pack8(v + 8);
+        }
       }
     }
     tmem_st_wait();
@@ -398,20 +441,22 @@ __global__ void __launch_bounds__(128, 1) tc_fwd_kernel(const __grid_constant__ 
     // ---------------------------------------------------------- MMA 2 ---
     if (tid == 0) {
       tc_fence_after();
-      if (gla)
+      if (gla && full)
         for (int s = 0; s < 8; ++s) mma_ts(tb + C_A, tb + C_QT + s * 8, desc_k(sbase + R_XK, s), id_128, s > 0);
       mma_commit(&bar_m2);
       // V of the previous tile into the G region (E has been consumed)
-      mbar_expect_tx(&bar_vp, TILE);
-      tma_load_3d(sm + R_G, &p.mv, &bar_vp, 0, t0 - T, bh);
-      tma_load_3d(sm + R_G + REG, &p.mv, &bar_vp, 64, t0 - T, bh);
+      mbar_expect_tx(&bar_vp, swa ? TILE : 0);
+      if (swa) {
+        tma_load_3d(sm + R_G, &p.mv, &bar_vp, 0, t0 - T, bh);
+        tma_load_3d(sm + R_G + REG, &p.mv, &bar_vp, 64, t0 - T, bh);
+      }
     }
     ok = mbar_wait(&bar_m2, par, err, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) { s_fail = 1; break; }
     tc_fence_after();
 
     // ------------------------------------------ rows: masked intra A ---
-    if (gla) {
+    if (gla && full) {
       for (int c16 = 0; c16 < 8; ++c16) {
         float v[16];
         tmem_ld16(tb + lane_off + C_A + c16 * 16, v);
@@ -437,7 +482,7 @@ __global__ void __launch_bounds__(128, 1) tc_fwd_kernel(const __grid_constant__ 
       tc_fence_after();
       const uint32_t sp = sbase + R_XQ, v = sbase + R_V, vp = sbase + R_G, kt = sbase + R_XK;
       uint32_t accum = 0;
-      if (gla) {
+      if (gla && full) {
         for (int s = 0; s < 8; ++s) { mma_ts(tb + C_O, tb + C_QT + s * 8, desc_mn(sp, s), id_mn, accum); accum = 1; }
         for (int s = 0; s < 8; ++s) mma_ts(tb + C_O, tb + C_AH + s * 8, desc_mn(v, s), id_mn, 1);
       }
@@ -452,10 +497,10 @@ __global__ void __launch_bounds__(128, 1) tc_fwd_kernel(const __grid_constant__ 
     ok = mbar_wait(&bar_m3, par, err, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) { s_fail = 1; break; }
     tc_fence_after();
-    if (tid == 0 && c + 1 < ntiles) issue_tile_loads(p, sm, &bar_tma, bh, t0 + T);
+    if (tid == 0 && c + 1 < cend) issue_tile_loads(p, sm, &bar_tma, bh, t0 + T, full);
 
     // -------------------------------------------------------- epilogue ---
-    {
+    if (full) {
       // tcgen05.ld is warp-collective: every lane loads, valid rows store
       __nv_bfloat16 *orow = p.o + ((size_t)bh * p.L + (qvalid ? tq : 0)) * D;
       for (int c16 = 0; c16 < 8; ++c16) {
@@ -485,9 +530,15 @@ __global__ void __launch_bounds__(128, 1) tc_fwd_kernel(const __grid_constant__ 
     __syncthreads();
   }
 
-  if (!s_fail && p.state_out && gla) {
+  float *sdst = nullptr;
+  if (full && p.state_out && gla && seg == p.nseg - 1) sdst = p.state_out + ((size_t)bh * D + row) * D;
+  if (!full) {
+    sdst = p.seg_state + (((size_t)bh * p.nseg + seg) * D + row) * D;
+    p.seg_decay[((size_t)bh * p.nseg + seg) * D + row] = tot_decay;
+  }
+  if (!s_fail && sdst) {
     tc_fence_after();
-    float *dst = p.state_out + ((size_t)bh * D + row) * D;
+    float *dst = sdst;
     for (int c16 = 0; c16 < 8; ++c16) {
       float v[16];
       tmem_ld16(tb + lane_off + C_S + c16 * 16, v);
@@ -504,13 +555,64 @@ __global__ void __launch_bounds__(128, 1) tc_fwd_kernel(const __grid_constant__ 
   if (warp == 0) tmem_dealloc(tb, 512);
 }
 
+// Start state of every segment: S_0 = state_in (or 0),
+// S_{s+1} = diag(exp(decay_s)) S_s + local_s.
+__global__ void __launch_bounds__(256) seg_combine_kernel(const float *seg_state, const float *seg_decay,
+                                                          const float *state_in, float *seg_start, int nseg) {
+  const int bh = blockIdx.x;
+  for (int e = threadIdx.x; e < D * D; e += 256) {
+    const int i = e / D;
+    float sv = state_in ? state_in[(size_t)bh * D * D + e] : 0.f;
+    seg_start[((size_t)bh * nseg) * D * D + e] = sv;
+    for (int sg = 1; sg < nseg; ++sg) {
+      const size_t prev = (size_t)bh * nseg + sg - 1;
+      sv = expf(seg_decay[prev * D + i]) * sv + seg_state[prev * D * D + e];
+      seg_start[((size_t)bh * nseg + sg) * D * D + e] = sv;
+    }
+  }
+}
+
 }  // namespace
 
 bool tc_fwd_supported(int dk, int dv, int window, int M, bool bf16) {
   return bf16 && dk == D && dv == D && window <= T && M <= MAXM;
 }
 
-cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t s) {
+// Segments per sequence: enough (batch, head, segment) CTAs to cover the
+// 148 SMs once, each segment at least two tiles long.
+void tc_fwd_segments(int BH, int L, int *nseg, int *tiles_per_seg) {
+  const int ntiles = (L + T - 1) / T;
+  int n = BH >= 120 ? 1 : 148 / (BH > 0 ? BH : 1);
+  n = n < ntiles / 2 ? n : ntiles / 2;
+  if (n < 1) n = 1;
+  const int tps = (ntiles + n - 1) / n;
+  *tiles_per_seg = tps > 0 ? tps : 1;
+  *nseg = tps > 0 ? (ntiles + tps - 1) / tps : 1;
+}
+
+size_t tc_fwd_workspace_bytes(int BH, int L) {
+  int nseg, tps;
+  tc_fwd_segments(BH, L, &nseg, &tps);
+  if (nseg <= 1) return 0;
+  return (size_t)BH * nseg * (2 * (size_t)D * D + D) * sizeof(float);
+}
+
+int tc_fwd_stage_count(int BH, int L) {
+  int nseg, tps;
+  tc_fwd_segments(BH, L, &nseg, &tps);
+  return nseg > 1 ? 3 : 1;
+}
+
+cudaError_t launch_tc_fwd(const TcFwdArgs &a, int stage, cudaStream_t s) {
+  int nseg, tps;
+  tc_fwd_segments(a.BH, a.L, &nseg, &tps);
+  float *seg_state = static_cast<float *>(a.seg_ws);
+  float *seg_start = seg_state ? seg_state + (size_t)a.BH * nseg * D * D : nullptr;
+  float *seg_decay = seg_start ? seg_start + (size_t)a.BH * nseg * D * D : nullptr;
+  if (nseg > 1 && stage == 1) {
+    seg_combine_kernel<<<a.BH, 256, 0, s>>>(seg_state, seg_decay, a.state_in, seg_start, nseg);
+    return cudaGetLastError();
+  }
   Params p;
   memset(&p, 0, sizeof(p));
   const uint64_t rows = (uint64_t)a.L;
@@ -528,11 +630,16 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t s) {
   p.state_out = a.state_out;
   p.lse = a.lse;
   p.status = a.status;
+  p.seg_start = seg_start;
+  p.seg_state = seg_state;
+  p.seg_decay = seg_decay;
   p.H = a.H;
   p.L = a.L;
   p.M = a.M;
   p.window = a.window;
   p.branch = a.branch;
+  p.nseg = nseg;
+  p.tiles_per_seg = tps;
   p.inv_tau = a.inv_tau;
   p.scale = a.scale;
   static size_t configured[64] = {};
@@ -544,7 +651,13 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) configured[dev] = SMEM_BYTES;
   }
-  tc_fwd_kernel<<<a.BH, 128, SMEM_BYTES, s>>>(p);
+  if (nseg > 1 && stage == 0) {          // state pass over every segment but the last
+    p.mode = 1;
+    tc_fwd_kernel<<<dim3(a.BH, nseg - 1), 128, SMEM_BYTES, s>>>(p);
+  } else {                               // full pass
+    p.mode = 0;
+    tc_fwd_kernel<<<dim3(a.BH, nseg), 128, SMEM_BYTES, s>>>(p);
+  }
   return cudaGetLastError();
 }
 

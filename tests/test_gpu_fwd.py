@@ -164,6 +164,28 @@ def test_segmented_equals_one_shot(lz, impl):
     check("S", r2["state_out"], to64(full["state_out"]), dtype)
 
 
+@pytest.mark.parametrize("L", [1000, 3000])
+def test_tc_segmented_long_sequence(lz, L):
+    """Few (batch, head) pairs and a long sequence: the tensor-core forward
+    splits the sequence into segments (state pass, combine, full pass)."""
+    w = Workload("tcseg", B=1, H=2, L=L, d=128, window=128, M=4, dtype="bf16", seed=L)
+    inp = make_inputs(w)
+    inp["state_in"] = torch.randn(1, 2, 128, 128, generator=torch.Generator().manual_seed(3)) * 0.1
+    inp["alpha"] = random_alpha(2, seed=L)
+    x = to_device(inp)
+    plan = lz.attn_fwd(x["q"], x["k"], x["v"], x["g"], window=w.window, gate_temp=w.gate_temp,
+                       fmap_wq=x["fmap_wq"], fmap_wk=x["fmap_wk"], meta_k=x["meta_k"],
+                       meta_v=x["meta_v"], alpha=x["alpha"], state_in=x["state_in"],
+                       impl=lz.IMPL_TC, plan_only=True)
+    assert len(plan) == 3, plan
+    got = _run(lz, x, w, lz.IMPL_TC, want_state=True, want_lse=True)
+    assert lz.workspace_status(got["workspace"]) == lz.OK
+    want = oracle_forward(inp, window=w.window, tau=w.gate_temp)
+    check("o", got["o"], want["o"], "bf16")
+    check("state_out", got["state_out"], want["state_out"], "bf16")
+    check("lse", got["lse"], want["lse"], "bf16")
+
+
 def test_empty_sequence_passes_state_through(lz):
     w = Workload("empty", B=1, H=2, L=0, d=64, window=4, M=0, dtype="bf16")
     inp = make_inputs(w)
