@@ -80,10 +80,16 @@ FwdLayout fwd_layout(const lizard_fwd_args *a) {
   return l;
 }
 
+// Whether the backward's anchor branch runs on the tensor-core kernels.
+bool bwd_swa_uses_tc(const lizard_fwd_args *a, int impl) {
+  const bool ok = lz::tc_swa_bwd_supported(a->dk, a->dv, a->window, a->M, a->dtype == LIZARD_BF16);
+  return (impl == LIZARD_IMPL_AUTO || impl == LIZARD_IMPL_TC) && ok;
+}
+
 struct BwdLayout {
-  size_t phq, phk, a, sprev, dphq, dphk, da, dv_gla, dq_swa, dk_swa, dv_swa, lse, Dterm, total;
+  size_t phq, phk, a, sprev, dphq, dphk, da, dv_gla, dq_swa, dk_swa, dv_swa, lse, Dterm, dsm, pm, total;
 };
-BwdLayout bwd_layout(const lizard_fwd_args *a) {
+BwdLayout bwd_layout(const lizard_fwd_args *a, int impl) {
   const size_t BH = (size_t)a->B * a->H;
   const size_t N = BH * a->L;
   const size_t nd = up(N * a->dk * sizeof(float));
@@ -107,6 +113,10 @@ BwdLayout bwd_layout(const lizard_fwd_args *a) {
     l.dv_swa = off; off += nv;
     l.lse = off; off += up(N * sizeof(float));
     l.Dterm = off; off += up(N * sizeof(float));
+    if (bwd_swa_uses_tc(a, impl)) {
+      l.dsm = off; off += up(N * 16 * sizeof(float));
+      l.pm = off; off += up(N * 16 * sizeof(float));
+    }
   }
   l.total = off;
   return l;
@@ -181,7 +191,7 @@ void fwd_plan(const lizard_fwd_args *a, void *ws, cudaStream_t s, Plan &plan) {
 
 void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan) {
   const lizard_fwd_args *a = &b->fwd;
-  const BwdLayout lay = bwd_layout(a);
+  const BwdLayout lay = bwd_layout(a, b->impl);
   const int BH = a->B * a->H, D = a->dk;
   const bool bf16 = a->dtype == LIZARD_BF16;
   const float inv_tau = 1.f / a->gate_temp;
@@ -197,7 +207,17 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan) {
                       at<float>(ws, lay.da), at<float>(ws, lay.dv_gla), b->dstate_in, a->L};
     plan.add("gla_bwd_simt", [=] { return lz::launch_gla_bwd_simt(ga, BH, D, bf16, s); });
   }
-  if (w) {
+  if (w && bwd_swa_uses_tc(a, b->impl)) {
+    lz::TcSwaBwdArgs t{a->q, a->k, a->v, b->dout, a->meta_k, a->meta_v, a->alpha,
+                       at<float>(ws, lay.dq_swa), at<float>(ws, lay.dk_swa), at<float>(ws, lay.dv_swa),
+                       at<float>(ws, lay.lse), at<float>(ws, lay.Dterm), at<float>(ws, lay.dsm),
+                       at<float>(ws, lay.pm), b->dmeta_k, b->dmeta_v, b->dalpha, static_cast<uint32_t *>(ws),
+                       a->B, a->H, BH, a->L, a->M, a->window, scale_of(a)};
+    plan.add("tc_swa_bwd_q_kernel", [=] { return lz::launch_tc_swa_bwd(t, 0, s); });
+    plan.add("tc_swa_bwd_kv_kernel", [=] { return lz::launch_tc_swa_bwd(t, 1, s); });
+    if (a->M > 0 && (b->dmeta_k || b->dmeta_v))
+      plan.add("meta_grad_kernel", [=] { return lz::launch_tc_swa_bwd(t, 2, s); });
+  } else if (w) {
     lz::SwaBwdQArgs qa{a->q, a->k, a->v, b->dout, a->meta_k, a->meta_v, a->alpha,
                        at<float>(ws, lay.dq_swa), at<float>(ws, lay.lse), at<float>(ws, lay.Dterm),
                        b->dmeta_k, b->dmeta_v, b->dalpha, a->H, a->L, a->window, a->M, scale_of(a)};
@@ -301,15 +321,15 @@ size_t lizard_bwd_workspace_size(const lizard_bwd_args *args) {
     a.o = reinterpret_cast<void *>(16);
   }
   if (check_fwd(&a) != LIZARD_OK) return 0;
-  return bwd_layout(&a).total;
+  return bwd_layout(&a, args->impl).total;
 }
 
 lizard_status lizard_attn_bwd(const lizard_bwd_args *b, lizard_stream_t stream) {
   lizard_status st = check_bwd(b);
   if (st != LIZARD_OK) return st;
-  if (b->impl == LIZARD_IMPL_TC) return LIZARD_ERR_UNSUPPORTED;
   const lizard_fwd_args *a = &b->fwd;
-  const BwdLayout lay = bwd_layout(a);
+  if (b->impl == LIZARD_IMPL_TC && swa_on(a) && !bwd_swa_uses_tc(a, b->impl)) return LIZARD_ERR_UNSUPPORTED;
+  const BwdLayout lay = bwd_layout(a, b->impl);
   if (!b->workspace || b->workspace_bytes < lay.total) return LIZARD_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int BH = a->B * a->H, D = a->dk, F = D / 2;

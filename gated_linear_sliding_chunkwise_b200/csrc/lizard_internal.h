@@ -102,6 +102,18 @@ struct TcFwdArgs {
   float inv_tau, scale;
 };
 
+struct TcSwaBwdArgs {
+  const void *q, *k, *v, *dout;
+  const float *meta_k, *meta_v, *alpha;
+  float *dq, *dk, *dv;          // anchor-branch parts, fp32 [B*H*L][128]
+  float *lse, *Dterm;           // [B*H*L]
+  float *dsm, *pm;              // per-row meta-token terms, [B*H*L][16]
+  float *dmeta_k, *dmeta_v, *dalpha;
+  uint32_t *status;
+  int B, H, BH, L, M, window;
+  float scale;
+};
+
 constexpr int kBwdC = 32;   // GLA chunk used by the portable backward
 
 cudaError_t launch_prep(const PrepArgs &a, int BH, int D, bool bf16, cudaStream_t s);
@@ -118,6 +130,9 @@ cudaError_t launch_gla_states(const GlaStatesArgs &a, int BH, int D, bool bf16, 
 cudaError_t launch_gla_bwd_simt(const GlaBwdArgs &a, int BH, int D, bool bf16, cudaStream_t s);
 cudaError_t launch_swa_bwd_q(const SwaBwdQArgs &a, int BH, int D, bool bf16, cudaStream_t s);
 cudaError_t launch_swa_bwd_kv(const SwaBwdKVArgs &a, int BH, int D, bool bf16, cudaStream_t s);
+bool tc_swa_bwd_supported(int dk, int dv, int window, int M, bool bf16);
+// stage 0: dq pass, 1: dk/dv pass, 2: meta-token gradients
+cudaError_t launch_tc_swa_bwd(const TcSwaBwdArgs &a, int stage, cudaStream_t s);
 cudaError_t launch_finish_bwd(const FinishBwdArgs &a, int BH, int D, bool bf16, cudaStream_t s);
 
 }  // namespace lz

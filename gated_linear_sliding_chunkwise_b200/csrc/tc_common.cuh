@@ -179,5 +179,42 @@ __host__ __device__ __forceinline__ uint32_t sw128_offset(int row, int col) {
   return (uint32_t)(row * 128 + chunk * 16 + (col & 7) * 2);
 }
 
+// ---------------------------------------------- 128 x 128 bf16 tiles -----
+// A 128-row tile of 128 bf16 columns, as TMA writes it with the 128-byte
+// swizzle: two 16 KB regions of 64 columns, each 1024-byte aligned.
+constexpr uint32_t kReg = 16384;
+constexpr uint32_t kTile = 2 * kReg;
+
+// 16-byte chunk c (columns 8c .. 8c+7) of row `row`
+__device__ __forceinline__ uint4 *chunk_ptr(unsigned char *base, uint32_t region_off, int row, int c) {
+  return reinterpret_cast<uint4 *>(base + region_off + (c >> 3) * kReg + sw128_offset(row, (c & 7) * 8));
+}
+__device__ __forceinline__ void unpack8(const uint4 &u, float *f) {
+  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 v = __bfloat1622float2(h[i]);
+    f[2 * i] = v.x;
+    f[2 * i + 1] = v.y;
+  }
+}
+__device__ __forceinline__ uint4 pack8(const float *f) {
+  uint4 u;
+  u.x = pack_bf16(f[0], f[1]);
+  u.y = pack_bf16(f[2], f[3]);
+  u.z = pack_bf16(f[4], f[5]);
+  u.w = pack_bf16(f[6], f[7]);
+  return u;
+}
+// K-major operand descriptor, k-step s (16 columns) of a 128-row tile
+__device__ __forceinline__ uint64_t desc_k(uint32_t tile_addr, int s) {
+  return sdesc_sw128(tile_addr + (s >> 2) * kReg + (s & 3) * 32, 0, 1024);
+}
+// MN-major operand descriptor, k-step s (16 rows) of a tile whose rows are K
+// and whose two 64-column regions are M/N blocks
+__device__ __forceinline__ uint64_t desc_mn(uint32_t tile_addr, int s) {
+  return sdesc_sw128(tile_addr + s * 2048, kReg, 1024);
+}
+
 }  // namespace tc
 }  // namespace lz

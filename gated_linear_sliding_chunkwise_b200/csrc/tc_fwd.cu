@@ -54,8 +54,8 @@ using namespace tc;
 constexpr int T = 128;             // tokens per tile
 constexpr int D = 128;             // dk = dv
 constexpr int F = D / 2;           // feature-map width per half
-constexpr uint32_t REG = 16384;    // one 64-column swizzled region of a 128-row tile
-constexpr uint32_t TILE = 2 * REG; // a 128 x 128 bf16 tile
+constexpr uint32_t REG = kReg;     // one 64-column swizzled region of a 128-row tile
+constexpr uint32_t TILE = kTile;   // a 128 x 128 bf16 tile
 constexpr int MAXM = 16;
 
 // shared-memory regions (offsets from the 1024-aligned base)
@@ -93,39 +93,6 @@ struct Params {
 // logsigmoid(g) / tau with the fast exp/log: bf16 inputs make the last ulps moot
 __device__ __forceinline__ float log_decay_fast(float g, float inv_tau) {
   return (fminf(g, 0.f) - __logf(1.f + __expf(-fabsf(g)))) * inv_tau;
-}
-
-// 16-byte chunk c (8 consecutive columns 8c..8c+7) of row `row`
-__device__ __forceinline__ uint4 *chunk_ptr(unsigned char *base, uint32_t region_off, int row, int c) {
-  return reinterpret_cast<uint4 *>(base + region_off + (c >> 3) * REG + sw128_offset(row, (c & 7) * 8));
-}
-
-__device__ __forceinline__ void unpack8(const uint4 &u, float *f) {
-  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 v = __bfloat1622float2(h[i]);
-    f[2 * i] = v.x;
-    f[2 * i + 1] = v.y;
-  }
-}
-__device__ __forceinline__ uint4 pack8(const float *f) {
-  uint4 u;
-  u.x = pack_bf16(f[0], f[1]);
-  u.y = pack_bf16(f[2], f[3]);
-  u.z = pack_bf16(f[4], f[5]);
-  u.w = pack_bf16(f[6], f[7]);
-  return u;
-}
-
-// K-major operand descriptor, k-step s (16 columns) of a 128-row tile
-__device__ __forceinline__ uint64_t desc_k(uint32_t tile_addr, int s) {
-  return sdesc_sw128(tile_addr + (s >> 2) * REG + (s & 3) * 32, 0, 1024);
-}
-// MN-major operand descriptor, k-step s (16 rows) of a tile whose rows are K
-// and whose two 64-column regions are M/N blocks
-__device__ __forceinline__ uint64_t desc_mn(uint32_t tile_addr, int s) {
-  return sdesc_sw128(tile_addr + s * 2048, REG, 1024);
 }
 
 __device__ __forceinline__ void issue_tile_loads(const Params &p, unsigned char *sm, uint64_t *bar, int bh,

@@ -1,0 +1,517 @@
+// Tensor-core (tcgen05 / TMEM / TMA) backward of the anchor branch: sliding
+// window softmax with meta-token sinks (English gist.science summary,
+// section 2.A "Anchor Window Attention"), bf16, d = 128, window <= 128.
+//
+// Softmax backward for query t with weights p over its window keys and the
+// meta tokens, dO_swa = alpha dout:
+//   D_t = dO_swa . o_swa_t,   dS = p (dO_swa . value - D_t)
+//   dq_t = scale sum dS key,  dkey += scale dS q_t,  dvalue += p dO_swa
+//
+// tc_swa_bwd_q_kernel   one CTA per (sequence, 128-query tile): logits and
+//                       softmax again, o_swa = P V for D, dP, dS, dq; writes
+//                       dq, the log-normaliser, D and the per-row meta terms.
+// tc_swa_bwd_kv_kernel  one CTA per (sequence, 128-key block): the two query
+//                       tiles that see the block; dK and dV accumulate in TMEM.
+// meta_grad_kernel      meta-token gradients: per head, sums over tokens.
+//
+// Every mbarrier wait is bounded; a wait that gives up sets the TIMEOUT bit
+// of the status word and the CTA leaves after freeing its TMEM.
+#include "common.cuh"
+#include "lizard_internal.h"
+#include "tc_common.cuh"
+#include "tc_host.h"
+
+namespace lz {
+namespace {
+
+using namespace tc;
+
+constexpr int T = 128;
+constexpr int D = 128;
+constexpr int MAXM = 16;
+constexpr uint32_t TILE = kTile;
+constexpr size_t SMEM_BYTES = 6 * TILE + 1024;
+constexpr uint32_t ST_TIMEOUT = 1u;
+
+struct QParams {
+  CUtensorMap mq, mk, mv, mo;
+  const float *meta_k, *meta_v, *alpha;
+  float *dq, *lse, *Dterm, *dsm, *pm, *dalpha;
+  uint32_t *status;
+  int H, L, M, window;
+  float scale;
+};
+
+struct KVParams {
+  CUtensorMap mq, mk, mv, mo;
+  const float *alpha, *lse, *Dterm;
+  float *dk, *dv;
+  uint32_t *status;
+  int H, L, window;
+  float scale;
+};
+
+__device__ __forceinline__ void setup_cta(uint32_t *tmem_slot, uint64_t *bars, int nbars, int tid) {
+  if ((tid >> 5) == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int i = 0; i < nbars; ++i) mbar_init(&bars[i], 1);
+    fence_barrier_init();
+  }
+}
+
+// ------------------------------------------------------------- dq pass ----
+__global__ void __launch_bounds__(128, 1) tc_swa_bwd_q_kernel(const __grid_constant__ QParams p) {
+  extern __shared__ unsigned char smraw[];
+  unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
+  __shared__ float s_mk[MAXM][D], s_mv[MAXM][D];
+  __shared__ float s_red[4];
+  __shared__ uint64_t bars[5];
+  __shared__ uint32_t s_tmem;
+  // regions: Q, dO, K_prev, K, V_prev, V
+  constexpr uint32_t R_Q = 0, R_O = TILE, R_KP = 2 * TILE, R_K = 3 * TILE, R_VP = 4 * TILE, R_V = 5 * TILE;
+  // TMEM: P^ [0,128) (over the logits [0,256)), O' [256,384), dP' [128,384),
+  // dS [384,512), dq' [128,256)
+  constexpr uint32_t C_L = 0, C_P = 0, C_O = 256, C_DP = 128, C_DS = 384, C_DQ = 128;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, row = tid;
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const int bh = blockIdx.y, h = bh % p.H, t0 = blockIdx.x * T, tq = t0 + row;
+  const bool qvalid = tq < p.L;
+  const float alpha = p.alpha ? p.alpha[h] : 1.f;
+  const uint32_t sbase = smem_u32(sm);
+  uint64_t *bar_tma = &bars[0], *bar_m = &bars[1];
+  setup_cta(&s_tmem, bars, 5, tid);
+  for (int e = tid; e < p.M * D; e += 128) {
+    s_mk[e / D][e % D] = p.meta_k[(size_t)h * p.M * D + e];
+    s_mv[e / D][e % D] = p.meta_v ? p.meta_v[(size_t)h * p.M * D + e] : 0.f;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = s_tmem;
+  if (tid == 0) {
+    mbar_expect_tx(bar_tma, 6 * TILE);
+    for (int r = 0; r < 2; ++r) {
+      tma_load_3d(sm + R_Q + r * kReg, &p.mq, bar_tma, 64 * r, t0, bh);
+      tma_load_3d(sm + R_O + r * kReg, &p.mo, bar_tma, 64 * r, t0, bh);
+      tma_load_3d(sm + R_KP + r * kReg, &p.mk, bar_tma, 64 * r, t0 - T, bh);
+      tma_load_3d(sm + R_K + r * kReg, &p.mk, bar_tma, 64 * r, t0, bh);
+      tma_load_3d(sm + R_VP + r * kReg, &p.mv, bar_tma, 64 * r, t0 - T, bh);
+      tma_load_3d(sm + R_V + r * kReg, &p.mv, bar_tma, 64 * r, t0, bh);
+    }
+  }
+  const uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
+  const uint32_t id_mn = idesc_bf16(128, 128, 0, 1);
+  bool ok = mbar_wait(bar_tma, 0, p.status, ST_TIMEOUT);
+  if (__syncthreads_or(!ok)) goto done;
+
+  // 1. logits L = Q [K_prev ; K]^T
+  if (tid == 0) {
+    tc_fence_after();
+    for (int s = 0; s < 8; ++s) mma_ss(tb + C_L, desc_k(sbase + R_Q, s), desc_k(sbase + R_KP, s), id_kk, s > 0);
+    for (int s = 0; s < 8; ++s) mma_ss(tb + C_L + 128, desc_k(sbase + R_Q, s), desc_k(sbase + R_K, s), id_kk, s > 0);
+    mma_commit(&bars[1]);
+  }
+  {
+    // meta logits on the CUDA cores while the MMAs run
+    float ml[MAXM], em[MAXM], dom[MAXM];
+#pragma unroll
+    for (int m = 0; m < MAXM; ++m) { ml[m] = 0.f; dom[m] = 0.f; }
+    for (int ch = 0; ch < 16; ++ch) {
+      float q8[8], o8[8];
+      unpack8(*chunk_ptr(sm, R_Q, row, ch), q8);
+      unpack8(*chunk_ptr(sm, R_O, row, ch), o8);
+#pragma unroll
+      for (int m = 0; m < MAXM; ++m) {
+        if (m < p.M) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            ml[m] = fmaf(q8[u], s_mk[m][ch * 8 + u], ml[m]);
+            dom[m] = fmaf(o8[u], s_mv[m][ch * 8 + u], dom[m]);
+          }
+        }
+      }
+    }
+    float mx = kNegBig;
+#pragma unroll
+    for (int m = 0; m < MAXM; ++m)
+      if (m < p.M) { ml[m] *= p.scale; mx = fmaxf(mx, ml[m]); }
+    ok = mbar_wait(bar_m, 0, p.status, ST_TIMEOUT);
+    if (__syncthreads_or(!ok)) goto done;
+    tc_fence_after();
+
+    // 2. softmax: max, then exp and sum with P^ = exp(l - max) packed over L
+    const int jlo = max(tq - p.window + 1, 0);
+    for (int ch = 0; ch < 8; ++ch) {
+      float v[32];
+      tmem_ld32(tb + lane_off + C_L + ch * 32, v);
+#pragma unroll
+      for (int u = 0; u < 32; ++u) {
+        const int j = t0 - T + ch * 32 + u;
+        if (j >= jlo && j <= tq) mx = fmaxf(mx, v[u] * p.scale);
+      }
+    }
+    float lsum = 0.f;
+    for (int ch = 0; ch < 8; ++ch) {
+      float v[32];
+      tmem_ld32(tb + lane_off + C_L + ch * 32, v);
+      uint32_t pk[16];
+      float part = 0.f;
+#pragma unroll
+      for (int u = 0; u < 32; u += 2) {
+        const int j = t0 - T + ch * 32 + u;
+        const float e0 = (j >= jlo && j <= tq) ? __expf(v[u] * p.scale - mx) : 0.f;
+        const float e1 = (j + 1 >= jlo && j + 1 <= tq) ? __expf(v[u + 1] * p.scale - mx) : 0.f;
+        part += e0 + e1;
+        pk[u / 2] = pack_bf16(e0, e1);
+      }
+      lsum += part;
+      tmem_st8(tb + lane_off + C_P + ch * 16, pk);
+      tmem_st8(tb + lane_off + C_P + ch * 16 + 8, pk + 8);
+    }
+#pragma unroll
+    for (int m = 0; m < MAXM; ++m)
+      if (m < p.M) { em[m] = __expf(ml[m] - mx); lsum += em[m]; } else em[m] = 0.f;
+    const float inv_l = 1.f / lsum;
+    if (qvalid) p.lse[(size_t)bh * p.L + tq] = mx + logf(lsum);
+    tmem_st_wait();
+    tc_fence_before();
+    __syncthreads();
+
+    // 3. O' = P^ [V_prev ; V]   (o_swa = (O' + sum_m em_m mv_m) / l)
+    if (tid == 0) {
+      tc_fence_after();
+      for (int s = 0; s < 8; ++s) mma_ts(tb + C_O, tb + C_P + s * 8, desc_mn(sbase + R_VP, s), id_mn, s > 0);
+      for (int s = 0; s < 8; ++s) mma_ts(tb + C_O, tb + C_P + 64 + s * 8, desc_mn(sbase + R_V, s), id_mn, 1);
+      mma_commit(&bars[2]);
+    }
+    ok = mbar_wait(&bars[2], 0, p.status, ST_TIMEOUT);
+    if (__syncthreads_or(!ok)) goto done;
+    tc_fence_after();
+    float dal = 0.f;                      // dout . o_swa for this row
+    for (int ch = 0; ch < 4; ++ch) {
+      float v[32];
+      tmem_ld32(tb + lane_off + C_O + ch * 32, v);
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8) {
+        float o8[8];
+        unpack8(*chunk_ptr(sm, R_O, row, ch * 4 + c8), o8);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) dal = fmaf(o8[u], v[c8 * 8 + u], dal);
+      }
+    }
+#pragma unroll
+    for (int m = 0; m < MAXM; ++m) dal = fmaf(em[m], dom[m], dal);
+    dal *= inv_l;
+    if (!qvalid) dal = 0.f;
+    const float Dt = alpha * dal;
+    if (qvalid) p.Dterm[(size_t)bh * p.L + tq] = Dt;
+    if (p.dalpha) {
+      const float w = warp_sum(dal);
+      if (lane == 0) s_red[warp] = w;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0 && p.dalpha) atomicAdd(p.dalpha + h, s_red[0] + s_red[1] + s_red[2] + s_red[3]);
+
+    // 4. dP' = dO [V_prev ; V]^T
+    if (tid == 0) {
+      tc_fence_after();
+      for (int s = 0; s < 8; ++s) mma_ss(tb + C_DP, desc_k(sbase + R_O, s), desc_k(sbase + R_VP, s), id_kk, s > 0);
+      for (int s = 0; s < 8; ++s) mma_ss(tb + C_DP + 128, desc_k(sbase + R_O, s), desc_k(sbase + R_V, s), id_kk, s > 0);
+      mma_commit(&bars[3]);
+    }
+    ok = mbar_wait(&bars[3], 0, p.status, ST_TIMEOUT);
+    if (__syncthreads_or(!ok)) goto done;
+    tc_fence_after();
+
+    // 5. dS = P (alpha dP' - D), P = P^ / l; the meta terms go to memory
+    for (int ch = 0; ch < 8; ++ch) {
+      float dp[32], pp[32];
+      tmem_ld32(tb + lane_off + C_DP + ch * 32, dp);
+      float pk16[16];
+      tmem_ld16(tb + lane_off + C_P + ch * 16, pk16);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const uint32_t w = __float_as_uint(pk16[u]);
+        pp[2 * u] = __uint_as_float(w << 16);
+        pp[2 * u + 1] = __uint_as_float(w & 0xffff0000u);
+      }
+      uint32_t ds[16];
+#pragma unroll
+      for (int u = 0; u < 32; u += 2)
+        ds[u / 2] = pack_bf16(pp[u] * inv_l * (alpha * dp[u] - Dt), pp[u + 1] * inv_l * (alpha * dp[u + 1] - Dt));
+      tmem_st8(tb + lane_off + C_DS + ch * 16, ds);
+      tmem_st8(tb + lane_off + C_DS + ch * 16 + 8, ds + 8);
+    }
+    float dsm[MAXM];
+#pragma unroll
+    for (int m = 0; m < MAXM; ++m) {
+      const float pm = em[m] * inv_l;
+      dsm[m] = pm * (alpha * dom[m] - Dt);
+      if (m < p.M && qvalid) {
+        p.dsm[((size_t)bh * p.L + tq) * MAXM + m] = dsm[m];
+        p.pm[((size_t)bh * p.L + tq) * MAXM + m] = pm;
+      }
+    }
+    tmem_st_wait();
+    tc_fence_before();
+    __syncthreads();
+
+    // 6. dq' = dS [K_prev ; K]
+    if (tid == 0) {
+      tc_fence_after();
+      for (int s = 0; s < 8; ++s) mma_ts(tb + C_DQ, tb + C_DS + s * 8, desc_mn(sbase + R_KP, s), id_mn, s > 0);
+      for (int s = 0; s < 8; ++s) mma_ts(tb + C_DQ, tb + C_DS + 64 + s * 8, desc_mn(sbase + R_K, s), id_mn, 1);
+      mma_commit(&bars[4]);
+    }
+    ok = mbar_wait(&bars[4], 0, p.status, ST_TIMEOUT);
+    if (__syncthreads_or(!ok)) goto done;
+    tc_fence_after();
+    float *dst = p.dq + ((size_t)bh * p.L + (qvalid ? tq : 0)) * D;
+    for (int ch = 0; ch < 4; ++ch) {
+      float v[32];
+      tmem_ld32(tb + lane_off + C_DQ + ch * 32, v);
+#pragma unroll
+      for (int m = 0; m < MAXM; ++m)
+        if (m < p.M)
+#pragma unroll
+          for (int u = 0; u < 32; ++u) v[u] = fmaf(dsm[m], s_mk[m][ch * 32 + u], v[u]);
+      if (qvalid)
+#pragma unroll
+        for (int u = 0; u < 32; u += 4)
+          *reinterpret_cast<float4 *>(dst + ch * 32 + u) =
+              make_float4(v[u] * p.scale, v[u + 1] * p.scale, v[u + 2] * p.scale, v[u + 3] * p.scale);
+    }
+  }
+done:
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(s_tmem, 512);
+}
+
+// ------------------------------------------------------------ dk, dv ------
+__global__ void __launch_bounds__(128, 1) tc_swa_bwd_kv_kernel(const __grid_constant__ KVParams p) {
+  extern __shared__ unsigned char smraw[];
+  unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
+  __shared__ float s_lse[2 * T], s_D[2 * T];
+  __shared__ uint64_t bars[5];
+  __shared__ uint32_t s_tmem;
+  // regions: K, V, Q_a, dO_a, Q_b, dO_b  (query tiles kb and kb + 1)
+  constexpr uint32_t R_K = 0, R_V = TILE, R_Q0 = 2 * TILE, R_O0 = 3 * TILE;
+  // TMEM: S^T / P [0,128), dP^T / dS [128,256), dV [256,384), dK [384,512)
+  constexpr uint32_t C_S = 0, C_P = 0, C_DP = 128, C_DS = 128, C_DV = 256, C_DK = 384;
+
+  const int tid = threadIdx.x, warp = tid >> 5, row = tid;
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const int bh = blockIdx.y, h = bh % p.H, j0 = blockIdx.x * T, tk = j0 + row;
+  const float alpha = p.alpha ? p.alpha[h] : 1.f;
+  const uint32_t sbase = smem_u32(sm);
+  setup_cta(&s_tmem, bars, 5, tid);
+  for (int e = tid; e < 2 * T; e += 128) {
+    const int t = j0 + e;
+    s_lse[e] = t < p.L ? p.lse[(size_t)bh * p.L + t] : 0.f;
+    s_D[e] = t < p.L ? p.Dterm[(size_t)bh * p.L + t] : 0.f;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = s_tmem;
+  if (tid == 0) {
+    mbar_expect_tx(&bars[0], 6 * TILE);
+    for (int r = 0; r < 2; ++r) {
+      tma_load_3d(sm + R_K + r * kReg, &p.mk, &bars[0], 64 * r, j0, bh);
+      tma_load_3d(sm + R_V + r * kReg, &p.mv, &bars[0], 64 * r, j0, bh);
+      for (int it = 0; it < 2; ++it) {
+        tma_load_3d(sm + R_Q0 + it * 2 * TILE + r * kReg, &p.mq, &bars[0], 64 * r, j0 + it * T, bh);
+        tma_load_3d(sm + R_O0 + it * 2 * TILE + r * kReg, &p.mo, &bars[0], 64 * r, j0 + it * T, bh);
+      }
+    }
+  }
+  const uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
+  const uint32_t id_mn = idesc_bf16(128, 128, 0, 1);
+  bool ok = mbar_wait(&bars[0], 0, p.status, ST_TIMEOUT);
+  if (__syncthreads_or(!ok)) goto done;
+  for (int it = 0; it < 2; ++it) {
+    const uint32_t rq = R_Q0 + it * 2 * TILE, ro = R_O0 + it * 2 * TILE;
+    // S^T = K Q^T, dP^T = V dO^T   (rows = keys of this block)
+    if (tid == 0) {
+      tc_fence_after();
+      for (int s = 0; s < 8; ++s) mma_ss(tb + C_S, desc_k(sbase + R_K, s), desc_k(sbase + rq, s), id_kk, s > 0);
+      for (int s = 0; s < 8; ++s) mma_ss(tb + C_DP, desc_k(sbase + R_V, s), desc_k(sbase + ro, s), id_kk, s > 0);
+      mma_commit(&bars[1 + 2 * it]);
+    }
+    ok = mbar_wait(&bars[1 + 2 * it], 0, p.status, ST_TIMEOUT);
+    if (__syncthreads_or(!ok)) goto done;
+    tc_fence_after();
+    // P = exp(scale s - lse_t), dS = P (alpha dP - D_t) on the band t - w < j <= t
+    for (int ch = 0; ch < 4; ++ch) {
+      float sv[32], dv[32];
+      tmem_ld32(tb + lane_off + C_S + ch * 32, sv);
+      tmem_ld32(tb + lane_off + C_DP + ch * 32, dv);
+      uint32_t pk[16], dk[16];
+#pragma unroll
+      for (int u = 0; u < 32; u += 2) {
+        float pr[2], ds[2];
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          const int qi = it * T + ch * 32 + u + w;       // query row within the two tiles
+          const int t = j0 + qi;
+          const bool valid = t < p.L && tk < p.L && t >= tk && t - tk < p.window;
+          pr[w] = valid ? __expf(sv[u + w] * p.scale - s_lse[qi]) : 0.f;
+          ds[w] = pr[w] * (alpha * dv[u + w] - s_D[qi]);
+        }
+        pk[u / 2] = pack_bf16(pr[0], pr[1]);
+        dk[u / 2] = pack_bf16(ds[0], ds[1]);
+      }
+      tmem_st8(tb + lane_off + C_P + ch * 16, pk);
+      tmem_st8(tb + lane_off + C_P + ch * 16 + 8, pk + 8);
+      tmem_st8(tb + lane_off + C_DS + ch * 16, dk);
+      tmem_st8(tb + lane_off + C_DS + ch * 16 + 8, dk + 8);
+    }
+    tmem_st_wait();
+    tc_fence_before();
+    __syncthreads();
+    // dV += P dO, dK += dS Q   (K dimension = the 128 queries of this tile)
+    if (tid == 0) {
+      tc_fence_after();
+      for (int s = 0; s < 8; ++s) mma_ts(tb + C_DV, tb + C_P + s * 8, desc_mn(sbase + ro, s), id_mn, it > 0 || s > 0);
+      for (int s = 0; s < 8; ++s) mma_ts(tb + C_DK, tb + C_DS + s * 8, desc_mn(sbase + rq, s), id_mn, it > 0 || s > 0);
+      mma_commit(&bars[2 + 2 * it]);
+    }
+    ok = mbar_wait(&bars[2 + 2 * it], 0, p.status, ST_TIMEOUT);
+    if (__syncthreads_or(!ok)) goto done;
+    tc_fence_after();
+  }
+  {
+    const bool kvalid = tk < p.L;
+    float *dkr = p.dk + ((size_t)bh * p.L + (kvalid ? tk : 0)) * D;
+    float *dvr = p.dv + ((size_t)bh * p.L + (kvalid ? tk : 0)) * D;
+    for (int ch = 0; ch < 4; ++ch) {
+      float a[32], b[32];
+      tmem_ld32(tb + lane_off + C_DK + ch * 32, a);
+      tmem_ld32(tb + lane_off + C_DV + ch * 32, b);
+      if (kvalid)
+#pragma unroll
+        for (int u = 0; u < 32; u += 4) {
+          *reinterpret_cast<float4 *>(dkr + ch * 32 + u) =
+              make_float4(a[u] * p.scale, a[u + 1] * p.scale, a[u + 2] * p.scale, a[u + 3] * p.scale);
+          *reinterpret_cast<float4 *>(dvr + ch * 32 + u) =
+              make_float4(b[u] * alpha, b[u + 1] * alpha, b[u + 2] * alpha, b[u + 3] * alpha);
+        }
+    }
+  }
+done:
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(s_tmem, 512);
+}
+
+// ------------------------------------------------------- meta gradients ---
+// dmeta_k[h][m] += scale sum_t dSm[t][m] q_t ; dmeta_v[h][m] += alpha sum_t pm[t][m] dout_t
+constexpr int kMetaTok = 1024;
+__global__ void __launch_bounds__(128) meta_grad_kernel(const __nv_bfloat16 *q, const __nv_bfloat16 *dout,
+                                                         const float *dsm, const float *pm, const float *alpha,
+                                                         float *dmk, float *dmv, int B, int H, int L, int M,
+                                                         float scale) {
+  const int h = blockIdx.y, i = threadIdx.x;
+  const int n0 = blockIdx.x * kMetaTok;
+  const int ntok = B * L;
+  float ak[MAXM], av[MAXM];
+#pragma unroll
+  for (int m = 0; m < MAXM; ++m) { ak[m] = 0.f; av[m] = 0.f; }
+  for (int n = n0; n < min(ntok, n0 + kMetaTok); ++n) {
+    const int b = n / L, t = n % L;
+    const size_t tok = ((size_t)b * H + h) * L + t;
+    const float qi = __bfloat162float(q[tok * D + i]);
+    const float oi = __bfloat162float(dout[tok * D + i]);
+#pragma unroll
+    for (int m = 0; m < MAXM; ++m) {
+      if (m < M) {
+        ak[m] = fmaf(dsm[tok * MAXM + m], qi, ak[m]);
+        av[m] = fmaf(pm[tok * MAXM + m], oi, av[m]);
+      }
+    }
+  }
+  const float a = alpha ? alpha[h] : 1.f;
+#pragma unroll
+  for (int m = 0; m < MAXM; ++m) {
+    if (m < M) {
+      if (dmk) atomicAdd(dmk + ((size_t)h * M + m) * D + i, ak[m] * scale);
+      if (dmv) atomicAdd(dmv + ((size_t)h * M + m) * D + i, av[m] * a);
+    }
+  }
+}
+
+}  // namespace
+
+bool tc_swa_bwd_supported(int dk, int dv, int window, int M, bool bf16) {
+  return bf16 && dk == D && dv == D && window <= T && M <= MAXM;
+}
+
+cudaError_t launch_tc_swa_bwd(const TcSwaBwdArgs &a, int stage, cudaStream_t s) {
+  const int ntiles = (a.L + T - 1) / T;
+  const uint64_t rows = (uint64_t)a.L;
+  if (stage == 2) {
+    if (a.M == 0 || (!a.dmeta_k && !a.dmeta_v)) return cudaSuccess;
+    dim3 grid((a.B * a.L + kMetaTok - 1) / kMetaTok, a.H);
+    meta_grad_kernel<<<grid, 128, 0, s>>>(static_cast<const __nv_bfloat16 *>(a.q),
+                                          static_cast<const __nv_bfloat16 *>(a.dout), a.dsm, a.pm, a.alpha,
+                                          a.dmeta_k, a.dmeta_v, a.B, a.H, a.L, a.M, a.scale);
+    return cudaGetLastError();
+  }
+  // the attribute is per device: set it every launch on devices not yet seen
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (stage == 0) {
+    QParams p;
+    memset(&p, 0, sizeof(p));
+    if (!make_map_bf16_3d(&p.mq, a.q, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mk, a.k, D, rows, a.BH, T) ||
+        !make_map_bf16_3d(&p.mv, a.v, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mo, a.dout, D, rows, a.BH, T))
+      return cudaErrorInvalidValue;
+    p.meta_k = a.meta_k;
+    p.meta_v = a.meta_v;
+    p.alpha = a.alpha;
+    p.dq = a.dq;
+    p.lse = a.lse;
+    p.Dterm = a.Dterm;
+    p.dsm = a.dsm;
+    p.pm = a.pm;
+    p.dalpha = a.dalpha;
+    p.status = a.status;
+    p.H = a.H;
+    p.L = a.L;
+    p.M = a.M;
+    p.window = a.window;
+    p.scale = a.scale;
+    e = cudaFuncSetAttribute(tc_swa_bwd_q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    tc_swa_bwd_q_kernel<<<dim3(ntiles, a.BH), 128, SMEM_BYTES, s>>>(p);
+    return cudaGetLastError();
+  }
+  KVParams p;
+  memset(&p, 0, sizeof(p));
+  if (!make_map_bf16_3d(&p.mq, a.q, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mk, a.k, D, rows, a.BH, T) ||
+      !make_map_bf16_3d(&p.mv, a.v, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mo, a.dout, D, rows, a.BH, T))
+    return cudaErrorInvalidValue;
+  p.alpha = a.alpha;
+  p.lse = a.lse;
+  p.Dterm = a.Dterm;
+  p.dk = a.dk;
+  p.dv = a.dv;
+  p.status = a.status;
+  p.H = a.H;
+  p.L = a.L;
+  p.window = a.window;
+  p.scale = a.scale;
+  e = cudaFuncSetAttribute(tc_swa_bwd_kv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  tc_swa_bwd_kv_kernel<<<dim3(ntiles, a.BH), 128, SMEM_BYTES, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace lz

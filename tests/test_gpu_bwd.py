@@ -12,7 +12,13 @@ pytestmark = pytest.mark.gpu
 
 GRADS = ["dq", "dk", "dv", "dg", "dmeta_k", "dmeta_v", "dfmap_wq", "dfmap_wk", "dalpha",
          "dstate_in"]
-IMPLS = ["simt"]
+IMPLS = ["simt", "tc"]
+
+
+def _skip_unsupported(impl, dtype, d, window, M):
+    """The tensor-core backward kernels cover bf16, d = 128, window <= 128, M <= 16."""
+    if impl == "tc" and not (dtype == "bf16" and d == 128 and window <= 128 and M <= 16):
+        pytest.skip("shape outside the tensor-core backward")
 
 
 @pytest.fixture(scope="module")
@@ -55,6 +61,7 @@ SWEEP = [
 @pytest.mark.parametrize("impl", IMPLS)
 @pytest.mark.parametrize("dtype,d,L,window,M,with_mv,with_state,rand_alpha", SWEEP)
 def test_backward_sweep(lz, impl, dtype, d, L, window, M, with_mv, with_state, rand_alpha):
+    _skip_unsupported(impl, dtype, d, window, M)
     w = Workload("bsweep", B=2, H=2, L=L, d=d, window=window, M=M, dtype=dtype,
                  seed=100 + L, kind="train")
     inp = make_inputs(w)
@@ -78,17 +85,37 @@ def test_backward_sweep(lz, impl, dtype, d, L, window, M, with_mv, with_state, r
 @pytest.mark.parametrize("impl", IMPLS)
 @pytest.mark.parametrize("branch", [ref.BRANCH_GLA_ONLY, ref.BRANCH_SWA_ONLY])
 def test_backward_branch_hooks(lz, impl, branch):
-    w = Workload("bbranch", B=1, H=2, L=90, d=64, window=10, M=4, dtype="fp32", seed=5,
+    dtype, d = ("fp32", 64) if impl == "simt" else ("bf16", 128)
+    w = Workload("bbranch", B=1, H=2, L=90, d=d, window=10, M=4, dtype=dtype, seed=5,
                  kind="train")
     inp = make_inputs(w)
     inp["alpha"] = random_alpha(2, seed=1)
     got = _run(lz, to_device(inp), w, _impl(lz, impl), branch=branch)
     want = oracle_backward(inp, window=w.window, tau=w.gate_temp, branch=branch)
     for name in GRADS:
-        check(name, got[name], want[name], "fp32")
+        check(name, got[name], want[name], dtype)
 
 
 @pytest.mark.parametrize("impl", IMPLS)
+def test_backward_alpha_zero_and_sink_only(lz, impl):
+    """alpha = 0 on one head (the anchor branch still has a gradient for
+    alpha) and sink-only meta tokens (no meta values)."""
+    dtype, d = ("fp32", 64) if impl == "simt" else ("bf16", 128)
+    w = Workload("balpha", B=2, H=2, L=200, d=d, window=64, M=4, dtype=dtype, seed=41,
+                 kind="train")
+    inp = make_inputs(w)
+    inp["alpha"] = torch.tensor([0.0, 1.3])
+    inp["meta_v"] = None
+    got = _run(lz, to_device(inp), w, _impl(lz, impl))
+    want = oracle_backward(inp, window=w.window, tau=w.gate_temp)
+    for name in GRADS:
+        if want[name] is None:
+            assert got[name] is None
+            continue
+        check(name, got[name], want[name], dtype)
+
+
+@pytest.mark.parametrize("impl", ["simt"])
 def test_backward_extreme_decay(lz, impl):
     w = Workload("bextreme", B=1, H=2, L=100, d=64, window=6, M=2, dtype="fp32", seed=6,
                  kind="train")
