@@ -86,8 +86,15 @@ bool bwd_swa_uses_tc(const lizard_fwd_args *a, int impl) {
   return (impl == LIZARD_IMPL_AUTO || impl == LIZARD_IMPL_TC) && ok;
 }
 
+// Whether the backward's GLA branch runs on the tensor-core kernels.
+bool bwd_gla_uses_tc(const lizard_fwd_args *a, int impl) {
+  const bool ok = a->dtype == LIZARD_BF16 && a->dk == 128 && a->dv == 128;
+  return (impl == LIZARD_IMPL_AUTO || impl == LIZARD_IMPL_TC) && ok;
+}
+
 struct BwdLayout {
-  size_t phq, phk, a, sprev, dphq, dphk, da, dv_gla, dq_swa, dk_swa, dv_swa, lse, Dterm, dsm, pm, total;
+  size_t phq, phk, a, sprev, dphq, dphk, da, dv_gla, dq_swa, dk_swa, dv_swa, lse, Dterm, dsm, pm, snap_s,
+      snap_ds, total;
 };
 BwdLayout bwd_layout(const lizard_fwd_args *a, int impl) {
   const size_t BH = (size_t)a->B * a->H;
@@ -97,7 +104,15 @@ BwdLayout bwd_layout(const lizard_fwd_args *a, int impl) {
   const size_t nch = (a->L + lz::kBwdC - 1) / lz::kBwdC;
   BwdLayout l{};
   size_t off = kHeader;
-  if (gla_on(a)) {
+  if (gla_on(a) && bwd_gla_uses_tc(a, impl)) {
+    const size_t snap = up(lz::tc_gla_bwd_snapshot_bytes((int)BH, a->L));
+    l.snap_s = off; off += snap;
+    l.snap_ds = off; off += snap;
+    l.dphq = off; off += nd;
+    l.dphk = off; off += nd;
+    l.da = off; off += nd;       // dB: gradient of the in-tile cumulative log-decay
+    l.dv_gla = off; off += nv;
+  } else if (gla_on(a)) {
     l.phq = off; off += nd;
     l.phk = off; off += nd;
     l.a = off; off += nd;
@@ -196,7 +211,20 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan) {
   const bool bf16 = a->dtype == LIZARD_BF16;
   const float inv_tau = 1.f / a->gate_temp;
   const bool g = gla_on(a), w = swa_on(a);
-  if (g) {
+  const bool gla_tc = g && bwd_gla_uses_tc(a, b->impl);
+  if (gla_tc) {
+    lz::TcFwdArgs f{a->q, a->k, a->v, a->g, a->fmap_wq, a->fmap_wk, a->meta_k, a->meta_v, a->alpha,
+                    a->state_in, nullptr, nullptr, nullptr, static_cast<uint32_t *>(ws), nullptr, BH, a->H,
+                    a->L, a->M, a->window, 0, inv_tau, scale_of(a)};
+    void *snap_s = at<void>(ws, lay.snap_s);
+    plan.add("tc_fwd_kernel(state copies)", [=] { return lz::launch_tc_state_snapshots(f, snap_s, s); });
+    lz::TcGlaBwdArgs t{a->q, a->k, a->v, a->g, b->dout, a->fmap_wq, a->fmap_wk, snap_s,
+                       at<void>(ws, lay.snap_ds), at<float>(ws, lay.dphq), at<float>(ws, lay.dphk),
+                       at<float>(ws, lay.da), at<float>(ws, lay.dv_gla), b->dg, b->dstate_in,
+                       static_cast<uint32_t *>(ws), a->H, BH, a->L, inv_tau};
+    plan.add("tc_gla_dstates_kernel", [=] { return lz::launch_tc_gla_bwd(t, 0, s); });
+    plan.add("tc_gla_bwd_tile_kernel", [=] { return lz::launch_tc_gla_bwd(t, 1, s); });
+  } else if (g) {
     lz::PrepArgs pa{a->q, a->k, a->g, a->fmap_wq, a->fmap_wk, at<float>(ws, lay.phq), at<float>(ws, lay.phk),
                     at<float>(ws, lay.a), a->H, a->L, inv_tau};
     plan.add("prep_kernel", [=] { return lz::launch_prep(pa, BH, D, bf16, s); });
@@ -232,8 +260,16 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan) {
                        g ? at<float>(ws, lay.da) : nullptr, g ? at<float>(ws, lay.dv_gla) : nullptr,
                        w ? at<float>(ws, lay.dq_swa) : nullptr, w ? at<float>(ws, lay.dk_swa) : nullptr,
                        w ? at<float>(ws, lay.dv_swa) : nullptr,
-                       b->dq, b->dk, b->dv, b->dg, b->dfmap_wq, b->dfmap_wk, a->H, a->L, inv_tau};
+                       b->dq, b->dk, b->dv, b->dg, b->dfmap_wq, b->dfmap_wk, a->H, a->L, inv_tau,
+                       gla_tc ? 0 : 1};
+  if (gla_tc) fa.da = nullptr;   // the gate gradient comes from gate_grad_kernel
   plan.add("finish_bwd", [=] { return lz::launch_finish_bwd(fa, BH, D, bf16, s); });
+  if (gla_tc) {
+    lz::TcGlaBwdArgs t{a->q, a->k, a->v, a->g, b->dout, a->fmap_wq, a->fmap_wk, nullptr, nullptr, nullptr,
+                       nullptr, at<float>(ws, lay.da), nullptr, b->dg, nullptr, static_cast<uint32_t *>(ws),
+                       a->H, BH, a->L, inv_tau};
+    plan.add("gate_grad_kernel", [=] { return lz::launch_tc_gla_bwd(t, 2, s); });
+  }
 }
 
 }  // namespace
@@ -329,6 +365,7 @@ lizard_status lizard_attn_bwd(const lizard_bwd_args *b, lizard_stream_t stream) 
   if (st != LIZARD_OK) return st;
   const lizard_fwd_args *a = &b->fwd;
   if (b->impl == LIZARD_IMPL_TC && swa_on(a) && !bwd_swa_uses_tc(a, b->impl)) return LIZARD_ERR_UNSUPPORTED;
+  if (b->impl == LIZARD_IMPL_TC && gla_on(a) && !bwd_gla_uses_tc(a, b->impl)) return LIZARD_ERR_UNSUPPORTED;
   const BwdLayout lay = bwd_layout(a, b->impl);
   if (!b->workspace || b->workspace_bytes < lay.total) return LIZARD_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

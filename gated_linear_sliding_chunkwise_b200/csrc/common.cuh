@@ -48,6 +48,7 @@ LZ_DEV int warp_min_int(int v) {
 // stays inside the fp32/bf16 exponent range with margin.  Chunks whose
 // cumulative decay exceeds it take the per-element exact path instead.
 constexpr float kMaxSpread = 64.f;
+constexpr float kMaxSpreadExp = 6.2351490808e27f;   // exp(kMaxSpread)
 
 // Sentinel for "no valid logit yet" in online softmax (finite, so that
 // exp(m_old - m_new) never forms inf - inf).

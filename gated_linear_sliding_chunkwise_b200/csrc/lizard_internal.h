@@ -89,6 +89,7 @@ struct FinishBwdArgs {
   float *dg, *dwq, *dwk;                    // dwq/dwk accumulated atomically; may be null
   int H, L;
   float inv_tau;
+  int write_dg;                             // 0 when another kernel writes dg
 };
 
 struct TcFwdArgs {
@@ -114,6 +115,17 @@ struct TcSwaBwdArgs {
   float scale;
 };
 
+struct TcGlaBwdArgs {
+  const void *q, *k, *v, *g, *dout;
+  const float *wq, *wk;
+  void *snap_s, *snap_ds;       // bf16 [B*H][L/128][128][128]: S' and dS of every tile
+  float *dphq, *dphk, *dB, *dv; // fp32 [B*H*L][128]
+  float *dg, *dstate_in;
+  uint32_t *status;
+  int H, BH, L;
+  float inv_tau;
+};
+
 constexpr int kBwdC = 32;   // GLA chunk used by the portable backward
 
 cudaError_t launch_prep(const PrepArgs &a, int BH, int D, bool bf16, cudaStream_t s);
@@ -133,6 +145,10 @@ cudaError_t launch_swa_bwd_kv(const SwaBwdKVArgs &a, int BH, int D, bool bf16, c
 bool tc_swa_bwd_supported(int dk, int dv, int window, int M, bool bf16);
 // stage 0: dq pass, 1: dk/dv pass, 2: meta-token gradients
 cudaError_t launch_tc_swa_bwd(const TcSwaBwdArgs &a, int stage, cudaStream_t s);
+size_t tc_gla_bwd_snapshot_bytes(int BH, int L);
+cudaError_t launch_tc_state_snapshots(const TcFwdArgs &a, void *snap, cudaStream_t s);
+// stage 0: reverse dS pass, 1: per-tile gradients, 2: gate-logit gradient
+cudaError_t launch_tc_gla_bwd(const TcGlaBwdArgs &a, int stage, cudaStream_t s);
 cudaError_t launch_finish_bwd(const FinishBwdArgs &a, int BH, int D, bool bf16, cudaStream_t s);
 
 }  // namespace lz

@@ -759,9 +759,11 @@ __global__ void __launch_bounds__(256) finish_bwd(FinishBwdArgs p) {
           if (p.dv_gla) dvv += p.dv_gla[row + i];
           if (p.dv_swa) dvv += p.dv_swa[row + i];
           dvdst[row + i] = from_f32<T>(dvv);
-          float dg = 0.f;
-          if (p.da) dg = p.da[row + i] * dlogsigmoid(to_f32(gsrc[row + i])) * p.inv_tau;
-          p.dg[row + i] = dg;
+          if (p.write_dg) {
+            float dg = 0.f;
+            if (p.da) dg = p.da[row + i] * dlogsigmoid(to_f32(gsrc[row + i])) * p.inv_tau;
+            p.dg[row + i] = dg;
+          }
         }
       }
     }

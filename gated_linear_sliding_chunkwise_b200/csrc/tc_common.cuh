@@ -216,5 +216,56 @@ __device__ __forceinline__ uint64_t desc_mn(uint32_t tile_addr, int s) {
   return sdesc_sw128(tile_addr + s * 2048, kReg, 1024);
 }
 
+// logsigmoid(g) / tau with the fast exp/log (bf16 inputs make the last ulps moot)
+__device__ __forceinline__ float log_decay_fast(float g, float inv_tau) {
+  return (fminf(g, 0.f) - __logf(1.f + __expf(-fabsf(g)))) * inv_tau;
+}
+
+// In-tile decay factors in fp32, thread = tile row t (128 threads, 4 warps),
+// for the 16 key dimensions 16 c16 .. 16 c16 + 15:
+//   E[u]   = exp(sum_{s > t} -a_s)   (= exp(b_t - r), b the in-tile cumsum)
+//   tot[u] = sum_{all s} -a_s         (= -r)
+// from the bf16 gate logits of a 128 x 128 tile (a_s = logsigmoid(g)/tau,
+// zero for rows at or beyond L).  Suffix sums: a shuffle scan within each
+// warp, then the later warps' totals from shared memory `wtot` [4][16].
+// All 128 threads must call it (it synchronises the block twice).
+__device__ __forceinline__ void row_decay16(unsigned char *gtile, int row, int c16, bool valid, float inv_tau,
+                                            float (*wtot)[16], float *E, float *tot) {
+  const int lane = row & 31, warp = row >> 5;
+  float na[16], x[16];
+  unpack8(*chunk_ptr(gtile, 0, row, 2 * c16), na);
+  unpack8(*chunk_ptr(gtile, 0, row, 2 * c16 + 1), na + 8);
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    na[u] = valid ? -log_decay_fast(na[u], inv_tau) : 0.f;
+    x[u] = na[u];
+  }
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const float y = __shfl_down_sync(0xffffffffu, x[u], off);
+      if (lane + off < 32) x[u] += y;
+    }
+  }
+  if (lane == 0)
+#pragma unroll
+    for (int u = 0; u < 16; ++u) wtot[warp][u] = x[u];
+  __syncthreads();
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    float later = 0.f, all = 0.f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const float v = wtot[w][u];
+      all += v;
+      if (w > warp) later += v;
+    }
+    E[u] = __expf(x[u] - na[u] + later);
+    tot[u] = all;
+  }
+  __syncthreads();
+}
+
 }  // namespace tc
 }  // namespace lz

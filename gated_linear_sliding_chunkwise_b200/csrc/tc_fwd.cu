@@ -84,16 +84,13 @@ struct Params {
   const float *seg_start;   // [BH][nseg][D][D] start state of each segment (nseg > 1)
   float *seg_state;         // mode 1: [BH][nseg][D][D] local end state (zero start)
   float *seg_decay;         // mode 1: [BH][nseg][D] summed log-decay of the segment
+  __nv_bfloat16 *snap;      // mode 1 with nseg == 1: [BH][ntiles][D][D] bf16 S' of every tile
   int H, L, M, window, branch;
   int mode;                 // 0: full forward, 1: state pass
   int nseg, tiles_per_seg;
   float inv_tau, scale;
 };
 
-// logsigmoid(g) / tau with the fast exp/log: bf16 inputs make the last ulps moot
-__device__ __forceinline__ float log_decay_fast(float g, float inv_tau) {
-  return (fminf(g, 0.f) - __logf(1.f + __expf(-fabsf(g)))) * inv_tau;
-}
 
 __device__ __forceinline__ void issue_tile_loads(const Params &p, unsigned char *sm, uint64_t *bar, int bh,
                                                  int t0, bool full) {
@@ -134,6 +131,7 @@ __global__ void __launch_bounds__(128, 1) tc_fwd_kernel(const __grid_constant__ 
   unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
   __shared__ float s_mk[MAXM][D], s_mv[MAXM][D];
   __shared__ float s_dec[D];
+  __shared__ float s_wtot[4][16];
   __shared__ uint64_t bar_tma, bar_vp, bar_m1, bar_m2, bar_m3;
   __shared__ uint32_t s_tmem;
   __shared__ int s_fail;
@@ -191,6 +189,7 @@ __global__ void __launch_bounds__(128, 1) tc_fwd_kernel(const __grid_constant__ 
     const float *src = nullptr;
     if (full && p.nseg > 1) src = p.seg_start + (((size_t)bh * p.nseg + seg) * D + row) * D;
     else if (full && p.state_in) src = p.state_in + ((size_t)bh * D + row) * D;
+    else if (p.snap && p.state_in) src = p.state_in + ((size_t)bh * D + row) * D;
 #pragma unroll
     for (int c = 0; c < D; c += 8) {
       uint32_t r[8];
@@ -235,7 +234,7 @@ __global__ void __launch_bounds__(128, 1) tc_fwd_kernel(const __grid_constant__ 
     }
 
     // ---------------------------------------------- gates (thread = dim) ---
-    {
+    if (full) {
       // 8 tokens per step: the logsigmoids and exps are independent, only
       // the running suffix sum is a chain
       const int i = row;
@@ -361,20 +360,61 @@ __global__ void __launch_bounds__(128, 1) tc_fwd_kernel(const __grid_constant__ 
       }
       }
       // phi_k -> Kt = phi_k / E, bf16 into shared memory over X_k
-      tmem_ld32(tb + lane_off + C_ZK, z);
-      tmem_ld32(tb + lane_off + C_ZK + 32, z + 32);
-      feature_map_row(z, neg);
+      if (full) {
+        tmem_ld32(tb + lane_off + C_ZK, z);
+        tmem_ld32(tb + lane_off + C_ZK + 32, z + 32);
+        feature_map_row(z, neg);
 #pragma unroll
-      for (int c8 = 0; c8 < 16; ++c8) {
-        float e8[8], k8[8];
-        unpack8(*chunk_ptr(sm, R_G, row, c8), e8);
+        for (int c8 = 0; c8 < 16; ++c8) {
+          float e8[8], k8[8];
+          unpack8(*chunk_ptr(sm, R_G, row, c8), e8);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int i = c8 * 8 + u;
-          const float ph = i < F ? z[i] : neg[i - F];
-          k8[u] = ph * __fdividef(1.f, e8[u]);
+          for (int u = 0; u < 8; ++u) {
+            const int i = c8 * 8 + u;
+            const float ph = i < F ? z[i] : neg[i - F];
+            k8[u] = ph * __fdividef(1.f, e8[u]);
+          }
+          *chunk_ptr(sm, R_XK, row, c8) = pack8(k8);
         }
-        *chunk_ptr(sm, R_XK, row, c8) = pack8(k8);
+      } else {
+        // state pass: E in fp32 from row-wise suffix sums (its states feed
+        // the backward and the segment chain), staged in the unused logits
+        // columns of TMEM
+        for (int c16 = 0; c16 < 8; ++c16) {
+          float E[16], tot[16];
+          row_decay16(sm + R_G, row, c16, qvalid, p.inv_tau, s_wtot, E, tot);
+          uint32_t r[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(E[u]);
+          tmem_st8(tb + lane_off + C_L + c16 * 16, r);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(E[8 + u]);
+          tmem_st8(tb + lane_off + C_L + c16 * 16 + 8, r);
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            if (row == c16 * 16 + u) {   // this thread's dimension
+              s_dec[row] = __expf(-tot[u]);   // exp(r)
+              tot_decay -= tot[u];             // r, the tile's log-decay
+            }
+            if (row == 0 && E[u] > kMaxSpreadExp && gla) atomicOr(err, ST_RANGE);
+          }
+        }
+        tmem_st_wait();
+        tmem_ld32(tb + lane_off + C_ZK, z);
+        tmem_ld32(tb + lane_off + C_ZK + 32, z + 32);
+        feature_map_row(z, neg);
+#pragma unroll
+        for (int c16 = 0; c16 < 8; ++c16) {
+          float E[16], k16[16];
+          tmem_ld16(tb + lane_off + C_L + c16 * 16, E);
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const int i = c16 * 16 + u;
+            k16[u] = (i < F ? z[i] : neg[i - F]) * __fdividef(1.f, E[u]);
+          }
+          *chunk_ptr(sm, R_XK, row, 2 * c16) = pack8(k16);
+          *chunk_ptr(sm, R_XK, row, 2 * c16 + 1) = pack8(k16 + 8);
+        }
       }
     }
 
@@ -397,6 +437,10 @@ __global__ void __launch_bounds__(128, 1) tc_fwd_kernel(const __grid_constant__ 
         if (full) {   // bf16 copy S'[i][v], MN-major: rows = i (K of the O = Qt S' product)
           *chunk_ptr(sm, R_XQ, i, 2 * c16) = pack8(v);
           *chunk_ptr(sm, R_XQ, i, 2 * c16 + 1) = pack8(v + 8);
+        } else if (p.snap) {   // the backward's copy of S', row-major [i][v]
+          uint4 *dst = reinterpret_cast<uint4 *>(p.snap + (((size_t)bh * ntiles_all + c) * D + i) * D + c16 * 16);
+          dst[0] = pack8(v);
+          dst[1] = pack8(v + 8);
         }
       }
     }
@@ -499,7 +543,7 @@ __global__ void __launch_bounds__(128, 1) tc_fwd_kernel(const __grid_constant__ 
 
   float *sdst = nullptr;
   if (full && p.state_out && gla && seg == p.nseg - 1) sdst = p.state_out + ((size_t)bh * D + row) * D;
-  if (!full) {
+  if (!full && p.seg_state) {
     sdst = p.seg_state + (((size_t)bh * p.nseg + seg) * D + row) * D;
     p.seg_decay[((size_t)bh * p.nseg + seg) * D + row] = tot_decay;
   }
@@ -568,6 +612,44 @@ int tc_fwd_stage_count(int BH, int L) {
   int nseg, tps;
   tc_fwd_segments(BH, L, &nseg, &tps);
   return nseg > 1 ? 3 : 1;
+}
+
+// Forward state pass over whole sequences that keeps, for every 128-token
+// tile, the bf16 state at the tile's start already decayed by the tile's
+// gates, S' = diag(exp r) S (the backward's input).
+cudaError_t launch_tc_state_snapshots(const TcFwdArgs &a, void *snap, cudaStream_t s) {
+  Params p;
+  memset(&p, 0, sizeof(p));
+  const uint64_t rows = (uint64_t)a.L;
+  if (!make_map_bf16_3d(&p.mq, a.q, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mk, a.k, D, rows, a.BH, T) ||
+      !make_map_bf16_3d(&p.mv, a.v, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mg, a.g, D, rows, a.BH, T))
+    return cudaErrorInvalidValue;
+  p.wq = a.wq;
+  p.wk = a.wk;
+  p.meta_k = a.meta_k;
+  p.meta_v = a.meta_v;
+  p.alpha = a.alpha;
+  p.state_in = a.state_in;
+  p.status = a.status;
+  p.snap = static_cast<__nv_bfloat16 *>(snap);
+  p.H = a.H;
+  p.L = a.L;
+  p.M = a.M;
+  p.window = a.window;
+  p.branch = 0;
+  p.mode = 1;
+  p.nseg = 1;
+  p.tiles_per_seg = (a.L + T - 1) / T;
+  p.inv_tau = a.inv_tau;
+  p.scale = a.scale;
+  // the state pass starts from state_in when there is one
+  p.seg_start = a.state_in;
+  p.seg_state = nullptr;
+  p.seg_decay = nullptr;
+  cudaError_t e = cudaFuncSetAttribute(tc_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  tc_fwd_kernel<<<dim3(a.BH, 1), 128, SMEM_BYTES, s>>>(p);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_tc_fwd(const TcFwdArgs &a, int stage, cudaStream_t s) {

@@ -1,0 +1,566 @@
+// Tensor-core (tcgen05 / TMEM / TMA) backward of the GLA branch, bf16,
+// dk = dv = 128, 128-token tiles (English gist.science summary, section
+// 2.A "State Update"; the gate absorbed into q and k in log space as the
+// Chinese summary, section 2.3, describes).
+//
+// Per tile, with E = exp(b - r) (b the in-tile cumulative log-decay, r its
+// value at the tile's end), Qt = phi_q E, Kt = phi_k / E, S' = diag(exp r) S
+// the tile's start state decayed over the tile, and dS the gradient into the
+// tile's end state:
+//   dA   = tril(dO V^T)                       (query x key)
+//   GQ   = dO S'^T + dA Kt                    dphi_q = E GQ
+//   GK   = dA^T Qt + V dS^T                   dphi_k = GK / E
+//   dv   = tril(Qt Kt^T)^T dO + Kt dS
+//   dB   = Qt GQ - Kt GK  (gradient of b; its reverse cumulative sum over the
+//          sequence is the log-decay gradient)
+//   dS_prev = diag(exp r) (dS + Qt^T dO)
+//
+// tc_gla_dstates_kernel  reverse pass per sequence: dS of every tile (bf16
+//                        copies) and the gradient of the initial state.
+// tc_gla_bwd_tile_kernel one CTA per (tile, sequence): the formulas above,
+//                        given the S' and dS copies.
+// gate_grad_kernel       reverse cumulative sum of dB -> gate-logit gradient.
+#include "common.cuh"
+#include "lizard_internal.h"
+#include "tc_common.cuh"
+#include "tc_host.h"
+
+namespace lz {
+namespace {
+
+using namespace tc;
+
+constexpr int T = 128;
+constexpr int D = 128;
+constexpr int F = D / 2;
+constexpr uint32_t TILE = kTile;
+constexpr uint32_t REG = kReg;
+constexpr uint32_t ST_TIMEOUT = 1u, ST_RANGE = 2u;
+
+struct DsParams {
+  CUtensorMap mq, mg, mo;
+  const float *wq;
+  __nv_bfloat16 *snap;      // [BH][ntiles][D][D] dS at each tile's end
+  float *dstate_in;         // [BH][D][D] or null
+  uint32_t *status;
+  int H, L;
+  float inv_tau;
+};
+
+struct TileParams {
+  CUtensorMap mq, mk, mv, mo, mg, msp, mds;   // msp / mds: [BH*ntiles][D][D] snapshots
+  const float *wq, *wk;
+  float *dphq, *dphk, *dB, *dv;
+  uint32_t *status;
+  int H, L, ntiles;
+  float inv_tau;
+};
+
+
+// feature map of one row: z (64 projections) -> [softmax(z), softmax(-z)]
+__device__ __forceinline__ void feature_map_row(float *z, float *neg) {
+  float mx = z[0], mn = z[0];
+#pragma unroll
+  for (int f = 1; f < F; ++f) { mx = fmaxf(mx, z[f]); mn = fminf(mn, z[f]); }
+  float sp = 0.f, sn = 0.f;
+#pragma unroll
+  for (int f = 0; f < F; ++f) {
+    neg[f] = __expf(mn - z[f]);
+    z[f] = __expf(z[f] - mx);
+    sp += z[f];
+    sn += neg[f];
+  }
+  const float ip = 1.f / sp, in_ = 1.f / sn;
+#pragma unroll
+  for (int f = 0; f < F; ++f) { z[f] *= ip; neg[f] *= in_; }
+}
+
+// W (fp32 [D][F] of head h) -> bf16 shared memory, [dk row][feature], MN-major
+__device__ __forceinline__ void stage_weights(unsigned char *dst, const float *W, int h, int row) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    float f[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) f[u] = W ? W[((size_t)h * D + row) * F + c * 8 + u] : 0.f;
+    *reinterpret_cast<uint4 *>(dst + sw128_offset(row, c * 8)) = pack8(f);
+  }
+}
+
+// ------------------------------------------------------ reverse dS pass ---
+__global__ void __launch_bounds__(128, 1) tc_gla_dstates_kernel(const __grid_constant__ DsParams p) {
+  extern __shared__ unsigned char smraw[];
+  unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
+  __shared__ float s_dec[D];
+  __shared__ float s_wtot[4][16];
+  __shared__ uint64_t bar_tma, bar_m1, bar_m2;
+  __shared__ uint32_t s_tmem;
+  constexpr uint32_t R_XQ = 0, R_G = TILE, R_O = 2 * TILE, R_W = 3 * TILE;
+  constexpr uint32_t C_S = 0, C_Z = 128, C_E = 256;
+  const int tid = threadIdx.x, warp = tid >> 5, row = tid;
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const int bh = blockIdx.x, h = bh % p.H;
+  const uint32_t sbase = smem_u32(sm);
+  const int ntiles = (p.L + T - 1) / T;
+  if (warp == 0) { tmem_alloc(&s_tmem, 512); tmem_relinquish(); }
+  if (tid == 0) {
+    mbar_init(&bar_tma, 1);
+    mbar_init(&bar_m1, 1);
+    mbar_init(&bar_m2, 1);
+    fence_barrier_init();
+  }
+  stage_weights(sm + R_W, p.wq, h, row);
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = s_tmem;
+  {   // dS starts at zero: nothing flows into the last tile's end state
+    uint32_t z[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int c = 0; c < D; c += 8) tmem_st8(tb + lane_off + C_S + c, z);
+    tmem_st_wait();
+  }
+  const uint32_t id_z = idesc_bf16(128, 64, 0, 1);
+  const uint32_t id_st = idesc_bf16(128, 128, 1, 1);
+  auto loads = [&](int c) {
+    mbar_expect_tx(&bar_tma, 3 * TILE);
+    for (int r = 0; r < 2; ++r) {
+      tma_load_3d(sm + R_XQ + r * REG, &p.mq, &bar_tma, 64 * r, c * T, bh);
+      tma_load_3d(sm + R_G + r * REG, &p.mg, &bar_tma, 64 * r, c * T, bh);
+      tma_load_3d(sm + R_O + r * REG, &p.mo, &bar_tma, 64 * r, c * T, bh);
+    }
+  };
+  if (tid == 0 && ntiles > 0) loads(ntiles - 1);
+  bool fail = false;
+  for (int c = ntiles - 1; c >= 0; --c) {
+    const uint32_t par = (ntiles - 1 - c) & 1;
+    const int t0 = c * T;
+    bool ok = mbar_wait(&bar_tma, par, p.status, ST_TIMEOUT);
+    if (__syncthreads_or(!ok)) { fail = true; break; }
+    if (tid == 0) {
+      tc_fence_after();
+      for (int s = 0; s < 8; ++s) mma_ss(tb + C_Z, desc_k(sbase + R_XQ, s), desc_mn(sbase + R_W, s), id_z, s > 0);
+      mma_commit(&bar_m1);
+    }
+    // copy of dS (the gradient into this tile's end state)
+    {
+      __nv_bfloat16 *dst = p.snap + (((size_t)bh * ntiles + c) * D + row) * D;
+      for (int ch = 0; ch < 4; ++ch) {
+        float v[32];
+        tmem_ld32(tb + lane_off + C_S + ch * 32, v);
+#pragma unroll
+        for (int u = 0; u < 32; u += 8) *reinterpret_cast<uint4 *>(dst + ch * 32 + u) = pack8(v + u);
+      }
+    }
+    ok = mbar_wait(&bar_m1, par, p.status, ST_TIMEOUT);
+    if (__syncthreads_or(!ok)) { fail = true; break; }
+    tc_fence_after();
+    // E in fp32 (row-wise suffix sums) into TMEM; the tile's decay exp(r)
+    for (int c16 = 0; c16 < 8; ++c16) {
+      float E[16], tot[16];
+      row_decay16(sm + R_G, row, c16, t0 + row < p.L, p.inv_tau, s_wtot, E, tot);
+      uint32_t r[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(E[u]);
+      tmem_st8(tb + lane_off + C_E + c16 * 16, r);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(E[8 + u]);
+      tmem_st8(tb + lane_off + C_E + c16 * 16 + 8, r);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        if (row == u) s_dec[c16 * 16 + u] = __expf(-tot[u]);
+        if (row == 0 && E[u] > kMaxSpreadExp) atomicOr(p.status, ST_RANGE);
+      }
+    }
+    tmem_st_wait();
+    {   // Qt = phi_q E into shared memory over X_q (row = token)
+      float z[F], neg[F];
+      tmem_ld32(tb + lane_off + C_Z, z);
+      tmem_ld32(tb + lane_off + C_Z + 32, z + 32);
+      feature_map_row(z, neg);
+#pragma unroll
+      for (int c16 = 0; c16 < 8; ++c16) {
+        float E[16], q16[16];
+        tmem_ld16(tb + lane_off + C_E + c16 * 16, E);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int i = c16 * 16 + u;
+          q16[u] = (i < F ? z[i] : neg[i - F]) * E[u];
+        }
+        *chunk_ptr(sm, R_XQ, row, 2 * c16) = pack8(q16);
+        *chunk_ptr(sm, R_XQ, row, 2 * c16 + 1) = pack8(q16 + 8);
+      }
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {   // dS += Qt^T dO
+      tc_fence_after();
+      for (int s = 0; s < 8; ++s) mma_ss(tb + C_S, desc_mn(sbase + R_XQ, s), desc_mn(sbase + R_O, s), id_st, 1);
+      mma_commit(&bar_m2);
+    }
+    ok = mbar_wait(&bar_m2, par, p.status, ST_TIMEOUT);
+    if (__syncthreads_or(!ok)) { fail = true; break; }
+    tc_fence_after();
+    if (tid == 0 && c > 0) loads(c - 1);
+    {   // dS_prev = diag(exp r) (dS + Qt^T dO)
+      const float dec = s_dec[row];
+      for (int ch = 0; ch < 8; ++ch) {
+        float v[16];
+        tmem_ld16(tb + lane_off + C_S + ch * 16, v);
+        uint32_t r[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(v[u] * dec);
+        tmem_st8(tb + lane_off + C_S + ch * 16, r);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(v[8 + u] * dec);
+        tmem_st8(tb + lane_off + C_S + ch * 16 + 8, r);
+      }
+      tmem_st_wait();
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
+  if (!fail && p.dstate_in) {
+    tc_fence_after();
+    float *dst = p.dstate_in + ((size_t)bh * D + row) * D;
+    for (int ch = 0; ch < 4; ++ch) {
+      float v[32];
+      tmem_ld32(tb + lane_off + C_S + ch * 32, v);
+#pragma unroll
+      for (int u = 0; u < 32; u += 4)
+        *reinterpret_cast<float4 *>(dst + ch * 32 + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tb, 512);
+}
+
+// ------------------------------------------------------------ per tile ----
+__global__ void __launch_bounds__(128, 1) tc_gla_bwd_tile_kernel(const __grid_constant__ TileParams p) {
+  extern __shared__ unsigned char smraw[];
+  unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
+  __shared__ float s_wtot[4][16];
+  __shared__ uint64_t bars[7];
+  __shared__ uint32_t s_tmem;
+  // X_q -> Qt, X_k -> Kt, V, dO, G (gate logits), [W_q | W_k] -> S' -> dS
+  constexpr uint32_t R_XQ = 0, R_XK = TILE, R_V = 2 * TILE, R_O = 3 * TILE, R_G = 4 * TILE, R_W = 5 * TILE;
+  // TMEM, in order of use:
+  //   dA [128,256) dA^T [256,384) Zq [384,448) Zk [448,512)
+  //   dA^ [128,192) dA^T^ [192,256) E (fp32) [0,128)
+  //   A^T [0,128) -> A^T^ [0,64)
+  //   GQ [256,384) GK [384,512) ; DV [128,256)
+  constexpr uint32_t C_E = 0, C_DA = 128, C_DAT = 256, C_ZQ = 384, C_ZK = 448, C_DAH = 128, C_DATH = 192;
+  constexpr uint32_t C_AT = 0, C_ATH = 0, C_GQ = 256, C_GK = 384, C_DV = 128;
+  const int tid = threadIdx.x, warp = tid >> 5, row = tid;
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const int c = blockIdx.x, bh = blockIdx.y, h = bh % p.H, t0 = c * T, tq = t0 + row;
+  const bool valid = tq < p.L;
+  const uint32_t sbase = smem_u32(sm);
+  if (warp == 0) { tmem_alloc(&s_tmem, 512); tmem_relinquish(); }
+  if (tid == 0) {
+    for (int i = 0; i < 7; ++i) mbar_init(&bars[i], 1);
+    fence_barrier_init();
+  }
+  stage_weights(sm + R_W, p.wq, h, row);
+  stage_weights(sm + R_W + REG, p.wk, h, row);
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = s_tmem;
+  const int snap_idx = bh * p.ntiles + c;
+  if (tid == 0) {
+    mbar_expect_tx(&bars[0], 5 * TILE);
+    for (int r = 0; r < 2; ++r) {
+      tma_load_3d(sm + R_XQ + r * REG, &p.mq, &bars[0], 64 * r, t0, bh);
+      tma_load_3d(sm + R_XK + r * REG, &p.mk, &bars[0], 64 * r, t0, bh);
+      tma_load_3d(sm + R_V + r * REG, &p.mv, &bars[0], 64 * r, t0, bh);
+      tma_load_3d(sm + R_O + r * REG, &p.mo, &bars[0], 64 * r, t0, bh);
+      tma_load_3d(sm + R_G + r * REG, &p.mg, &bars[0], 64 * r, t0, bh);
+    }
+  }
+  const uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
+  const uint32_t id_mn = idesc_bf16(128, 128, 0, 1);
+  const uint32_t id_z = idesc_bf16(128, 64, 0, 1);
+  bool ok = mbar_wait(&bars[0], 0, p.status, ST_TIMEOUT);
+  if (__syncthreads_or(!ok)) goto done;
+  // 1. dA = dO V^T, dA^T = V dO^T, Zq = X_q W_q, Zk = X_k W_k
+  if (tid == 0) {
+    tc_fence_after();
+    for (int s = 0; s < 8; ++s) mma_ss(tb + C_DA, desc_k(sbase + R_O, s), desc_k(sbase + R_V, s), id_kk, s > 0);
+    for (int s = 0; s < 8; ++s) mma_ss(tb + C_DAT, desc_k(sbase + R_V, s), desc_k(sbase + R_O, s), id_kk, s > 0);
+    for (int s = 0; s < 8; ++s) mma_ss(tb + C_ZQ, desc_k(sbase + R_XQ, s), desc_mn(sbase + R_W, s), id_z, s > 0);
+    for (int s = 0; s < 8; ++s) mma_ss(tb + C_ZK, desc_k(sbase + R_XK, s), desc_mn(sbase + R_W + REG, s), id_z, s > 0);
+    mma_commit(&bars[1]);
+  }
+  ok = mbar_wait(&bars[1], 0, p.status, ST_TIMEOUT);
+  if (__syncthreads_or(!ok)) goto done;
+  tc_fence_after();
+  if (tid == 0) {   // the weights are consumed: S' goes into their place
+    mbar_expect_tx(&bars[2], TILE);
+    tma_load_3d(sm + R_W, &p.msp, &bars[2], 0, 0, snap_idx);
+    tma_load_3d(sm + R_W + REG, &p.msp, &bars[2], 64, 0, snap_idx);
+  }
+  // 2. masked dA (row = query; written over its own columns as read) ...
+  for (int ch = 0; ch < 4; ++ch) {
+    float v[32];
+    tmem_ld32(tb + lane_off + C_DA + ch * 32, v);
+    uint32_t a[16];
+#pragma unroll
+    for (int u = 0; u < 32; u += 2) {
+      const int j = ch * 32 + u;          // key j <= query row
+      a[u / 2] = pack_bf16(j <= row ? v[u] : 0.f, j + 1 <= row ? v[u + 1] : 0.f);
+    }
+    tmem_st8(tb + lane_off + C_DAH + ch * 16, a);
+    tmem_st8(tb + lane_off + C_DAH + ch * 16 + 8, a + 8);
+  }
+  //    ... then masked dA^T (row = key) into the consumed upper half of dA
+  for (int ch = 0; ch < 4; ++ch) {
+    float w[32];
+    tmem_ld32(tb + lane_off + C_DAT + ch * 32, w);
+    uint32_t b[16];
+#pragma unroll
+    for (int u = 0; u < 32; u += 2) {
+      const int j = ch * 32 + u;          // query j >= key row
+      b[u / 2] = pack_bf16(j >= row ? w[u] : 0.f, j + 1 >= row ? w[u + 1] : 0.f);
+    }
+    tmem_st8(tb + lane_off + C_DATH + ch * 16, b);
+    tmem_st8(tb + lane_off + C_DATH + ch * 16 + 8, b + 8);
+  }
+  //    E in fp32 (row-wise suffix sums) into TMEM, then Qt = phi_q E, Kt = phi_k / E
+  for (int c16 = 0; c16 < 8; ++c16) {
+    float E[16], tot[16];
+    row_decay16(sm + R_G, row, c16, valid, p.inv_tau, s_wtot, E, tot);
+    uint32_t r[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(E[u]);
+    tmem_st8(tb + lane_off + C_E + c16 * 16, r);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(E[8 + u]);
+    tmem_st8(tb + lane_off + C_E + c16 * 16 + 8, r);
+#pragma unroll
+    for (int u = 0; u < 16; ++u)
+      if (row == 0 && E[u] > kMaxSpreadExp) atomicOr(p.status, ST_RANGE);
+  }
+  tmem_st_wait();
+  {
+    float z[F], neg[F];
+    tmem_ld32(tb + lane_off + C_ZQ, z);
+    tmem_ld32(tb + lane_off + C_ZQ + 32, z + 32);
+    feature_map_row(z, neg);
+#pragma unroll
+    for (int c16 = 0; c16 < 8; ++c16) {
+      float E[16], q16[16];
+      tmem_ld16(tb + lane_off + C_E + c16 * 16, E);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int i = c16 * 16 + u;
+        q16[u] = (i < F ? z[i] : neg[i - F]) * E[u];
+      }
+      *chunk_ptr(sm, R_XQ, row, 2 * c16) = pack8(q16);
+      *chunk_ptr(sm, R_XQ, row, 2 * c16 + 1) = pack8(q16 + 8);
+    }
+    tmem_ld32(tb + lane_off + C_ZK, z);
+    tmem_ld32(tb + lane_off + C_ZK + 32, z + 32);
+    feature_map_row(z, neg);
+#pragma unroll
+    for (int c16 = 0; c16 < 8; ++c16) {
+      float E[16], k16[16];
+      tmem_ld16(tb + lane_off + C_E + c16 * 16, E);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int i = c16 * 16 + u;
+        k16[u] = (i < F ? z[i] : neg[i - F]) * __fdividef(1.f, E[u]);
+      }
+      *chunk_ptr(sm, R_XK, row, 2 * c16) = pack8(k16);
+      *chunk_ptr(sm, R_XK, row, 2 * c16 + 1) = pack8(k16 + 8);
+    }
+  }
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+  // 3. A^T = Kt Qt^T (rows = keys), over E
+  if (tid == 0) {
+    tc_fence_after();
+    for (int s = 0; s < 8; ++s) mma_ss(tb + C_AT, desc_k(sbase + R_XK, s), desc_k(sbase + R_XQ, s), id_kk, s > 0);
+    mma_commit(&bars[3]);
+  }
+  ok = mbar_wait(&bars[3], 0, p.status, ST_TIMEOUT);
+  if (__syncthreads_or(!ok)) goto done;
+  tc_fence_after();
+  for (int ch = 0; ch < 4; ++ch) {
+    float v[32];
+    tmem_ld32(tb + lane_off + C_AT + ch * 32, v);
+    uint32_t a[16];
+#pragma unroll
+    for (int u = 0; u < 32; u += 2) {
+      const int j = ch * 32 + u;                 // query index, row = key
+      a[u / 2] = pack_bf16(j >= row ? v[u] : 0.f, j + 1 >= row ? v[u + 1] : 0.f);
+    }
+    tmem_st8(tb + lane_off + C_ATH + ch * 16, a);
+    tmem_st8(tb + lane_off + C_ATH + ch * 16 + 8, a + 8);
+  }
+  tmem_st_wait();
+  tc_fence_before();
+  ok = mbar_wait(&bars[2], 0, p.status, ST_TIMEOUT);
+  if (__syncthreads_or(!ok)) goto done;
+  // 4a. GQ = dO S'^T + dA^ Kt ;  GK = dA^T^ Qt
+  if (tid == 0) {
+    tc_fence_after();
+    for (int s = 0; s < 8; ++s) mma_ss(tb + C_GQ, desc_k(sbase + R_O, s), desc_k(sbase + R_W, s), id_kk, s > 0);
+    for (int s = 0; s < 8; ++s) mma_ts(tb + C_GQ, tb + C_DAH + s * 8, desc_mn(sbase + R_XK, s), id_mn, 1);
+    for (int s = 0; s < 8; ++s) mma_ts(tb + C_GK, tb + C_DATH + s * 8, desc_mn(sbase + R_XQ, s), id_mn, s > 0);
+    mma_commit(&bars[4]);
+  }
+  ok = mbar_wait(&bars[4], 0, p.status, ST_TIMEOUT);
+  if (__syncthreads_or(!ok)) goto done;
+  tc_fence_after();
+  if (tid == 0) {   // S' consumed: dS goes into its place
+    mbar_expect_tx(&bars[5], TILE);
+    tma_load_3d(sm + R_W, &p.mds, &bars[5], 0, 0, snap_idx);
+    tma_load_3d(sm + R_W + REG, &p.mds, &bars[5], 64, 0, snap_idx);
+  }
+  ok = mbar_wait(&bars[5], 0, p.status, ST_TIMEOUT);
+  if (__syncthreads_or(!ok)) goto done;
+  // 4b. GK += V dS^T ;  DV = A^T^ dO + Kt dS
+  if (tid == 0) {
+    tc_fence_after();
+    for (int s = 0; s < 8; ++s) mma_ss(tb + C_GK, desc_k(sbase + R_V, s), desc_k(sbase + R_W, s), id_kk, 1);
+    for (int s = 0; s < 8; ++s) mma_ts(tb + C_DV, tb + C_ATH + s * 8, desc_mn(sbase + R_O, s), id_mn, s > 0);
+    for (int s = 0; s < 8; ++s) mma_ss(tb + C_DV, desc_k(sbase + R_XK, s), desc_mn(sbase + R_W, s), id_mn, 1);
+    mma_commit(&bars[6]);
+  }
+  ok = mbar_wait(&bars[6], 0, p.status, ST_TIMEOUT);
+  if (__syncthreads_or(!ok)) goto done;
+  tc_fence_after();
+  // 5. rows: dphi_q = E GQ, dphi_k = GK / E, dB = Qt GQ - Kt GK (E in fp32 again), dv
+  {
+    const size_t off = ((size_t)bh * p.L + (valid ? tq : 0)) * D;
+    for (int c16 = 0; c16 < 8; ++c16) {
+      float E[16], tot[16], gq[16], gk[16];
+      row_decay16(sm + R_G, row, c16, valid, p.inv_tau, s_wtot, E, tot);
+      tmem_ld16(tb + lane_off + C_GQ + c16 * 16, gq);
+      tmem_ld16(tb + lane_off + C_GK + c16 * 16, gk);
+      float q16[16], k16[16], oq[16], ok16[16], ob[16];
+      unpack8(*chunk_ptr(sm, R_XQ, row, 2 * c16), q16);
+      unpack8(*chunk_ptr(sm, R_XQ, row, 2 * c16 + 1), q16 + 8);
+      unpack8(*chunk_ptr(sm, R_XK, row, 2 * c16), k16);
+      unpack8(*chunk_ptr(sm, R_XK, row, 2 * c16 + 1), k16 + 8);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        oq[u] = E[u] * gq[u];
+        ok16[u] = gk[u] * __fdividef(1.f, E[u]);
+        ob[u] = q16[u] * gq[u] - k16[u] * gk[u];
+      }
+      if (valid) {
+#pragma unroll
+        for (int u = 0; u < 16; u += 4) {
+          *reinterpret_cast<float4 *>(p.dphq + off + c16 * 16 + u) = make_float4(oq[u], oq[u + 1], oq[u + 2], oq[u + 3]);
+          *reinterpret_cast<float4 *>(p.dphk + off + c16 * 16 + u) = make_float4(ok16[u], ok16[u + 1], ok16[u + 2], ok16[u + 3]);
+          *reinterpret_cast<float4 *>(p.dB + off + c16 * 16 + u) = make_float4(ob[u], ob[u + 1], ob[u + 2], ob[u + 3]);
+        }
+      }
+    }
+    for (int ch = 0; ch < 4; ++ch) {
+      float dv[32];
+      tmem_ld32(tb + lane_off + C_DV + ch * 32, dv);
+      if (valid)
+#pragma unroll
+        for (int u = 0; u < 32; u += 4)
+          *reinterpret_cast<float4 *>(p.dv + off + ch * 32 + u) = make_float4(dv[u], dv[u + 1], dv[u + 2], dv[u + 3]);
+    }
+  }
+done:
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(s_tmem, 512);
+}
+
+// ------------------------------------------------------- gate gradient ----
+// dg_t = (sum_{s >= t} dB_s) * sigmoid(-g_t) / tau, one thread per dimension
+__global__ void __launch_bounds__(128) gate_grad_kernel(const float *dB, const __nv_bfloat16 *g, float *dg, int L,
+                                                       float inv_tau) {
+  const int bh = blockIdx.x, i = threadIdx.x;
+  const size_t base = (size_t)bh * L * D + i;
+  float carry = 0.f;
+  int t = L - 1;
+  for (; t >= 7; t -= 8) {
+    float b[8], gv[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      b[u] = dB[base + (size_t)(t - u) * D];
+      gv[u] = __bfloat162float(g[base + (size_t)(t - u) * D]);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      carry += b[u];
+      dg[base + (size_t)(t - u) * D] = carry * dlogsigmoid(gv[u]) * inv_tau;
+    }
+  }
+  for (; t >= 0; --t) {
+    carry += dB[base + (size_t)t * D];
+    dg[base + (size_t)t * D] = carry * dlogsigmoid(__bfloat162float(g[base + (size_t)t * D])) * inv_tau;
+  }
+}
+
+constexpr size_t DS_SMEM = 3 * TILE + TILE / 2 + 1024;
+constexpr size_t TILE_SMEM = 6 * TILE + 1024;
+
+}  // namespace
+
+size_t tc_gla_bwd_snapshot_bytes(int BH, int L) {
+  return (size_t)BH * ((L + T - 1) / T) * D * D * sizeof(__nv_bfloat16);
+}
+
+cudaError_t launch_tc_gla_bwd(const TcGlaBwdArgs &a, int stage, cudaStream_t s) {
+  const int ntiles = (a.L + T - 1) / T;
+  const uint64_t rows = (uint64_t)a.L;
+  if (stage == 0) {   // reverse dS pass
+    DsParams p;
+    memset(&p, 0, sizeof(p));
+    if (!make_map_bf16_3d(&p.mq, a.q, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mg, a.g, D, rows, a.BH, T) ||
+        !make_map_bf16_3d(&p.mo, a.dout, D, rows, a.BH, T))
+      return cudaErrorInvalidValue;
+    p.wq = a.wq;
+    p.snap = static_cast<__nv_bfloat16 *>(a.snap_ds);
+    p.dstate_in = a.dstate_in;
+    p.status = a.status;
+    p.H = a.H;
+    p.L = a.L;
+    p.inv_tau = a.inv_tau;
+    cudaError_t e = cudaFuncSetAttribute(tc_gla_dstates_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DS_SMEM);
+    if (e != cudaSuccess) return e;
+    tc_gla_dstates_kernel<<<a.BH, 128, DS_SMEM, s>>>(p);
+    return cudaGetLastError();
+  }
+  if (stage == 1) {   // per-tile gradients
+    TileParams p;
+    memset(&p, 0, sizeof(p));
+    if (!make_map_bf16_3d(&p.mq, a.q, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mk, a.k, D, rows, a.BH, T) ||
+        !make_map_bf16_3d(&p.mv, a.v, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mo, a.dout, D, rows, a.BH, T) ||
+        !make_map_bf16_3d(&p.mg, a.g, D, rows, a.BH, T) ||
+        !make_map_bf16_3d(&p.msp, a.snap_s, D, D, (uint64_t)a.BH * ntiles, T) ||
+        !make_map_bf16_3d(&p.mds, a.snap_ds, D, D, (uint64_t)a.BH * ntiles, T))
+      return cudaErrorInvalidValue;
+    p.wq = a.wq;
+    p.wk = a.wk;
+    p.dphq = a.dphq;
+    p.dphk = a.dphk;
+    p.dB = a.dB;
+    p.dv = a.dv;
+    p.status = a.status;
+    p.H = a.H;
+    p.L = a.L;
+    p.ntiles = ntiles;
+    p.inv_tau = a.inv_tau;
+    cudaError_t e = cudaFuncSetAttribute(tc_gla_bwd_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TILE_SMEM);
+    if (e != cudaSuccess) return e;
+    tc_gla_bwd_tile_kernel<<<dim3(ntiles, a.BH), 128, TILE_SMEM, s>>>(p);
+    return cudaGetLastError();
+  }
+  gate_grad_kernel<<<a.BH, 128, 0, s>>>(a.dB, static_cast<const __nv_bfloat16 *>(a.g), a.dg, a.L, a.inv_tau);
+  return cudaGetLastError();
+}
+
+}  // namespace lz

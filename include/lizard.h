@@ -78,8 +78,9 @@ enum { LIZARD_BRANCH_BOTH = 0, LIZARD_BRANCH_GLA_ONLY = 1, LIZARD_BRANCH_SWA_ONL
 enum {
   LIZARD_IMPL_AUTO = 0,  /* tensor-core path where it applies, else portable */
   LIZARD_IMPL_SIMT = 1,  /* portable fp32 CUDA-core kernels (exact fp32 math) */
-  LIZARD_IMPL_TC = 2     /* tcgen05/TMEM tensor-core kernels: forward only,
-                            bf16, dk = dv = 128, window <= 128, M <= 16 */
+  LIZARD_IMPL_TC = 2     /* tcgen05/TMEM tensor-core kernels: bf16, dk = dv =
+                            128, window <= 128, M <= 16 (the GLA part of the
+                            backward needs only bf16 and d = 128) */
 };
 
 /*
