@@ -261,9 +261,12 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan) {
                        w ? at<float>(ws, lay.dq_swa) : nullptr, w ? at<float>(ws, lay.dk_swa) : nullptr,
                        w ? at<float>(ws, lay.dv_swa) : nullptr,
                        b->dq, b->dk, b->dv, b->dg, b->dfmap_wq, b->dfmap_wk, a->H, a->L, inv_tau,
-                       gla_tc ? 0 : 1};
+                       gla_tc ? 0 : 1, static_cast<uint32_t *>(ws)};
   if (gla_tc) fa.da = nullptr;   // the gate gradient comes from gate_grad_kernel
-  plan.add("finish_bwd", [=] { return lz::launch_finish_bwd(fa, BH, D, bf16, s); });
+  if (gla_tc && a->fmap_wq && a->fmap_wk)
+    plan.add("tc_finish_kernel", [=] { return lz::launch_tc_finish(fa, BH, s); });
+  else
+    plan.add("finish_bwd", [=] { return lz::launch_finish_bwd(fa, BH, D, bf16, s); });
   if (gla_tc) {
     lz::TcGlaBwdArgs t{a->q, a->k, a->v, a->g, b->dout, a->fmap_wq, a->fmap_wk, nullptr, nullptr, nullptr,
                        nullptr, at<float>(ws, lay.da), nullptr, b->dg, nullptr, static_cast<uint32_t *>(ws),

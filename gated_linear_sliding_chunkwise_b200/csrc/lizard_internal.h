@@ -90,6 +90,7 @@ struct FinishBwdArgs {
   int H, L;
   float inv_tau;
   int write_dg;                             // 0 when another kernel writes dg
+  uint32_t *status;                         // workspace status word (tensor-core finish)
 };
 
 struct TcFwdArgs {
@@ -149,6 +150,8 @@ size_t tc_gla_bwd_snapshot_bytes(int BH, int L);
 cudaError_t launch_tc_state_snapshots(const TcFwdArgs &a, void *snap, cudaStream_t s);
 // stage 0: reverse dS pass, 1: per-tile gradients, 2: gate-logit gradient
 cudaError_t launch_tc_gla_bwd(const TcGlaBwdArgs &a, int stage, cudaStream_t s);
+// tensor-core finish: bf16, d = 128, both feature maps present
+cudaError_t launch_tc_finish(const FinishBwdArgs &a, int BH, cudaStream_t s);
 cudaError_t launch_finish_bwd(const FinishBwdArgs &a, int BH, int D, bool bf16, cudaStream_t s);
 
 }  // namespace lz

@@ -1,0 +1,267 @@
+// Tensor-core (tcgen05) end of the backward, bf16, d = 128: the feature-map
+// backward and the sums of the two branches' gradients.
+//
+// phi(x) = [softmax(x W), softmax(-x W)] (the non-negative Hedgehog map of
+// the Chinese gist.science summary, section 2.3).  With p = softmax(z),
+// n = softmax(-z), z = x W and dphi = [dp, dn]:
+//   dz = p (dp - <dp, p>) - n (dn - <dn, n>)
+//   dx = dz W^T,   dW += x^T dz
+// One CTA per sequence walks its 128-token tiles; dW_q and dW_k accumulate
+// in TMEM across the tiles and are added to the output once per CTA.  dz is
+// formed in fp32 (the subtraction above cancels) and only then rounded to
+// bf16 as an MMA operand.
+#include "common.cuh"
+#include "lizard_internal.h"
+#include "tc_common.cuh"
+#include "tc_host.h"
+
+namespace lz {
+namespace {
+
+using namespace tc;
+
+constexpr int T = 128;
+constexpr int D = 128;
+constexpr int F = D / 2;
+constexpr uint32_t TILE = kTile;
+constexpr uint32_t REG = kReg;
+constexpr uint32_t ST_TIMEOUT = 1u;
+
+struct Params {
+  CUtensorMap mq, mk;
+  const float *wq, *wk;
+  const float *dphq, *dphk, *dv_gla;       // GLA parts (fp32), null when the branch is off
+  const float *dq_swa, *dk_swa, *dv_swa;   // anchor parts (fp32), null when the branch is off
+  __nv_bfloat16 *dq, *dk, *dv;
+  float *dwq, *dwk;
+  uint32_t *status;
+  int H, L;
+};
+
+__global__ void __launch_bounds__(128, 1) tc_finish_kernel(const __grid_constant__ Params p) {
+  extern __shared__ unsigned char smraw[];
+  unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
+  __shared__ uint64_t bar_tma, bar_z, bar_d;
+  __shared__ uint32_t s_tmem;
+  // X_q, X_k, W_q | W_k (64-column tiles), dZ_q | dZ_k (64-column tiles)
+  constexpr uint32_t R_XQ = 0, R_XK = TILE, R_WQ = 2 * TILE, R_WK = 2 * TILE + REG, R_ZQ = 3 * TILE,
+                     R_ZK = 3 * TILE + REG;
+  // TMEM: dWq [0,64) dWk [64,128) Zq [128,192) Zk [192,256) dXq [256,384) dXk [384,512)
+  constexpr uint32_t C_WQ = 0, C_WK = 64, C_ZQ = 128, C_ZK = 192, C_XQ = 256, C_XK = 384;
+  const int tid = threadIdx.x, warp = tid >> 5, row = tid;
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const int bh = blockIdx.x, h = bh % p.H;
+  const uint32_t sbase = smem_u32(sm);
+  const bool gla = p.dphq != nullptr;
+  if (warp == 0) { tmem_alloc(&s_tmem, 512); tmem_relinquish(); }
+  if (tid == 0) {
+    mbar_init(&bar_tma, 1);
+    mbar_init(&bar_z, 1);
+    mbar_init(&bar_d, 1);
+    fence_barrier_init();
+  }
+  // weights -> bf16 [dk row][feature] (MN-major for z = x W, K-major for dz W^T)
+#pragma unroll
+  for (int m = 0; m < 2; ++m) {
+    const float *W = m == 0 ? p.wq : p.wk;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      float f[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) f[u] = W[((size_t)h * D + row) * F + c * 8 + u];
+      *reinterpret_cast<uint4 *>(sm + (m == 0 ? R_WQ : R_WK) + sw128_offset(row, c * 8)) = pack8(f);
+    }
+  }
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = s_tmem;
+  const int ntiles = (p.L + T - 1) / T;
+  const uint32_t id_z = idesc_bf16(128, 64, 0, 1);     // X (K-major) x W (MN-major, N = 64)
+  const uint32_t id_dx = idesc_bf16(128, 128, 0, 0);   // dZ (K-major) x W^T (K-major, N = 128)
+  const uint32_t id_dw = idesc_bf16(128, 64, 1, 1);    // X^T (MN-major) x dZ (MN-major, N = 64)
+  auto loads = [&](int c) {
+    mbar_expect_tx(&bar_tma, 2 * TILE);
+    for (int r = 0; r < 2; ++r) {
+      tma_load_3d(sm + R_XQ + r * REG, &p.mq, &bar_tma, 64 * r, c * T, bh);
+      tma_load_3d(sm + R_XK + r * REG, &p.mk, &bar_tma, 64 * r, c * T, bh);
+    }
+  };
+  if (tid == 0 && ntiles > 0 && gla) loads(0);
+  bool fail = false;
+  for (int c = 0; c < ntiles; ++c) {
+    const uint32_t par = c & 1;
+    const int tq = c * T + row;
+    const bool valid = tq < p.L;
+    const size_t off = ((size_t)bh * p.L + (valid ? tq : 0)) * D;
+    if (gla) {
+      bool ok = mbar_wait(&bar_tma, par, p.status, ST_TIMEOUT);
+      if (__syncthreads_or(!ok)) { fail = true; break; }
+      if (tid == 0) {
+        tc_fence_after();
+        for (int s = 0; s < 8; ++s) mma_ss(tb + C_ZQ, desc_k(sbase + R_XQ, s), desc_mn(sbase + R_WQ, s), id_z, s > 0);
+        for (int s = 0; s < 8; ++s) mma_ss(tb + C_ZK, desc_k(sbase + R_XK, s), desc_mn(sbase + R_WK, s), id_z, s > 0);
+        mma_commit(&bar_z);
+      }
+      ok = mbar_wait(&bar_z, par, p.status, ST_TIMEOUT);
+      if (__syncthreads_or(!ok)) { fail = true; break; }
+      tc_fence_after();
+      // dz rows (fp32 math) -> bf16 dZ tiles
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        float pos[F], neg[F];
+        tmem_ld32(tb + lane_off + (m == 0 ? C_ZQ : C_ZK), pos);
+        tmem_ld32(tb + lane_off + (m == 0 ? C_ZQ : C_ZK) + 32, pos + 32);
+        const float *src = (m == 0 ? p.dphq : p.dphk) + off;
+        float mx = pos[0], mn = pos[0];
+#pragma unroll
+        for (int f = 1; f < F; ++f) { mx = fmaxf(mx, pos[f]); mn = fminf(mn, pos[f]); }
+        float sp = 0.f, sn = 0.f;
+#pragma unroll
+        for (int f = 0; f < F; ++f) {
+          neg[f] = __expf(mn - pos[f]);
+          pos[f] = __expf(pos[f] - mx);
+          sp += pos[f];
+          sn += neg[f];
+        }
+        const float ip = 1.f / sp, in_ = 1.f / sn;
+        // pass 1: <dp, p> and <dn, n>
+        float dotp = 0.f, dotn = 0.f;
+#pragma unroll
+        for (int f = 0; f < F; ++f) { pos[f] *= ip; neg[f] *= in_; }
+        if (valid) {
+#pragma unroll
+          for (int u = 0; u < F; u += 4) {
+            const float4 a = *reinterpret_cast<const float4 *>(src + u);
+            const float4 b = *reinterpret_cast<const float4 *>(src + F + u);
+            dotp += a.x * pos[u] + a.y * pos[u + 1] + a.z * pos[u + 2] + a.w * pos[u + 3];
+            dotn += b.x * neg[u] + b.y * neg[u + 1] + b.z * neg[u + 2] + b.w * neg[u + 3];
+          }
+        }
+        // pass 2: dz = p (dp - <dp,p>) - n (dn - <dn,n>), 8 features at a time
+        const uint32_t reg = m == 0 ? R_ZQ : R_ZK;
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) {
+          float dz[8];
+          if (valid) {
+            const float4 a0 = *reinterpret_cast<const float4 *>(src + c8 * 8);
+            const float4 a1 = *reinterpret_cast<const float4 *>(src + c8 * 8 + 4);
+            const float4 b0 = *reinterpret_cast<const float4 *>(src + F + c8 * 8);
+            const float4 b1 = *reinterpret_cast<const float4 *>(src + F + c8 * 8 + 4);
+            const float dpv[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float dnv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int f = c8 * 8 + u;
+              dz[u] = pos[f] * (dpv[u] - dotp) - neg[f] * (dnv[u] - dotn);
+            }
+          } else {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) dz[u] = 0.f;
+          }
+          *reinterpret_cast<uint4 *>(sm + reg + sw128_offset(row, c8 * 8)) = pack8(dz);
+        }
+      }
+      fence_proxy_async();
+      tc_fence_before();
+      __syncthreads();
+      if (tid == 0) {
+        tc_fence_after();
+        for (int s = 0; s < 4; ++s) mma_ss(tb + C_XQ, desc_k(sbase + R_ZQ, s), desc_k(sbase + R_WQ, s), id_dx, s > 0);
+        for (int s = 0; s < 4; ++s) mma_ss(tb + C_XK, desc_k(sbase + R_ZK, s), desc_k(sbase + R_WK, s), id_dx, s > 0);
+        for (int s = 0; s < 8; ++s) mma_ss(tb + C_WQ, desc_mn(sbase + R_XQ, s), desc_mn(sbase + R_ZQ, s), id_dw, c > 0 || s > 0);
+        for (int s = 0; s < 8; ++s) mma_ss(tb + C_WK, desc_mn(sbase + R_XK, s), desc_mn(sbase + R_ZK, s), id_dw, c > 0 || s > 0);
+        mma_commit(&bar_d);
+      }
+      ok = mbar_wait(&bar_d, par, p.status, ST_TIMEOUT);
+      if (__syncthreads_or(!ok)) { fail = true; break; }
+      tc_fence_after();
+      if (tid == 0 && c + 1 < ntiles) loads(c + 1);   // X tiles consumed by the dW products
+    }
+    // dq, dk = GLA (dz W^T) + anchor parts; dv = both parts
+#pragma unroll
+    for (int m = 0; m < 3; ++m) {
+      const float *swa = m == 0 ? p.dq_swa : (m == 1 ? p.dk_swa : p.dv_swa);
+      __nv_bfloat16 *dst = m == 0 ? p.dq : (m == 1 ? p.dk : p.dv);
+      for (int ch = 0; ch < 4; ++ch) {
+        float v[32];
+        if (m < 2 && gla) {
+          tmem_ld32(tb + lane_off + (m == 0 ? C_XQ : C_XK) + ch * 32, v);
+        } else {
+#pragma unroll
+          for (int u = 0; u < 32; ++u) v[u] = 0.f;
+        }
+        if (!valid) continue;
+        if (m == 2 && p.dv_gla)
+#pragma unroll
+          for (int u = 0; u < 32; u += 4) {
+            const float4 a = *reinterpret_cast<const float4 *>(p.dv_gla + off + ch * 32 + u);
+            v[u] += a.x; v[u + 1] += a.y; v[u + 2] += a.z; v[u + 3] += a.w;
+          }
+        if (swa)
+#pragma unroll
+          for (int u = 0; u < 32; u += 4) {
+            const float4 a = *reinterpret_cast<const float4 *>(swa + off + ch * 32 + u);
+            v[u] += a.x; v[u + 1] += a.y; v[u + 2] += a.z; v[u + 3] += a.w;
+          }
+#pragma unroll
+        for (int u = 0; u < 32; u += 8) *reinterpret_cast<uint4 *>(dst + off + ch * 32 + u) = pack8(v + u);
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
+  if (gla && !fail) {
+    tc_fence_after();
+    // dW rows: lane = dk index, 64 feature columns per map
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      float *dW = m == 0 ? p.dwq : p.dwk;
+      if (!dW) continue;
+      float v[32];
+      for (int ch = 0; ch < 2; ++ch) {
+        tmem_ld32(tb + lane_off + (m == 0 ? C_WQ : C_WK) + ch * 32, v);
+#pragma unroll
+        for (int u = 0; u < 32; ++u) atomicAdd(dW + ((size_t)h * D + row) * F + ch * 32 + u, v[u]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(s_tmem, 512);
+}
+
+constexpr size_t SMEM_BYTES = 4 * TILE + 1024;
+
+}  // namespace
+
+cudaError_t launch_tc_finish(const FinishBwdArgs &a, int BH, cudaStream_t s) {
+  Params p;
+  memset(&p, 0, sizeof(p));
+  const uint64_t rows = (uint64_t)a.L;
+  if (!make_map_bf16_3d(&p.mq, a.q, D, rows, BH, T) || !make_map_bf16_3d(&p.mk, a.k, D, rows, BH, T))
+    return cudaErrorInvalidValue;
+  p.wq = a.wq;
+  p.wk = a.wk;
+  p.dphq = a.dphq;
+  p.dphk = a.dphk;
+  p.dv_gla = a.dv_gla;
+  p.dq_swa = a.dq_swa;
+  p.dk_swa = a.dk_swa;
+  p.dv_swa = a.dv_swa;
+  p.dq = static_cast<__nv_bfloat16 *>(a.dq);
+  p.dk = static_cast<__nv_bfloat16 *>(a.dk);
+  p.dv = static_cast<__nv_bfloat16 *>(a.dv);
+  p.dwq = a.dwq;
+  p.dwk = a.dwk;
+  p.status = a.status;
+  p.H = a.H;
+  p.L = a.L;
+  cudaError_t e = cudaFuncSetAttribute(tc_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  tc_finish_kernel<<<BH, 128, SMEM_BYTES, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace lz

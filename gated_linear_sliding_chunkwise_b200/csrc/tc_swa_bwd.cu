@@ -412,27 +412,35 @@ done:
 
 // ------------------------------------------------------- meta gradients ---
 // dmeta_k[h][m] += scale sum_t dSm[t][m] q_t ; dmeta_v[h][m] += alpha sum_t pm[t][m] dout_t
-constexpr int kMetaTok = 1024;
+constexpr int kMetaTok = 256;
 __global__ void __launch_bounds__(128) meta_grad_kernel(const __nv_bfloat16 *q, const __nv_bfloat16 *dout,
                                                          const float *dsm, const float *pm, const float *alpha,
                                                          float *dmk, float *dmv, int B, int H, int L, int M,
                                                          float scale) {
   const int h = blockIdx.y, i = threadIdx.x;
   const int n0 = blockIdx.x * kMetaTok;
-  const int ntok = B * L;
+  const int n1 = min(B * L, n0 + kMetaTok);
   float ak[MAXM], av[MAXM];
 #pragma unroll
   for (int m = 0; m < MAXM; ++m) { ak[m] = 0.f; av[m] = 0.f; }
-  for (int n = n0; n < min(ntok, n0 + kMetaTok); ++n) {
-    const int b = n / L, t = n % L;
-    const size_t tok = ((size_t)b * H + h) * L + t;
-    const float qi = __bfloat162float(q[tok * D + i]);
-    const float oi = __bfloat162float(dout[tok * D + i]);
+  for (int nb = n0; nb < n1; nb += 8) {
+    float qi[8], oi[8];
+    size_t tok[8];
 #pragma unroll
-    for (int m = 0; m < MAXM; ++m) {
-      if (m < M) {
-        ak[m] = fmaf(dsm[tok * MAXM + m], qi, ak[m]);
-        av[m] = fmaf(pm[tok * MAXM + m], oi, av[m]);
+    for (int u = 0; u < 8; ++u) {       // all loads of 8 tokens in flight together
+      const int n = min(nb + u, n1 - 1);
+      tok[u] = ((size_t)(n / L) * H + h) * L + n % L;
+      qi[u] = nb + u < n1 ? __bfloat162float(q[tok[u] * D + i]) : 0.f;
+      oi[u] = nb + u < n1 ? __bfloat162float(dout[tok[u] * D + i]) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+#pragma unroll
+      for (int m = 0; m < MAXM; ++m) {
+        if (m < M) {
+          ak[m] = fmaf(dsm[tok[u] * MAXM + m], qi[u], ak[m]);
+          av[m] = fmaf(pm[tok[u] * MAXM + m], oi[u], av[m]);
+        }
       }
     }
   }
