@@ -371,6 +371,35 @@ def run_forward(args, lz, dev, rank, world, peaks, name, steps):
     return out
 
 
+def run_backward(args, lz, dev, rank, world, peaks, name, steps):
+    """Time lizard_attn_bwd alone on one workload (inputs resident)."""
+    from gated_linear_sliding_chunkwise_b200.synth import WORKLOADS, make_inputs
+
+    w = WORKLOADS[name]
+    impl = {"auto": lz.IMPL_AUTO, "simt": lz.IMPL_SIMT, "tc": lz.IMPL_TC}[args.kernels]
+    inp = make_inputs(w, seed=w.seed + rank, with_dout=True)
+    x = {k: v.to(dev).contiguous() for k, v in inp.items()}
+    kw = dict(window=w.window, chunk=w.chunk, gate_temp=w.gate_temp, fmap_wq=x["fmap_wq"],
+              fmap_wk=x["fmap_wk"], meta_k=x["meta_k"], meta_v=x["meta_v"], alpha=x["alpha"],
+              impl=impl)
+    names = lz.attn_bwd(x["q"], x["k"], x["v"], x["g"], x["dout"], plan_only=True, **kw)
+    ws = lz.attn_bwd(x["q"], x["k"], x["v"], x["g"], x["dout"], **kw)["workspace"]
+    for _ in range(max(args.warmup, 1)):
+        lz.attn_bwd(x["q"], x["k"], x["v"], x["g"], x["dout"], workspace=ws, **kw)
+    evs = [lz.make_events(len(names) + 1) for _ in range(steps)]
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for i in range(steps):
+        lz.attn_bwd(x["q"], x["k"], x["v"], x["g"], x["dout"], workspace=ws, events=evs[i], **kw)
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / steps
+    per = {n: statistics.mean(ev[j].elapsed_time(ev[j + 1]) for ev in evs) for j, n in enumerate(names)}
+    return {"workload": f"{name} backward: B={w.B} H={w.H} L={w.L} d={w.d}", "ms": ms,
+            "kernel_ms": {n: round(t, 4) for n, t in per.items()}, "launches": len(names)}
+
+
 def run_decode(args, lz, dev, rank, world, peaks):
     from gated_linear_sliding_chunkwise_b200.synth import WORKLOADS, make_inputs
 
@@ -492,19 +521,20 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-fwd-long", action="store_true")
-    ap.add_argument("--only", choices=["train", "fwd"], default="train",
-                    help="fwd: time lizard_attn_fwd alone on --workload (profiling aid)")
+    ap.add_argument("--only", choices=["train", "fwd", "bwd"], default="train",
+                    help="fwd / bwd: time one entry point alone on --workload (profiling aid)")
     ap.add_argument("--workload", default="llama8b_layer_fwd")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         print("note: --warmup below 3 is not a valid measurement", file=sys.stderr)
     rank, world, local = dist_env()
-    if args.only == "fwd":
-        # forward-only timing of one workload (used for kernel profiles)
+    if args.only in ("fwd", "bwd"):
+        # one entry point alone on one workload (used for kernel profiles)
         from gated_linear_sliding_chunkwise_b200 import lizard as lz
         dev = torch.device("cuda", local)
         torch.cuda.set_device(dev)
-        print(json.dumps(run_forward(args, lz, dev, rank, 1, load_peaks(), args.workload, args.steps)))
+        fn = run_forward if args.only == "fwd" else run_backward
+        print(json.dumps(fn(args, lz, dev, rank, 1, load_peaks(), args.workload, args.steps)))
         return
     if world > 1:
         import torch.distributed as dist

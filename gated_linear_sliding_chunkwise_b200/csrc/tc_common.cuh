@@ -44,6 +44,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32
   if (err) atomicOr(err, code);
   return false;
 }
+// Named CTA barriers (id 0 is __syncthreads): `bar_sync` waits until
+// `count` threads have arrived at barrier `id`; `bar_arrive` only counts.
+__device__ __forceinline__ void bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ void bar_arrive(int id, int count) {
+  asm volatile("bar.arrive %0, %1;\n" ::"r"(id), "r"(count) : "memory");
+}
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
 }
@@ -228,9 +236,11 @@ __device__ __forceinline__ float log_decay_fast(float g, float inv_tau) {
 // from the bf16 gate logits of a 128 x 128 tile (a_s = logsigmoid(g)/tau,
 // zero for rows at or beyond L).  Suffix sums: a shuffle scan within each
 // warp, then the later warps' totals from shared memory `wtot` [4][16].
-// All 128 threads must call it (it synchronises the block twice).
+// All 128 threads of the group must call it: it synchronises them twice,
+// through __syncthreads (bar_id 0, a 128-thread CTA) or through named
+// barrier bar_id over 128 threads (one warpgroup of a larger CTA).
 __device__ __forceinline__ void row_decay16(unsigned char *gtile, int row, int c16, bool valid, float inv_tau,
-                                            float (*wtot)[16], float *E, float *tot) {
+                                            float (*wtot)[16], float *E, float *tot, int bar_id = 0) {
   const int lane = row & 31, warp = row >> 5;
   float na[16], x[16];
   unpack8(*chunk_ptr(gtile, 0, row, 2 * c16), na);
@@ -251,7 +261,7 @@ __device__ __forceinline__ void row_decay16(unsigned char *gtile, int row, int c
   if (lane == 0)
 #pragma unroll
     for (int u = 0; u < 16; ++u) wtot[warp][u] = x[u];
-  __syncthreads();
+  if (bar_id) bar_sync(bar_id, 128); else __syncthreads();
 #pragma unroll
   for (int u = 0; u < 16; ++u) {
     float later = 0.f, all = 0.f;
@@ -264,7 +274,7 @@ __device__ __forceinline__ void row_decay16(unsigned char *gtile, int row, int c
     E[u] = __expf(x[u] - na[u] + later);
     tot[u] = all;
   }
-  __syncthreads();
+  if (bar_id) bar_sync(bar_id, 128); else __syncthreads();
 }
 
 }  // namespace tc

@@ -57,6 +57,7 @@ constexpr int F = D / 2;           // feature-map width per half
 constexpr uint32_t REG = kReg;     // one 64-column swizzled region of a 128-row tile
 constexpr uint32_t TILE = kTile;   // a 128 x 128 bf16 tile
 constexpr int MAXM = 16;
+constexpr int NTHREADS = 256;     // two warpgroups
 
 // shared-memory regions (offsets from the 1024-aligned base)
 constexpr uint32_t R_XQ = 0;            // X_q, then S' (bf16, MN-major)
@@ -107,38 +108,123 @@ __device__ __forceinline__ void issue_tile_loads(const Params &p, unsigned char 
   }
 }
 
-// phi(x) = [softmax(z), softmax(-z)] of the 64 projections z of this
-// thread's row: z is overwritten with the first half, neg gets the second.
-__device__ __forceinline__ void feature_map_row(float *z, float *neg) {
-  float mx = z[0], mn = z[0];
+// One half of the feature map of this thread's row, from the 64
+// projections z in TMEM: half 0 is softmax(z), half 1 is softmax(-z).  ph
+// gets the unnormalised terms exp(+-z_f - max); the result is 1 / their sum.
+__device__ __forceinline__ float feature_half(uint32_t taddr, int half, float *ph) {
+  tmem_ld32(taddr, ph);
+  tmem_ld32(taddr + 32, ph + 32);
+  const float sg = half ? -1.f : 1.f;
+  float m[4];
 #pragma unroll
-  for (int f = 1; f < F; ++f) { mx = fmaxf(mx, z[f]); mn = fminf(mn, z[f]); }
-  float sp = 0.f, sn = 0.f;
+  for (int k = 0; k < 4; ++k) m[k] = sg * ph[k];
+#pragma unroll
+  for (int f = 4; f < F; ++f) m[f & 3] = fmaxf(m[f & 3], sg * ph[f]);
+  const float mx = fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+  float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int f = 0; f < F; ++f) {
-    neg[f] = __expf(mn - z[f]);
-    z[f] = __expf(z[f] - mx);
-    sp += z[f];
-    sn += neg[f];
+    ph[f] = __expf(fmaf(sg, ph[f], -mx));
+    s[f & 3] += ph[f];
   }
-  const float ip = 1.f / sp, in_ = 1.f / sn;
-#pragma unroll
-  for (int f = 0; f < F; ++f) { z[f] *= ip; neg[f] *= in_; }
+  return 1.f / ((s[0] + s[1]) + (s[2] + s[3]));
 }
 
-__global__ void __launch_bounds__(128, 1) tc_fwd_kernel(const __grid_constant__ Params p) {
+// Gates, thread = key dimension i: in-tile suffix sums of the log-decay,
+// E_t = exp(sum_{s>t} -a_s) = exp(b_t - r) written as bf16 over the gate
+// logits, exp(r) (the tile's decay) into s_dec[i].  16 tokens per step; the
+// next step's logits are read before this step's factors are written.
+// Returns the largest exponent of E in this dimension (its value at t = 0).
+__device__ __forceinline__ float gates_by_dim(unsigned char *sm, int i, int t0, int L, float inv_tau,
+                                              float *s_dec) {
+  unsigned char *gcol = sm + R_G + (i >> 6) * REG;
+  const int ci = i & 63;
+  float acc = 0.f, spread = 0.f, gn[16];
+#pragma unroll
+  for (int u = 0; u < 16; ++u)
+    gn[u] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(gcol + sw128_offset(T - 16 + u, ci)));
+#pragma unroll 1
+  for (int tb = T - 16; tb >= 0; tb -= 16) {
+    float a[16], pre[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) a[u] = (t0 + tb + u < L) ? log_decay_fast(gn[u], inv_tau) : 0.f;
+    if (tb > 0) {
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+        gn[u] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(gcol + sw128_offset(tb - 16 + u, ci)));
+    }
+#pragma unroll
+    for (int u = 15; u >= 0; --u) { pre[u] = acc; acc -= a[u]; }
+#pragma unroll
+    for (int u = 0; u < 16; ++u)
+      *reinterpret_cast<__nv_bfloat16 *>(gcol + sw128_offset(tb + u, ci)) = __float2bfloat16_rn(__expf(pre[u]));
+    spread = pre[0];
+  }
+  s_dec[i] = __expf(-acc);
+  return spread;
+}
+
+// Qt for dimensions 64 h .. 64 h + 63: phi_q E gscale, bf16 pairs into TMEM.
+__device__ __forceinline__ void qt_half(unsigned char *sm, uint32_t tl, int row, int h, float gscale) {
+  float ph[F];
+  const float s = feature_half(tl + C_ZQ, h, ph) * gscale;
+#pragma unroll
+  for (int c16 = 0; c16 < 4; ++c16) {     // 16 dims = 8 TMEM columns
+    float e16[16];
+    unpack8(*chunk_ptr(sm, R_G, row, 8 * h + 2 * c16), e16);
+    unpack8(*chunk_ptr(sm, R_G, row, 8 * h + 2 * c16 + 1), e16 + 8);
+    uint32_t r8[8];
+#pragma unroll
+    for (int u = 0; u < 16; u += 2)
+      r8[u / 2] = pack_bf16(ph[16 * c16 + u] * e16[u] * s, ph[16 * c16 + u + 1] * e16[u + 1] * s);
+    tmem_st8(tl + C_QT + 32 * h + 8 * c16, r8);
+  }
+}
+
+// Kt for dimensions 64 h .. 64 h + 63: phi_k / E, bf16 into shared memory
+// over X_k.  E comes as bf16 from the gate region (full pass) or as fp32
+// from TMEM (state pass).
+__device__ __forceinline__ void kt_half(unsigned char *sm, uint32_t tl, int row, int h, bool e_in_tmem) {
+  float ph[F];
+  const float s = feature_half(tl + C_ZK, h, ph);
+#pragma unroll
+  for (int c16 = 0; c16 < 4; ++c16) {
+    float e16[16], k16[16];
+    if (e_in_tmem) {
+      tmem_ld16(tl + C_L + 64 * h + 16 * c16, e16);
+    } else {
+      unpack8(*chunk_ptr(sm, R_G, row, 8 * h + 2 * c16), e16);
+      unpack8(*chunk_ptr(sm, R_G, row, 8 * h + 2 * c16 + 1), e16 + 8);
+    }
+#pragma unroll
+    for (int u = 0; u < 16; ++u) k16[u] = __fdividef(ph[16 * c16 + u] * s, e16[u]);
+    *chunk_ptr(sm, R_XK, row, 8 * h + 2 * c16) = pack8(k16);
+    *chunk_ptr(sm, R_XK, row, 8 * h + 2 * c16 + 1) = pack8(k16 + 8);
+  }
+}
+
+// Named barriers between the two warpgroups (id 0 is __syncthreads).
+constexpr int BAR_E = 1;       // gate factors E written (group 1 -> group 0)
+constexpr int BAR_G = 2;       // row scales of the anchor softmax written (group 0 -> group 1)
+constexpr int BAR_DECAY = 3;   // + group: the row-wise decay scan inside one group
+
+__global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_constant__ Params p) {
   extern __shared__ unsigned char smraw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
-  __shared__ float s_mk[MAXM][D], s_mv[MAXM][D];
+  __shared__ __align__(16) float s_mk[MAXM][D];
+  __shared__ __align__(16) float s_mv[MAXM][D];
+  __shared__ float s_ml[MAXM][T];     // meta logits, then their mixing weights, per row
   __shared__ float s_dec[D];
-  __shared__ float s_wtot[4][16];
+  __shared__ float s_gscale[T], s_oscale[T];
+  __shared__ float s_wtot[2][4][16];
   __shared__ uint64_t bar_tma, bar_vp, bar_m1, bar_m2, bar_m3;
   __shared__ uint32_t s_tmem;
   __shared__ int s_fail;
 
   const int tid = threadIdx.x, warp = tid >> 5;
-  const int row = tid;                                 // TMEM lane == tile row
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const int wg = tid >> 7;                             // warpgroup
+  const int row = tid & 127;                           // TMEM lane == tile row
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
   const int bh = blockIdx.x, h = bh % p.H, seg = blockIdx.y;
   const float alpha = p.alpha ? p.alpha[h] : 1.f;
   const bool full = p.mode == 0;
@@ -158,44 +244,44 @@ __global__ void __launch_bounds__(128, 1) tc_fwd_kernel(const __grid_constant__ 
     fence_barrier_init();
     s_fail = 0;
   }
-  // feature-map weights -> bf16, MN-major [dk row][feature]
+  // feature-map weights -> bf16, MN-major [dk row][feature]; group 0 W_q, group 1 W_k
   {
     const int i = row;
+    const float *W = wg == 0 ? p.wq : p.wk;
+    const uint32_t reg = wg == 0 ? R_WQ : R_WK;
 #pragma unroll
-    for (int m = 0; m < 2; ++m) {
-      const float *W = m == 0 ? p.wq : p.wk;
-      const uint32_t reg = m == 0 ? R_WQ : R_WK;
+    for (int c = 0; c < 8; ++c) {
+      float f[8];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        float f[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) f[u] = W ? W[((size_t)h * D + i) * F + c * 8 + u] : 0.f;
-        *reinterpret_cast<uint4 *>(sm + reg + sw128_offset(i, c * 8)) = pack8(f);
-      }
+      for (int u = 0; u < 8; ++u) f[u] = W ? W[((size_t)h * D + i) * F + c * 8 + u] : 0.f;
+      *reinterpret_cast<uint4 *>(sm + reg + sw128_offset(i, c * 8)) = pack8(f);
     }
   }
-  for (int e = tid; e < p.M * D; e += 128) {
-    s_mk[e / D][e % D] = p.meta_k[(size_t)h * p.M * D + e];
-    s_mv[e / D][e % D] = p.meta_v ? p.meta_v[(size_t)h * p.M * D + e] : 0.f;
+  for (int e = tid; e < MAXM * D; e += NTHREADS) {
+    const int m = e / D;
+    s_mk[m][e % D] = m < p.M ? p.meta_k[(size_t)h * p.M * D + e] : 0.f;
+    s_mv[m][e % D] = (m < p.M && p.meta_v) ? p.meta_v[(size_t)h * p.M * D + e] : 0.f;
   }
   fence_proxy_async();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = s_tmem;
+  const uint32_t tl = tb + lane_off;
 
-  // initial state -> TMEM columns [0, 128), lane = key dimension
+  // initial state -> TMEM columns [0, 128), lane = key dimension; each
+  // group writes one half of the columns
   {
     const float *src = nullptr;
     if (full && p.nseg > 1) src = p.seg_start + (((size_t)bh * p.nseg + seg) * D + row) * D;
     else if (full && p.state_in) src = p.state_in + ((size_t)bh * D + row) * D;
     else if (p.snap && p.state_in) src = p.state_in + ((size_t)bh * D + row) * D;
 #pragma unroll
-    for (int c = 0; c < D; c += 8) {
+    for (int c = 64 * wg; c < 64 * wg + 64; c += 8) {
       uint32_t r[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(src ? src[c + u] : 0.f);
-      tmem_st8(tb + lane_off + C_S + c, r);
+      tmem_st8(tl + C_S + c, r);
     }
     tmem_st_wait();
   }
@@ -204,7 +290,7 @@ __global__ void __launch_bounds__(128, 1) tc_fwd_kernel(const __grid_constant__ 
   const int cbeg = seg * p.tiles_per_seg;
   const int cend = min(ntiles_all, cbeg + p.tiles_per_seg);
   uint32_t *err = p.status;
-  float tot_decay = 0.f;                      // mode 1: summed log-decay of this dimension
+  float tot_decay = 0.f;                      // state pass: summed log-decay of the dimension this thread owns
   if (tid == 0 && cbeg < cend) issue_tile_loads(p, sm, &bar_tma, bh, cbeg * T, full);
   const uint32_t id_128 = idesc_bf16(128, 128, 0, 0);
   const uint32_t id_z = idesc_bf16(128, 64, 0, 1);
@@ -233,221 +319,155 @@ __global__ void __launch_bounds__(128, 1) tc_fwd_kernel(const __grid_constant__ 
       mma_commit(&bar_m1);
     }
 
-    // ---------------------------------------------- gates (thread = dim) ---
-    if (full) {
-      // 8 tokens per step: the logsigmoids and exps are independent, only
-      // the running suffix sum is a chain
-      const int i = row;
-      unsigned char *gcol = sm + R_G + (i >> 6) * REG;
-      float acc = 0.f, spread = 0.f;
-      for (int tb8 = T - 8; tb8 >= 0; tb8 -= 8) {
-        float a[8], pre[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int t = tb8 + u;
-          const __nv_bfloat16 g = *reinterpret_cast<const __nv_bfloat16 *>(gcol + sw128_offset(t, i & 63));
-          a[u] = (t0 + t < p.L) ? log_decay_fast(__bfloat162float(g), p.inv_tau) : 0.f;
-        }
-#pragma unroll
-        for (int u = 7; u >= 0; --u) { pre[u] = acc; acc -= a[u]; }
-#pragma unroll
-        for (int u = 0; u < 8; ++u)      // E_t = exp(b_t - r) = exp(sum_{s>t} -a_s)
-          *reinterpret_cast<__nv_bfloat16 *>(gcol + sw128_offset(tb8 + u, i & 63)) = __float2bfloat16_rn(__expf(pre[u]));
-        if (tb8 == 0) spread = pre[0];
-      }
-      s_dec[i] = __expf(-acc);                     // exp(r): the tile's total decay
-      tot_decay -= acc;
+    if (full && wg == 1) {
+      // ------------------------------- group 1: gates, then phi half 1 ---
+      const float spread = gates_by_dim(sm, row, t0, p.L, p.inv_tau, s_dec);
       if (spread > kMaxSpread && gla) atomicOr(err, ST_RANGE);
-    }
-
-    ok = mbar_wait(&bar_m1, par, err, ST_TIMEOUT);
-    if (__syncthreads_or(!ok)) { s_fail = 1; break; }
-    tc_fence_after();
-
-    // ------------------------------------------- rows: anchor softmax ---
-    float lsum = 1.f, mx = 0.f;           // row normaliser and max (scaled logits)
-    float em[MAXM];                       // exp(meta logit - max)
+      bar_arrive(BAR_E, NTHREADS);
+      ok &= mbar_wait(&bar_m1, par, err, ST_TIMEOUT);
+      tc_fence_after();
+      kt_half(sm, tl, row, 1, false);
+      bar_sync(BAR_G, NTHREADS);
+      qt_half(sm, tl, row, 1, s_gscale[row]);
+    } else if (full) {
+      // ---------------------- group 0: anchor softmax, then phi half 0 ---
+      ok &= mbar_wait(&bar_m1, par, err, ST_TIMEOUT);
+      tc_fence_after();
+      float lsum = 1.f, mx = 0.f;                 // row normaliser and max (scaled logits)
+      if (swa) {
+        // meta logits q . mk_m (scaled) into s_ml, four meta tokens per pass
+        for (int m0 = 0; m0 < p.M; m0 += 4) {
+          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+          for (int ch = 0; ch < 16; ++ch) {
+            float q8[8];
+            unpack8(*chunk_ptr(sm, R_XQ, row, ch), q8);
 #pragma unroll
-    for (int m = 0; m < MAXM; ++m) em[m] = 0.f;
-    if (swa) {
-      float ml[MAXM];
-      mx = kNegBig;
-#pragma unroll
-      for (int m = 0; m < MAXM; ++m) ml[m] = 0.f;
-      for (int ch = 0; ch < 16; ++ch) {
-        float q8[8];
-        unpack8(*chunk_ptr(sm, R_XQ, row, ch), q8);
-#pragma unroll
-        for (int m = 0; m < MAXM; ++m) {
-          if (m < p.M) {
-#pragma unroll
-            for (int u = 0; u < 8; ++u) ml[m] = fmaf(q8[u], s_mk[m][ch * 8 + u], ml[m]);
-          }
-        }
-      }
-#pragma unroll
-      for (int m = 0; m < MAXM; ++m) {
-        if (m < p.M) {
-          ml[m] *= p.scale;
-          mx = fmaxf(mx, ml[m]);
-        }
-      }
-      const int jlo = max(tq - p.window + 1, 0);     // valid keys j in [jlo, tq]
-      for (int ch = 0; ch < 8; ++ch) {
-        float v[32];
-        tmem_ld32(tb + lane_off + C_L + ch * 32, v);
-#pragma unroll
-        for (int u = 0; u < 32; ++u) {
-          const int j = t0 - T + ch * 32 + u;
-          if (j >= jlo && j <= tq) mx = fmaxf(mx, v[u] * p.scale);
-        }
-      }
-      lsum = 0.f;
-      for (int ch = 0; ch < 8; ++ch) {
-        float v[32];
-        tmem_ld32(tb + lane_off + C_L + ch * 32, v);
-        uint32_t pk[16];
-        float part = 0.f;
-#pragma unroll
-        for (int u = 0; u < 32; u += 2) {
-          const int j = t0 - T + ch * 32 + u;
-          const float e0 = (j >= jlo && j <= tq) ? __expf(v[u] * p.scale - mx) : 0.f;
-          const float e1 = (j + 1 >= jlo && j + 1 <= tq) ? __expf(v[u + 1] * p.scale - mx) : 0.f;
-          part += e0 + e1;
-          pk[u / 2] = alpha != 0.f ? pack_bf16(e0, e1) : 0u;
-        }
-        lsum += part;
-        tmem_st8(tb + lane_off + C_P + ch * 16, pk);
-        tmem_st8(tb + lane_off + C_P + ch * 16 + 8, pk + 8);
-      }
-#pragma unroll
-      for (int m = 0; m < MAXM; ++m) {
-        if (m < p.M) {
-          em[m] = __expf(ml[m] - mx);
-          lsum += em[m];
-        }
-      }
-      if (!qvalid) lsum = 1.f;
-    }
-    // GLA operands carry l/alpha so that one accumulator holds both terms
-    const bool mixed = swa && alpha != 0.f;
-    const float gscale = mixed ? lsum / alpha : 1.f;
-    const float oscale = mixed ? alpha / lsum : 1.f;
-    const float mscale = mixed ? alpha / lsum : 0.f;   // meta-value weight per em
-
-    // -------------------------------------------- rows: feature maps ---
-    {
-      float z[F], neg[F];
-      // phi_q -> Qt = phi_q E gscale, packed bf16 pairs into TMEM
-      if (full) {
-      tmem_ld32(tb + lane_off + C_ZQ, z);
-      tmem_ld32(tb + lane_off + C_ZQ + 32, z + 32);
-      feature_map_row(z, neg);
-#pragma unroll
-      for (int c16 = 0; c16 < 8; ++c16) {     // 16 dims = 8 TMEM columns
-        float e16[16];
-        unpack8(*chunk_ptr(sm, R_G, row, 2 * c16), e16);
-        unpack8(*chunk_ptr(sm, R_G, row, 2 * c16 + 1), e16 + 8);
-        uint32_t r8[8];
-#pragma unroll
-        for (int u = 0; u < 16; u += 2) {
-          const int i = c16 * 16 + u;
-          const float ph0 = i < F ? z[i] : neg[i - F];
-          const float ph1 = i + 1 < F ? z[i + 1] : neg[i + 1 - F];
-          r8[u / 2] = pack_bf16(ph0 * e16[u] * gscale, ph1 * e16[u + 1] * gscale);
-        }
-        tmem_st8(tb + lane_off + C_QT + c16 * 8, r8);
-      }
-      }
-      // phi_k -> Kt = phi_k / E, bf16 into shared memory over X_k
-      if (full) {
-        tmem_ld32(tb + lane_off + C_ZK, z);
-        tmem_ld32(tb + lane_off + C_ZK + 32, z + 32);
-        feature_map_row(z, neg);
-#pragma unroll
-        for (int c8 = 0; c8 < 16; ++c8) {
-          float e8[8], k8[8];
-          unpack8(*chunk_ptr(sm, R_G, row, c8), e8);
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int i = c8 * 8 + u;
-            const float ph = i < F ? z[i] : neg[i - F];
-            k8[u] = ph * __fdividef(1.f, e8[u]);
-          }
-          *chunk_ptr(sm, R_XK, row, c8) = pack8(k8);
-        }
-      } else {
-        // state pass: E in fp32 from row-wise suffix sums (its states feed
-        // the backward and the segment chain), staged in the unused logits
-        // columns of TMEM
-        for (int c16 = 0; c16 < 8; ++c16) {
-          float E[16], tot[16];
-          row_decay16(sm + R_G, row, c16, qvalid, p.inv_tau, s_wtot, E, tot);
-          uint32_t r[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(E[u]);
-          tmem_st8(tb + lane_off + C_L + c16 * 16, r);
-#pragma unroll
-          for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(E[8 + u]);
-          tmem_st8(tb + lane_off + C_L + c16 * 16 + 8, r);
-#pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            if (row == c16 * 16 + u) {   // this thread's dimension
-              s_dec[row] = __expf(-tot[u]);   // exp(r)
-              tot_decay -= tot[u];             // r, the tile's log-decay
+            for (int k = 0; k < 4; ++k) {
+              const float4 a = *reinterpret_cast<const float4 *>(&s_mk[m0 + k][ch * 8]);
+              const float4 b = *reinterpret_cast<const float4 *>(&s_mk[m0 + k][ch * 8 + 4]);
+              acc[2 * k] = fmaf(q8[0], a.x, fmaf(q8[1], a.y, fmaf(q8[2], a.z, fmaf(q8[3], a.w, acc[2 * k]))));
+              acc[2 * k + 1] = fmaf(q8[4], b.x, fmaf(q8[5], b.y, fmaf(q8[6], b.z, fmaf(q8[7], b.w, acc[2 * k + 1]))));
             }
-            if (row == 0 && E[u] > kMaxSpreadExp && gla) atomicOr(err, ST_RANGE);
+          }
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            if (m0 + k < p.M) s_ml[m0 + k][row] = (acc[2 * k] + acc[2 * k + 1]) * p.scale;
+        }
+        mx = kNegBig;
+        for (int m = 0; m < p.M; ++m) mx = fmaxf(mx, s_ml[m][row]);
+        // Logit column cl holds key t0 - T + cl.  Row r sees columns
+        // [r + T + 1 - window, r + T] (and keys >= 0), so warp w4 only
+        // visits 32-column chunks w4 + (T + 1 - window) / 32 .. w4 + 4, and
+        // only the first and last of those need the band mask.
+        const int w4 = warp & 3;
+        const int cbase = t0 - T;
+        const int lo_c = max(tq - p.window + 1, 0) - cbase, hi_c = tq - cbase;
+        int ch_lo = (32 * w4 + T + 1 - p.window) >> 5;
+        if (cbase < 0) ch_lo = max(ch_lo, 4);
+        const int ch_hi = w4 + 4;
+        const int in_lo = 32 * w4 + 31 + T + 1 - p.window;   // interior chunk: 32 ch >= in_lo
+        for (int ch = ch_lo; ch <= ch_hi; ++ch) {
+          float v[32];
+          tmem_ld32(tl + C_L + ch * 32, v);
+          float m4[4] = {kNegBig, kNegBig, kNegBig, kNegBig};
+          if (32 * ch >= in_lo && 32 * ch + 31 <= 32 * w4 + T && 32 * ch + cbase >= 0) {
+#pragma unroll
+            for (int u = 0; u < 32; ++u) m4[u & 3] = fmaxf(m4[u & 3], v[u]);
+          } else {
+#pragma unroll
+            for (int u = 0; u < 32; ++u) {
+              const int cl = 32 * ch + u;
+              if (cl >= lo_c && cl <= hi_c) m4[u & 3] = fmaxf(m4[u & 3], v[u]);
+            }
+          }
+          const float cm = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+          if (cm > kNegBig) mx = fmaxf(mx, cm * p.scale);
+        }
+        float s4[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int ch = ch_lo; ch <= ch_hi; ++ch) {
+          float v[32];
+          tmem_ld32(tl + C_L + ch * 32, v);
+          const bool inner = 32 * ch >= in_lo && 32 * ch + 31 <= 32 * w4 + T && 32 * ch + cbase >= 0;
+          uint32_t pk[16];
+#pragma unroll
+          for (int u = 0; u < 32; u += 2) {
+            float e0 = __expf(fmaf(v[u], p.scale, -mx));
+            float e1 = __expf(fmaf(v[u + 1], p.scale, -mx));
+            if (!inner) {
+              const int cl = 32 * ch + u;
+              e0 = (cl >= lo_c && cl <= hi_c) ? e0 : 0.f;
+              e1 = (cl + 1 >= lo_c && cl + 1 <= hi_c) ? e1 : 0.f;
+            }
+            s4[(u >> 1) & 3] += e0 + e1;
+            pk[u / 2] = alpha != 0.f ? pack_bf16(e0, e1) : 0u;
+          }
+          tmem_st8(tl + C_P + ch * 16, pk);
+          tmem_st8(tl + C_P + ch * 16 + 8, pk + 8);
+        }
+        // chunks outside the band: P = 0 (written after the band's logits
+        // were read, since P column 16 ch overlays logit chunk ch / 2)
+        {
+          uint32_t zero[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+          for (int ch = 0; ch < 8; ++ch) {
+            if (ch >= ch_lo && ch <= ch_hi) continue;
+            tmem_st8(tl + C_P + ch * 16, zero);
+            tmem_st8(tl + C_P + ch * 16 + 8, zero);
           }
         }
-        tmem_st_wait();
-        tmem_ld32(tb + lane_off + C_ZK, z);
-        tmem_ld32(tb + lane_off + C_ZK + 32, z + 32);
-        feature_map_row(z, neg);
-#pragma unroll
-        for (int c16 = 0; c16 < 8; ++c16) {
-          float E[16], k16[16];
-          tmem_ld16(tb + lane_off + C_L + c16 * 16, E);
-#pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const int i = c16 * 16 + u;
-            k16[u] = (i < F ? z[i] : neg[i - F]) * __fdividef(1.f, E[u]);
-          }
-          *chunk_ptr(sm, R_XK, row, 2 * c16) = pack8(k16);
-          *chunk_ptr(sm, R_XK, row, 2 * c16 + 1) = pack8(k16 + 8);
+        float sm_meta = 0.f;
+        for (int m = 0; m < p.M; ++m) {
+          const float e = __expf(s_ml[m][row] - mx);
+          sm_meta += e;
+          s_ml[m][row] = e;
         }
+        lsum = ((s4[0] + s4[1]) + (s4[2] + s4[3])) + sm_meta;
+        if (!qvalid) lsum = 1.f;
+        if (qvalid && p.lse) p.lse[(size_t)bh * p.L + tq] = mx + logf(lsum);
       }
-    }
-
-    // ------------------------------- state rescale (thread = dimension) ---
-    if (gla) {
-      const int i = row;
-      const float dec = s_dec[i];
-      for (int c16 = 0; c16 < 8; ++c16) {
-        float v[16];
-        tmem_ld16(tb + lane_off + C_S + c16 * 16, v);
+      // GLA operands carry l/alpha so that one accumulator holds both terms
+      const bool mixed = swa && alpha != 0.f;
+      const float gscale = mixed ? lsum / alpha : 1.f;
+      s_gscale[row] = gscale;
+      s_oscale[row] = mixed ? alpha / lsum : 1.f;
+      if (swa) {
+        const float mscale = mixed ? alpha / lsum : 0.f;   // meta-value weight per exp
+        for (int m = 0; m < p.M; ++m) s_ml[m][row] *= mscale;
+      }
+      bar_arrive(BAR_G, NTHREADS);
+      bar_sync(BAR_E, NTHREADS);
+      qt_half(sm, tl, row, 0, gscale);
+      kt_half(sm, tl, row, 0, false);
+    } else {
+      // ------------- state pass: fp32 decay factors, phi_k half per group ---
+      for (int c16 = 4 * wg; c16 < 4 * wg + 4; ++c16) {
+        float E[16], tot[16];
+        row_decay16(sm + R_G, row, c16, qvalid, p.inv_tau, s_wtot[wg], E, tot, BAR_DECAY + wg);
         uint32_t r[8];
 #pragma unroll
-        for (int u = 0; u < 16; ++u) v[u] *= dec;
+        for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(E[u]);
+        tmem_st8(tl + C_L + c16 * 16, r);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(v[u]);
-        tmem_st8(tb + lane_off + C_S + c16 * 16, r);
+        for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(E[8 + u]);
+        tmem_st8(tl + C_L + c16 * 16 + 8, r);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(v[8 + u]);
-        tmem_st8(tb + lane_off + C_S + c16 * 16 + 8, r);
-        if (full) {   // bf16 copy S'[i][v], MN-major: rows = i (K of the O = Qt S' product)
-          *chunk_ptr(sm, R_XQ, i, 2 * c16) = pack8(v);
-          *chunk_ptr(sm, R_XQ, i, 2 * c16 + 1) = pack8(v + 8);
-        } else if (p.snap) {   // the backward's copy of S', row-major [i][v]
-          uint4 *dst = reinterpret_cast<uint4 *>(p.snap + (((size_t)bh * ntiles_all + c) * D + i) * D + c16 * 16);
-          dst[0] = pack8(v);
-          dst[1] = pack8(v + 8);
+        for (int u = 0; u < 16; ++u) {
+          if (row == c16 * 16 + u) {   // the dimension this thread owns
+            s_dec[row] = __expf(-tot[u]);   // exp(r)
+            tot_decay -= tot[u];             // r, the tile's log-decay
+          }
+          if (row == 0 && E[u] > kMaxSpreadExp && gla) atomicOr(err, ST_RANGE);
         }
       }
+      tmem_st_wait();
+      ok &= mbar_wait(&bar_m1, par, err, ST_TIMEOUT);
+      tc_fence_after();
+      kt_half(sm, tl, row, wg, true);
     }
     tmem_st_wait();
     fence_proxy_async();
     tc_fence_before();
-    __syncthreads();
+    if (__syncthreads_or(!ok)) { s_fail = 1; break; }
 
     // ---------------------------------------------------------- MMA 2 ---
     if (tid == 0) {
@@ -462,15 +482,42 @@ __global__ void __launch_bounds__(128, 1) tc_fwd_kernel(const __grid_constant__ 
         tma_load_3d(sm + R_G + REG, &p.mv, &bar_vp, 64, t0 - T, bh);
       }
     }
+
+    // -------------- state rescale (thread = dimension, column half per group) ---
+    if (gla) {
+      tc_fence_after();
+      const int i = row;
+      const float dec = s_dec[i];
+      for (int c16 = 4 * wg; c16 < 4 * wg + 4; ++c16) {
+        float v[16];
+        tmem_ld16(tl + C_S + c16 * 16, v);
+        uint32_t r[8];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) v[u] *= dec;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(v[u]);
+        tmem_st8(tl + C_S + c16 * 16, r);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(v[8 + u]);
+        tmem_st8(tl + C_S + c16 * 16 + 8, r);
+        if (full) {   // bf16 copy S'[i][v], MN-major: rows = i (K of the O = Qt S' product)
+          *chunk_ptr(sm, R_XQ, i, 2 * c16) = pack8(v);
+          *chunk_ptr(sm, R_XQ, i, 2 * c16 + 1) = pack8(v + 8);
+        } else if (p.snap) {   // the backward's copy of S', row-major [i][v]
+          uint4 *dst = reinterpret_cast<uint4 *>(p.snap + (((size_t)bh * ntiles_all + c) * D + i) * D + c16 * 16);
+          dst[0] = pack8(v);
+          dst[1] = pack8(v + 8);
+        }
+      }
+    }
     ok = mbar_wait(&bar_m2, par, err, ST_TIMEOUT);
-    if (__syncthreads_or(!ok)) { s_fail = 1; break; }
     tc_fence_after();
 
-    // ------------------------------------------ rows: masked intra A ---
+    // ---------------------- masked intra A (column half per group) ---
     if (gla && full) {
-      for (int c16 = 0; c16 < 8; ++c16) {
+      for (int c16 = 4 * wg; c16 < 4 * wg + 4; ++c16) {
         float v[16];
-        tmem_ld16(tb + lane_off + C_A + c16 * 16, v);
+        tmem_ld16(tl + C_A + c16 * 16, v);
         uint32_t r[8];
 #pragma unroll
         for (int u = 0; u < 16; u += 2) {
@@ -480,12 +527,13 @@ __global__ void __launch_bounds__(128, 1) tc_fwd_kernel(const __grid_constant__ 
           const float a1 = (j + 1 <= row) ? v[u + 1] : 0.f;
           r[u / 2] = pack_bf16(a0, a1);
         }
-        tmem_st8(tb + lane_off + C_AH + c16 * 8, r);
+        tmem_st8(tl + C_AH + c16 * 8, r);
       }
     }
     tmem_st_wait();
+    fence_proxy_async();
     tc_fence_before();
-    ok = mbar_wait(&bar_vp, par, err, ST_TIMEOUT);
+    ok &= mbar_wait(&bar_vp, par, err, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) { s_fail = 1; break; }
 
     // ---------------------------------------------------------- MMA 3 ---
@@ -510,22 +558,27 @@ __global__ void __launch_bounds__(128, 1) tc_fwd_kernel(const __grid_constant__ 
     tc_fence_after();
     if (tid == 0 && c + 1 < cend) issue_tile_loads(p, sm, &bar_tma, bh, t0 + T, full);
 
-    // -------------------------------------------------------- epilogue ---
+    // ---------------------------- epilogue (column half per group) ---
     if (full) {
       // tcgen05.ld is warp-collective: every lane loads, valid rows store
       __nv_bfloat16 *orow = p.o + ((size_t)bh * p.L + (qvalid ? tq : 0)) * D;
-      for (int c16 = 0; c16 < 8; ++c16) {
+      const float oscale = s_oscale[row];
+      for (int c16 = 4 * wg; c16 < 4 * wg + 4; ++c16) {
         float v[16];
-        tmem_ld16(tb + lane_off + C_O + c16 * 16, v);
+        tmem_ld16(tl + C_O + c16 * 16, v);
 #pragma unroll
         for (int u = 0; u < 16; ++u) v[u] *= oscale;
         if (swa && p.meta_v) {
+          for (int m = 0; m < p.M; ++m) {
+            const float w = s_ml[m][row];
+            const float4 *mv = reinterpret_cast<const float4 *>(&s_mv[m][c16 * 16]);
 #pragma unroll
-          for (int m = 0; m < MAXM; ++m) {
-            if (m < p.M) {
-              const float w = mscale * em[m];
-#pragma unroll
-              for (int u = 0; u < 16; ++u) v[u] = fmaf(w, s_mv[m][c16 * 16 + u], v[u]);
+            for (int q4 = 0; q4 < 4; ++q4) {
+              const float4 x = mv[q4];
+              v[4 * q4] = fmaf(w, x.x, v[4 * q4]);
+              v[4 * q4 + 1] = fmaf(w, x.y, v[4 * q4 + 1]);
+              v[4 * q4 + 2] = fmaf(w, x.z, v[4 * q4 + 2]);
+              v[4 * q4 + 3] = fmaf(w, x.w, v[4 * q4 + 3]);
             }
           }
         }
@@ -535,7 +588,6 @@ __global__ void __launch_bounds__(128, 1) tc_fwd_kernel(const __grid_constant__ 
           dst[1] = pack8(v + 8);
         }
       }
-      if (qvalid && p.lse && swa) p.lse[(size_t)bh * p.L + tq] = mx + logf(lsum);
     }
     tc_fence_before();
     __syncthreads();
@@ -545,16 +597,16 @@ __global__ void __launch_bounds__(128, 1) tc_fwd_kernel(const __grid_constant__ 
   if (full && p.state_out && gla && seg == p.nseg - 1) sdst = p.state_out + ((size_t)bh * D + row) * D;
   if (!full && p.seg_state) {
     sdst = p.seg_state + (((size_t)bh * p.nseg + seg) * D + row) * D;
-    p.seg_decay[((size_t)bh * p.nseg + seg) * D + row] = tot_decay;
+    if ((row >> 6) == wg) p.seg_decay[((size_t)bh * p.nseg + seg) * D + row] = tot_decay;
   }
   if (!s_fail && sdst) {
     tc_fence_after();
-    float *dst = sdst;
-    for (int c16 = 0; c16 < 8; ++c16) {
+    for (int c16 = 4 * wg; c16 < 4 * wg + 4; ++c16) {
       float v[16];
-      tmem_ld16(tb + lane_off + C_S + c16 * 16, v);
+      tmem_ld16(tl + C_S + c16 * 16, v);
 #pragma unroll
-      for (int u = 0; u < 16; u += 4) *reinterpret_cast<float4 *>(dst + c16 * 16 + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
+      for (int u = 0; u < 16; u += 4)
+        *reinterpret_cast<float4 *>(sdst + c16 * 16 + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
     }
   }
   if (s_fail && tid == 0) {
@@ -648,7 +700,7 @@ cudaError_t launch_tc_state_snapshots(const TcFwdArgs &a, void *snap, cudaStream
   p.seg_decay = nullptr;
   cudaError_t e = cudaFuncSetAttribute(tc_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  tc_fwd_kernel<<<dim3(a.BH, 1), 128, SMEM_BYTES, s>>>(p);
+  tc_fwd_kernel<<<dim3(a.BH, 1), NTHREADS, SMEM_BYTES, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -702,10 +754,10 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, int stage, cudaStream_t s) {
   }
   if (nseg > 1 && stage == 0) {          // state pass over every segment but the last
     p.mode = 1;
-    tc_fwd_kernel<<<dim3(a.BH, nseg - 1), 128, SMEM_BYTES, s>>>(p);
+    tc_fwd_kernel<<<dim3(a.BH, nseg - 1), NTHREADS, SMEM_BYTES, s>>>(p);
   } else {                               // full pass
     p.mode = 0;
-    tc_fwd_kernel<<<dim3(a.BH, nseg), 128, SMEM_BYTES, s>>>(p);
+    tc_fwd_kernel<<<dim3(a.BH, nseg), NTHREADS, SMEM_BYTES, s>>>(p);
   }
   return cudaGetLastError();
 }
