@@ -59,14 +59,32 @@ def bytes_per_token_head(d, esz=2):
     return {"fwd": fwd, "bwd": bwd, "train": fwd + bwd}
 
 
+def tc_segments(BH, L, T=128):
+    """Segments per sequence of the tensor-core forward (mirrors the library:
+    enough (batch, head, segment) CTAs to cover the SMs once, each segment at
+    least two tiles long)."""
+    nt = math.ceil(L / T)
+    n = 1 if BH >= 120 else SM_COUNT // max(BH, 1)
+    n = max(1, min(n, nt // 2))
+    tps = math.ceil(nt / n)
+    return math.ceil(nt / tps)
+
+
 def kernel_model(name, w, N, BH):
     """(algorithmic bytes, algorithmic flops) of one launch of a kernel of the
-    library over N token-heads (BH sequences).  Workspace arrays are fp32."""
+    library over N token-heads (BH sequences): every input and output of the
+    kernel counted once (workspace arrays at their stored width), and the
+    dense contractions it exists to perform."""
     d, esz = w.d, 2 if w.dtype == "bf16" else 4
     Nd = N * d
     fl = flops_per_token_head(d, w.chunk, w.window, w.M)
     phi = 2 * d * d   # two feature maps: x W for q and k, d x d/2 each
     nch32 = math.ceil(w.L / 32)
+    nt = math.ceil(w.L / 128)
+    snaps = BH * nt * d * d * 2          # one bf16 d x d state per 128-token tile
+    nseg = tc_segments(BH, w.L)
+    seg_states = BH * nseg * d * d * 4
+    mw = 16                               # per-row meta buffers [N][16] fp32
     table = {
         # portable kernels
         "prep_kernel": (3 * Nd * esz + 3 * Nd * 4, N * phi),
@@ -78,6 +96,22 @@ def kernel_model(name, w, N, BH):
         "swa_bwd_q": (4 * Nd * esz + Nd * 4 + 2 * N * 4, N * 1.5 * fl["swa_fwd"]),
         "swa_bwd_kv": (4 * Nd * esz + 2 * N * 4 + 2 * Nd * 4, N * 1.0 * fl["swa_fwd"]),
         "finish_bwd": (3 * Nd * esz + 7 * Nd * 4 + 3 * Nd * esz + Nd * 4, N * 2 * phi),
+        # tensor-core kernels
+        "tc_fwd_kernel": (5 * Nd * esz + N * 4 + (seg_states if nseg > 1 else 0),
+                          N * (fl["fwd"] + phi)),
+        "tc_fwd_kernel(state pass)": (3 * Nd * esz * (nseg - 1) / nseg + seg_states,
+                                      N * (nseg - 1) / nseg * (2 * d * d + phi / 2)),
+        "seg_combine_kernel": (3 * seg_states, 0),
+        "tc_fwd_kernel(state copies)": (3 * Nd * esz + snaps, N * (2 * d * d + phi / 2)),
+        "tc_gla_dstates_kernel": (3 * Nd * esz + snaps + BH * d * d * 4, N * (2 * d * d + phi / 2)),
+        "tc_gla_bwd_tile_kernel": (5 * Nd * esz + 2 * snaps + 4 * Nd * 4,
+                                   N * (2 * fl["gla_fwd"] + phi)),
+        "tc_swa_bwd_q_kernel": (4 * Nd * esz + Nd * 4 + 2 * N * 4 + 2 * N * mw * 4,
+                                N * 1.5 * fl["swa_fwd"]),
+        "tc_swa_bwd_kv_kernel": (4 * Nd * esz + 2 * N * 4 + 2 * Nd * 4, N * 2.0 * fl["swa_fwd"]),
+        "meta_grad_kernel": (2 * Nd * esz + 2 * N * mw * 4, N * 4 * d * w.M),
+        "tc_finish_kernel": (5 * Nd * esz + 6 * Nd * 4, N * 3 * phi),
+        "gate_grad_kernel": (Nd * 4 + Nd * esz + Nd * 4, 0),
     }
     return table.get(name, (0, 0))
 
@@ -243,7 +277,8 @@ def run_ours(args, rank, world, local):
     dbytes, dflops = kernel_model(dom, w, N, BH)
     dt = per[dom] / 1e3
     ai = dflops / max(dbytes, 1)
-    if dom.endswith("_simt") or dom in ("prep_kernel", "swa_bwd_q", "swa_bwd_kv", "finish_bwd"):
+    if dom.endswith("_simt") or dom in ("prep_kernel", "swa_bwd_q", "swa_bwd_kv", "finish_bwd",
+                                         "meta_grad_kernel", "gate_grad_kernel"):
         # CUDA-core kernels: fp32 FMA peak from unit counts and clock
         alu_peak = SM_COUNT * FP32_LANES_PER_SM * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
         ridge = alu_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)

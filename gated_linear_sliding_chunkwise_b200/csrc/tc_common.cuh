@@ -229,6 +229,28 @@ __device__ __forceinline__ float log_decay_fast(float g, float inv_tau) {
   return (fminf(g, 0.f) - __logf(1.f + __expf(-fabsf(g)))) * inv_tau;
 }
 
+// One half of the feature map of this thread's row, from the 64
+// projections z in TMEM: half 0 is softmax(z), half 1 is softmax(-z).  ph
+// gets the unnormalised terms exp(+-z_f - max); the result is 1 / their sum.
+__device__ __forceinline__ float feature_half(uint32_t taddr, int half, float *ph) {
+  tmem_ld32(taddr, ph);
+  tmem_ld32(taddr + 32, ph + 32);
+  const float sg = half ? -1.f : 1.f;
+  float m[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) m[k] = sg * ph[k];
+#pragma unroll
+  for (int f = 4; f < 64; ++f) m[f & 3] = fmaxf(m[f & 3], sg * ph[f]);
+  const float mx = fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+  float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int f = 0; f < 64; ++f) {
+    ph[f] = __expf(fmaf(sg, ph[f], -mx));
+    s[f & 3] += ph[f];
+  }
+  return 1.f / ((s[0] + s[1]) + (s[2] + s[3]));
+}
+
 // In-tile decay factors in fp32, thread = tile row t (128 threads, 4 warps),
 // for the 16 key dimensions 16 c16 .. 16 c16 + 15:
 //   E[u]   = exp(sum_{s > t} -a_s)   (= exp(b_t - r), b the in-tile cumsum)

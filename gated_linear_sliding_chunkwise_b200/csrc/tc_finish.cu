@@ -38,7 +38,11 @@ struct Params {
   int H, L;
 };
 
-__global__ void __launch_bounds__(128, 1) tc_finish_kernel(const __grid_constant__ Params p) {
+// Two warpgroups (256 threads), thread = tile row `row` of its group:
+// group 0 forms dz of the q map and writes dq, group 1 those of the k map
+// and dk; each writes half of dv's columns.
+constexpr int NTHREADS = 256;
+__global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_constant__ Params p) {
   extern __shared__ unsigned char smraw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
   __shared__ uint64_t bar_tma, bar_z, bar_d;
@@ -48,8 +52,8 @@ __global__ void __launch_bounds__(128, 1) tc_finish_kernel(const __grid_constant
                      R_ZK = 3 * TILE + REG;
   // TMEM: dWq [0,64) dWk [64,128) Zq [128,192) Zk [192,256) dXq [256,384) dXk [384,512)
   constexpr uint32_t C_WQ = 0, C_WK = 64, C_ZQ = 128, C_ZK = 192, C_XQ = 256, C_XK = 384;
-  const int tid = threadIdx.x, warp = tid >> 5, row = tid;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const int tid = threadIdx.x, warp = tid >> 5, wg = tid >> 7, row = tid & 127;
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
   const int bh = blockIdx.x, h = bh % p.H;
   const uint32_t sbase = smem_u32(sm);
   const bool gla = p.dphq != nullptr;
@@ -60,23 +64,23 @@ __global__ void __launch_bounds__(128, 1) tc_finish_kernel(const __grid_constant
     mbar_init(&bar_d, 1);
     fence_barrier_init();
   }
-  // weights -> bf16 [dk row][feature] (MN-major for z = x W, K-major for dz W^T)
-#pragma unroll
-  for (int m = 0; m < 2; ++m) {
-    const float *W = m == 0 ? p.wq : p.wk;
+  // weights -> bf16 [dk row][feature] (MN-major for z = x W, K-major for dz W^T);
+  // group 0 W_q, group 1 W_k
+  {
+    const float *W = wg == 0 ? p.wq : p.wk;
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
       float f[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) f[u] = W[((size_t)h * D + row) * F + c * 8 + u];
-      *reinterpret_cast<uint4 *>(sm + (m == 0 ? R_WQ : R_WK) + sw128_offset(row, c * 8)) = pack8(f);
+      *reinterpret_cast<uint4 *>(sm + (wg == 0 ? R_WQ : R_WK) + sw128_offset(row, c * 8)) = pack8(f);
     }
   }
   fence_proxy_async();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tb = s_tmem;
+  const uint32_t tb = s_tmem, tl = tb + lane_off;
   const int ntiles = (p.L + T - 1) / T;
   const uint32_t id_z = idesc_bf16(128, 64, 0, 1);     // X (K-major) x W (MN-major, N = 64)
   const uint32_t id_dx = idesc_bf16(128, 128, 0, 0);   // dZ (K-major) x W^T (K-major, N = 128)
@@ -107,40 +111,29 @@ __global__ void __launch_bounds__(128, 1) tc_finish_kernel(const __grid_constant
       ok = mbar_wait(&bar_z, par, p.status, ST_TIMEOUT);
       if (__syncthreads_or(!ok)) { fail = true; break; }
       tc_fence_after();
-      // dz rows (fp32 math) -> bf16 dZ tiles
-#pragma unroll
-      for (int m = 0; m < 2; ++m) {
+      // dz row of this group's map (fp32 math) -> bf16 dZ tile
+      {
         float pos[F], neg[F];
-        tmem_ld32(tb + lane_off + (m == 0 ? C_ZQ : C_ZK), pos);
-        tmem_ld32(tb + lane_off + (m == 0 ? C_ZQ : C_ZK) + 32, pos + 32);
-        const float *src = (m == 0 ? p.dphq : p.dphk) + off;
-        float mx = pos[0], mn = pos[0];
+        const float sp = feature_half(tl + (wg == 0 ? C_ZQ : C_ZK), 0, pos);
+        const float sn = feature_half(tl + (wg == 0 ? C_ZQ : C_ZK), 1, neg);
+        const float *__restrict__ src = (wg == 0 ? p.dphq : p.dphk) + off;
 #pragma unroll
-        for (int f = 1; f < F; ++f) { mx = fmaxf(mx, pos[f]); mn = fminf(mn, pos[f]); }
-        float sp = 0.f, sn = 0.f;
-#pragma unroll
-        for (int f = 0; f < F; ++f) {
-          neg[f] = __expf(mn - pos[f]);
-          pos[f] = __expf(pos[f] - mx);
-          sp += pos[f];
-          sn += neg[f];
-        }
-        const float ip = 1.f / sp, in_ = 1.f / sn;
+        for (int f = 0; f < F; ++f) { pos[f] *= sp; neg[f] *= sn; }
         // pass 1: <dp, p> and <dn, n>
-        float dotp = 0.f, dotn = 0.f;
-#pragma unroll
-        for (int f = 0; f < F; ++f) { pos[f] *= ip; neg[f] *= in_; }
+        float dp4[4] = {0.f, 0.f, 0.f, 0.f}, dn4[4] = {0.f, 0.f, 0.f, 0.f};
         if (valid) {
 #pragma unroll
           for (int u = 0; u < F; u += 4) {
             const float4 a = *reinterpret_cast<const float4 *>(src + u);
             const float4 b = *reinterpret_cast<const float4 *>(src + F + u);
-            dotp += a.x * pos[u] + a.y * pos[u + 1] + a.z * pos[u + 2] + a.w * pos[u + 3];
-            dotn += b.x * neg[u] + b.y * neg[u + 1] + b.z * neg[u + 2] + b.w * neg[u + 3];
+            dp4[(u >> 2) & 3] += a.x * pos[u] + a.y * pos[u + 1] + a.z * pos[u + 2] + a.w * pos[u + 3];
+            dn4[(u >> 2) & 3] += b.x * neg[u] + b.y * neg[u + 1] + b.z * neg[u + 2] + b.w * neg[u + 3];
           }
         }
+        const float dotp = (dp4[0] + dp4[1]) + (dp4[2] + dp4[3]);
+        const float dotn = (dn4[0] + dn4[1]) + (dn4[2] + dn4[3]);
         // pass 2: dz = p (dp - <dp,p>) - n (dn - <dn,n>), 8 features at a time
-        const uint32_t reg = m == 0 ? R_ZQ : R_ZK;
+        const uint32_t reg = wg == 0 ? R_ZQ : R_ZK;
 #pragma unroll
         for (int c8 = 0; c8 < 8; ++c8) {
           float dz[8];
@@ -179,34 +172,40 @@ __global__ void __launch_bounds__(128, 1) tc_finish_kernel(const __grid_constant
       tc_fence_after();
       if (tid == 0 && c + 1 < ntiles) loads(c + 1);   // X tiles consumed by the dW products
     }
-    // dq, dk = GLA (dz W^T) + anchor parts; dv = both parts
+    // dq (group 0), dk (group 1) = GLA (dz W^T) + anchor parts; dv = both
+    // parts, 64 columns per group
 #pragma unroll
-    for (int m = 0; m < 3; ++m) {
-      const float *swa = m == 0 ? p.dq_swa : (m == 1 ? p.dk_swa : p.dv_swa);
-      __nv_bfloat16 *dst = m == 0 ? p.dq : (m == 1 ? p.dk : p.dv);
-      for (int ch = 0; ch < 4; ++ch) {
+    for (int k = 0; k < 2; ++k) {
+      const int m = k == 0 ? wg : 2;
+      const float *__restrict__ swa = m == 0 ? p.dq_swa : (m == 1 ? p.dk_swa : p.dv_swa);
+      const float *__restrict__ gpart = m == 2 ? p.dv_gla : nullptr;
+      __nv_bfloat16 *__restrict__ dst = m == 0 ? p.dq : (m == 1 ? p.dk : p.dv);
+      const int ch0 = m == 2 ? 2 * wg : 0, ch1 = m == 2 ? 2 * wg + 2 : 4;
+      for (int ch = ch0; ch < ch1; ++ch) {
         float v[32];
         if (m < 2 && gla) {
-          tmem_ld32(tb + lane_off + (m == 0 ? C_XQ : C_XK) + ch * 32, v);
+          tmem_ld32(tl + (m == 0 ? C_XQ : C_XK) + ch * 32, v);
         } else {
 #pragma unroll
           for (int u = 0; u < 32; ++u) v[u] = 0.f;
         }
-        if (!valid) continue;
-        if (m == 2 && p.dv_gla)
+        if (valid) {
+        float4 ga[8], sa[8];
 #pragma unroll
-          for (int u = 0; u < 32; u += 4) {
-            const float4 a = *reinterpret_cast<const float4 *>(p.dv_gla + off + ch * 32 + u);
-            v[u] += a.x; v[u + 1] += a.y; v[u + 2] += a.z; v[u + 3] += a.w;
-          }
-        if (swa)
+        for (int u = 0; u < 8; ++u) {
+          ga[u] = gpart ? *reinterpret_cast<const float4 *>(gpart + off + ch * 32 + 4 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+          sa[u] = swa ? *reinterpret_cast<const float4 *>(swa + off + ch * 32 + 4 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
 #pragma unroll
-          for (int u = 0; u < 32; u += 4) {
-            const float4 a = *reinterpret_cast<const float4 *>(swa + off + ch * 32 + u);
-            v[u] += a.x; v[u + 1] += a.y; v[u + 2] += a.z; v[u + 3] += a.w;
-          }
+        for (int u = 0; u < 8; ++u) {
+          v[4 * u] += ga[u].x + sa[u].x;
+          v[4 * u + 1] += ga[u].y + sa[u].y;
+          v[4 * u + 2] += ga[u].z + sa[u].z;
+          v[4 * u + 3] += ga[u].w + sa[u].w;
+        }
 #pragma unroll
         for (int u = 0; u < 32; u += 8) *reinterpret_cast<uint4 *>(dst + off + ch * 32 + u) = pack8(v + u);
+        }
       }
     }
     tc_fence_before();
@@ -214,14 +213,12 @@ __global__ void __launch_bounds__(128, 1) tc_finish_kernel(const __grid_constant
   }
   if (gla && !fail) {
     tc_fence_after();
-    // dW rows: lane = dk index, 64 feature columns per map
-#pragma unroll
-    for (int m = 0; m < 2; ++m) {
-      float *dW = m == 0 ? p.dwq : p.dwk;
-      if (!dW) continue;
+    // dW rows: lane = dk index, 64 feature columns per map; group 0 dW_q, group 1 dW_k
+    float *dW = wg == 0 ? p.dwq : p.dwk;
+    if (dW) {
       float v[32];
       for (int ch = 0; ch < 2; ++ch) {
-        tmem_ld32(tb + lane_off + (m == 0 ? C_WQ : C_WK) + ch * 32, v);
+        tmem_ld32(tl + (wg == 0 ? C_WQ : C_WK) + ch * 32, v);
 #pragma unroll
         for (int u = 0; u < 32; ++u) atomicAdd(dW + ((size_t)h * D + row) * F + ch * 32 + u, v[u]);
       }
@@ -260,7 +257,7 @@ cudaError_t launch_tc_finish(const FinishBwdArgs &a, int BH, cudaStream_t s) {
   p.L = a.L;
   cudaError_t e = cudaFuncSetAttribute(tc_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  tc_finish_kernel<<<BH, 128, SMEM_BYTES, s>>>(p);
+  tc_finish_kernel<<<BH, NTHREADS, SMEM_BYTES, s>>>(p);
   return cudaGetLastError();
 }
 

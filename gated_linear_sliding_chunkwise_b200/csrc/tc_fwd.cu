@@ -108,28 +108,6 @@ __device__ __forceinline__ void issue_tile_loads(const Params &p, unsigned char 
   }
 }
 
-// One half of the feature map of this thread's row, from the 64
-// projections z in TMEM: half 0 is softmax(z), half 1 is softmax(-z).  ph
-// gets the unnormalised terms exp(+-z_f - max); the result is 1 / their sum.
-__device__ __forceinline__ float feature_half(uint32_t taddr, int half, float *ph) {
-  tmem_ld32(taddr, ph);
-  tmem_ld32(taddr + 32, ph + 32);
-  const float sg = half ? -1.f : 1.f;
-  float m[4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) m[k] = sg * ph[k];
-#pragma unroll
-  for (int f = 4; f < F; ++f) m[f & 3] = fmaxf(m[f & 3], sg * ph[f]);
-  const float mx = fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
-  float s[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-  for (int f = 0; f < F; ++f) {
-    ph[f] = __expf(fmaf(sg, ph[f], -mx));
-    s[f & 3] += ph[f];
-  }
-  return 1.f / ((s[0] + s[1]) + (s[2] + s[3]));
-}
-
 // Gates, thread = key dimension i: in-tile suffix sums of the log-decay,
 // E_t = exp(sum_{s>t} -a_s) = exp(b_t - r) written as bf16 over the gate
 // logits, exp(r) (the tile's decay) into s_dec[i].  16 tokens per step; the

@@ -237,38 +237,41 @@ __global__ void __launch_bounds__(128, 1) tc_gla_dstates_kernel(const __grid_con
 }
 
 // ------------------------------------------------------------ per tile ----
-__global__ void __launch_bounds__(128, 1) tc_gla_bwd_tile_kernel(const __grid_constant__ TileParams p) {
+// Two warpgroups (256 threads): each thread owns tile row `row` (TMEM lane)
+// in its group; the groups split the row work by columns (dimension halves
+// for E, phi, dphi and dB; one mask each for dA and dA^T).
+constexpr int NT_TILE = 256;
+__global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __grid_constant__ TileParams p) {
   extern __shared__ unsigned char smraw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
-  __shared__ float s_wtot[4][16];
-  __shared__ uint64_t bars[7];
+  __shared__ float s_wtot[2][4][16];
+  __shared__ uint64_t bars[8];
   __shared__ uint32_t s_tmem;
-  // X_q -> Qt, X_k -> Kt, V, dO, G (gate logits), [W_q | W_k] -> S' -> dS
+  // X_q -> Qt, X_k -> Kt, V, dO, G (gate logits) -> A^T^ (bf16, rows = keys),
+  // [W_q | W_k] -> S' -> dS
   constexpr uint32_t R_XQ = 0, R_XK = TILE, R_V = 2 * TILE, R_O = 3 * TILE, R_G = 4 * TILE, R_W = 5 * TILE;
   // TMEM, in order of use:
   //   dA [128,256) dA^T [256,384) Zq [384,448) Zk [448,512)
-  //   dA^ [128,192) dA^T^ [192,256) E (fp32) [0,128)
-  //   A^T [0,128) -> A^T^ [0,64)
-  //   GQ [256,384) GK [384,512) ; DV [128,256)
-  constexpr uint32_t C_E = 0, C_DA = 128, C_DAT = 256, C_ZQ = 384, C_ZK = 448, C_DAH = 128, C_DATH = 192;
-  constexpr uint32_t C_AT = 0, C_ATH = 0, C_GQ = 256, C_GK = 384, C_DV = 128;
-  const int tid = threadIdx.x, warp = tid >> 5, row = tid;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  //   dA^ [0,64) dA^T^ [64,128) ; E (fp32, kept to the end) [128,256)
+  //   A^T [256,384) ; GQ [256,384) GK [384,512) ; DV [0,128)
+  constexpr uint32_t C_DAH = 0, C_DATH = 64, C_DV = 0, C_DA = 128, C_E = 128, C_DAT = 256, C_AT = 256,
+                     C_GQ = 256, C_ZQ = 384, C_ZK = 448, C_GK = 384;
+  const int tid = threadIdx.x, warp = tid >> 5, wg = tid >> 7, row = tid & 127;
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
   const int c = blockIdx.x, bh = blockIdx.y, h = bh % p.H, t0 = c * T, tq = t0 + row;
   const bool valid = tq < p.L;
   const uint32_t sbase = smem_u32(sm);
   if (warp == 0) { tmem_alloc(&s_tmem, 512); tmem_relinquish(); }
   if (tid == 0) {
-    for (int i = 0; i < 7; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < 8; ++i) mbar_init(&bars[i], 1);
     fence_barrier_init();
   }
-  stage_weights(sm + R_W, p.wq, h, row);
-  stage_weights(sm + R_W + REG, p.wk, h, row);
+  stage_weights(sm + R_W + wg * REG, wg == 0 ? p.wq : p.wk, h, row);
   fence_proxy_async();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tb = s_tmem;
+  const uint32_t tb = s_tmem, tl = tb + lane_off;
   const int snap_idx = bh * p.ntiles + c;
   if (tid == 0) {
     mbar_expect_tx(&bars[0], 5 * TILE);
@@ -302,85 +305,65 @@ __global__ void __launch_bounds__(128, 1) tc_gla_bwd_tile_kernel(const __grid_co
     tma_load_3d(sm + R_W, &p.msp, &bars[2], 0, 0, snap_idx);
     tma_load_3d(sm + R_W + REG, &p.msp, &bars[2], 64, 0, snap_idx);
   }
-  // 2. masked dA (row = query; written over its own columns as read) ...
-  for (int ch = 0; ch < 4; ++ch) {
-    float v[32];
-    tmem_ld32(tb + lane_off + C_DA + ch * 32, v);
-    uint32_t a[16];
+  // 2. group 0: masked dA (row = query, key j <= row); group 1: masked dA^T
+  //    (row = key, query j >= row); packed bf16 into [0,128)
+  {
+    const uint32_t src = wg == 0 ? C_DA : C_DAT, dst = wg == 0 ? C_DAH : C_DATH;
+    for (int ch = 0; ch < 4; ++ch) {
+      float v[32];
+      tmem_ld32(tl + src + ch * 32, v);
+      uint32_t a[16];
 #pragma unroll
-    for (int u = 0; u < 32; u += 2) {
-      const int j = ch * 32 + u;          // key j <= query row
-      a[u / 2] = pack_bf16(j <= row ? v[u] : 0.f, j + 1 <= row ? v[u + 1] : 0.f);
+      for (int u = 0; u < 32; u += 2) {
+        const int j = ch * 32 + u;
+        const bool k0 = wg == 0 ? j <= row : j >= row, k1 = wg == 0 ? j + 1 <= row : j + 1 >= row;
+        a[u / 2] = pack_bf16(k0 ? v[u] : 0.f, k1 ? v[u + 1] : 0.f);
+      }
+      tmem_st8(tl + dst + ch * 16, a);
+      tmem_st8(tl + dst + ch * 16 + 8, a + 8);
     }
-    tmem_st8(tb + lane_off + C_DAH + ch * 16, a);
-    tmem_st8(tb + lane_off + C_DAH + ch * 16 + 8, a + 8);
   }
-  //    ... then masked dA^T (row = key) into the consumed upper half of dA
-  for (int ch = 0; ch < 4; ++ch) {
-    float w[32];
-    tmem_ld32(tb + lane_off + C_DAT + ch * 32, w);
-    uint32_t b[16];
-#pragma unroll
-    for (int u = 0; u < 32; u += 2) {
-      const int j = ch * 32 + u;          // query j >= key row
-      b[u / 2] = pack_bf16(j >= row ? w[u] : 0.f, j + 1 >= row ? w[u + 1] : 0.f);
-    }
-    tmem_st8(tb + lane_off + C_DATH + ch * 16, b);
-    tmem_st8(tb + lane_off + C_DATH + ch * 16 + 8, b + 8);
-  }
-  //    E in fp32 (row-wise suffix sums) into TMEM, then Qt = phi_q E, Kt = phi_k / E
-  for (int c16 = 0; c16 < 8; ++c16) {
+  tmem_st_wait();
+  tc_fence_before();
+  __syncthreads();   // dA read out before E overwrites its columns
+  tc_fence_after();
+  //    E in fp32 (row-wise suffix sums, dimensions 64 wg ..) into TMEM, then
+  //    Qt = phi_q E and Kt = phi_k / E for the same dimensions
+  for (int c16 = 4 * wg; c16 < 4 * wg + 4; ++c16) {
     float E[16], tot[16];
-    row_decay16(sm + R_G, row, c16, valid, p.inv_tau, s_wtot, E, tot);
+    row_decay16(sm + R_G, row, c16, valid, p.inv_tau, s_wtot[wg], E, tot, 3 + wg);
     uint32_t r[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(E[u]);
-    tmem_st8(tb + lane_off + C_E + c16 * 16, r);
+    tmem_st8(tl + C_E + c16 * 16, r);
 #pragma unroll
     for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(E[8 + u]);
-    tmem_st8(tb + lane_off + C_E + c16 * 16 + 8, r);
+    tmem_st8(tl + C_E + c16 * 16 + 8, r);
 #pragma unroll
     for (int u = 0; u < 16; ++u)
       if (row == 0 && E[u] > kMaxSpreadExp) atomicOr(p.status, ST_RANGE);
   }
   tmem_st_wait();
-  {
-    float z[F], neg[F];
-    tmem_ld32(tb + lane_off + C_ZQ, z);
-    tmem_ld32(tb + lane_off + C_ZQ + 32, z + 32);
-    feature_map_row(z, neg);
 #pragma unroll
-    for (int c16 = 0; c16 < 8; ++c16) {
-      float E[16], q16[16];
-      tmem_ld16(tb + lane_off + C_E + c16 * 16, E);
+  for (int m = 0; m < 2; ++m) {
+    float ph[F];
+    const float s = feature_half(tl + (m == 0 ? C_ZQ : C_ZK), wg, ph);
+    const uint32_t reg = m == 0 ? R_XQ : R_XK;
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int i = c16 * 16 + u;
-        q16[u] = (i < F ? z[i] : neg[i - F]) * E[u];
-      }
-      *chunk_ptr(sm, R_XQ, row, 2 * c16) = pack8(q16);
-      *chunk_ptr(sm, R_XQ, row, 2 * c16 + 1) = pack8(q16 + 8);
-    }
-    tmem_ld32(tb + lane_off + C_ZK, z);
-    tmem_ld32(tb + lane_off + C_ZK + 32, z + 32);
-    feature_map_row(z, neg);
+    for (int c16 = 0; c16 < 4; ++c16) {
+      float E[16], x16[16];
+      tmem_ld16(tl + C_E + 64 * wg + 16 * c16, E);
 #pragma unroll
-    for (int c16 = 0; c16 < 8; ++c16) {
-      float E[16], k16[16];
-      tmem_ld16(tb + lane_off + C_E + c16 * 16, E);
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int i = c16 * 16 + u;
-        k16[u] = (i < F ? z[i] : neg[i - F]) * __fdividef(1.f, E[u]);
-      }
-      *chunk_ptr(sm, R_XK, row, 2 * c16) = pack8(k16);
-      *chunk_ptr(sm, R_XK, row, 2 * c16 + 1) = pack8(k16 + 8);
+      for (int u = 0; u < 16; ++u)
+        x16[u] = m == 0 ? ph[16 * c16 + u] * s * E[u] : __fdividef(ph[16 * c16 + u] * s, E[u]);
+      *chunk_ptr(sm, reg, row, 8 * wg + 2 * c16) = pack8(x16);
+      *chunk_ptr(sm, reg, row, 8 * wg + 2 * c16 + 1) = pack8(x16 + 8);
     }
   }
   fence_proxy_async();
   tc_fence_before();
   __syncthreads();
-  // 3. A^T = Kt Qt^T (rows = keys), over E
+  // 3. A^T = Kt Qt^T (rows = keys)
   if (tid == 0) {
     tc_fence_after();
     for (int s = 0; s < 8; ++s) mma_ss(tb + C_AT, desc_k(sbase + R_XK, s), desc_k(sbase + R_XQ, s), id_kk, s > 0);
@@ -389,59 +372,57 @@ __global__ void __launch_bounds__(128, 1) tc_gla_bwd_tile_kernel(const __grid_co
   ok = mbar_wait(&bars[3], 0, p.status, ST_TIMEOUT);
   if (__syncthreads_or(!ok)) goto done;
   tc_fence_after();
-  for (int ch = 0; ch < 4; ++ch) {
+  //    A^T^ = A^T masked to queries j >= key row, bf16 K-major over the gate
+  //    tile (consumed), 64 query columns per group
+  for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
     float v[32];
-    tmem_ld32(tb + lane_off + C_AT + ch * 32, v);
-    uint32_t a[16];
+    tmem_ld32(tl + C_AT + ch * 32, v);
 #pragma unroll
-    for (int u = 0; u < 32; u += 2) {
-      const int j = ch * 32 + u;                 // query index, row = key
-      a[u / 2] = pack_bf16(j >= row ? v[u] : 0.f, j + 1 >= row ? v[u + 1] : 0.f);
-    }
-    tmem_st8(tb + lane_off + C_ATH + ch * 16, a);
-    tmem_st8(tb + lane_off + C_ATH + ch * 16 + 8, a + 8);
+    for (int u = 0; u < 32; ++u) v[u] = (ch * 32 + u >= row) ? v[u] : 0.f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) *chunk_ptr(sm, R_G, row, 4 * ch + k) = pack8(v + 8 * k);
   }
-  tmem_st_wait();
+  fence_proxy_async();
   tc_fence_before();
   ok = mbar_wait(&bars[2], 0, p.status, ST_TIMEOUT);
   if (__syncthreads_or(!ok)) goto done;
-  // 4a. GQ = dO S'^T + dA^ Kt ;  GK = dA^T^ Qt
+  // 4a. GQ = dO S'^T + dA^ Kt ;  GK = dA^T^ Qt ; dS replaces S' once its product is done
   if (tid == 0) {
     tc_fence_after();
     for (int s = 0; s < 8; ++s) mma_ss(tb + C_GQ, desc_k(sbase + R_O, s), desc_k(sbase + R_W, s), id_kk, s > 0);
+    mma_commit(&bars[4]);
     for (int s = 0; s < 8; ++s) mma_ts(tb + C_GQ, tb + C_DAH + s * 8, desc_mn(sbase + R_XK, s), id_mn, 1);
     for (int s = 0; s < 8; ++s) mma_ts(tb + C_GK, tb + C_DATH + s * 8, desc_mn(sbase + R_XQ, s), id_mn, s > 0);
-    mma_commit(&bars[4]);
-  }
-  ok = mbar_wait(&bars[4], 0, p.status, ST_TIMEOUT);
-  if (__syncthreads_or(!ok)) goto done;
-  tc_fence_after();
-  if (tid == 0) {   // S' consumed: dS goes into its place
-    mbar_expect_tx(&bars[5], TILE);
-    tma_load_3d(sm + R_W, &p.mds, &bars[5], 0, 0, snap_idx);
-    tma_load_3d(sm + R_W + REG, &p.mds, &bars[5], 64, 0, snap_idx);
+    mma_commit(&bars[5]);
+    if (mbar_wait(&bars[4], 0, p.status, ST_TIMEOUT)) {
+      mbar_expect_tx(&bars[6], TILE);
+      tma_load_3d(sm + R_W, &p.mds, &bars[6], 0, 0, snap_idx);
+      tma_load_3d(sm + R_W + REG, &p.mds, &bars[6], 64, 0, snap_idx);
+    }
   }
   ok = mbar_wait(&bars[5], 0, p.status, ST_TIMEOUT);
+  ok &= mbar_wait(&bars[6], 0, p.status, ST_TIMEOUT);
   if (__syncthreads_or(!ok)) goto done;
   // 4b. GK += V dS^T ;  DV = A^T^ dO + Kt dS
   if (tid == 0) {
     tc_fence_after();
     for (int s = 0; s < 8; ++s) mma_ss(tb + C_GK, desc_k(sbase + R_V, s), desc_k(sbase + R_W, s), id_kk, 1);
-    for (int s = 0; s < 8; ++s) mma_ts(tb + C_DV, tb + C_ATH + s * 8, desc_mn(sbase + R_O, s), id_mn, s > 0);
+    for (int s = 0; s < 8; ++s) mma_ss(tb + C_DV, desc_k(sbase + R_G, s), desc_mn(sbase + R_O, s), id_mn, s > 0);
     for (int s = 0; s < 8; ++s) mma_ss(tb + C_DV, desc_k(sbase + R_XK, s), desc_mn(sbase + R_W, s), id_mn, 1);
-    mma_commit(&bars[6]);
+    mma_commit(&bars[7]);
   }
-  ok = mbar_wait(&bars[6], 0, p.status, ST_TIMEOUT);
+  ok = mbar_wait(&bars[7], 0, p.status, ST_TIMEOUT);
   if (__syncthreads_or(!ok)) goto done;
   tc_fence_after();
-  // 5. rows: dphi_q = E GQ, dphi_k = GK / E, dB = Qt GQ - Kt GK (E in fp32 again), dv
+  // 5. rows, dimension half per group: dphi_q = E GQ, dphi_k = GK / E,
+  //    dB = Qt GQ - Kt GK; then dv (64 columns per group)
   {
     const size_t off = ((size_t)bh * p.L + (valid ? tq : 0)) * D;
-    for (int c16 = 0; c16 < 8; ++c16) {
-      float E[16], tot[16], gq[16], gk[16];
-      row_decay16(sm + R_G, row, c16, valid, p.inv_tau, s_wtot, E, tot);
-      tmem_ld16(tb + lane_off + C_GQ + c16 * 16, gq);
-      tmem_ld16(tb + lane_off + C_GK + c16 * 16, gk);
+    for (int c16 = 4 * wg; c16 < 4 * wg + 4; ++c16) {
+      float E[16], gq[16], gk[16];
+      tmem_ld16(tl + C_E + c16 * 16, E);
+      tmem_ld16(tl + C_GQ + c16 * 16, gq);
+      tmem_ld16(tl + C_GK + c16 * 16, gk);
       float q16[16], k16[16], oq[16], ok16[16], ob[16];
       unpack8(*chunk_ptr(sm, R_XQ, row, 2 * c16), q16);
       unpack8(*chunk_ptr(sm, R_XQ, row, 2 * c16 + 1), q16 + 8);
@@ -450,7 +431,7 @@ __global__ void __launch_bounds__(128, 1) tc_gla_bwd_tile_kernel(const __grid_co
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
         oq[u] = E[u] * gq[u];
-        ok16[u] = gk[u] * __fdividef(1.f, E[u]);
+        ok16[u] = __fdividef(gk[u], E[u]);
         ob[u] = q16[u] * gq[u] - k16[u] * gk[u];
       }
       if (valid) {
@@ -462,9 +443,9 @@ __global__ void __launch_bounds__(128, 1) tc_gla_bwd_tile_kernel(const __grid_co
         }
       }
     }
-    for (int ch = 0; ch < 4; ++ch) {
+    for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
       float dv[32];
-      tmem_ld32(tb + lane_off + C_DV + ch * 32, dv);
+      tmem_ld32(tl + C_DV + ch * 32, dv);
       if (valid)
 #pragma unroll
         for (int u = 0; u < 32; u += 4)
@@ -479,13 +460,33 @@ done:
 
 // ------------------------------------------------------- gate gradient ----
 // dg_t = (sum_{s >= t} dB_s) * sigmoid(-g_t) / tau, one thread per dimension
-__global__ void __launch_bounds__(128) gate_grad_kernel(const float *dB, const __nv_bfloat16 *g, float *dg, int L,
+// dg_t = dlogsigmoid(g_t) / tau * sum_{s >= t} dB_s, per (sequence, key
+// dimension).  One CTA per (sequence, 32 dimensions): warp w owns token
+// segment w of 8 (lane = dimension, so each token row is one coalesced
+// 128-byte read); a first pass sums each segment, the later segments' sums
+// give its carry, and a second pass walks it backwards writing dg.
+constexpr int kGateSeg = 8;
+__global__ void __launch_bounds__(256) gate_grad_kernel(const float *dB, const __nv_bfloat16 *g, float *dg, int L,
                                                        float inv_tau) {
-  const int bh = blockIdx.x, i = threadIdx.x;
+  __shared__ float s_tot[kGateSeg][32];
+  const int bh = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int i = blockIdx.y * 32 + lane;
+  const int seg = (L + kGateSeg - 1) / kGateSeg;
+  const int ta = min(L, warp * seg), tz = min(L, ta + seg);   // this warp's tokens [ta, tz)
   const size_t base = (size_t)bh * L * D + i;
+  float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  int t = ta;
+  for (; t + 8 <= tz; t += 8) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) part[u] += dB[base + (size_t)(t + u) * D];
+  }
+  for (; t < tz; ++t) part[0] += dB[base + (size_t)t * D];
+  s_tot[warp][lane] = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
+  __syncthreads();
   float carry = 0.f;
-  int t = L - 1;
-  for (; t >= 7; t -= 8) {
+  for (int w = warp + 1; w < kGateSeg; ++w) carry += s_tot[w][lane];
+  t = tz - 1;
+  for (; t - 7 >= ta; t -= 8) {
     float b[8], gv[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
@@ -498,7 +499,7 @@ __global__ void __launch_bounds__(128) gate_grad_kernel(const float *dB, const _
       dg[base + (size_t)(t - u) * D] = carry * dlogsigmoid(gv[u]) * inv_tau;
     }
   }
-  for (; t >= 0; --t) {
+  for (; t >= ta; --t) {
     carry += dB[base + (size_t)t * D];
     dg[base + (size_t)t * D] = carry * dlogsigmoid(__bfloat162float(g[base + (size_t)t * D])) * inv_tau;
   }
@@ -556,10 +557,11 @@ cudaError_t launch_tc_gla_bwd(const TcGlaBwdArgs &a, int stage, cudaStream_t s) 
     p.inv_tau = a.inv_tau;
     cudaError_t e = cudaFuncSetAttribute(tc_gla_bwd_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TILE_SMEM);
     if (e != cudaSuccess) return e;
-    tc_gla_bwd_tile_kernel<<<dim3(ntiles, a.BH), 128, TILE_SMEM, s>>>(p);
+    tc_gla_bwd_tile_kernel<<<dim3(ntiles, a.BH), NT_TILE, TILE_SMEM, s>>>(p);
     return cudaGetLastError();
   }
-  gate_grad_kernel<<<a.BH, 128, 0, s>>>(a.dB, static_cast<const __nv_bfloat16 *>(a.g), a.dg, a.L, a.inv_tau);
+  gate_grad_kernel<<<dim3(a.BH, D / 32), 256, 0, s>>>(a.dB, static_cast<const __nv_bfloat16 *>(a.g), a.dg, a.L,
+                                                      a.inv_tau);
   return cudaGetLastError();
 }
 

@@ -412,45 +412,79 @@ done:
 
 // ------------------------------------------------------- meta gradients ---
 // dmeta_k[h][m] += scale sum_t dSm[t][m] q_t ; dmeta_v[h][m] += alpha sum_t pm[t][m] dout_t
-constexpr int kMetaTok = 256;
-__global__ void __launch_bounds__(128) meta_grad_kernel(const __nv_bfloat16 *q, const __nv_bfloat16 *dout,
+//
+// A streaming reduction over the tokens of one head: each warp walks every
+// 8th token of the CTA's range reading whole 256-byte rows of q and dout
+// (lane = 4 dimensions); the per-row meta terms are broadcast loads.  MM is
+// the meta-token count rounded up to 4, 8 or 16; U tokens are in flight per
+// warp.  Warps combine in shared memory, then one global add per element.
+constexpr int kMetaTok = 1024;
+template <int MM, int U>
+__global__ void __launch_bounds__(256) meta_grad_kernel(const __nv_bfloat16 *q, const __nv_bfloat16 *dout,
                                                          const float *dsm, const float *pm, const float *alpha,
                                                          float *dmk, float *dmv, int B, int H, int L, int M,
                                                          float scale) {
-  const int h = blockIdx.y, i = threadIdx.x;
+  __shared__ float s_red[2][MM][D];
+  const int h = blockIdx.y, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int n0 = blockIdx.x * kMetaTok;
   const int n1 = min(B * L, n0 + kMetaTok);
-  float ak[MAXM], av[MAXM];
+  for (int e = threadIdx.x; e < 2 * MM * D; e += 256) (&s_red[0][0][0])[e] = 0.f;
+  float ak[MM][4], av[MM][4];
 #pragma unroll
-  for (int m = 0; m < MAXM; ++m) { ak[m] = 0.f; av[m] = 0.f; }
-  for (int nb = n0; nb < n1; nb += 8) {
-    float qi[8], oi[8];
-    size_t tok[8];
+  for (int m = 0; m < MM; ++m)
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {       // all loads of 8 tokens in flight together
-      const int n = min(nb + u, n1 - 1);
-      tok[u] = ((size_t)(n / L) * H + h) * L + n % L;
-      qi[u] = nb + u < n1 ? __bfloat162float(q[tok[u] * D + i]) : 0.f;
-      oi[u] = nb + u < n1 ? __bfloat162float(dout[tok[u] * D + i]) : 0.f;
+    for (int j = 0; j < 4; ++j) { ak[m][j] = 0.f; av[m][j] = 0.f; }
+  for (int nb = n0 + warp; nb < n1; nb += 8 * U) {
+    uint2 qv[U], ov[U];
+    float4 ds[U][MM / 4], pw[U][MM / 4];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {       // all loads of U tokens in flight together
+      const int n = nb + 8 * u;
+      const bool in = n < n1;
+      const size_t tok = ((size_t)((in ? n : n0) / L) * H + h) * L + (in ? n : n0) % L;
+      qv[u] = in ? *reinterpret_cast<const uint2 *>(q + tok * D + lane * 4) : make_uint2(0u, 0u);
+      ov[u] = in ? *reinterpret_cast<const uint2 *>(dout + tok * D + lane * 4) : make_uint2(0u, 0u);
+#pragma unroll
+      for (int k = 0; k < MM / 4; ++k) {
+        ds[u][k] = in ? *reinterpret_cast<const float4 *>(dsm + tok * MAXM + 4 * k) : make_float4(0.f, 0.f, 0.f, 0.f);
+        pw[u][k] = in ? *reinterpret_cast<const float4 *>(pm + tok * MAXM + 4 * k) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
     }
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < U; ++u) {
+      const float2 q01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&qv[u].x));
+      const float2 q23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&qv[u].y));
+      const float2 o01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ov[u].x));
+      const float2 o23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ov[u].y));
+      const float qf[4] = {q01.x, q01.y, q23.x, q23.y}, of[4] = {o01.x, o01.y, o23.x, o23.y};
 #pragma unroll
-      for (int m = 0; m < MAXM; ++m) {
-        if (m < M) {
-          ak[m] = fmaf(dsm[tok[u] * MAXM + m], qi[u], ak[m]);
-          av[m] = fmaf(pm[tok[u] * MAXM + m], oi[u], av[m]);
-        }
+      for (int k = 0; k < MM / 4; ++k) {
+        const float dk4[4] = {ds[u][k].x, ds[u][k].y, ds[u][k].z, ds[u][k].w};
+        const float pv4[4] = {pw[u][k].x, pw[u][k].y, pw[u][k].z, pw[u][k].w};
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            ak[4 * k + r][j] = fmaf(dk4[r], qf[j], ak[4 * k + r][j]);
+            av[4 * k + r][j] = fmaf(pv4[r], of[j], av[4 * k + r][j]);
+          }
       }
     }
   }
-  const float a = alpha ? alpha[h] : 1.f;
+  __syncthreads();
 #pragma unroll
-  for (int m = 0; m < MAXM; ++m) {
-    if (m < M) {
-      if (dmk) atomicAdd(dmk + ((size_t)h * M + m) * D + i, ak[m] * scale);
-      if (dmv) atomicAdd(dmv + ((size_t)h * M + m) * D + i, av[m] * a);
+  for (int m = 0; m < MM; ++m)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      atomicAdd(&s_red[0][m][lane * 4 + j], ak[m][j]);
+      atomicAdd(&s_red[1][m][lane * 4 + j], av[m][j]);
     }
+  __syncthreads();
+  const float a = alpha ? alpha[h] : 1.f;
+  for (int e = threadIdx.x; e < M * D; e += 256) {
+    const int m = e / D, i = e % D;
+    if (dmk) atomicAdd(dmk + ((size_t)h * M + m) * D + i, s_red[0][m][i] * scale);
+    if (dmv) atomicAdd(dmv + ((size_t)h * M + m) * D + i, s_red[1][m][i] * a);
   }
 }
 
@@ -466,9 +500,17 @@ cudaError_t launch_tc_swa_bwd(const TcSwaBwdArgs &a, int stage, cudaStream_t s) 
   if (stage == 2) {
     if (a.M == 0 || (!a.dmeta_k && !a.dmeta_v)) return cudaSuccess;
     dim3 grid((a.B * a.L + kMetaTok - 1) / kMetaTok, a.H);
-    meta_grad_kernel<<<grid, 128, 0, s>>>(static_cast<const __nv_bfloat16 *>(a.q),
-                                          static_cast<const __nv_bfloat16 *>(a.dout), a.dsm, a.pm, a.alpha,
-                                          a.dmeta_k, a.dmeta_v, a.B, a.H, a.L, a.M, a.scale);
+    const auto *qp = static_cast<const __nv_bfloat16 *>(a.q);
+    const auto *op = static_cast<const __nv_bfloat16 *>(a.dout);
+    if (a.M <= 4)
+      meta_grad_kernel<4, 4><<<grid, 256, 0, s>>>(qp, op, a.dsm, a.pm, a.alpha, a.dmeta_k, a.dmeta_v, a.B, a.H,
+                                                  a.L, a.M, a.scale);
+    else if (a.M <= 8)
+      meta_grad_kernel<8, 2><<<grid, 256, 0, s>>>(qp, op, a.dsm, a.pm, a.alpha, a.dmeta_k, a.dmeta_v, a.B, a.H,
+                                                  a.L, a.M, a.scale);
+    else
+      meta_grad_kernel<16, 1><<<grid, 256, 0, s>>>(qp, op, a.dsm, a.pm, a.alpha, a.dmeta_k, a.dmeta_v, a.B, a.H,
+                                                   a.L, a.M, a.scale);
     return cudaGetLastError();
   }
   // the attribute is per device: set it every launch on devices not yet seen
