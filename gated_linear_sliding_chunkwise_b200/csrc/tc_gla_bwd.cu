@@ -57,25 +57,6 @@ struct TileParams {
 };
 
 
-// feature map of one row: z (64 projections) -> [softmax(z), softmax(-z)]
-__device__ __forceinline__ void feature_map_row(float *z, float *neg) {
-  float mx = z[0], mn = z[0];
-#pragma unroll
-  for (int f = 1; f < F; ++f) { mx = fmaxf(mx, z[f]); mn = fminf(mn, z[f]); }
-  float sp = 0.f, sn = 0.f;
-#pragma unroll
-  for (int f = 0; f < F; ++f) {
-    neg[f] = __expf(mn - z[f]);
-    z[f] = __expf(z[f] - mx);
-    sp += z[f];
-    sn += neg[f];
-  }
-  const float ip = 1.f / sp, in_ = 1.f / sn;
-#pragma unroll
-  for (int f = 0; f < F; ++f) { z[f] *= ip; neg[f] *= in_; }
-}
-
-// W (fp32 [D][F] of head h) -> bf16 shared memory, [dk row][feature], MN-major
 __device__ __forceinline__ void stage_weights(unsigned char *dst, const float *W, int h, int row) {
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
@@ -87,17 +68,21 @@ __device__ __forceinline__ void stage_weights(unsigned char *dst, const float *W
 }
 
 // ------------------------------------------------------ reverse dS pass ---
-__global__ void __launch_bounds__(128, 1) tc_gla_dstates_kernel(const __grid_constant__ DsParams p) {
+// Two warpgroups (256 threads): thread = tile row / state row `row` of its
+// group; the groups take halves of the key dimensions (E, phi_q) and of the
+// state's columns (copy and rescale).
+constexpr int NT_DS = 256;
+__global__ void __launch_bounds__(NT_DS, 1) tc_gla_dstates_kernel(const __grid_constant__ DsParams p) {
   extern __shared__ unsigned char smraw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
   __shared__ float s_dec[D];
-  __shared__ float s_wtot[4][16];
+  __shared__ float s_wtot[2][4][16];
   __shared__ uint64_t bar_tma, bar_m1, bar_m2;
   __shared__ uint32_t s_tmem;
   constexpr uint32_t R_XQ = 0, R_G = TILE, R_O = 2 * TILE, R_W = 3 * TILE;
   constexpr uint32_t C_S = 0, C_Z = 128, C_E = 256;
-  const int tid = threadIdx.x, warp = tid >> 5, row = tid;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const int tid = threadIdx.x, warp = tid >> 5, wg = tid >> 7, row = tid & 127;
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
   const int bh = blockIdx.x, h = bh % p.H;
   const uint32_t sbase = smem_u32(sm);
   const int ntiles = (p.L + T - 1) / T;
@@ -108,15 +93,15 @@ __global__ void __launch_bounds__(128, 1) tc_gla_dstates_kernel(const __grid_con
     mbar_init(&bar_m2, 1);
     fence_barrier_init();
   }
-  stage_weights(sm + R_W, p.wq, h, row);
+  if (wg == 0) stage_weights(sm + R_W, p.wq, h, row);
   fence_proxy_async();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tb = s_tmem;
+  const uint32_t tb = s_tmem, tl = tb + lane_off;
   {   // dS starts at zero: nothing flows into the last tile's end state
     uint32_t z[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int c = 0; c < D; c += 8) tmem_st8(tb + lane_off + C_S + c, z);
+    for (int c = 64 * wg; c < 64 * wg + 64; c += 8) tmem_st8(tl + C_S + c, z);
     tmem_st_wait();
   }
   const uint32_t id_z = idesc_bf16(128, 64, 0, 1);
@@ -141,30 +126,28 @@ __global__ void __launch_bounds__(128, 1) tc_gla_dstates_kernel(const __grid_con
       for (int s = 0; s < 8; ++s) mma_ss(tb + C_Z, desc_k(sbase + R_XQ, s), desc_mn(sbase + R_W, s), id_z, s > 0);
       mma_commit(&bar_m1);
     }
-    // copy of dS (the gradient into this tile's end state)
+    // copy of dS (the gradient into this tile's end state), column half per group
     {
       __nv_bfloat16 *dst = p.snap + (((size_t)bh * ntiles + c) * D + row) * D;
-      for (int ch = 0; ch < 4; ++ch) {
+      for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
         float v[32];
-        tmem_ld32(tb + lane_off + C_S + ch * 32, v);
+        tmem_ld32(tl + C_S + ch * 32, v);
 #pragma unroll
         for (int u = 0; u < 32; u += 8) *reinterpret_cast<uint4 *>(dst + ch * 32 + u) = pack8(v + u);
       }
     }
-    ok = mbar_wait(&bar_m1, par, p.status, ST_TIMEOUT);
-    if (__syncthreads_or(!ok)) { fail = true; break; }
-    tc_fence_after();
-    // E in fp32 (row-wise suffix sums) into TMEM; the tile's decay exp(r)
-    for (int c16 = 0; c16 < 8; ++c16) {
+    // E in fp32 (row-wise suffix sums, dimensions 64 wg ..) into TMEM; the
+    // tile's decay exp(r)
+    for (int c16 = 4 * wg; c16 < 4 * wg + 4; ++c16) {
       float E[16], tot[16];
-      row_decay16(sm + R_G, row, c16, t0 + row < p.L, p.inv_tau, s_wtot, E, tot);
+      row_decay16(sm + R_G, row, c16, t0 + row < p.L, p.inv_tau, s_wtot[wg], E, tot, 3 + wg);
       uint32_t r[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(E[u]);
-      tmem_st8(tb + lane_off + C_E + c16 * 16, r);
+      tmem_st8(tl + C_E + c16 * 16, r);
 #pragma unroll
       for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(E[8 + u]);
-      tmem_st8(tb + lane_off + C_E + c16 * 16 + 8, r);
+      tmem_st8(tl + C_E + c16 * 16 + 8, r);
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
         if (row == u) s_dec[c16 * 16 + u] = __expf(-tot[u]);
@@ -172,27 +155,24 @@ __global__ void __launch_bounds__(128, 1) tc_gla_dstates_kernel(const __grid_con
       }
     }
     tmem_st_wait();
-    {   // Qt = phi_q E into shared memory over X_q (row = token)
-      float z[F], neg[F];
-      tmem_ld32(tb + lane_off + C_Z, z);
-      tmem_ld32(tb + lane_off + C_Z + 32, z + 32);
-      feature_map_row(z, neg);
+    ok = mbar_wait(&bar_m1, par, p.status, ST_TIMEOUT);
+    tc_fence_after();
+    {   // Qt = phi_q E into shared memory over X_q (row = token), dimension half per group
+      float ph[F];
+      const float sc = feature_half(tl + C_Z, wg, ph);
 #pragma unroll
-      for (int c16 = 0; c16 < 8; ++c16) {
+      for (int c16 = 0; c16 < 4; ++c16) {
         float E[16], q16[16];
-        tmem_ld16(tb + lane_off + C_E + c16 * 16, E);
+        tmem_ld16(tl + C_E + 64 * wg + 16 * c16, E);
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int i = c16 * 16 + u;
-          q16[u] = (i < F ? z[i] : neg[i - F]) * E[u];
-        }
-        *chunk_ptr(sm, R_XQ, row, 2 * c16) = pack8(q16);
-        *chunk_ptr(sm, R_XQ, row, 2 * c16 + 1) = pack8(q16 + 8);
+        for (int u = 0; u < 16; ++u) q16[u] = ph[16 * c16 + u] * sc * E[u];
+        *chunk_ptr(sm, R_XQ, row, 8 * wg + 2 * c16) = pack8(q16);
+        *chunk_ptr(sm, R_XQ, row, 8 * wg + 2 * c16 + 1) = pack8(q16 + 8);
       }
     }
     fence_proxy_async();
     tc_fence_before();
-    __syncthreads();
+    if (__syncthreads_or(!ok)) { fail = true; break; }
     if (tid == 0) {   // dS += Qt^T dO
       tc_fence_after();
       for (int s = 0; s < 8; ++s) mma_ss(tb + C_S, desc_mn(sbase + R_XQ, s), desc_mn(sbase + R_O, s), id_st, 1);
@@ -202,18 +182,18 @@ __global__ void __launch_bounds__(128, 1) tc_gla_dstates_kernel(const __grid_con
     if (__syncthreads_or(!ok)) { fail = true; break; }
     tc_fence_after();
     if (tid == 0 && c > 0) loads(c - 1);
-    {   // dS_prev = diag(exp r) (dS + Qt^T dO)
+    {   // dS_prev = diag(exp r) (dS + Qt^T dO), column half per group
       const float dec = s_dec[row];
-      for (int ch = 0; ch < 8; ++ch) {
+      for (int ch = 4 * wg; ch < 4 * wg + 4; ++ch) {
         float v[16];
-        tmem_ld16(tb + lane_off + C_S + ch * 16, v);
+        tmem_ld16(tl + C_S + ch * 16, v);
         uint32_t r[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(v[u] * dec);
-        tmem_st8(tb + lane_off + C_S + ch * 16, r);
+        tmem_st8(tl + C_S + ch * 16, r);
 #pragma unroll
         for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(v[8 + u] * dec);
-        tmem_st8(tb + lane_off + C_S + ch * 16 + 8, r);
+        tmem_st8(tl + C_S + ch * 16 + 8, r);
       }
       tmem_st_wait();
     }
@@ -223,9 +203,9 @@ __global__ void __launch_bounds__(128, 1) tc_gla_dstates_kernel(const __grid_con
   if (!fail && p.dstate_in) {
     tc_fence_after();
     float *dst = p.dstate_in + ((size_t)bh * D + row) * D;
-    for (int ch = 0; ch < 4; ++ch) {
+    for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
       float v[32];
-      tmem_ld32(tb + lane_off + C_S + ch * 32, v);
+      tmem_ld32(tl + C_S + ch * 32, v);
 #pragma unroll
       for (int u = 0; u < 32; u += 4)
         *reinterpret_cast<float4 *>(dst + ch * 32 + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
@@ -532,7 +512,7 @@ cudaError_t launch_tc_gla_bwd(const TcGlaBwdArgs &a, int stage, cudaStream_t s) 
     p.inv_tau = a.inv_tau;
     cudaError_t e = cudaFuncSetAttribute(tc_gla_dstates_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DS_SMEM);
     if (e != cudaSuccess) return e;
-    tc_gla_dstates_kernel<<<a.BH, 128, DS_SMEM, s>>>(p);
+    tc_gla_dstates_kernel<<<a.BH, NT_DS, DS_SMEM, s>>>(p);
     return cudaGetLastError();
   }
   if (stage == 1) {   // per-tile gradients

@@ -63,10 +63,18 @@ __device__ __forceinline__ void setup_cta(uint32_t *tmem_slot, uint64_t *bars, i
 }
 
 // ------------------------------------------------------------- dq pass ----
-__global__ void __launch_bounds__(128, 1) tc_swa_bwd_q_kernel(const __grid_constant__ QParams p) {
+// Two warpgroups (256 threads): thread = query row `row` of its group.  The
+// groups split the band's logit chunks (alternate chunks), the columns of O'
+// and dq', and the meta dot products (group 0 q . mk, group 1 dO . mv);
+// row sums and maxima meet in shared memory.
+constexpr int NT_Q = 256;
+__global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_constant__ QParams p) {
   extern __shared__ unsigned char smraw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
-  __shared__ float s_mk[MAXM][D], s_mv[MAXM][D];
+  __shared__ __align__(16) float s_mk[MAXM][D];
+  __shared__ __align__(16) float s_mv[MAXM][D];
+  __shared__ float s_x[MAXM][T];        // dO . mv_m per row, later the meta dS per row
+  __shared__ float s_pmax[2][T], s_psum[2][T];
   __shared__ float s_red[4];
   __shared__ uint64_t bars[5];
   __shared__ uint32_t s_tmem;
@@ -76,22 +84,23 @@ __global__ void __launch_bounds__(128, 1) tc_swa_bwd_q_kernel(const __grid_const
   // dS [384,512), dq' [128,256)
   constexpr uint32_t C_L = 0, C_P = 0, C_O = 256, C_DP = 128, C_DS = 384, C_DQ = 128;
 
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, row = tid;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wg = tid >> 7, row = tid & 127;
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
   const int bh = blockIdx.y, h = bh % p.H, t0 = blockIdx.x * T, tq = t0 + row;
   const bool qvalid = tq < p.L;
   const float alpha = p.alpha ? p.alpha[h] : 1.f;
   const uint32_t sbase = smem_u32(sm);
   uint64_t *bar_tma = &bars[0], *bar_m = &bars[1];
   setup_cta(&s_tmem, bars, 5, tid);
-  for (int e = tid; e < p.M * D; e += 128) {
-    s_mk[e / D][e % D] = p.meta_k[(size_t)h * p.M * D + e];
-    s_mv[e / D][e % D] = p.meta_v ? p.meta_v[(size_t)h * p.M * D + e] : 0.f;
+  for (int e = tid; e < MAXM * D; e += NT_Q) {
+    const int m = e / D;
+    s_mk[m][e % D] = m < p.M ? p.meta_k[(size_t)h * p.M * D + e] : 0.f;
+    s_mv[m][e % D] = (m < p.M && p.meta_v) ? p.meta_v[(size_t)h * p.M * D + e] : 0.f;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tb = s_tmem;
+  const uint32_t tb = s_tmem, tl = tb + lane_off;
   if (tid == 0) {
     mbar_expect_tx(bar_tma, 6 * TILE);
     for (int r = 0; r < 2; ++r) {
@@ -113,70 +122,136 @@ __global__ void __launch_bounds__(128, 1) tc_swa_bwd_q_kernel(const __grid_const
     tc_fence_after();
     for (int s = 0; s < 8; ++s) mma_ss(tb + C_L, desc_k(sbase + R_Q, s), desc_k(sbase + R_KP, s), id_kk, s > 0);
     for (int s = 0; s < 8; ++s) mma_ss(tb + C_L + 128, desc_k(sbase + R_Q, s), desc_k(sbase + R_K, s), id_kk, s > 0);
-    mma_commit(&bars[1]);
+    mma_commit(bar_m);
   }
   {
-    // meta logits on the CUDA cores while the MMAs run
+    // meta dot products on the CUDA cores while the MMAs run: group 0
+    // q . mk_m (kept in registers), group 1 dO . mv_m (to shared memory);
+    // four meta tokens per pass, passes beyond M skipped
     float ml[MAXM], em[MAXM], dom[MAXM];
 #pragma unroll
-    for (int m = 0; m < MAXM; ++m) { ml[m] = 0.f; dom[m] = 0.f; }
-    for (int ch = 0; ch < 16; ++ch) {
-      float q8[8], o8[8];
-      unpack8(*chunk_ptr(sm, R_Q, row, ch), q8);
-      unpack8(*chunk_ptr(sm, R_O, row, ch), o8);
+    for (int m = 0; m < MAXM; ++m) { ml[m] = 0.f; em[m] = 0.f; dom[m] = 0.f; }
+    {
+      const uint32_t reg = wg == 0 ? R_Q : R_O;
+      const float(*W)[D] = wg == 0 ? s_mk : s_mv;
 #pragma unroll
-      for (int m = 0; m < MAXM; ++m) {
-        if (m < p.M) {
+      for (int g = 0; g < MAXM / 4; ++g) {
+        if (4 * g < p.M) {
+          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+          for (int ch = 0; ch < 16; ++ch) {
+            float x8[8];
+            unpack8(*chunk_ptr(sm, reg, row, ch), x8);
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            ml[m] = fmaf(q8[u], s_mk[m][ch * 8 + u], ml[m]);
-            dom[m] = fmaf(o8[u], s_mv[m][ch * 8 + u], dom[m]);
+            for (int k = 0; k < 4; ++k) {
+              const float4 a = *reinterpret_cast<const float4 *>(&W[4 * g + k][ch * 8]);
+              const float4 b = *reinterpret_cast<const float4 *>(&W[4 * g + k][ch * 8 + 4]);
+              acc[2 * k] = fmaf(x8[0], a.x, fmaf(x8[1], a.y, fmaf(x8[2], a.z, fmaf(x8[3], a.w, acc[2 * k]))));
+              acc[2 * k + 1] = fmaf(x8[4], b.x, fmaf(x8[5], b.y, fmaf(x8[6], b.z, fmaf(x8[7], b.w, acc[2 * k + 1]))));
+            }
           }
+#pragma unroll
+          for (int k = 0; k < 4; ++k) ml[4 * g + k] = acc[2 * k] + acc[2 * k + 1];
         }
       }
-    }
-    float mx = kNegBig;
+      if (wg == 1)
 #pragma unroll
-    for (int m = 0; m < MAXM; ++m)
-      if (m < p.M) { ml[m] *= p.scale; mx = fmaxf(mx, ml[m]); }
+        for (int m = 0; m < MAXM; ++m)
+          if (m < p.M) s_x[m][row] = ml[m];
+    }
     ok = mbar_wait(bar_m, 0, p.status, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) goto done;
     tc_fence_after();
-
-    // 2. softmax: max, then exp and sum with P^ = exp(l - max) packed over L
-    const int jlo = max(tq - p.window + 1, 0);
-    for (int ch = 0; ch < 8; ++ch) {
-      float v[32];
-      tmem_ld32(tb + lane_off + C_L + ch * 32, v);
+    float mx = kNegBig;
+    if (wg == 0) {
 #pragma unroll
-      for (int u = 0; u < 32; ++u) {
-        const int j = t0 - T + ch * 32 + u;
-        if (j >= jlo && j <= tq) mx = fmaxf(mx, v[u] * p.scale);
-      }
+      for (int m = 0; m < MAXM; ++m)
+        if (m < p.M) {
+          dom[m] = s_x[m][row];
+          ml[m] *= p.scale;
+          mx = fmaxf(mx, ml[m]);
+        }
     }
-    float lsum = 0.f;
-    for (int ch = 0; ch < 8; ++ch) {
+
+    // 2. softmax over the band (see the forward): logit column cl holds key
+    //    t0 - T + cl; warp w4 visits chunks ch_lo .. ch_hi, group wg the
+    //    chunks ch_lo + wg, ch_lo + wg + 2, ...
+    const int w4 = warp & 3, cbase = t0 - T;
+    const int lo_c = max(tq - p.window + 1, 0) - cbase, hi_c = tq - cbase;
+    int ch_lo = (32 * w4 + T + 1 - p.window) >> 5;
+    if (cbase < 0) ch_lo = max(ch_lo, 4);
+    const int ch_hi = w4 + 4;
+    const int in_lo = 32 * w4 + 31 + T + 1 - p.window;
+    for (int ch = ch_lo + wg; ch <= ch_hi; ch += 2) {
       float v[32];
-      tmem_ld32(tb + lane_off + C_L + ch * 32, v);
-      uint32_t pk[16];
-      float part = 0.f;
+      tmem_ld32(tl + C_L + ch * 32, v);
+      float m4[4] = {kNegBig, kNegBig, kNegBig, kNegBig};
+      if (32 * ch >= in_lo && 32 * ch + 31 <= 32 * w4 + T && 32 * ch + cbase >= 0) {
+#pragma unroll
+        for (int u = 0; u < 32; ++u) m4[u & 3] = fmaxf(m4[u & 3], v[u]);
+      } else {
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+          const int cl = 32 * ch + u;
+          if (cl >= lo_c && cl <= hi_c) m4[u & 3] = fmaxf(m4[u & 3], v[u]);
+        }
+      }
+      const float cm = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      if (cm > kNegBig) mx = fmaxf(mx, cm * p.scale);
+    }
+    s_pmax[wg][row] = mx;
+    bar_sync(1, NT_Q);
+    mx = fmaxf(s_pmax[0][row], s_pmax[1][row]);
+    //    P^ = exp(l - max) of this group's chunks, held in registers until
+    //    both groups have read their logits (P^ overlays logit chunks 0 .. 3)
+    uint32_t pk[3][16];
+    float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+      const int ch = ch_lo + wg + 2 * k;
+      if (ch > ch_hi) continue;
+      float v[32];
+      tmem_ld32(tl + C_L + ch * 32, v);
+      const bool inner = 32 * ch >= in_lo && 32 * ch + 31 <= 32 * w4 + T && 32 * ch + cbase >= 0;
 #pragma unroll
       for (int u = 0; u < 32; u += 2) {
-        const int j = t0 - T + ch * 32 + u;
-        const float e0 = (j >= jlo && j <= tq) ? __expf(v[u] * p.scale - mx) : 0.f;
-        const float e1 = (j + 1 >= jlo && j + 1 <= tq) ? __expf(v[u + 1] * p.scale - mx) : 0.f;
-        part += e0 + e1;
-        pk[u / 2] = pack_bf16(e0, e1);
+        float e0 = __expf(fmaf(v[u], p.scale, -mx));
+        float e1 = __expf(fmaf(v[u + 1], p.scale, -mx));
+        if (!inner) {
+          const int cl = 32 * ch + u;
+          e0 = (cl >= lo_c && cl <= hi_c) ? e0 : 0.f;
+          e1 = (cl + 1 >= lo_c && cl + 1 <= hi_c) ? e1 : 0.f;
+        }
+        s4[(u >> 1) & 3] += e0 + e1;
+        pk[k][u / 2] = pack_bf16(e0, e1);
       }
-      lsum += part;
-      tmem_st8(tb + lane_off + C_P + ch * 16, pk);
-      tmem_st8(tb + lane_off + C_P + ch * 16 + 8, pk + 8);
     }
+    float psum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+    if (wg == 0) {
 #pragma unroll
-    for (int m = 0; m < MAXM; ++m)
-      if (m < p.M) { em[m] = __expf(ml[m] - mx); lsum += em[m]; } else em[m] = 0.f;
+      for (int m = 0; m < MAXM; ++m)
+        if (m < p.M) { em[m] = __expf(ml[m] - mx); psum += em[m]; }
+    }
+    s_psum[wg][row] = psum;
+    bar_sync(2, NT_Q);
+    const float lsum = s_psum[0][row] + s_psum[1][row];
     const float inv_l = 1.f / lsum;
-    if (qvalid) p.lse[(size_t)bh * p.L + tq] = mx + logf(lsum);
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+      const int ch = ch_lo + wg + 2 * k;
+      if (ch > ch_hi) continue;
+      tmem_st8(tl + C_P + ch * 16, pk[k]);
+      tmem_st8(tl + C_P + ch * 16 + 8, pk[k] + 8);
+    }
+    {
+      uint32_t zero[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+      for (int ch = wg; ch < 8; ch += 2) {
+        if (ch >= ch_lo && ch <= ch_hi) continue;
+        tmem_st8(tl + C_P + ch * 16, zero);
+        tmem_st8(tl + C_P + ch * 16 + 8, zero);
+      }
+    }
+    if (wg == 0 && qvalid) p.lse[(size_t)bh * p.L + tq] = mx + logf(lsum);
     tmem_st_wait();
     tc_fence_before();
     __syncthreads();
@@ -191,27 +266,33 @@ __global__ void __launch_bounds__(128, 1) tc_swa_bwd_q_kernel(const __grid_const
     ok = mbar_wait(&bars[2], 0, p.status, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) goto done;
     tc_fence_after();
-    float dal = 0.f;                      // dout . o_swa for this row
-    for (int ch = 0; ch < 4; ++ch) {
+    float dpart = 0.f;                    // dout . o_swa for this row, column half per group
+    for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
       float v[32];
-      tmem_ld32(tb + lane_off + C_O + ch * 32, v);
+      tmem_ld32(tl + C_O + ch * 32, v);
 #pragma unroll
       for (int c8 = 0; c8 < 4; ++c8) {
         float o8[8];
         unpack8(*chunk_ptr(sm, R_O, row, ch * 4 + c8), o8);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) dal = fmaf(o8[u], v[c8 * 8 + u], dal);
+        for (int u = 0; u < 8; ++u) dpart = fmaf(o8[u], v[c8 * 8 + u], dpart);
       }
     }
+    if (wg == 0) {
 #pragma unroll
-    for (int m = 0; m < MAXM; ++m) dal = fmaf(em[m], dom[m], dal);
-    dal *= inv_l;
+      for (int m = 0; m < MAXM; ++m) dpart = fmaf(em[m], dom[m], dpart);
+    }
+    s_pmax[wg][row] = dpart;
+    bar_sync(3, NT_Q);
+    float dal = (s_pmax[0][row] + s_pmax[1][row]) * inv_l;
     if (!qvalid) dal = 0.f;
     const float Dt = alpha * dal;
-    if (qvalid) p.Dterm[(size_t)bh * p.L + tq] = Dt;
-    if (p.dalpha) {
-      const float w = warp_sum(dal);
-      if (lane == 0) s_red[warp] = w;
+    if (wg == 0) {
+      if (qvalid) p.Dterm[(size_t)bh * p.L + tq] = Dt;
+      if (p.dalpha) {
+        const float w = warp_sum(dal);
+        if (lane == 0) s_red[warp] = w;
+      }
     }
     tc_fence_before();
     __syncthreads();
@@ -228,33 +309,42 @@ __global__ void __launch_bounds__(128, 1) tc_swa_bwd_q_kernel(const __grid_const
     if (__syncthreads_or(!ok)) goto done;
     tc_fence_after();
 
-    // 5. dS = P (alpha dP' - D), P = P^ / l; the meta terms go to memory
-    for (int ch = 0; ch < 8; ++ch) {
-      float dp[32], pp[32];
-      tmem_ld32(tb + lane_off + C_DP + ch * 32, dp);
-      float pk16[16];
-      tmem_ld16(tb + lane_off + C_P + ch * 16, pk16);
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const uint32_t w = __float_as_uint(pk16[u]);
-        pp[2 * u] = __uint_as_float(w << 16);
-        pp[2 * u + 1] = __uint_as_float(w & 0xffff0000u);
-      }
+    // 5. dS = P (alpha dP' - D), P = P^ / l, on the band (zero elsewhere,
+    //    as P^ is); alternate chunks per group; the meta terms go to memory
+    for (int ch = wg; ch < 8; ch += 2) {
       uint32_t ds[16];
+      if (ch >= ch_lo && ch <= ch_hi) {
+        float dp[32], pp[32], pk16[16];
+        tmem_ld32(tl + C_DP + ch * 32, dp);
+        tmem_ld16(tl + C_P + ch * 16, pk16);
 #pragma unroll
-      for (int u = 0; u < 32; u += 2)
-        ds[u / 2] = pack_bf16(pp[u] * inv_l * (alpha * dp[u] - Dt), pp[u + 1] * inv_l * (alpha * dp[u + 1] - Dt));
-      tmem_st8(tb + lane_off + C_DS + ch * 16, ds);
-      tmem_st8(tb + lane_off + C_DS + ch * 16 + 8, ds + 8);
+        for (int u = 0; u < 16; ++u) {
+          const uint32_t w = __float_as_uint(pk16[u]);
+          pp[2 * u] = __uint_as_float(w << 16);
+          pp[2 * u + 1] = __uint_as_float(w & 0xffff0000u);
+        }
+#pragma unroll
+        for (int u = 0; u < 32; u += 2)
+          ds[u / 2] = pack_bf16(pp[u] * inv_l * (alpha * dp[u] - Dt), pp[u + 1] * inv_l * (alpha * dp[u + 1] - Dt));
+      } else {
+#pragma unroll
+        for (int u = 0; u < 16; ++u) ds[u] = 0u;
+      }
+      tmem_st8(tl + C_DS + ch * 16, ds);
+      tmem_st8(tl + C_DS + ch * 16 + 8, ds + 8);
     }
-    float dsm[MAXM];
+    if (wg == 0) {
 #pragma unroll
-    for (int m = 0; m < MAXM; ++m) {
-      const float pm = em[m] * inv_l;
-      dsm[m] = pm * (alpha * dom[m] - Dt);
-      if (m < p.M && qvalid) {
-        p.dsm[((size_t)bh * p.L + tq) * MAXM + m] = dsm[m];
-        p.pm[((size_t)bh * p.L + tq) * MAXM + m] = pm;
+      for (int m = 0; m < MAXM; ++m) {
+        if (m < p.M) {
+          const float pm = em[m] * inv_l;
+          const float dsm = pm * (alpha * dom[m] - Dt);
+          s_x[m][row] = dsm;
+          if (qvalid) {
+            p.dsm[((size_t)bh * p.L + tq) * MAXM + m] = dsm;
+            p.pm[((size_t)bh * p.L + tq) * MAXM + m] = pm;
+          }
+        }
       }
     }
     tmem_st_wait();
@@ -272,14 +362,21 @@ __global__ void __launch_bounds__(128, 1) tc_swa_bwd_q_kernel(const __grid_const
     if (__syncthreads_or(!ok)) goto done;
     tc_fence_after();
     float *dst = p.dq + ((size_t)bh * p.L + (qvalid ? tq : 0)) * D;
-    for (int ch = 0; ch < 4; ++ch) {
+    for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
       float v[32];
-      tmem_ld32(tb + lane_off + C_DQ + ch * 32, v);
+      tmem_ld32(tl + C_DQ + ch * 32, v);
+      for (int m = 0; m < p.M; ++m) {
+        const float w = s_x[m][row];
+        const float4 *mk = reinterpret_cast<const float4 *>(&s_mk[m][ch * 32]);
 #pragma unroll
-      for (int m = 0; m < MAXM; ++m)
-        if (m < p.M)
-#pragma unroll
-          for (int u = 0; u < 32; ++u) v[u] = fmaf(dsm[m], s_mk[m][ch * 32 + u], v[u]);
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const float4 x = mk[q4];
+          v[4 * q4] = fmaf(w, x.x, v[4 * q4]);
+          v[4 * q4 + 1] = fmaf(w, x.y, v[4 * q4 + 1]);
+          v[4 * q4 + 2] = fmaf(w, x.z, v[4 * q4 + 2]);
+          v[4 * q4 + 3] = fmaf(w, x.w, v[4 * q4 + 3]);
+        }
+      }
       if (qvalid)
 #pragma unroll
         for (int u = 0; u < 32; u += 4)
@@ -294,7 +391,11 @@ done:
 }
 
 // ------------------------------------------------------------ dk, dv ------
-__global__ void __launch_bounds__(128, 1) tc_swa_bwd_kv_kernel(const __grid_constant__ KVParams p) {
+// Two warpgroups (256 threads): thread = key row `row` of its group; group h
+// forms P and dS for query chunks 2h, 2h + 1 of each query tile and writes
+// columns 64 h .. of dK and dV.
+constexpr int NT_KV = 256;
+__global__ void __launch_bounds__(NT_KV, 1) tc_swa_bwd_kv_kernel(const __grid_constant__ KVParams p) {
   extern __shared__ unsigned char smraw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
   __shared__ float s_lse[2 * T], s_D[2 * T];
@@ -305,13 +406,13 @@ __global__ void __launch_bounds__(128, 1) tc_swa_bwd_kv_kernel(const __grid_cons
   // TMEM: S^T / P [0,128), dP^T / dS [128,256), dV [256,384), dK [384,512)
   constexpr uint32_t C_S = 0, C_P = 0, C_DP = 128, C_DS = 128, C_DV = 256, C_DK = 384;
 
-  const int tid = threadIdx.x, warp = tid >> 5, row = tid;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const int tid = threadIdx.x, warp = tid >> 5, wg = tid >> 7, row = tid & 127;
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
   const int bh = blockIdx.y, h = bh % p.H, j0 = blockIdx.x * T, tk = j0 + row;
   const float alpha = p.alpha ? p.alpha[h] : 1.f;
   const uint32_t sbase = smem_u32(sm);
   setup_cta(&s_tmem, bars, 5, tid);
-  for (int e = tid; e < 2 * T; e += 128) {
+  for (int e = tid; e < 2 * T; e += NT_KV) {
     const int t = j0 + e;
     s_lse[e] = t < p.L ? p.lse[(size_t)bh * p.L + t] : 0.f;
     s_D[e] = t < p.L ? p.Dterm[(size_t)bh * p.L + t] : 0.f;
@@ -319,7 +420,7 @@ __global__ void __launch_bounds__(128, 1) tc_swa_bwd_kv_kernel(const __grid_cons
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tb = s_tmem;
+  const uint32_t tb = s_tmem, tl = tb + lane_off;
   if (tid == 0) {
     mbar_expect_tx(&bars[0], 6 * TILE);
     for (int r = 0; r < 2; ++r) {
@@ -333,6 +434,7 @@ __global__ void __launch_bounds__(128, 1) tc_swa_bwd_kv_kernel(const __grid_cons
   }
   const uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
   const uint32_t id_mn = idesc_bf16(128, 128, 0, 1);
+  const int r0 = 32 * (warp & 3);          // first key row of this warp
   bool ok = mbar_wait(&bars[0], 0, p.status, ST_TIMEOUT);
   if (__syncthreads_or(!ok)) goto done;
   for (int it = 0; it < 2; ++it) {
@@ -347,30 +449,49 @@ __global__ void __launch_bounds__(128, 1) tc_swa_bwd_kv_kernel(const __grid_cons
     ok = mbar_wait(&bars[1 + 2 * it], 0, p.status, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) goto done;
     tc_fence_after();
-    // P = exp(scale s - lse_t), dS = P (alpha dP - D_t) on the band t - w < j <= t
-    for (int ch = 0; ch < 4; ++ch) {
-      float sv[32], dv[32];
-      tmem_ld32(tb + lane_off + C_S + ch * 32, sv);
-      tmem_ld32(tb + lane_off + C_DP + ch * 32, dv);
-      uint32_t pk[16], dk[16];
+    // P = exp(scale s - lse_t), dS = P (alpha dP - D_t) on the band t - w < j <= t.
+    // Query column qc of this tile is token j0 + it T + qc; the warp's keys
+    // j0 + r0 .. j0 + r0 + 31 see columns qc with 0 <= it T + qc - row < w.
+    // Packed results are held until both groups have read their logits
+    // (P and dS overlay the logit columns of the lower chunks).
+    {
+      const int qlo = max(0, r0 - it * T), qhi = min(T - 1, r0 + 31 + p.window - 1 - it * T);
+      uint32_t pk[2][16], dk[2][16];
 #pragma unroll
-      for (int u = 0; u < 32; u += 2) {
-        float pr[2], ds[2];
+      for (int k = 0; k < 2; ++k) {
+        const int ch = 2 * wg + k;
+        if (32 * ch + 31 < qlo || 32 * ch > qhi) {     // no query of this chunk sees the warp's keys
 #pragma unroll
-        for (int w = 0; w < 2; ++w) {
-          const int qi = it * T + ch * 32 + u + w;       // query row within the two tiles
-          const int t = j0 + qi;
-          const bool valid = t < p.L && tk < p.L && t >= tk && t - tk < p.window;
-          pr[w] = valid ? __expf(sv[u + w] * p.scale - s_lse[qi]) : 0.f;
-          ds[w] = pr[w] * (alpha * dv[u + w] - s_D[qi]);
+          for (int u = 0; u < 16; ++u) { pk[k][u] = 0u; dk[k][u] = 0u; }
+          continue;
         }
-        pk[u / 2] = pack_bf16(pr[0], pr[1]);
-        dk[u / 2] = pack_bf16(ds[0], ds[1]);
+        float sv[32], dv[32];
+        tmem_ld32(tl + C_S + ch * 32, sv);
+        tmem_ld32(tl + C_DP + ch * 32, dv);
+#pragma unroll
+        for (int u = 0; u < 32; u += 2) {
+          float pr[2], ds[2];
+#pragma unroll
+          for (int w = 0; w < 2; ++w) {
+            const int qi = it * T + ch * 32 + u + w;       // query row within the two tiles
+            const int t = j0 + qi;
+            const bool valid = t < p.L && tk < p.L && t >= tk && t - tk < p.window;
+            pr[w] = valid ? __expf(sv[u + w] * p.scale - s_lse[qi]) : 0.f;
+            ds[w] = pr[w] * (alpha * dv[u + w] - s_D[qi]);
+          }
+          pk[k][u / 2] = pack_bf16(pr[0], pr[1]);
+          dk[k][u / 2] = pack_bf16(ds[0], ds[1]);
+        }
       }
-      tmem_st8(tb + lane_off + C_P + ch * 16, pk);
-      tmem_st8(tb + lane_off + C_P + ch * 16 + 8, pk + 8);
-      tmem_st8(tb + lane_off + C_DS + ch * 16, dk);
-      tmem_st8(tb + lane_off + C_DS + ch * 16 + 8, dk + 8);
+      bar_sync(1, NT_KV);
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int ch = 2 * wg + k;
+        tmem_st8(tl + C_P + ch * 16, pk[k]);
+        tmem_st8(tl + C_P + ch * 16 + 8, pk[k] + 8);
+        tmem_st8(tl + C_DS + ch * 16, dk[k]);
+        tmem_st8(tl + C_DS + ch * 16 + 8, dk[k] + 8);
+      }
     }
     tmem_st_wait();
     tc_fence_before();
@@ -390,10 +511,10 @@ __global__ void __launch_bounds__(128, 1) tc_swa_bwd_kv_kernel(const __grid_cons
     const bool kvalid = tk < p.L;
     float *dkr = p.dk + ((size_t)bh * p.L + (kvalid ? tk : 0)) * D;
     float *dvr = p.dv + ((size_t)bh * p.L + (kvalid ? tk : 0)) * D;
-    for (int ch = 0; ch < 4; ++ch) {
+    for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
       float a[32], b[32];
-      tmem_ld32(tb + lane_off + C_DK + ch * 32, a);
-      tmem_ld32(tb + lane_off + C_DV + ch * 32, b);
+      tmem_ld32(tl + C_DK + ch * 32, a);
+      tmem_ld32(tl + C_DV + ch * 32, b);
       if (kvalid)
 #pragma unroll
         for (int u = 0; u < 32; u += 4) {
@@ -540,7 +661,7 @@ cudaError_t launch_tc_swa_bwd(const TcSwaBwdArgs &a, int stage, cudaStream_t s) 
     p.scale = a.scale;
     e = cudaFuncSetAttribute(tc_swa_bwd_q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    tc_swa_bwd_q_kernel<<<dim3(ntiles, a.BH), 128, SMEM_BYTES, s>>>(p);
+    tc_swa_bwd_q_kernel<<<dim3(ntiles, a.BH), NT_Q, SMEM_BYTES, s>>>(p);
     return cudaGetLastError();
   }
   KVParams p;
@@ -560,7 +681,7 @@ cudaError_t launch_tc_swa_bwd(const TcSwaBwdArgs &a, int stage, cudaStream_t s) 
   p.scale = a.scale;
   e = cudaFuncSetAttribute(tc_swa_bwd_kv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  tc_swa_bwd_kv_kernel<<<dim3(ntiles, a.BH), 128, SMEM_BYTES, s>>>(p);
+  tc_swa_bwd_kv_kernel<<<dim3(ntiles, a.BH), NT_KV, SMEM_BYTES, s>>>(p);
   return cudaGetLastError();
 }
 
