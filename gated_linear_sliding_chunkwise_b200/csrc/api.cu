@@ -430,7 +430,17 @@ lizard_status lizard_decode_step(const lizard_decode_args *a, lizard_stream_t st
                    a->H, a->window, a->M, 1.f / a->gate_temp,
                    a->softmax_scale > 0.f ? a->softmax_scale : 1.f / sqrtf((float)a->dk)};
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  return cuda_status(lz::launch_decode(d, a->B, a->dk, a->dtype == LIZARD_BF16, a->pos, s));
+  const bool bf16 = a->dtype == LIZARD_BF16;
+  if (lz::decode_stream_supported(a->dk, bf16, a->window, a->M))
+    return cuda_status(lz::launch_decode_stream(d, a->B, a->pos, s));
+  return cuda_status(lz::launch_decode(d, a->B, a->dk, bf16, a->pos, s));
+}
+
+lizard_status lizard_decode_status(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return LIZARD_ERR_CUDA;
+  const int v = lz::decode_stream_status_take();
+  if (v < 0) return LIZARD_ERR_CUDA;
+  return (v & 1) ? LIZARD_ERR_TIMEOUT : LIZARD_OK;
 }
 
 lizard_status lizard_workspace_status(void *workspace, lizard_stream_t stream) {

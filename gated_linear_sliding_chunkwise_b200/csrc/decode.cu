@@ -21,6 +21,11 @@ namespace lz {
 
 constexpr int kDecWB = 128;   // window slots staged in shared memory per block
 
+__global__ void advance_pos_kernel(int64_t *pos, int B) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < B) pos[b] += 1;
+}
+
 LZ_DEV void cp_async16(void *smem, const void *gmem) {
   const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem) : "memory");
@@ -324,9 +329,461 @@ __global__ void __launch_bounds__(256, 2) decode_kernel(DecodeArgs p) {
   }
 }
 
-__global__ void advance_pos_kernel(int64_t *pos, int B) {
-  const int b = blockIdx.x * blockDim.x + threadIdx.x;
-  if (b < B) pos[b] += 1;
+
+// ------------------------------------------------------------------------
+// Streaming decode (bf16, d = 128, window <= 128, M <= 16): a persistent
+// kernel, one CTA per SM.  The (batch, head) pairs are taken in head-major
+// order, a contiguous run per CTA, so a CTA keeps the feature-map weights and
+// meta tokens of its current head in shared memory.  Each pair is four
+// chunks of at most 32 KB -- the key window (with the new token's q, k, v, g
+// riding along), state rows 0..63, state rows 64..127, the value window --
+// that a producer warp copies into a ring of shared-memory slots with bulk
+// copies (cp.async.bulk, completion on an mbarrier), up to kStreamSlots
+// chunks ahead of the consumers, so HBM keeps streaming while the CTA
+// computes.  The updated state goes back with 16-byte stores straight from
+// registers.
+namespace {
+
+constexpr int kStreamSlots = 4;
+constexpr uint32_t kChunkBytes = 32768;
+constexpr int SD = 128, SF = 64;
+constexpr int kMaxRunPairs = 64;                  // pairs whose (n, slot) are precomputed
+constexpr size_t kRingOff = 0;
+constexpr size_t kWOff = kStreamSlots * (size_t)kChunkBytes;   // W_q | W_k, fp32 [128][64] each
+constexpr size_t kTokOff = kWOff + 2 * SD * SF * 4;           // [slot][q, k, v, g][128] bf16
+constexpr size_t kMetaOff = kTokOff + kStreamSlots * 4 * SD * 2;   // meta_k | meta_v, fp32 [M][128]
+
+__device__ uint32_t g_decode_status;   // bit 1: a bounded wait gave up
+
+LZ_DEV uint32_t s_addr(const void *p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
+LZ_DEV void s_mbar_init(uint64_t *bar) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(s_addr(bar)) : "memory");
+}
+LZ_DEV void s_mbar_expect(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(s_addr(bar)), "r"(bytes) : "memory");
+}
+LZ_DEV bool s_mbar_wait(uint64_t *bar, uint32_t parity) {
+  for (uint32_t i = 0; i < (1u << 22); ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(s_addr(bar)), "r"(parity)
+        : "memory");
+    if (ok) return true;
+  }
+  return false;
+}
+LZ_DEV void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(s_addr(dst)),
+      "l"(src), "r"(bytes), "r"(s_addr(bar))
+      : "memory");
+}
+
+struct PairInfo {
+  int bh, h, n, slot;
+};
+
+// Pair k of this CTA's run (head-major order: q -> head q / B, batch q % B).
+LZ_DEV PairInfo pair_info(const DecodeArgs &p, int B, int first, int k, const int *s_n, const int *s_slot) {
+  PairInfo r;
+  const int q = first + k, h = q / B, b = q % B;
+  r.bh = b * p.H + h;
+  r.h = h;
+  if (k < kMaxRunPairs) {
+    r.n = s_n[k];
+    r.slot = s_slot[k];
+  } else {
+    const long long pos = p.pos[b];
+    r.n = (int)(pos + 1 < (long long)p.window ? pos + 1 : p.window);
+    r.slot = (int)(pos % p.window);
+  }
+  return r;
+}
+
+// Thread roles: warps 0..7 consume (256 threads, thread = column group or
+// slot pair as below), warp 8 produces: one lane walks the same chunk
+// sequence, waits until all eight consumer warps have released a slot
+// (`empty` mbarrier, one arrival per warp) and refills it.  The consumers
+// meet on named barrier 1 only where data flows between them.
+constexpr int kConsumers = 256;
+LZ_DEV void s_mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(s_addr(bar)) : "memory");
+}
+LZ_DEV void s_mbar_init_n(uint64_t *bar, uint32_t n) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(s_addr(bar)), "r"(n) : "memory");
+}
+LZ_DEV void consumers_sync() { asm volatile("bar.sync 1, %0;\n" ::"n"(kConsumers) : "memory"); }
+// Barrier over the consumers that also returns whether any of them passed true.
+LZ_DEV bool consumers_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, 1, %2, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"((uint32_t)v), "n"(kConsumers)
+      : "memory");
+  return r != 0;
+}
+
+__global__ void __launch_bounds__(kConsumers + 32, 1) decode_stream_kernel(const __grid_constant__ DecodeArgs p, int B, int run) {
+  extern __shared__ __align__(1024) unsigned char dsm[];
+  unsigned char *ring = dsm + kRingOff;
+  float *Wq = reinterpret_cast<float *>(dsm + kWOff), *Wk = Wq + SD * SF;
+  __nv_bfloat16 *tokring = reinterpret_cast<__nv_bfloat16 *>(dsm + kTokOff);
+  float *mk_s = reinterpret_cast<float *>(dsm + kMetaOff), *mv_s = mk_s + p.M * SD;
+  __shared__ uint64_t full[kStreamSlots], empty[kStreamSlots];
+  __shared__ uint64_t wfull, wempty;
+  __shared__ float xq[SD], xk[SD], xv[SD], gam[SD], phq[SD], phk[SD];
+  __shared__ __align__(16) float zpart[2][8][SF];   // z partials, later the read-out partials [8][128]
+  __shared__ float prob[128 + 16];
+  __shared__ float red[8][SD];
+  __shared__ float s_inv;
+  __shared__ int s_n[kMaxRunPairs], s_slot[kMaxRunPairs];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int BH = B * p.H;
+  const int first = blockIdx.x * run;
+  const int npairs = max(0, min(run, BH - first));
+  const int nchunks = 4 * npairs;
+  for (int k = tid; k < npairs && k < kMaxRunPairs; k += blockDim.x) {
+    const long long pos = p.pos[(first + k) % B];
+    s_n[k] = (int)(pos + 1 < (long long)p.window ? pos + 1 : p.window);
+    s_slot[k] = (int)(pos % p.window);
+  }
+  if (tid == 0) {
+    for (int i = 0; i < kStreamSlots; ++i) {
+      s_mbar_init_n(&full[i], 1);
+      s_mbar_init_n(&empty[i], kConsumers / 32);
+    }
+    s_mbar_init_n(&wfull, 1);
+    s_mbar_init_n(&wempty, kConsumers / 32);
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  __syncthreads();
+
+  if (warp == kConsumers / 32) {
+    // ------------------------------------------------------- producer ---
+    if (lane == 0) {
+      int prev_head = -1, nh = 0;
+      bool ok = true;
+      for (int c = 0; c < nchunks && ok; ++c) {
+        const PairInfo pi = pair_info(p, B, first, c >> 2, s_n, s_slot);
+        const int kind = c & 3, sl = c % kStreamSlots;
+        if (kind == 0 && pi.h != prev_head) {
+          // weights and meta tokens of the next head, once the consumers are
+          // done with the current ones
+          if (nh > 0) ok = s_mbar_wait(&wempty, (uint32_t)(nh - 1) & 1u);
+          if (!ok) break;
+          const uint32_t wb = (p.wq ? SD * SF * 4 : 0) + (p.wk ? SD * SF * 4 : 0);
+          const uint32_t mb = (uint32_t)p.M * SD * 4 * (p.meta_v ? 2 : 1);
+          s_mbar_expect(&wfull, wb + mb);
+          if (p.wq) bulk_load(Wq, p.wq + (size_t)pi.h * SD * SF, SD * SF * 4, &wfull);
+          if (p.wk) bulk_load(Wk, p.wk + (size_t)pi.h * SD * SF, SD * SF * 4, &wfull);
+          if (p.M > 0) bulk_load(mk_s, p.meta_k + (size_t)pi.h * p.M * SD, p.M * SD * 4, &wfull);
+          if (p.M > 0 && p.meta_v) bulk_load(mv_s, p.meta_v + (size_t)pi.h * p.M * SD, p.M * SD * 4, &wfull);
+          prev_head = pi.h;
+          ++nh;
+        }
+        if (c >= kStreamSlots) ok = s_mbar_wait(&empty[sl], (uint32_t)(c / kStreamSlots - 1) & 1u);
+        if (!ok) break;
+        uint64_t *bar = &full[sl];
+        unsigned char *dst = ring + (size_t)sl * kChunkBytes;
+        if (kind == 0 || kind == 3) {
+          const uint32_t bytes = (uint32_t)pi.n * SD * 2;
+          const __nv_bfloat16 *src = static_cast<const __nv_bfloat16 *>(kind == 0 ? p.k_cache : p.v_cache) +
+                                     (size_t)pi.bh * p.window * SD;
+          s_mbar_expect(bar, bytes + (kind == 0 ? 4 * SD * 2 : 0));
+          bulk_load(dst, src, bytes, bar);
+          if (kind == 0) {   // the new token's q, k, v, g ride along
+            __nv_bfloat16 *tk = tokring + (size_t)sl * 4 * SD;
+            const void *srcs[4] = {p.q, p.k, p.v, p.g};
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              bulk_load(tk + u * SD, static_cast<const __nv_bfloat16 *>(srcs[u]) + (size_t)pi.bh * SD, SD * 2, bar);
+          }
+        } else {
+          s_mbar_expect(bar, kChunkBytes);
+          bulk_load(dst, p.state + (size_t)pi.bh * SD * SD + (size_t)(kind - 1) * 64 * SD, kChunkBytes, bar);
+        }
+      }
+      if (!ok) atomicOr(&g_decode_status, 1u);
+    }
+    return;
+  }
+
+  // ---------------------------------------------------------- consumers ---
+  const int cg = tid & 31, rg = tid >> 5;   // state: float4 column group, row group (8 rows)
+  const int vg = tid & 15, eg = tid >> 4;   // values: 8 columns, slot group
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  int cur_head = -1, nh = 0;
+  bool failed = false;
+  int c_stop = nchunks;
+  PairInfo pi{0, 0, 0, 0};
+  for (int c = 0; c < nchunks; ++c) {
+    const int kind = c & 3, sl = c % kStreamSlots;
+    const unsigned char *chunk = ring + (size_t)sl * kChunkBytes;
+    bool new_head = false;
+    if (kind == 0) {
+      pi = pair_info(p, B, first, c >> 2, s_n, s_slot);
+      new_head = pi.h != cur_head;
+      acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    bool ok = s_mbar_wait(&full[sl], (uint32_t)(c / kStreamSlots) & 1u);
+    if (new_head) {
+      ok &= s_mbar_wait(&wfull, (uint32_t)nh & 1u);
+      ++nh;
+      cur_head = pi.h;
+    }
+    if (!ok) {
+      atomicOr(&g_decode_status, 1u);
+      failed = true;
+    }
+    // A failed (bounded) wait inside a pair only leaves stale slot data; the
+    // consumers decide together, at the next pair, to stop.
+    if (kind == 0 && consumers_any(failed)) {
+      c_stop = c;
+      break;
+    }
+    const int n = pi.n, slot = pi.slot, h = pi.h, bh = pi.bh;
+    if (kind == 0) {
+      // ---- token vectors and decay (the token rode along with this chunk);
+      //      the vote above also ends the previous pair's read-out
+      const __nv_bfloat16 *tk = tokring + (size_t)sl * 4 * SD;
+      if (tid < SD) {
+        xq[tid] = __bfloat162float(tk[tid]);
+        xk[tid] = __bfloat162float(tk[SD + tid]);
+        xv[tid] = __bfloat162float(tk[2 * SD + tid]);
+        gam[tid] = expf(log_decay(__bfloat162float(tk[3 * SD + tid]), p.inv_tau));
+      }
+      consumers_sync();
+      {   // z = x W from shared memory: thread = (map, 4 features, 16 rows of W)
+        const int map = tid >> 7, r = tid & 127, fg = r & 15, ip = r >> 4;
+        const float *Wm = map == 0 ? Wq : Wk;
+        const float *x = map == 0 ? xq : xk;
+        float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float4 wv = *reinterpret_cast<const float4 *>(Wm + (ip * 16 + i) * SF + fg * 4);
+          const float xi = x[ip * 16 + i];
+          z.x = fmaf(xi, wv.x, z.x);
+          z.y = fmaf(xi, wv.y, z.y);
+          z.z = fmaf(xi, wv.z, z.z);
+          z.w = fmaf(xi, wv.w, z.w);
+        }
+        *reinterpret_cast<float4 *>(&zpart[map][ip][fg * 4]) = z;
+      }
+      // ---- window logits: two threads per slot (64 dimensions each); the
+      //      slot being replaced takes the new key
+      {
+        const int j = tid >> 1, half = tid & 1;
+        float d = 0.f;
+        if (j < n) {
+          const __nv_bfloat16 *kr = reinterpret_cast<const __nv_bfloat16 *>(chunk) + (size_t)j * SD + half * 64;
+          if (j == slot) {
+#pragma unroll 8
+            for (int i = 0; i < 64; ++i) d = fmaf(xq[half * 64 + i], xk[half * 64 + i], d);
+          } else {
+#pragma unroll
+            for (int c0 = 0; c0 < 8; ++c0) {
+              const int cc = (c0 + j) & 7;   // spread a warp's reads over the banks
+              float kv[8];
+              load8(kr + cc * 8, kv);
+#pragma unroll
+              for (int u = 0; u < 8; ++u) d = fmaf(xq[half * 64 + cc * 8 + u], kv[u], d);
+            }
+          }
+        }
+        d += __shfl_xor_sync(0xffffffffu, d, 1);
+        if (j < n && half == 0) prob[j] = d * p.scale;
+      }
+      __syncwarp();
+      if (lane == 0) s_mbar_arrive(&empty[sl]);   // the key window and the token are read
+      consumers_sync();
+      if (warp < 2) {   // feature maps from the z partials
+        const int map = warp;
+        const bool has_w = map == 0 ? p.wq != nullptr : p.wk != nullptr;
+        float *out = map == 0 ? phq : phk;
+        const float *x = map == 0 ? xq : xk;
+        if (!has_w) {
+          for (int i = lane; i < SD; i += 32) out[i] = x[i];
+        } else {
+          float z[2], mx = kNegBig, mn = -kNegBig;
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            float a = 0.f;
+#pragma unroll
+            for (int pp = 0; pp < 8; ++pp) a += zpart[map][pp][lane + 32 * j];
+            z[j] = a;
+            mx = fmaxf(mx, a);
+            mn = fminf(mn, a);
+          }
+          mx = warp_max(mx);
+          mn = -warp_max(-mn);
+          float ep[2], en[2], sp = 0.f, sn = 0.f;
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            ep[j] = expf(z[j] - mx);
+            en[j] = expf(mn - z[j]);
+            sp += ep[j];
+            sn += en[j];
+          }
+          sp = 1.f / warp_sum(sp);
+          sn = 1.f / warp_sum(sn);
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            out[lane + 32 * j] = ep[j] * sp;
+            out[SF + lane + 32 * j] = en[j] * sn;
+          }
+        }
+      } else if (warp == 2) {   // meta logits, then the softmax over n + M
+        for (int m = 0; m < p.M; ++m) {
+          float d = 0.f;
+#pragma unroll
+          for (int i = lane; i < SD; i += 32) d = fmaf(xq[i], mk_s[m * SD + i], d);
+          d = warp_sum(d);
+          if (lane == 0) prob[n + m] = d * p.scale;
+        }
+        __syncwarp();
+        const int ntot = n + p.M;
+        float mx = kNegBig;
+        for (int j = lane; j < ntot; j += 32) mx = fmaxf(mx, prob[j]);
+        mx = warp_max(mx);
+        float sum = 0.f;
+        for (int j = lane; j < ntot; j += 32) {
+          const float e = expf(prob[j] - mx);
+          prob[j] = e;
+          sum += e;
+        }
+        sum = warp_sum(sum);
+        if (lane == 0) s_inv = 1.f / sum;
+      }
+      consumers_sync();   // phi_q, phi_k and the probabilities are ready
+    } else if (kind == 1 || kind == 2) {
+      // ---- state rows (kind - 1) * 64 .. + 63: update, store, read out
+      const float4 v4 = make_float4(xv[cg * 4], xv[cg * 4 + 1], xv[cg * 4 + 2], xv[cg * 4 + 3]);
+      float *S = p.state + (size_t)bh * SD * SD;
+      float4 sv[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) sv[r] = *reinterpret_cast<const float4 *>(chunk + (size_t)(rg * 8 + r) * SD * 4 + cg * 16);
+      __syncwarp();
+      if (lane == 0) s_mbar_arrive(&empty[sl]);
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const int i = (kind - 1) * 64 + rg * 8 + r;
+        const float gi = gam[i], ki = phk[i], qi = phq[i];
+        float4 s = sv[r];
+        s.x = fmaf(gi, s.x, ki * v4.x);
+        s.y = fmaf(gi, s.y, ki * v4.y);
+        s.z = fmaf(gi, s.z, ki * v4.z);
+        s.w = fmaf(gi, s.w, ki * v4.w);
+        *reinterpret_cast<float4 *>(S + (size_t)i * SD + cg * 4) = s;
+        acc.x = fmaf(qi, s.x, acc.x);
+        acc.y = fmaf(qi, s.y, acc.y);
+        acc.z = fmaf(qi, s.z, acc.z);
+        acc.w = fmaf(qi, s.w, acc.w);
+      }
+    } else {
+      // ---- o_swa = sum_j p_j v_j (+ meta values); the replaced slot takes
+      //      the new value; then o = o_gla + alpha o_swa / l
+      float a8[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) a8[u] = 0.f;
+      for (int j = eg; j < n; j += 16) {
+        float vv[8];
+        if (j == slot) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) vv[u] = xv[vg * 8 + u];
+        } else {
+          load8(reinterpret_cast<const __nv_bfloat16 *>(chunk) + (size_t)j * SD + vg * 8, vv);
+        }
+        const float pj = prob[j];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) a8[u] = fmaf(pj, vv[u], a8[u]);
+      }
+      __syncwarp();
+      if (lane == 0) s_mbar_arrive(&empty[sl]);
+      if (p.meta_v)
+        for (int m = eg; m < p.M; m += 16) {
+          const float pj = prob[n + m];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) a8[u] = fmaf(pj, mv_s[m * SD + vg * 8 + u], a8[u]);
+        }
+      __syncwarp();
+      if (lane == 0 && ((c >> 2) + 1 >= npairs || pair_info(p, B, first, (c >> 2) + 1, s_n, s_slot).h != h))
+        s_mbar_arrive(&wempty);   // last pair of this head: its weights and meta tokens are read
+#pragma unroll
+      for (int u = 0; u < 8; ++u) a8[u] += __shfl_xor_sync(0xffffffffu, a8[u], 16);
+      if (lane < 16)
+#pragma unroll
+        for (int u = 0; u < 8; ++u) red[warp][vg * 8 + u] = a8[u];
+      // the read-out partials of the two state chunks, per row group
+      *reinterpret_cast<float4 *>(&zpart[0][0][0] + rg * SD + cg * 4) = acc;
+      consumers_sync();
+      if (tid < SD) {
+        float so = 0.f, sg = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) so += red[w][tid];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) sg += (&zpart[0][0][0])[r * SD + tid];
+        const float alpha = p.alpha ? p.alpha[h] : 1.f;
+        static_cast<__nv_bfloat16 *>(p.o)[(size_t)bh * SD + tid] = __float2bfloat16_rn(sg + alpha * so * s_inv);
+        // the new token enters the ring (both windows were read above); xk
+        // and xv hold it exactly (bf16 -> fp32 -> bf16 is lossless)
+        const size_t cw = ((size_t)bh * p.window + slot) * SD + tid;
+        static_cast<__nv_bfloat16 *>(p.k_cache)[cw] = __float2bfloat16_rn(xk[tid]);
+        static_cast<__nv_bfloat16 *>(p.v_cache)[cw] = __float2bfloat16_rn(xv[tid]);
+      }
+    }
+  }
+  if (c_stop < nchunks && tid == 0) {
+    // stopped after a failed wait: let the copies the producer may still have
+    // in flight (chunks c_stop .. c_stop + slots - 1, and a weight copy) land
+    // before the shared memory goes away; every wait is bounded
+    for (int c = c_stop; c < c_stop + kStreamSlots && c < nchunks; ++c)
+      s_mbar_wait(&full[c % kStreamSlots], (uint32_t)(c / kStreamSlots) & 1u);
+    s_mbar_wait(&wfull, (uint32_t)nh & 1u);
+  }
+}
+
+}  // namespace
+
+bool decode_stream_supported(int D, bool bf16, int window, int M) {
+  return bf16 && D == SD && window <= 128 && M <= 16;
+}
+
+cudaError_t launch_decode_stream(const DecodeArgs &a, int B, int64_t *pos, cudaStream_t s) {
+  const size_t smem = kMetaOff + 2 * (size_t)16 * SD * 4;   // room for M <= 16 meta keys and values
+  static int sms[64] = {};
+  static bool configured[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!configured[dev]) {
+    e = cudaFuncSetAttribute(decode_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  const int BH = B * a.H;
+  const int run = (BH + sms[dev] - 1) / sms[dev];   // pairs per CTA
+  const int grid = (BH + run - 1) / run;
+  decode_stream_kernel<<<grid, kConsumers + 32, smem, s>>>(a, B, run);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  advance_pos_kernel<<<(B + 127) / 128, 128, 0, s>>>(pos, B);
+  return cudaGetLastError();
+}
+
+int decode_stream_status_take() {
+  uint32_t v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_decode_status, sizeof(v)) != cudaSuccess) return -1;
+  if (v) {
+    const uint32_t z = 0;
+    if (cudaMemcpyToSymbol(g_decode_status, &z, sizeof(z)) != cudaSuccess) return -1;
+  }
+  return (int)v;
 }
 
 template <typename T, int D>

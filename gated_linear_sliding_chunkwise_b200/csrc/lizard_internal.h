@@ -138,6 +138,11 @@ int tc_fwd_stage_count(int BH, int L);
 // stage 0: state pass, 1: combine (both only when the sequence is split), 2: full pass
 cudaError_t launch_tc_fwd(const TcFwdArgs &a, int stage, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs &a, int B, int D, bool bf16, int64_t *pos, cudaStream_t s);
+// Persistent streaming decode for bf16, d = 128, window <= 128, M <= 16.
+bool decode_stream_supported(int D, bool bf16, int window, int M);
+cudaError_t launch_decode_stream(const DecodeArgs &a, int B, int64_t *pos, cudaStream_t s);
+// The streaming kernel's timeout flag (bit 1), cleared by reading; -1 on error.
+int decode_stream_status_take();
 
 cudaError_t launch_gla_states(const GlaStatesArgs &a, int BH, int D, bool bf16, cudaStream_t s);
 cudaError_t launch_gla_bwd_simt(const GlaBwdArgs &a, int BH, int D, bool bf16, cudaStream_t s);

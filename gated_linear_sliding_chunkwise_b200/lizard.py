@@ -77,6 +77,8 @@ _lib.lizard_bwd_launch_plan.argtypes = [ctypes.POINTER(BwdArgs), ctypes.POINTER(
 _lib.lizard_bwd_launch_plan.restype = _i32
 _lib.lizard_decode_step.argtypes = [ctypes.POINTER(DecodeArgs), _vp]
 _lib.lizard_decode_step.restype = ctypes.c_int
+_lib.lizard_decode_status.argtypes = []
+_lib.lizard_decode_status.restype = ctypes.c_int
 _lib.lizard_workspace_status.argtypes = [_vp, _vp]
 _lib.lizard_workspace_status.restype = ctypes.c_int
 _lib.lizard_status_string.argtypes = [ctypes.c_int]
@@ -287,3 +289,9 @@ def decode_step(q, k, v, g, state, k_cache, v_cache, pos, *, gate_temp=16.0,
 def workspace_status(workspace, stream=None) -> int:
     """Status word left in a workspace by kernels with bounded waits."""
     return int(_lib.lizard_workspace_status(workspace.data_ptr(), _stream(stream)))
+
+
+def decode_status() -> int:
+    """Timeout flag of the decode steps run on the current device since the
+    last call (OK or ERR_TIMEOUT); reading clears it and synchronises."""
+    return int(_lib.lizard_decode_status())

@@ -215,6 +215,15 @@ typedef struct {
 lizard_status lizard_decode_step(const lizard_decode_args *args, lizard_stream_t stream);
 
 /*
+ * Status of the decode steps run on the current device since the last call:
+ * LIZARD_ERR_TIMEOUT when a step's bounded wait for its own copies gave up
+ * (its outputs are then undefined), else LIZARD_OK; LIZARD_ERR_CUDA when
+ * the flag cannot be read.  Reading clears the flag.  Synchronises the
+ * device.  (Decode has no workspace, so the flag lives in the library.)
+ */
+lizard_status lizard_decode_status(void);
+
+/*
  * Forward for callers that cannot allocate device memory.
  *
  * Some callers have no way to obtain a device workspace: a plug-in living

@@ -53,9 +53,13 @@ def test_decode_full_batch_one_step(lz):
     assert torch.equal(x["pos"].cpu(), torch.from_numpy(want_pos))
 
 
+# bf16 with d = 128, window <= 128 and M <= 16 runs the streaming kernel;
+# the other rows run the general one.
 @pytest.mark.parametrize("dtype,d,window,M,pos0", [
     ("fp32", 64, 16, 4, 0), ("fp32", 128, 128, 0, 3), ("fp32", 64, 5, 16, 1000),
     ("bf16", 128, 128, 4, 127), ("bf16", 64, 33, 2, 32),
+    ("bf16", 128, 100, 0, 3), ("bf16", 128, 5, 16, 1000), ("bf16", 128, 1, 4, 7),
+    ("bf16", 128, 129, 4, 500),
 ])
 def test_decode_small_cases(lz, dtype, d, window, M, pos0):
     w = Workload("dec", B=3, H=2, L=1, d=d, window=window, M=M, dtype=dtype, seed=pos0 + d,
@@ -75,11 +79,11 @@ def test_decode_small_cases(lz, dtype, d, window, M, pos0):
         assert torch.equal(x["pos"].cpu(), torch.from_numpy(want[4]))
 
 
-@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
-def test_decode_replay_equals_forward(lz, dtype):
+@pytest.mark.parametrize("dtype,d", [("fp32", 64), ("bf16", 64), ("bf16", 128)])
+def test_decode_replay_equals_forward(lz, dtype, d):
     """Prefill nothing, decode L tokens one by one: every output equals the
     parallel forward at the same position (GPU vs GPU and vs the oracle)."""
-    B, H, L, d, window, M = 2, 2, 40, 64, 12, 4
+    B, H, L, window, M = 2, 2, 40, 12, 4
     w = Workload("replay", B=B, H=H, L=L, d=d, window=window, M=M, dtype=dtype, seed=77)
     inp = make_inputs(w)
     x = to_device(inp)
@@ -105,3 +109,21 @@ def test_decode_replay_equals_forward(lz, dtype):
     check("forward vs oracle", fwd["o"], want["o"], dtype)
     check("decode state", st["state"], want["state_out"], "fp32" if dtype == "fp32" else dtype)
     assert torch.equal(st["pos"].cpu(), torch.full((B,), L, dtype=torch.int64))
+
+
+def test_decode_streaming_without_meta_values_and_status(lz):
+    """Sink-only meta tokens (no meta values) on the streaming kernel, more
+    (batch, head) pairs than SMs, and the timeout flag stays clear."""
+    w = Workload("dec_sink", B=40, H=8, L=1, d=128, window=64, M=4, dtype="bf16", seed=9,
+                 kind="decode", decode_pos=200)
+    inp = make_inputs(w)
+    inp["meta_v"] = None
+    x = to_device(inp)
+    want = _oracle_step({k_: (v_.cpu() if v_ is not None else None) for k_, v_ in x.items()}, w)
+    o = _gpu_step(lz, x, w)
+    torch.cuda.synchronize()
+    check("o", o, want[0], "bf16")
+    check("state", x["state"], want[1], "fp32")
+    assert torch.equal(x["k_cache"].cpu(), torch.from_numpy(want[2]).to(x["k_cache"].dtype))
+    assert torch.equal(x["v_cache"].cpu(), torch.from_numpy(want[3]).to(x["v_cache"].dtype))
+    assert lz.decode_status() == lz.OK
