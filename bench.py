@@ -102,6 +102,7 @@ def kernel_model(name, w, N, BH):
         "tc_fwd_kernel(state pass)": (3 * Nd * esz * (nseg - 1) / nseg + seg_states,
                                       N * (nseg - 1) / nseg * (2 * d * d + phi / 2)),
         "seg_combine_kernel": (3 * seg_states, 0),
+        "gate_prep_kernel": (Nd * esz * 2 + BH * nt * d * 4, 0),
         "tc_fwd_kernel(state copies)": (3 * Nd * esz + snaps, N * (2 * d * d + phi / 2)),
         "tc_gla_dstates_kernel": (3 * Nd * esz + snaps + BH * d * d * 4, N * (2 * d * d + phi / 2)),
         "tc_gla_bwd_tile_kernel": (5 * Nd * esz + 2 * snaps + 4 * Nd * 4,
@@ -278,7 +279,7 @@ def run_ours(args, rank, world, local):
     dt = per[dom] / 1e3
     ai = dflops / max(dbytes, 1)
     if dom.endswith("_simt") or dom in ("prep_kernel", "swa_bwd_q", "swa_bwd_kv", "finish_bwd",
-                                         "meta_grad_kernel", "gate_grad_kernel"):
+                                         "meta_grad_kernel", "gate_grad_kernel", "gate_prep_kernel"):
         # CUDA-core kernels: fp32 FMA peak from unit counts and clock
         alu_peak = SM_COUNT * FP32_LANES_PER_SM * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
         ridge = alu_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)

@@ -94,7 +94,7 @@ bool bwd_gla_uses_tc(const lizard_fwd_args *a, int impl) {
 
 struct BwdLayout {
   size_t phq, phk, a, sprev, dphq, dphk, da, dv_gla, dq_swa, dk_swa, dv_swa, lse, Dterm, dsm, pm, snap_s,
-      snap_ds, total;
+      snap_ds, e32, gr, total;
 };
 BwdLayout bwd_layout(const lizard_fwd_args *a, int impl) {
   const size_t BH = (size_t)a->B * a->H;
@@ -112,6 +112,8 @@ BwdLayout bwd_layout(const lizard_fwd_args *a, int impl) {
     l.dphk = off; off += nd;
     l.da = off; off += nd;       // dB: gradient of the in-tile cumulative log-decay
     l.dv_gla = off; off += nv;
+    l.e32 = off; off += nd;      // fp32 decay factors E of every tile
+    l.gr = off; off += up(BH * ((a->L + 127) / 128) * a->dk * sizeof(float));   // tiles' log-decays
   } else if (gla_on(a)) {
     l.phq = off; off += nd;
     l.phk = off; off += nd;
@@ -182,6 +184,7 @@ void fwd_plan(const lizard_fwd_args *a, void *ws, cudaStream_t s, Plan &plan) {
                     a->state_in, a->o, gla_on(a) ? a->state_out : nullptr, swa_on(a) ? a->lse : nullptr,
                     static_cast<uint32_t *>(ws), at<void>(ws, lay.phq), BH, a->H, a->L, a->M, a->window,
                     a->branch, 1.f / a->gate_temp, scale_of(a)};
+    if (gla_on(a)) plan.add("gate_prep_kernel", [=] { return lz::launch_tc_fwd(t, 3, s); });
     if (lz::tc_fwd_stage_count(BH, a->L) > 1) {
       plan.add("tc_fwd_kernel(state pass)", [=] { return lz::launch_tc_fwd(t, 0, s); });
       plan.add("seg_combine_kernel", [=] { return lz::launch_tc_fwd(t, 1, s); });
@@ -217,11 +220,15 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan) {
                     a->state_in, nullptr, nullptr, nullptr, static_cast<uint32_t *>(ws), nullptr, BH, a->H,
                     a->L, a->M, a->window, 0, inv_tau, scale_of(a)};
     void *snap_s = at<void>(ws, lay.snap_s);
-    plan.add("tc_fwd_kernel(state copies)", [=] { return lz::launch_tc_state_snapshots(f, snap_s, s); });
+    float *e32 = at<float>(ws, lay.e32), *gr = at<float>(ws, lay.gr);
+    uint32_t *status = static_cast<uint32_t *>(ws);
+    plan.add("gate_prep_kernel",
+             [=] { return lz::launch_gate_prep(a->g, nullptr, e32, gr, status, BH, a->L, inv_tau, s); });
+    plan.add("tc_fwd_kernel(state copies)", [=] { return lz::launch_tc_state_snapshots(f, snap_s, e32, gr, s); });
     lz::TcGlaBwdArgs t{a->q, a->k, a->v, a->g, b->dout, a->fmap_wq, a->fmap_wk, snap_s,
                        at<void>(ws, lay.snap_ds), at<float>(ws, lay.dphq), at<float>(ws, lay.dphk),
                        at<float>(ws, lay.da), at<float>(ws, lay.dv_gla), b->dg, b->dstate_in,
-                       static_cast<uint32_t *>(ws), a->H, BH, a->L, inv_tau};
+                       status, a->H, BH, a->L, inv_tau, e32, gr};
     plan.add("tc_gla_dstates_kernel", [=] { return lz::launch_tc_gla_bwd(t, 0, s); });
     plan.add("tc_gla_bwd_tile_kernel", [=] { return lz::launch_tc_gla_bwd(t, 1, s); });
   } else if (g) {

@@ -99,7 +99,7 @@ struct TcFwdArgs {
   void *o;
   float *state_out, *lse;
   uint32_t *status;   // workspace status word (bit 0 timeout, bit 1 range)
-  void *seg_ws;       // segment states, tc_fwd_workspace_bytes() bytes (may be null when 0)
+  void *seg_ws;       // tc_fwd_workspace_bytes() bytes: segment states, then the gate factors
   int BH, H, L, M, window, branch;
   float inv_tau, scale;
 };
@@ -125,6 +125,8 @@ struct TcGlaBwdArgs {
   uint32_t *status;
   int H, BH, L;
   float inv_tau;
+  const float *e32;             // fp32 [B*H*L][128] decay factors of every tile (launch_gate_prep)
+  const float *gate_r;          // fp32 [B*H][L/128][128] log-decay of every tile
 };
 
 constexpr int kBwdC = 32;   // GLA chunk used by the portable backward
@@ -135,6 +137,7 @@ cudaError_t launch_swa_mix_simt(const SwaMixArgs &a, int BH, int D, bool bf16, c
 bool tc_fwd_supported(int dk, int dv, int window, int M, bool bf16);
 size_t tc_fwd_workspace_bytes(int BH, int L);
 int tc_fwd_stage_count(int BH, int L);
+// stage 3: gate factors of every tile (first, when the GLA branch is on);
 // stage 0: state pass, 1: combine (both only when the sequence is split), 2: full pass
 cudaError_t launch_tc_fwd(const TcFwdArgs &a, int stage, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs &a, int B, int D, bool bf16, int64_t *pos, cudaStream_t s);
@@ -152,7 +155,13 @@ bool tc_swa_bwd_supported(int dk, int dv, int window, int M, bool bf16);
 // stage 0: dq pass, 1: dk/dv pass, 2: meta-token gradients
 cudaError_t launch_tc_swa_bwd(const TcSwaBwdArgs &a, int stage, cudaStream_t s);
 size_t tc_gla_bwd_snapshot_bytes(int BH, int L);
-cudaError_t launch_tc_state_snapshots(const TcFwdArgs &a, void *snap, cudaStream_t s);
+cudaError_t launch_tc_state_snapshots(const TcFwdArgs &a, void *snap, const float *e32, const float *r,
+                                      cudaStream_t s);
+// Decay factors of every 128-token tile (bf16 E16 and/or fp32 E32, [BH][L][128],
+// either may be null) and the tiles' log-decays r [BH][ntiles][128], from bf16
+// gate logits g [BH][L][128]; sets bit 2 of *status when a tile's spread is too wide.
+cudaError_t launch_gate_prep(const void *g, void *E16, float *E32, float *r, uint32_t *status, int BH, int L,
+                             float inv_tau, cudaStream_t s);
 // stage 0: reverse dS pass, 1: per-tile gradients, 2: gate-logit gradient
 cudaError_t launch_tc_gla_bwd(const TcGlaBwdArgs &a, int stage, cudaStream_t s);
 // tensor-core finish: bf16, d = 128, both feature maps present

@@ -190,6 +190,7 @@ __host__ __device__ __forceinline__ uint32_t sw128_offset(int row, int col) {
 // ---------------------------------------------- 128 x 128 bf16 tiles -----
 // A 128-row tile of 128 bf16 columns, as TMA writes it with the 128-byte
 // swizzle: two 16 KB regions of 64 columns, each 1024-byte aligned.
+constexpr int kTileRows = 128;       // tokens per tensor-core tile
 constexpr uint32_t kReg = 16384;
 constexpr uint32_t kTile = 2 * kReg;
 
@@ -249,54 +250,6 @@ __device__ __forceinline__ float feature_half(uint32_t taddr, int half, float *p
     s[f & 3] += ph[f];
   }
   return 1.f / ((s[0] + s[1]) + (s[2] + s[3]));
-}
-
-// In-tile decay factors in fp32, thread = tile row t (128 threads, 4 warps),
-// for the 16 key dimensions 16 c16 .. 16 c16 + 15:
-//   E[u]   = exp(sum_{s > t} -a_s)   (= exp(b_t - r), b the in-tile cumsum)
-//   tot[u] = sum_{all s} -a_s         (= -r)
-// from the bf16 gate logits of a 128 x 128 tile (a_s = logsigmoid(g)/tau,
-// zero for rows at or beyond L).  Suffix sums: a shuffle scan within each
-// warp, then the later warps' totals from shared memory `wtot` [4][16].
-// All 128 threads of the group must call it: it synchronises them twice,
-// through __syncthreads (bar_id 0, a 128-thread CTA) or through named
-// barrier bar_id over 128 threads (one warpgroup of a larger CTA).
-__device__ __forceinline__ void row_decay16(unsigned char *gtile, int row, int c16, bool valid, float inv_tau,
-                                            float (*wtot)[16], float *E, float *tot, int bar_id = 0) {
-  const int lane = row & 31, warp = row >> 5;
-  float na[16], x[16];
-  unpack8(*chunk_ptr(gtile, 0, row, 2 * c16), na);
-  unpack8(*chunk_ptr(gtile, 0, row, 2 * c16 + 1), na + 8);
-#pragma unroll
-  for (int u = 0; u < 16; ++u) {
-    na[u] = valid ? -log_decay_fast(na[u], inv_tau) : 0.f;
-    x[u] = na[u];
-  }
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      const float y = __shfl_down_sync(0xffffffffu, x[u], off);
-      if (lane + off < 32) x[u] += y;
-    }
-  }
-  if (lane == 0)
-#pragma unroll
-    for (int u = 0; u < 16; ++u) wtot[warp][u] = x[u];
-  if (bar_id) bar_sync(bar_id, 128); else __syncthreads();
-#pragma unroll
-  for (int u = 0; u < 16; ++u) {
-    float later = 0.f, all = 0.f;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const float v = wtot[w][u];
-      all += v;
-      if (w > warp) later += v;
-    }
-    E[u] = __expf(x[u] - na[u] + later);
-    tot[u] = all;
-  }
-  if (bar_id) bar_sync(bar_id, 128); else __syncthreads();
 }
 
 }  // namespace tc

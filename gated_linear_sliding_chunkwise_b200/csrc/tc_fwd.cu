@@ -1,24 +1,27 @@
 // Tensor-core (tcgen05 / TMEM / TMA) forward of the Lizard hybrid layer,
 // bf16 activations, dk = dv = 128, window <= 128, M <= 16.
 //
-// One CTA (128 threads, one TMEM lane per thread) walks one (batch, head)
-// sequence in tiles of T = 128 tokens, i.e. two 64-token chunks per tile with
-// the cumulative gate absorbed once per tile.  Per tile:
+// One CTA walks one (batch, head) sequence in tiles of T = 128 tokens, i.e.
+// two 64-token chunks per tile with the cumulative gate absorbed once per
+// tile.  The CTA has two warpgroups (256 threads); warps w and w + 4 address
+// the same 32 TMEM lanes, so thread = tile row (lane) in both groups and the
+// groups split each row's work.  The decay factors of every tile come from
+// a separate, fully parallel pass (gate_prep_kernel):
+//   E_t = exp(sum_{s>t} -a_s) = exp(b_t - r) (bf16) and exp(r) (fp32).
+// Per tile:
 //
-//   TMA     X_q, X_k, V, G (gate logits) of the tile and K of the previous
-//           tile, 128-byte swizzled; later V of the previous tile.
+//   TMA     X_q, X_k, V, E of the tile and K of the previous tile, 128-byte
+//           swizzled; later V of the previous tile.
 //   MMA 1   L  = X_q [K_prev ; X_k]^T            (window logits, 128 x 256)
 //           Zq = X_q W_q, Zk = X_k W_k           (feature-map projections)
-//   gates   thread = key dimension i, tokens in reverse:
-//             acc_t = sum_{s>t} -a_s,  E_t = exp(acc_t) = exp(b_t - r)
-//           written as bf16 over G; exp(r) = exp(-acc_{-1}) decays the state.
-//   rows    thread = token t:
-//             anchor softmax over the 256 logits (band mask) and the M meta
-//             logits -> P^ = exp(l - max), unnormalised, into TMEM;
-//             phi_q, phi_k from Zq, Zk; Qt = phi_q E l/alpha (TMEM),
-//             Kt = phi_k / E (shared memory);
+//   rows    anchor softmax over the band of L (each warp visits only the
+//           <= 5 32-column chunks its rows can see; group 1 takes alternate
+//           chunks, group 0 the others and the M meta logits; maxima and
+//           sums meet in shared memory) -> P^ = exp(l - max) into TMEM;
+//           group h builds half h of phi = [softmax(z), softmax(-z)]:
+//           Qt = phi_q E l/alpha (TMEM), Kt = phi_k / E (shared memory);
 //           thread = key dimension i: S' = diag(exp r) S in TMEM, and its
-//           bf16 copy in shared memory.
+//           bf16 copy in shared memory (column half per group).
 //   MMA 2   A  = Qt Kt^T
 //   rows    A^ = tril(A) (TMEM; l/alpha comes in through Qt)
 //   MMA 3   O  = Qt S' + A^ V + P^ [V_prev ; V];   S = S' + Kt^T V
@@ -32,7 +35,8 @@
 //
 // Long sequences with few (batch, head) pairs are split into segments so
 // that every SM has a sequence slice: a state pass (the same kernel in
-// mode 1: gates, phi_k, state update only) gives each segment's local end
+// mode 1: the decay factors in fp32 by a row-wise suffix scan of the gate
+// logits, phi_k, state update only) gives each segment's local end
 // state and total log-decay, a combine kernel chains them into each
 // segment's start state, and the full pass runs all segments in parallel.
 //
@@ -86,6 +90,8 @@ struct Params {
   float *seg_state;         // mode 1: [BH][nseg][D][D] local end state (zero start)
   float *seg_decay;         // mode 1: [BH][nseg][D] summed log-decay of the segment
   __nv_bfloat16 *snap;      // mode 1 with nseg == 1: [BH][ntiles][D][D] bf16 S' of every tile
+  const float *gate_r;      // [BH][ntiles][D] log-decay r of every tile (gate_prep_kernel)
+  const float *gate_e32;    // mode 1: [BH][L][D] fp32 decay factors E (mode 0 loads bf16 E as the G tiles)
   int H, L, M, window, branch;
   int mode;                 // 0: full forward, 1: state pass
   int nseg, tiles_per_seg;
@@ -95,51 +101,17 @@ struct Params {
 
 __device__ __forceinline__ void issue_tile_loads(const Params &p, unsigned char *sm, uint64_t *bar, int bh,
                                                  int t0, bool full) {
-  mbar_expect_tx(bar, (full ? 5 : 3) * TILE);
+  mbar_expect_tx(bar, (full ? 5 : 2) * TILE);
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
     if (full) {
       tma_load_3d(sm + R_XQ + r * REG, &p.mq, bar, 64 * r, t0, bh);
       tma_load_3d(sm + R_KP + r * REG, &p.mk, bar, 64 * r, t0 - T, bh);
+      tma_load_3d(sm + R_G + r * REG, &p.mg, bar, 64 * r, t0, bh);
     }
     tma_load_3d(sm + R_XK + r * REG, &p.mk, bar, 64 * r, t0, bh);
     tma_load_3d(sm + R_V + r * REG, &p.mv, bar, 64 * r, t0, bh);
-    tma_load_3d(sm + R_G + r * REG, &p.mg, bar, 64 * r, t0, bh);
   }
-}
-
-// Gates, thread = key dimension i: in-tile suffix sums of the log-decay,
-// E_t = exp(sum_{s>t} -a_s) = exp(b_t - r) written as bf16 over the gate
-// logits, exp(r) (the tile's decay) into s_dec[i].  16 tokens per step; the
-// next step's logits are read before this step's factors are written.
-// Returns the largest exponent of E in this dimension (its value at t = 0).
-__device__ __forceinline__ float gates_by_dim(unsigned char *sm, int i, int t0, int L, float inv_tau,
-                                              float *s_dec) {
-  unsigned char *gcol = sm + R_G + (i >> 6) * REG;
-  const int ci = i & 63;
-  float acc = 0.f, spread = 0.f, gn[16];
-#pragma unroll
-  for (int u = 0; u < 16; ++u)
-    gn[u] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(gcol + sw128_offset(T - 16 + u, ci)));
-#pragma unroll 1
-  for (int tb = T - 16; tb >= 0; tb -= 16) {
-    float a[16], pre[16];
-#pragma unroll
-    for (int u = 0; u < 16; ++u) a[u] = (t0 + tb + u < L) ? log_decay_fast(gn[u], inv_tau) : 0.f;
-    if (tb > 0) {
-#pragma unroll
-      for (int u = 0; u < 16; ++u)
-        gn[u] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(gcol + sw128_offset(tb - 16 + u, ci)));
-    }
-#pragma unroll
-    for (int u = 15; u >= 0; --u) { pre[u] = acc; acc -= a[u]; }
-#pragma unroll
-    for (int u = 0; u < 16; ++u)
-      *reinterpret_cast<__nv_bfloat16 *>(gcol + sw128_offset(tb + u, ci)) = __float2bfloat16_rn(__expf(pre[u]));
-    spread = pre[0];
-  }
-  s_dec[i] = __expf(-acc);
-  return spread;
 }
 
 // Qt for dimensions 64 h .. 64 h + 63: phi_q E gscale, bf16 pairs into TMEM.
@@ -161,10 +133,13 @@ __device__ __forceinline__ void qt_half(unsigned char *sm, uint32_t tl, int row,
 
 // Kt for dimensions 64 h .. 64 h + 63: phi_k / E, bf16 into shared memory
 // over X_k.  E comes as bf16 from the gate region (full pass) or as fp32
-// from TMEM (state pass).
-__device__ __forceinline__ void kt_half(unsigned char *sm, uint32_t tl, int row, int h, bool e_in_tmem) {
+// from TMEM (state pass).  Rows past L (where the full pass's E is zero)
+// get Kt = 0.
+__device__ __forceinline__ void kt_half(unsigned char *sm, uint32_t tl, int row, int h, bool e_in_tmem,
+                                        bool valid) {
   float ph[F];
-  const float s = feature_half(tl + C_ZK, h, ph);
+  float s = feature_half(tl + C_ZK, h, ph);   // warp-collective TMEM loads: every lane
+  if (!valid) s = 0.f;
 #pragma unroll
   for (int c16 = 0; c16 < 4; ++c16) {
     float e16[16], k16[16];
@@ -175,16 +150,15 @@ __device__ __forceinline__ void kt_half(unsigned char *sm, uint32_t tl, int row,
       unpack8(*chunk_ptr(sm, R_G, row, 8 * h + 2 * c16 + 1), e16 + 8);
     }
 #pragma unroll
-    for (int u = 0; u < 16; ++u) k16[u] = __fdividef(ph[16 * c16 + u] * s, e16[u]);
+    for (int u = 0; u < 16; ++u) k16[u] = valid ? __fdividef(ph[16 * c16 + u] * s, e16[u]) : 0.f;
     *chunk_ptr(sm, R_XK, row, 8 * h + 2 * c16) = pack8(k16);
     *chunk_ptr(sm, R_XK, row, 8 * h + 2 * c16 + 1) = pack8(k16 + 8);
   }
 }
 
-// Named barriers between the two warpgroups (id 0 is __syncthreads).
-constexpr int BAR_E = 1;       // gate factors E written (group 1 -> group 0)
-constexpr int BAR_G = 2;       // row scales of the anchor softmax written (group 0 -> group 1)
-constexpr int BAR_DECAY = 3;   // + group: the row-wise decay scan inside one group
+// Named barriers (id 0 is __syncthreads).
+constexpr int BAR_A = 1;       // both groups' row maxima written
+constexpr int BAR_B = 2;       // both groups' row sums written, all logits read
 
 __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_constant__ Params p) {
   extern __shared__ unsigned char smraw[];
@@ -193,8 +167,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
   __shared__ __align__(16) float s_mv[MAXM][D];
   __shared__ float s_ml[MAXM][T];     // meta logits, then their mixing weights, per row
   __shared__ float s_dec[D];
-  __shared__ float s_gscale[T], s_oscale[T];
-  __shared__ float s_wtot[2][4][16];
+  __shared__ float s_oscale[T];
+  __shared__ float s_pmax[2][T], s_psum[2][T];   // per-group row maxima and sums of the softmax
   __shared__ uint64_t bar_tma, bar_vp, bar_m1, bar_m2, bar_m3;
   __shared__ uint32_t s_tmem;
   __shared__ int s_fail;
@@ -268,7 +242,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
   const int cbeg = seg * p.tiles_per_seg;
   const int cend = min(ntiles_all, cbeg + p.tiles_per_seg);
   uint32_t *err = p.status;
-  float tot_decay = 0.f;                      // state pass: summed log-decay of the dimension this thread owns
+  float tot_decay = 0.f;                      // state pass: summed log-decay of dimension `row` (group 0)
   if (tid == 0 && cbeg < cend) issue_tile_loads(p, sm, &bar_tma, bh, cbeg * T, full);
   const uint32_t id_128 = idesc_bf16(128, 128, 0, 0);
   const uint32_t id_z = idesc_bf16(128, 64, 0, 1);
@@ -297,55 +271,55 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       mma_commit(&bar_m1);
     }
 
-    if (full && wg == 1) {
-      // ------------------------------- group 1: gates, then phi half 1 ---
-      const float spread = gates_by_dim(sm, row, t0, p.L, p.inv_tau, s_dec);
-      if (spread > kMaxSpread && gla) atomicOr(err, ST_RANGE);
-      bar_arrive(BAR_E, NTHREADS);
+    if (full) {
+      // ---- full pass: the anchor softmax split between the groups (group 1
+      //      the band chunks ch_lo, ch_lo + 2, ..., group 0 the others and
+      //      the meta logits), then one half of phi_q, phi_k per group
       ok &= mbar_wait(&bar_m1, par, err, ST_TIMEOUT);
       tc_fence_after();
-      kt_half(sm, tl, row, 1, false);
-      bar_sync(BAR_G, NTHREADS);
-      qt_half(sm, tl, row, 1, s_gscale[row]);
-    } else if (full) {
-      // ---------------------- group 0: anchor softmax, then phi half 0 ---
-      ok &= mbar_wait(&bar_m1, par, err, ST_TIMEOUT);
-      tc_fence_after();
+      if (wg == 1 && gla) s_dec[row] = __expf(p.gate_r[((size_t)bh * ntiles_all + c) * D + row]);   // exp(r)
       float lsum = 1.f, mx = 0.f;                 // row normaliser and max (scaled logits)
+      // Logit column cl holds key t0 - T + cl.  Row r sees columns
+      // [r + T + 1 - window, r + T] (and keys >= 0), so warp w4 only visits
+      // 32-column chunks w4 + (T + 1 - window) / 32 .. w4 + 4, and only the
+      // first and last of those need the band mask.
+      const int w4 = warp & 3;
+      const int cbase = t0 - T;
+      const int lo_c = max(tq - p.window + 1, 0) - cbase, hi_c = tq - cbase;
+      int ch_lo = (32 * w4 + T + 1 - p.window) >> 5;
+      if (cbase < 0) ch_lo = max(ch_lo, 4);
+      const int ch_hi = w4 + 4;
+      const int in_lo = 32 * w4 + 31 + T + 1 - p.window;   // interior chunk: 32 ch >= in_lo
+      const int ch_first = ch_lo + 1 - wg;                 // this group's first chunk
+      uint32_t pk[3][16];
       if (swa) {
-        // meta logits q . mk_m (scaled) into s_ml, four meta tokens per pass
-        for (int m0 = 0; m0 < p.M; m0 += 4) {
-          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        float pmax = kNegBig;
+        if (wg == 0) {
+          // meta logits q . mk_m (scaled) into s_ml, four meta tokens per pass
+          for (int m0 = 0; m0 < p.M; m0 += 4) {
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll 4
-          for (int ch = 0; ch < 16; ++ch) {
-            float q8[8];
-            unpack8(*chunk_ptr(sm, R_XQ, row, ch), q8);
+            for (int ch = 0; ch < 16; ++ch) {
+              float q8[8];
+              unpack8(*chunk_ptr(sm, R_XQ, row, ch), q8);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const float4 a = *reinterpret_cast<const float4 *>(&s_mk[m0 + k][ch * 8]);
-              const float4 b = *reinterpret_cast<const float4 *>(&s_mk[m0 + k][ch * 8 + 4]);
-              acc[2 * k] = fmaf(q8[0], a.x, fmaf(q8[1], a.y, fmaf(q8[2], a.z, fmaf(q8[3], a.w, acc[2 * k]))));
-              acc[2 * k + 1] = fmaf(q8[4], b.x, fmaf(q8[5], b.y, fmaf(q8[6], b.z, fmaf(q8[7], b.w, acc[2 * k + 1]))));
+              for (int k = 0; k < 4; ++k) {
+                const float4 a = *reinterpret_cast<const float4 *>(&s_mk[m0 + k][ch * 8]);
+                const float4 b = *reinterpret_cast<const float4 *>(&s_mk[m0 + k][ch * 8 + 4]);
+                acc[2 * k] = fmaf(q8[0], a.x, fmaf(q8[1], a.y, fmaf(q8[2], a.z, fmaf(q8[3], a.w, acc[2 * k]))));
+                acc[2 * k + 1] = fmaf(q8[4], b.x, fmaf(q8[5], b.y, fmaf(q8[6], b.z, fmaf(q8[7], b.w, acc[2 * k + 1]))));
+              }
             }
-          }
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            if (m0 + k < p.M) s_ml[m0 + k][row] = (acc[2 * k] + acc[2 * k + 1]) * p.scale;
+            for (int k = 0; k < 4; ++k)
+              if (m0 + k < p.M) {
+                const float l = (acc[2 * k] + acc[2 * k + 1]) * p.scale;
+                s_ml[m0 + k][row] = l;
+                pmax = fmaxf(pmax, l);
+              }
+          }
         }
-        mx = kNegBig;
-        for (int m = 0; m < p.M; ++m) mx = fmaxf(mx, s_ml[m][row]);
-        // Logit column cl holds key t0 - T + cl.  Row r sees columns
-        // [r + T + 1 - window, r + T] (and keys >= 0), so warp w4 only
-        // visits 32-column chunks w4 + (T + 1 - window) / 32 .. w4 + 4, and
-        // only the first and last of those need the band mask.
-        const int w4 = warp & 3;
-        const int cbase = t0 - T;
-        const int lo_c = max(tq - p.window + 1, 0) - cbase, hi_c = tq - cbase;
-        int ch_lo = (32 * w4 + T + 1 - p.window) >> 5;
-        if (cbase < 0) ch_lo = max(ch_lo, 4);
-        const int ch_hi = w4 + 4;
-        const int in_lo = 32 * w4 + 31 + T + 1 - p.window;   // interior chunk: 32 ch >= in_lo
-        for (int ch = ch_lo; ch <= ch_hi; ++ch) {
+        for (int ch = ch_first; ch <= ch_hi; ch += 2) {
           float v[32];
           tmem_ld32(tl + C_L + ch * 32, v);
           float m4[4] = {kNegBig, kNegBig, kNegBig, kNegBig};
@@ -360,14 +334,23 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
             }
           }
           const float cm = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-          if (cm > kNegBig) mx = fmaxf(mx, cm * p.scale);
+          if (cm > kNegBig) pmax = fmaxf(pmax, cm * p.scale);
         }
+        s_pmax[wg][row] = pmax;
+      }
+      bar_sync(BAR_A, NTHREADS);
+      if (swa) {
+        mx = fmaxf(s_pmax[0][row], s_pmax[1][row]);
+        // P^ = exp(l - max), packed and held until both groups have read
+        // their logits (P^ column 16 ch overlays logit chunk ch / 2)
         float s4[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int ch = ch_lo; ch <= ch_hi; ++ch) {
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+          const int ch = ch_first + 2 * k;
+          if (ch > ch_hi) continue;
           float v[32];
           tmem_ld32(tl + C_L + ch * 32, v);
           const bool inner = 32 * ch >= in_lo && 32 * ch + 31 <= 32 * w4 + T && 32 * ch + cbase >= 0;
-          uint32_t pk[16];
 #pragma unroll
           for (int u = 0; u < 32; u += 2) {
             float e0 = __expf(fmaf(v[u], p.scale, -mx));
@@ -378,69 +361,75 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
               e1 = (cl + 1 >= lo_c && cl + 1 <= hi_c) ? e1 : 0.f;
             }
             s4[(u >> 1) & 3] += e0 + e1;
-            pk[u / 2] = alpha != 0.f ? pack_bf16(e0, e1) : 0u;
-          }
-          tmem_st8(tl + C_P + ch * 16, pk);
-          tmem_st8(tl + C_P + ch * 16 + 8, pk + 8);
-        }
-        // chunks outside the band: P = 0 (written after the band's logits
-        // were read, since P column 16 ch overlays logit chunk ch / 2)
-        {
-          uint32_t zero[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-          for (int ch = 0; ch < 8; ++ch) {
-            if (ch >= ch_lo && ch <= ch_hi) continue;
-            tmem_st8(tl + C_P + ch * 16, zero);
-            tmem_st8(tl + C_P + ch * 16 + 8, zero);
+            pk[k][u / 2] = alpha != 0.f ? pack_bf16(e0, e1) : 0u;
           }
         }
-        float sm_meta = 0.f;
-        for (int m = 0; m < p.M; ++m) {
-          const float e = __expf(s_ml[m][row] - mx);
-          sm_meta += e;
-          s_ml[m][row] = e;
-        }
-        lsum = ((s4[0] + s4[1]) + (s4[2] + s4[3])) + sm_meta;
+        float psum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+        if (wg == 0)
+          for (int m = 0; m < p.M; ++m) {
+            const float e = __expf(s_ml[m][row] - mx);
+            psum += e;
+            s_ml[m][row] = e;
+          }
+        s_psum[wg][row] = psum;
+      }
+      bar_sync(BAR_B, NTHREADS);
+      if (swa) {
+        lsum = s_psum[0][row] + s_psum[1][row];
         if (!qvalid) lsum = 1.f;
-        if (qvalid && p.lse) p.lse[(size_t)bh * p.L + tq] = mx + logf(lsum);
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+          const int ch = ch_first + 2 * k;
+          if (ch > ch_hi) continue;
+          tmem_st8(tl + C_P + ch * 16, pk[k]);
+          tmem_st8(tl + C_P + ch * 16 + 8, pk[k] + 8);
+        }
+        uint32_t zero[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+        for (int ch = wg; ch < 8; ch += 2) {   // chunks outside the band: P = 0
+          if (ch >= ch_lo && ch <= ch_hi) continue;
+          tmem_st8(tl + C_P + ch * 16, zero);
+          tmem_st8(tl + C_P + ch * 16 + 8, zero);
+        }
+        if (wg == 0 && qvalid && p.lse) p.lse[(size_t)bh * p.L + tq] = mx + logf(lsum);
       }
       // GLA operands carry l/alpha so that one accumulator holds both terms
       const bool mixed = swa && alpha != 0.f;
       const float gscale = mixed ? lsum / alpha : 1.f;
-      s_gscale[row] = gscale;
-      s_oscale[row] = mixed ? alpha / lsum : 1.f;
-      if (swa) {
-        const float mscale = mixed ? alpha / lsum : 0.f;   // meta-value weight per exp
-        for (int m = 0; m < p.M; ++m) s_ml[m][row] *= mscale;
+      if (wg == 0) {
+        s_oscale[row] = mixed ? alpha / lsum : 1.f;
+        if (swa) {
+          const float mscale = mixed ? alpha / lsum : 0.f;   // meta-value weight per exp
+          for (int m = 0; m < p.M; ++m) s_ml[m][row] *= mscale;
+        }
       }
-      bar_arrive(BAR_G, NTHREADS);
-      bar_sync(BAR_E, NTHREADS);
-      qt_half(sm, tl, row, 0, gscale);
-      kt_half(sm, tl, row, 0, false);
+      qt_half(sm, tl, row, wg, gscale);
+      kt_half(sm, tl, row, wg, false, qvalid);
     } else {
-      // ------------- state pass: fp32 decay factors, phi_k half per group ---
-      for (int c16 = 4 * wg; c16 < 4 * wg + 4; ++c16) {
-        float E[16], tot[16];
-        row_decay16(sm + R_G, row, c16, qvalid, p.inv_tau, s_wtot[wg], E, tot, BAR_DECAY + wg);
-        uint32_t r[8];
+      // ------ state pass: fp32 decay factors of this row's dimension half
+      //        (from gate_prep_kernel) into TMEM, phi_k half per group ---
+      {
+        const float *er = p.gate_e32 + ((size_t)bh * p.L + (qvalid ? tq : 0)) * D + 64 * wg;
+        float4 e[16];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(E[u]);
-        tmem_st8(tl + C_L + c16 * 16, r);
+        for (int u = 0; u < 16; ++u)
+          e[u] = qvalid ? *reinterpret_cast<const float4 *>(er + 4 * u) : make_float4(1.f, 1.f, 1.f, 1.f);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(E[8 + u]);
-        tmem_st8(tl + C_L + c16 * 16 + 8, r);
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          if (row == c16 * 16 + u) {   // the dimension this thread owns
-            s_dec[row] = __expf(-tot[u]);   // exp(r)
-            tot_decay -= tot[u];             // r, the tile's log-decay
-          }
-          if (row == 0 && E[u] > kMaxSpreadExp && gla) atomicOr(err, ST_RANGE);
+        for (int u = 0; u < 8; ++u) {
+          const uint32_t r8[8] = {__float_as_uint(e[2 * u].x), __float_as_uint(e[2 * u].y), __float_as_uint(e[2 * u].z),
+                                  __float_as_uint(e[2 * u].w), __float_as_uint(e[2 * u + 1].x), __float_as_uint(e[2 * u + 1].y),
+                                  __float_as_uint(e[2 * u + 1].z), __float_as_uint(e[2 * u + 1].w)};
+          tmem_st8(tl + C_L + 64 * wg + 8 * u, r8);
+        }
+        if (wg == 0) {   // thread row = key dimension: the tile's decay
+          const float r = p.gate_r[((size_t)bh * ntiles_all + c) * D + row];
+          s_dec[row] = __expf(r);
+          tot_decay += r;
         }
       }
       tmem_st_wait();
       ok &= mbar_wait(&bar_m1, par, err, ST_TIMEOUT);
       tc_fence_after();
-      kt_half(sm, tl, row, wg, true);
+      kt_half(sm, tl, row, wg, true, qvalid);
     }
     tmem_st_wait();
     fence_proxy_async();
@@ -575,7 +564,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
   if (full && p.state_out && gla && seg == p.nseg - 1) sdst = p.state_out + ((size_t)bh * D + row) * D;
   if (!full && p.seg_state) {
     sdst = p.seg_state + (((size_t)bh * p.nseg + seg) * D + row) * D;
-    if ((row >> 6) == wg) p.seg_decay[((size_t)bh * p.nseg + seg) * D + row] = tot_decay;
+    if (wg == 0) p.seg_decay[((size_t)bh * p.nseg + seg) * D + row] = tot_decay;
   }
   if (!s_fail && sdst) {
     tc_fence_after();
@@ -595,6 +584,81 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
   __syncthreads();
   if (warp == 0) tmem_dealloc(tb, 512);
 }
+
+}  // namespace
+
+// Decay factors of every 128-token tile, computed apart from the kernels
+// that use them so that they cost no time on a sequential critical path:
+//   E_t = exp(sum_{s>t} -a_s) = exp(b_t - r)   (bf16 E16 and/or fp32 E32,
+//                                               in the layout of g)
+//   r   = sum_s a_s                            (fp32, per tile and dimension)
+// with a = logsigmoid(g)/tau and s, t inside the tile.  One CTA per
+// (64 key dimensions, tile, sequence): lane = two dimensions (each token row
+// is one coalesced 128-byte read), warp w = tokens 16 w .. 16 w + 15, whose
+// 16 loads are all in flight together; the warps' totals give each warp its
+// carry from the later tokens.  Rows past L are not written (readers treat
+// them as zero).  A tile whose spread r - b_0 exceeds kMaxSpread sets the
+// RANGE bit of *status.
+__global__ void __launch_bounds__(256) gate_prep_kernel(const __nv_bfloat16 *g, __nv_bfloat16 *E16, float *E32,
+                                                        float *rr, uint32_t *status, int L, int ntiles,
+                                                        float inv_tau) {
+  __shared__ float2 s_tot[8][32];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int i = blockIdx.x * 64 + 2 * lane, c = blockIdx.y, bh = blockIdx.z;
+  const int tb = c * tc::kTileRows + 16 * w;     // first token of this warp
+  const size_t base = (size_t)bh * L * 128 + i;
+  float2 a[16];
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    const int t = tb + u;
+    a[u] = t < L ? __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(g + base + (size_t)t * 128))
+                 : make_float2(0.f, 0.f);
+  }
+  float2 tot = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    const bool in = tb + u < L;
+    a[u].x = in ? -tc::log_decay_fast(a[u].x, inv_tau) : 0.f;   // -a_s >= 0
+    a[u].y = in ? -tc::log_decay_fast(a[u].y, inv_tau) : 0.f;
+    tot.x += a[u].x;
+    tot.y += a[u].y;
+  }
+  s_tot[w][lane] = tot;
+  __syncthreads();
+  float2 carry = make_float2(0.f, 0.f);          // sum of -a_s over the later warps' tokens
+  for (int w2 = w + 1; w2 < 8; ++w2) {
+    carry.x += s_tot[w2][lane].x;
+    carry.y += s_tot[w2][lane].y;
+  }
+#pragma unroll
+  for (int u = 15; u >= 0; --u) {
+    if (tb + u < L) {
+      const float e0 = __expf(carry.x), e1 = __expf(carry.y);
+      const size_t o = base + (size_t)(tb + u) * 128;
+      if (E16) *reinterpret_cast<__nv_bfloat162 *>(E16 + o) = __floats2bfloat162_rn(e0, e1);
+      if (E32) *reinterpret_cast<float2 *>(E32 + o) = make_float2(e0, e1);
+    }
+    carry.x += a[u].x;
+    carry.y += a[u].y;
+  }
+  if (w == 0) {   // carry = -r: the whole tile
+    *reinterpret_cast<float2 *>(rr + ((size_t)bh * ntiles + c) * 128 + i) = make_float2(-carry.x, -carry.y);
+    const float spread = fmaxf(carry.x - a[0].x, carry.y - a[0].y);   // sum over s > 0
+    if (spread > kMaxSpread) atomicOr(status, 2u);
+  }
+}
+
+cudaError_t launch_gate_prep(const void *g, void *E16, float *E32, float *r, uint32_t *status, int BH, int L,
+                             float inv_tau, cudaStream_t s) {
+  if (L == 0) return cudaSuccess;
+  const int ntiles = (L + tc::kTileRows - 1) / tc::kTileRows;
+  gate_prep_kernel<<<dim3(2, ntiles, BH), 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(g),
+                                                       static_cast<__nv_bfloat16 *>(E16), E32, r, status, L,
+                                                       ntiles, inv_tau);
+  return cudaGetLastError();
+}
+
+namespace {
 
 // Start state of every segment: S_0 = state_in (or 0),
 // S_{s+1} = diag(exp(decay_s)) S_s + local_s.
@@ -631,12 +695,53 @@ void tc_fwd_segments(int BH, int L, int *nseg, int *tiles_per_seg) {
   *nseg = tps > 0 ? (ntiles + tps - 1) / tps : 1;
 }
 
-size_t tc_fwd_workspace_bytes(int BH, int L) {
+// Workspace of the tensor-core forward: the segment states (when the
+// sequences are split), then the gate factors E (bf16, [BH][L][D]) and the
+// per-tile decays (fp32, [BH][ntiles][D]), each 256-byte aligned.
+static size_t seg_bytes(int BH, int L) {
   int nseg, tps;
   tc_fwd_segments(BH, L, &nseg, &tps);
   if (nseg <= 1) return 0;
-  return (size_t)BH * nseg * (2 * (size_t)D * D + D) * sizeof(float);
+  return ((size_t)BH * nseg * (2 * (size_t)D * D + D) * sizeof(float) + 255) & ~size_t(255);
 }
+static size_t up256(size_t b) { return (b + 255) & ~size_t(255); }
+
+// Workspace of the tensor-core forward, in order: the segment states (when
+// the sequences are split), the tiles' bf16 decay factors E16 [BH][L][D],
+// their fp32 E32 (only for a state pass), and the tiles' log-decays r
+// [BH][ntiles][D].
+struct FwdWs {
+  float *seg_state, *seg_start, *seg_decay;
+  __nv_bfloat16 *e16;
+  float *e32, *r;
+  size_t total;
+};
+static FwdWs fwd_ws(void *base, int BH, int L) {
+  int nseg, tps;
+  tc_fwd_segments(BH, L, &nseg, &tps);
+  unsigned char *b = static_cast<unsigned char *>(base);
+  FwdWs w{};
+  size_t off = 0;
+  if (nseg > 1) {
+    w.seg_state = reinterpret_cast<float *>(b + off);
+    w.seg_start = w.seg_state + (size_t)BH * nseg * D * D;
+    w.seg_decay = w.seg_start + (size_t)BH * nseg * D * D;
+  }
+  off += seg_bytes(BH, L);
+  w.e16 = reinterpret_cast<__nv_bfloat16 *>(b + off);
+  off += up256((size_t)BH * L * D * 2);
+  if (nseg > 1) {
+    w.e32 = reinterpret_cast<float *>(b + off);
+    off += up256((size_t)BH * L * D * 4);
+  }
+  w.r = reinterpret_cast<float *>(b + off);
+  off += up256((size_t)BH * ((L + T - 1) / T) * D * 4);
+  w.total = off;
+  if (!base) w = FwdWs{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, off};
+  return w;
+}
+
+size_t tc_fwd_workspace_bytes(int BH, int L) { return fwd_ws(nullptr, BH, L).total; }
 
 int tc_fwd_stage_count(int BH, int L) {
   int nseg, tps;
@@ -646,14 +751,18 @@ int tc_fwd_stage_count(int BH, int L) {
 
 // Forward state pass over whole sequences that keeps, for every 128-token
 // tile, the bf16 state at the tile's start already decayed by the tile's
-// gates, S' = diag(exp r) S (the backward's input).
-cudaError_t launch_tc_state_snapshots(const TcFwdArgs &a, void *snap, cudaStream_t s) {
+// gates, S' = diag(exp r) S (the backward's input).  e32 and r come from
+// launch_gate_prep over the same gate logits.
+cudaError_t launch_tc_state_snapshots(const TcFwdArgs &a, void *snap, const float *e32, const float *r,
+                                      cudaStream_t s) {
   Params p;
   memset(&p, 0, sizeof(p));
   const uint64_t rows = (uint64_t)a.L;
   if (!make_map_bf16_3d(&p.mq, a.q, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mk, a.k, D, rows, a.BH, T) ||
       !make_map_bf16_3d(&p.mv, a.v, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mg, a.g, D, rows, a.BH, T))
     return cudaErrorInvalidValue;
+  p.gate_e32 = e32;
+  p.gate_r = r;
   p.wq = a.wq;
   p.wk = a.wk;
   p.meta_k = a.meta_k;
@@ -685,20 +794,27 @@ cudaError_t launch_tc_state_snapshots(const TcFwdArgs &a, void *snap, cudaStream
 cudaError_t launch_tc_fwd(const TcFwdArgs &a, int stage, cudaStream_t s) {
   int nseg, tps;
   tc_fwd_segments(a.BH, a.L, &nseg, &tps);
-  float *seg_state = static_cast<float *>(a.seg_ws);
-  float *seg_start = seg_state ? seg_state + (size_t)a.BH * nseg * D * D : nullptr;
-  float *seg_decay = seg_start ? seg_start + (size_t)a.BH * nseg * D * D : nullptr;
+  const FwdWs w = fwd_ws(a.seg_ws, a.BH, a.L);
+  const bool gla = a.branch != 2 && a.g != nullptr;
+  if (stage == 3) {
+    if (!gla) return cudaSuccess;
+    return launch_gate_prep(a.g, w.e16, w.e32, w.r, a.status, a.BH, a.L, a.inv_tau, s);
+  }
   if (nseg > 1 && stage == 1) {
-    seg_combine_kernel<<<a.BH, 256, 0, s>>>(seg_state, seg_decay, a.state_in, seg_start, nseg);
+    seg_combine_kernel<<<a.BH, 256, 0, s>>>(w.seg_state, w.seg_decay, a.state_in, w.seg_start, nseg);
     return cudaGetLastError();
   }
   Params p;
   memset(&p, 0, sizeof(p));
   const uint64_t rows = (uint64_t)a.L;
+  // the full pass loads the bf16 factors E from stage 3 as its gate tiles
+  // (unused without the GLA branch)
+  const void *gsrc = gla ? static_cast<const void *>(w.e16) : a.q;
   if (!make_map_bf16_3d(&p.mq, a.q, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mk, a.k, D, rows, a.BH, T) ||
-      !make_map_bf16_3d(&p.mv, a.v, D, rows, a.BH, T) ||
-      !make_map_bf16_3d(&p.mg, a.g ? a.g : a.q, D, rows, a.BH, T))   // g unused without the GLA branch
+      !make_map_bf16_3d(&p.mv, a.v, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mg, gsrc, D, rows, a.BH, T))
     return cudaErrorInvalidValue;
+  p.gate_r = gla ? w.r : nullptr;
+  p.gate_e32 = gla ? w.e32 : nullptr;
   p.wq = a.wq;
   p.wk = a.wk;
   p.meta_k = a.meta_k;
@@ -709,9 +825,9 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, int stage, cudaStream_t s) {
   p.state_out = a.state_out;
   p.lse = a.lse;
   p.status = a.status;
-  p.seg_start = seg_start;
-  p.seg_state = seg_state;
-  p.seg_decay = seg_decay;
+  p.seg_start = w.seg_start;
+  p.seg_state = w.seg_state;
+  p.seg_decay = w.seg_decay;
   p.H = a.H;
   p.L = a.L;
   p.M = a.M;

@@ -15,6 +15,9 @@
 //          sequence is the log-decay gradient)
 //   dS_prev = diag(exp r) (dS + Qt^T dO)
 //
+// The decay factors E (fp32) and the tiles' log-decays r come precomputed
+// from launch_gate_prep.
+//
 // tc_gla_dstates_kernel  reverse pass per sequence: dS of every tile (bf16
 //                        copies) and the gradient of the initial state.
 // tc_gla_bwd_tile_kernel one CTA per (tile, sequence): the formulas above,
@@ -40,6 +43,7 @@ constexpr uint32_t ST_TIMEOUT = 1u, ST_RANGE = 2u;
 struct DsParams {
   CUtensorMap mq, mg, mo;
   const float *wq;
+  const float *e32, *gate_r;   // fp32 decay factors [BH*L][D] and tile log-decays [BH][ntiles][D]
   __nv_bfloat16 *snap;      // [BH][ntiles][D][D] dS at each tile's end
   float *dstate_in;         // [BH][D][D] or null
   uint32_t *status;
@@ -50,6 +54,7 @@ struct DsParams {
 struct TileParams {
   CUtensorMap mq, mk, mv, mo, mg, msp, mds;   // msp / mds: [BH*ntiles][D][D] snapshots
   const float *wq, *wk;
+  const float *e32;            // fp32 decay factors [BH*L][D]
   float *dphq, *dphk, *dB, *dv;
   uint32_t *status;
   int H, L, ntiles;
@@ -67,6 +72,23 @@ __device__ __forceinline__ void stage_weights(unsigned char *dst, const float *W
   }
 }
 
+// fp32 decay factors of tile row `t` (< L, else 1), dimensions 64 h ..
+// 64 h + 63, from the precomputed array into TMEM columns col .. col + 63.
+__device__ __forceinline__ void e_half_to_tmem(const float *e32, size_t row_off, bool valid, int h, uint32_t taddr) {
+  const float *er = e32 + row_off + 64 * h;
+  float4 e[16];
+#pragma unroll
+  for (int u = 0; u < 16; ++u)
+    e[u] = valid ? *reinterpret_cast<const float4 *>(er + 4 * u) : make_float4(1.f, 1.f, 1.f, 1.f);
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const uint32_t r8[8] = {__float_as_uint(e[2 * u].x), __float_as_uint(e[2 * u].y), __float_as_uint(e[2 * u].z),
+                            __float_as_uint(e[2 * u].w), __float_as_uint(e[2 * u + 1].x), __float_as_uint(e[2 * u + 1].y),
+                            __float_as_uint(e[2 * u + 1].z), __float_as_uint(e[2 * u + 1].w)};
+    tmem_st8(taddr + 8 * u, r8);
+  }
+}
+
 // ------------------------------------------------------ reverse dS pass ---
 // Two warpgroups (256 threads): thread = tile row / state row `row` of its
 // group; the groups take halves of the key dimensions (E, phi_q) and of the
@@ -76,7 +98,6 @@ __global__ void __launch_bounds__(NT_DS, 1) tc_gla_dstates_kernel(const __grid_c
   extern __shared__ unsigned char smraw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
   __shared__ float s_dec[D];
-  __shared__ float s_wtot[2][4][16];
   __shared__ uint64_t bar_tma, bar_m1, bar_m2;
   __shared__ uint32_t s_tmem;
   constexpr uint32_t R_XQ = 0, R_G = TILE, R_O = 2 * TILE, R_W = 3 * TILE;
@@ -107,10 +128,9 @@ __global__ void __launch_bounds__(NT_DS, 1) tc_gla_dstates_kernel(const __grid_c
   const uint32_t id_z = idesc_bf16(128, 64, 0, 1);
   const uint32_t id_st = idesc_bf16(128, 128, 1, 1);
   auto loads = [&](int c) {
-    mbar_expect_tx(&bar_tma, 3 * TILE);
+    mbar_expect_tx(&bar_tma, 2 * TILE);
     for (int r = 0; r < 2; ++r) {
       tma_load_3d(sm + R_XQ + r * REG, &p.mq, &bar_tma, 64 * r, c * T, bh);
-      tma_load_3d(sm + R_G + r * REG, &p.mg, &bar_tma, 64 * r, c * T, bh);
       tma_load_3d(sm + R_O + r * REG, &p.mo, &bar_tma, 64 * r, c * T, bh);
     }
   };
@@ -136,24 +156,10 @@ __global__ void __launch_bounds__(NT_DS, 1) tc_gla_dstates_kernel(const __grid_c
         for (int u = 0; u < 32; u += 8) *reinterpret_cast<uint4 *>(dst + ch * 32 + u) = pack8(v + u);
       }
     }
-    // E in fp32 (row-wise suffix sums, dimensions 64 wg ..) into TMEM; the
-    // tile's decay exp(r)
-    for (int c16 = 4 * wg; c16 < 4 * wg + 4; ++c16) {
-      float E[16], tot[16];
-      row_decay16(sm + R_G, row, c16, t0 + row < p.L, p.inv_tau, s_wtot[wg], E, tot, 3 + wg);
-      uint32_t r[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(E[u]);
-      tmem_st8(tl + C_E + c16 * 16, r);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(E[8 + u]);
-      tmem_st8(tl + C_E + c16 * 16 + 8, r);
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        if (row == u) s_dec[c16 * 16 + u] = __expf(-tot[u]);
-        if (row == 0 && E[u] > kMaxSpreadExp) atomicOr(p.status, ST_RANGE);
-      }
-    }
+    // E in fp32 (dimensions 64 wg ..) into TMEM; the tile's decay exp(r)
+    e_half_to_tmem(p.e32, ((size_t)bh * p.L + (t0 + row < p.L ? t0 + row : 0)) * D, t0 + row < p.L, wg,
+                   tl + C_E + 64 * wg);
+    if (wg == 0) s_dec[row] = __expf(p.gate_r[((size_t)bh * ntiles + c) * D + row]);
     tmem_st_wait();
     ok = mbar_wait(&bar_m1, par, p.status, ST_TIMEOUT);
     tc_fence_after();
@@ -224,11 +230,9 @@ constexpr int NT_TILE = 256;
 __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __grid_constant__ TileParams p) {
   extern __shared__ unsigned char smraw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
-  __shared__ float s_wtot[2][4][16];
   __shared__ uint64_t bars[8];
   __shared__ uint32_t s_tmem;
-  // X_q -> Qt, X_k -> Kt, V, dO, G (gate logits) -> A^T^ (bf16, rows = keys),
-  // [W_q | W_k] -> S' -> dS
+  // X_q -> Qt, X_k -> Kt, V, dO, A^T^ (bf16, rows = keys), [W_q | W_k] -> S' -> dS
   constexpr uint32_t R_XQ = 0, R_XK = TILE, R_V = 2 * TILE, R_O = 3 * TILE, R_G = 4 * TILE, R_W = 5 * TILE;
   // TMEM, in order of use:
   //   dA [128,256) dA^T [256,384) Zq [384,448) Zk [448,512)
@@ -254,13 +258,12 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
   const uint32_t tb = s_tmem, tl = tb + lane_off;
   const int snap_idx = bh * p.ntiles + c;
   if (tid == 0) {
-    mbar_expect_tx(&bars[0], 5 * TILE);
+    mbar_expect_tx(&bars[0], 4 * TILE);
     for (int r = 0; r < 2; ++r) {
       tma_load_3d(sm + R_XQ + r * REG, &p.mq, &bars[0], 64 * r, t0, bh);
       tma_load_3d(sm + R_XK + r * REG, &p.mk, &bars[0], 64 * r, t0, bh);
       tma_load_3d(sm + R_V + r * REG, &p.mv, &bars[0], 64 * r, t0, bh);
       tma_load_3d(sm + R_O + r * REG, &p.mo, &bars[0], 64 * r, t0, bh);
-      tma_load_3d(sm + R_G + r * REG, &p.mg, &bars[0], 64 * r, t0, bh);
     }
   }
   const uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
@@ -307,22 +310,9 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
   tc_fence_before();
   __syncthreads();   // dA read out before E overwrites its columns
   tc_fence_after();
-  //    E in fp32 (row-wise suffix sums, dimensions 64 wg ..) into TMEM, then
-  //    Qt = phi_q E and Kt = phi_k / E for the same dimensions
-  for (int c16 = 4 * wg; c16 < 4 * wg + 4; ++c16) {
-    float E[16], tot[16];
-    row_decay16(sm + R_G, row, c16, valid, p.inv_tau, s_wtot[wg], E, tot, 3 + wg);
-    uint32_t r[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(E[u]);
-    tmem_st8(tl + C_E + c16 * 16, r);
-#pragma unroll
-    for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(E[8 + u]);
-    tmem_st8(tl + C_E + c16 * 16 + 8, r);
-#pragma unroll
-    for (int u = 0; u < 16; ++u)
-      if (row == 0 && E[u] > kMaxSpreadExp) atomicOr(p.status, ST_RANGE);
-  }
+  //    E in fp32 (dimensions 64 wg ..) into TMEM, then Qt = phi_q E and
+  //    Kt = phi_k / E for the same dimensions (rows past L: Kt = 0)
+  e_half_to_tmem(p.e32, ((size_t)bh * p.L + (valid ? tq : 0)) * D, valid, wg, tl + C_E + 64 * wg);
   tmem_st_wait();
 #pragma unroll
   for (int m = 0; m < 2; ++m) {
@@ -335,7 +325,7 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
       tmem_ld16(tl + C_E + 64 * wg + 16 * c16, E);
 #pragma unroll
       for (int u = 0; u < 16; ++u)
-        x16[u] = m == 0 ? ph[16 * c16 + u] * s * E[u] : __fdividef(ph[16 * c16 + u] * s, E[u]);
+        x16[u] = m == 0 ? ph[16 * c16 + u] * s * E[u] : (valid ? __fdividef(ph[16 * c16 + u] * s, E[u]) : 0.f);
       *chunk_ptr(sm, reg, row, 8 * wg + 2 * c16) = pack8(x16);
       *chunk_ptr(sm, reg, row, 8 * wg + 2 * c16 + 1) = pack8(x16 + 8);
     }
@@ -504,6 +494,8 @@ cudaError_t launch_tc_gla_bwd(const TcGlaBwdArgs &a, int stage, cudaStream_t s) 
         !make_map_bf16_3d(&p.mo, a.dout, D, rows, a.BH, T))
       return cudaErrorInvalidValue;
     p.wq = a.wq;
+    p.e32 = a.e32;
+    p.gate_r = a.gate_r;
     p.snap = static_cast<__nv_bfloat16 *>(a.snap_ds);
     p.dstate_in = a.dstate_in;
     p.status = a.status;
@@ -526,6 +518,7 @@ cudaError_t launch_tc_gla_bwd(const TcGlaBwdArgs &a, int stage, cudaStream_t s) 
       return cudaErrorInvalidValue;
     p.wq = a.wq;
     p.wk = a.wk;
+    p.e32 = a.e32;
     p.dphq = a.dphq;
     p.dphk = a.dphk;
     p.dB = a.dB;

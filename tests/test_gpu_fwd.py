@@ -167,7 +167,8 @@ def test_segmented_equals_one_shot(lz, impl):
 @pytest.mark.parametrize("L", [1000, 3000])
 def test_tc_segmented_long_sequence(lz, L):
     """Few (batch, head) pairs and a long sequence: the tensor-core forward
-    splits the sequence into segments (state pass, combine, full pass)."""
+    splits the sequence into segments (gate factors, state pass, combine,
+    full pass)."""
     w = Workload("tcseg", B=1, H=2, L=L, d=128, window=128, M=4, dtype="bf16", seed=L)
     inp = make_inputs(w)
     inp["state_in"] = torch.randn(1, 2, 128, 128, generator=torch.Generator().manual_seed(3)) * 0.1
@@ -177,7 +178,8 @@ def test_tc_segmented_long_sequence(lz, L):
                        fmap_wq=x["fmap_wq"], fmap_wk=x["fmap_wk"], meta_k=x["meta_k"],
                        meta_v=x["meta_v"], alpha=x["alpha"], state_in=x["state_in"],
                        impl=lz.IMPL_TC, plan_only=True)
-    assert len(plan) == 3, plan
+    assert plan == ["gate_prep_kernel", "tc_fwd_kernel(state pass)", "seg_combine_kernel",
+                    "tc_fwd_kernel"], plan
     got = _run(lz, x, w, lz.IMPL_TC, want_state=True, want_lse=True)
     assert lz.workspace_status(got["workspace"]) == lz.OK
     want = oracle_forward(inp, window=w.window, tau=w.gate_temp)
