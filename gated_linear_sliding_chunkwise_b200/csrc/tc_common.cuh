@@ -69,6 +69,20 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, u
       : "memory");
 }
 
+// TMA store of a staged shared-memory box to global memory (no negative
+// coordinates: rows past the map's extent are clipped), grouped per thread.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, const void *src, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];\n" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
+// wait until the shared memory of every committed store has been read
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory"); }
+// wait until every committed store has completed
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
+
 // -------------------------------------------------------------- tcgen05 ---
 // One full warp allocates / frees; the allocated TMEM address is written to
 // *dst in shared memory.
@@ -195,6 +209,14 @@ constexpr uint32_t kReg = 16384;
 constexpr uint32_t kTile = 2 * kReg;
 
 // 16-byte chunk c (columns 8c .. 8c+7) of row `row`
+// A 128 x 128 fp32 tile staged for TMA stores as four 128 x 32 boxes of
+// 16 KB, each 128-byte swizzled: the 16-byte chunk holding columns
+// col .. col + 3 (col % 4 == 0) of row `row`.
+__device__ __forceinline__ float4 *f32_stage_ptr(unsigned char *stage, int row, int col) {
+  const int b = col >> 5, j = (col & 31) >> 2;
+  return reinterpret_cast<float4 *>(stage + b * 16384 + row * 128 + ((j ^ (row & 7)) << 4));
+}
+
 __device__ __forceinline__ uint4 *chunk_ptr(unsigned char *base, uint32_t region_off, int row, int c) {
   return reinterpret_cast<uint4 *>(base + region_off + (c >> 3) * kReg + sw128_offset(row, (c & 7) * 8));
 }

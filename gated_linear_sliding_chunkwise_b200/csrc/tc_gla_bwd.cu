@@ -53,6 +53,7 @@ struct DsParams {
 
 struct TileParams {
   CUtensorMap mq, mk, mv, mo, mg, msp, mds;   // msp / mds: [BH*ntiles][D][D] snapshots
+  CUtensorMap mdq, mdk, mdb, mdv;             // fp32 outputs dphi_q, dphi_k, dB, dv (TMA stores)
   const float *wq, *wk;
   const float *e32;            // fp32 decay factors [BH*L][D]
   float *dphq, *dphk, *dB, *dv;
@@ -384,42 +385,67 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
   ok = mbar_wait(&bars[7], 0, p.status, ST_TIMEOUT);
   if (__syncthreads_or(!ok)) goto done;
   tc_fence_after();
-  // 5. rows, dimension half per group: dphi_q = E GQ, dphi_k = GK / E,
-  //    dB = Qt GQ - Kt GK; then dv (64 columns per group)
+  // 5. rows, dimension half per group: dphi_q = E GQ, dphi_k = GK / E, then
+  //    dB = Qt GQ - Kt GK and dv, staged as fp32 tiles over the free V | dO
+  //    and A^T^ | dS regions and written with TMA stores (rows past L are
+  //    clipped by the maps)
   {
-    const size_t off = ((size_t)bh * p.L + (valid ? tq : 0)) * D;
+    unsigned char *st0 = sm + R_V, *st1 = sm + R_G;
     for (int c16 = 4 * wg; c16 < 4 * wg + 4; ++c16) {
       float E[16], gq[16], gk[16];
       tmem_ld16(tl + C_E + c16 * 16, E);
       tmem_ld16(tl + C_GQ + c16 * 16, gq);
       tmem_ld16(tl + C_GK + c16 * 16, gk);
-      float q16[16], k16[16], oq[16], ok16[16], ob[16];
+#pragma unroll
+      for (int u = 0; u < 16; u += 4) {
+        *f32_stage_ptr(st0, row, c16 * 16 + u) =
+            make_float4(E[u] * gq[u], E[u + 1] * gq[u + 1], E[u + 2] * gq[u + 2], E[u + 3] * gq[u + 3]);
+        *f32_stage_ptr(st1, row, c16 * 16 + u) =
+            make_float4(__fdividef(gk[u], E[u]), __fdividef(gk[u + 1], E[u + 1]), __fdividef(gk[u + 2], E[u + 2]),
+                        __fdividef(gk[u + 3], E[u + 3]));
+      }
+    }
+    fence_proxy_async();
+    __syncthreads();
+    if (tid == 0) {
+      for (int bx = 0; bx < 4; ++bx) {
+        tma_store_3d(&p.mdq, st0 + bx * 16384, 32 * bx, t0, bh);
+        tma_store_3d(&p.mdk, st1 + bx * 16384, 32 * bx, t0, bh);
+      }
+      bulk_commit();
+      bulk_wait_read();
+    }
+    __syncthreads();
+    for (int c16 = 4 * wg; c16 < 4 * wg + 4; ++c16) {
+      float gq[16], gk[16], q16[16], k16[16];
+      tmem_ld16(tl + C_GQ + c16 * 16, gq);
+      tmem_ld16(tl + C_GK + c16 * 16, gk);
       unpack8(*chunk_ptr(sm, R_XQ, row, 2 * c16), q16);
       unpack8(*chunk_ptr(sm, R_XQ, row, 2 * c16 + 1), q16 + 8);
       unpack8(*chunk_ptr(sm, R_XK, row, 2 * c16), k16);
       unpack8(*chunk_ptr(sm, R_XK, row, 2 * c16 + 1), k16 + 8);
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        oq[u] = E[u] * gq[u];
-        ok16[u] = __fdividef(gk[u], E[u]);
-        ob[u] = q16[u] * gq[u] - k16[u] * gk[u];
-      }
-      if (valid) {
-#pragma unroll
-        for (int u = 0; u < 16; u += 4) {
-          *reinterpret_cast<float4 *>(p.dphq + off + c16 * 16 + u) = make_float4(oq[u], oq[u + 1], oq[u + 2], oq[u + 3]);
-          *reinterpret_cast<float4 *>(p.dphk + off + c16 * 16 + u) = make_float4(ok16[u], ok16[u + 1], ok16[u + 2], ok16[u + 3]);
-          *reinterpret_cast<float4 *>(p.dB + off + c16 * 16 + u) = make_float4(ob[u], ob[u + 1], ob[u + 2], ob[u + 3]);
-        }
-      }
+      for (int u = 0; u < 16; u += 4)
+        *f32_stage_ptr(st0, row, c16 * 16 + u) =
+            make_float4(q16[u] * gq[u] - k16[u] * gk[u], q16[u + 1] * gq[u + 1] - k16[u + 1] * gk[u + 1],
+                        q16[u + 2] * gq[u + 2] - k16[u + 2] * gk[u + 2], q16[u + 3] * gq[u + 3] - k16[u + 3] * gk[u + 3]);
     }
     for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
       float dv[32];
       tmem_ld32(tl + C_DV + ch * 32, dv);
-      if (valid)
 #pragma unroll
-        for (int u = 0; u < 32; u += 4)
-          *reinterpret_cast<float4 *>(p.dv + off + ch * 32 + u) = make_float4(dv[u], dv[u + 1], dv[u + 2], dv[u + 3]);
+      for (int u = 0; u < 32; u += 4)
+        *f32_stage_ptr(st1, row, ch * 32 + u) = make_float4(dv[u], dv[u + 1], dv[u + 2], dv[u + 3]);
+    }
+    fence_proxy_async();
+    __syncthreads();
+    if (tid == 0) {
+      for (int bx = 0; bx < 4; ++bx) {
+        tma_store_3d(&p.mdb, st0 + bx * 16384, 32 * bx, t0, bh);
+        tma_store_3d(&p.mdv, st1 + bx * 16384, 32 * bx, t0, bh);
+      }
+      bulk_commit();
+      bulk_wait_all();
     }
   }
 done:
@@ -514,7 +540,9 @@ cudaError_t launch_tc_gla_bwd(const TcGlaBwdArgs &a, int stage, cudaStream_t s) 
         !make_map_bf16_3d(&p.mv, a.v, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mo, a.dout, D, rows, a.BH, T) ||
         !make_map_bf16_3d(&p.mg, a.g, D, rows, a.BH, T) ||
         !make_map_bf16_3d(&p.msp, a.snap_s, D, D, (uint64_t)a.BH * ntiles, T) ||
-        !make_map_bf16_3d(&p.mds, a.snap_ds, D, D, (uint64_t)a.BH * ntiles, T))
+        !make_map_bf16_3d(&p.mds, a.snap_ds, D, D, (uint64_t)a.BH * ntiles, T) ||
+        !make_map_f32_3d(&p.mdq, a.dphq, D, rows, a.BH, T) || !make_map_f32_3d(&p.mdk, a.dphk, D, rows, a.BH, T) ||
+        !make_map_f32_3d(&p.mdb, a.dB, D, rows, a.BH, T) || !make_map_f32_3d(&p.mdv, a.dv, D, rows, a.BH, T))
       return cudaErrorInvalidValue;
     p.wq = a.wq;
     p.wk = a.wk;

@@ -35,6 +35,7 @@ constexpr uint32_t ST_TIMEOUT = 1u;
 
 struct QParams {
   CUtensorMap mq, mk, mv, mo;
+  CUtensorMap mdq;            // fp32 dq output (TMA stores)
   const float *meta_k, *meta_v, *alpha;
   float *dq, *lse, *Dterm, *dsm, *pm, *dalpha;
   uint32_t *status;
@@ -44,6 +45,7 @@ struct QParams {
 
 struct KVParams {
   CUtensorMap mq, mk, mv, mo;
+  CUtensorMap mdk, mdv;       // fp32 dk, dv outputs (TMA stores)
   const float *alpha, *lse, *Dterm;
   float *dk, *dv;
   uint32_t *status;
@@ -361,7 +363,9 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
     ok = mbar_wait(&bars[4], 0, p.status, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) goto done;
     tc_fence_after();
-    float *dst = p.dq + ((size_t)bh * p.L + (qvalid ? tq : 0)) * D;
+    // dq, staged as an fp32 tile over the free Q | dO regions and written
+    // with TMA stores (rows past L are clipped by the map)
+    unsigned char *st = sm + R_Q;
     for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
       float v[32];
       tmem_ld32(tl + C_DQ + ch * 32, v);
@@ -377,11 +381,17 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
           v[4 * q4 + 3] = fmaf(w, x.w, v[4 * q4 + 3]);
         }
       }
-      if (qvalid)
 #pragma unroll
-        for (int u = 0; u < 32; u += 4)
-          *reinterpret_cast<float4 *>(dst + ch * 32 + u) =
-              make_float4(v[u] * p.scale, v[u + 1] * p.scale, v[u + 2] * p.scale, v[u + 3] * p.scale);
+      for (int u = 0; u < 32; u += 4)
+        *f32_stage_ptr(st, row, ch * 32 + u) =
+            make_float4(v[u] * p.scale, v[u + 1] * p.scale, v[u + 2] * p.scale, v[u + 3] * p.scale);
+    }
+    fence_proxy_async();
+    __syncthreads();
+    if (tid == 0) {
+      for (int bx = 0; bx < 4; ++bx) tma_store_3d(&p.mdq, st + bx * 16384, 32 * bx, t0, bh);
+      bulk_commit();
+      bulk_wait_all();
     }
   }
 done:
@@ -508,21 +518,30 @@ __global__ void __launch_bounds__(NT_KV, 1) tc_swa_bwd_kv_kernel(const __grid_co
     tc_fence_after();
   }
   {
-    const bool kvalid = tk < p.L;
-    float *dkr = p.dk + ((size_t)bh * p.L + (kvalid ? tk : 0)) * D;
-    float *dvr = p.dv + ((size_t)bh * p.L + (kvalid ? tk : 0)) * D;
+    // dK, dV, staged as fp32 tiles over the free K | V and Q_a | dO_a regions
+    // and written with TMA stores (rows past L are clipped by the maps)
+    unsigned char *st0 = sm + R_K, *st1 = sm + R_Q0;
     for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
       float a[32], b[32];
       tmem_ld32(tl + C_DK + ch * 32, a);
       tmem_ld32(tl + C_DV + ch * 32, b);
-      if (kvalid)
 #pragma unroll
-        for (int u = 0; u < 32; u += 4) {
-          *reinterpret_cast<float4 *>(dkr + ch * 32 + u) =
-              make_float4(a[u] * p.scale, a[u + 1] * p.scale, a[u + 2] * p.scale, a[u + 3] * p.scale);
-          *reinterpret_cast<float4 *>(dvr + ch * 32 + u) =
-              make_float4(b[u] * alpha, b[u + 1] * alpha, b[u + 2] * alpha, b[u + 3] * alpha);
-        }
+      for (int u = 0; u < 32; u += 4) {
+        *f32_stage_ptr(st0, row, ch * 32 + u) =
+            make_float4(a[u] * p.scale, a[u + 1] * p.scale, a[u + 2] * p.scale, a[u + 3] * p.scale);
+        *f32_stage_ptr(st1, row, ch * 32 + u) =
+            make_float4(b[u] * alpha, b[u + 1] * alpha, b[u + 2] * alpha, b[u + 3] * alpha);
+      }
+    }
+    fence_proxy_async();
+    __syncthreads();
+    if (tid == 0) {
+      for (int bx = 0; bx < 4; ++bx) {
+        tma_store_3d(&p.mdk, st0 + bx * 16384, 32 * bx, j0, bh);
+        tma_store_3d(&p.mdv, st1 + bx * 16384, 32 * bx, j0, bh);
+      }
+      bulk_commit();
+      bulk_wait_all();
     }
   }
 done:
@@ -642,7 +661,8 @@ cudaError_t launch_tc_swa_bwd(const TcSwaBwdArgs &a, int stage, cudaStream_t s) 
     QParams p;
     memset(&p, 0, sizeof(p));
     if (!make_map_bf16_3d(&p.mq, a.q, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mk, a.k, D, rows, a.BH, T) ||
-        !make_map_bf16_3d(&p.mv, a.v, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mo, a.dout, D, rows, a.BH, T))
+        !make_map_bf16_3d(&p.mv, a.v, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mo, a.dout, D, rows, a.BH, T) ||
+        !make_map_f32_3d(&p.mdq, a.dq, D, rows, a.BH, T))
       return cudaErrorInvalidValue;
     p.meta_k = a.meta_k;
     p.meta_v = a.meta_v;
@@ -667,7 +687,8 @@ cudaError_t launch_tc_swa_bwd(const TcSwaBwdArgs &a, int stage, cudaStream_t s) 
   KVParams p;
   memset(&p, 0, sizeof(p));
   if (!make_map_bf16_3d(&p.mq, a.q, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mk, a.k, D, rows, a.BH, T) ||
-      !make_map_bf16_3d(&p.mv, a.v, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mo, a.dout, D, rows, a.BH, T))
+      !make_map_bf16_3d(&p.mv, a.v, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mo, a.dout, D, rows, a.BH, T) ||
+      !make_map_f32_3d(&p.mdk, a.dk, D, rows, a.BH, T) || !make_map_f32_3d(&p.mdv, a.dv, D, rows, a.BH, T))
     return cudaErrorInvalidValue;
   p.alpha = a.alpha;
   p.lse = a.lse;
