@@ -242,12 +242,43 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan) {
                       at<float>(ws, lay.da), at<float>(ws, lay.dv_gla), b->dstate_in, a->L};
     plan.add("gla_bwd_simt", [=] { return lz::launch_gla_bwd_simt(ga, BH, D, bf16, s); });
   }
-  if (w && bwd_swa_uses_tc(a, b->impl)) {
+  const bool swa_tc = w && bwd_swa_uses_tc(a, b->impl);
+  const bool finish_tc = gla_tc && a->fmap_wq && a->fmap_wk;
+  // With both branches on the tensor cores, the feature-map backward runs
+  // first and hands its parts (bf16) to the anchor kernels, which add them
+  // and write the final dq, dk, dv; otherwise the finish kernel sums fp32
+  // parts of both branches at the end.
+  const bool fused = finish_tc && swa_tc;
+  lz::FinishBwdArgs fa{a->q, a->k, a->g,
+                       a->fmap_wq, a->fmap_wk,
+                       g ? at<float>(ws, lay.dphq) : nullptr, g ? at<float>(ws, lay.dphk) : nullptr,
+                       g ? at<float>(ws, lay.da) : nullptr, g ? at<float>(ws, lay.dv_gla) : nullptr,
+                       w ? at<float>(ws, lay.dq_swa) : nullptr, w ? at<float>(ws, lay.dk_swa) : nullptr,
+                       w ? at<float>(ws, lay.dv_swa) : nullptr,
+                       b->dq, b->dk, b->dv, b->dg, b->dfmap_wq, b->dfmap_wk, a->H, a->L, inv_tau,
+                       gla_tc ? 0 : 1, static_cast<uint32_t *>(ws)};
+  if (gla_tc) fa.da = nullptr;   // the gate gradient comes from gate_grad_kernel
+  if (fused) {
+    fa.xq_part = at<void>(ws, lay.dq_swa);   // bf16 parts in the anchor part slots
+    fa.xk_part = at<void>(ws, lay.dk_swa);
+    fa.dq_swa = fa.dk_swa = fa.dv_swa = nullptr;
+    plan.add("tc_finish_kernel", [=] { return lz::launch_tc_finish(fa, BH, s); });
+  }
+  if (swa_tc) {
     lz::TcSwaBwdArgs t{a->q, a->k, a->v, b->dout, a->meta_k, a->meta_v, a->alpha,
                        at<float>(ws, lay.dq_swa), at<float>(ws, lay.dk_swa), at<float>(ws, lay.dv_swa),
                        at<float>(ws, lay.lse), at<float>(ws, lay.Dterm), at<float>(ws, lay.dsm),
                        at<float>(ws, lay.pm), b->dmeta_k, b->dmeta_v, b->dalpha, static_cast<uint32_t *>(ws),
                        a->B, a->H, BH, a->L, a->M, a->window, scale_of(a)};
+    if (fused) {
+      t.dq = t.dk = t.dv = nullptr;
+      t.xq_part = at<void>(ws, lay.dq_swa);
+      t.xk_part = at<void>(ws, lay.dk_swa);
+      t.dv_gla = at<float>(ws, lay.dv_gla);
+      t.dq_out = b->dq;
+      t.dk_out = b->dk;
+      t.dv_out = b->dv;
+    }
     plan.add("tc_swa_bwd_q_kernel", [=] { return lz::launch_tc_swa_bwd(t, 0, s); });
     plan.add("tc_swa_bwd_kv_kernel", [=] { return lz::launch_tc_swa_bwd(t, 1, s); });
     if (a->M > 0 && (b->dmeta_k || b->dmeta_v))
@@ -261,19 +292,12 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan) {
                         at<float>(ws, lay.dk_swa), at<float>(ws, lay.dv_swa), a->H, a->L, a->window, scale_of(a)};
     plan.add("swa_bwd_kv", [=] { return lz::launch_swa_bwd_kv(ka, BH, D, bf16, s); });
   }
-  lz::FinishBwdArgs fa{a->q, a->k, a->g,
-                       a->fmap_wq, a->fmap_wk,
-                       g ? at<float>(ws, lay.dphq) : nullptr, g ? at<float>(ws, lay.dphk) : nullptr,
-                       g ? at<float>(ws, lay.da) : nullptr, g ? at<float>(ws, lay.dv_gla) : nullptr,
-                       w ? at<float>(ws, lay.dq_swa) : nullptr, w ? at<float>(ws, lay.dk_swa) : nullptr,
-                       w ? at<float>(ws, lay.dv_swa) : nullptr,
-                       b->dq, b->dk, b->dv, b->dg, b->dfmap_wq, b->dfmap_wk, a->H, a->L, inv_tau,
-                       gla_tc ? 0 : 1, static_cast<uint32_t *>(ws)};
-  if (gla_tc) fa.da = nullptr;   // the gate gradient comes from gate_grad_kernel
-  if (gla_tc && a->fmap_wq && a->fmap_wk)
-    plan.add("tc_finish_kernel", [=] { return lz::launch_tc_finish(fa, BH, s); });
-  else
-    plan.add("finish_bwd", [=] { return lz::launch_finish_bwd(fa, BH, D, bf16, s); });
+  if (!fused) {
+    if (finish_tc)
+      plan.add("tc_finish_kernel", [=] { return lz::launch_tc_finish(fa, BH, s); });
+    else
+      plan.add("finish_bwd", [=] { return lz::launch_finish_bwd(fa, BH, D, bf16, s); });
+  }
   if (gla_tc) {
     lz::TcGlaBwdArgs t{a->q, a->k, a->v, a->g, b->dout, a->fmap_wq, a->fmap_wk, nullptr, nullptr, nullptr,
                        nullptr, at<float>(ws, lay.da), nullptr, b->dg, nullptr, static_cast<uint32_t *>(ws),

@@ -91,6 +91,10 @@ struct FinishBwdArgs {
   float inv_tau;
   int write_dg;                             // 0 when another kernel writes dg
   uint32_t *status;                         // workspace status word (tensor-core finish)
+  // Tensor-core finish only: when set, write the GLA feature-map parts dx_q,
+  // dx_k here (bf16 [B*H*L][128]) for the anchor kernels to add, and leave
+  // dq, dk, dv to them.
+  void *xq_part, *xk_part;
 };
 
 struct TcFwdArgs {
@@ -114,6 +118,11 @@ struct TcSwaBwdArgs {
   uint32_t *status;
   int B, H, BH, L, M, window;
   float scale;
+  // Fused with the tensor-core GLA backward (when xq_part is set): add the
+  // GLA parts and write the final gradients instead of the fp32 parts above.
+  const void *xq_part, *xk_part;   // bf16 [B*H*L][128] feature-map parts dx_q, dx_k
+  const float *dv_gla;             // fp32 [B*H*L][128] value part
+  void *dq_out, *dk_out, *dv_out;  // bf16 dq, dk, dv
 };
 
 struct TcGlaBwdArgs {

@@ -29,6 +29,7 @@ constexpr uint32_t ST_TIMEOUT = 1u;
 
 struct Params {
   CUtensorMap mq, mk;
+  CUtensorMap mxq, mxk;                    // bf16 dx_q, dx_k parts (fused mode)
   const float *wq, *wk;
   const float *dphq, *dphk, *dv_gla;       // GLA parts (fp32), null when the branch is off
   const float *dq_swa, *dk_swa, *dv_swa;   // anchor parts (fp32), null when the branch is off
@@ -36,6 +37,7 @@ struct Params {
   float *dwq, *dwk;
   uint32_t *status;
   int H, L;
+  int fused;                               // write dx_q, dx_k parts; the anchor kernels finish dq, dk, dv
 };
 
 // Two warpgroups (256 threads), thread = tile row `row` of its group:
@@ -49,7 +51,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
   __shared__ uint32_t s_tmem;
   // X_q, X_k, W_q | W_k (64-column tiles), dZ_q | dZ_k (64-column tiles)
   constexpr uint32_t R_XQ = 0, R_XK = TILE, R_WQ = 2 * TILE, R_WK = 2 * TILE + REG, R_ZQ = 3 * TILE,
-                     R_ZK = 3 * TILE + REG;
+                     R_ZK = 3 * TILE + REG, R_STG = 4 * TILE;   // R_STG: dx_q | dx_k staging (fused mode)
   // TMEM: dWq [0,64) dWk [64,128) Zq [128,192) Zk [192,256) dXq [256,384) dXk [384,512)
   constexpr uint32_t C_WQ = 0, C_WK = 64, C_ZQ = 128, C_ZK = 192, C_XQ = 256, C_XK = 384;
   const int tid = threadIdx.x, warp = tid >> 5, wg = tid >> 7, row = tid & 127;
@@ -172,10 +174,31 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
       tc_fence_after();
       if (tid == 0 && c + 1 < ntiles) loads(c + 1);   // X tiles consumed by the dW products
     }
+    if (p.fused) {
+      // dx of this group's map, bf16, staged over R_STG and written with TMA
+      // stores (rows past L are clipped by the map)
+      unsigned char *st = sm + R_STG + wg * TILE;
+      for (int ch = 0; ch < 4; ++ch) {
+        float v[32];
+        tmem_ld32(tl + (wg == 0 ? C_XQ : C_XK) + ch * 32, v);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) *chunk_ptr(st, 0, row, 4 * ch + k) = pack8(v + 8 * k);
+      }
+      fence_proxy_async();
+      __syncthreads();
+      if (tid == 0) {
+        tma_store_3d(&p.mxq, sm + R_STG, 0, c * T, bh);
+        tma_store_3d(&p.mxq, sm + R_STG + REG, 64, c * T, bh);
+        tma_store_3d(&p.mxk, sm + R_STG + TILE, 0, c * T, bh);
+        tma_store_3d(&p.mxk, sm + R_STG + TILE + REG, 64, c * T, bh);
+        bulk_commit();
+        bulk_wait_read();
+      }
+    }
     // dq (group 0), dk (group 1) = GLA (dz W^T) + anchor parts; dv = both
     // parts, 64 columns per group
 #pragma unroll
-    for (int k = 0; k < 2; ++k) {
+    for (int k = 0; k < 2 && !p.fused; ++k) {
       const int m = k == 0 ? wg : 2;
       const float *__restrict__ swa = m == 0 ? p.dq_swa : (m == 1 ? p.dk_swa : p.dv_swa);
       const float *__restrict__ gpart = m == 2 ? p.dv_gla : nullptr;
@@ -224,12 +247,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
       }
     }
   }
+  if (p.fused && tid == 0) bulk_wait_all();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(s_tmem, 512);
 }
 
-constexpr size_t SMEM_BYTES = 4 * TILE + 1024;
+constexpr size_t SMEM_BYTES = 6 * TILE + 1024;
 
 }  // namespace
 
@@ -238,6 +262,10 @@ cudaError_t launch_tc_finish(const FinishBwdArgs &a, int BH, cudaStream_t s) {
   memset(&p, 0, sizeof(p));
   const uint64_t rows = (uint64_t)a.L;
   if (!make_map_bf16_3d(&p.mq, a.q, D, rows, BH, T) || !make_map_bf16_3d(&p.mk, a.k, D, rows, BH, T))
+    return cudaErrorInvalidValue;
+  p.fused = a.xq_part != nullptr;
+  if (p.fused && (!make_map_bf16_3d(&p.mxq, a.xq_part, D, rows, BH, T) ||
+                  !make_map_bf16_3d(&p.mxk, a.xk_part, D, rows, BH, T)))
     return cudaErrorInvalidValue;
   p.wq = a.wq;
   p.wk = a.wk;

@@ -36,21 +36,26 @@ constexpr uint32_t ST_TIMEOUT = 1u;
 struct QParams {
   CUtensorMap mq, mk, mv, mo;
   CUtensorMap mdq;            // fp32 dq output (TMA stores)
+  CUtensorMap mxq, mdqo;      // fused: bf16 GLA part dx_q (load), bf16 final dq (store)
   const float *meta_k, *meta_v, *alpha;
   float *dq, *lse, *Dterm, *dsm, *pm, *dalpha;
   uint32_t *status;
   int H, L, M, window;
   float scale;
+  int fused;
 };
 
 struct KVParams {
   CUtensorMap mq, mk, mv, mo;
   CUtensorMap mdk, mdv;       // fp32 dk, dv outputs (TMA stores)
+  CUtensorMap mxk, mdvg;      // fused: bf16 GLA part dx_k, fp32 GLA dv (loads)
+  CUtensorMap mdko, mdvo;     // fused: bf16 final dk, dv (stores)
   const float *alpha, *lse, *Dterm;
   float *dk, *dv;
   uint32_t *status;
   int H, L, window;
   float scale;
+  int fused;
 };
 
 __device__ __forceinline__ void setup_cta(uint32_t *tmem_slot, uint64_t *bars, int nbars, int tid) {
@@ -78,7 +83,7 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
   __shared__ float s_x[MAXM][T];        // dO . mv_m per row, later the meta dS per row
   __shared__ float s_pmax[2][T], s_psum[2][T];
   __shared__ float s_red[4];
-  __shared__ uint64_t bars[5];
+  __shared__ uint64_t bars[6];
   __shared__ uint32_t s_tmem;
   // regions: Q, dO, K_prev, K, V_prev, V
   constexpr uint32_t R_Q = 0, R_O = TILE, R_KP = 2 * TILE, R_K = 3 * TILE, R_VP = 4 * TILE, R_V = 5 * TILE;
@@ -93,7 +98,7 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
   const float alpha = p.alpha ? p.alpha[h] : 1.f;
   const uint32_t sbase = smem_u32(sm);
   uint64_t *bar_tma = &bars[0], *bar_m = &bars[1];
-  setup_cta(&s_tmem, bars, 5, tid);
+  setup_cta(&s_tmem, bars, 6, tid);
   for (int e = tid; e < MAXM * D; e += NT_Q) {
     const int m = e / D;
     s_mk[m][e % D] = m < p.M ? p.meta_k[(size_t)h * p.M * D + e] : 0.f;
@@ -310,6 +315,11 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
     ok = mbar_wait(&bars[3], 0, p.status, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) goto done;
     tc_fence_after();
+    if (p.fused && tid == 0) {   // the GLA part of dq into the free V region
+      mbar_expect_tx(&bars[5], TILE);
+      tma_load_3d(sm + R_V, &p.mxq, &bars[5], 0, t0, bh);
+      tma_load_3d(sm + R_V + kReg, &p.mxq, &bars[5], 64, t0, bh);
+    }
 
     // 5. dS = P (alpha dP' - D), P = P^ / l, on the band (zero elsewhere,
     //    as P^ is); alternate chunks per group; the meta terms go to memory
@@ -363,6 +373,46 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
     ok = mbar_wait(&bars[4], 0, p.status, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) goto done;
     tc_fence_after();
+    if (p.fused) {
+      // dq = anchor part + GLA part, bf16, written in place over the GLA
+      // part in the V region and stored with TMA (rows past L are clipped)
+      ok = mbar_wait(&bars[5], 0, p.status, ST_TIMEOUT);
+      if (__syncthreads_or(!ok)) goto done;
+      for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
+        float v[32];
+        tmem_ld32(tl + C_DQ + ch * 32, v);
+        for (int m = 0; m < p.M; ++m) {
+          const float w = s_x[m][row];
+          const float4 *mk = reinterpret_cast<const float4 *>(&s_mk[m][ch * 32]);
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const float4 x = mk[q4];
+            v[4 * q4] = fmaf(w, x.x, v[4 * q4]);
+            v[4 * q4 + 1] = fmaf(w, x.y, v[4 * q4 + 1]);
+            v[4 * q4 + 2] = fmaf(w, x.z, v[4 * q4 + 2]);
+            v[4 * q4 + 3] = fmaf(w, x.w, v[4 * q4 + 3]);
+          }
+        }
+#pragma unroll
+        for (int k8 = 0; k8 < 4; ++k8) {
+          uint4 *cp = chunk_ptr(sm, R_V, row, 4 * ch + k8);
+          float g8[8];
+          unpack8(*cp, g8);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) g8[u] = fmaf(v[8 * k8 + u], p.scale, g8[u]);
+          *cp = pack8(g8);
+        }
+      }
+      fence_proxy_async();
+      __syncthreads();
+      if (tid == 0) {
+        tma_store_3d(&p.mdqo, sm + R_V, 0, t0, bh);
+        tma_store_3d(&p.mdqo, sm + R_V + kReg, 64, t0, bh);
+        bulk_commit();
+        bulk_wait_all();
+      }
+      goto done;
+    }
     // dq, staged as an fp32 tile over the free Q | dO regions and written
     // with TMA stores (rows past L are clipped by the map)
     unsigned char *st = sm + R_Q;
@@ -409,7 +459,7 @@ __global__ void __launch_bounds__(NT_KV, 1) tc_swa_bwd_kv_kernel(const __grid_co
   extern __shared__ unsigned char smraw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
   __shared__ float s_lse[2 * T], s_D[2 * T];
-  __shared__ uint64_t bars[5];
+  __shared__ uint64_t bars[7];
   __shared__ uint32_t s_tmem;
   // regions: K, V, Q_a, dO_a, Q_b, dO_b  (query tiles kb and kb + 1)
   constexpr uint32_t R_K = 0, R_V = TILE, R_Q0 = 2 * TILE, R_O0 = 3 * TILE;
@@ -421,7 +471,7 @@ __global__ void __launch_bounds__(NT_KV, 1) tc_swa_bwd_kv_kernel(const __grid_co
   const int bh = blockIdx.y, h = bh % p.H, j0 = blockIdx.x * T, tk = j0 + row;
   const float alpha = p.alpha ? p.alpha[h] : 1.f;
   const uint32_t sbase = smem_u32(sm);
-  setup_cta(&s_tmem, bars, 5, tid);
+  setup_cta(&s_tmem, bars, 7, tid);
   for (int e = tid; e < 2 * T; e += NT_KV) {
     const int t = j0 + e;
     s_lse[e] = t < p.L ? p.lse[(size_t)bh * p.L + t] : 0.f;
@@ -459,6 +509,11 @@ __global__ void __launch_bounds__(NT_KV, 1) tc_swa_bwd_kv_kernel(const __grid_co
     ok = mbar_wait(&bars[1 + 2 * it], 0, p.status, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) goto done;
     tc_fence_after();
+    if (p.fused && it == 1 && tid == 0) {   // K and V are read: the GLA part of dk into K
+      mbar_expect_tx(&bars[6], TILE);
+      tma_load_3d(sm + R_K, &p.mxk, &bars[6], 0, j0, bh);
+      tma_load_3d(sm + R_K + kReg, &p.mxk, &bars[6], 64, j0, bh);
+    }
     // P = exp(scale s - lse_t), dS = P (alpha dP - D_t) on the band t - w < j <= t.
     // Query column qc of this tile is token j0 + it T + qc; the warp's keys
     // j0 + r0 .. j0 + r0 + 31 see columns qc with 0 <= it T + qc - row < w.
@@ -516,6 +571,50 @@ __global__ void __launch_bounds__(NT_KV, 1) tc_swa_bwd_kv_kernel(const __grid_co
     ok = mbar_wait(&bars[2 + 2 * it], 0, p.status, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) goto done;
     tc_fence_after();
+    if (p.fused && it == 0 && tid == 0) {   // query tile a is done: the GLA dv into its regions
+      mbar_expect_tx(&bars[5], 2 * TILE);
+      for (int bx = 0; bx < 4; ++bx) tma_load_3d(sm + R_Q0 + bx * 16384, &p.mdvg, &bars[5], 32 * bx, j0, bh);
+    }
+  }
+  if (p.fused) {
+    // dk = anchor part + GLA part (bf16, in place over the GLA part in K);
+    // dv = anchor part + GLA dv (fp32 in Q_a | dO_a) as bf16 into V; both
+    // stored with TMA (rows past L are clipped by the maps)
+    ok = mbar_wait(&bars[5], 0, p.status, ST_TIMEOUT);
+    ok &= mbar_wait(&bars[6], 0, p.status, ST_TIMEOUT);
+    if (__syncthreads_or(!ok)) goto done;
+    for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
+      float a[32], b[32];
+      tmem_ld32(tl + C_DK + ch * 32, a);
+      tmem_ld32(tl + C_DV + ch * 32, b);
+#pragma unroll
+      for (int k8 = 0; k8 < 4; ++k8) {
+        uint4 *cp = chunk_ptr(sm, R_K, row, 4 * ch + k8);
+        float g8[8], v8[8];
+        unpack8(*cp, g8);
+        const float4 d0 = *f32_stage_ptr(sm + R_Q0, row, 32 * ch + 8 * k8);
+        const float4 d1 = *f32_stage_ptr(sm + R_Q0, row, 32 * ch + 8 * k8 + 4);
+        const float dg[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          g8[u] = fmaf(a[8 * k8 + u], p.scale, g8[u]);
+          v8[u] = fmaf(b[8 * k8 + u], alpha, dg[u]);
+        }
+        *cp = pack8(g8);
+        *chunk_ptr(sm, R_V, row, 4 * ch + k8) = pack8(v8);
+      }
+    }
+    fence_proxy_async();
+    __syncthreads();
+    if (tid == 0) {
+      tma_store_3d(&p.mdko, sm + R_K, 0, j0, bh);
+      tma_store_3d(&p.mdko, sm + R_K + kReg, 64, j0, bh);
+      tma_store_3d(&p.mdvo, sm + R_V, 0, j0, bh);
+      tma_store_3d(&p.mdvo, sm + R_V + kReg, 64, j0, bh);
+      bulk_commit();
+      bulk_wait_all();
+    }
+    goto done;
   }
   {
     // dK, dV, staged as fp32 tiles over the free K | V and Q_a | dO_a regions
@@ -662,7 +761,11 @@ cudaError_t launch_tc_swa_bwd(const TcSwaBwdArgs &a, int stage, cudaStream_t s) 
     memset(&p, 0, sizeof(p));
     if (!make_map_bf16_3d(&p.mq, a.q, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mk, a.k, D, rows, a.BH, T) ||
         !make_map_bf16_3d(&p.mv, a.v, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mo, a.dout, D, rows, a.BH, T) ||
-        !make_map_f32_3d(&p.mdq, a.dq, D, rows, a.BH, T))
+        !make_map_f32_3d(&p.mdq, a.dq ? a.dq : static_cast<float *>(a.dq_out), D, rows, a.BH, T))
+      return cudaErrorInvalidValue;
+    p.fused = a.xq_part != nullptr;
+    if (p.fused && (!make_map_bf16_3d(&p.mxq, a.xq_part, D, rows, a.BH, T) ||
+                    !make_map_bf16_3d(&p.mdqo, a.dq_out, D, rows, a.BH, T)))
       return cudaErrorInvalidValue;
     p.meta_k = a.meta_k;
     p.meta_v = a.meta_v;
@@ -688,7 +791,14 @@ cudaError_t launch_tc_swa_bwd(const TcSwaBwdArgs &a, int stage, cudaStream_t s) 
   memset(&p, 0, sizeof(p));
   if (!make_map_bf16_3d(&p.mq, a.q, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mk, a.k, D, rows, a.BH, T) ||
       !make_map_bf16_3d(&p.mv, a.v, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mo, a.dout, D, rows, a.BH, T) ||
-      !make_map_f32_3d(&p.mdk, a.dk, D, rows, a.BH, T) || !make_map_f32_3d(&p.mdv, a.dv, D, rows, a.BH, T))
+      !make_map_f32_3d(&p.mdk, a.dk ? a.dk : static_cast<float *>(a.dk_out), D, rows, a.BH, T) ||
+      !make_map_f32_3d(&p.mdv, a.dv ? a.dv : static_cast<float *>(a.dv_out), D, rows, a.BH, T))
+    return cudaErrorInvalidValue;
+  p.fused = a.xq_part != nullptr;
+  if (p.fused && (!make_map_bf16_3d(&p.mxk, a.xk_part, D, rows, a.BH, T) ||
+                  !make_map_f32_3d(&p.mdvg, a.dv_gla, D, rows, a.BH, T) ||
+                  !make_map_bf16_3d(&p.mdko, a.dk_out, D, rows, a.BH, T) ||
+                  !make_map_bf16_3d(&p.mdvo, a.dv_out, D, rows, a.BH, T)))
     return cudaErrorInvalidValue;
   p.alpha = a.alpha;
   p.lse = a.lse;
