@@ -113,50 +113,71 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
       ok = mbar_wait(&bar_z, par, p.status, ST_TIMEOUT);
       if (__syncthreads_or(!ok)) { fail = true; break; }
       tc_fence_after();
-      // dz row of this group's map (fp32 math) -> bf16 dZ tile
-      {
-        float pos[F], neg[F];
-        const float sp = feature_half(tl + (wg == 0 ? C_ZQ : C_ZK), 0, pos);
-        const float sn = feature_half(tl + (wg == 0 ? C_ZQ : C_ZK), 1, neg);
-        const float *__restrict__ src = (wg == 0 ? p.dphq : p.dphk) + off;
+      // dz of both maps, one map at a time (fp32 math, bf16 dZ tiles): group
+      // 0 owns the softmax(z) half (p, dp), group 1 the softmax(-z) half
+      // (n, dn); each loads its 64 dphi values once, all in flight, and forms
+      //   A_f = p_f (dp_f - <dp, p>)   or   B_f = n_f (dn_f - <dn, n>).
+      // The half-terms meet in shared memory (R_STG, one swizzled 128 x 32
+      // fp32 box per map and group): group 0 writes dz_f = A_f - B_f for
+      // f < 32, group 1 for f >= 32.
+#pragma unroll 1
+      for (int m = 0; m < 2; ++m) {
+        float ph[F];
+        const float sc = feature_half(tl + (m == 0 ? C_ZQ : C_ZK), wg, ph);
+        const float *__restrict__ src = (m == 0 ? p.dphq : p.dphk) + off + wg * F;
+        float4 d[16];
 #pragma unroll
-        for (int f = 0; f < F; ++f) { pos[f] *= sp; neg[f] *= sn; }
-        // pass 1: <dp, p> and <dn, n>
-        float dp4[4] = {0.f, 0.f, 0.f, 0.f}, dn4[4] = {0.f, 0.f, 0.f, 0.f};
-        if (valid) {
+        for (int u = 0; u < 16; ++u)
+          d[u] = valid ? *reinterpret_cast<const float4 *>(src + 4 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+        float dot4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int u = 0; u < F; u += 4) {
-            const float4 a = *reinterpret_cast<const float4 *>(src + u);
-            const float4 b = *reinterpret_cast<const float4 *>(src + F + u);
-            dp4[(u >> 2) & 3] += a.x * pos[u] + a.y * pos[u + 1] + a.z * pos[u + 2] + a.w * pos[u + 3];
-            dn4[(u >> 2) & 3] += b.x * neg[u] + b.y * neg[u + 1] + b.z * neg[u + 2] + b.w * neg[u + 3];
-          }
+        for (int u = 0; u < 16; ++u) {
+          ph[4 * u] *= sc;
+          ph[4 * u + 1] *= sc;
+          ph[4 * u + 2] *= sc;
+          ph[4 * u + 3] *= sc;
+          dot4[u & 3] += d[u].x * ph[4 * u] + d[u].y * ph[4 * u + 1] + d[u].z * ph[4 * u + 2] + d[u].w * ph[4 * u + 3];
         }
-        const float dotp = (dp4[0] + dp4[1]) + (dp4[2] + dp4[3]);
-        const float dotn = (dn4[0] + dn4[1]) + (dn4[2] + dn4[3]);
-        // pass 2: dz = p (dp - <dp,p>) - n (dn - <dn,n>), 8 features at a time
-        const uint32_t reg = wg == 0 ? R_ZQ : R_ZK;
+        const float dot = (dot4[0] + dot4[1]) + (dot4[2] + dot4[3]);
 #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
-          float dz[8];
-          if (valid) {
-            const float4 a0 = *reinterpret_cast<const float4 *>(src + c8 * 8);
-            const float4 a1 = *reinterpret_cast<const float4 *>(src + c8 * 8 + 4);
-            const float4 b0 = *reinterpret_cast<const float4 *>(src + F + c8 * 8);
-            const float4 b1 = *reinterpret_cast<const float4 *>(src + F + c8 * 8 + 4);
-            const float dpv[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-            const float dnv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+        for (int u = 0; u < 16; ++u) {   // ph <- this group's half-term
+          ph[4 * u] *= d[u].x - dot;
+          ph[4 * u + 1] *= d[u].y - dot;
+          ph[4 * u + 2] *= d[u].z - dot;
+          ph[4 * u + 3] *= d[u].w - dot;
+        }
+        // send the half-terms of the other group's features
+        unsigned char *mine = sm + R_STG + (2 * m + wg) * 16384;
+        const unsigned char *theirs = sm + R_STG + (2 * m + 1 - wg) * 16384;
+        if (wg == 0) {
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const int f = c8 * 8 + u;
-              dz[u] = pos[f] * (dpv[u] - dotp) - neg[f] * (dnv[u] - dotn);
-            }
+          for (int j = 0; j < 8; ++j)
+            *f32_stage_ptr(mine, row, 4 * j) = make_float4(ph[32 + 4 * j], ph[33 + 4 * j], ph[34 + 4 * j], ph[35 + 4 * j]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *f32_stage_ptr(mine, row, 4 * j) = make_float4(ph[4 * j], ph[1 + 4 * j], ph[2 + 4 * j], ph[3 + 4 * j]);
+        }
+        bar_sync(1, NTHREADS);
+        const int fm = 32 * wg;            // this group's 32 dz features
+        float dz[32];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float4 t = *f32_stage_ptr(const_cast<unsigned char *>(theirs), row, 4 * j);
+          const float tv[4] = {t.x, t.y, t.z, t.w};
+          // group 0: A_f - B_f with B from group 1; group 1: A_{32+f} - B_{32+f} with A from group 0
+          if (wg == 0) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) dz[4 * j + u] = valid ? ph[4 * j + u] - tv[u] : 0.f;
           } else {
 #pragma unroll
-            for (int u = 0; u < 8; ++u) dz[u] = 0.f;
+            for (int u = 0; u < 4; ++u) dz[4 * j + u] = valid ? tv[u] - ph[32 + 4 * j + u] : 0.f;
           }
-          *reinterpret_cast<uint4 *>(sm + reg + sw128_offset(row, c8 * 8)) = pack8(dz);
         }
+        const uint32_t reg = m == 0 ? R_ZQ : R_ZK;
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8)
+          *reinterpret_cast<uint4 *>(sm + reg + sw128_offset(row, fm + 8 * c8)) = pack8(dz + 8 * c8);
       }
       fence_proxy_async();
       tc_fence_before();
