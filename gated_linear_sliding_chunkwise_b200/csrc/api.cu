@@ -52,8 +52,13 @@ bool gla_on(const lizard_fwd_args *a) { return a->branch != LIZARD_BRANCH_SWA_ON
 bool swa_on(const lizard_fwd_args *a) { return a->branch != LIZARD_BRANCH_GLA_ONLY; }
 
 // Kernel family the forward runs for these arguments.
+// The tensor-core kernels build the Hedgehog map from its weights; without
+// them (the identity map) the GLA branch takes the portable kernels.
+bool fmap_weights(const lizard_fwd_args *a) { return a->fmap_wq != nullptr && a->fmap_wk != nullptr; }
+
 bool fwd_uses_tc(const lizard_fwd_args *a) {
-  const bool ok = lz::tc_fwd_supported(a->dk, a->dv, a->window, a->M, a->dtype == LIZARD_BF16);
+  const bool ok = lz::tc_fwd_supported(a->dk, a->dv, a->window, a->M, a->dtype == LIZARD_BF16) &&
+                  (fmap_weights(a) || a->branch == LIZARD_BRANCH_SWA_ONLY);
   if (a->impl == LIZARD_IMPL_TC) return ok;
   return a->impl == LIZARD_IMPL_AUTO && ok;
 }
@@ -88,7 +93,7 @@ bool bwd_swa_uses_tc(const lizard_fwd_args *a, int impl) {
 
 // Whether the backward's GLA branch runs on the tensor-core kernels.
 bool bwd_gla_uses_tc(const lizard_fwd_args *a, int impl) {
-  const bool ok = a->dtype == LIZARD_BF16 && a->dk == 128 && a->dv == 128;
+  const bool ok = a->dtype == LIZARD_BF16 && a->dk == 128 && a->dv == 128 && fmap_weights(a);
   return (impl == LIZARD_IMPL_AUTO || impl == LIZARD_IMPL_TC) && ok;
 }
 

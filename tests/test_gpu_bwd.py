@@ -156,3 +156,25 @@ def test_train_step_full_size_sampled_heads(lz, impl):
     for (b, h), r in want.items():
         for name in ("dq", "dk", "dv", "dg", "dstate_in"):
             check(f"{name}[{b},{h}]", got[name][b:b + 1, h:h + 1], r[name], "bf16")
+
+
+@pytest.mark.parametrize("case", ["swa_portable", "no_fmap_weights"])
+def test_backward_mixed_paths(lz, case):
+    """bf16, d = 128 combinations outside the fused tensor-core configuration:
+    a window above 128 (tensor-core GLA backward, portable anchor backward,
+    the tensor-core finish summing fp32 parts) and no feature-map weights
+    (identity map: tensor-core GLA backward, portable finish)."""
+    window = 200 if case == "swa_portable" else 64
+    w = Workload("bmixed", B=1, H=2, L=300, d=128, window=window, M=4, dtype="bf16", seed=61,
+                 kind="train")
+    inp = make_inputs(w)
+    inp["alpha"] = random_alpha(2, seed=5)
+    if case == "no_fmap_weights":
+        inp["fmap_wq"] = inp["fmap_wk"] = None
+    got = _run(lz, to_device(inp), w, lz.IMPL_AUTO)
+    want = oracle_backward(inp, window=w.window, tau=w.gate_temp)
+    for name in GRADS:
+        if want[name] is None:
+            assert got[name] is None
+            continue
+        check(name, got[name], want[name], "bf16")

@@ -216,3 +216,18 @@ def test_full_size_sampled_heads(lz, impl, name, pairs):
         check(f"o[{b},{h}]", got["o"][b:b + 1, h:h + 1], r["o"], "bf16")
         check(f"S[{b},{h}]", got["state_out"][b:b + 1, h:h + 1], r["state_out"], "bf16")
         check(f"lse[{b},{h}]", got["lse"][b:b + 1, h:h + 1], r["lse"], "bf16")
+
+
+def test_identity_feature_map_at_tensor_core_shape(lz):
+    """No feature-map weights (the identity map) at bf16, d = 128: the
+    forward takes the portable GLA kernels and matches the oracle; forcing
+    the tensor-core kernels is refused."""
+    w = Workload("ident", B=1, H=2, L=300, d=128, window=64, M=4, dtype="bf16", seed=71)
+    inp = make_inputs(w)
+    inp["fmap_wq"] = inp["fmap_wk"] = None
+    x = to_device(inp)
+    got = _run(lz, x, w, lz.IMPL_AUTO, want_state=True)
+    want = oracle_forward(inp, window=w.window, tau=w.gate_temp)
+    check("o", got["o"], want["o"], "bf16")
+    with pytest.raises(RuntimeError):
+        _run(lz, x, w, lz.IMPL_TC)
