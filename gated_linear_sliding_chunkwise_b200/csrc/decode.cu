@@ -402,12 +402,17 @@ LZ_DEV PairInfo pair_info(const DecodeArgs &p, int B, int first, int k, const in
   return r;
 }
 
-// Thread roles: warps 0..7 consume (256 threads, thread = column group or
-// slot pair as below), warp 8 produces: one lane walks the same chunk
-// sequence, waits until all eight consumer warps have released a slot
-// (`empty` mbarrier, one arrival per warp) and refills it.  The consumers
-// meet on named barrier 1 only where data flows between them.
+// Thread roles: warps 0..7 consume (256 threads), warp 8 produces (one lane
+// walks the chunk sequence, waits until a slot is released -- `empty`
+// mbarrier, one arrival per reading warp -- and refills it), warps 9..12
+// prepare (128 threads): for each pair, as soon as its key chunk and token
+// have landed, they form phi_q, phi_k, the decay gamma and the meta logits
+// into a two-entry record ring, so that the consumers of the pair before
+// are not held up by that work.  Consumers meet on named barrier 1, the
+// prep warps on named barrier 2, only where data flows between them.
 constexpr int kConsumers = 256;
+constexpr int kPrep = 128;
+constexpr int kDecThreads = kConsumers + 32 + kPrep;
 LZ_DEV void s_mbar_arrive(uint64_t *bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(s_addr(bar)) : "memory");
 }
@@ -415,6 +420,17 @@ LZ_DEV void s_mbar_init_n(uint64_t *bar, uint32_t n) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(s_addr(bar)), "r"(n) : "memory");
 }
 LZ_DEV void consumers_sync() { asm volatile("bar.sync 1, %0;\n" ::"n"(kConsumers) : "memory"); }
+LZ_DEV void prep_sync() { asm volatile("bar.sync 2, %0;\n" ::"n"(kPrep) : "memory"); }
+// Barrier over the prep warps that also returns whether any of them passed true.
+LZ_DEV bool prep_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, 2, %2, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"((uint32_t)v), "n"(kPrep)
+      : "memory");
+  return r != 0;
+}
 // Barrier over the consumers that also returns whether any of them passed true.
 LZ_DEV bool consumers_any(bool v) {
   uint32_t r;
@@ -426,19 +442,25 @@ LZ_DEV bool consumers_any(bool v) {
   return r != 0;
 }
 
-__global__ void __launch_bounds__(kConsumers + 32, 1) decode_stream_kernel(const __grid_constant__ DecodeArgs p, int B, int run) {
+struct PairRec {                 // what the prep warps hand to the consumers for one pair
+  float phq[SD], phk[SD], gam[SD], ml[16];
+};
+
+__global__ void __launch_bounds__(kDecThreads, 1) decode_stream_kernel(const __grid_constant__ DecodeArgs p, int B, int run) {
   extern __shared__ __align__(1024) unsigned char dsm[];
   unsigned char *ring = dsm + kRingOff;
   float *Wq = reinterpret_cast<float *>(dsm + kWOff), *Wk = Wq + SD * SF;
   __nv_bfloat16 *tokring = reinterpret_cast<__nv_bfloat16 *>(dsm + kTokOff);
   float *mk_s = reinterpret_cast<float *>(dsm + kMetaOff), *mv_s = mk_s + p.M * SD;
   __shared__ uint64_t full[kStreamSlots], empty[kStreamSlots];
-  __shared__ uint64_t wfull, wempty;
-  __shared__ float xq[SD], xk[SD], xv[SD], gam[SD], phq[SD], phk[SD];
-  __shared__ __align__(16) float zpart[2][8][SF];   // z partials, later the read-out partials [8][128]
+  __shared__ uint64_t wfull, wempty, rfull[2], rempty[2];
+  __shared__ PairRec rec[2];
+  __shared__ float xk_c[SD], xv_c[SD];               // the consumers' copy of the token's k, v
+  __shared__ __align__(16) float zpart[8][SD];       // read-out partials per row group
   __shared__ float prob[128 + 16];
   __shared__ float red[8][SD];
   __shared__ float s_inv;
+  __shared__ float p_red[4][2];                      // prep: per-warp maxima, then sums
   __shared__ int s_n[kMaxRunPairs], s_slot[kMaxRunPairs];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int BH = B * p.H;
@@ -451,12 +473,18 @@ __global__ void __launch_bounds__(kConsumers + 32, 1) decode_stream_kernel(const
     s_slot[k] = (int)(pos % p.window);
   }
   if (tid == 0) {
+    // slot 0 always holds a key chunk and its token (4 chunks per pair, 4
+    // slots): the prep warps read it too
     for (int i = 0; i < kStreamSlots; ++i) {
       s_mbar_init_n(&full[i], 1);
-      s_mbar_init_n(&empty[i], kConsumers / 32);
+      s_mbar_init_n(&empty[i], kConsumers / 32 + (i == 0 ? kPrep / 32 : 0));
     }
     s_mbar_init_n(&wfull, 1);
-    s_mbar_init_n(&wempty, kConsumers / 32);
+    s_mbar_init_n(&wempty, kConsumers / 32 + kPrep / 32);
+    for (int i = 0; i < 2; ++i) {
+      s_mbar_init_n(&rfull[i], kPrep / 32);
+      s_mbar_init_n(&rempty[i], kConsumers / 32);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
   __syncthreads();
@@ -470,7 +498,7 @@ __global__ void __launch_bounds__(kConsumers + 32, 1) decode_stream_kernel(const
         const PairInfo pi = pair_info(p, B, first, c >> 2, s_n, s_slot);
         const int kind = c & 3, sl = c % kStreamSlots;
         if (kind == 0 && pi.h != prev_head) {
-          // weights and meta tokens of the next head, once the consumers are
+          // weights and meta tokens of the next head, once every reader is
           // done with the current ones
           if (nh > 0) ok = s_mbar_wait(&wempty, (uint32_t)(nh - 1) & 1u);
           if (!ok) break;
@@ -511,6 +539,84 @@ __global__ void __launch_bounds__(kConsumers + 32, 1) decode_stream_kernel(const
     return;
   }
 
+  if (warp > kConsumers / 32) {
+    // ----------------------------------------------------------- prep ---
+    const int pt = tid - (kConsumers + 32), pw = pt >> 5;
+    const __nv_bfloat16 *tk = tokring;   // slot 0
+    int cur_head = -1, nh = 0;
+    for (int k = 0; k < npairs; ++k) {
+      const PairInfo pi = pair_info(p, B, first, k, s_n, s_slot);
+      bool ok = s_mbar_wait(&full[0], (uint32_t)k & 1u);
+      if (pi.h != cur_head) {
+        ok &= s_mbar_wait(&wfull, (uint32_t)nh & 1u);
+        ++nh;
+        cur_head = pi.h;
+      }
+      if (k >= 2) ok &= s_mbar_wait(&rempty[k & 1], (uint32_t)((k >> 1) - 1) & 1u);
+      if (prep_any(!ok)) {   // all prep warps stop together; the consumers time out on the record
+        atomicOr(&g_decode_status, 1u);
+        return;
+      }
+      PairRec &R = rec[k & 1];
+      R.gam[pt] = expf(log_decay(__bfloat162float(tk[3 * SD + pt]), p.inv_tau));
+      // z = x W: thread = (map, feature); 4 partial sums over the 128 rows
+      const int map = pt >> 6, f = pt & 63;
+      const __nv_bfloat16 *x = tk + map * SD;
+      const float *W = map == 0 ? Wq : Wk;
+      const bool has_w = map == 0 ? p.wq != nullptr : p.wk != nullptr;
+      float z = 0.f;
+      if (has_w) {
+        float a4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+        for (int i = 0; i < SD; ++i) a4[i & 3] = fmaf(__bfloat162float(x[i]), W[i * SF + f], a4[i & 3]);
+        z = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+      }
+      // phi = [softmax(z), softmax(-z)] over the 64 features of this map
+      // (two warps per map meet through p_red)
+      float mx = warp_max(z), mn = warp_max(-z);
+      if (lane == 0) { p_red[pw][0] = mx; p_red[pw][1] = mn; }
+      prep_sync();
+      mx = fmaxf(p_red[pw][0], p_red[pw ^ 1][0]);
+      mn = fmaxf(p_red[pw][1], p_red[pw ^ 1][1]);
+      const float ep = expf(z - mx), en = expf(-z - mn);
+      const float sp = warp_sum(ep), sn = warp_sum(en);
+      prep_sync();
+      if (lane == 0) { p_red[pw][0] = sp; p_red[pw][1] = sn; }
+      prep_sync();
+      const float isp = 1.f / (p_red[pw][0] + p_red[pw ^ 1][0]);
+      const float isn = 1.f / (p_red[pw][1] + p_red[pw ^ 1][1]);
+      float *ph = map == 0 ? R.phq : R.phk;
+      if (has_w) {
+        ph[f] = ep * isp;
+        ph[SF + f] = en * isn;
+      } else {   // identity map
+        ph[f] = __bfloat162float(x[f]);
+        ph[SF + f] = __bfloat162float(x[SF + f]);
+      }
+      // meta logits: thread = (meta token m, 16 dimensions), 8 lanes per token
+      {
+        const int m = pt >> 3, part = pt & 7;
+        float d = 0.f;
+        if (m < p.M) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) d = fmaf(__bfloat162float(tk[part * 16 + i]), mk_s[m * SD + part * 16 + i], d);
+        }
+        d += __shfl_xor_sync(0xffffffffu, d, 4);
+        d += __shfl_xor_sync(0xffffffffu, d, 2);
+        d += __shfl_xor_sync(0xffffffffu, d, 1);
+        if (m < p.M && part == 0) R.ml[m] = d * p.scale;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        s_mbar_arrive(&rfull[k & 1]);
+        s_mbar_arrive(&empty[0]);   // the token and the weights are read
+        if (k + 1 >= npairs || pair_info(p, B, first, k + 1, s_n, s_slot).h != pi.h) s_mbar_arrive(&wempty);
+      }
+      prep_sync();   // p_red is reused by the next pair
+    }
+    return;
+  }
+
   // ---------------------------------------------------------- consumers ---
   const int cg = tid & 31, rg = tid >> 5;   // state: float4 column group, row group (8 rows)
   const int vg = tid & 15, eg = tid >> 4;   // values: 8 columns, slot group
@@ -520,17 +626,18 @@ __global__ void __launch_bounds__(kConsumers + 32, 1) decode_stream_kernel(const
   int c_stop = nchunks;
   PairInfo pi{0, 0, 0, 0};
   for (int c = 0; c < nchunks; ++c) {
-    const int kind = c & 3, sl = c % kStreamSlots;
+    const int kind = c & 3, sl = c % kStreamSlots, kp = c >> 2;
     const unsigned char *chunk = ring + (size_t)sl * kChunkBytes;
     bool new_head = false;
     if (kind == 0) {
-      pi = pair_info(p, B, first, c >> 2, s_n, s_slot);
+      pi = pair_info(p, B, first, kp, s_n, s_slot);
       new_head = pi.h != cur_head;
       acc = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     bool ok = s_mbar_wait(&full[sl], (uint32_t)(c / kStreamSlots) & 1u);
+    if (kind == 0) ok &= s_mbar_wait(&rfull[kp & 1], (uint32_t)(kp >> 1) & 1u);
     if (new_head) {
-      ok &= s_mbar_wait(&wfull, (uint32_t)nh & 1u);
+      ok &= s_mbar_wait(&wfull, (uint32_t)nh & 1u);   // meta values
       ++nh;
       cur_head = pi.h;
     }
@@ -539,38 +646,19 @@ __global__ void __launch_bounds__(kConsumers + 32, 1) decode_stream_kernel(const
       failed = true;
     }
     // A failed (bounded) wait inside a pair only leaves stale slot data; the
-    // consumers decide together, at the next pair, to stop.
+    // consumers decide together, at the next pair, to stop.  The vote is
+    // also the barrier that ends the previous pair's read-out.
     if (kind == 0 && consumers_any(failed)) {
       c_stop = c;
       break;
     }
     const int n = pi.n, slot = pi.slot, h = pi.h, bh = pi.bh;
+    const PairRec &R = rec[kp & 1];
     if (kind == 0) {
-      // ---- token vectors and decay (the token rode along with this chunk);
-      //      the vote above also ends the previous pair's read-out
       const __nv_bfloat16 *tk = tokring + (size_t)sl * 4 * SD;
-      if (tid < SD) {
-        xq[tid] = __bfloat162float(tk[tid]);
-        xk[tid] = __bfloat162float(tk[SD + tid]);
-        xv[tid] = __bfloat162float(tk[2 * SD + tid]);
-        gam[tid] = expf(log_decay(__bfloat162float(tk[3 * SD + tid]), p.inv_tau));
-      }
-      consumers_sync();
-      {   // z = x W from shared memory: thread = (map, 4 features, 16 rows of W)
-        const int map = tid >> 7, r = tid & 127, fg = r & 15, ip = r >> 4;
-        const float *Wm = map == 0 ? Wq : Wk;
-        const float *x = map == 0 ? xq : xk;
-        float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float4 wv = *reinterpret_cast<const float4 *>(Wm + (ip * 16 + i) * SF + fg * 4);
-          const float xi = x[ip * 16 + i];
-          z.x = fmaf(xi, wv.x, z.x);
-          z.y = fmaf(xi, wv.y, z.y);
-          z.z = fmaf(xi, wv.z, z.z);
-          z.w = fmaf(xi, wv.w, z.w);
-        }
-        *reinterpret_cast<float4 *>(&zpart[map][ip][fg * 4]) = z;
+      if (tid < SD) {   // keep k and v: the token slot is refilled once everyone has read it
+        xk_c[tid] = __bfloat162float(tk[SD + tid]);
+        xv_c[tid] = __bfloat162float(tk[2 * SD + tid]);
       }
       // ---- window logits: two threads per slot (64 dimensions each); the
       //      slot being replaced takes the new key
@@ -578,19 +666,17 @@ __global__ void __launch_bounds__(kConsumers + 32, 1) decode_stream_kernel(const
         const int j = tid >> 1, half = tid & 1;
         float d = 0.f;
         if (j < n) {
-          const __nv_bfloat16 *kr = reinterpret_cast<const __nv_bfloat16 *>(chunk) + (size_t)j * SD + half * 64;
-          if (j == slot) {
-#pragma unroll 8
-            for (int i = 0; i < 64; ++i) d = fmaf(xq[half * 64 + i], xk[half * 64 + i], d);
-          } else {
+          const __nv_bfloat16 *kr = j == slot ? tk + SD + half * 64
+                                              : reinterpret_cast<const __nv_bfloat16 *>(chunk) + (size_t)j * SD + half * 64;
+          const __nv_bfloat16 *qr = tk + half * 64;
 #pragma unroll
-            for (int c0 = 0; c0 < 8; ++c0) {
-              const int cc = (c0 + j) & 7;   // spread a warp's reads over the banks
-              float kv[8];
-              load8(kr + cc * 8, kv);
+          for (int c0 = 0; c0 < 8; ++c0) {
+            const int cc = (c0 + j) & 7;   // spread a warp's reads over the banks
+            float kv[8], q8[8];
+            load8(kr + cc * 8, kv);
+            load8(qr + cc * 8, q8);
 #pragma unroll
-              for (int u = 0; u < 8; ++u) d = fmaf(xq[half * 64 + cc * 8 + u], kv[u], d);
-            }
+            for (int u = 0; u < 8; ++u) d = fmaf(q8[u], kv[u], d);
           }
         }
         d += __shfl_xor_sync(0xffffffffu, d, 1);
@@ -599,68 +685,24 @@ __global__ void __launch_bounds__(kConsumers + 32, 1) decode_stream_kernel(const
       __syncwarp();
       if (lane == 0) s_mbar_arrive(&empty[sl]);   // the key window and the token are read
       consumers_sync();
-      if (warp < 2) {   // feature maps from the z partials
-        const int map = warp;
-        const bool has_w = map == 0 ? p.wq != nullptr : p.wk != nullptr;
-        float *out = map == 0 ? phq : phk;
-        const float *x = map == 0 ? xq : xk;
-        if (!has_w) {
-          for (int i = lane; i < SD; i += 32) out[i] = x[i];
-        } else {
-          float z[2], mx = kNegBig, mn = -kNegBig;
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            float a = 0.f;
-#pragma unroll
-            for (int pp = 0; pp < 8; ++pp) a += zpart[map][pp][lane + 32 * j];
-            z[j] = a;
-            mx = fmaxf(mx, a);
-            mn = fminf(mn, a);
-          }
-          mx = warp_max(mx);
-          mn = -warp_max(-mn);
-          float ep[2], en[2], sp = 0.f, sn = 0.f;
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            ep[j] = expf(z[j] - mx);
-            en[j] = expf(mn - z[j]);
-            sp += ep[j];
-            sn += en[j];
-          }
-          sp = 1.f / warp_sum(sp);
-          sn = 1.f / warp_sum(sn);
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            out[lane + 32 * j] = ep[j] * sp;
-            out[SF + lane + 32 * j] = en[j] * sn;
-          }
-        }
-      } else if (warp == 2) {   // meta logits, then the softmax over n + M
-        for (int m = 0; m < p.M; ++m) {
-          float d = 0.f;
-#pragma unroll
-          for (int i = lane; i < SD; i += 32) d = fmaf(xq[i], mk_s[m * SD + i], d);
-          d = warp_sum(d);
-          if (lane == 0) prob[n + m] = d * p.scale;
-        }
-        __syncwarp();
+      if (warp == 0) {   // softmax over the n window logits and the M meta logits
         const int ntot = n + p.M;
         float mx = kNegBig;
-        for (int j = lane; j < ntot; j += 32) mx = fmaxf(mx, prob[j]);
+        for (int j = lane; j < ntot; j += 32) mx = fmaxf(mx, j < n ? prob[j] : R.ml[j - n]);
         mx = warp_max(mx);
         float sum = 0.f;
         for (int j = lane; j < ntot; j += 32) {
-          const float e = expf(prob[j] - mx);
+          const float e = expf((j < n ? prob[j] : R.ml[j - n]) - mx);
           prob[j] = e;
           sum += e;
         }
         sum = warp_sum(sum);
         if (lane == 0) s_inv = 1.f / sum;
       }
-      consumers_sync();   // phi_q, phi_k and the probabilities are ready
+      consumers_sync();   // the probabilities are ready
     } else if (kind == 1 || kind == 2) {
       // ---- state rows (kind - 1) * 64 .. + 63: update, store, read out
-      const float4 v4 = make_float4(xv[cg * 4], xv[cg * 4 + 1], xv[cg * 4 + 2], xv[cg * 4 + 3]);
+      const float4 v4 = make_float4(xv_c[cg * 4], xv_c[cg * 4 + 1], xv_c[cg * 4 + 2], xv_c[cg * 4 + 3]);
       float *S = p.state + (size_t)bh * SD * SD;
       float4 sv[8];
 #pragma unroll
@@ -670,7 +712,7 @@ __global__ void __launch_bounds__(kConsumers + 32, 1) decode_stream_kernel(const
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
         const int i = (kind - 1) * 64 + rg * 8 + r;
-        const float gi = gam[i], ki = phk[i], qi = phq[i];
+        const float gi = R.gam[i], ki = R.phk[i], qi = R.phq[i];
         float4 s = sv[r];
         s.x = fmaf(gi, s.x, ki * v4.x);
         s.y = fmaf(gi, s.y, ki * v4.y);
@@ -682,6 +724,10 @@ __global__ void __launch_bounds__(kConsumers + 32, 1) decode_stream_kernel(const
         acc.z = fmaf(qi, s.z, acc.z);
         acc.w = fmaf(qi, s.w, acc.w);
       }
+      if (kind == 2) {   // the record of this pair is no longer read
+        __syncwarp();
+        if (lane == 0) s_mbar_arrive(&rempty[kp & 1]);
+      }
     } else {
       // ---- o_swa = sum_j p_j v_j (+ meta values); the replaced slot takes
       //      the new value; then o = o_gla + alpha o_swa / l
@@ -692,7 +738,7 @@ __global__ void __launch_bounds__(kConsumers + 32, 1) decode_stream_kernel(const
         float vv[8];
         if (j == slot) {
 #pragma unroll
-          for (int u = 0; u < 8; ++u) vv[u] = xv[vg * 8 + u];
+          for (int u = 0; u < 8; ++u) vv[u] = xv_c[vg * 8 + u];
         } else {
           load8(reinterpret_cast<const __nv_bfloat16 *>(chunk) + (size_t)j * SD + vg * 8, vv);
         }
@@ -709,29 +755,29 @@ __global__ void __launch_bounds__(kConsumers + 32, 1) decode_stream_kernel(const
           for (int u = 0; u < 8; ++u) a8[u] = fmaf(pj, mv_s[m * SD + vg * 8 + u], a8[u]);
         }
       __syncwarp();
-      if (lane == 0 && ((c >> 2) + 1 >= npairs || pair_info(p, B, first, (c >> 2) + 1, s_n, s_slot).h != h))
-        s_mbar_arrive(&wempty);   // last pair of this head: its weights and meta tokens are read
+      if (lane == 0 && (kp + 1 >= npairs || pair_info(p, B, first, kp + 1, s_n, s_slot).h != h))
+        s_mbar_arrive(&wempty);   // last pair of this head: its meta values are read
 #pragma unroll
       for (int u = 0; u < 8; ++u) a8[u] += __shfl_xor_sync(0xffffffffu, a8[u], 16);
       if (lane < 16)
 #pragma unroll
         for (int u = 0; u < 8; ++u) red[warp][vg * 8 + u] = a8[u];
       // the read-out partials of the two state chunks, per row group
-      *reinterpret_cast<float4 *>(&zpart[0][0][0] + rg * SD + cg * 4) = acc;
+      *reinterpret_cast<float4 *>(&zpart[rg][cg * 4]) = acc;
       consumers_sync();
       if (tid < SD) {
         float so = 0.f, sg = 0.f;
 #pragma unroll
         for (int w = 0; w < 8; ++w) so += red[w][tid];
 #pragma unroll
-        for (int r = 0; r < 8; ++r) sg += (&zpart[0][0][0])[r * SD + tid];
+        for (int r = 0; r < 8; ++r) sg += zpart[r][tid];
         const float alpha = p.alpha ? p.alpha[h] : 1.f;
         static_cast<__nv_bfloat16 *>(p.o)[(size_t)bh * SD + tid] = __float2bfloat16_rn(sg + alpha * so * s_inv);
-        // the new token enters the ring (both windows were read above); xk
-        // and xv hold it exactly (bf16 -> fp32 -> bf16 is lossless)
+        // the new token enters the ring (both windows were read above); the
+        // fp32 copies hold it exactly (bf16 -> fp32 -> bf16 is lossless)
         const size_t cw = ((size_t)bh * p.window + slot) * SD + tid;
-        static_cast<__nv_bfloat16 *>(p.k_cache)[cw] = __float2bfloat16_rn(xk[tid]);
-        static_cast<__nv_bfloat16 *>(p.v_cache)[cw] = __float2bfloat16_rn(xv[tid]);
+        static_cast<__nv_bfloat16 *>(p.k_cache)[cw] = __float2bfloat16_rn(xk_c[tid]);
+        static_cast<__nv_bfloat16 *>(p.v_cache)[cw] = __float2bfloat16_rn(xv_c[tid]);
       }
     }
   }
@@ -769,7 +815,7 @@ cudaError_t launch_decode_stream(const DecodeArgs &a, int B, int64_t *pos, cudaS
   const int BH = B * a.H;
   const int run = (BH + sms[dev] - 1) / sms[dev];   // pairs per CTA
   const int grid = (BH + run - 1) / run;
-  decode_stream_kernel<<<grid, kConsumers + 32, smem, s>>>(a, B, run);
+  decode_stream_kernel<<<grid, kDecThreads, smem, s>>>(a, B, run);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   advance_pos_kernel<<<(B + 127) / 128, 128, 0, s>>>(pos, B);
