@@ -472,6 +472,21 @@ lizard_status lizard_decode_step(const lizard_decode_args *a, lizard_stream_t st
   return cuda_status(lz::launch_decode(d, a->B, a->dk, bf16, a->pos, s));
 }
 
+lizard_status lizard_prefill_cache(const lizard_cache_args *a, lizard_stream_t stream) {
+  if (!a) return LIZARD_ERR_INVALID_ARG;
+  if (a->B < 1 || a->H < 1 || a->L < 0 || a->dk <= 0 || a->dv <= 0 || a->window < 1) return LIZARD_ERR_INVALID_ARG;
+  if (a->dtype != LIZARD_BF16 && a->dtype != LIZARD_FP32) return LIZARD_ERR_INVALID_ARG;
+  if (a->dk != a->dv || (a->dk != 64 && a->dk != 128) || a->window > 16384) return LIZARD_ERR_UNSUPPORTED;
+  if (!a->k_cache || !a->v_cache || !a->pos || (a->L > 0 && (!a->k || !a->v))) return LIZARD_ERR_INVALID_ARG;
+  const void *ptrs[] = {a->k, a->v, a->k_cache, a->v_cache, a->pos};
+  for (const void *p : ptrs)
+    if (!ok_ptr(p)) return LIZARD_ERR_INVALID_ARG;
+  const size_t esz = a->dtype == LIZARD_BF16 ? 2 : 4;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return cuda_status(lz::launch_prefill_cache(a->k, a->v, a->k_cache, a->v_cache, a->pos, a->B, a->H, a->L,
+                                              a->window, a->dk * esz, a->dv * esz, s));
+}
+
 lizard_status lizard_decode_status(void) {
   if (cudaDeviceSynchronize() != cudaSuccess) return LIZARD_ERR_CUDA;
   const int v = lz::decode_stream_status_take();

@@ -822,6 +822,31 @@ cudaError_t launch_decode_stream(const DecodeArgs &a, int B, int64_t *pos, cudaS
   return cudaGetLastError();
 }
 
+// Window caches from a prefix: slot s of sequence (b, h) receives the last
+// prefix token t < L with t mod W == s (zeros when no token reached it);
+// pos[b] = L.  Thread = one 16-byte vector of a slot's key and value rows.
+__global__ void prefill_cache_kernel(const uint4 *k, const uint4 *v, uint4 *kc, uint4 *vc, int64_t *pos, int L,
+                                     int W, int vec_k, int vec_v, int H) {
+  const int s = blockIdx.x, bh = blockIdx.y;
+  const int t = s < L ? s + W * ((L - 1 - s) / W) : -1;
+  for (int e = threadIdx.x; e < vec_k + vec_v; e += blockDim.x) {
+    const bool isk = e < vec_k;
+    const int u = isk ? e : e - vec_k, vec = isk ? vec_k : vec_v;
+    const uint4 *src = isk ? k : v;
+    uint4 *dst = isk ? kc : vc;
+    dst[((size_t)bh * W + s) * vec + u] = t >= 0 ? src[((size_t)bh * L + t) * vec + u] : make_uint4(0u, 0u, 0u, 0u);
+  }
+  if (s == 0 && threadIdx.x == 0 && bh % H == 0) pos[bh / H] = L;
+}
+
+cudaError_t launch_prefill_cache(const void *k, const void *v, void *kc, void *vc, int64_t *pos, int B, int H,
+                                 int L, int W, size_t row_bytes_k, size_t row_bytes_v, cudaStream_t s) {
+  prefill_cache_kernel<<<dim3(W, B * H), 128, 0, s>>>(
+      static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), static_cast<uint4 *>(kc),
+      static_cast<uint4 *>(vc), pos, L, W, (int)(row_bytes_k / 16), (int)(row_bytes_v / 16), H);
+  return cudaGetLastError();
+}
+
 int decode_stream_status_take() {
   uint32_t v = 0;
   if (cudaMemcpyFromSymbol(&v, g_decode_status, sizeof(v)) != cudaSuccess) return -1;

@@ -153,6 +153,9 @@ cudaError_t launch_decode(const DecodeArgs &a, int B, int D, bool bf16, int64_t 
 // Persistent streaming decode for bf16, d = 128, window <= 128, M <= 16.
 bool decode_stream_supported(int D, bool bf16, int window, int M);
 cudaError_t launch_decode_stream(const DecodeArgs &a, int B, int64_t *pos, cudaStream_t s);
+// Prefill -> decode handoff of the window caches (rows are 16-byte multiples).
+cudaError_t launch_prefill_cache(const void *k, const void *v, void *kc, void *vc, int64_t *pos, int B, int H,
+                                 int L, int W, size_t row_bytes_k, size_t row_bytes_v, cudaStream_t s);
 // The streaming kernel's timeout flag (bit 1), cleared by reading; -1 on error.
 int decode_stream_status_take();
 

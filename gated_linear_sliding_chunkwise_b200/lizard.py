@@ -77,6 +77,14 @@ _lib.lizard_bwd_launch_plan.argtypes = [ctypes.POINTER(BwdArgs), ctypes.POINTER(
 _lib.lizard_bwd_launch_plan.restype = _i32
 _lib.lizard_decode_step.argtypes = [ctypes.POINTER(DecodeArgs), _vp]
 _lib.lizard_decode_step.restype = ctypes.c_int
+class CacheArgs(ctypes.Structure):
+    _fields_ = [("B", _i32), ("H", _i32), ("L", _i32), ("dk", _i32), ("dv", _i32), ("window", _i32),
+                ("dtype", _i32), ("k", _vp), ("v", _vp), ("k_cache", _vp), ("v_cache", _vp),
+                ("pos", _vp)]
+
+
+_lib.lizard_prefill_cache.argtypes = [ctypes.POINTER(CacheArgs), _vp]
+_lib.lizard_prefill_cache.restype = ctypes.c_int
 _lib.lizard_decode_status.argtypes = []
 _lib.lizard_decode_status.restype = ctypes.c_int
 _lib.lizard_workspace_status.argtypes = [_vp, _vp]
@@ -295,3 +303,16 @@ def decode_status() -> int:
     """Timeout flag of the decode steps run on the current device since the
     last call (OK or ERR_TIMEOUT); reading clears it and synchronises."""
     return int(_lib.lizard_decode_status())
+
+
+def prefill_cache(k, v, k_cache, v_cache, pos, stream=None):
+    """Prefill -> decode handoff (lizard_prefill_cache): fill the window
+    caches from the prefix keys and values k, v [B, H, L, d] and set
+    pos = L, in place."""
+    B, H, L, dk = k.shape
+    a = CacheArgs()
+    a.B, a.H, a.L, a.dk, a.dv, a.window = B, H, L, dk, v.shape[-1], k_cache.shape[2]
+    a.dtype = _dtype_code(k)
+    a.k, a.v = _ptr(k), _ptr(v)
+    a.k_cache, a.v_cache, a.pos = _ptr(k_cache), _ptr(v_cache), _ptr(pos)
+    _check(_lib.lizard_prefill_cache(ctypes.byref(a), _stream(stream)), "lizard_prefill_cache")

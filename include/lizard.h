@@ -215,6 +215,31 @@ typedef struct {
 lizard_status lizard_decode_step(const lizard_decode_args *args, lizard_stream_t stream);
 
 /*
+ * Prefill -> decode handoff: after lizard_attn_fwd over a prefix of L tokens
+ * (its state_out is the decode state), fill the decode window caches from
+ * the prefix so that lizard_decode_step continues the sequence (the
+ * constant-memory generation of the English summary, section 2.A, with the
+ * fixed-size cache of the Chinese summary, section 2.1).
+ *
+ *   k, v       [B, H, L, dk|dv] dtype: the prefix's keys and values
+ *   k_cache    [B, H, window, dk] dtype, v_cache [B, H, window, dv] dtype,
+ *              written: token t of the last min(L, window) goes to slot
+ *              t mod window (the slot lizard_decode_step would have used);
+ *              slots no token reached are zeroed
+ *   pos        [B] int64, written: L
+ * L = 0 clears the caches.  No workspace.  Errors as lizard_decode_step.
+ */
+typedef struct {
+  int32_t B, H, L, dk, dv, window;
+  int32_t dtype;
+  const void *k, *v;
+  void *k_cache, *v_cache;
+  int64_t *pos;
+} lizard_cache_args;
+
+lizard_status lizard_prefill_cache(const lizard_cache_args *args, lizard_stream_t stream);
+
+/*
  * Status of the decode steps run on the current device since the last call:
  * LIZARD_ERR_TIMEOUT when a step's bounded wait for its own copies gave up
  * (its outputs are then undefined), else LIZARD_OK; LIZARD_ERR_CUDA when

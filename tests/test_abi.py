@@ -47,7 +47,7 @@ def test_struct_layouts_match_c(lz, tmp_path):
     """Compile a C program against the header and compare sizeof/offsetof."""
     fields = {
         "lizard_fwd_args": lz.FwdArgs, "lizard_bwd_args": lz.BwdArgs,
-        "lizard_decode_args": lz.DecodeArgs,
+        "lizard_decode_args": lz.DecodeArgs, "lizard_cache_args": lz.CacheArgs,
     }
     lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "lizard.h"',
              "int main(void) {"]
@@ -166,3 +166,11 @@ def test_decode_rejects_bad_arguments_on_host(lz):
     d.pos = fake
     d.M = 2                    # meta tokens without meta keys
     assert lz.lib().lizard_decode_step(ctypes.byref(d), None) == lz.ERR_INVALID_ARG
+
+
+def test_prefill_cache_rejects_bad_arguments_on_host(lz):
+    a = lz.CacheArgs()
+    a.B, a.H, a.L, a.dk, a.dv, a.window, a.dtype = 1, 1, 4, 128, 128, 8, lz.BF16
+    assert lz.lib().lizard_prefill_cache(ctypes.byref(a), None) == lz.ERR_INVALID_ARG   # no buffers
+    a.dk = a.dv = 96
+    assert lz.lib().lizard_prefill_cache(ctypes.byref(a), None) == lz.ERR_UNSUPPORTED

@@ -127,3 +127,42 @@ def test_decode_streaming_without_meta_values_and_status(lz):
     assert torch.equal(x["k_cache"].cpu(), torch.from_numpy(want[2]).to(x["k_cache"].dtype))
     assert torch.equal(x["v_cache"].cpu(), torch.from_numpy(want[3]).to(x["v_cache"].dtype))
     assert lz.decode_status() == lz.OK
+
+
+@pytest.mark.parametrize("dtype,d,window,L0", [("bf16", 128, 128, 300), ("bf16", 128, 64, 37),
+                                                ("fp32", 64, 12, 50), ("bf16", 128, 32, 0)])
+def test_prefill_handoff_then_decode(lz, dtype, d, window, L0):
+    """Forward over a prefix of L0 tokens (its end state) and lizard_prefill_cache
+    (its window), then decode steps: every decoded output equals the whole
+    sequence's forward at that position (oracle), and pos advances from L0."""
+    B, H, Ld = 2, 2, 6
+    L = L0 + Ld
+    w = Workload("handoff", B=B, H=H, L=L, d=d, window=window, M=4, dtype=dtype, seed=L0 + d)
+    inp = make_inputs(w)
+    x = to_device(inp)
+    par = dict(fmap_wq=x["fmap_wq"], fmap_wk=x["fmap_wk"], meta_k=x["meta_k"], meta_v=x["meta_v"],
+               alpha=x["alpha"])
+    pre = {n: x[n][:, :, :L0].contiguous() for n in ("q", "k", "v", "g")}
+    dt = x["q"].dtype
+    if L0 > 0:
+        fwd = lz.attn_fwd(pre["q"], pre["k"], pre["v"], pre["g"], window=window, gate_temp=w.gate_temp,
+                          want_state=True, **par)
+        state = fwd["state_out"]
+    else:
+        state = torch.zeros(B, H, d, d, device="cuda")
+    kc = torch.full((B, H, window, d), 7.0, dtype=dt, device="cuda")   # stale contents
+    vc = torch.full((B, H, window, d), 7.0, dtype=dt, device="cuda")
+    pos = torch.full((B,), 99, dtype=torch.int64, device="cuda")
+    lz.prefill_cache(pre["k"], pre["v"], kc, vc, pos)
+    torch.cuda.synchronize()
+    assert torch.equal(pos.cpu(), torch.full((B,), L0, dtype=torch.int64))
+    st = {"state": state, "k_cache": kc, "v_cache": vc, "pos": pos}
+    outs = []
+    for t in range(L0, L):
+        step = {n: x[n][:, :, t].contiguous() for n in ("q", "k", "v", "g")}
+        outs.append(_gpu_step(lz, {**step, **par, **st}, w))
+    dec = torch.stack(outs, 2)
+    torch.cuda.synchronize()
+    want = oracle_forward(inp, window=window, tau=w.gate_temp)
+    check("decode after prefill", dec, want["o"][:, :, L0:], dtype)
+    assert torch.equal(pos.cpu(), torch.full((B,), L, dtype=torch.int64))
