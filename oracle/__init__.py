@@ -7,6 +7,7 @@ product path (the CUDA library and its Python binding) never does.
 
 from .lizard_ref import (  # noqa: F401
     gate_log_decay,
+    layer_log_decay,
     feature_map,
     feature_map_backward,
     gla_forward,
@@ -19,4 +20,6 @@ from .lizard_ref import (  # noqa: F401
     BRANCH_BOTH,
     BRANCH_GLA_ONLY,
     BRANCH_SWA_ONLY,
+    GATE_PER_DIM,
+    GATE_SCALAR,
 )

@@ -25,6 +25,10 @@ What the pages fix, and the reading taken where they are silent:
   the inputs are the gate logits g.  The log-decay is
   a_t = logsigmoid(g_t) / tau per key dimension, with tau a temperature
   (tau = 1 gives the pages' literal sigmoid gate; the workloads use 16).
+* Gate granularity: per key dimension (g [B,H,L,dk]) by default.  The
+  Chinese summary's ablation ([ZH] 4, "消融实验") finds a light scalar gate
+  the most effective; gate="scalar" takes one logit per token and head
+  (g [B,H,L]) whose decay applies to every key dimension.
 * State update: S_t = diag(Gamma_t) S_{t-1} + phi(k_t) v_t^T ([EN] 2.A
   "State Update").  Read-out (a reading): o_t = S_t^T phi(q_t), with S_t
   already containing token t.  No normaliser.  The recurrence spans the
@@ -61,6 +65,9 @@ BRANCH_BOTH = 0
 BRANCH_GLA_ONLY = 1
 BRANCH_SWA_ONLY = 2
 
+GATE_PER_DIM = "dim"
+GATE_SCALAR = "scalar"
+
 
 def _f64(x):
     return None if x is None else np.asarray(x, dtype=np.float64)
@@ -79,6 +86,21 @@ def gate_log_decay(g, tau=16.0):
     """
     g = _f64(g)
     return (np.minimum(g, 0.0) - np.log1p(np.exp(-np.abs(g)))) / float(tau)
+
+
+def layer_log_decay(g, tau, gate, dk):
+    """The per-dimension log-decay a [..., dk] the recurrence uses.
+
+    gate="dim": g [..., dk], a = logsigmoid(g)/tau elementwise.
+    gate="scalar": g [...] (one logit per token and head, [ZH] 4 ablation);
+    every key dimension decays by the same logsigmoid(g)/tau.
+    """
+    a = gate_log_decay(g, tau)
+    if gate == GATE_SCALAR:
+        return np.repeat(a[..., None], dk, axis=-1)
+    if gate != GATE_PER_DIM:
+        raise ValueError(f"gate must be {GATE_PER_DIM!r} or {GATE_SCALAR!r}")
+    return a
 
 
 def _softmax_last(z):
@@ -293,7 +315,8 @@ def _defaults(q, alpha, scale, meta_k):
 
 def lizard_forward(q, k, v, g, *, window, tau=16.0, scale=None,
                    fmap_wq=None, fmap_wk=None, meta_k=None, meta_v=None,
-                   alpha=None, state_in=None, branch=BRANCH_BOTH):
+                   alpha=None, state_in=None, branch=BRANCH_BOTH,
+                   gate=GATE_PER_DIM):
     """Hybrid layer forward: o = o_gla + alpha_h * o_swa.
 
     Mixing rule: [FR] 2.A last line, [EN] 2.A "Final Output".  `branch`
@@ -309,7 +332,7 @@ def lizard_forward(q, k, v, g, *, window, tau=16.0, scale=None,
     out = {"o": np.zeros(v.shape), "state_out": None, "lse": None,
            "o_gla": None, "o_swa": None}
     if branch != BRANCH_SWA_ONLY:
-        a = gate_log_decay(g, tau)
+        a = layer_log_decay(g, tau, gate, q.shape[-1])
         o_gla, S_L, _ = gla_forward(feature_map(q, fmap_wq),
                                     feature_map(k, fmap_wk), v, a, state_in)
         out["o"] += o_gla
@@ -323,10 +346,12 @@ def lizard_forward(q, k, v, g, *, window, tau=16.0, scale=None,
 
 def lizard_backward(q, k, v, g, dout, *, window, tau=16.0, scale=None,
                     fmap_wq=None, fmap_wk=None, meta_k=None, meta_v=None,
-                    alpha=None, state_in=None, branch=BRANCH_BOTH):
+                    alpha=None, state_in=None, branch=BRANCH_BOTH,
+                    gate=GATE_PER_DIM):
     """Gradients of sum(dout * lizard_forward(...)['o']) w.r.t. every input.
 
-    Returns a dict: dq, dk, dv, dg [B,H,L,dk], dmeta_k, dmeta_v, dfmap_wq,
+    Returns a dict: dq, dk, dv, dg (the shape of g: [B,H,L,dk], or [B,H,L]
+    for gate="scalar"), dmeta_k, dmeta_v, dfmap_wq,
     dfmap_wk (None where the input is None), dalpha [H], dstate_in [B,H,dk,dv].
     """
     q, k, v, g, dout = _f64(q), _f64(k), _f64(v), _f64(g), _f64(dout)
@@ -343,7 +368,7 @@ def lizard_backward(q, k, v, g, dout, *, window, tau=16.0, scale=None,
            "dfmap_wk": None if fmap_wk is None else np.zeros(_f64(fmap_wk).shape),
            "dalpha": np.zeros(H), "dstate_in": np.zeros((B, H, dk, dv_))}
     if branch != BRANCH_SWA_ONLY:
-        a = gate_log_decay(g, tau)
+        a = layer_log_decay(g, tau, gate, dk)
         phq = feature_map(q, fmap_wq)
         phk = feature_map(k, fmap_wk)
         dphq, dphk, dv_g, da, dS0 = gla_backward(phq, phk, v, a, state_in, dout)
@@ -352,7 +377,10 @@ def lizard_backward(q, k, v, g, dout, *, window, tau=16.0, scale=None,
         res["dq"] += dq_g
         res["dk"] += dk_g
         res["dv"] += dv_g
-        # d logsigmoid(g)/dg = sigmoid(-g)
+        # d logsigmoid(g)/dg = sigmoid(-g); a scalar logit feeds every
+        # key dimension's decay, so its gradient sums over them
+        if gate == GATE_SCALAR:
+            da = da.sum(axis=-1)
         res["dg"] = da / (1.0 + np.exp(g)) / float(tau)
         res["dstate_in"] = dS0
         if fmap_wq is not None:
@@ -381,10 +409,11 @@ def lizard_backward(q, k, v, g, dout, *, window, tau=16.0, scale=None,
 
 def lizard_decode_step(q, k, v, g, state, k_cache, v_cache, pos, *, window,
                        tau=16.0, scale=None, fmap_wq=None, fmap_wk=None,
-                       meta_k=None, meta_v=None, alpha=None):
+                       meta_k=None, meta_v=None, alpha=None, gate=GATE_PER_DIM):
     """One generation step for every (batch, head); inputs are not modified.
 
-    q, k, g: [B,H,dk]; v: [B,H,dv]; state: [B,H,dk,dv]; k_cache: [B,H,w,dk];
+    q, k: [B,H,dk]; g: [B,H,dk] ([B,H] for gate="scalar"); v: [B,H,dv];
+    state: [B,H,dk,dv]; k_cache: [B,H,w,dk];
     v_cache: [B,H,w,dv]; pos: [B] tokens already seen.  The new token goes to
     ring slot pos mod w; the softmax covers the min(pos+1, w) filled slots and
     the meta tokens.  Returns (o [B,H,dv], state, k_cache, v_cache, pos + 1).
@@ -398,7 +427,7 @@ def lizard_decode_step(q, k, v, g, state, k_cache, v_cache, pos, *, window,
     if meta_k is None:
         meta_v = None
     B, H, dk = q.shape
-    a = gate_log_decay(g, tau)
+    a = layer_log_decay(g, tau, gate, dk)
     phq = feature_map(q[:, :, None], fmap_wq)[:, :, 0]
     phk = feature_map(k[:, :, None], fmap_wk)[:, :, 0]
     S = np.exp(a)[..., None] * S + phk[..., None] * v[:, :, None, :]
