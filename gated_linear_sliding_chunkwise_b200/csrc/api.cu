@@ -30,6 +30,7 @@ lizard_status check_fwd(const lizard_fwd_args *a) {
   if (a->dtype != LIZARD_BF16 && a->dtype != LIZARD_FP32) return LIZARD_ERR_INVALID_ARG;
   if (a->branch < LIZARD_BRANCH_BOTH || a->branch > LIZARD_BRANCH_SWA_ONLY) return LIZARD_ERR_INVALID_ARG;
   if (a->impl < LIZARD_IMPL_AUTO || a->impl > LIZARD_IMPL_TC) return LIZARD_ERR_INVALID_ARG;
+  if (a->gate != LIZARD_GATE_PER_DIM && a->gate != LIZARD_GATE_SCALAR) return LIZARD_ERR_INVALID_ARG;
   if (!(a->gate_temp > 0.f) || !isfinite(a->gate_temp)) return LIZARD_ERR_INVALID_ARG;
   if (!(a->softmax_scale >= 0.f) || !isfinite(a->softmax_scale)) return LIZARD_ERR_INVALID_ARG;
   if (a->dk != a->dv || (a->dk != 64 && a->dk != 128)) return LIZARD_ERR_UNSUPPORTED;
@@ -49,6 +50,7 @@ lizard_status check_fwd(const lizard_fwd_args *a) {
 }
 
 bool gla_on(const lizard_fwd_args *a) { return a->branch != LIZARD_BRANCH_SWA_ONLY; }
+int scalar_gate(const lizard_fwd_args *a) { return a->gate == LIZARD_GATE_SCALAR ? 1 : 0; }
 bool swa_on(const lizard_fwd_args *a) { return a->branch != LIZARD_BRANCH_GLA_ONLY; }
 
 // Kernel family the forward runs for these arguments.
@@ -188,7 +190,7 @@ void fwd_plan(const lizard_fwd_args *a, void *ws, cudaStream_t s, Plan &plan) {
     lz::TcFwdArgs t{a->q, a->k, a->v, a->g, a->fmap_wq, a->fmap_wk, a->meta_k, a->meta_v, a->alpha,
                     a->state_in, a->o, gla_on(a) ? a->state_out : nullptr, swa_on(a) ? a->lse : nullptr,
                     static_cast<uint32_t *>(ws), at<void>(ws, lay.phq), BH, a->H, a->L, a->M, a->window,
-                    a->branch, 1.f / a->gate_temp, scale_of(a)};
+                    a->branch, 1.f / a->gate_temp, scale_of(a), scalar_gate(a)};
     if (gla_on(a)) plan.add("gate_prep_kernel", [=] { return lz::launch_tc_fwd(t, 3, s); });
     if (lz::tc_fwd_stage_count(BH, a->L) > 1) {
       plan.add("tc_fwd_kernel(state pass)", [=] { return lz::launch_tc_fwd(t, 0, s); });
@@ -200,7 +202,7 @@ void fwd_plan(const lizard_fwd_args *a, void *ws, cudaStream_t s, Plan &plan) {
   float *o_gla = nullptr;
   if (gla_on(a)) {
     lz::PrepArgs pa{a->q, a->k, a->g, a->fmap_wq, a->fmap_wk, at<float>(ws, lay.phq), at<float>(ws, lay.phk),
-                    at<float>(ws, lay.a), a->H, a->L, 1.f / a->gate_temp};
+                    at<float>(ws, lay.a), a->H, a->L, 1.f / a->gate_temp, scalar_gate(a)};
     plan.add("prep_kernel", [=] { return lz::launch_prep(pa, BH, D, bf16, s); });
     o_gla = at<float>(ws, lay.o_gla);
     lz::GlaFwdArgs ga{at<float>(ws, lay.phq), at<float>(ws, lay.phk), at<float>(ws, lay.a), a->v, a->state_in,
@@ -223,22 +225,23 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan) {
   if (gla_tc) {
     lz::TcFwdArgs f{a->q, a->k, a->v, a->g, a->fmap_wq, a->fmap_wk, a->meta_k, a->meta_v, a->alpha,
                     a->state_in, nullptr, nullptr, nullptr, static_cast<uint32_t *>(ws), nullptr, BH, a->H,
-                    a->L, a->M, a->window, 0, inv_tau, scale_of(a)};
+                    a->L, a->M, a->window, 0, inv_tau, scale_of(a), scalar_gate(a)};
     void *snap_s = at<void>(ws, lay.snap_s);
     float *e32 = at<float>(ws, lay.e32), *gr = at<float>(ws, lay.gr);
     uint32_t *status = static_cast<uint32_t *>(ws);
     plan.add("gate_prep_kernel",
-             [=] { return lz::launch_gate_prep(a->g, nullptr, e32, gr, status, BH, a->L, inv_tau, s); });
+             [=] { return lz::launch_gate_prep(a->g, nullptr, e32, gr, status, BH, a->L, inv_tau, f.scalar_gate != 0,
+                                               s); });
     plan.add("tc_fwd_kernel(state copies)", [=] { return lz::launch_tc_state_snapshots(f, snap_s, e32, gr, s); });
     lz::TcGlaBwdArgs t{a->q, a->k, a->v, a->g, b->dout, a->fmap_wq, a->fmap_wk, snap_s,
                        at<void>(ws, lay.snap_ds), at<float>(ws, lay.dphq), at<float>(ws, lay.dphk),
                        at<float>(ws, lay.da), at<float>(ws, lay.dv_gla), b->dg, b->dstate_in,
-                       status, a->H, BH, a->L, inv_tau, e32, gr};
+                       status, a->H, BH, a->L, inv_tau, e32, gr, scalar_gate(a)};
     plan.add("tc_gla_dstates_kernel", [=] { return lz::launch_tc_gla_bwd(t, 0, s); });
     plan.add("tc_gla_bwd_tile_kernel", [=] { return lz::launch_tc_gla_bwd(t, 1, s); });
   } else if (g) {
     lz::PrepArgs pa{a->q, a->k, a->g, a->fmap_wq, a->fmap_wk, at<float>(ws, lay.phq), at<float>(ws, lay.phk),
-                    at<float>(ws, lay.a), a->H, a->L, inv_tau};
+                    at<float>(ws, lay.a), a->H, a->L, inv_tau, scalar_gate(a)};
     plan.add("prep_kernel", [=] { return lz::launch_prep(pa, BH, D, bf16, s); });
     lz::GlaStatesArgs sa{at<float>(ws, lay.phk), at<float>(ws, lay.a), a->v, a->state_in, at<float>(ws, lay.sprev), a->L};
     plan.add("gla_states_simt", [=] { return lz::launch_gla_states(sa, BH, D, bf16, s); });
@@ -261,7 +264,7 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan) {
                        w ? at<float>(ws, lay.dq_swa) : nullptr, w ? at<float>(ws, lay.dk_swa) : nullptr,
                        w ? at<float>(ws, lay.dv_swa) : nullptr,
                        b->dq, b->dk, b->dv, b->dg, b->dfmap_wq, b->dfmap_wk, a->H, a->L, inv_tau,
-                       gla_tc ? 0 : 1, static_cast<uint32_t *>(ws)};
+                       gla_tc ? 0 : 1, static_cast<uint32_t *>(ws), nullptr, nullptr, scalar_gate(a)};
   if (gla_tc) fa.da = nullptr;   // the gate gradient comes from gate_grad_kernel
   if (fused) {
     fa.xq_part = at<void>(ws, lay.dq_swa);   // bf16 parts in the anchor part slots
@@ -306,7 +309,7 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan) {
   if (gla_tc) {
     lz::TcGlaBwdArgs t{a->q, a->k, a->v, a->g, b->dout, a->fmap_wq, a->fmap_wk, nullptr, nullptr, nullptr,
                        nullptr, at<float>(ws, lay.da), nullptr, b->dg, nullptr, static_cast<uint32_t *>(ws),
-                       a->H, BH, a->L, inv_tau};
+                       a->H, BH, a->L, inv_tau, nullptr, nullptr, scalar_gate(a)};
     plan.add("gate_grad_kernel", [=] { return lz::launch_tc_gla_bwd(t, 2, s); });
   }
 }
@@ -449,6 +452,7 @@ lizard_status lizard_decode_step(const lizard_decode_args *a, lizard_stream_t st
   if (!a) return LIZARD_ERR_INVALID_ARG;
   if (a->B < 1 || a->H < 1 || a->dk <= 0 || a->dv <= 0 || a->window < 1 || a->M < 0) return LIZARD_ERR_INVALID_ARG;
   if (a->dtype != LIZARD_BF16 && a->dtype != LIZARD_FP32) return LIZARD_ERR_INVALID_ARG;
+  if (a->gate != LIZARD_GATE_PER_DIM && a->gate != LIZARD_GATE_SCALAR) return LIZARD_ERR_INVALID_ARG;
   if (!(a->gate_temp > 0.f) || !isfinite(a->gate_temp)) return LIZARD_ERR_INVALID_ARG;
   if (!(a->softmax_scale >= 0.f) || !isfinite(a->softmax_scale)) return LIZARD_ERR_INVALID_ARG;
   if (a->dk != a->dv || (a->dk != 64 && a->dk != 128)) return LIZARD_ERR_UNSUPPORTED;
@@ -464,7 +468,8 @@ lizard_status lizard_decode_step(const lizard_decode_args *a, lizard_stream_t st
   lz::DecodeArgs d{a->q, a->k, a->v, a->g, a->state, a->k_cache, a->v_cache, a->pos,
                    a->fmap_wq, a->fmap_wk, a->meta_k, a->meta_v, a->alpha, a->o,
                    a->H, a->window, a->M, 1.f / a->gate_temp,
-                   a->softmax_scale > 0.f ? a->softmax_scale : 1.f / sqrtf((float)a->dk)};
+                   a->softmax_scale > 0.f ? a->softmax_scale : 1.f / sqrtf((float)a->dk),
+                   a->gate == LIZARD_GATE_SCALAR ? 1 : 0};
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool bf16 = a->dtype == LIZARD_BF16;
   if (lz::decode_stream_supported(a->dk, bf16, a->window, a->M))

@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(256, 2) decode_kernel(DecodeArgs p) {
   const T *qs = static_cast<const T *>(p.q) + (size_t)bh * D;
   const T *ks = static_cast<const T *>(p.k) + (size_t)bh * D;
   const T *vs = static_cast<const T *>(p.v) + (size_t)bh * D;
-  const T *gs = static_cast<const T *>(p.g) + (size_t)bh * D;
+  const T *gs = static_cast<const T *>(p.g) + (size_t)bh * (p.scalar_gate ? 1 : D);
   float *S = p.state + (size_t)bh * D * D;
   const long long pos = p.pos[b];
   const int W = p.window;
@@ -113,7 +113,7 @@ __global__ void __launch_bounds__(256, 2) decode_kernel(DecodeArgs p) {
     xq[tid] = to_f32(qs[tid]);
     xk[tid] = to_f32(ks[tid]);
     xv[tid] = to_f32(vs[tid]);
-    gam[tid] = expf(log_decay(to_f32(gs[tid]), p.inv_tau));
+    gam[tid] = expf(log_decay(to_f32(gs[p.scalar_gate ? 0 : tid]), p.inv_tau));
   }
   __syncthreads();
 
@@ -520,14 +520,19 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_stream_kernel(const __g
           const uint32_t bytes = (uint32_t)pi.n * SD * 2;
           const __nv_bfloat16 *src = static_cast<const __nv_bfloat16 *>(kind == 0 ? p.k_cache : p.v_cache) +
                                      (size_t)pi.bh * p.window * SD;
-          s_mbar_expect(bar, bytes + (kind == 0 ? 4 * SD * 2 : 0));
+          // the new token's q, k, v and (per-dimension) g ride along with kind 0;
+          // a scalar gate is a single value that the prep warps read directly
+          const int ntok = p.scalar_gate ? 3 : 4;
+          s_mbar_expect(bar, bytes + (kind == 0 ? (uint32_t)ntok * SD * 2 : 0));
           bulk_load(dst, src, bytes, bar);
-          if (kind == 0) {   // the new token's q, k, v, g ride along
+          if (kind == 0) {
             __nv_bfloat16 *tk = tokring + (size_t)sl * 4 * SD;
             const void *srcs[4] = {p.q, p.k, p.v, p.g};
 #pragma unroll
             for (int u = 0; u < 4; ++u)
-              bulk_load(tk + u * SD, static_cast<const __nv_bfloat16 *>(srcs[u]) + (size_t)pi.bh * SD, SD * 2, bar);
+              if (u < ntok)
+                bulk_load(tk + u * SD, static_cast<const __nv_bfloat16 *>(srcs[u]) + (size_t)pi.bh * SD, SD * 2,
+                          bar);
           }
         } else {
           s_mbar_expect(bar, kChunkBytes);
@@ -558,7 +563,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_stream_kernel(const __g
         return;
       }
       PairRec &R = rec[k & 1];
-      R.gam[pt] = expf(log_decay(__bfloat162float(tk[3 * SD + pt]), p.inv_tau));
+      const __nv_bfloat16 gv = p.scalar_gate ? static_cast<const __nv_bfloat16 *>(p.g)[pi.bh] : tk[3 * SD + pt];
+      R.gam[pt] = expf(log_decay(__bfloat162float(gv), p.inv_tau));
       // z = x W: thread = (map, feature); 4 partial sums over the 128 rows
       const int map = pt >> 6, f = pt & 63;
       const __nv_bfloat16 *x = tk + map * SD;

@@ -13,6 +13,7 @@ struct PrepArgs {
   float *phq, *phk, *a;
   int H, L;
   float inv_tau;
+  int scalar_gate;   // g holds one logit per (token, head): [B*H][L]
 };
 
 struct GlaFwdArgs {
@@ -43,6 +44,7 @@ struct DecodeArgs {
   void *o;
   int H, window, M;
   float inv_tau, scale;
+  int scalar_gate;   // g holds one logit per (batch, head): [B*H]
 };
 
 // Backward (portable fp32 kernels).
@@ -95,6 +97,7 @@ struct FinishBwdArgs {
   // dx_k here (bf16 [B*H*L][128]) for the anchor kernels to add, and leave
   // dq, dk, dv to them.
   void *xq_part, *xk_part;
+  int scalar_gate;   // g and dg hold one value per (token, head): [B*H][L]
 };
 
 struct TcFwdArgs {
@@ -106,6 +109,7 @@ struct TcFwdArgs {
   void *seg_ws;       // tc_fwd_workspace_bytes() bytes: segment states, then the gate factors
   int BH, H, L, M, window, branch;
   float inv_tau, scale;
+  int scalar_gate;    // g holds one logit per (token, head): [B*H][L]
 };
 
 struct TcSwaBwdArgs {
@@ -136,6 +140,7 @@ struct TcGlaBwdArgs {
   float inv_tau;
   const float *e32;             // fp32 [B*H*L][128] decay factors of every tile (launch_gate_prep)
   const float *gate_r;          // fp32 [B*H][L/128][128] log-decay of every tile
+  int scalar_gate;              // g and dg hold one value per (token, head): [B*H][L]
 };
 
 constexpr int kBwdC = 32;   // GLA chunk used by the portable backward
@@ -171,9 +176,10 @@ cudaError_t launch_tc_state_snapshots(const TcFwdArgs &a, void *snap, const floa
                                       cudaStream_t s);
 // Decay factors of every 128-token tile (bf16 E16 and/or fp32 E32, [BH][L][128],
 // either may be null) and the tiles' log-decays r [BH][ntiles][128], from bf16
-// gate logits g [BH][L][128]; sets bit 2 of *status when a tile's spread is too wide.
+// gate logits g [BH][L][128] (scalar_gate: [BH][L], one logit for all 128
+// dimensions); sets bit 2 of *status when a tile's spread is too wide.
 cudaError_t launch_gate_prep(const void *g, void *E16, float *E32, float *r, uint32_t *status, int BH, int L,
-                             float inv_tau, cudaStream_t s);
+                             float inv_tau, bool scalar_gate, cudaStream_t s);
 // stage 0: reverse dS pass, 1: per-tile gradients, 2: gate-logit gradient
 cudaError_t launch_tc_gla_bwd(const TcGlaBwdArgs &a, int stage, cudaStream_t s);
 // tensor-core finish: bf16, d = 128, both feature maps present

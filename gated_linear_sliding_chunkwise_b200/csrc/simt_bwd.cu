@@ -759,11 +759,22 @@ __global__ void __launch_bounds__(256) finish_bwd(FinishBwdArgs p) {
           if (p.dv_gla) dvv += p.dv_gla[row + i];
           if (p.dv_swa) dvv += p.dv_swa[row + i];
           dvdst[row + i] = from_f32<T>(dvv);
-          if (p.write_dg) {
+          if (p.write_dg && !p.scalar_gate) {
             float dg = 0.f;
             if (p.da) dg = p.da[row + i] * dlogsigmoid(to_f32(gsrc[row + i])) * p.inv_tau;
             p.dg[row + i] = dg;
           }
+        }
+      }
+      if (p.write_dg && p.scalar_gate) {   // one logit feeds every dimension: sum over them
+        float s = 0.f;
+        if (live && p.da)
+#pragma unroll
+          for (int j = 0; j < XJ; ++j) s += p.da[row + lane + 32 * j];
+        s = warp_sum(s);
+        if (live && lane == 0) {
+          const size_t gi = (size_t)bh * p.L + t;
+          p.dg[gi] = p.da ? s * dlogsigmoid(to_f32(gsrc[gi])) * p.inv_tau : 0.f;
         }
       }
     }

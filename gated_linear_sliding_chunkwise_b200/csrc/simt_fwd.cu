@@ -51,10 +51,12 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepArgs p) {
     const int t = t0 + tt;
     if (t >= p.L) break;
     const size_t row = ((size_t)bh * p.L + t) * D;
+    // scalar gate: one logit per token and head, the same decay for every dimension
+    const float a_tok = p.scalar_gate ? log_decay(to_f32(gs[(size_t)bh * p.L + t]), p.inv_tau) : 0.f;
 #pragma unroll
     for (int j = 0; j < XJ; ++j) {
       const int i = lane + 32 * j;
-      p.a[row + i] = log_decay(to_f32(gs[row + i]), p.inv_tau);
+      p.a[row + i] = p.scalar_gate ? a_tok : log_decay(to_f32(gs[row + i]), p.inv_tau);
     }
 #pragma unroll
     for (int which = 0; which < 2; ++which) {

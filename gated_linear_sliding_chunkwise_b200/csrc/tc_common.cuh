@@ -80,6 +80,10 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, const void 
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
 // wait until the shared memory of every committed store has been read
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory"); }
+// the same, except for the most recently committed group
+__device__ __forceinline__ void bulk_wait_read_but_last() {
+  asm volatile("cp.async.bulk.wait_group.read 1;\n" ::: "memory");
+}
 // wait until every committed store has completed
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
 
@@ -236,6 +240,16 @@ __device__ __forceinline__ uint4 pack8(const float *f) {
   u.z = pack_bf16(f[4], f[5]);
   u.w = pack_bf16(f[6], f[7]);
   return u;
+}
+// Eight fp32 values as a bf16 pair hi + lo (hi = RNE(x), lo = RNE(x - hi)):
+// two MMAs over hi and lo carry about 16 significant bits of x.
+__device__ __forceinline__ void split8(const float *f, uint4 &hi, uint4 &lo) {
+  hi = pack8(f);
+  float h[8], r[8];
+  unpack8(hi, h);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) r[i] = f[i] - h[i];
+  lo = pack8(r);
 }
 // K-major operand descriptor, k-step s (16 columns) of a 128-row tile
 __device__ __forceinline__ uint64_t desc_k(uint32_t tile_addr, int s) {

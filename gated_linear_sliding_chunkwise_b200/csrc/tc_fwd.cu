@@ -598,7 +598,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
 // 16 loads are all in flight together; the warps' totals give each warp its
 // carry from the later tokens.  Rows past L are not written (readers treat
 // them as zero).  A tile whose spread r - b_0 exceeds kMaxSpread sets the
-// RANGE bit of *status.
+// RANGE bit of *status.  SCALAR: g is [BH][L], one logit per token and head
+// (the scalar gate of the Chinese summary's ablation, section 4) that every
+// dimension shares; the factors come out in the same per-dimension layout.
+template <bool SCALAR>
 __global__ void __launch_bounds__(256) gate_prep_kernel(const __nv_bfloat16 *g, __nv_bfloat16 *E16, float *E32,
                                                         float *rr, uint32_t *status, int L, int ntiles,
                                                         float inv_tau) {
@@ -611,8 +614,13 @@ __global__ void __launch_bounds__(256) gate_prep_kernel(const __nv_bfloat16 *g, 
 #pragma unroll
   for (int u = 0; u < 16; ++u) {
     const int t = tb + u;
-    a[u] = t < L ? __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(g + base + (size_t)t * 128))
-                 : make_float2(0.f, 0.f);
+    if (SCALAR) {
+      const float gv = t < L ? __bfloat162float(g[(size_t)bh * L + t]) : 0.f;
+      a[u] = make_float2(gv, gv);
+    } else {
+      a[u] = t < L ? __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(g + base + (size_t)t * 128))
+                   : make_float2(0.f, 0.f);
+    }
   }
   float2 tot = make_float2(0.f, 0.f);
 #pragma unroll
@@ -649,12 +657,16 @@ __global__ void __launch_bounds__(256) gate_prep_kernel(const __nv_bfloat16 *g, 
 }
 
 cudaError_t launch_gate_prep(const void *g, void *E16, float *E32, float *r, uint32_t *status, int BH, int L,
-                             float inv_tau, cudaStream_t s) {
+                             float inv_tau, bool scalar_gate, cudaStream_t s) {
   if (L == 0) return cudaSuccess;
   const int ntiles = (L + tc::kTileRows - 1) / tc::kTileRows;
-  gate_prep_kernel<<<dim3(2, ntiles, BH), 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(g),
-                                                       static_cast<__nv_bfloat16 *>(E16), E32, r, status, L,
-                                                       ntiles, inv_tau);
+  const dim3 grid(2, ntiles, BH);
+  const __nv_bfloat16 *gp = static_cast<const __nv_bfloat16 *>(g);
+  __nv_bfloat16 *e16 = static_cast<__nv_bfloat16 *>(E16);
+  if (scalar_gate)
+    gate_prep_kernel<true><<<grid, 256, 0, s>>>(gp, e16, E32, r, status, L, ntiles, inv_tau);
+  else
+    gate_prep_kernel<false><<<grid, 256, 0, s>>>(gp, e16, E32, r, status, L, ntiles, inv_tau);
   return cudaGetLastError();
 }
 
@@ -759,9 +771,9 @@ cudaError_t launch_tc_state_snapshots(const TcFwdArgs &a, void *snap, const floa
   memset(&p, 0, sizeof(p));
   const uint64_t rows = (uint64_t)a.L;
   if (!make_map_bf16_3d(&p.mq, a.q, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mk, a.k, D, rows, a.BH, T) ||
-      !make_map_bf16_3d(&p.mv, a.v, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mg, a.g, D, rows, a.BH, T))
+      !make_map_bf16_3d(&p.mv, a.v, D, rows, a.BH, T))
     return cudaErrorInvalidValue;
-  p.gate_e32 = e32;
+  p.gate_e32 = e32;   // the state pass loads no gate tiles (p.mg stays unset)
   p.gate_r = r;
   p.wq = a.wq;
   p.wk = a.wk;
@@ -798,7 +810,7 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, int stage, cudaStream_t s) {
   const bool gla = a.branch != 2 && a.g != nullptr;
   if (stage == 3) {
     if (!gla) return cudaSuccess;
-    return launch_gate_prep(a.g, w.e16, w.e32, w.r, a.status, a.BH, a.L, a.inv_tau, s);
+    return launch_gate_prep(a.g, w.e16, w.e32, w.r, a.status, a.BH, a.L, a.inv_tau, a.scalar_gate != 0, s);
   }
   if (nseg > 1 && stage == 1) {
     seg_combine_kernel<<<a.BH, 256, 0, s>>>(w.seg_state, w.seg_decay, a.state_in, w.seg_start, nseg);

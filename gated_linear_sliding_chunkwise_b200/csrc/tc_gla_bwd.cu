@@ -18,6 +18,12 @@
 // The decay factors E (fp32) and the tiles' log-decays r come precomputed
 // from launch_gate_prep.
 //
+// Qt and Kt enter the GK and GQ products as bf16 pairs hi + lo.  At small
+// feature-map weights phi is close to uniform, so dphi carries a large
+// component shared by all features that the feature-map backward removes
+// again; one bf16 rounding of Qt or Kt would leave errors of a few percent
+// of what remains in dW_k and dW_q.
+//
 // tc_gla_dstates_kernel  reverse pass per sequence: dS of every tile (bf16
 //                        copies) and the gradient of the initial state.
 // tc_gla_bwd_tile_kernel one CTA per (tile, sequence): the formulas above,
@@ -41,7 +47,7 @@ constexpr uint32_t REG = kReg;
 constexpr uint32_t ST_TIMEOUT = 1u, ST_RANGE = 2u;
 
 struct DsParams {
-  CUtensorMap mq, mg, mo;
+  CUtensorMap mq, mo;
   const float *wq;
   const float *e32, *gate_r;   // fp32 decay factors [BH*L][D] and tile log-decays [BH][ntiles][D]
   __nv_bfloat16 *snap;      // [BH][ntiles][D][D] dS at each tile's end
@@ -52,7 +58,7 @@ struct DsParams {
 };
 
 struct TileParams {
-  CUtensorMap mq, mk, mv, mo, mg, msp, mds;   // msp / mds: [BH*ntiles][D][D] snapshots
+  CUtensorMap mq, mk, mv, mo, msp, mds;       // msp / mds: [BH*ntiles][D][D] snapshots
   CUtensorMap mdq, mdk, mdb, mdv;             // fp32 outputs dphi_q, dphi_k, dB, dv (TMA stores)
   const float *wq, *wk;
   const float *e32;            // fp32 decay factors [BH*L][D]
@@ -233,14 +239,15 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
   unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
   __shared__ uint64_t bars[8];
   __shared__ uint32_t s_tmem;
-  // X_q -> Qt, X_k -> Kt, V, dO, A^T^ (bf16, rows = keys), [W_q | W_k] -> S' -> dS
-  constexpr uint32_t R_XQ = 0, R_XK = TILE, R_V = 2 * TILE, R_O = 3 * TILE, R_G = 4 * TILE, R_W = 5 * TILE;
+  // X_q -> Qt (hi), X_k -> Kt (hi), V, dO, Qt (lo), [W_q | W_k] -> S' -> dS, Kt (lo)
+  constexpr uint32_t R_XQ = 0, R_XK = TILE, R_V = 2 * TILE, R_O = 3 * TILE, R_QL = 4 * TILE, R_W = 5 * TILE,
+                     R_KL = 6 * TILE;
   // TMEM, in order of use:
   //   dA [128,256) dA^T [256,384) Zq [384,448) Zk [448,512)
-  //   dA^ [0,64) dA^T^ [64,128) ; E (fp32, kept to the end) [128,256)
-  //   A^T [256,384) ; GQ [256,384) GK [384,512) ; DV [0,128)
-  constexpr uint32_t C_DAH = 0, C_DATH = 64, C_DV = 0, C_DA = 128, C_E = 128, C_DAT = 256, C_AT = 256,
-                     C_GQ = 256, C_ZQ = 384, C_ZK = 448, C_GK = 384;
+  //   dA^ [0,64) dA^T^ [64,128) ; E (fp32, while Qt and Kt are formed) [128,256)
+  //   A^T [256,384) ; A^T^ (bf16) [128,192) ; GQ [256,384) GK [384,512) ; DV [0,128)
+  constexpr uint32_t C_DAH = 0, C_DATH = 64, C_DV = 0, C_DA = 128, C_E = 128, C_ATH = 128, C_DAT = 256,
+                     C_AT = 256, C_GQ = 256, C_ZQ = 384, C_ZK = 448, C_GK = 384;
   const int tid = threadIdx.x, warp = tid >> 5, wg = tid >> 7, row = tid & 127;
   const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
   const int c = blockIdx.x, bh = blockIdx.y, h = bh % p.H, t0 = c * T, tq = t0 + row;
@@ -312,14 +319,15 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
   __syncthreads();   // dA read out before E overwrites its columns
   tc_fence_after();
   //    E in fp32 (dimensions 64 wg ..) into TMEM, then Qt = phi_q E and
-  //    Kt = phi_k / E for the same dimensions (rows past L: Kt = 0)
+  //    Kt = phi_k / E for the same dimensions (rows past L: Kt = 0), each as
+  //    a bf16 pair hi + lo
   e_half_to_tmem(p.e32, ((size_t)bh * p.L + (valid ? tq : 0)) * D, valid, wg, tl + C_E + 64 * wg);
   tmem_st_wait();
 #pragma unroll
   for (int m = 0; m < 2; ++m) {
     float ph[F];
     const float s = feature_half(tl + (m == 0 ? C_ZQ : C_ZK), wg, ph);
-    const uint32_t reg = m == 0 ? R_XQ : R_XK;
+    const uint32_t reg = m == 0 ? R_XQ : R_XK, reg_lo = m == 0 ? R_QL : R_KL;
 #pragma unroll
     for (int c16 = 0; c16 < 4; ++c16) {
       float E[16], x16[16];
@@ -327,8 +335,13 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
 #pragma unroll
       for (int u = 0; u < 16; ++u)
         x16[u] = m == 0 ? ph[16 * c16 + u] * s * E[u] : (valid ? __fdividef(ph[16 * c16 + u] * s, E[u]) : 0.f);
-      *chunk_ptr(sm, reg, row, 8 * wg + 2 * c16) = pack8(x16);
-      *chunk_ptr(sm, reg, row, 8 * wg + 2 * c16 + 1) = pack8(x16 + 8);
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint4 hi, lo;
+        split8(x16 + 8 * hh, hi, lo);
+        *chunk_ptr(sm, reg, row, 8 * wg + 2 * c16 + hh) = hi;
+        *chunk_ptr(sm, reg_lo, row, 8 * wg + 2 * c16 + hh) = lo;
+      }
     }
   }
   fence_proxy_async();
@@ -343,27 +356,34 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
   ok = mbar_wait(&bars[3], 0, p.status, ST_TIMEOUT);
   if (__syncthreads_or(!ok)) goto done;
   tc_fence_after();
-  //    A^T^ = A^T masked to queries j >= key row, bf16 K-major over the gate
-  //    tile (consumed), 64 query columns per group
+  //    A^T^ = A^T masked to queries j >= key row, packed bf16 into TMEM over
+  //    the spent E columns, 64 query columns per group
   for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
     float v[32];
     tmem_ld32(tl + C_AT + ch * 32, v);
+    uint32_t a[16];
 #pragma unroll
-    for (int u = 0; u < 32; ++u) v[u] = (ch * 32 + u >= row) ? v[u] : 0.f;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) *chunk_ptr(sm, R_G, row, 4 * ch + k) = pack8(v + 8 * k);
+    for (int u = 0; u < 32; u += 2) {
+      const int j = ch * 32 + u;
+      a[u / 2] = pack_bf16(j >= row ? v[u] : 0.f, j + 1 >= row ? v[u + 1] : 0.f);
+    }
+    tmem_st8(tl + C_ATH + ch * 16, a);
+    tmem_st8(tl + C_ATH + ch * 16 + 8, a + 8);
   }
-  fence_proxy_async();
+  tmem_st_wait();
   tc_fence_before();
   ok = mbar_wait(&bars[2], 0, p.status, ST_TIMEOUT);
   if (__syncthreads_or(!ok)) goto done;
-  // 4a. GQ = dO S'^T + dA^ Kt ;  GK = dA^T^ Qt ; dS replaces S' once its product is done
+  // 4a. GQ = dO S'^T + dA^ (Kt hi + lo) ;  GK = dA^T^ (Qt hi + lo) ; dS
+  //     replaces S' once its product is done
   if (tid == 0) {
     tc_fence_after();
     for (int s = 0; s < 8; ++s) mma_ss(tb + C_GQ, desc_k(sbase + R_O, s), desc_k(sbase + R_W, s), id_kk, s > 0);
     mma_commit(&bars[4]);
     for (int s = 0; s < 8; ++s) mma_ts(tb + C_GQ, tb + C_DAH + s * 8, desc_mn(sbase + R_XK, s), id_mn, 1);
+    for (int s = 0; s < 8; ++s) mma_ts(tb + C_GQ, tb + C_DAH + s * 8, desc_mn(sbase + R_KL, s), id_mn, 1);
     for (int s = 0; s < 8; ++s) mma_ts(tb + C_GK, tb + C_DATH + s * 8, desc_mn(sbase + R_XQ, s), id_mn, s > 0);
+    for (int s = 0; s < 8; ++s) mma_ts(tb + C_GK, tb + C_DATH + s * 8, desc_mn(sbase + R_QL, s), id_mn, 1);
     mma_commit(&bars[5]);
     if (mbar_wait(&bars[4], 0, p.status, ST_TIMEOUT)) {
       mbar_expect_tx(&bars[6], TILE);
@@ -378,72 +398,93 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
   if (tid == 0) {
     tc_fence_after();
     for (int s = 0; s < 8; ++s) mma_ss(tb + C_GK, desc_k(sbase + R_V, s), desc_k(sbase + R_W, s), id_kk, 1);
-    for (int s = 0; s < 8; ++s) mma_ss(tb + C_DV, desc_k(sbase + R_G, s), desc_mn(sbase + R_O, s), id_mn, s > 0);
+    for (int s = 0; s < 8; ++s) mma_ts(tb + C_DV, tb + C_ATH + s * 8, desc_mn(sbase + R_O, s), id_mn, s > 0);
     for (int s = 0; s < 8; ++s) mma_ss(tb + C_DV, desc_k(sbase + R_XK, s), desc_mn(sbase + R_W, s), id_mn, 1);
     mma_commit(&bars[7]);
   }
-  ok = mbar_wait(&bars[7], 0, p.status, ST_TIMEOUT);
-  if (__syncthreads_or(!ok)) goto done;
-  tc_fence_after();
-  // 5. rows, dimension half per group: dphi_q = E GQ, dphi_k = GK / E, then
-  //    dB = Qt GQ - Kt GK and dv, staged as fp32 tiles over the free V | dO
-  //    and A^T^ | dS regions and written with TMA stores (rows past L are
-  //    clipped by the maps)
   {
-    unsigned char *st0 = sm + R_V, *st1 = sm + R_G;
-    for (int c16 = 4 * wg; c16 < 4 * wg + 4; ++c16) {
-      float E[16], gq[16], gk[16];
-      tmem_ld16(tl + C_E + c16 * 16, E);
-      tmem_ld16(tl + C_GQ + c16 * 16, gq);
-      tmem_ld16(tl + C_GK + c16 * 16, gk);
+    // 5. rows, dimension half per group, staged as fp32 tiles in the spent
+    //    regions and written with TMA stores (rows past L are clipped by the
+    //    maps): dB = Qt GQ - Kt GK (Qt, Kt as hi + lo, so that dB matches the
+    //    products) over V | dO; then dphi_q = E GQ over Qt lo | dS and
+    //    dphi_k = GK / E over Qt hi | Kt hi; then dv over V | dO again.  E
+    //    (fp32) is read again from global memory, its loads in flight while
+    //    the last products run.
+    float4 e4[16];
+    const float *er = p.e32 + ((size_t)bh * p.L + (valid ? tq : 0)) * D + 64 * wg;
 #pragma unroll
-      for (int u = 0; u < 16; u += 4) {
-        *f32_stage_ptr(st0, row, c16 * 16 + u) =
-            make_float4(E[u] * gq[u], E[u + 1] * gq[u + 1], E[u + 2] * gq[u + 2], E[u + 3] * gq[u + 3]);
-        *f32_stage_ptr(st1, row, c16 * 16 + u) =
-            make_float4(__fdividef(gk[u], E[u]), __fdividef(gk[u + 1], E[u + 1]), __fdividef(gk[u + 2], E[u + 2]),
-                        __fdividef(gk[u + 3], E[u + 3]));
-      }
-    }
-    fence_proxy_async();
-    __syncthreads();
-    if (tid == 0) {
-      for (int bx = 0; bx < 4; ++bx) {
-        tma_store_3d(&p.mdq, st0 + bx * 16384, 32 * bx, t0, bh);
-        tma_store_3d(&p.mdk, st1 + bx * 16384, 32 * bx, t0, bh);
-      }
-      bulk_commit();
-      bulk_wait_read();
-    }
-    __syncthreads();
+    for (int u = 0; u < 16; ++u)
+      e4[u] = valid ? *reinterpret_cast<const float4 *>(er + 4 * u) : make_float4(1.f, 1.f, 1.f, 1.f);
+    ok = mbar_wait(&bars[7], 0, p.status, ST_TIMEOUT);
+    if (__syncthreads_or(!ok)) goto done;
+    tc_fence_after();
+    unsigned char *st0 = sm + R_V, *st1 = sm + R_QL, *st2 = sm + R_XQ;
     for (int c16 = 4 * wg; c16 < 4 * wg + 4; ++c16) {
-      float gq[16], gk[16], q16[16], k16[16];
+      float gq[16], gk[16], q16[16], k16[16], lo[16];
       tmem_ld16(tl + C_GQ + c16 * 16, gq);
       tmem_ld16(tl + C_GK + c16 * 16, gk);
       unpack8(*chunk_ptr(sm, R_XQ, row, 2 * c16), q16);
       unpack8(*chunk_ptr(sm, R_XQ, row, 2 * c16 + 1), q16 + 8);
+      unpack8(*chunk_ptr(sm, R_QL, row, 2 * c16), lo);
+      unpack8(*chunk_ptr(sm, R_QL, row, 2 * c16 + 1), lo + 8);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) q16[u] += lo[u];
       unpack8(*chunk_ptr(sm, R_XK, row, 2 * c16), k16);
       unpack8(*chunk_ptr(sm, R_XK, row, 2 * c16 + 1), k16 + 8);
+      unpack8(*chunk_ptr(sm, R_KL, row, 2 * c16), lo);
+      unpack8(*chunk_ptr(sm, R_KL, row, 2 * c16 + 1), lo + 8);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) k16[u] += lo[u];
 #pragma unroll
       for (int u = 0; u < 16; u += 4)
         *f32_stage_ptr(st0, row, c16 * 16 + u) =
             make_float4(q16[u] * gq[u] - k16[u] * gk[u], q16[u + 1] * gq[u + 1] - k16[u + 1] * gk[u + 1],
                         q16[u + 2] * gq[u + 2] - k16[u + 2] * gk[u + 2], q16[u + 3] * gq[u + 3] - k16[u + 3] * gk[u + 3]);
     }
-    for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
-      float dv[32];
-      tmem_ld32(tl + C_DV + ch * 32, dv);
+    fence_proxy_async();
+    __syncthreads();   // also: every Qt / Kt read is done before their regions are reused
+    if (tid == 0) {
+      for (int bx = 0; bx < 4; ++bx) tma_store_3d(&p.mdb, st0 + bx * 16384, 32 * bx, t0, bh);
+      bulk_commit();
+    }
 #pragma unroll
-      for (int u = 0; u < 32; u += 4)
-        *f32_stage_ptr(st1, row, ch * 32 + u) = make_float4(dv[u], dv[u + 1], dv[u + 2], dv[u + 3]);
+    for (int k4 = 0; k4 < 4; ++k4) {
+      const int c16 = 4 * wg + k4;
+      float gq[16], gk[16];
+      tmem_ld16(tl + C_GQ + c16 * 16, gq);
+      tmem_ld16(tl + C_GK + c16 * 16, gk);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float4 E = e4[4 * k4 + u];
+        *f32_stage_ptr(st1, row, c16 * 16 + 4 * u) =
+            make_float4(E.x * gq[4 * u], E.y * gq[4 * u + 1], E.z * gq[4 * u + 2], E.w * gq[4 * u + 3]);
+        *f32_stage_ptr(st2, row, c16 * 16 + 4 * u) =
+            make_float4(__fdividef(gk[4 * u], E.x), __fdividef(gk[4 * u + 1], E.y),
+                        __fdividef(gk[4 * u + 2], E.z), __fdividef(gk[4 * u + 3], E.w));
+      }
     }
     fence_proxy_async();
     __syncthreads();
     if (tid == 0) {
       for (int bx = 0; bx < 4; ++bx) {
-        tma_store_3d(&p.mdb, st0 + bx * 16384, 32 * bx, t0, bh);
-        tma_store_3d(&p.mdv, st1 + bx * 16384, 32 * bx, t0, bh);
+        tma_store_3d(&p.mdq, st1 + bx * 16384, 32 * bx, t0, bh);
+        tma_store_3d(&p.mdk, st2 + bx * 16384, 32 * bx, t0, bh);
       }
+      bulk_commit();
+      bulk_wait_read_but_last();   // the dB tile has been read out of V | dO
+    }
+    __syncthreads();
+    for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
+      float dv[32];
+      tmem_ld32(tl + C_DV + ch * 32, dv);
+#pragma unroll
+      for (int u = 0; u < 32; u += 4)
+        *f32_stage_ptr(st0, row, ch * 32 + u) = make_float4(dv[u], dv[u + 1], dv[u + 2], dv[u + 3]);
+    }
+    fence_proxy_async();
+    __syncthreads();
+    if (tid == 0) {
+      for (int bx = 0; bx < 4; ++bx) tma_store_3d(&p.mdv, st0 + bx * 16384, 32 * bx, t0, bh);
       bulk_commit();
       bulk_wait_all();
     }
@@ -455,7 +496,6 @@ done:
 }
 
 // ------------------------------------------------------- gate gradient ----
-// dg_t = (sum_{s >= t} dB_s) * sigmoid(-g_t) / tau, one thread per dimension
 // dg_t = dlogsigmoid(g_t) / tau * sum_{s >= t} dB_s, per (sequence, key
 // dimension).  One CTA per (sequence, 32 dimensions): warp w owns token
 // segment w of 8 (lane = dimension, so each token row is one coalesced
@@ -501,8 +541,65 @@ __global__ void __launch_bounds__(256) gate_grad_kernel(const float *dB, const _
   }
 }
 
+// Scalar gate (one logit per token and head, shared by every key dimension):
+// dg_t = dlogsigmoid(g_t) / tau * sum_{s >= t} sum_i dB_s[i].  One CTA per
+// sequence; warp w owns token segment w of 8.  Pass 1: each warp reduces
+// its rows over the 128 dimensions (lane = 4 dimensions, one float4 each,
+// 8 rows in flight) and parks the row sums in dg; pass 2 walks the segment
+// backwards 32 rows at a time with a warp-wide suffix scan, starting from
+// the later segments' totals.
+__global__ void __launch_bounds__(256) gate_grad_scalar_kernel(const float *dB, const __nv_bfloat16 *g, float *dg,
+                                                              int L, float inv_tau) {
+  __shared__ float s_tot[kGateSeg];
+  const int bh = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int seg = (L + kGateSeg - 1) / kGateSeg;
+  const int ta = min(L, warp * seg), tz = min(L, ta + seg);
+  const float *src = dB + (size_t)bh * L * D + lane * 4;
+  float *dst = dg + (size_t)bh * L;
+  float total = 0.f;
+  for (int t = ta; t < tz; t += 8) {
+    float r[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      r[u] = 0.f;
+      if (t + u < tz) {
+        const float4 x = *reinterpret_cast<const float4 *>(src + (size_t)(t + u) * D);
+        r[u] = (x.x + x.y) + (x.z + x.w);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+      for (int u = 0; u < 8; ++u) r[u] += __shfl_xor_sync(0xffffffffu, r[u], o);
+    if (lane < 8 && t + lane < tz) {
+      float mine = r[0];
+#pragma unroll
+      for (int u = 1; u < 8; ++u) mine = lane == u ? r[u] : mine;
+      dst[t + lane] = mine;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) total += t + u < tz ? r[u] : 0.f;
+  }
+  if (lane == 0) s_tot[warp] = total;
+  __syncthreads();   // also orders each warp's parked row sums before pass 2
+  float carry = 0.f;
+  for (int w = warp + 1; w < kGateSeg; ++w) carry += s_tot[w];
+  for (int hi = tz - 1; hi >= ta; hi -= 32) {
+    const int t = hi - lane;                   // lane 0 takes the latest row
+    const bool in = t >= ta;
+    float x = in ? dst[t] : 0.f;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {         // suffix sum toward lane 0
+      const float y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (in) dst[t] = (carry + x) * dlogsigmoid(__bfloat162float(g[(size_t)bh * L + t])) * inv_tau;
+    carry += __shfl_sync(0xffffffffu, x, 31);
+  }
+}
+
 constexpr size_t DS_SMEM = 3 * TILE + TILE / 2 + 1024;
-constexpr size_t TILE_SMEM = 6 * TILE + 1024;
+constexpr size_t TILE_SMEM = 7 * TILE + 1024;
 
 }  // namespace
 
@@ -516,8 +613,7 @@ cudaError_t launch_tc_gla_bwd(const TcGlaBwdArgs &a, int stage, cudaStream_t s) 
   if (stage == 0) {   // reverse dS pass
     DsParams p;
     memset(&p, 0, sizeof(p));
-    if (!make_map_bf16_3d(&p.mq, a.q, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mg, a.g, D, rows, a.BH, T) ||
-        !make_map_bf16_3d(&p.mo, a.dout, D, rows, a.BH, T))
+    if (!make_map_bf16_3d(&p.mq, a.q, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mo, a.dout, D, rows, a.BH, T))
       return cudaErrorInvalidValue;
     p.wq = a.wq;
     p.e32 = a.e32;
@@ -538,7 +634,6 @@ cudaError_t launch_tc_gla_bwd(const TcGlaBwdArgs &a, int stage, cudaStream_t s) 
     memset(&p, 0, sizeof(p));
     if (!make_map_bf16_3d(&p.mq, a.q, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mk, a.k, D, rows, a.BH, T) ||
         !make_map_bf16_3d(&p.mv, a.v, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mo, a.dout, D, rows, a.BH, T) ||
-        !make_map_bf16_3d(&p.mg, a.g, D, rows, a.BH, T) ||
         !make_map_bf16_3d(&p.msp, a.snap_s, D, D, (uint64_t)a.BH * ntiles, T) ||
         !make_map_bf16_3d(&p.mds, a.snap_ds, D, D, (uint64_t)a.BH * ntiles, T) ||
         !make_map_f32_3d(&p.mdq, a.dphq, D, rows, a.BH, T) || !make_map_f32_3d(&p.mdk, a.dphk, D, rows, a.BH, T) ||
@@ -561,8 +656,12 @@ cudaError_t launch_tc_gla_bwd(const TcGlaBwdArgs &a, int stage, cudaStream_t s) 
     tc_gla_bwd_tile_kernel<<<dim3(ntiles, a.BH), NT_TILE, TILE_SMEM, s>>>(p);
     return cudaGetLastError();
   }
-  gate_grad_kernel<<<dim3(a.BH, D / 32), 256, 0, s>>>(a.dB, static_cast<const __nv_bfloat16 *>(a.g), a.dg, a.L,
-                                                      a.inv_tau);
+  if (a.scalar_gate)
+    gate_grad_scalar_kernel<<<a.BH, 256, 0, s>>>(a.dB, static_cast<const __nv_bfloat16 *>(a.g), a.dg, a.L,
+                                                 a.inv_tau);
+  else
+    gate_grad_kernel<<<dim3(a.BH, D / 32), 256, 0, s>>>(a.dB, static_cast<const __nv_bfloat16 *>(a.g), a.dg, a.L,
+                                                        a.inv_tau);
   return cudaGetLastError();
 }
 

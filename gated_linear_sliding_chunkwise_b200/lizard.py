@@ -28,6 +28,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE, ERR_
 BF16, FP32 = 0, 1
 BRANCH_BOTH, BRANCH_GLA_ONLY, BRANCH_SWA_ONLY = 0, 1, 2
 IMPL_AUTO, IMPL_SIMT, IMPL_TC = 0, 1, 2
+GATE_PER_DIM, GATE_SCALAR = 0, 1
 
 _vp = ctypes.c_void_p
 _i32 = ctypes.c_int32
@@ -37,7 +38,7 @@ _f32 = ctypes.c_float
 class FwdArgs(ctypes.Structure):
     _fields_ = [("B", _i32), ("H", _i32), ("L", _i32), ("dk", _i32), ("dv", _i32),
                 ("chunk", _i32), ("window", _i32), ("M", _i32), ("dtype", _i32),
-                ("branch", _i32), ("impl", _i32), ("gate_temp", _f32),
+                ("branch", _i32), ("impl", _i32), ("gate", _i32), ("gate_temp", _f32),
                 ("softmax_scale", _f32),
                 ("q", _vp), ("k", _vp), ("v", _vp), ("g", _vp),
                 ("fmap_wq", _vp), ("fmap_wk", _vp), ("meta_k", _vp), ("meta_v", _vp),
@@ -56,7 +57,8 @@ class BwdArgs(ctypes.Structure):
 
 class DecodeArgs(ctypes.Structure):
     _fields_ = [("B", _i32), ("H", _i32), ("dk", _i32), ("dv", _i32), ("window", _i32),
-                ("M", _i32), ("dtype", _i32), ("gate_temp", _f32), ("softmax_scale", _f32),
+                ("M", _i32), ("dtype", _i32), ("gate", _i32), ("gate_temp", _f32),
+                ("softmax_scale", _f32),
                 ("q", _vp), ("k", _vp), ("v", _vp), ("g", _vp), ("state", _vp),
                 ("k_cache", _vp), ("v_cache", _vp), ("pos", _vp),
                 ("fmap_wq", _vp), ("fmap_wk", _vp), ("meta_k", _vp), ("meta_v", _vp),
@@ -137,10 +139,23 @@ def _check(code: int, where: str):
         raise LizardError(code, where)
 
 
+def _gate_code(q, g):
+    """The gate granularity from g's shape: the shape of q (one logit per key
+    dimension) or q's without the last axis (one scalar logit per token and
+    head)."""
+    if g is None or tuple(g.shape) == tuple(q.shape):
+        return GATE_PER_DIM
+    if tuple(g.shape) == tuple(q.shape[:-1]):
+        return GATE_SCALAR
+    raise ValueError(f"gate logits of shape {tuple(g.shape)} fit neither {tuple(q.shape)} "
+                     f"nor {tuple(q.shape[:-1])}")
+
+
 def _fwd_struct(q, k, v, g, *, window, chunk, gate_temp, softmax_scale, fmap_wq,
                 fmap_wk, meta_k, meta_v, alpha, state_in, branch, impl):
     B, H, L, dk = q.shape
     a = FwdArgs()
+    a.gate = _gate_code(q, g)
     a.B, a.H, a.L, a.dk, a.dv = B, H, L, dk, v.shape[-1]
     a.chunk, a.window = chunk, window
     a.M = 0 if meta_k is None else meta_k.shape[1]
@@ -245,7 +260,7 @@ def attn_bwd(q, k, v, g, dout, *, window, chunk=64, gate_temp=16.0, softmax_scal
     f32 = torch.float32
     res = {
         "dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
-        "dg": torch.empty(B, H, L, dk, dtype=f32, device=dev),
+        "dg": torch.empty(g.shape if g is not None else (B, H, L, dk), dtype=f32, device=dev),
         "dmeta_k": None if meta_k is None else torch.empty_like(meta_k),
         "dmeta_v": None if meta_v is None else torch.empty_like(meta_v),
         "dfmap_wq": None if fmap_wq is None else torch.empty_like(fmap_wq),
@@ -283,6 +298,7 @@ def decode_step(q, k, v, g, state, k_cache, v_cache, pos, *, gate_temp=16.0,
     a.window = k_cache.shape[2]
     a.M = 0 if meta_k is None else meta_k.shape[1]
     a.dtype = _dtype_code(q)
+    a.gate = _gate_code(q, g)
     a.gate_temp, a.softmax_scale = gate_temp, softmax_scale
     a.q, a.k, a.v, a.g = _ptr(q), _ptr(k), _ptr(v), _ptr(g)
     a.state, a.k_cache, a.v_cache, a.pos = _ptr(state), _ptr(k_cache), _ptr(v_cache), _ptr(pos)

@@ -9,7 +9,8 @@ Recipe (one torch.Generator on the CPU, seeded per workload, drawn in this
 fixed order, fp32 then rounded once to the activation dtype with RNE):
 
   q, k, v      ~ N(0, 1) / 8          [B, H, L, d]
-  g            ~ N(gate_mean, 1)      [B, H, L, d]   gate logits
+  g            ~ N(gate_mean, 1)      [B, H, L, d]   gate logits ([B, H, L] for
+                                                     the scalar gate)
   fmap_wq, wk  ~ N(0, 1) * 0.02       [H, d, d/2]    fp32 (parameters)
   meta_k, v    ~ N(0, 1) / 8          [H, M, d]      fp32 (parameters)
   alpha        = 1                    [H]            fp32
@@ -43,6 +44,7 @@ class Workload:
     seed: int = 0
     kind: str = "fwd"            # "fwd" | "train" | "decode"
     decode_pos: int = 65536
+    gate: str = "dim"            # "dim": a logit per key dimension | "scalar": one per token-head
 
     def as_dict(self):
         return asdict(self)
@@ -72,7 +74,7 @@ def torch_dtype(name: str) -> torch.dtype:
 
 
 def make_inputs(w: Workload, *, B=None, H=None, L=None, d=None, seed=None,
-                M=None, with_dout=None):
+                M=None, with_dout=None, gate=None):
     """Draw one workload's inputs on the CPU (optionally with new sizes).
 
     Returns a dict of CPU tensors: activations in the workload's dtype,
@@ -84,6 +86,7 @@ def make_inputs(w: Workload, *, B=None, H=None, L=None, d=None, seed=None,
     d = w.d if d is None else d
     M = w.M if M is None else M
     seed = w.seed if seed is None else seed
+    gd = () if (w.gate if gate is None else gate) == "scalar" else (d,)
     dt = torch_dtype(w.dtype)
     gen = torch.Generator().manual_seed(seed)
 
@@ -95,7 +98,7 @@ def make_inputs(w: Workload, *, B=None, H=None, L=None, d=None, seed=None,
         out["q"] = (rn(B, H, d) / 8).to(dt)
         out["k"] = (rn(B, H, d) / 8).to(dt)
         out["v"] = (rn(B, H, d) / 8).to(dt)
-        out["g"] = (rn(B, H, d) + w.gate_mean).to(dt)
+        out["g"] = (rn(B, H, *gd) + w.gate_mean).to(dt)
         out["state"] = rn(B, H, d, d) * 0.1
         out["k_cache"] = (rn(B, H, w.window, d) / 8).to(dt)
         out["v_cache"] = (rn(B, H, w.window, d) / 8).to(dt)
@@ -104,7 +107,7 @@ def make_inputs(w: Workload, *, B=None, H=None, L=None, d=None, seed=None,
         out["q"] = (rn(B, H, L, d) / 8).to(dt)
         out["k"] = (rn(B, H, L, d) / 8).to(dt)
         out["v"] = (rn(B, H, L, d) / 8).to(dt)
-        out["g"] = (rn(B, H, L, d) + w.gate_mean).to(dt)
+        out["g"] = (rn(B, H, L, *gd) + w.gate_mean).to(dt)
     out["fmap_wq"] = rn(H, d, d // 2) * 0.02
     out["fmap_wk"] = rn(H, d, d // 2) * 0.02
     out["meta_k"] = rn(H, M, d) / 8

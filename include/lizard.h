@@ -6,7 +6,8 @@
  * English, French, Spanish and Chinese describe it) mixes two branches:
  *
  *   GLA branch (English summary, section 2.A "State Update"):
- *     a_t   = logsigmoid(g_t) / gate_temp                   (per key dim)
+ *     a_t   = logsigmoid(g_t) / gate_temp                   (per key dim, or
+ *             one value for every key dim with LIZARD_GATE_SCALAR)
  *     S_t   = diag(exp a_t) S_{t-1} + phi_k(k_t) v_t^T      (fp32 state)
  *     o^gla = S_t^T phi_q(q_t)
  *   with phi(x) = [softmax(x W), softmax(-x W)], W in R^{dk x dk/2} per head
@@ -74,6 +75,14 @@ typedef enum { LIZARD_BF16 = 0, LIZARD_FP32 = 1 } lizard_dtype;
 /* Which terms of o = o^gla + alpha_h o^swa to compute (test hook). */
 enum { LIZARD_BRANCH_BOTH = 0, LIZARD_BRANCH_GLA_ONLY = 1, LIZARD_BRANCH_SWA_ONLY = 2 };
 
+/* Gate granularity (lizard_fwd_args.gate, lizard_decode_args.gate).
+ * PER_DIM: one gate logit per key dimension, g [..., dk].  SCALAR: one logit
+ * per token and head, g [...] without the dk axis, whose decay every key
+ * dimension shares (the light scalar gate that the Chinese summary's
+ * ablation, section 4, finds most effective); its gradient dg has the same
+ * shape as g. */
+enum { LIZARD_GATE_PER_DIM = 0, LIZARD_GATE_SCALAR = 1 };
+
 /* Kernel family selection (lizard_fwd_args.impl / lizard_bwd_args.impl). */
 enum {
   LIZARD_IMPL_AUTO = 0,  /* tensor-core path where it applies, else portable */
@@ -87,8 +96,10 @@ enum {
  * Forward of the hybrid layer over whole sequences.
  *
  * Shapes (B batch, H heads, L tokens, dk = dv = d):
- *   q, k, g    [B, H, L, dk] dtype   (g: gate logits; the gate projection
- *                                      W_gamma x itself is the caller's)
+ *   q, k       [B, H, L, dk] dtype
+ *   g          [B, H, L, dk] dtype gate logits, or [B, H, L] with
+ *              gate = LIZARD_GATE_SCALAR (the gate projection W_gamma x
+ *              itself is the caller's)
  *   v          [B, H, L, dv] dtype
  *   fmap_wq/wk [H, dk, dk/2] fp32, or NULL for the identity map
  *   meta_k     [H, M, dk] fp32 (NULL iff M == 0)
@@ -109,6 +120,7 @@ typedef struct {
   int32_t dtype;   /* lizard_dtype */
   int32_t branch;  /* LIZARD_BRANCH_* */
   int32_t impl;    /* LIZARD_IMPL_* */
+  int32_t gate;    /* LIZARD_GATE_* */
   float gate_temp;
   float softmax_scale;
   const void *q, *k, *v, *g;
@@ -145,7 +157,8 @@ lizard_status lizard_attn_fwd(const lizard_fwd_args *args, lizard_stream_t strea
  *   dout     [B, H, L, dv] dtype
  *   dq, dk   [B, H, L, dk] dtype, written
  *   dv       [B, H, L, dv] dtype, written
- *   dg       [B, H, L, dk] fp32 gradient of the gate logits, written
+ *   dg       [B, H, L, dk] fp32 gradient of the gate logits ([B, H, L] with
+ *            LIZARD_GATE_SCALAR), written
  *   dmeta_k, dmeta_v, dfmap_wq, dfmap_wk, dalpha, dstate_in   fp32, same
  *            shapes as the inputs, written (overwritten, not accumulated);
  *            each may be NULL when not wanted (and must be NULL when the
@@ -182,7 +195,8 @@ int32_t lizard_bwd_launch_plan(const lizard_bwd_args *args, const char **names, 
  * English summary (section 2.A "State Update") with the fixed-size window
  * cache of the Chinese summary (section 2.1).
  *
- *   q, k, g    [B, H, dk] dtype;  v [B, H, dv] dtype: the new token
+ *   q, k       [B, H, dk] dtype;  v [B, H, dv] dtype: the new token
+ *   g          [B, H, dk] dtype, or [B, H] with gate = LIZARD_GATE_SCALAR
  *   state      [B, H, dk, dv] fp32, updated in place:
  *              S <- diag(exp a) S + phi_k(k) v^T
  *   k_cache    [B, H, window, dk] dtype, v_cache [B, H, window, dv] dtype:
@@ -200,6 +214,7 @@ int32_t lizard_bwd_launch_plan(const lizard_bwd_args *args, const char **names, 
 typedef struct {
   int32_t B, H, dk, dv, window, M;
   int32_t dtype;
+  int32_t gate;    /* LIZARD_GATE_* */
   float gate_temp;
   float softmax_scale;
   const void *q, *k, *v, *g;

@@ -51,6 +51,12 @@ def head_inputs(inp, b, h, keys=("q", "k", "v", "g", "dout")):
     return out
 
 
+def gate_of(x):
+    """Scalar gate when the logits lack q's last axis (one per token and head)."""
+    g, q = x.get("g"), x["q"]
+    return ref.GATE_SCALAR if g is not None and g.ndim == q.ndim - 1 else ref.GATE_PER_DIM
+
+
 def oracle_forward(inp, *, window, tau, branch=ref.BRANCH_BOTH, pairs=None):
     """Oracle forward on all pairs (pairs None) or on listed (b, h) pairs.
     Returns {(b, h) or 'all': result dict}."""
@@ -60,7 +66,7 @@ def oracle_forward(inp, *, window, tau, branch=ref.BRANCH_BOTH, pairs=None):
                                   fmap_wq=x.get("fmap_wq"), fmap_wk=x.get("fmap_wk"),
                                   meta_k=x.get("meta_k"), meta_v=x.get("meta_v"),
                                   alpha=x.get("alpha"), state_in=x.get("state_in"),
-                                  branch=branch)
+                                  branch=branch, gate=gate_of(x))
     res = {}
     for (b, h) in pairs:
         x = head_inputs(inp, b, h)
@@ -68,7 +74,8 @@ def oracle_forward(inp, *, window, tau, branch=ref.BRANCH_BOTH, pairs=None):
                                          tau=tau, fmap_wq=x.get("fmap_wq"),
                                          fmap_wk=x.get("fmap_wk"), meta_k=x.get("meta_k"),
                                          meta_v=x.get("meta_v"), alpha=x.get("alpha"),
-                                         state_in=x.get("state_in"), branch=branch)
+                                         state_in=x.get("state_in"), branch=branch,
+                                         gate=gate_of(x))
     return res
 
 
@@ -79,7 +86,7 @@ def oracle_backward(inp, *, window, tau, branch=ref.BRANCH_BOTH, pairs=None):
                                    tau=tau, fmap_wq=x.get("fmap_wq"), fmap_wk=x.get("fmap_wk"),
                                    meta_k=x.get("meta_k"), meta_v=x.get("meta_v"),
                                    alpha=x.get("alpha"), state_in=x.get("state_in"),
-                                   branch=branch)
+                                   branch=branch, gate=gate_of(x))
     res = {}
     for (b, h) in pairs:
         x = head_inputs(inp, b, h)
@@ -87,7 +94,8 @@ def oracle_backward(inp, *, window, tau, branch=ref.BRANCH_BOTH, pairs=None):
                                           window=window, tau=tau, fmap_wq=x.get("fmap_wq"),
                                           fmap_wk=x.get("fmap_wk"), meta_k=x.get("meta_k"),
                                           meta_v=x.get("meta_v"), alpha=x.get("alpha"),
-                                          state_in=x.get("state_in"), branch=branch)
+                                          state_in=x.get("state_in"), branch=branch,
+                                         gate=gate_of(x))
     return res
 
 

@@ -8,6 +8,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "lizard.h")
@@ -99,6 +100,8 @@ def _fwd(lz, **over):
     ({"B": 0}, 1),
     ({"dtype": 7}, 1),
     ({"branch": 3}, 1),
+    ({"gate": 2}, 1),
+    ({"gate": -1}, 1),
     ({"gate_temp": 0.0}, 1),
     ({"gate_temp": float("nan")}, 1),
     ({"softmax_scale": -1.0}, 1),
@@ -164,8 +167,21 @@ def test_decode_rejects_bad_arguments_on_host(lz):
     d.pos = None
     assert lz.lib().lizard_decode_step(ctypes.byref(d), None) == lz.ERR_INVALID_ARG
     d.pos = fake
+    d.gate = 5                 # neither per-dimension nor scalar
+    assert lz.lib().lizard_decode_step(ctypes.byref(d), None) == lz.ERR_INVALID_ARG
+    d.gate = lz.GATE_SCALAR
     d.M = 2                    # meta tokens without meta keys
     assert lz.lib().lizard_decode_step(ctypes.byref(d), None) == lz.ERR_INVALID_ARG
+
+
+def test_gate_granularity_follows_the_logits_shape(lz):
+    """The binding marks the gate scalar when g lacks q's last axis."""
+    q = torch.zeros(2, 3, 5, 8)
+    assert lz._gate_code(q, torch.zeros(2, 3, 5, 8)) == lz.GATE_PER_DIM
+    assert lz._gate_code(q, torch.zeros(2, 3, 5)) == lz.GATE_SCALAR
+    assert lz._gate_code(q, None) == lz.GATE_PER_DIM
+    with pytest.raises(ValueError):
+        lz._gate_code(q, torch.zeros(2, 3, 8))
 
 
 def test_prefill_cache_rejects_bad_arguments_on_host(lz):
