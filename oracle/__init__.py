@@ -17,6 +17,8 @@ from .lizard_ref import (  # noqa: F401
     lizard_forward,
     lizard_backward,
     lizard_decode_step,
+    attention_mse,
+    lizard_stage1_step,
     BRANCH_BOTH,
     BRANCH_GLA_ONLY,
     BRANCH_SWA_ONLY,

@@ -404,6 +404,39 @@ def lizard_backward(q, k, v, g, dout, *, window, tau=16.0, scale=None,
 
 
 # ---------------------------------------------------------------------------
+# Stage 1 of training: attention approximation
+# ---------------------------------------------------------------------------
+
+def attention_mse(o, target):
+    """Stage-1 attention-approximation loss and its gradient.
+
+    [EN] 2.B "Stage 1", [ZH] 2.2, [FR] 2.B: the layer is trained to reproduce
+    the teacher's softmax-attention output under a mean squared error.
+    Reading: the mean runs over every element (batch, head, token, value
+    dimension), loss = sum((o - y)^2) / n, so dL/do = 2 (o - y) / n.
+    """
+    diff = _f64(o) - _f64(target)
+    n = diff.size
+    return float(np.sum(diff * diff) / n), 2.0 * diff / n
+
+
+def lizard_stage1_step(q, k, v, g, target, *, window, tau=16.0, scale=None,
+                       fmap_wq=None, fmap_wk=None, meta_k=None, meta_v=None,
+                       alpha=None, state_in=None, gate=GATE_PER_DIM):
+    """One stage-1 training step: forward, the MSE against the teacher output
+    `target` [B,H,L,dv], and the gradients of that loss with respect to every
+    input (as lizard_backward, with dout = dL/do).  Returns the backward's
+    dict plus "loss" and "o"."""
+    kw = dict(window=window, tau=tau, scale=scale, fmap_wq=fmap_wq, fmap_wk=fmap_wk,
+              meta_k=meta_k, meta_v=meta_v, alpha=alpha, state_in=state_in, gate=gate)
+    o = lizard_forward(q, k, v, g, **kw)["o"]
+    loss, dout = attention_mse(o, target)
+    res = lizard_backward(q, k, v, g, dout, **kw)
+    res["loss"], res["o"] = loss, o
+    return res
+
+
+# ---------------------------------------------------------------------------
 # Decode: one token, constant-size state plus a ring-buffer window
 # ---------------------------------------------------------------------------
 
