@@ -176,6 +176,14 @@ class ClockSampler:
 
 
 # -------------------------------------------------------------- helpers ----
+# dram__bytes_read.sum + dram__bytes_write.sum of one launch on the
+# train_step workload (B=8, H=32, L=2048), from an ncu capture of the current
+# kernel build.
+MEASURED_TRAFFIC = {
+    "tc_gla_bwd_tile_kernel": 1.091525e9 + 1.023677e9,
+}
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -299,7 +307,9 @@ def run_ours(args, rank, world, local):
             roof = {"bound": "hbm", "achieved": dbytes / dt / 1e9, "peak": peaks["hbm_gbs"],
                     "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = None
+    # DRAM bytes (read + write) of one ncu capture of the kernel on this
+    # workload, per launch; kernels changed since their capture are left out
+    roof["traffic"] = MEASURED_TRAFFIC.get(dom) if args.kernels in ("auto", "tc") else None
     roof["kernel"] = dom
     roof["ms_per_launch"] = per[dom]
     roof["peak_source"] = peaks["source"]
@@ -387,6 +397,8 @@ def run_ours(args, rank, world, local):
     decode = None if args.no_decode else run_decode(args, lz, dev, rank, world, peaks)
     fwd_long = None if args.no_fwd_long else run_forward(args, lz, dev, rank, world, peaks,
                                                          "long_fwd_16k", max(K, 5))
+    variants = None if args.no_variants else run_variants(args, lz, dev, rank, world, peaks,
+                                                          max(min(K, 30), 5))
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
@@ -404,6 +416,7 @@ def run_ours(args, rank, world, local):
         "roofline": roof, "kernel_ms": kernels,
         "gpu_launches": K * (len(fwd_names) + len(bwd_names)),
         "clocks": clk, "e2e": e2e, "decode": decode, "fwd_long_16k": fwd_long,
+        "variants": variants,
     }
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(inp, w, budget_s=args.cpu_budget)
@@ -483,6 +496,80 @@ def run_backward(args, lz, dev, rank, world, peaks, name, steps):
     per = {n: statistics.mean(ev[j].elapsed_time(ev[j + 1]) for ev in evs) for j, n in enumerate(names)}
     return {"workload": f"{name} backward: B={w.B} H={w.H} L={w.L} d={w.d}", "ms": ms,
             "kernel_ms": {n: round(t, 4) for n, t in per.items()}, "launches": len(names)}
+
+
+def _time_steps(step, names, lz, world, dev, warmup, steps):
+    """Device time per call of step(events) and per kernel (launch events)."""
+    for _ in range(max(warmup, 1)):
+        step(None)
+    evs = [lz.make_events(len(names) + 1) for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for i in range(steps):
+        step(evs[i])
+    e.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(s.elapsed_time(e) / steps, world, dev)
+    per = {}
+    for j, n in enumerate(names):
+        per[n] = per.get(n, 0.0) + statistics.mean(ev[j].elapsed_time(ev[j + 1]) for ev in evs)
+    return ms, {n: round(t, 4) for n, t in per.items()}
+
+
+def run_variants(args, lz, dev, rank, world, peaks, steps):
+    """The training-step shape in the two variants beside the headline step:
+    the stage-1 step (forward, mean squared error against a teacher output,
+    backward: lizard_stage1_step) and the forward + backward with the scalar
+    per-head gate (g [B, H, L])."""
+    from gated_linear_sliding_chunkwise_b200.synth import WORKLOADS, make_inputs
+
+    w = WORKLOADS["train_step"]
+    impl = {"auto": lz.IMPL_AUTO, "simt": lz.IMPL_SIMT, "tc": lz.IMPL_TC}[args.kernels]
+    out = {}
+    tokens = w.B * w.L
+    fl = flops_per_token_head(w.d, w.chunk, w.window, w.M)["train"] * w.B * w.H * w.L
+
+    inp = make_inputs(w, seed=w.seed + rank)
+    x = {k: v.to(dev).contiguous() for k, v in inp.items()}
+    gen = torch.Generator().manual_seed(1000 + rank)
+    target = (torch.randn(*x["q"].shape, generator=gen) / 8).to(x["q"].dtype).to(dev)
+    kw = dict(window=w.window, chunk=w.chunk, gate_temp=w.gate_temp, fmap_wq=x["fmap_wq"],
+              fmap_wk=x["fmap_wk"], meta_k=x["meta_k"], meta_v=x["meta_v"], alpha=x["alpha"],
+              impl=impl)
+    names = lz.stage1_step(x["q"], x["k"], x["v"], x["g"], target, plan_only=True, **kw)
+    ws = lz.stage1_step(x["q"], x["k"], x["v"], x["g"], target, **kw)["workspace"]
+    ms, per = _time_steps(lambda ev: lz.stage1_step(x["q"], x["k"], x["v"], x["g"], target, workspace=ws,
+                                                    events=ev, **kw),
+                          names, lz, world, dev, args.warmup, steps)
+    out["stage1_step"] = {
+        "workload": f"train_step shape, stage-1 step (loss fused in the forward): B={w.B} H={w.H} L={w.L}",
+        "ms": ms, "tokens_per_s": world * tokens / (ms / 1e3),
+        "tflops": world * fl / (ms / 1e3) / 1e12, "kernel_ms": per, "launches": len(names)}
+    del x, ws
+
+    inp = make_inputs(w, seed=w.seed + rank, gate="scalar")
+    x = {k: v.to(dev).contiguous() for k, v in inp.items()}
+    kw = dict(window=w.window, chunk=w.chunk, gate_temp=w.gate_temp, fmap_wq=x["fmap_wq"],
+              fmap_wk=x["fmap_wk"], meta_k=x["meta_k"], meta_v=x["meta_v"], alpha=x["alpha"],
+              impl=impl)
+    fn = lz.attn_fwd(x["q"], x["k"], x["v"], x["g"], plan_only=True, **kw)
+    bn = lz.attn_bwd(x["q"], x["k"], x["v"], x["g"], x["dout"], plan_only=True, **kw)
+    o = torch.empty_like(x["q"])
+    fws = lz.attn_fwd(x["q"], x["k"], x["v"], x["g"], out=o, **kw)["workspace"]
+    bws = lz.attn_bwd(x["q"], x["k"], x["v"], x["g"], x["dout"], **kw)["workspace"]
+    msf, perf = _time_steps(lambda ev: lz.attn_fwd(x["q"], x["k"], x["v"], x["g"], out=o, workspace=fws,
+                                                   events=ev, **kw), fn, lz, world, dev, args.warmup, steps)
+    msb, perb = _time_steps(lambda ev: lz.attn_bwd(x["q"], x["k"], x["v"], x["g"], x["dout"], workspace=bws,
+                                                   events=ev, **kw), bn, lz, world, dev, args.warmup, steps)
+    out["scalar_gate_train_step"] = {
+        "workload": f"train_step shape, scalar per-head gate g [B,H,L]: B={w.B} H={w.H} L={w.L}",
+        "ms": msf + msb, "fwd_ms": msf, "bwd_ms": msb,
+        "tokens_per_s": world * tokens / ((msf + msb) / 1e3),
+        "kernel_ms": {**perf, **{("bwd:" + n): t for n, t in perb.items()}},
+        "launches": len(fn) + len(bn)}
+    return out
 
 
 def run_decode(args, lz, dev, rank, world, peaks):
@@ -606,6 +693,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-fwd-long", action="store_true")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the stage-1 step and scalar-gate timings")
     ap.add_argument("--only", choices=["train", "fwd", "bwd"], default="train",
                     help="fwd / bwd: time one entry point alone on --workload (profiling aid)")
     ap.add_argument("--workload", default="llama8b_layer_fwd")

@@ -157,7 +157,7 @@ float scale_of(const lizard_fwd_args *a) {
 // A call's kernels in launch order.  The same list serves the launch and the
 // host-only plan query, so the names always match what runs.
 struct Plan {
-  static constexpr int kMax = 16;
+  static constexpr int kMax = 24;
   const char *names[kMax];
   std::function<cudaError_t()> fns[kMax];
   int n = 0;
@@ -182,7 +182,10 @@ struct Plan {
   }
 };
 
-void fwd_plan(const lizard_fwd_args *a, void *ws, cudaStream_t s, Plan &plan) {
+// `target`, `dmse`, `loss`: the stage-1 loss, which the tensor-core forward
+// forms in its epilogue (null otherwise).
+void fwd_plan(const lizard_fwd_args *a, void *ws, cudaStream_t s, Plan &plan, const void *target = nullptr,
+              void *dmse = nullptr, float *loss = nullptr) {
   const FwdLayout lay = fwd_layout(a);
   const int BH = a->B * a->H, D = a->dk;
   const bool bf16 = a->dtype == LIZARD_BF16;
@@ -190,7 +193,7 @@ void fwd_plan(const lizard_fwd_args *a, void *ws, cudaStream_t s, Plan &plan) {
     lz::TcFwdArgs t{a->q, a->k, a->v, a->g, a->fmap_wq, a->fmap_wk, a->meta_k, a->meta_v, a->alpha,
                     a->state_in, a->o, gla_on(a) ? a->state_out : nullptr, swa_on(a) ? a->lse : nullptr,
                     static_cast<uint32_t *>(ws), at<void>(ws, lay.phq), BH, a->H, a->L, a->M, a->window,
-                    a->branch, 1.f / a->gate_temp, scale_of(a), scalar_gate(a)};
+                    a->branch, 1.f / a->gate_temp, scale_of(a), scalar_gate(a), target, dmse, loss};
     if (gla_on(a)) plan.add("gate_prep_kernel", [=] { return lz::launch_tc_fwd(t, 3, s); });
     if (lz::tc_fwd_stage_count(BH, a->L) > 1) {
       plan.add("tc_fwd_kernel(state pass)", [=] { return lz::launch_tc_fwd(t, 0, s); });
@@ -402,6 +405,23 @@ size_t lizard_bwd_workspace_size(const lizard_bwd_args *args) {
   return bwd_layout(&a, args->impl).total;
 }
 
+// Gradient outputs that the kernels accumulate atomically start at zero; so
+// does dstate_in when no kernel writes it.
+static cudaError_t bwd_zero_outputs(const lizard_bwd_args *b, cudaStream_t s) {
+  const lizard_fwd_args *a = &b->fwd;
+  const int BH = a->B * a->H, D = a->dk, F = D / 2;
+  cudaError_t e = cudaSuccess;
+  struct Z { void *p; size_t n; } zs[] = {
+      {b->dmeta_k, (size_t)a->H * a->M * a->dk * 4}, {b->dmeta_v, (size_t)a->H * a->M * a->dv * 4},
+      {b->dfmap_wq, (size_t)a->H * D * F * 4},       {b->dfmap_wk, (size_t)a->H * D * F * 4},
+      {b->dalpha, (size_t)a->H * 4}};
+  for (const Z &z : zs)
+    if (z.p && z.n && (e = cudaMemsetAsync(z.p, 0, z.n, s)) != cudaSuccess) return e;
+  const size_t BHdd = (size_t)BH * a->dk * a->dv * sizeof(float);
+  if ((a->L == 0 || !gla_on(a)) && b->dstate_in) e = cudaMemsetAsync(b->dstate_in, 0, BHdd, s);
+  return e;
+}
+
 lizard_status lizard_attn_bwd(const lizard_bwd_args *b, lizard_stream_t stream) {
   lizard_status st = check_bwd(b);
   if (st != LIZARD_OK) return st;
@@ -411,25 +431,138 @@ lizard_status lizard_attn_bwd(const lizard_bwd_args *b, lizard_stream_t stream) 
   const BwdLayout lay = bwd_layout(a, b->impl);
   if (!b->workspace || b->workspace_bytes < lay.total) return LIZARD_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int BH = a->B * a->H, D = a->dk, F = D / 2;
-  void *ws = b->workspace;
-  cudaError_t e = cudaSuccess;
-  // outputs that are accumulated atomically start at zero
-  struct Z { void *p; size_t n; } zs[] = {
-      {b->dmeta_k, (size_t)a->H * a->M * a->dk * 4}, {b->dmeta_v, (size_t)a->H * a->M * a->dv * 4},
-      {b->dfmap_wq, (size_t)a->H * D * F * 4},       {b->dfmap_wk, (size_t)a->H * D * F * 4},
-      {b->dalpha, (size_t)a->H * 4}};
-  for (const Z &z : zs)
-    if (z.p && z.n && (e = cudaMemsetAsync(z.p, 0, z.n, s)) != cudaSuccess) return LIZARD_ERR_CUDA;
-  const size_t BHdd = (size_t)BH * a->dk * a->dv * sizeof(float);
-  if (a->L == 0 || !gla_on(a)) {
-    if (b->dstate_in && (e = cudaMemsetAsync(b->dstate_in, 0, BHdd, s)) != cudaSuccess) return LIZARD_ERR_CUDA;
-  }
+  if (bwd_zero_outputs(b, s) != cudaSuccess) return LIZARD_ERR_CUDA;
   if (a->L == 0) return LIZARD_OK;
+  void *ws = b->workspace;
   if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), s) != cudaSuccess) return LIZARD_ERR_CUDA;
   Plan plan;
   bwd_plan(b, ws, s, plan);
   return plan.run(s, b->launch_events, b->n_launch_events);
+}
+
+// ---------------------------------------------------------- stage 1 ----
+// One workspace for the whole step: the forward's and the backward's scratch
+// share its start (the backward begins after the forward's last kernel, and
+// both keep the status word at offset 0), then dL/do, then the output when
+// the portable forward needs one and the caller gave none.
+}  // extern "C"
+
+namespace {
+
+struct S1Layout {
+  size_t dmse, o, total;
+};
+S1Layout s1_layout(const lizard_stage1_args *a) {
+  const lizard_bwd_args *b = &a->bwd;
+  const lizard_fwd_args *f = &b->fwd;
+  const size_t fw = fwd_layout(f).total, bw = bwd_layout(f, b->impl).total;
+  const size_t nel = (size_t)f->B * f->H * f->L * f->dv, esz = f->dtype == LIZARD_BF16 ? 2 : 4;
+  S1Layout l{};
+  size_t off = up(fw > bw ? fw : bw);
+  l.dmse = off;
+  off += up(nel * esz);
+  if (!f->o && !fwd_uses_tc(f)) {
+    l.o = off;
+    off += up(nel * esz);
+  }
+  l.total = off;
+  return l;
+}
+
+lizard_status check_stage1(const lizard_stage1_args *a) {
+  if (!a) return LIZARD_ERR_INVALID_ARG;
+  lizard_bwd_args b = a->bwd;
+  b.dout = b.dq;   // dL/do comes from the loss; dq stands in for the pointer check
+  const lizard_status st = check_bwd(&b);
+  if (st != LIZARD_OK) return st;
+  if (b.fwd.L > 0 && (!a->target || !a->loss)) return LIZARD_ERR_INVALID_ARG;
+  if (!ok_ptr(a->target) || !ok_ptr(a->loss) || !ok_ptr(b.fwd.o)) return LIZARD_ERR_INVALID_ARG;
+  return LIZARD_OK;
+}
+
+// The forward and backward argument views that the step's kernels read; they
+// must outlive the plan's run.
+struct S1Views {
+  lizard_fwd_args f;
+  lizard_bwd_args b;
+};
+
+void stage1_plan(const lizard_stage1_args *a, S1Views &v, void *ws, cudaStream_t s, Plan &plan) {
+  const S1Layout lay = s1_layout(a);
+  v.b = a->bwd;
+  v.f = a->bwd.fwd;
+  v.f.workspace = ws;
+  void *dmse = at<void>(ws, lay.dmse);
+  const lizard_fwd_args *f = &v.f;
+  if (fwd_uses_tc(f)) {
+    fwd_plan(f, ws, s, plan, a->target, dmse, a->loss);
+  } else {
+    if (!v.f.o) v.f.o = at<void>(ws, lay.o);
+    fwd_plan(f, ws, s, plan);
+    const size_t nel = (size_t)f->B * f->H * f->L * f->dv;
+    const bool bf16 = f->dtype == LIZARD_BF16;
+    const void *target = a->target;
+    float *loss = a->loss;
+    plan.add("mse_kernel", [=] { return lz::launch_mse(f->o, target, dmse, loss, nel, bf16, s); });
+  }
+  v.b.dout = dmse;
+  bwd_plan(&v.b, ws, s, plan);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t lizard_stage1_workspace_size(const lizard_stage1_args *args) {
+  if (!args) return 0;
+  lizard_stage1_args a = *args;
+  lizard_fwd_args &f = a.bwd.fwd;
+  f.impl = args->bwd.fwd.impl;
+  const bool keep_o = f.o != nullptr;
+  f.q = f.k = f.v = f.g = nullptr;
+  f.o = nullptr;
+  f.fmap_wq = f.fmap_wk = f.alpha = f.state_in = nullptr;
+  f.state_out = f.lse = nullptr;
+  f.meta_k = f.M > 0 ? reinterpret_cast<const float *>(16) : nullptr;
+  f.meta_v = nullptr;
+  if (f.L > 0) f.q = f.k = f.v = f.g = reinterpret_cast<const void *>(16);
+  f.workspace = nullptr;
+  lizard_fwd_args chk = f;
+  chk.o = reinterpret_cast<void *>(16);
+  if (check_fwd(&chk) != LIZARD_OK) return 0;
+  if (keep_o) f.o = reinterpret_cast<void *>(16);
+  return s1_layout(&a).total;
+}
+
+lizard_status lizard_stage1_step(const lizard_stage1_args *a, lizard_stream_t stream) {
+  lizard_status st = check_stage1(a);
+  if (st != LIZARD_OK) return st;
+  const lizard_bwd_args *b = &a->bwd;
+  const lizard_fwd_args *f = &b->fwd;
+  if (f->impl == LIZARD_IMPL_TC && !fwd_uses_tc(f)) return LIZARD_ERR_UNSUPPORTED;
+  if (b->impl == LIZARD_IMPL_TC && swa_on(f) && !bwd_swa_uses_tc(f, b->impl)) return LIZARD_ERR_UNSUPPORTED;
+  if (b->impl == LIZARD_IMPL_TC && gla_on(f) && !bwd_gla_uses_tc(f, b->impl)) return LIZARD_ERR_UNSUPPORTED;
+  const S1Layout lay = s1_layout(a);
+  if (!b->workspace || b->workspace_bytes < lay.total) return LIZARD_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (bwd_zero_outputs(b, s) != cudaSuccess) return LIZARD_ERR_CUDA;
+  if (a->loss && cudaMemsetAsync(a->loss, 0, sizeof(float), s) != cudaSuccess) return LIZARD_ERR_CUDA;
+  if (f->L == 0) return LIZARD_OK;
+  void *ws = b->workspace;
+  if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), s) != cudaSuccess) return LIZARD_ERR_CUDA;
+  S1Views views;
+  Plan plan;
+  stage1_plan(a, views, ws, s, plan);
+  return plan.run(s, b->launch_events, b->n_launch_events);
+}
+
+int32_t lizard_stage1_launch_plan(const lizard_stage1_args *a, const char **names, int32_t cap) {
+  if (check_stage1(a) != LIZARD_OK) return -1;
+  if (a->bwd.fwd.L == 0) return 0;
+  S1Views views;
+  Plan plan;
+  stage1_plan(a, views, a->bwd.workspace, nullptr, plan);
+  return plan.names_out(names, cap);
 }
 
 int32_t lizard_fwd_launch_plan(const lizard_fwd_args *a, const char **names, int32_t cap) {

@@ -110,6 +110,12 @@ struct TcFwdArgs {
   int BH, H, L, M, window, branch;
   float inv_tau, scale;
   int scalar_gate;    // g holds one logit per (token, head): [B*H][L]
+  // Stage-1 loss in the full pass's epilogue (target null: off): with
+  // n = B*H*L*128, dmse = 2 (o - target) / n (bf16) and *loss += sum (o - target)^2 / n.
+  // o may be null when the loss is on.
+  const void *target;
+  void *dmse;
+  float *loss;
 };
 
 struct TcSwaBwdArgs {
@@ -178,6 +184,10 @@ cudaError_t launch_tc_state_snapshots(const TcFwdArgs &a, void *snap, const floa
 // either may be null) and the tiles' log-decays r [BH][ntiles][128], from bf16
 // gate logits g [BH][L][128] (scalar_gate: [BH][L], one logit for all 128
 // dimensions); sets bit 2 of *status when a tile's spread is too wide.
+// Stage-1 loss over n elements of o and target (dtype): dout = 2 (o - target) / n,
+// *loss += sum (o - target)^2 / n (the caller zeroes *loss first).
+cudaError_t launch_mse(const void *o, const void *target, void *dout, float *loss, size_t n, bool bf16,
+                       cudaStream_t s);
 cudaError_t launch_gate_prep(const void *g, void *E16, float *E32, float *r, uint32_t *status, int BH, int L,
                              float inv_tau, bool scalar_gate, cudaStream_t s);
 // stage 0: reverse dS pass, 1: per-tile gradients, 2: gate-logit gradient

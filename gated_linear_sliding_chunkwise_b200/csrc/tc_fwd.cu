@@ -96,6 +96,11 @@ struct Params {
   int mode;                 // 0: full forward, 1: state pass
   int nseg, tiles_per_seg;
   float inv_tau, scale;
+  // stage-1 loss (target null: off): dmse = mse_grad (o - target), *loss += mse_loss sum (o - target)^2
+  const __nv_bfloat16 *target;
+  __nv_bfloat16 *dmse;
+  float *loss;
+  float mse_grad, mse_loss;
 };
 
 
@@ -160,6 +165,9 @@ __device__ __forceinline__ void kt_half(unsigned char *sm, uint32_t tl, int row,
 constexpr int BAR_A = 1;       // both groups' row maxima written
 constexpr int BAR_B = 2;       // both groups' row sums written, all logits read
 
+// LOSS: the full pass also forms the stage-1 loss (p.target set).  A separate
+// instance, so that the plain forward keeps its register budget.
+template <bool LOSS>
 __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_constant__ Params p) {
   extern __shared__ unsigned char smraw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
@@ -172,6 +180,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
   __shared__ uint64_t bar_tma, bar_vp, bar_m1, bar_m2, bar_m3;
   __shared__ uint32_t s_tmem;
   __shared__ int s_fail;
+  __shared__ float s_mse[NTHREADS / 32];
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const int wg = tid >> 7;                             // warpgroup
@@ -249,11 +258,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
   const uint32_t id_mn = idesc_bf16(128, 128, 0, 1);
   const uint32_t id_st = idesc_bf16(128, 128, 1, 1);
 
+  float mse_acc = 0.f;                        // this thread's share of sum (o - target)^2
   for (int c = cbeg; c < cend; ++c) {
     const uint32_t par = (c - cbeg) & 1;
     const int t0 = c * T;
     const int tq = t0 + row;                  // this thread's query token
     const bool qvalid = tq < p.L;
+    if (LOSS && full && qvalid)               // the epilogue's target half-row, toward L2 early
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(p.target + ((size_t)bh * p.L + tq) * D + 64 * wg));
 
     // ---------------------------------------------------------- MMA 1 ---
     bool ok = mbar_wait(&bar_tma, par, err, ST_TIMEOUT);
@@ -520,6 +532,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         for (int s = 0; s < 8; ++s) mma_ss(tb + C_S, desc_mn(kt, s), desc_mn(v, s), id_st, 1);
       mma_commit(&bar_m3);
     }
+    // stage-1 loss: this thread's half-row of the target, in flight during MMA 3
+    uint4 ytgt[8];
+    if (LOSS && full && qvalid) {
+      const uint4 *yp = reinterpret_cast<const uint4 *>(p.target + ((size_t)bh * p.L + tq) * D + 64 * wg);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) ytgt[u] = yp[u];
+    }
     ok = mbar_wait(&bar_m3, par, err, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) { s_fail = 1; break; }
     tc_fence_after();
@@ -528,9 +547,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
     // ---------------------------- epilogue (column half per group) ---
     if (full) {
       // tcgen05.ld is warp-collective: every lane loads, valid rows store
-      __nv_bfloat16 *orow = p.o + ((size_t)bh * p.L + (qvalid ? tq : 0)) * D;
+      const size_t roff = ((size_t)bh * p.L + (qvalid ? tq : 0)) * D;
       const float oscale = s_oscale[row];
-      for (int c16 = 4 * wg; c16 < 4 * wg + 4; ++c16) {
+#pragma unroll(LOSS ? 4 : 1)
+      for (int k4 = 0; k4 < 4; ++k4) {
+        const int c16 = 4 * wg + k4;
         float v[16];
         tmem_ld16(tl + C_O + c16 * 16, v);
 #pragma unroll
@@ -549,10 +570,24 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
             }
           }
         }
-        if (qvalid) {
-          uint4 *dst = reinterpret_cast<uint4 *>(orow + c16 * 16);
+        if (qvalid && p.o) {
+          uint4 *dst = reinterpret_cast<uint4 *>(p.o + roff + c16 * 16);
           dst[0] = pack8(v);
           dst[1] = pack8(v + 8);
+        }
+        if (LOSS && qvalid) {       // stage-1 loss: (o - y)^2 and dL/do from the fp32 o
+          float y[16];
+          unpack8(ytgt[2 * k4], y);
+          unpack8(ytgt[2 * k4 + 1], y + 8);
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const float d = v[u] - y[u];
+            mse_acc = fmaf(d, d, mse_acc);
+            y[u] = d * p.mse_grad;
+          }
+          uint4 *dd = reinterpret_cast<uint4 *>(p.dmse + roff + c16 * 16);
+          dd[0] = pack8(y);
+          dd[1] = pack8(y + 8);
         }
       }
     }
@@ -560,6 +595,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
     __syncthreads();
   }
 
+  if (LOSS && full) {       // one atomic per CTA
+    const float t = warp_sum(mse_acc);
+    if ((tid & 31) == 0) s_mse[warp] = t;
+    __syncthreads();
+    if (tid == 0) {
+      float tot = 0.f;
+      for (int w = 0; w < NTHREADS / 32; ++w) tot += s_mse[w];
+      atomicAdd(p.loss, tot * p.mse_loss);
+    }
+  }
   float *sdst = nullptr;
   if (full && p.state_out && gla && seg == p.nseg - 1) sdst = p.state_out + ((size_t)bh * D + row) * D;
   if (!full && p.seg_state) {
@@ -797,9 +842,10 @@ cudaError_t launch_tc_state_snapshots(const TcFwdArgs &a, void *snap, const floa
   p.seg_start = a.state_in;
   p.seg_state = nullptr;
   p.seg_decay = nullptr;
-  cudaError_t e = cudaFuncSetAttribute(tc_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+  cudaError_t e =
+      cudaFuncSetAttribute(tc_fwd_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  tc_fwd_kernel<<<dim3(a.BH, 1), NTHREADS, SMEM_BYTES, s>>>(p);
+  tc_fwd_kernel<false><<<dim3(a.BH, 1), NTHREADS, SMEM_BYTES, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -834,6 +880,14 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, int stage, cudaStream_t s) {
   p.alpha = a.alpha;
   p.state_in = a.state_in;
   p.o = static_cast<__nv_bfloat16 *>(a.o);
+  p.target = static_cast<const __nv_bfloat16 *>(a.target);
+  p.dmse = static_cast<__nv_bfloat16 *>(a.dmse);
+  p.loss = a.loss;
+  {
+    const double n = (double)a.BH * a.L * D;
+    p.mse_grad = (float)(2.0 / n);
+    p.mse_loss = (float)(1.0 / n);
+  }
   p.state_out = a.state_out;
   p.lse = a.lse;
   p.status = a.status;
@@ -854,16 +908,21 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, int stage, cudaStream_t s) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64 || configured[dev] < SMEM_BYTES) {
-    e = cudaFuncSetAttribute(tc_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    e = cudaFuncSetAttribute(tc_fwd_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(tc_fwd_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) configured[dev] = SMEM_BYTES;
   }
   if (nseg > 1 && stage == 0) {          // state pass over every segment but the last
     p.mode = 1;
-    tc_fwd_kernel<<<dim3(a.BH, nseg - 1), NTHREADS, SMEM_BYTES, s>>>(p);
+    tc_fwd_kernel<false><<<dim3(a.BH, nseg - 1), NTHREADS, SMEM_BYTES, s>>>(p);
   } else {                               // full pass
     p.mode = 0;
-    tc_fwd_kernel<<<dim3(a.BH, nseg), NTHREADS, SMEM_BYTES, s>>>(p);
+    if (p.target)
+      tc_fwd_kernel<true><<<dim3(a.BH, nseg), NTHREADS, SMEM_BYTES, s>>>(p);
+    else
+      tc_fwd_kernel<false><<<dim3(a.BH, nseg), NTHREADS, SMEM_BYTES, s>>>(p);
   }
   return cudaGetLastError();
 }

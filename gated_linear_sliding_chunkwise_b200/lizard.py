@@ -65,6 +65,10 @@ class DecodeArgs(ctypes.Structure):
                 ("alpha", _vp), ("o", _vp)]
 
 
+class Stage1Args(ctypes.Structure):
+    _fields_ = [("bwd", BwdArgs), ("target", _vp), ("loss", _vp)]
+
+
 _lib.lizard_fwd_workspace_size.argtypes = [ctypes.POINTER(FwdArgs)]
 _lib.lizard_fwd_workspace_size.restype = ctypes.c_size_t
 _lib.lizard_attn_fwd.argtypes = [ctypes.POINTER(FwdArgs), _vp]
@@ -77,6 +81,12 @@ _lib.lizard_fwd_launch_plan.argtypes = [ctypes.POINTER(FwdArgs), ctypes.POINTER(
 _lib.lizard_fwd_launch_plan.restype = _i32
 _lib.lizard_bwd_launch_plan.argtypes = [ctypes.POINTER(BwdArgs), ctypes.POINTER(ctypes.c_char_p), _i32]
 _lib.lizard_bwd_launch_plan.restype = _i32
+_lib.lizard_stage1_workspace_size.argtypes = [ctypes.POINTER(Stage1Args)]
+_lib.lizard_stage1_workspace_size.restype = ctypes.c_size_t
+_lib.lizard_stage1_step.argtypes = [ctypes.POINTER(Stage1Args), _vp]
+_lib.lizard_stage1_step.restype = ctypes.c_int
+_lib.lizard_stage1_launch_plan.argtypes = [ctypes.POINTER(Stage1Args), ctypes.POINTER(ctypes.c_char_p), _i32]
+_lib.lizard_stage1_launch_plan.restype = _i32
 _lib.lizard_decode_step.argtypes = [ctypes.POINTER(DecodeArgs), _vp]
 _lib.lizard_decode_step.restype = ctypes.c_int
 class CacheArgs(ctypes.Structure):
@@ -245,15 +255,8 @@ def attn_fwd(q, k, v, g, *, window, chunk=64, gate_temp=16.0, softmax_scale=0.0,
     return {"o": o, "state_out": S, "lse": lse, "workspace": ws}
 
 
-def attn_bwd(q, k, v, g, dout, *, window, chunk=64, gate_temp=16.0, softmax_scale=0.0,
-             fmap_wq=None, fmap_wk=None, meta_k=None, meta_v=None, alpha=None,
-             state_in=None, branch=BRANCH_BOTH, impl=IMPL_AUTO, want_dstate=True,
-             workspace=None, stream=None, events=None, plan_only=False):
-    """Backward of the hybrid layer (lizard_attn_bwd); returns every gradient."""
-    f = _fwd_struct(q, k, v, g, window=window, chunk=chunk, gate_temp=gate_temp,
-                    softmax_scale=softmax_scale, fmap_wq=fmap_wq, fmap_wk=fmap_wk,
-                    meta_k=meta_k, meta_v=meta_v, alpha=alpha, state_in=state_in,
-                    branch=branch, impl=impl)
+def _bwd_struct(f, q, k, v, g, dout, *, meta_k, meta_v, fmap_wq, fmap_wk, impl, want_dstate):
+    """Gradient buffers and the lizard_bwd_args that point at them."""
     B, H, L, dk = q.shape
     dv_ = v.shape[-1]
     dev = q.device
@@ -275,6 +278,21 @@ def attn_bwd(q, k, v, g, dout, *, window, chunk=64, gate_temp=16.0, softmax_scal
                  "dalpha", "dstate_in"):
         setattr(b, name, _ptr(res[name]))
     b.impl = impl
+    return b, res
+
+
+def attn_bwd(q, k, v, g, dout, *, window, chunk=64, gate_temp=16.0, softmax_scale=0.0,
+             fmap_wq=None, fmap_wk=None, meta_k=None, meta_v=None, alpha=None,
+             state_in=None, branch=BRANCH_BOTH, impl=IMPL_AUTO, want_dstate=True,
+             workspace=None, stream=None, events=None, plan_only=False):
+    """Backward of the hybrid layer (lizard_attn_bwd); returns every gradient."""
+    f = _fwd_struct(q, k, v, g, window=window, chunk=chunk, gate_temp=gate_temp,
+                    softmax_scale=softmax_scale, fmap_wq=fmap_wq, fmap_wk=fmap_wk,
+                    meta_k=meta_k, meta_v=meta_v, alpha=alpha, state_in=state_in,
+                    branch=branch, impl=impl)
+    b, res = _bwd_struct(f, q, k, v, g, dout, meta_k=meta_k, meta_v=meta_v, fmap_wq=fmap_wq,
+                         fmap_wk=fmap_wk, impl=impl, want_dstate=want_dstate)
+    dev = q.device
     nbytes = bwd_workspace_bytes(b)
     ws = _workspace(nbytes, dev, workspace)
     b.workspace, b.workspace_bytes = ws.data_ptr(), ws.numel() * ws.element_size()
@@ -284,6 +302,38 @@ def attn_bwd(q, k, v, g, dout, *, window, chunk=64, gate_temp=16.0, softmax_scal
     _check(_lib.lizard_attn_bwd(ctypes.byref(b), _stream(stream)), "lizard_attn_bwd")
     del keep
     res["workspace"] = ws
+    return res
+
+
+def stage1_step(q, k, v, g, target, *, window, chunk=64, gate_temp=16.0, softmax_scale=0.0,
+                fmap_wq=None, fmap_wk=None, meta_k=None, meta_v=None, alpha=None,
+                state_in=None, branch=BRANCH_BOTH, impl=IMPL_AUTO, want_o=False,
+                want_dstate=True, workspace=None, stream=None, events=None, plan_only=False):
+    """One stage-1 training step (lizard_stage1_step): forward, the mean squared
+    error against the teacher output `target`, and every gradient of it.
+    Returns the gradients plus "loss" (a one-element fp32 tensor) and "o"
+    (when want_o)."""
+    f = _fwd_struct(q, k, v, g, window=window, chunk=chunk, gate_temp=gate_temp,
+                    softmax_scale=softmax_scale, fmap_wq=fmap_wq, fmap_wk=fmap_wk,
+                    meta_k=meta_k, meta_v=meta_v, alpha=alpha, state_in=state_in,
+                    branch=branch, impl=impl)
+    o = torch.empty(*q.shape[:-1], v.shape[-1], dtype=q.dtype, device=q.device) if want_o else None
+    f.o = _ptr(o)
+    b, res = _bwd_struct(f, q, k, v, g, None, meta_k=meta_k, meta_v=meta_v, fmap_wq=fmap_wq,
+                         fmap_wk=fmap_wk, impl=impl, want_dstate=want_dstate)
+    loss = torch.zeros(1, dtype=torch.float32, device=q.device)
+    a = Stage1Args()
+    a.bwd = b
+    a.target, a.loss = _ptr(target), _ptr(loss)
+    nbytes = int(_lib.lizard_stage1_workspace_size(ctypes.byref(a)))
+    ws = _workspace(nbytes, q.device, workspace)
+    a.bwd.workspace, a.bwd.workspace_bytes = ws.data_ptr(), ws.numel() * ws.element_size()
+    if plan_only:
+        return _plan(_lib.lizard_stage1_launch_plan, a)
+    keep = _attach_events(a.bwd, events)
+    _check(_lib.lizard_stage1_step(ctypes.byref(a), _stream(stream)), "lizard_stage1_step")
+    del keep
+    res.update(loss=loss, o=o, workspace=ws)
     return res
 
 

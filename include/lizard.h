@@ -184,11 +184,43 @@ typedef struct {
 size_t lizard_bwd_workspace_size(const lizard_bwd_args *args);
 lizard_status lizard_attn_bwd(const lizard_bwd_args *args, lizard_stream_t stream);
 
-/* Kernels lizard_attn_fwd / lizard_attn_bwd launch for these arguments, in
+/*
+ * One stage-1 training step (attention approximation: the layer learns to
+ * reproduce a teacher's softmax-attention output under a mean squared error;
+ * English summary, section 2.B "Stage 1"; Chinese summary, section 2.2):
+ * the forward, the loss, and the gradients of the loss with respect to every
+ * input, in one call.
+ *
+ *   bwd      inputs and gradient outputs exactly as in lizard_attn_bwd, with
+ *            two differences: bwd.dout is ignored (dL/do comes from the loss),
+ *            and bwd.fwd.o may be NULL (the output is then not kept) or
+ *            receives o.  bwd.fwd.impl selects the forward's kernels,
+ *            bwd.impl the backward's.  bwd.workspace and bwd.launch_events
+ *            serve the whole step.
+ *   target   [B, H, L, dv] dtype: the teacher's attention output y
+ *   loss     one fp32, written: sum over every element of (o - y)^2 divided
+ *            by the element count B H L dv; dL/do = 2 (o - y) / (B H L dv)
+ *            (o before its rounding to dtype)
+ * The tensor-core forward forms the loss and dL/do in its epilogue; the
+ * portable path adds one elementwise kernel.  The workspace (at least
+ * lizard_stage1_workspace_size() bytes) holds dL/do between the two halves.
+ * Errors as lizard_attn_bwd.
+ */
+typedef struct {
+  lizard_bwd_args bwd;
+  const void *target;
+  float *loss;
+} lizard_stage1_args;
+
+size_t lizard_stage1_workspace_size(const lizard_stage1_args *args);
+lizard_status lizard_stage1_step(const lizard_stage1_args *args, lizard_stream_t stream);
+
+/* Kernels lizard_attn_fwd / lizard_attn_bwd / lizard_stage1_step launch for these arguments, in
  * launch order: fills names[0 .. min(count, cap)) with static strings and
  * returns count (-1 when the arguments are invalid).  Host only. */
 int32_t lizard_fwd_launch_plan(const lizard_fwd_args *args, const char **names, int32_t cap);
 int32_t lizard_bwd_launch_plan(const lizard_bwd_args *args, const char **names, int32_t cap);
+int32_t lizard_stage1_launch_plan(const lizard_stage1_args *args, const char **names, int32_t cap);
 
 /*
  * One decode step for every sequence: the constant-memory generation of the

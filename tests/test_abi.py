@@ -49,6 +49,7 @@ def test_struct_layouts_match_c(lz, tmp_path):
     fields = {
         "lizard_fwd_args": lz.FwdArgs, "lizard_bwd_args": lz.BwdArgs,
         "lizard_decode_args": lz.DecodeArgs, "lizard_cache_args": lz.CacheArgs,
+        "lizard_stage1_args": lz.Stage1Args,
     }
     lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "lizard.h"',
              "int main(void) {"]
@@ -190,3 +191,42 @@ def test_prefill_cache_rejects_bad_arguments_on_host(lz):
     assert lz.lib().lizard_prefill_cache(ctypes.byref(a), None) == lz.ERR_INVALID_ARG   # no buffers
     a.dk = a.dv = 96
     assert lz.lib().lizard_prefill_cache(ctypes.byref(a), None) == lz.ERR_UNSUPPORTED
+
+
+def _stage1(lz, **over):
+    a = lz.Stage1Args()
+    a.bwd.fwd = _fwd(lz, dk=128, dv=128)
+    fake = 0x10000
+    a.bwd.dq = a.bwd.dk = a.bwd.dv = a.bwd.dg = fake
+    a.target, a.loss = fake, 0x30000
+    for k_, v_ in over.items():
+        setattr(a, k_, v_)
+    return a
+
+
+def test_stage1_rejects_bad_arguments_on_host(lz):
+    a = _stage1(lz)
+    need = lz.lib().lizard_stage1_workspace_size(ctypes.byref(a))
+    # dL/do lives in the workspace: it outgrows the backward's own
+    assert need > lz.bwd_workspace_bytes(a.bwd)
+    a.bwd.workspace, a.bwd.workspace_bytes = 0x20000, need - 1
+    assert lz.lib().lizard_stage1_step(ctypes.byref(a), None) == lz.ERR_WORKSPACE
+    for over in ({"target": None}, {"loss": None}, {"target": 0x10008}):
+        b = _stage1(lz, **over)
+        assert lz.lib().lizard_stage1_step(ctypes.byref(b), None) == lz.ERR_INVALID_ARG, over
+    assert lz.lib().lizard_stage1_step(None, None) == lz.ERR_INVALID_ARG
+
+
+def test_stage1_launch_plan_fuses_the_loss_on_tensor_cores(lz):
+    """The tensor-core forward forms the loss in its epilogue; the portable
+    forward adds one elementwise kernel before the backward."""
+    import ctypes as ct
+    for impl, fused in ((lz.IMPL_TC, True), (lz.IMPL_SIMT, False)):
+        a = _stage1(lz)
+        a.bwd.fwd.impl = a.bwd.impl = impl
+        a.bwd.fwd.fmap_wq = a.bwd.fwd.fmap_wk = 0x10000
+        names = (ct.c_char_p * 24)()
+        n = lz.lib().lizard_stage1_launch_plan(ct.byref(a), names, 24)
+        got = [names[i].decode() for i in range(n)]
+        assert ("mse_kernel" in got) != fused, got
+        assert got[-1] in ("gate_grad_kernel", "finish_bwd"), got
