@@ -89,7 +89,8 @@ struct Params {
   const float *seg_start;   // [BH][nseg][D][D] start state of each segment (nseg > 1)
   float *seg_state;         // mode 1: [BH][nseg][D][D] local end state (zero start)
   float *seg_decay;         // mode 1: [BH][nseg][D] summed log-decay of the segment
-  __nv_bfloat16 *snap;      // mode 1 with nseg == 1: [BH][ntiles][D][D] bf16 S' of every tile
+  __nv_bfloat16 *snap;      // mode 1 with nseg == 1: [BH][ntiles][D][D] bf16 S' - 1 S'[0] of every tile
+  float *snap_r0;           // ... and [BH][ntiles][D] fp32 row 0 of S' (the part taken out of every row)
   const float *gate_r;      // [BH][ntiles][D] log-decay r of every tile (gate_prep_kernel)
   const float *gate_e32;    // mode 1: [BH][L][D] fp32 decay factors E (mode 0 loads bf16 E as the G tiles)
   int H, L, M, window, branch;
@@ -138,8 +139,9 @@ __device__ __forceinline__ void qt_half(unsigned char *sm, uint32_t tl, int row,
 
 // Kt for dimensions 64 h .. 64 h + 63: phi_k / E, bf16 into shared memory
 // over X_k.  E comes as bf16 from the gate region (full pass) or as fp32
-// from TMEM (state pass).  Rows past L (where the full pass's E is zero)
-// get Kt = 0.
+// from TMEM (state pass, which also writes the rounding remainder Kt - bf16(Kt)
+// over the K_prev region, so that its state update runs on hi + lo).  Rows
+// past L (where the full pass's E is zero) get Kt = 0.
 __device__ __forceinline__ void kt_half(unsigned char *sm, uint32_t tl, int row, int h, bool e_in_tmem,
                                         bool valid) {
   float ph[F];
@@ -156,8 +158,18 @@ __device__ __forceinline__ void kt_half(unsigned char *sm, uint32_t tl, int row,
     }
 #pragma unroll
     for (int u = 0; u < 16; ++u) k16[u] = valid ? __fdividef(ph[16 * c16 + u] * s, e16[u]) : 0.f;
-    *chunk_ptr(sm, R_XK, row, 8 * h + 2 * c16) = pack8(k16);
-    *chunk_ptr(sm, R_XK, row, 8 * h + 2 * c16 + 1) = pack8(k16 + 8);
+    if (e_in_tmem) {
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint4 hi, lo;
+        split8(k16 + 8 * hh, hi, lo);
+        *chunk_ptr(sm, R_XK, row, 8 * h + 2 * c16 + hh) = hi;
+        *chunk_ptr(sm, R_KP, row, 8 * h + 2 * c16 + hh) = lo;
+      }
+    } else {
+      *chunk_ptr(sm, R_XK, row, 8 * h + 2 * c16) = pack8(k16);
+      *chunk_ptr(sm, R_XK, row, 8 * h + 2 * c16 + 1) = pack8(k16 + 8);
+    }
   }
 }
 
@@ -181,6 +193,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
   __shared__ uint32_t s_tmem;
   __shared__ int s_fail;
   __shared__ float s_mse[NTHREADS / 32];
+  __shared__ __align__(16) float s_row0[D];   // state pass: row 0 of S' (taken out of the copies)
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const int wg = tid >> 7;                             // warpgroup
@@ -482,11 +495,29 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         if (full) {   // bf16 copy S'[i][v], MN-major: rows = i (K of the O = Qt S' product)
           *chunk_ptr(sm, R_XQ, i, 2 * c16) = pack8(v);
           *chunk_ptr(sm, R_XQ, i, 2 * c16 + 1) = pack8(v + 8);
-        } else if (p.snap) {   // the backward's copy of S', row-major [i][v]
-          uint4 *dst = reinterpret_cast<uint4 *>(p.snap + (((size_t)bh * ntiles_all + c) * D + i) * D + c16 * 16);
+        } else if (p.snap && i == 0) {
+#pragma unroll
+          for (int u = 0; u < 16; ++u) s_row0[c16 * 16 + u] = v[u];
+        }
+      }
+      if (!full && p.snap) {
+        // The backward's copy of S', row-major [i][v], stored as S' - 1 S'[0]
+        // in bf16 with row 0 in fp32: the rows of S' share a large common
+        // part (the feature map is close to uniform), which a plain bf16
+        // copy would round element by element.
+        tmem_st_wait();
+        __syncthreads();
+        const size_t tile = (size_t)bh * ntiles_all + c;
+        for (int c16 = 4 * wg; c16 < 4 * wg + 4; ++c16) {
+          float v[16];
+          tmem_ld16(tl + C_S + c16 * 16, v);
+#pragma unroll
+          for (int u = 0; u < 16; ++u) v[u] -= s_row0[c16 * 16 + u];
+          uint4 *dst = reinterpret_cast<uint4 *>(p.snap + (tile * D + i) * D + c16 * 16);
           dst[0] = pack8(v);
           dst[1] = pack8(v + 8);
         }
+        if (tid < D) p.snap_r0[tile * D + tid] = s_row0[tid];
       }
     }
     ok = mbar_wait(&bar_m2, par, err, ST_TIMEOUT);
@@ -530,6 +561,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       }
       if (gla)
         for (int s = 0; s < 8; ++s) mma_ss(tb + C_S, desc_mn(kt, s), desc_mn(v, s), id_st, 1);
+      if (gla && !full)   // the state pass's Kt remainder
+        for (int s = 0; s < 8; ++s) mma_ss(tb + C_S, desc_mn(sbase + R_KP, s), desc_mn(v, s), id_st, 1);
       mma_commit(&bar_m3);
     }
     // stage-1 loss: this thread's half-row of the target, in flight during MMA 3
@@ -828,6 +861,7 @@ cudaError_t launch_tc_state_snapshots(const TcFwdArgs &a, void *snap, const floa
   p.state_in = a.state_in;
   p.status = a.status;
   p.snap = static_cast<__nv_bfloat16 *>(snap);
+  p.snap_r0 = reinterpret_cast<float *>(p.snap + (size_t)a.BH * ((a.L + T - 1) / T) * D * D);
   p.H = a.H;
   p.L = a.L;
   p.M = a.M;

@@ -50,7 +50,8 @@ struct DsParams {
   CUtensorMap mq, mo;
   const float *wq;
   const float *e32, *gate_r;   // fp32 decay factors [BH*L][D] and tile log-decays [BH][ntiles][D]
-  __nv_bfloat16 *snap;      // [BH][ntiles][D][D] dS at each tile's end
+  __nv_bfloat16 *snap;      // [BH][ntiles][D][D] dS - 1 dS[0] at each tile's end (bf16)
+  float *snap_r0;           // [BH][ntiles][D] row 0 of that dS (fp32)
   float *dstate_in;         // [BH][D][D] or null
   uint32_t *status;
   int H, L;
@@ -62,6 +63,7 @@ struct TileParams {
   CUtensorMap mdq, mdk, mdb, mdv;             // fp32 outputs dphi_q, dphi_k, dB, dv (TMA stores)
   const float *wq, *wk;
   const float *e32;            // fp32 decay factors [BH*L][D]
+  const float *sp_r0, *ds_r0;  // [BH*ntiles][D] row 0 of S' and of dS (the copies hold the rest)
   float *dphq, *dphk, *dB, *dv;
   uint32_t *status;
   int H, L, ntiles;
@@ -105,9 +107,11 @@ __global__ void __launch_bounds__(NT_DS, 1) tc_gla_dstates_kernel(const __grid_c
   extern __shared__ unsigned char smraw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
   __shared__ float s_dec[D];
+  __shared__ __align__(16) float s_row0[D];   // row 0 of dS, taken out of the bf16 copy
   __shared__ uint64_t bar_tma, bar_m1, bar_m2;
   __shared__ uint32_t s_tmem;
-  constexpr uint32_t R_XQ = 0, R_G = TILE, R_O = 2 * TILE, R_W = 3 * TILE;
+  // Qt (hi) over X_q, the remainder Qt - bf16(Qt) in R_QL, dO, W_q
+  constexpr uint32_t R_XQ = 0, R_QL = TILE, R_O = 2 * TILE, R_W = 3 * TILE;
   constexpr uint32_t C_S = 0, C_Z = 128, C_E = 256;
   const int tid = threadIdx.x, warp = tid >> 5, wg = tid >> 7, row = tid & 127;
   const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
@@ -153,15 +157,31 @@ __global__ void __launch_bounds__(NT_DS, 1) tc_gla_dstates_kernel(const __grid_c
       for (int s = 0; s < 8; ++s) mma_ss(tb + C_Z, desc_k(sbase + R_XQ, s), desc_mn(sbase + R_W, s), id_z, s > 0);
       mma_commit(&bar_m1);
     }
-    // copy of dS (the gradient into this tile's end state), column half per group
+    // copy of dS (the gradient into this tile's end state), column half per
+    // group, as dS - 1 dS[0] in bf16 with row 0 in fp32 (the rows share a
+    // large common part that a plain bf16 copy would round element by element)
     {
-      __nv_bfloat16 *dst = p.snap + (((size_t)bh * ntiles + c) * D + row) * D;
+      const size_t tile = (size_t)bh * ntiles + c;
+      if ((warp & 3) == 0) {   // the warps holding TMEM lane 0: row 0 to shared memory
+        for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
+          float v[32];
+          tmem_ld32(tl + C_S + ch * 32, v);
+          if (row == 0)
+#pragma unroll
+            for (int u = 0; u < 32; ++u) s_row0[ch * 32 + u] = v[u];
+        }
+      }
+      __syncthreads();
+      __nv_bfloat16 *dst = p.snap + (tile * D + row) * D;
       for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
         float v[32];
         tmem_ld32(tl + C_S + ch * 32, v);
 #pragma unroll
+        for (int u = 0; u < 32; ++u) v[u] -= s_row0[ch * 32 + u];
+#pragma unroll
         for (int u = 0; u < 32; u += 8) *reinterpret_cast<uint4 *>(dst + ch * 32 + u) = pack8(v + u);
       }
+      if (tid < D) p.snap_r0[tile * D + tid] = s_row0[tid];
     }
     // E in fp32 (dimensions 64 wg ..) into TMEM; the tile's decay exp(r)
     e_half_to_tmem(p.e32, ((size_t)bh * p.L + (t0 + row < p.L ? t0 + row : 0)) * D, t0 + row < p.L, wg,
@@ -179,16 +199,22 @@ __global__ void __launch_bounds__(NT_DS, 1) tc_gla_dstates_kernel(const __grid_c
         tmem_ld16(tl + C_E + 64 * wg + 16 * c16, E);
 #pragma unroll
         for (int u = 0; u < 16; ++u) q16[u] = ph[16 * c16 + u] * sc * E[u];
-        *chunk_ptr(sm, R_XQ, row, 8 * wg + 2 * c16) = pack8(q16);
-        *chunk_ptr(sm, R_XQ, row, 8 * wg + 2 * c16 + 1) = pack8(q16 + 8);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          uint4 hi, lo;
+          split8(q16 + 8 * hh, hi, lo);
+          *chunk_ptr(sm, R_XQ, row, 8 * wg + 2 * c16 + hh) = hi;
+          *chunk_ptr(sm, R_QL, row, 8 * wg + 2 * c16 + hh) = lo;
+        }
       }
     }
     fence_proxy_async();
     tc_fence_before();
     if (__syncthreads_or(!ok)) { fail = true; break; }
-    if (tid == 0) {   // dS += Qt^T dO
+    if (tid == 0) {   // dS += (Qt hi + lo)^T dO
       tc_fence_after();
       for (int s = 0; s < 8; ++s) mma_ss(tb + C_S, desc_mn(sbase + R_XQ, s), desc_mn(sbase + R_O, s), id_st, 1);
+      for (int s = 0; s < 8; ++s) mma_ss(tb + C_S, desc_mn(sbase + R_QL, s), desc_mn(sbase + R_O, s), id_st, 1);
       mma_commit(&bar_m2);
     }
     ok = mbar_wait(&bar_m2, par, p.status, ST_TIMEOUT);
@@ -239,6 +265,9 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
   unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
   __shared__ uint64_t bars[8];
   __shared__ uint32_t s_tmem;
+  // Per row: dO . S'[0], V . dS[0], sum_i Kt[i] -- the rank-one parts of GQ,
+  // GK and dv that the copies (S' - 1 S'[0], dS - 1 dS[0]) leave out
+  __shared__ float s_r1[3][T];
   // X_q -> Qt (hi), X_k -> Kt (hi), V, dO, Qt (lo), [W_q | W_k] -> S' -> dS, Kt (lo)
   constexpr uint32_t R_XQ = 0, R_XK = TILE, R_V = 2 * TILE, R_O = 3 * TILE, R_QL = 4 * TILE, R_W = 5 * TILE,
                      R_KL = 6 * TILE;
@@ -277,6 +306,7 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
   const uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
   const uint32_t id_mn = idesc_bf16(128, 128, 0, 1);
   const uint32_t id_z = idesc_bf16(128, 64, 0, 1);
+  float r1[3];   // this half's dO . S'[0], V . dS[0], sum Kt
   bool ok = mbar_wait(&bars[0], 0, p.status, ST_TIMEOUT);
   if (__syncthreads_or(!ok)) goto done;
   // 1. dA = dO V^T, dA^T = V dO^T, Zq = X_q W_q, Zk = X_k W_k
@@ -323,6 +353,24 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
   //    a bf16 pair hi + lo
   e_half_to_tmem(p.e32, ((size_t)bh * p.L + (valid ? tq : 0)) * D, valid, wg, tl + C_E + 64 * wg);
   tmem_st_wait();
+  r1[0] = r1[1] = r1[2] = 0.f;
+  {
+    const float *ms = p.sp_r0 + (size_t)snap_idx * D + 64 * wg, *md = p.ds_r0 + (size_t)snap_idx * D + 64 * wg;
+#pragma unroll 2
+    for (int ch = 0; ch < 8; ++ch) {
+      float o8[8], v8[8];
+      unpack8(*chunk_ptr(sm, R_O, row, 8 * wg + ch), o8);
+      unpack8(*chunk_ptr(sm, R_V, row, 8 * wg + ch), v8);
+      const float4 a0 = __ldg(reinterpret_cast<const float4 *>(ms + 8 * ch)),
+                   a1 = __ldg(reinterpret_cast<const float4 *>(ms + 8 * ch + 4));
+      const float4 b0 = __ldg(reinterpret_cast<const float4 *>(md + 8 * ch)),
+                   b1 = __ldg(reinterpret_cast<const float4 *>(md + 8 * ch + 4));
+      r1[0] += o8[0] * a0.x + o8[1] * a0.y + o8[2] * a0.z + o8[3] * a0.w + o8[4] * a1.x + o8[5] * a1.y +
+               o8[6] * a1.z + o8[7] * a1.w;
+      r1[1] += v8[0] * b0.x + v8[1] * b0.y + v8[2] * b0.z + v8[3] * b0.w + v8[4] * b1.x + v8[5] * b1.y +
+               v8[6] * b1.z + v8[7] * b1.w;
+    }
+  }
 #pragma unroll
   for (int m = 0; m < 2; ++m) {
     float ph[F];
@@ -335,6 +383,9 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
 #pragma unroll
       for (int u = 0; u < 16; ++u)
         x16[u] = m == 0 ? ph[16 * c16 + u] * s * E[u] : (valid ? __fdividef(ph[16 * c16 + u] * s, E[u]) : 0.f);
+      if (m == 1)
+#pragma unroll
+        for (int u = 0; u < 16; ++u) r1[2] += x16[u];
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         uint4 hi, lo;
@@ -344,9 +395,15 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
       }
     }
   }
+  if (wg == 1)
+#pragma unroll
+    for (int k = 0; k < 3; ++k) s_r1[k][row] = r1[k];
   fence_proxy_async();
   tc_fence_before();
   __syncthreads();
+  if (wg == 0)   // the two halves' sums meet; read after the next barrier
+#pragma unroll
+    for (int k = 0; k < 3; ++k) s_r1[k][row] += r1[k];
   // 3. A^T = Kt Qt^T (rows = keys)
   if (tid == 0) {
     tc_fence_after();
@@ -419,10 +476,17 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
     if (__syncthreads_or(!ok)) goto done;
     tc_fence_after();
     unsigned char *st0 = sm + R_V, *st1 = sm + R_QL, *st2 = sm + R_XQ;
+    // rank-one parts of GQ and GK left out of the S' and dS copies
+    const float cq = s_r1[0][row], ck = s_r1[1][row], kap = s_r1[2][row];
     for (int c16 = 4 * wg; c16 < 4 * wg + 4; ++c16) {
       float gq[16], gk[16], q16[16], k16[16], lo[16];
       tmem_ld16(tl + C_GQ + c16 * 16, gq);
       tmem_ld16(tl + C_GK + c16 * 16, gk);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        gq[u] += cq;
+        gk[u] += ck;
+      }
       unpack8(*chunk_ptr(sm, R_XQ, row, 2 * c16), q16);
       unpack8(*chunk_ptr(sm, R_XQ, row, 2 * c16 + 1), q16 + 8);
       unpack8(*chunk_ptr(sm, R_QL, row, 2 * c16), lo);
@@ -454,6 +518,11 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
       tmem_ld16(tl + C_GQ + c16 * 16, gq);
       tmem_ld16(tl + C_GK + c16 * 16, gk);
 #pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        gq[u] += cq;
+        gk[u] += ck;
+      }
+#pragma unroll
       for (int u = 0; u < 4; ++u) {
         const float4 E = e4[4 * k4 + u];
         *f32_stage_ptr(st1, row, c16 * 16 + 4 * u) =
@@ -474,12 +543,16 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
       bulk_wait_read_but_last();   // the dB tile has been read out of V | dO
     }
     __syncthreads();
+    const float *md = p.ds_r0 + (size_t)snap_idx * D;
     for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
       float dv[32];
       tmem_ld32(tl + C_DV + ch * 32, dv);
 #pragma unroll
-      for (int u = 0; u < 32; u += 4)
-        *f32_stage_ptr(st0, row, ch * 32 + u) = make_float4(dv[u], dv[u + 1], dv[u + 2], dv[u + 3]);
+      for (int u = 0; u < 32; u += 4) {   // + (sum_i Kt[i]) dS[0]
+        const float4 m4 = __ldg(reinterpret_cast<const float4 *>(md + ch * 32 + u));
+        *f32_stage_ptr(st0, row, ch * 32 + u) = make_float4(fmaf(kap, m4.x, dv[u]), fmaf(kap, m4.y, dv[u + 1]),
+                                                            fmaf(kap, m4.z, dv[u + 2]), fmaf(kap, m4.w, dv[u + 3]));
+      }
     }
     fence_proxy_async();
     __syncthreads();
@@ -603,8 +676,15 @@ constexpr size_t TILE_SMEM = 7 * TILE + 1024;
 
 }  // namespace
 
+// One copy region: [BH][ntiles][D][D] bf16 (each tile's matrix minus its
+// row 0), then [BH][ntiles][D] fp32 (row 0).
 size_t tc_gla_bwd_snapshot_bytes(int BH, int L) {
-  return (size_t)BH * ((L + T - 1) / T) * D * D * sizeof(__nv_bfloat16);
+  const size_t n = (size_t)BH * ((L + T - 1) / T);
+  return n * D * D * sizeof(__nv_bfloat16) + n * D * sizeof(float);
+}
+static const float *snapshot_row0(const void *snap, int BH, int L) {
+  return reinterpret_cast<const float *>(static_cast<const __nv_bfloat16 *>(snap) +
+                                         (size_t)BH * ((L + T - 1) / T) * D * D);
 }
 
 cudaError_t launch_tc_gla_bwd(const TcGlaBwdArgs &a, int stage, cudaStream_t s) {
@@ -619,6 +699,7 @@ cudaError_t launch_tc_gla_bwd(const TcGlaBwdArgs &a, int stage, cudaStream_t s) 
     p.e32 = a.e32;
     p.gate_r = a.gate_r;
     p.snap = static_cast<__nv_bfloat16 *>(a.snap_ds);
+    p.snap_r0 = const_cast<float *>(snapshot_row0(a.snap_ds, a.BH, a.L));
     p.dstate_in = a.dstate_in;
     p.status = a.status;
     p.H = a.H;
@@ -642,6 +723,8 @@ cudaError_t launch_tc_gla_bwd(const TcGlaBwdArgs &a, int stage, cudaStream_t s) 
     p.wq = a.wq;
     p.wk = a.wk;
     p.e32 = a.e32;
+    p.sp_r0 = snapshot_row0(a.snap_s, a.BH, a.L);
+    p.ds_r0 = snapshot_row0(a.snap_ds, a.BH, a.L);
     p.dphq = a.dphq;
     p.dphk = a.dphk;
     p.dB = a.dB;

@@ -130,3 +130,20 @@ def test_scalar_gate_decode_step(lz, dtype, d, window, M, pos0):
     check("state", x["state"], want_S, "fp32")
     assert torch.equal(x["k_cache"].cpu(), torch.from_numpy(want_kc).to(x["k_cache"].dtype))
     assert np.array_equal(x["pos"].cpu().numpy(), want_pos)
+
+
+@pytest.mark.parametrize("gate", ["dim", "scalar"])
+def test_feature_map_weight_gradients_keep_their_cancellation(lz, gate):
+    """At the workloads' small feature-map weights the weight gradients are a
+    small remainder of large per-feature terms; the tensor-core backward keeps
+    them well inside the bf16 bar (hi + lo operands, row-0-centred state
+    copies).  A regression guard at a quarter of the bar."""
+    w = Workload("wprec", B=2, H=2, L=512, d=128, dtype="bf16", seed=13, kind="train", gate=gate)
+    inp = make_inputs(w)
+    x = to_device(inp)
+    got = lz.attn_bwd(x["q"], x["k"], x["v"], x["g"], x["dout"], impl=lz.IMPL_TC, **_kw(x, w))
+    want = oracle_backward(inp, window=w.window, tau=w.gate_temp)
+    for name in ("dfmap_wq", "dfmap_wk", "dg", "dstate_in"):
+        g_, r_ = to64(got[name]), want[name]
+        rel = float(np.max(np.abs(g_ - r_)) / np.max(np.abs(r_)))
+        assert rel <= 5e-3, f"{name}: {rel:.2e}"
