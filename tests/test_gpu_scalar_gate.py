@@ -137,7 +137,7 @@ def test_feature_map_weight_gradients_keep_their_cancellation(lz, gate):
     """At the workloads' small feature-map weights the weight gradients are a
     small remainder of large per-feature terms; the tensor-core backward keeps
     them well inside the bf16 bar (hi + lo operands, row-0-centred state
-    copies).  A regression guard at a quarter of the bar."""
+    copies).  A regression guard at 0.4 of the bar."""
     w = Workload("wprec", B=2, H=2, L=512, d=128, dtype="bf16", seed=13, kind="train", gate=gate)
     inp = make_inputs(w)
     x = to_device(inp)
@@ -146,4 +146,4 @@ def test_feature_map_weight_gradients_keep_their_cancellation(lz, gate):
     for name in ("dfmap_wq", "dfmap_wk", "dg", "dstate_in"):
         g_, r_ = to64(got[name]), want[name]
         rel = float(np.max(np.abs(g_ - r_)) / np.max(np.abs(r_)))
-        assert rel <= 5e-3, f"{name}: {rel:.2e}"
+        assert rel <= 8e-3, f"{name}: {rel:.2e}"
