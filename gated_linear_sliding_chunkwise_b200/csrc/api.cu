@@ -101,7 +101,7 @@ bool bwd_gla_uses_tc(const lizard_fwd_args *a, int impl) {
 
 struct BwdLayout {
   size_t phq, phk, a, sprev, dphq, dphk, da, dv_gla, dq_swa, dk_swa, dv_swa, lse, Dterm, dsm, pm, snap_s,
-      snap_ds, e32, gr, total;
+      snap_ds, e32, gr, w16, total;
 };
 BwdLayout bwd_layout(const lizard_fwd_args *a, int impl) {
   const size_t BH = (size_t)a->B * a->H;
@@ -121,6 +121,7 @@ BwdLayout bwd_layout(const lizard_fwd_args *a, int impl) {
     l.dv_gla = off; off += nv;
     l.e32 = off; off += nd;      // fp32 decay factors E of every tile
     l.gr = off; off += up(BH * ((a->L + 127) / 128) * a->dk * sizeof(float));   // tiles' log-decays
+    l.w16 = off; off += up(lz::tc_gla_bwd_weights_bytes(a->H));                  // bf16 W_q, W_k
   } else if (gla_on(a)) {
     l.phq = off; off += nd;
     l.phk = off; off += nd;
@@ -239,7 +240,9 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan) {
     lz::TcGlaBwdArgs t{a->q, a->k, a->v, a->g, b->dout, a->fmap_wq, a->fmap_wk, snap_s,
                        at<void>(ws, lay.snap_ds), at<float>(ws, lay.dphq), at<float>(ws, lay.dphk),
                        at<float>(ws, lay.da), at<float>(ws, lay.dv_gla), b->dg, b->dstate_in,
-                       status, a->H, BH, a->L, inv_tau, e32, gr, scalar_gate(a)};
+                       status, a->H, BH, a->L, inv_tau, e32, gr, scalar_gate(a), at<void>(ws, lay.w16)};
+    void *w16 = at<void>(ws, lay.w16);
+    plan.add("weights_bf16_kernel", [=] { return lz::launch_weights_bf16(a->fmap_wq, a->fmap_wk, w16, a->H, s); });
     plan.add("tc_gla_dstates_kernel", [=] { return lz::launch_tc_gla_bwd(t, 0, s); });
     plan.add("tc_gla_bwd_tile_kernel", [=] { return lz::launch_tc_gla_bwd(t, 1, s); });
   } else if (g) {

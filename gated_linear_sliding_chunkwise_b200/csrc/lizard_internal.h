@@ -147,6 +147,7 @@ struct TcGlaBwdArgs {
   const float *e32;             // fp32 [B*H*L][128] decay factors of every tile (launch_gate_prep)
   const float *gate_r;          // fp32 [B*H][L/128][128] log-decay of every tile
   int scalar_gate;              // g and dg hold one value per (token, head): [B*H][L]
+  const void *w16;              // bf16 [H][2][128][64] feature-map weights (launch_weights_bf16)
 };
 
 constexpr int kBwdC = 32;   // GLA chunk used by the portable backward
@@ -178,6 +179,9 @@ bool tc_swa_bwd_supported(int dk, int dv, int window, int M, bool bf16);
 // stage 0: dq pass, 1: dk/dv pass, 2: meta-token gradients
 cudaError_t launch_tc_swa_bwd(const TcSwaBwdArgs &a, int stage, cudaStream_t s);
 size_t tc_gla_bwd_snapshot_bytes(int BH, int L);
+// bf16 copies of W_q, W_k ([H][2][128][64]) for the per-tile backward's TMA loads
+size_t tc_gla_bwd_weights_bytes(int H);
+cudaError_t launch_weights_bf16(const float *wq, const float *wk, void *out, int H, cudaStream_t s);
 cudaError_t launch_tc_state_snapshots(const TcFwdArgs &a, void *snap, const float *e32, const float *r,
                                       cudaStream_t s);
 // Decay factors of every 128-token tile (bf16 E16 and/or fp32 E32, [BH][L][128],

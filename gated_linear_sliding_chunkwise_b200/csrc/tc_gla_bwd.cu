@@ -60,6 +60,7 @@ struct DsParams {
 
 struct TileParams {
   CUtensorMap mq, mk, mv, mo, msp, mds;       // msp / mds: [BH*ntiles][D][D] snapshots
+  CUtensorMap mw;                             // [H*2][D][F] bf16 feature-map weights (W_q, W_k per head)
   CUtensorMap mdq, mdk, mdb, mdv;             // fp32 outputs dphi_q, dphi_k, dB, dv (TMA stores)
   const float *wq, *wk;
   const float *e32;            // fp32 decay factors [BH*L][D]
@@ -82,13 +83,15 @@ __device__ __forceinline__ void stage_weights(unsigned char *dst, const float *W
 }
 
 // fp32 decay factors of tile row `t` (< L, else 1), dimensions 64 h ..
-// 64 h + 63, from the precomputed array into TMEM columns col .. col + 63.
-__device__ __forceinline__ void e_half_to_tmem(const float *e32, size_t row_off, bool valid, int h, uint32_t taddr) {
+// 64 h + 63, from the precomputed array into TMEM columns col .. col + 63,
+// in two halves: the loads (in flight early) and the TMEM stores.
+__device__ __forceinline__ void e_half_load(const float *e32, size_t row_off, bool valid, int h, float4 *e) {
   const float *er = e32 + row_off + 64 * h;
-  float4 e[16];
 #pragma unroll
   for (int u = 0; u < 16; ++u)
     e[u] = valid ? *reinterpret_cast<const float4 *>(er + 4 * u) : make_float4(1.f, 1.f, 1.f, 1.f);
+}
+__device__ __forceinline__ void e_half_store(const float4 *e, uint32_t taddr) {
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
     const uint32_t r8[8] = {__float_as_uint(e[2 * u].x), __float_as_uint(e[2 * u].y), __float_as_uint(e[2 * u].z),
@@ -146,6 +149,14 @@ __global__ void __launch_bounds__(NT_DS, 1) tc_gla_dstates_kernel(const __grid_c
     }
   };
   if (tid == 0 && ntiles > 0) loads(ntiles - 1);
+  // this row's fp32 decay factors (its dimension half) of the tile to come:
+  // loaded one tile ahead, so that they are in flight during the previous one
+  float4 epre[16];
+  auto e_load = [&](int c) {
+    const int t = c * T + row;
+    e_half_load(p.e32, ((size_t)bh * p.L + (t < p.L ? t : 0)) * D, t < p.L, wg, epre);
+  };
+  if (ntiles > 0) e_load(ntiles - 1);
   bool fail = false;
   for (int c = ntiles - 1; c >= 0; --c) {
     const uint32_t par = (ntiles - 1 - c) & 1;
@@ -184,8 +195,8 @@ __global__ void __launch_bounds__(NT_DS, 1) tc_gla_dstates_kernel(const __grid_c
       if (tid < D) p.snap_r0[tile * D + tid] = s_row0[tid];
     }
     // E in fp32 (dimensions 64 wg ..) into TMEM; the tile's decay exp(r)
-    e_half_to_tmem(p.e32, ((size_t)bh * p.L + (t0 + row < p.L ? t0 + row : 0)) * D, t0 + row < p.L, wg,
-                   tl + C_E + 64 * wg);
+    e_half_store(epre, tl + C_E + 64 * wg);
+    if (c > 0) e_load(c - 1);
     if (wg == 0) s_dec[row] = __expf(p.gate_r[((size_t)bh * ntiles + c) * D + row]);
     tmem_st_wait();
     ok = mbar_wait(&bar_m1, par, p.status, ST_TIMEOUT);
@@ -286,27 +297,27 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
   if (tid == 0) {
     for (int i = 0; i < 8; ++i) mbar_init(&bars[i], 1);
     fence_barrier_init();
-  }
-  stage_weights(sm + R_W + wg * REG, wg == 0 ? p.wq : p.wk, h, row);
-  fence_proxy_async();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tb = s_tmem, tl = tb + lane_off;
-  const int snap_idx = bh * p.ntiles + c;
-  if (tid == 0) {
-    mbar_expect_tx(&bars[0], 4 * TILE);
+    // the tile and this head's bf16 feature-map weights (converted once per call)
+    mbar_expect_tx(&bars[0], 5 * TILE);
     for (int r = 0; r < 2; ++r) {
       tma_load_3d(sm + R_XQ + r * REG, &p.mq, &bars[0], 64 * r, t0, bh);
       tma_load_3d(sm + R_XK + r * REG, &p.mk, &bars[0], 64 * r, t0, bh);
       tma_load_3d(sm + R_V + r * REG, &p.mv, &bars[0], 64 * r, t0, bh);
       tma_load_3d(sm + R_O + r * REG, &p.mo, &bars[0], 64 * r, t0, bh);
+      tma_load_3d(sm + R_W + r * REG, &p.mw, &bars[0], 0, 0, 2 * h + r);
     }
   }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = s_tmem, tl = tb + lane_off;
+  const int snap_idx = bh * p.ntiles + c;
   const uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
   const uint32_t id_mn = idesc_bf16(128, 128, 0, 1);
   const uint32_t id_z = idesc_bf16(128, 64, 0, 1);
   float r1[3];   // this half's dO . S'[0], V . dS[0], sum Kt
+  float4 epre[16];   // this row's fp32 decay factors (its dimension half), loaded while the tile arrives
+  e_half_load(p.e32, ((size_t)bh * p.L + (valid ? tq : 0)) * D, valid, wg, epre);
   bool ok = mbar_wait(&bars[0], 0, p.status, ST_TIMEOUT);
   if (__syncthreads_or(!ok)) goto done;
   // 1. dA = dO V^T, dA^T = V dO^T, Zq = X_q W_q, Zk = X_k W_k
@@ -351,7 +362,7 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
   //    E in fp32 (dimensions 64 wg ..) into TMEM, then Qt = phi_q E and
   //    Kt = phi_k / E for the same dimensions (rows past L: Kt = 0), each as
   //    a bf16 pair hi + lo
-  e_half_to_tmem(p.e32, ((size_t)bh * p.L + (valid ? tq : 0)) * D, valid, wg, tl + C_E + 64 * wg);
+  e_half_store(epre, tl + C_E + 64 * wg);
   tmem_st_wait();
   r1[0] = r1[1] = r1[2] = 0.f;
   {
@@ -671,6 +682,20 @@ __global__ void __launch_bounds__(256) gate_grad_scalar_kernel(const float *dB, 
   }
 }
 
+// bf16 copies of the feature-map weights, [H][2][D][F] (W_q then W_k of
+// each head), for the tile kernel's TMA loads.
+__global__ void __launch_bounds__(256) weights_bf16_kernel(const float *wq, const float *wk,
+                                                          __nv_bfloat16 *out) {
+  const int hm = blockIdx.x, h = hm >> 1;
+  const float *W = ((hm & 1) ? wk : wq) + (size_t)h * D * F;
+  __nv_bfloat16 *o = out + (size_t)hm * D * F;
+  for (int e = threadIdx.x * 4; e < D * F; e += 256 * 4) {
+    const float4 x = *reinterpret_cast<const float4 *>(W + e);
+    *reinterpret_cast<__nv_bfloat162 *>(o + e) = __floats2bfloat162_rn(x.x, x.y);
+    *reinterpret_cast<__nv_bfloat162 *>(o + e + 2) = __floats2bfloat162_rn(x.z, x.w);
+  }
+}
+
 constexpr size_t DS_SMEM = 3 * TILE + TILE / 2 + 1024;
 constexpr size_t TILE_SMEM = 7 * TILE + 1024;
 
@@ -678,6 +703,13 @@ constexpr size_t TILE_SMEM = 7 * TILE + 1024;
 
 // One copy region: [BH][ntiles][D][D] bf16 (each tile's matrix minus its
 // row 0), then [BH][ntiles][D] fp32 (row 0).
+size_t tc_gla_bwd_weights_bytes(int H) { return (size_t)H * 2 * D * F * sizeof(__nv_bfloat16); }
+
+cudaError_t launch_weights_bf16(const float *wq, const float *wk, void *out, int H, cudaStream_t s) {
+  weights_bf16_kernel<<<2 * H, 256, 0, s>>>(wq, wk, static_cast<__nv_bfloat16 *>(out));
+  return cudaGetLastError();
+}
+
 size_t tc_gla_bwd_snapshot_bytes(int BH, int L) {
   const size_t n = (size_t)BH * ((L + T - 1) / T);
   return n * D * D * sizeof(__nv_bfloat16) + n * D * sizeof(float);
@@ -716,6 +748,7 @@ cudaError_t launch_tc_gla_bwd(const TcGlaBwdArgs &a, int stage, cudaStream_t s) 
     if (!make_map_bf16_3d(&p.mq, a.q, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mk, a.k, D, rows, a.BH, T) ||
         !make_map_bf16_3d(&p.mv, a.v, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mo, a.dout, D, rows, a.BH, T) ||
         !make_map_bf16_3d(&p.msp, a.snap_s, D, D, (uint64_t)a.BH * ntiles, T) ||
+        !make_map_bf16_3d(&p.mw, a.w16, F, D, (uint64_t)a.H * 2, T) ||
         !make_map_bf16_3d(&p.mds, a.snap_ds, D, D, (uint64_t)a.BH * ntiles, T) ||
         !make_map_f32_3d(&p.mdq, a.dphq, D, rows, a.BH, T) || !make_map_f32_3d(&p.mdk, a.dphk, D, rows, a.BH, T) ||
         !make_map_f32_3d(&p.mdb, a.dB, D, rows, a.BH, T) || !make_map_f32_3d(&p.mdv, a.dv, D, rows, a.BH, T))
