@@ -177,10 +177,13 @@ __device__ __forceinline__ void kt_half(unsigned char *sm, uint32_t tl, int row,
 constexpr int BAR_A = 1;       // both groups' row maxima written
 constexpr int BAR_B = 2;       // both groups' row sums written, all logits read
 
-// LOSS: the full pass also forms the stage-1 loss (p.target set).  A separate
-// instance, so that the plain forward keeps its register budget.
-template <bool LOSS>
+// Kernel instances: the full pass, the full pass that also forms the
+// stage-1 loss (p.target set), and the state pass.  Each keeps its own
+// register budget.
+constexpr int K_FULL = 0, K_LOSS = 1, K_STATE = 2;
+template <int KIND>
 __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_constant__ Params p) {
+  constexpr bool LOSS = KIND == K_LOSS;
   extern __shared__ unsigned char smraw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
   __shared__ __align__(16) float s_mk[MAXM][D];
@@ -201,7 +204,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
   const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
   const int bh = blockIdx.x, h = bh % p.H, seg = blockIdx.y;
   const float alpha = p.alpha ? p.alpha[h] : 1.f;
-  const bool full = p.mode == 0;
+  constexpr bool full = KIND != K_STATE;
   const bool gla = p.branch != 2, swa = full && p.branch != 1;
   const uint32_t sbase = smem_u32(sm);
 
@@ -272,6 +275,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
   const uint32_t id_st = idesc_bf16(128, 128, 1, 1);
 
   float mse_acc = 0.f;                        // this thread's share of sum (o - target)^2
+  // state pass: this row's fp32 decay factors (its dimension half) of the
+  // next tile, loaded one tile ahead
+  float4 epre[16];
+  auto e_load = [&](int c) {
+    const int t = c * T + row;
+    const float *er = p.gate_e32 + ((size_t)bh * p.L + (t < p.L ? t : 0)) * D + 64 * wg;
+#pragma unroll
+    for (int u = 0; u < 16; ++u)
+      epre[u] = t < p.L ? *reinterpret_cast<const float4 *>(er + 4 * u) : make_float4(1.f, 1.f, 1.f, 1.f);
+  };
+  if (!full && cbeg < cend) e_load(cbeg);
   for (int c = cbeg; c < cend; ++c) {
     const uint32_t par = (c - cbeg) & 1;
     const int t0 = c * T;
@@ -433,11 +447,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       // ------ state pass: fp32 decay factors of this row's dimension half
       //        (from gate_prep_kernel) into TMEM, phi_k half per group ---
       {
-        const float *er = p.gate_e32 + ((size_t)bh * p.L + (qvalid ? tq : 0)) * D + 64 * wg;
-        float4 e[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u)
-          e[u] = qvalid ? *reinterpret_cast<const float4 *>(er + 4 * u) : make_float4(1.f, 1.f, 1.f, 1.f);
+        const float4 *e = epre;
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const uint32_t r8[8] = {__float_as_uint(e[2 * u].x), __float_as_uint(e[2 * u].y), __float_as_uint(e[2 * u].z),
@@ -445,6 +455,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
                                   __float_as_uint(e[2 * u + 1].z), __float_as_uint(e[2 * u + 1].w)};
           tmem_st8(tl + C_L + 64 * wg + 8 * u, r8);
         }
+        if (c + 1 < cend) e_load(c + 1);
         if (wg == 0) {   // thread row = key dimension: the tile's decay
           const float r = p.gate_r[((size_t)bh * ntiles_all + c) * D + row];
           s_dec[row] = __expf(r);
@@ -877,9 +888,9 @@ cudaError_t launch_tc_state_snapshots(const TcFwdArgs &a, void *snap, const floa
   p.seg_state = nullptr;
   p.seg_decay = nullptr;
   cudaError_t e =
-      cudaFuncSetAttribute(tc_fwd_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+      cudaFuncSetAttribute(tc_fwd_kernel<K_STATE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  tc_fwd_kernel<false><<<dim3(a.BH, 1), NTHREADS, SMEM_BYTES, s>>>(p);
+  tc_fwd_kernel<K_STATE><<<dim3(a.BH, 1), NTHREADS, SMEM_BYTES, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -942,21 +953,23 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, int stage, cudaStream_t s) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64 || configured[dev] < SMEM_BYTES) {
-    e = cudaFuncSetAttribute(tc_fwd_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    e = cudaFuncSetAttribute(tc_fwd_kernel<K_FULL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(tc_fwd_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    e = cudaFuncSetAttribute(tc_fwd_kernel<K_LOSS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(tc_fwd_kernel<K_STATE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) configured[dev] = SMEM_BYTES;
   }
   if (nseg > 1 && stage == 0) {          // state pass over every segment but the last
     p.mode = 1;
-    tc_fwd_kernel<false><<<dim3(a.BH, nseg - 1), NTHREADS, SMEM_BYTES, s>>>(p);
+    tc_fwd_kernel<K_STATE><<<dim3(a.BH, nseg - 1), NTHREADS, SMEM_BYTES, s>>>(p);
   } else {                               // full pass
     p.mode = 0;
     if (p.target)
-      tc_fwd_kernel<true><<<dim3(a.BH, nseg), NTHREADS, SMEM_BYTES, s>>>(p);
+      tc_fwd_kernel<K_LOSS><<<dim3(a.BH, nseg), NTHREADS, SMEM_BYTES, s>>>(p);
     else
-      tc_fwd_kernel<false><<<dim3(a.BH, nseg), NTHREADS, SMEM_BYTES, s>>>(p);
+      tc_fwd_kernel<K_FULL><<<dim3(a.BH, nseg), NTHREADS, SMEM_BYTES, s>>>(p);
   }
   return cudaGetLastError();
 }
