@@ -66,6 +66,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
     mbar_init(&bar_d, 1);
     fence_barrier_init();
   }
+  const int ntiles = (p.L + T - 1) / T;
+  auto loads = [&](int c) {
+    mbar_expect_tx(&bar_tma, 2 * TILE);
+    for (int r = 0; r < 2; ++r) {
+      tma_load_3d(sm + R_XQ + r * REG, &p.mq, &bar_tma, 64 * r, c * T, bh);
+      tma_load_3d(sm + R_XK + r * REG, &p.mk, &bar_tma, 64 * r, c * T, bh);
+    }
+  };
+  if (tid == 0 && ntiles > 0 && gla) loads(0);   // in flight while the weights are staged
   // weights -> bf16 [dk row][feature] (MN-major for z = x W, K-major for dz W^T);
   // group 0 W_q, group 1 W_k
   {
@@ -83,18 +92,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = s_tmem, tl = tb + lane_off;
-  const int ntiles = (p.L + T - 1) / T;
   const uint32_t id_z = idesc_bf16(128, 64, 0, 1);     // X (K-major) x W (MN-major, N = 64)
   const uint32_t id_dx = idesc_bf16(128, 128, 0, 0);   // dZ (K-major) x W^T (K-major, N = 128)
   const uint32_t id_dw = idesc_bf16(128, 64, 1, 1);    // X^T (MN-major) x dZ (MN-major, N = 64)
-  auto loads = [&](int c) {
-    mbar_expect_tx(&bar_tma, 2 * TILE);
-    for (int r = 0; r < 2; ++r) {
-      tma_load_3d(sm + R_XQ + r * REG, &p.mq, &bar_tma, 64 * r, c * T, bh);
-      tma_load_3d(sm + R_XK + r * REG, &p.mk, &bar_tma, 64 * r, c * T, bh);
-    }
-  };
-  if (tid == 0 && ntiles > 0 && gla) loads(0);
   bool fail = false;
   for (int c = 0; c < ntiles; ++c) {
     const uint32_t par = c & 1;

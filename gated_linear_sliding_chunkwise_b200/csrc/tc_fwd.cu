@@ -207,6 +207,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
   constexpr bool full = KIND != K_STATE;
   const bool gla = p.branch != 2, swa = full && p.branch != 1;
   const uint32_t sbase = smem_u32(sm);
+  const int ntiles_all = (p.L + T - 1) / T;
+  const int cbeg = seg * p.tiles_per_seg;
+  const int cend = min(ntiles_all, cbeg + p.tiles_per_seg);
 
   if (warp == 0) {
     tmem_alloc(&s_tmem, 512);
@@ -221,6 +224,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
     fence_barrier_init();
     s_fail = 0;
   }
+  // the first tile's loads go out before the weights and meta tokens are staged
+  if (tid == 0 && cbeg < cend) issue_tile_loads(p, sm, &bar_tma, bh, cbeg * T, full);
   // feature-map weights -> bf16, MN-major [dk row][feature]; group 0 W_q, group 1 W_k
   {
     const int i = row;
@@ -263,12 +268,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
     tmem_st_wait();
   }
 
-  const int ntiles_all = (p.L + T - 1) / T;
-  const int cbeg = seg * p.tiles_per_seg;
-  const int cend = min(ntiles_all, cbeg + p.tiles_per_seg);
   uint32_t *err = p.status;
   float tot_decay = 0.f;                      // state pass: summed log-decay of dimension `row` (group 0)
-  if (tid == 0 && cbeg < cend) issue_tile_loads(p, sm, &bar_tma, bh, cbeg * T, full);
   const uint32_t id_128 = idesc_bf16(128, 128, 0, 0);
   const uint32_t id_z = idesc_bf16(128, 64, 0, 1);
   const uint32_t id_mn = idesc_bf16(128, 128, 0, 1);

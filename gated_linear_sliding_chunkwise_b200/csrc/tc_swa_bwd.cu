@@ -99,15 +99,7 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
   const uint32_t sbase = smem_u32(sm);
   uint64_t *bar_tma = &bars[0], *bar_m = &bars[1];
   setup_cta(&s_tmem, bars, 6, tid);
-  for (int e = tid; e < MAXM * D; e += NT_Q) {
-    const int m = e / D;
-    s_mk[m][e % D] = m < p.M ? p.meta_k[(size_t)h * p.M * D + e] : 0.f;
-    s_mv[m][e % D] = (m < p.M && p.meta_v) ? p.meta_v[(size_t)h * p.M * D + e] : 0.f;
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tb = s_tmem, tl = tb + lane_off;
+  // the tiles first, so that they arrive while the meta tokens are staged
   if (tid == 0) {
     mbar_expect_tx(bar_tma, 6 * TILE);
     for (int r = 0; r < 2; ++r) {
@@ -119,6 +111,15 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
       tma_load_3d(sm + R_V + r * kReg, &p.mv, bar_tma, 64 * r, t0, bh);
     }
   }
+  for (int e = tid; e < MAXM * D; e += NT_Q) {
+    const int m = e / D;
+    s_mk[m][e % D] = m < p.M ? p.meta_k[(size_t)h * p.M * D + e] : 0.f;
+    s_mv[m][e % D] = (m < p.M && p.meta_v) ? p.meta_v[(size_t)h * p.M * D + e] : 0.f;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = s_tmem, tl = tb + lane_off;
   const uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
   const uint32_t id_mn = idesc_bf16(128, 128, 0, 1);
   bool ok = mbar_wait(bar_tma, 0, p.status, ST_TIMEOUT);
@@ -472,15 +473,7 @@ __global__ void __launch_bounds__(NT_KV, 1) tc_swa_bwd_kv_kernel(const __grid_co
   const float alpha = p.alpha ? p.alpha[h] : 1.f;
   const uint32_t sbase = smem_u32(sm);
   setup_cta(&s_tmem, bars, 7, tid);
-  for (int e = tid; e < 2 * T; e += NT_KV) {
-    const int t = j0 + e;
-    s_lse[e] = t < p.L ? p.lse[(size_t)bh * p.L + t] : 0.f;
-    s_D[e] = t < p.L ? p.Dterm[(size_t)bh * p.L + t] : 0.f;
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tb = s_tmem, tl = tb + lane_off;
+  // the tiles first, so that they arrive while the softmax statistics are staged
   if (tid == 0) {
     mbar_expect_tx(&bars[0], 6 * TILE);
     for (int r = 0; r < 2; ++r) {
@@ -492,6 +485,15 @@ __global__ void __launch_bounds__(NT_KV, 1) tc_swa_bwd_kv_kernel(const __grid_co
       }
     }
   }
+  for (int e = tid; e < 2 * T; e += NT_KV) {
+    const int t = j0 + e;
+    s_lse[e] = t < p.L ? p.lse[(size_t)bh * p.L + t] : 0.f;
+    s_D[e] = t < p.L ? p.Dterm[(size_t)bh * p.L + t] : 0.f;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = s_tmem, tl = tb + lane_off;
   const uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
   const uint32_t id_mn = idesc_bf16(128, 128, 0, 1);
   const int r0 = 32 * (warp & 3);          // first key row of this warp
