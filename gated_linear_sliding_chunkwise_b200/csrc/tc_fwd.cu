@@ -239,7 +239,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       *reinterpret_cast<uint4 *>(sm + reg + sw128_offset(i, c * 8)) = pack8(f);
     }
   }
-  for (int e = tid; e < MAXM * D; e += NTHREADS) {
+  // meta tokens (groups of four are read, so rows up to the next multiple of
+  // four are zero-filled)
+  const int m_rows = (p.M + 3) / 4 * 4;
+  for (int e = tid; e < m_rows * D; e += NTHREADS) {
     const int m = e / D;
     s_mk[m][e % D] = m < p.M ? p.meta_k[(size_t)h * p.M * D + e] : 0.f;
     s_mv[m][e % D] = (m < p.M && p.meta_v) ? p.meta_v[(size_t)h * p.M * D + e] : 0.f;

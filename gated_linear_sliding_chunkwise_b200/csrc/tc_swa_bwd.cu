@@ -43,6 +43,7 @@ struct QParams {
   int H, L, M, window;
   float scale;
   int fused;
+  int BH;
 };
 
 struct KVParams {
@@ -93,36 +94,61 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wg = tid >> 7, row = tid & 127;
   const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-  const int bh = blockIdx.y, h = bh % p.H, t0 = blockIdx.x * T, tq = t0 + row;
-  const bool qvalid = tq < p.L;
-  const float alpha = p.alpha ? p.alpha[h] : 1.f;
   const uint32_t sbase = smem_u32(sm);
   uint64_t *bar_tma = &bars[0], *bar_m = &bars[1];
   setup_cta(&s_tmem, bars, 6, tid);
-  // the tiles first, so that they arrive while the meta tokens are staged
-  if (tid == 0) {
-    mbar_expect_tx(bar_tma, 6 * TILE);
+  // Persistent: CTA b walks the contiguous run [w0, w1) of (sequence, tile)
+  // items, the tiles of a sequence in order; the meta tokens are staged again
+  // only when the head changes, and the next item's tiles are loaded as soon
+  // as this item's shared memory is free.
+  const int ntiles = (p.L + T - 1) / T, nwork = ntiles * p.BH;
+  const int w0 = (int)((long long)blockIdx.x * nwork / gridDim.x);
+  const int w1 = (int)((long long)(blockIdx.x + 1) * nwork / gridDim.x);
+  // Tile loads of item w, in two parts: `early` = the regions free once the
+  // dq' product has run (all but V when the GLA part arrives in V, all but
+  // Q | dO when dq is staged there), `late` = the rest, after the store.
+  auto tile_loads = [&](int w, bool early, bool late) {
+    const int lbh = w / ntiles, lt0 = (w % ntiles) * T;
+    if (early) mbar_expect_tx(bar_tma, 6 * TILE);
+    const bool qo_early = p.fused != 0, v_early = p.fused == 0;
     for (int r = 0; r < 2; ++r) {
-      tma_load_3d(sm + R_Q + r * kReg, &p.mq, bar_tma, 64 * r, t0, bh);
-      tma_load_3d(sm + R_O + r * kReg, &p.mo, bar_tma, 64 * r, t0, bh);
-      tma_load_3d(sm + R_KP + r * kReg, &p.mk, bar_tma, 64 * r, t0 - T, bh);
-      tma_load_3d(sm + R_K + r * kReg, &p.mk, bar_tma, 64 * r, t0, bh);
-      tma_load_3d(sm + R_VP + r * kReg, &p.mv, bar_tma, 64 * r, t0 - T, bh);
-      tma_load_3d(sm + R_V + r * kReg, &p.mv, bar_tma, 64 * r, t0, bh);
+      if (qo_early ? early : late) {
+        tma_load_3d(sm + R_Q + r * kReg, &p.mq, bar_tma, 64 * r, lt0, lbh);
+        tma_load_3d(sm + R_O + r * kReg, &p.mo, bar_tma, 64 * r, lt0, lbh);
+      }
+      if (early) {
+        tma_load_3d(sm + R_KP + r * kReg, &p.mk, bar_tma, 64 * r, lt0 - T, lbh);
+        tma_load_3d(sm + R_K + r * kReg, &p.mk, bar_tma, 64 * r, lt0, lbh);
+        tma_load_3d(sm + R_VP + r * kReg, &p.mv, bar_tma, 64 * r, lt0 - T, lbh);
+      }
+      if (v_early ? early : late) tma_load_3d(sm + R_V + r * kReg, &p.mv, bar_tma, 64 * r, lt0, lbh);
     }
-  }
-  for (int e = tid; e < MAXM * D; e += NT_Q) {
-    const int m = e / D;
-    s_mk[m][e % D] = m < p.M ? p.meta_k[(size_t)h * p.M * D + e] : 0.f;
-    s_mv[m][e % D] = (m < p.M && p.meta_v) ? p.meta_v[(size_t)h * p.M * D + e] : 0.f;
-  }
+  };
+  if (tid == 0 && w0 < w1) tile_loads(w0, true, true);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = s_tmem, tl = tb + lane_off;
   const uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
   const uint32_t id_mn = idesc_bf16(128, 128, 0, 1);
-  bool ok = mbar_wait(bar_tma, 0, p.status, ST_TIMEOUT);
+  const int m_rows = (p.M + 3) / 4 * 4;   // meta rows read (groups of four; zero past M)
+  int cur_h = -1;
+  bool ok = true;
+  for (int w = w0, it = 0; w < w1; ++w, ++it) {
+  const uint32_t par = (uint32_t)it & 1u;
+  const int bh = w / ntiles, h = bh % p.H, t0 = (w % ntiles) * T, tq = t0 + row;
+  const bool qvalid = tq < p.L;
+  const float alpha = p.alpha ? p.alpha[h] : 1.f;
+  if (h != cur_h) {
+    cur_h = h;
+    for (int e = tid; e < m_rows * D; e += NT_Q) {
+      const int m = e / D;
+      s_mk[m][e % D] = m < p.M ? p.meta_k[(size_t)h * p.M * D + e] : 0.f;
+      s_mv[m][e % D] = (m < p.M && p.meta_v) ? p.meta_v[(size_t)h * p.M * D + e] : 0.f;
+    }
+    __syncthreads();
+  }
+  ok = mbar_wait(bar_tma, par, p.status, ST_TIMEOUT);
   if (__syncthreads_or(!ok)) goto done;
 
   // 1. logits L = Q [K_prev ; K]^T
@@ -167,7 +193,7 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
         for (int m = 0; m < MAXM; ++m)
           if (m < p.M) s_x[m][row] = ml[m];
     }
-    ok = mbar_wait(bar_m, 0, p.status, ST_TIMEOUT);
+    ok = mbar_wait(bar_m, par, p.status, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) goto done;
     tc_fence_after();
     float mx = kNegBig;
@@ -271,7 +297,7 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
       for (int s = 0; s < 8; ++s) mma_ts(tb + C_O, tb + C_P + 64 + s * 8, desc_mn(sbase + R_V, s), id_mn, 1);
       mma_commit(&bars[2]);
     }
-    ok = mbar_wait(&bars[2], 0, p.status, ST_TIMEOUT);
+    ok = mbar_wait(&bars[2], par, p.status, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) goto done;
     tc_fence_after();
     float dpart = 0.f;                    // dout . o_swa for this row, column half per group
@@ -313,7 +339,7 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
       for (int s = 0; s < 8; ++s) mma_ss(tb + C_DP + 128, desc_k(sbase + R_O, s), desc_k(sbase + R_V, s), id_kk, s > 0);
       mma_commit(&bars[3]);
     }
-    ok = mbar_wait(&bars[3], 0, p.status, ST_TIMEOUT);
+    ok = mbar_wait(&bars[3], par, p.status, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) goto done;
     tc_fence_after();
     if (p.fused && tid == 0) {   // the GLA part of dq into the free V region
@@ -371,13 +397,16 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
       for (int s = 0; s < 8; ++s) mma_ts(tb + C_DQ, tb + C_DS + 64 + s * 8, desc_mn(sbase + R_K, s), id_mn, 1);
       mma_commit(&bars[4]);
     }
-    ok = mbar_wait(&bars[4], 0, p.status, ST_TIMEOUT);
+    ok = mbar_wait(&bars[4], par, p.status, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) goto done;
     tc_fence_after();
+    // the products are done with K_prev, K, V_prev (and Q, dO or V): the next
+    // item's tiles start arriving while this one finishes
+    if (tid == 0 && w + 1 < w1) tile_loads(w + 1, true, false);
     if (p.fused) {
       // dq = anchor part + GLA part, bf16, written in place over the GLA
       // part in the V region and stored with TMA (rows past L are clipped)
-      ok = mbar_wait(&bars[5], 0, p.status, ST_TIMEOUT);
+      ok = mbar_wait(&bars[5], par, p.status, ST_TIMEOUT);
       if (__syncthreads_or(!ok)) goto done;
       for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
         float v[32];
@@ -412,8 +441,7 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
         bulk_commit();
         bulk_wait_all();
       }
-      goto done;
-    }
+    } else {
     // dq, staged as an fp32 tile over the free Q | dO regions and written
     // with TMA stores (rows past L are clipped by the map)
     unsigned char *st = sm + R_Q;
@@ -444,6 +472,12 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
       bulk_commit();
       bulk_wait_all();
     }
+    }
+  }
+  // the store has read this item's staging: the rest of the next item's tiles
+  tc_fence_before();
+  __syncthreads();
+  if (tid == 0 && w + 1 < w1) tile_loads(w + 1, false, true);
   }
 done:
   tc_fence_before();
@@ -784,9 +818,14 @@ cudaError_t launch_tc_swa_bwd(const TcSwaBwdArgs &a, int stage, cudaStream_t s) 
     p.M = a.M;
     p.window = a.window;
     p.scale = a.scale;
+    p.BH = a.BH;
     e = cudaFuncSetAttribute(tc_swa_bwd_q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    tc_swa_bwd_q_kernel<<<dim3(ntiles, a.BH), NT_Q, SMEM_BYTES, s>>>(p);
+    int sms = 148;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const int nwork = ntiles * a.BH;
+    tc_swa_bwd_q_kernel<<<nwork < sms ? nwork : sms, NT_Q, SMEM_BYTES, s>>>(p);
     return cudaGetLastError();
   }
   KVParams p;
