@@ -693,7 +693,7 @@ done:
 // (lane = 4 dimensions); the per-row meta terms are broadcast loads.  MM is
 // the meta-token count rounded up to 4, 8 or 16; U tokens are in flight per
 // warp.  Warps combine in shared memory, then one global add per element.
-constexpr int kMetaTok = 1024;
+constexpr int kMetaTok = 256;   // tokens per CTA: enough CTAs that the last wave is a small share
 template <int MM, int U>
 __global__ void __launch_bounds__(256) meta_grad_kernel(const __nv_bfloat16 *q, const __nv_bfloat16 *dout,
                                                          const float *dsm, const float *pm, const float *alpha,
@@ -778,7 +778,7 @@ cudaError_t launch_tc_swa_bwd(const TcSwaBwdArgs &a, int stage, cudaStream_t s) 
     const auto *qp = static_cast<const __nv_bfloat16 *>(a.q);
     const auto *op = static_cast<const __nv_bfloat16 *>(a.dout);
     if (a.M <= 4)
-      meta_grad_kernel<4, 4><<<grid, 256, 0, s>>>(qp, op, a.dsm, a.pm, a.alpha, a.dmeta_k, a.dmeta_v, a.B, a.H,
+      meta_grad_kernel<4, 8><<<grid, 256, 0, s>>>(qp, op, a.dsm, a.pm, a.alpha, a.dmeta_k, a.dmeta_v, a.B, a.H,
                                                   a.L, a.M, a.scale);
     else if (a.M <= 8)
       meta_grad_kernel<8, 2><<<grid, 256, 0, s>>>(qp, op, a.dsm, a.pm, a.alpha, a.dmeta_k, a.dmeta_v, a.B, a.H,
