@@ -156,32 +156,108 @@ float scale_of(const lizard_fwd_args *a) {
 }
 
 // A call's kernels in launch order.  The same list serves the launch and the
-// host-only plan query, so the names always match what runs.
+// host-only plan query, so the names always match what runs.  Kernels on
+// lane 1 may run beside those on lane 0: fork() lets lane 1 start after
+// everything enqueued so far, join() makes lane 0 wait for lane 1.  The
+// lanes are the call's stream and a side stream of this host thread (created
+// on the first call on a device, outside any stream capture; inside a
+// capture without one, and whenever per-kernel timing events are requested,
+// everything runs in order on the call's stream).
 struct Plan {
-  static constexpr int kMax = 24;
-  const char *names[kMax];
-  std::function<cudaError_t()> fns[kMax];
+  static constexpr int kMax = 32;
+  struct Step {
+    const char *name;
+    std::function<cudaError_t(cudaStream_t)> fn;
+    int lane;
+    int sync;   // 0 kernel, 1 fork, 2 join
+  };
+  Step steps[kMax];
   int n = 0;
-  void add(const char *name, std::function<cudaError_t()> f) {
-    names[n] = name;
-    fns[n] = std::move(f);
-    ++n;
+  void add(const char *name, std::function<cudaError_t(cudaStream_t)> f, int lane = 0) {
+    steps[n++] = Step{name, std::move(f), lane, 0};
   }
-  lizard_status run(cudaStream_t s, void *const *events, int nev) const {
-    if (events && nev > 0 && cudaEventRecord(static_cast<cudaEvent_t>(events[0]), s) != cudaSuccess)
-      return LIZARD_ERR_CUDA;
-    for (int i = 0; i < n; ++i) {
-      if (fns[i]() != cudaSuccess) return LIZARD_ERR_CUDA;
-      if (events && i + 1 < nev && cudaEventRecord(static_cast<cudaEvent_t>(events[i + 1]), s) != cudaSuccess)
-        return LIZARD_ERR_CUDA;
-    }
-    return LIZARD_OK;
-  }
+  void fork() { steps[n++] = Step{nullptr, {}, 0, 1}; }
+  void join() { steps[n++] = Step{nullptr, {}, 0, 2}; }
+  lizard_status run(cudaStream_t s, void *const *events, int nev) const;
   int32_t names_out(const char **out, int32_t cap) const {
-    for (int i = 0; i < n && i < cap; ++i) out[i] = names[i];
-    return n;
+    int32_t k = 0;
+    for (int i = 0; i < n; ++i)
+      if (steps[i].sync == 0) {
+        if (k < cap) out[k] = steps[i].name;
+        ++k;
+      }
+    return k;
   }
 };
+
+// This host thread's side stream and fork / join events on the current
+// device; false when they cannot be had (creation failed, or the stream is
+// being captured and they do not exist yet).
+bool side_lane(cudaStream_t s, cudaStream_t *side, cudaEvent_t *ev_fork, cudaEvent_t *ev_join) {
+  constexpr int kDev = 64;
+  thread_local cudaStream_t t_side[kDev] = {};
+  thread_local cudaEvent_t t_fork[kDev] = {}, t_join[kDev] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDev) return false;
+  if (!t_side[dev]) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return false;
+    cudaStream_t st = nullptr;
+    cudaEvent_t ef = nullptr, ej = nullptr;
+    if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess) return false;
+    if (cudaEventCreateWithFlags(&ef, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ej, cudaEventDisableTiming) != cudaSuccess) {
+      if (ef) cudaEventDestroy(ef);
+      cudaStreamDestroy(st);
+      return false;
+    }
+    t_side[dev] = st;
+    t_fork[dev] = ef;
+    t_join[dev] = ej;
+  }
+  *side = t_side[dev];
+  *ev_fork = t_fork[dev];
+  *ev_join = t_join[dev];
+  return true;
+}
+
+lizard_status Plan::run(cudaStream_t s, void *const *events, int nev) const {
+  const bool timing = events && nev > 0;
+  bool any_fork = false;
+  for (int i = 0; i < n; ++i) any_fork |= steps[i].sync == 1;
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  const bool lanes = !timing && any_fork && side_lane(s, &side, &ev_fork, &ev_join);
+  if (timing && cudaEventRecord(static_cast<cudaEvent_t>(events[0]), s) != cudaSuccess) return LIZARD_ERR_CUDA;
+  int k = 0;
+  bool open = false;   // lane 1 has work that lane 0 has not joined
+  for (int i = 0; i < n; ++i) {
+    const Step &st = steps[i];
+    if (st.sync == 1) {
+      if (lanes && (cudaEventRecord(ev_fork, s) != cudaSuccess || cudaStreamWaitEvent(side, ev_fork, 0) != cudaSuccess))
+        return LIZARD_ERR_CUDA;
+      continue;
+    }
+    if (st.sync == 2) {
+      if (lanes && open) {
+        if (cudaEventRecord(ev_join, side) != cudaSuccess || cudaStreamWaitEvent(s, ev_join, 0) != cudaSuccess)
+          return LIZARD_ERR_CUDA;
+        open = false;
+      }
+      continue;
+    }
+    const bool on_side = lanes && st.lane == 1;
+    if (st.fn(on_side ? side : s) != cudaSuccess) return LIZARD_ERR_CUDA;
+    open |= on_side;
+    ++k;
+    if (timing && k < nev && cudaEventRecord(static_cast<cudaEvent_t>(events[k]), s) != cudaSuccess)
+      return LIZARD_ERR_CUDA;
+  }
+  if (lanes && open &&
+      (cudaEventRecord(ev_join, side) != cudaSuccess || cudaStreamWaitEvent(s, ev_join, 0) != cudaSuccess))
+    return LIZARD_ERR_CUDA;
+  return LIZARD_OK;
+}
 
 // `target`, `dmse`, `loss`: the stage-1 loss, which the tensor-core forward
 // forms in its epilogue (null otherwise).
@@ -195,27 +271,27 @@ void fwd_plan(const lizard_fwd_args *a, void *ws, cudaStream_t s, Plan &plan, co
                     a->state_in, a->o, gla_on(a) ? a->state_out : nullptr, swa_on(a) ? a->lse : nullptr,
                     static_cast<uint32_t *>(ws), at<void>(ws, lay.phq), BH, a->H, a->L, a->M, a->window,
                     a->branch, 1.f / a->gate_temp, scale_of(a), scalar_gate(a), target, dmse, loss};
-    if (gla_on(a)) plan.add("gate_prep_kernel", [=] { return lz::launch_tc_fwd(t, 3, s); });
+    if (gla_on(a)) plan.add("gate_prep_kernel", [=](cudaStream_t s) { return lz::launch_tc_fwd(t, 3, s); });
     if (lz::tc_fwd_stage_count(BH, a->L) > 1) {
-      plan.add("tc_fwd_kernel(state pass)", [=] { return lz::launch_tc_fwd(t, 0, s); });
-      plan.add("seg_combine_kernel", [=] { return lz::launch_tc_fwd(t, 1, s); });
+      plan.add("tc_fwd_kernel(state pass)", [=](cudaStream_t s) { return lz::launch_tc_fwd(t, 0, s); });
+      plan.add("seg_combine_kernel", [=](cudaStream_t s) { return lz::launch_tc_fwd(t, 1, s); });
     }
-    plan.add("tc_fwd_kernel", [=] { return lz::launch_tc_fwd(t, 2, s); });
+    plan.add("tc_fwd_kernel", [=](cudaStream_t s) { return lz::launch_tc_fwd(t, 2, s); });
     return;
   }
   float *o_gla = nullptr;
   if (gla_on(a)) {
     lz::PrepArgs pa{a->q, a->k, a->g, a->fmap_wq, a->fmap_wk, at<float>(ws, lay.phq), at<float>(ws, lay.phk),
                     at<float>(ws, lay.a), a->H, a->L, 1.f / a->gate_temp, scalar_gate(a)};
-    plan.add("prep_kernel", [=] { return lz::launch_prep(pa, BH, D, bf16, s); });
+    plan.add("prep_kernel", [=](cudaStream_t s) { return lz::launch_prep(pa, BH, D, bf16, s); });
     o_gla = at<float>(ws, lay.o_gla);
     lz::GlaFwdArgs ga{at<float>(ws, lay.phq), at<float>(ws, lay.phk), at<float>(ws, lay.a), a->v, a->state_in,
                       o_gla, a->state_out, a->L};
-    plan.add("gla_fwd_simt", [=] { return lz::launch_gla_fwd_simt(ga, BH, D, bf16, s); });
+    plan.add("gla_fwd_simt", [=](cudaStream_t s) { return lz::launch_gla_fwd_simt(ga, BH, D, bf16, s); });
   }
   lz::SwaMixArgs sa{a->q, a->k, a->v, a->meta_k, a->meta_v, a->alpha, o_gla, a->o,
                     swa_on(a) ? a->lse : nullptr, a->H, a->L, a->window, a->M, a->branch, scale_of(a)};
-  plan.add("swa_mix_simt", [=] { return lz::launch_swa_mix_simt(sa, BH, D, bf16, s); });
+  plan.add("swa_mix_simt", [=](cudaStream_t s) { return lz::launch_swa_mix_simt(sa, BH, D, bf16, s); });
 }
 
 void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan) {
@@ -234,27 +310,31 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan) {
     float *e32 = at<float>(ws, lay.e32), *gr = at<float>(ws, lay.gr);
     uint32_t *status = static_cast<uint32_t *>(ws);
     plan.add("gate_prep_kernel",
-             [=] { return lz::launch_gate_prep(a->g, nullptr, e32, gr, status, BH, a->L, inv_tau, f.scalar_gate != 0,
+             [=](cudaStream_t s) { return lz::launch_gate_prep(a->g, nullptr, e32, gr, status, BH, a->L, inv_tau, f.scalar_gate != 0,
                                                s); });
-    plan.add("tc_fwd_kernel(state copies)", [=] { return lz::launch_tc_state_snapshots(f, snap_s, e32, gr, s); });
+    // the state copies beside the weight conversion and the reverse dS pass
+    plan.fork();
+    plan.add("tc_fwd_kernel(state copies)",
+             [=](cudaStream_t s) { return lz::launch_tc_state_snapshots(f, snap_s, e32, gr, s); }, 1);
     lz::TcGlaBwdArgs t{a->q, a->k, a->v, a->g, b->dout, a->fmap_wq, a->fmap_wk, snap_s,
                        at<void>(ws, lay.snap_ds), at<float>(ws, lay.dphq), at<float>(ws, lay.dphk),
                        at<float>(ws, lay.da), at<float>(ws, lay.dv_gla), b->dg, b->dstate_in,
                        status, a->H, BH, a->L, inv_tau, e32, gr, scalar_gate(a), at<void>(ws, lay.w16)};
     void *w16 = at<void>(ws, lay.w16);
-    plan.add("weights_bf16_kernel", [=] { return lz::launch_weights_bf16(a->fmap_wq, a->fmap_wk, w16, a->H, s); });
-    plan.add("tc_gla_dstates_kernel", [=] { return lz::launch_tc_gla_bwd(t, 0, s); });
-    plan.add("tc_gla_bwd_tile_kernel", [=] { return lz::launch_tc_gla_bwd(t, 1, s); });
+    plan.add("weights_bf16_kernel", [=](cudaStream_t s) { return lz::launch_weights_bf16(a->fmap_wq, a->fmap_wk, w16, a->H, s); });
+    plan.add("tc_gla_dstates_kernel", [=](cudaStream_t s) { return lz::launch_tc_gla_bwd(t, 0, s); });
+    plan.join();
+    plan.add("tc_gla_bwd_tile_kernel", [=](cudaStream_t s) { return lz::launch_tc_gla_bwd(t, 1, s); });
   } else if (g) {
     lz::PrepArgs pa{a->q, a->k, a->g, a->fmap_wq, a->fmap_wk, at<float>(ws, lay.phq), at<float>(ws, lay.phk),
                     at<float>(ws, lay.a), a->H, a->L, inv_tau, scalar_gate(a)};
-    plan.add("prep_kernel", [=] { return lz::launch_prep(pa, BH, D, bf16, s); });
+    plan.add("prep_kernel", [=](cudaStream_t s) { return lz::launch_prep(pa, BH, D, bf16, s); });
     lz::GlaStatesArgs sa{at<float>(ws, lay.phk), at<float>(ws, lay.a), a->v, a->state_in, at<float>(ws, lay.sprev), a->L};
-    plan.add("gla_states_simt", [=] { return lz::launch_gla_states(sa, BH, D, bf16, s); });
+    plan.add("gla_states_simt", [=](cudaStream_t s) { return lz::launch_gla_states(sa, BH, D, bf16, s); });
     lz::GlaBwdArgs ga{at<float>(ws, lay.phq), at<float>(ws, lay.phk), at<float>(ws, lay.a), a->v, b->dout,
                       at<float>(ws, lay.sprev), at<float>(ws, lay.dphq), at<float>(ws, lay.dphk),
                       at<float>(ws, lay.da), at<float>(ws, lay.dv_gla), b->dstate_in, a->L};
-    plan.add("gla_bwd_simt", [=] { return lz::launch_gla_bwd_simt(ga, BH, D, bf16, s); });
+    plan.add("gla_bwd_simt", [=](cudaStream_t s) { return lz::launch_gla_bwd_simt(ga, BH, D, bf16, s); });
   }
   const bool swa_tc = w && bwd_swa_uses_tc(a, b->impl);
   const bool finish_tc = gla_tc && a->fmap_wq && a->fmap_wk;
@@ -272,11 +352,17 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan) {
                        b->dq, b->dk, b->dv, b->dg, b->dfmap_wq, b->dfmap_wk, a->H, a->L, inv_tau,
                        gla_tc ? 0 : 1, static_cast<uint32_t *>(ws), nullptr, nullptr, scalar_gate(a)};
   if (gla_tc) fa.da = nullptr;   // the gate gradient comes from gate_grad_kernel
+  lz::TcGlaBwdArgs tg{a->q, a->k, a->v, a->g, b->dout, a->fmap_wq, a->fmap_wk, nullptr, nullptr, nullptr,
+                      nullptr, at<float>(ws, lay.da), nullptr, b->dg, nullptr, static_cast<uint32_t *>(ws),
+                      a->H, BH, a->L, inv_tau, nullptr, nullptr, scalar_gate(a)};
   if (fused) {
+    // the gate-logit gradient (from dB) beside the feature-map and anchor passes
+    plan.fork();
+    plan.add("gate_grad_kernel", [=](cudaStream_t s) { return lz::launch_tc_gla_bwd(tg, 2, s); }, 1);
     fa.xq_part = at<void>(ws, lay.dq_swa);   // bf16 parts in the anchor part slots
     fa.xk_part = at<void>(ws, lay.dk_swa);
     fa.dq_swa = fa.dk_swa = fa.dv_swa = nullptr;
-    plan.add("tc_finish_kernel", [=] { return lz::launch_tc_finish(fa, BH, s); });
+    plan.add("tc_finish_kernel", [=](cudaStream_t s) { return lz::launch_tc_finish(fa, BH, s); });
   }
   if (swa_tc) {
     lz::TcSwaBwdArgs t{a->q, a->k, a->v, b->dout, a->meta_k, a->meta_v, a->alpha,
@@ -293,31 +379,30 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan) {
       t.dk_out = b->dk;
       t.dv_out = b->dv;
     }
-    plan.add("tc_swa_bwd_q_kernel", [=] { return lz::launch_tc_swa_bwd(t, 0, s); });
-    plan.add("tc_swa_bwd_kv_kernel", [=] { return lz::launch_tc_swa_bwd(t, 1, s); });
-    if (a->M > 0 && (b->dmeta_k || b->dmeta_v))
-      plan.add("meta_grad_kernel", [=] { return lz::launch_tc_swa_bwd(t, 2, s); });
+    plan.add("tc_swa_bwd_q_kernel", [=](cudaStream_t s) { return lz::launch_tc_swa_bwd(t, 0, s); });
+    if (a->M > 0 && (b->dmeta_k || b->dmeta_v)) {   // beside the dk / dv pass, after the dq pass's terms
+      plan.fork();
+      plan.add("meta_grad_kernel", [=](cudaStream_t s) { return lz::launch_tc_swa_bwd(t, 2, s); }, 1);
+    }
+    plan.add("tc_swa_bwd_kv_kernel", [=](cudaStream_t s) { return lz::launch_tc_swa_bwd(t, 1, s); });
+    plan.join();
   } else if (w) {
     lz::SwaBwdQArgs qa{a->q, a->k, a->v, b->dout, a->meta_k, a->meta_v, a->alpha,
                        at<float>(ws, lay.dq_swa), at<float>(ws, lay.lse), at<float>(ws, lay.Dterm),
                        b->dmeta_k, b->dmeta_v, b->dalpha, a->H, a->L, a->window, a->M, scale_of(a)};
-    plan.add("swa_bwd_q", [=] { return lz::launch_swa_bwd_q(qa, BH, D, bf16, s); });
+    plan.add("swa_bwd_q", [=](cudaStream_t s) { return lz::launch_swa_bwd_q(qa, BH, D, bf16, s); });
     lz::SwaBwdKVArgs ka{a->q, a->k, a->v, b->dout, a->alpha, at<float>(ws, lay.lse), at<float>(ws, lay.Dterm),
                         at<float>(ws, lay.dk_swa), at<float>(ws, lay.dv_swa), a->H, a->L, a->window, scale_of(a)};
-    plan.add("swa_bwd_kv", [=] { return lz::launch_swa_bwd_kv(ka, BH, D, bf16, s); });
+    plan.add("swa_bwd_kv", [=](cudaStream_t s) { return lz::launch_swa_bwd_kv(ka, BH, D, bf16, s); });
   }
   if (!fused) {
     if (finish_tc)
-      plan.add("tc_finish_kernel", [=] { return lz::launch_tc_finish(fa, BH, s); });
+      plan.add("tc_finish_kernel", [=](cudaStream_t s) { return lz::launch_tc_finish(fa, BH, s); });
     else
-      plan.add("finish_bwd", [=] { return lz::launch_finish_bwd(fa, BH, D, bf16, s); });
+      plan.add("finish_bwd", [=](cudaStream_t s) { return lz::launch_finish_bwd(fa, BH, D, bf16, s); });
   }
-  if (gla_tc) {
-    lz::TcGlaBwdArgs t{a->q, a->k, a->v, a->g, b->dout, a->fmap_wq, a->fmap_wk, nullptr, nullptr, nullptr,
-                       nullptr, at<float>(ws, lay.da), nullptr, b->dg, nullptr, static_cast<uint32_t *>(ws),
-                       a->H, BH, a->L, inv_tau, nullptr, nullptr, scalar_gate(a)};
-    plan.add("gate_grad_kernel", [=] { return lz::launch_tc_gla_bwd(t, 2, s); });
-  }
+  if (gla_tc && !fused)
+    plan.add("gate_grad_kernel", [=](cudaStream_t s) { return lz::launch_tc_gla_bwd(tg, 2, s); });
 }
 
 }  // namespace
@@ -506,7 +591,7 @@ void stage1_plan(const lizard_stage1_args *a, S1Views &v, void *ws, cudaStream_t
     const bool bf16 = f->dtype == LIZARD_BF16;
     const void *target = a->target;
     float *loss = a->loss;
-    plan.add("mse_kernel", [=] { return lz::launch_mse(f->o, target, dmse, loss, nel, bf16, s); });
+    plan.add("mse_kernel", [=](cudaStream_t s) { return lz::launch_mse(f->o, target, dmse, loss, nel, bf16, s); });
   }
   v.b.dout = dmse;
   bwd_plan(&v.b, ws, s, plan);
