@@ -25,7 +25,14 @@
  * Conventions shared by every entry point
  *   - All pointers are DEVICE pointers unless stated otherwise; the caller
  *     owns all memory, including the workspace.  The library allocates and
- *     frees nothing and keeps no state between calls.
+ *     frees no device memory and keeps no results between calls.  To run
+ *     independent backward kernels side by side, it creates on its first
+ *     backward call in each host thread and on each device one non-blocking
+ *     CUDA stream and two events (kept until the process exits); the work is
+ *     forked from and joined back into the call's stream with events, so a
+ *     stream capture of the call records it.  A first call made inside a
+ *     stream capture, or any call given per-kernel timing events, runs every
+ *     kernel in order on the call's stream instead.
  *   - Activations (q, k, v, g, o, caches, their gradients) use `dtype`
  *     (bf16 or fp32), contiguous row-major with the innermost dimension last
  *     (the shapes below).  Parameters (feature-map weights, meta tokens,
