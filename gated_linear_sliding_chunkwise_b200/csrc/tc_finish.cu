@@ -96,6 +96,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
   const uint32_t id_dx = idesc_bf16(128, 128, 0, 0);   // dZ (K-major) x W^T (K-major, N = 128)
   const uint32_t id_dw = idesc_bf16(128, 64, 1, 1);    // X^T (MN-major) x dZ (MN-major, N = 64)
   bool fail = false;
+  // this row's dphi values (its group's half) of one map, loaded ahead: map 0
+  // of the next tile while this tile finishes, map 1 while map 0 is used
+  float4 dpre[16];
+  auto dphi_load = [&](int m, int c) {
+    const int t = c * T + row;
+    const float *src = (m == 0 ? p.dphq : p.dphk) + ((size_t)bh * p.L + (t < p.L ? t : 0)) * D + wg * F;
+#pragma unroll
+    for (int u = 0; u < 16; ++u)
+      dpre[u] = t < p.L ? *reinterpret_cast<const float4 *>(src + 4 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+  };
+  if (gla && ntiles > 0) dphi_load(0, 0);
   for (int c = 0; c < ntiles; ++c) {
     const uint32_t par = c & 1;
     const int tq = c * T + row;
@@ -124,11 +135,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
       for (int m = 0; m < 2; ++m) {
         float ph[F];
         const float sc = feature_half(tl + (m == 0 ? C_ZQ : C_ZK), wg, ph);
-        const float *__restrict__ src = (m == 0 ? p.dphq : p.dphk) + off + wg * F;
-        float4 d[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u)
-          d[u] = valid ? *reinterpret_cast<const float4 *>(src + 4 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 *d = dpre;
         float dot4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
@@ -146,6 +153,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
           ph[4 * u + 2] *= d[u].z - dot;
           ph[4 * u + 3] *= d[u].w - dot;
         }
+        if (m == 0) dphi_load(1, c);   // the k map's values, in flight while this map finishes
+        else if (c + 1 < ntiles) dphi_load(0, c + 1);
         // send the half-terms of the other group's features
         unsigned char *mine = sm + R_STG + (2 * m + wg) * 16384;
         const unsigned char *theirs = sm + R_STG + (2 * m + 1 - wg) * 16384;

@@ -195,7 +195,9 @@ def test_side_by_side_backward_matches_in_order_run(lz):
     for name in ("dq", "dk", "dv", "dg", "dstate_in"):
         assert torch.equal(a[name], b[name]), name
     for name in ("dmeta_k", "dmeta_v", "dfmap_wq", "dfmap_wk", "dalpha"):
-        torch.testing.assert_close(a[name], b[name], rtol=1e-5, atol=1e-7)
+        # sums of fp32 atomics: their order varies from run to run
+        err = float((a[name] - b[name]).abs().max())
+        assert err <= 1e-4 * float(b[name].abs().max()), (name, err)
     # graph capture (the side stream exists by now)
     ws = a["workspace"]
     outs = {}
