@@ -767,10 +767,12 @@ namespace {
 
 // Start state of every segment: S_0 = state_in (or 0),
 // S_{s+1} = diag(exp(decay_s)) S_s + local_s.
+// One thread per state element: grid (B*H, D*D / 256).
 __global__ void __launch_bounds__(256) seg_combine_kernel(const float *seg_state, const float *seg_decay,
                                                           const float *state_in, float *seg_start, int nseg) {
   const int bh = blockIdx.x;
-  for (int e = threadIdx.x; e < D * D; e += 256) {
+  {
+    const int e = blockIdx.y * 256 + threadIdx.x;
     const int i = e / D;
     float sv = state_in ? state_in[(size_t)bh * D * D + e] : 0.f;
     seg_start[((size_t)bh * nseg) * D * D + e] = sv;
@@ -788,11 +790,23 @@ bool tc_fwd_supported(int dk, int dv, int window, int M, bool bf16) {
   return bf16 && dk == D && dv == D && window <= T && M <= MAXM;
 }
 
-// Segments per sequence: enough (batch, head, segment) CTAs to cover the
-// 148 SMs once, each segment at least two tiles long.
+// Segments per sequence, for few (batch, head) sequences: from enough
+// (sequence, segment) CTAs to cover the 148 SMs once up to twice that, the
+// count whose last wave is fullest (one CTA per SM), each segment at least
+// two tiles long.
 void tc_fwd_segments(int BH, int L, int *nseg, int *tiles_per_seg) {
+  constexpr int kSMs = 148;
   const int ntiles = (L + T - 1) / T;
-  int n = BH >= 120 ? 1 : 148 / (BH > 0 ? BH : 1);
+  int n = 1;
+  if (BH > 0 && BH < 120) {
+    const int n0 = kSMs / BH;
+    double best = -1.0;
+    for (int c = n0; c <= 2 * n0 + 1; ++c) {
+      const int ctas = BH * c, waves = (ctas + kSMs - 1) / kSMs;
+      const double fill = (double)ctas / ((double)waves * kSMs);
+      if (fill > best + 1e-9) { best = fill; n = c; }
+    }
+  }
   n = n < ntiles / 2 ? n : ntiles / 2;
   if (n < 1) n = 1;
   const int tps = (ntiles + n - 1) / n;
@@ -908,7 +922,8 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, int stage, cudaStream_t s) {
     return launch_gate_prep(a.g, w.e16, w.e32, w.r, a.status, a.BH, a.L, a.inv_tau, a.scalar_gate != 0, s);
   }
   if (nseg > 1 && stage == 1) {
-    seg_combine_kernel<<<a.BH, 256, 0, s>>>(w.seg_state, w.seg_decay, a.state_in, w.seg_start, nseg);
+    seg_combine_kernel<<<dim3(a.BH, D * D / 256), 256, 0, s>>>(w.seg_state, w.seg_decay, a.state_in, w.seg_start,
+                                                               nseg);
     return cudaGetLastError();
   }
   Params p;
