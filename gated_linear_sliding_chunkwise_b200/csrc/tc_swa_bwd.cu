@@ -57,6 +57,7 @@ struct KVParams {
   int H, L, window;
   float scale;
   int fused;
+  int BH;
 };
 
 __device__ __forceinline__ void setup_cta(uint32_t *tmem_slot, uint64_t *bars, int nbars, int tid) {
@@ -503,27 +504,31 @@ __global__ void __launch_bounds__(NT_KV, 1) tc_swa_bwd_kv_kernel(const __grid_co
 
   const int tid = threadIdx.x, warp = tid >> 5, wg = tid >> 7, row = tid & 127;
   const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-  const int bh = blockIdx.y, h = bh % p.H, j0 = blockIdx.x * T, tk = j0 + row;
-  const float alpha = p.alpha ? p.alpha[h] : 1.f;
   const uint32_t sbase = smem_u32(sm);
   setup_cta(&s_tmem, bars, 7, tid);
-  // the tiles first, so that they arrive while the softmax statistics are staged
-  if (tid == 0) {
-    mbar_expect_tx(&bars[0], 6 * TILE);
+  // Persistent: CTA b walks the contiguous run [w0, w1) of (sequence, key
+  // block) items; the next item's query tile b is loaded once this item's
+  // products are done with it, the rest after its store.
+  const int nblk = (p.L + T - 1) / T, nwork = nblk * p.BH;
+  const int w0 = (int)((long long)blockIdx.x * nwork / gridDim.x);
+  const int w1 = (int)((long long)(blockIdx.x + 1) * nwork / gridDim.x);
+  auto tile_loads = [&](int w, bool early, bool late) {
+    const int lbh = w / nblk, lj0 = (w % nblk) * T;
+    if (early) mbar_expect_tx(&bars[0], 6 * TILE);
     for (int r = 0; r < 2; ++r) {
-      tma_load_3d(sm + R_K + r * kReg, &p.mk, &bars[0], 64 * r, j0, bh);
-      tma_load_3d(sm + R_V + r * kReg, &p.mv, &bars[0], 64 * r, j0, bh);
-      for (int it = 0; it < 2; ++it) {
-        tma_load_3d(sm + R_Q0 + it * 2 * TILE + r * kReg, &p.mq, &bars[0], 64 * r, j0 + it * T, bh);
-        tma_load_3d(sm + R_O0 + it * 2 * TILE + r * kReg, &p.mo, &bars[0], 64 * r, j0 + it * T, bh);
+      if (late) {
+        tma_load_3d(sm + R_K + r * kReg, &p.mk, &bars[0], 64 * r, lj0, lbh);
+        tma_load_3d(sm + R_V + r * kReg, &p.mv, &bars[0], 64 * r, lj0, lbh);
+        tma_load_3d(sm + R_Q0 + r * kReg, &p.mq, &bars[0], 64 * r, lj0, lbh);
+        tma_load_3d(sm + R_O0 + r * kReg, &p.mo, &bars[0], 64 * r, lj0, lbh);
+      }
+      if (early) {
+        tma_load_3d(sm + R_Q0 + 2 * TILE + r * kReg, &p.mq, &bars[0], 64 * r, lj0 + T, lbh);
+        tma_load_3d(sm + R_O0 + 2 * TILE + r * kReg, &p.mo, &bars[0], 64 * r, lj0 + T, lbh);
       }
     }
-  }
-  for (int e = tid; e < 2 * T; e += NT_KV) {
-    const int t = j0 + e;
-    s_lse[e] = t < p.L ? p.lse[(size_t)bh * p.L + t] : 0.f;
-    s_D[e] = t < p.L ? p.Dterm[(size_t)bh * p.L + t] : 0.f;
-  }
+  };
+  if (tid == 0 && w0 < w1) tile_loads(w0, true, true);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -531,7 +536,17 @@ __global__ void __launch_bounds__(NT_KV, 1) tc_swa_bwd_kv_kernel(const __grid_co
   const uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
   const uint32_t id_mn = idesc_bf16(128, 128, 0, 1);
   const int r0 = 32 * (warp & 3);          // first key row of this warp
-  bool ok = mbar_wait(&bars[0], 0, p.status, ST_TIMEOUT);
+  bool ok = true;
+  for (int w = w0, itn = 0; w < w1; ++w, ++itn) {
+  const uint32_t par = (uint32_t)itn & 1u;
+  const int bh = w / nblk, h = bh % p.H, j0 = (w % nblk) * T, tk = j0 + row;
+  const float alpha = p.alpha ? p.alpha[h] : 1.f;
+  for (int e = tid; e < 2 * T; e += NT_KV) {   // the softmax statistics of the two query tiles
+    const int t = j0 + e;
+    s_lse[e] = t < p.L ? p.lse[(size_t)bh * p.L + t] : 0.f;
+    s_D[e] = t < p.L ? p.Dterm[(size_t)bh * p.L + t] : 0.f;
+  }
+  ok = mbar_wait(&bars[0], par, p.status, ST_TIMEOUT);
   if (__syncthreads_or(!ok)) goto done;
   for (int it = 0; it < 2; ++it) {
     const uint32_t rq = R_Q0 + it * 2 * TILE, ro = R_O0 + it * 2 * TILE;
@@ -542,7 +557,7 @@ __global__ void __launch_bounds__(NT_KV, 1) tc_swa_bwd_kv_kernel(const __grid_co
       for (int s = 0; s < 8; ++s) mma_ss(tb + C_DP, desc_k(sbase + R_V, s), desc_k(sbase + ro, s), id_kk, s > 0);
       mma_commit(&bars[1 + 2 * it]);
     }
-    ok = mbar_wait(&bars[1 + 2 * it], 0, p.status, ST_TIMEOUT);
+    ok = mbar_wait(&bars[1 + 2 * it], par, p.status, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) goto done;
     tc_fence_after();
     if (p.fused && it == 1 && tid == 0) {   // K and V are read: the GLA part of dk into K
@@ -604,9 +619,10 @@ __global__ void __launch_bounds__(NT_KV, 1) tc_swa_bwd_kv_kernel(const __grid_co
       for (int s = 0; s < 8; ++s) mma_ts(tb + C_DK, tb + C_DS + s * 8, desc_mn(sbase + rq, s), id_mn, it > 0 || s > 0);
       mma_commit(&bars[2 + 2 * it]);
     }
-    ok = mbar_wait(&bars[2 + 2 * it], 0, p.status, ST_TIMEOUT);
+    ok = mbar_wait(&bars[2 + 2 * it], par, p.status, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) goto done;
     tc_fence_after();
+    if (it == 1 && tid == 0 && w + 1 < w1) tile_loads(w + 1, true, false);   // query tile b is done
     if (p.fused && it == 0 && tid == 0) {   // query tile a is done: the GLA dv into its regions
       mbar_expect_tx(&bars[5], 2 * TILE);
       for (int bx = 0; bx < 4; ++bx) tma_load_3d(sm + R_Q0 + bx * 16384, &p.mdvg, &bars[5], 32 * bx, j0, bh);
@@ -616,8 +632,8 @@ __global__ void __launch_bounds__(NT_KV, 1) tc_swa_bwd_kv_kernel(const __grid_co
     // dk = anchor part + GLA part (bf16, in place over the GLA part in K);
     // dv = anchor part + GLA dv (fp32 in Q_a | dO_a) as bf16 into V; both
     // stored with TMA (rows past L are clipped by the maps)
-    ok = mbar_wait(&bars[5], 0, p.status, ST_TIMEOUT);
-    ok &= mbar_wait(&bars[6], 0, p.status, ST_TIMEOUT);
+    ok = mbar_wait(&bars[5], par, p.status, ST_TIMEOUT);
+    ok &= mbar_wait(&bars[6], par, p.status, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) goto done;
     for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
       float a[32], b[32];
@@ -650,9 +666,7 @@ __global__ void __launch_bounds__(NT_KV, 1) tc_swa_bwd_kv_kernel(const __grid_co
       bulk_commit();
       bulk_wait_all();
     }
-    goto done;
-  }
-  {
+  } else {
     // dK, dV, staged as fp32 tiles over the free K | V and Q_a | dO_a regions
     // and written with TMA stores (rows past L are clipped by the maps)
     unsigned char *st0 = sm + R_K, *st1 = sm + R_Q0;
@@ -678,6 +692,11 @@ __global__ void __launch_bounds__(NT_KV, 1) tc_swa_bwd_kv_kernel(const __grid_co
       bulk_commit();
       bulk_wait_all();
     }
+  }
+  // the store has read this item's staging: the rest of the next item's tiles
+  tc_fence_before();
+  __syncthreads();
+  if (tid == 0 && w + 1 < w1) tile_loads(w + 1, false, true);
   }
 done:
   tc_fence_before();
@@ -853,7 +872,14 @@ cudaError_t launch_tc_swa_bwd(const TcSwaBwdArgs &a, int stage, cudaStream_t s) 
   p.scale = a.scale;
   e = cudaFuncSetAttribute(tc_swa_bwd_kv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  tc_swa_bwd_kv_kernel<<<dim3(ntiles, a.BH), NT_KV, SMEM_BYTES, s>>>(p);
+  p.BH = a.BH;
+  {
+    int sms = 148;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const int nwork = ntiles * a.BH;
+    tc_swa_bwd_kv_kernel<<<nwork < sms ? nwork : sms, NT_KV, SMEM_BYTES, s>>>(p);
+  }
   return cudaGetLastError();
 }
 
