@@ -62,7 +62,6 @@ struct TileParams {
   CUtensorMap mq, mk, mv, mo, msp, mds;       // msp / mds: [BH*ntiles][D][D] snapshots
   CUtensorMap mw;                             // [H*2][D][F] bf16 feature-map weights (W_q, W_k per head)
   CUtensorMap mdq, mdk, mdb, mdv;             // fp32 outputs dphi_q, dphi_k, dB, dv (TMA stores)
-  const float *wq, *wk;
   const float *e32;            // fp32 decay factors [BH*L][D]
   const float *sp_r0, *ds_r0;  // [BH*ntiles][D] row 0 of S' and of dS (the copies hold the rest)
   float *dphq, *dphk, *dB, *dv;
@@ -753,8 +752,6 @@ cudaError_t launch_tc_gla_bwd(const TcGlaBwdArgs &a, int stage, cudaStream_t s) 
         !make_map_f32_3d(&p.mdq, a.dphq, D, rows, a.BH, T) || !make_map_f32_3d(&p.mdk, a.dphk, D, rows, a.BH, T) ||
         !make_map_f32_3d(&p.mdb, a.dB, D, rows, a.BH, T) || !make_map_f32_3d(&p.mdv, a.dv, D, rows, a.BH, T))
       return cudaErrorInvalidValue;
-    p.wq = a.wq;
-    p.wk = a.wk;
     p.e32 = a.e32;
     p.sp_r0 = snapshot_row0(a.snap_s, a.BH, a.L);
     p.ds_r0 = snapshot_row0(a.snap_ds, a.BH, a.L);
