@@ -459,7 +459,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_stream_kernel(const __g
   __shared__ __align__(16) float zpart[8][SD];       // read-out partials per row group
   __shared__ float prob[128 + 16];
   __shared__ float red[8][SD];
-  __shared__ float s_inv;
+  __shared__ float s_wmax[8], s_wsum[9];             // per-warp softmax maxima and sums (+ the meta sum)
   __shared__ float p_red[4][2];                      // prep: per-warp maxima, then sums
   __shared__ int s_n[kMaxRunPairs], s_slot[kMaxRunPairs];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -627,6 +627,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_stream_kernel(const __g
   const int cg = tid & 31, rg = tid >> 5;   // state: float4 column group, row group (8 rows)
   const int vg = tid & 15, eg = tid >> 4;   // values: 8 columns, slot group
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float inv_l = 0.f, alpha_h = 1.f;   // this pair's 1 / softmax sum; this head's alpha
   int cur_head = -1, nh = 0;
   bool failed = false;
   int c_stop = nchunks;
@@ -646,6 +647,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_stream_kernel(const __g
       ok &= s_mbar_wait(&wfull, (uint32_t)nh & 1u);   // meta values
       ++nh;
       cur_head = pi.h;
+      alpha_h = p.alpha ? p.alpha[pi.h] : 1.f;
     }
     if (!ok) {
       atomicOr(&g_decode_status, 1u);
@@ -668,8 +670,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_stream_kernel(const __g
       }
       // ---- window logits: two threads per slot (64 dimensions each); the
       //      slot being replaced takes the new key
+      const int j = tid >> 1, half = tid & 1;
+      float lj = kNegBig;   // the logit of slot j (both threads of the slot hold it)
       {
-        const int j = tid >> 1, half = tid & 1;
         float d = 0.f;
         if (j < n) {
           const __nv_bfloat16 *kr = j == slot ? tk + SD + half * 64
@@ -686,26 +689,40 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_stream_kernel(const __g
           }
         }
         d += __shfl_xor_sync(0xffffffffu, d, 1);
-        if (j < n && half == 0) prob[j] = d * p.scale;
+        if (j < n) lj = d * p.scale;
+      }
+      // softmax over the n window logits and the M meta logits, spread over
+      // the consumer warps: warp maxima, then one exp per slot and warp sums
+      {
+        const float wm = warp_max(lj);
+        if (lane == 0) s_wmax[warp] = wm;
       }
       __syncwarp();
       if (lane == 0) s_mbar_arrive(&empty[sl]);   // the key window and the token are read
       consumers_sync();
-      if (warp == 0) {   // softmax over the n window logits and the M meta logits
-        const int ntot = n + p.M;
-        float mx = kNegBig;
-        for (int j = lane; j < ntot; j += 32) mx = fmaxf(mx, j < n ? prob[j] : R.ml[j - n]);
-        mx = warp_max(mx);
-        float sum = 0.f;
-        for (int j = lane; j < ntot; j += 32) {
-          const float e = expf((j < n ? prob[j] : R.ml[j - n]) - mx);
-          prob[j] = e;
-          sum += e;
+      float mx = kNegBig;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) mx = fmaxf(mx, s_wmax[w]);
+      for (int m = 0; m < p.M; ++m) mx = fmaxf(mx, R.ml[m]);
+      {
+        const float e = j < n ? expf(lj - mx) : 0.f;
+        if (j < n && half == 0) prob[j] = e;
+        const float ws = warp_sum(half == 0 ? e : 0.f);
+        if (lane == 0) s_wsum[warp] = ws;
+        if (warp == 0) {   // the meta tokens
+          const float em = lane < p.M ? expf(R.ml[lane] - mx) : 0.f;
+          if (lane < p.M) prob[n + lane] = em;
+          const float ms = warp_sum(em);
+          if (lane == 0) s_wsum[8] = ms;
         }
-        sum = warp_sum(sum);
-        if (lane == 0) s_inv = 1.f / sum;
       }
       consumers_sync();   // the probabilities are ready
+      {
+        float sum = 0.f;
+#pragma unroll
+        for (int w = 0; w < 9; ++w) sum += s_wsum[w];
+        inv_l = 1.f / sum;
+      }
     } else if (kind == 1 || kind == 2) {
       // ---- state rows (kind - 1) * 64 .. + 63: update, store, read out
       const float4 v4 = make_float4(xv_c[cg * 4], xv_c[cg * 4 + 1], xv_c[cg * 4 + 2], xv_c[cg * 4 + 3]);
@@ -777,8 +794,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_stream_kernel(const __g
         for (int w = 0; w < 8; ++w) so += red[w][tid];
 #pragma unroll
         for (int r = 0; r < 8; ++r) sg += zpart[r][tid];
-        const float alpha = p.alpha ? p.alpha[h] : 1.f;
-        static_cast<__nv_bfloat16 *>(p.o)[(size_t)bh * SD + tid] = __float2bfloat16_rn(sg + alpha * so * s_inv);
+        static_cast<__nv_bfloat16 *>(p.o)[(size_t)bh * SD + tid] = __float2bfloat16_rn(sg + alpha_h * so * inv_l);
         // the new token enters the ring (both windows were read above); the
         // fp32 copies hold it exactly (bf16 -> fp32 -> bf16 is lossless)
         const size_t cw = ((size_t)bh * p.window + slot) * SD + tid;
