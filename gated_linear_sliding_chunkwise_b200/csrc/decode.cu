@@ -350,8 +350,8 @@ constexpr int SD = 128, SF = 64;
 constexpr int kMaxRunPairs = 64;                  // pairs whose (n, slot) are precomputed
 constexpr size_t kRingOff = 0;
 constexpr size_t kWOff = kStreamSlots * (size_t)kChunkBytes;   // W_q | W_k, fp32 [128][64] each
-constexpr size_t kTokOff = kWOff + 2 * SD * SF * 4;           // [slot][q, k, v, g][128] bf16
-constexpr size_t kMetaOff = kTokOff + kStreamSlots * 4 * SD * 2;   // meta_k | meta_v, fp32 [M][128]
+constexpr size_t kTokOff = kWOff + 2 * SD * SF * 4;           // [q, k, v, g][128] bf16 (slot 0's token)
+constexpr size_t kMetaOff = kTokOff + 4 * SD * 2;   // meta_k | meta_v, fp32 [M][128]
 
 __device__ uint32_t g_decode_status;   // bit 1: a bounded wait gave up
 
@@ -444,6 +444,8 @@ LZ_DEV bool consumers_any(bool v) {
 
 struct PairRec {                 // what the prep warps hand to the consumers for one pair
   float phq[SD], phk[SD], gam[SD], ml[16];
+  float lg[SD];                  // window logits (scaled), slots 0 .. n - 1
+  float xk[SD], xv[SD];          // the new token's k and v
 };
 
 __global__ void __launch_bounds__(kDecThreads, 1) decode_stream_kernel(const __grid_constant__ DecodeArgs p, int B, int run) {
@@ -455,7 +457,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_stream_kernel(const __g
   __shared__ uint64_t full[kStreamSlots], empty[kStreamSlots];
   __shared__ uint64_t wfull, wempty, rfull[2], rempty[2];
   __shared__ PairRec rec[2];
-  __shared__ float xk_c[SD], xv_c[SD];               // the consumers' copy of the token's k, v
   __shared__ __align__(16) float zpart[8][SD];       // read-out partials per row group
   __shared__ float prob[128 + 16];
   __shared__ float red[8][SD];
@@ -474,10 +475,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_stream_kernel(const __g
   }
   if (tid == 0) {
     // slot 0 always holds a key chunk and its token (4 chunks per pair, 4
-    // slots): the prep warps read it too
+    // slots): only the prep warps read it
     for (int i = 0; i < kStreamSlots; ++i) {
       s_mbar_init_n(&full[i], 1);
-      s_mbar_init_n(&empty[i], kConsumers / 32 + (i == 0 ? kPrep / 32 : 0));
+      s_mbar_init_n(&empty[i], i == 0 ? kPrep / 32 : kConsumers / 32);
     }
     s_mbar_init_n(&wfull, 1);
     s_mbar_init_n(&wempty, kConsumers / 32 + kPrep / 32);
@@ -526,7 +527,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_stream_kernel(const __g
           s_mbar_expect(bar, bytes + (kind == 0 ? (uint32_t)ntok * SD * 2 : 0));
           bulk_load(dst, src, bytes, bar);
           if (kind == 0) {
-            __nv_bfloat16 *tk = tokring + (size_t)sl * 4 * SD;
+            __nv_bfloat16 *tk = tokring;   // the key chunk is always slot 0
             const void *srcs[4] = {p.q, p.k, p.v, p.g};
 #pragma unroll
             for (int u = 0; u < 4; ++u)
@@ -563,6 +564,27 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_stream_kernel(const __g
         return;
       }
       PairRec &R = rec[k & 1];
+      // the new token's k, v for the consumers, and the window logits
+      // s q . k_j: thread = slot j (the slot being replaced takes the new key)
+      R.xk[pt] = __bfloat162float(tk[SD + pt]);
+      R.xv[pt] = __bfloat162float(tk[2 * SD + pt]);
+      if (pt < pi.n) {
+        const __nv_bfloat16 *kr = pt == pi.slot ? tk + SD : reinterpret_cast<const __nv_bfloat16 *>(ring) + (size_t)pt * SD;
+        float d0 = 0.f, d1 = 0.f;
+#pragma unroll 4
+        for (int c0 = 0; c0 < 16; ++c0) {
+          const int cc = (c0 + pt) & 15;   // spread a warp's reads over the banks
+          float kv[8], q8[8];
+          load8(kr + cc * 8, kv);
+          load8(tk + cc * 8, q8);
+#pragma unroll
+          for (int u = 0; u < 8; u += 2) {
+            d0 = fmaf(q8[u], kv[u], d0);
+            d1 = fmaf(q8[u + 1], kv[u + 1], d1);
+          }
+        }
+        R.lg[pt] = (d0 + d1) * p.scale;
+      }
       const __nv_bfloat16 gv = p.scalar_gate ? static_cast<const __nv_bfloat16 *>(p.g)[pi.bh] : tk[3 * SD + pt];
       R.gam[pt] = expf(log_decay(__bfloat162float(gv), p.inv_tau));
       // z = x W: thread = (map, feature); 4 partial sums over the 128 rows
@@ -641,8 +663,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_stream_kernel(const __g
       new_head = pi.h != cur_head;
       acc = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    bool ok = s_mbar_wait(&full[sl], (uint32_t)(c / kStreamSlots) & 1u);
-    if (kind == 0) ok &= s_mbar_wait(&rfull[kp & 1], (uint32_t)(kp >> 1) & 1u);
+    // the key chunk (slot 0) is read by the prep warps only: the consumers
+    // start a pair on its record
+    bool ok = kind == 0 ? s_mbar_wait(&rfull[kp & 1], (uint32_t)(kp >> 1) & 1u)
+                        : s_mbar_wait(&full[sl], (uint32_t)(c / kStreamSlots) & 1u);
     if (new_head) {
       ok &= s_mbar_wait(&wfull, (uint32_t)nh & 1u);   // meta values
       ++nh;
@@ -663,42 +687,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_stream_kernel(const __g
     const int n = pi.n, slot = pi.slot, h = pi.h, bh = pi.bh;
     const PairRec &R = rec[kp & 1];
     if (kind == 0) {
-      const __nv_bfloat16 *tk = tokring + (size_t)sl * 4 * SD;
-      if (tid < SD) {   // keep k and v: the token slot is refilled once everyone has read it
-        xk_c[tid] = __bfloat162float(tk[SD + tid]);
-        xv_c[tid] = __bfloat162float(tk[2 * SD + tid]);
-      }
-      // ---- window logits: two threads per slot (64 dimensions each); the
-      //      slot being replaced takes the new key
+      // softmax over the n window logits (from the prep warps) and the M
+      // meta logits, spread over the consumer warps: warp maxima, then one
+      // exp per slot and warp sums
       const int j = tid >> 1, half = tid & 1;
-      float lj = kNegBig;   // the logit of slot j (both threads of the slot hold it)
-      {
-        float d = 0.f;
-        if (j < n) {
-          const __nv_bfloat16 *kr = j == slot ? tk + SD + half * 64
-                                              : reinterpret_cast<const __nv_bfloat16 *>(chunk) + (size_t)j * SD + half * 64;
-          const __nv_bfloat16 *qr = tk + half * 64;
-#pragma unroll
-          for (int c0 = 0; c0 < 8; ++c0) {
-            const int cc = (c0 + j) & 7;   // spread a warp's reads over the banks
-            float kv[8], q8[8];
-            load8(kr + cc * 8, kv);
-            load8(qr + cc * 8, q8);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) d = fmaf(q8[u], kv[u], d);
-          }
-        }
-        d += __shfl_xor_sync(0xffffffffu, d, 1);
-        if (j < n) lj = d * p.scale;
-      }
-      // softmax over the n window logits and the M meta logits, spread over
-      // the consumer warps: warp maxima, then one exp per slot and warp sums
+      const float lj = j < n ? R.lg[j] : kNegBig;
       {
         const float wm = warp_max(lj);
         if (lane == 0) s_wmax[warp] = wm;
       }
-      __syncwarp();
-      if (lane == 0) s_mbar_arrive(&empty[sl]);   // the key window and the token are read
       consumers_sync();
       float mx = kNegBig;
 #pragma unroll
@@ -725,7 +722,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_stream_kernel(const __g
       }
     } else if (kind == 1 || kind == 2) {
       // ---- state rows (kind - 1) * 64 .. + 63: update, store, read out
-      const float4 v4 = make_float4(xv_c[cg * 4], xv_c[cg * 4 + 1], xv_c[cg * 4 + 2], xv_c[cg * 4 + 3]);
+      const float4 v4 = make_float4(R.xv[cg * 4], R.xv[cg * 4 + 1], R.xv[cg * 4 + 2], R.xv[cg * 4 + 3]);
       float *S = p.state + (size_t)bh * SD * SD;
       float4 sv[8];
 #pragma unroll
@@ -747,10 +744,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_stream_kernel(const __g
         acc.z = fmaf(qi, s.z, acc.z);
         acc.w = fmaf(qi, s.w, acc.w);
       }
-      if (kind == 2) {   // the record of this pair is no longer read
-        __syncwarp();
-        if (lane == 0) s_mbar_arrive(&rempty[kp & 1]);
-      }
     } else {
       // ---- o_swa = sum_j p_j v_j (+ meta values); the replaced slot takes
       //      the new value; then o = o_gla + alpha o_swa / l
@@ -761,7 +754,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_stream_kernel(const __g
         float vv[8];
         if (j == slot) {
 #pragma unroll
-          for (int u = 0; u < 8; ++u) vv[u] = xv_c[vg * 8 + u];
+          for (int u = 0; u < 8; ++u) vv[u] = R.xv[vg * 8 + u];
         } else {
           load8(reinterpret_cast<const __nv_bfloat16 *>(chunk) + (size_t)j * SD + vg * 8, vv);
         }
@@ -798,9 +791,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_stream_kernel(const __g
         // the new token enters the ring (both windows were read above); the
         // fp32 copies hold it exactly (bf16 -> fp32 -> bf16 is lossless)
         const size_t cw = ((size_t)bh * p.window + slot) * SD + tid;
-        static_cast<__nv_bfloat16 *>(p.k_cache)[cw] = __float2bfloat16_rn(xk_c[tid]);
-        static_cast<__nv_bfloat16 *>(p.v_cache)[cw] = __float2bfloat16_rn(xv_c[tid]);
+        static_cast<__nv_bfloat16 *>(p.k_cache)[cw] = __float2bfloat16_rn(R.xk[tid]);
+        static_cast<__nv_bfloat16 *>(p.v_cache)[cw] = __float2bfloat16_rn(R.xv[tid]);
       }
+      // the record of this pair is no longer read (the next pair's softmax
+      // starts on a consumer barrier, after every read above)
+      __syncwarp();
+      if (lane == 0) s_mbar_arrive(&rempty[kp & 1]);
     }
   }
   if (c_stop < nchunks && tid == 0) {
