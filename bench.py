@@ -180,7 +180,7 @@ class ClockSampler:
 # train_step workload (B=8, H=32, L=2048), from an ncu capture of the current
 # kernel build.
 MEASURED_TRAFFIC = {
-    "tc_gla_bwd_tile_kernel": 1.086746e9 + 1.021329e9,
+    "tc_gla_bwd_tile_kernel": 1.086681e9 + 1.020770e9,
 }
 
 
@@ -596,6 +596,9 @@ def run_decode(args, lz, dev, rank, world, peaks):
     from gated_linear_sliding_chunkwise_b200.synth import WORKLOADS, make_inputs
 
     w = WORKLOADS["decode_b64"]
+    if getattr(args, "decode_batch", None):   # a smaller batch for kernel profiles
+        import dataclasses
+        w = dataclasses.replace(w, B=args.decode_batch)
     inp = make_inputs(w, seed=w.seed + rank)
     x = {k: v.to(dev).contiguous() for k, v in inp.items()}
     o = torch.empty(w.B, w.H, w.d, dtype=x["q"].dtype, device=dev)
@@ -624,7 +627,7 @@ def run_decode(args, lz, dev, rank, world, peaks):
     gbs = world * step_bytes / (us * 1e-6) / 1e9
     return {"value": gbs, "unit": "GB/s", "frac_of_hbm": gbs / (world * peaks["hbm_gbs"]),
             "us_per_step": us, "steps": n, "bytes_per_step": step_bytes,
-            "workload": "decode_b64: B=64 H=32 d=128 window 128 M=4, pos 65536",
+            "workload": f"decode: B={w.B} H={w.H} d={w.d} window {w.window} M={w.M}, pos {w.decode_pos}",
             "launches_per_step": 2}
 
 
@@ -715,13 +718,21 @@ def main(argv=None):
     ap.add_argument("--no-fwd-long", action="store_true")
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the stage-1 step and scalar-gate timings")
-    ap.add_argument("--only", choices=["train", "fwd", "bwd"], default="train",
-                    help="fwd / bwd: time one entry point alone on --workload (profiling aid)")
+    ap.add_argument("--only", choices=["train", "fwd", "bwd", "decode"], default="train",
+                    help="fwd / bwd / decode: time one entry point alone (profiling aid)")
+    ap.add_argument("--decode-batch", type=int, default=None,
+                    help="with --only decode: batch size in place of the workload's 64")
     ap.add_argument("--workload", default="llama8b_layer_fwd")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         print("note: --warmup below 3 is not a valid measurement", file=sys.stderr)
     rank, world, local = dist_env()
+    if args.only == "decode":
+        from gated_linear_sliding_chunkwise_b200 import lizard as lz
+        dev = torch.device("cuda", local)
+        torch.cuda.set_device(dev)
+        print(json.dumps(run_decode(args, lz, dev, rank, 1, load_peaks())))
+        return
     if args.only in ("fwd", "bwd"):
         # one entry point alone on one workload (used for kernel profiles)
         from gated_linear_sliding_chunkwise_b200 import lizard as lz
