@@ -42,11 +42,21 @@ lizard_status check_fwd(const lizard_fwd_args *a) {
     if (!a->q || !a->k || !a->v || !a->o) return LIZARD_ERR_INVALID_ARG;
     if (a->branch != LIZARD_BRANCH_SWA_ONLY && !a->g) return LIZARD_ERR_INVALID_ARG;
   }
+  if (a->prefix_len < 0 || a->prefix_len > a->window) return LIZARD_ERR_INVALID_ARG;
+  if ((a->prefix_len > 0) != (a->k_prefix != nullptr) || (a->prefix_len > 0) != (a->v_prefix != nullptr))
+    return LIZARD_ERR_INVALID_ARG;
   const void *ptrs[] = {a->q, a->k, a->v, a->g, a->fmap_wq, a->fmap_wk, a->meta_k, a->meta_v,
-                        a->alpha, a->state_in, a->o, a->state_out, a->lse, a->workspace};
+                        a->alpha, a->state_in, a->o, a->state_out, a->lse, a->workspace,
+                        a->k_prefix, a->v_prefix};
   for (const void *p : ptrs)
     if (!ok_ptr(p)) return LIZARD_ERR_INVALID_ARG;
   return LIZARD_OK;
+}
+
+// Size queries ignore pointers: stand-ins for the prefix pointers that the
+// checks require when prefix_len > 0.
+void prefix_standin(lizard_fwd_args &a) {
+  a.k_prefix = a.v_prefix = a.prefix_len > 0 ? reinterpret_cast<const void *>(16) : nullptr;
 }
 
 bool gla_on(const lizard_fwd_args *a) { return a->branch != LIZARD_BRANCH_SWA_ONLY; }
@@ -270,7 +280,8 @@ void fwd_plan(const lizard_fwd_args *a, void *ws, cudaStream_t s, Plan &plan, co
     lz::TcFwdArgs t{a->q, a->k, a->v, a->g, a->fmap_wq, a->fmap_wk, a->meta_k, a->meta_v, a->alpha,
                     a->state_in, a->o, gla_on(a) ? a->state_out : nullptr, swa_on(a) ? a->lse : nullptr,
                     static_cast<uint32_t *>(ws), at<void>(ws, lay.phq), BH, a->H, a->L, a->M, a->window,
-                    a->branch, 1.f / a->gate_temp, scale_of(a), scalar_gate(a), target, dmse, loss};
+                    a->branch, 1.f / a->gate_temp, scale_of(a), scalar_gate(a), target, dmse, loss,
+                    a->k_prefix, a->v_prefix, a->prefix_len};
     if (gla_on(a)) plan.add("gate_prep_kernel", [=](cudaStream_t s) { return lz::launch_tc_fwd(t, 3, s); });
     if (lz::tc_fwd_stage_count(BH, a->L) > 1) {
       plan.add("tc_fwd_kernel(state pass)", [=](cudaStream_t s) { return lz::launch_tc_fwd(t, 0, s); });
@@ -290,7 +301,8 @@ void fwd_plan(const lizard_fwd_args *a, void *ws, cudaStream_t s, Plan &plan, co
     plan.add("gla_fwd_simt", [=](cudaStream_t s) { return lz::launch_gla_fwd_simt(ga, BH, D, bf16, s); });
   }
   lz::SwaMixArgs sa{a->q, a->k, a->v, a->meta_k, a->meta_v, a->alpha, o_gla, a->o,
-                    swa_on(a) ? a->lse : nullptr, a->H, a->L, a->window, a->M, a->branch, scale_of(a)};
+                    swa_on(a) ? a->lse : nullptr, a->H, a->L, a->window, a->M, a->branch, scale_of(a),
+                    a->k_prefix, a->v_prefix, a->prefix_len};
   plan.add("swa_mix_simt", [=](cudaStream_t s) { return lz::launch_swa_mix_simt(sa, BH, D, bf16, s); });
 }
 
@@ -426,6 +438,7 @@ size_t lizard_fwd_workspace_size(const lizard_fwd_args *args) {
     a.q = a.k = a.v = a.g = reinterpret_cast<const void *>(16);
     a.o = reinterpret_cast<void *>(16);
   }
+  prefix_standin(a);
   if (check_fwd(&a) != LIZARD_OK) return 0;
   return fwd_layout(&a).total;
 }
@@ -489,6 +502,7 @@ size_t lizard_bwd_workspace_size(const lizard_bwd_args *args) {
     a.q = a.k = a.v = a.g = reinterpret_cast<const void *>(16);
     a.o = reinterpret_cast<void *>(16);
   }
+  prefix_standin(a);
   if (check_fwd(&a) != LIZARD_OK) return 0;
   return bwd_layout(&a, args->impl).total;
 }
@@ -516,6 +530,7 @@ lizard_status lizard_attn_bwd(const lizard_bwd_args *b, lizard_stream_t stream) 
   const lizard_fwd_args *a = &b->fwd;
   if (b->impl == LIZARD_IMPL_TC && swa_on(a) && !bwd_swa_uses_tc(a, b->impl)) return LIZARD_ERR_UNSUPPORTED;
   if (b->impl == LIZARD_IMPL_TC && gla_on(a) && !bwd_gla_uses_tc(a, b->impl)) return LIZARD_ERR_UNSUPPORTED;
+  if (a->prefix_len != 0) return LIZARD_ERR_UNSUPPORTED;   // forward only
   const BwdLayout lay = bwd_layout(a, b->impl);
   if (!b->workspace || b->workspace_bytes < lay.total) return LIZARD_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -617,6 +632,7 @@ size_t lizard_stage1_workspace_size(const lizard_stage1_args *args) {
   f.workspace = nullptr;
   lizard_fwd_args chk = f;
   chk.o = reinterpret_cast<void *>(16);
+  prefix_standin(chk);
   if (check_fwd(&chk) != LIZARD_OK) return 0;
   if (keep_o) f.o = reinterpret_cast<void *>(16);
   return s1_layout(&a).total;
@@ -630,6 +646,7 @@ lizard_status lizard_stage1_step(const lizard_stage1_args *a, lizard_stream_t st
   if (f->impl == LIZARD_IMPL_TC && !fwd_uses_tc(f)) return LIZARD_ERR_UNSUPPORTED;
   if (b->impl == LIZARD_IMPL_TC && swa_on(f) && !bwd_swa_uses_tc(f, b->impl)) return LIZARD_ERR_UNSUPPORTED;
   if (b->impl == LIZARD_IMPL_TC && gla_on(f) && !bwd_gla_uses_tc(f, b->impl)) return LIZARD_ERR_UNSUPPORTED;
+  if (f->prefix_len != 0) return LIZARD_ERR_UNSUPPORTED;   // forward only
   const S1Layout lay = s1_layout(a);
   if (!b->workspace || b->workspace_bytes < lay.total) return LIZARD_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -746,5 +763,125 @@ const char *lizard_status_string(lizard_status s) {
 }
 
 const char *lizard_version(void) { return "0.1.0"; }
+
+}  // extern "C"
+
+// ------------------------------------------------- sequence parallelism ---
+namespace {
+
+// The segment summary runs on the tensor-core state pass for bf16, d = 128
+// with feature-map weights, else on the portable forward's kernels.
+bool seg_uses_tc(const lizard_fwd_args *a) {
+  const bool ok = a->dtype == LIZARD_BF16 && a->dk == 128 && a->dv == 128 && a->fmap_wk != nullptr;
+  return (a->impl == LIZARD_IMPL_AUTO || a->impl == LIZARD_IMPL_TC) && ok;
+}
+
+struct SegLayout {
+  size_t phq, phk, a, o_gla, tc, total;
+};
+SegLayout seg_layout(const lizard_fwd_args *a) {
+  const size_t N = (size_t)a->B * a->H * a->L;
+  SegLayout l{};
+  size_t off = kHeader;
+  if (seg_uses_tc(a)) {
+    l.tc = off;
+    off += up(lz::tc_segment_state_workspace_bytes(a->B * a->H, a->L));
+  } else {
+    const size_t nd = up(N * a->dk * sizeof(float));
+    l.phq = off; off += nd;
+    l.phk = off; off += nd;
+    l.a = off; off += nd;
+    l.o_gla = off; off += up(N * a->dv * sizeof(float));
+  }
+  l.total = off;
+  return l;
+}
+
+// The forward's checks on the arguments the summary reads: q and o are not
+// read (k and state_out stand in for them), nor are the meta tokens.
+lizard_status check_seg(const lizard_fwd_args *a, const float *log_decay) {
+  if (!a) return LIZARD_ERR_INVALID_ARG;
+  lizard_fwd_args f = *a;
+  f.q = a->k;
+  f.o = a->state_out;
+  f.lse = nullptr;
+  f.M = 0;
+  f.meta_k = f.meta_v = nullptr;
+  const lizard_status st = check_fwd(&f);
+  if (st != LIZARD_OK) return st;
+  if (a->branch == LIZARD_BRANCH_SWA_ONLY || a->state_in || a->prefix_len != 0) return LIZARD_ERR_INVALID_ARG;
+  if (!a->state_out || !log_decay || !aligned16(log_decay)) return LIZARD_ERR_INVALID_ARG;
+  return LIZARD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t lizard_segment_state_workspace_size(const lizard_fwd_args *args) {
+  if (!args) return 0;
+  lizard_fwd_args a = *args;
+  a.k = a.v = a.g = a.L > 0 ? reinterpret_cast<const void *>(16) : nullptr;
+  a.state_out = reinterpret_cast<float *>(16);
+  a.fmap_wq = a.fmap_wk = nullptr;
+  a.state_in = nullptr;
+  a.workspace = nullptr;
+  a.k_prefix = a.v_prefix = nullptr;
+  a.prefix_len = 0;
+  if (check_seg(&a, reinterpret_cast<const float *>(16)) != LIZARD_OK) return 0;
+  a.fmap_wk = args->fmap_wk ? reinterpret_cast<const float *>(16) : nullptr;   // selects the kernels
+  return seg_layout(&a).total;
+}
+
+lizard_status lizard_segment_state(const lizard_fwd_args *a, float *log_decay, lizard_stream_t stream) {
+  lizard_status st = check_seg(a, log_decay);
+  if (st != LIZARD_OK) return st;
+  if (a->impl == LIZARD_IMPL_TC && !seg_uses_tc(a)) return LIZARD_ERR_UNSUPPORTED;
+  const SegLayout lay = seg_layout(a);
+  if (!a->workspace || a->workspace_bytes < lay.total) return LIZARD_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int BH = a->B * a->H, D = a->dk;
+  if (a->L == 0) {
+    if (cudaMemsetAsync(a->state_out, 0, (size_t)BH * a->dk * a->dv * sizeof(float), s) != cudaSuccess ||
+        cudaMemsetAsync(log_decay, 0, (size_t)BH * a->dk * sizeof(float), s) != cudaSuccess)
+      return LIZARD_ERR_CUDA;
+    return LIZARD_OK;
+  }
+  void *ws = a->workspace;
+  if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), s) != cudaSuccess) return LIZARD_ERR_CUDA;
+  const float inv_tau = 1.f / a->gate_temp;
+  if (seg_uses_tc(a)) {
+    lz::TcFwdArgs t{a->k, a->k, a->v, a->g, nullptr, a->fmap_wk, nullptr, nullptr, nullptr, nullptr, nullptr,
+                    a->state_out, nullptr, static_cast<uint32_t *>(ws), nullptr, BH, a->H, a->L, 0, a->window,
+                    LIZARD_BRANCH_GLA_ONLY, inv_tau, scale_of(a), scalar_gate(a)};
+    return cuda_status(lz::launch_tc_segment_state(t, a->state_out, log_decay, at<void>(ws, lay.tc), s));
+  }
+  const bool bf16 = a->dtype == LIZARD_BF16;
+  // the portable forward's own kernels: the prep (phi of k stands in for the
+  // unused phi of q), the GLA pass from a zero start (its output is scratch),
+  // then the summed log-decay
+  lz::PrepArgs pa{a->k, a->k, a->g, a->fmap_wk, a->fmap_wk, at<float>(ws, lay.phq), at<float>(ws, lay.phk),
+                  at<float>(ws, lay.a), a->H, a->L, inv_tau, scalar_gate(a)};
+  cudaError_t e = lz::launch_prep(pa, BH, D, bf16, s);
+  if (e != cudaSuccess) return LIZARD_ERR_CUDA;
+  lz::GlaFwdArgs ga{at<float>(ws, lay.phq), at<float>(ws, lay.phk), at<float>(ws, lay.a), a->v, nullptr,
+                    at<float>(ws, lay.o_gla), a->state_out, a->L};
+  e = lz::launch_gla_fwd_simt(ga, BH, D, bf16, s);
+  if (e != cudaSuccess) return LIZARD_ERR_CUDA;
+  return cuda_status(lz::launch_decay_sum(at<float>(ws, lay.a), log_decay, BH, a->L, D, s));
+}
+
+lizard_status lizard_chain_states(const lizard_chain_args *a, lizard_stream_t stream) {
+  if (!a) return LIZARD_ERR_INVALID_ARG;
+  if (a->B <= 0 || a->H <= 0 || a->nseg < 0 || a->rank < 0 || a->rank > a->nseg) return LIZARD_ERR_INVALID_ARG;
+  if (a->dk != a->dv || (a->dk != 64 && a->dk != 128)) return LIZARD_ERR_UNSUPPORTED;
+  if (!a->state_out || (a->rank > 0 && (!a->seg_state || !a->seg_log_decay))) return LIZARD_ERR_INVALID_ARG;
+  const void *ptrs[] = {a->seg_state, a->seg_log_decay, a->state_in, a->state_out};
+  for (const void *p : ptrs)
+    if (!ok_ptr(p)) return LIZARD_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return cuda_status(lz::launch_chain_states(a->seg_state, a->seg_log_decay, a->state_in, a->state_out,
+                                             a->B * a->H, a->dk, a->rank, s));
+}
 
 }  // extern "C"

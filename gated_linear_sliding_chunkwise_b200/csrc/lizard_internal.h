@@ -33,6 +33,8 @@ struct SwaMixArgs {
   float *lse;
   int H, L, window, M, branch;
   float scale;
+  const void *k_prefix, *v_prefix;   // [B*H][P][D]: the P tokens before token 0 (P = 0: none)
+  int P;
 };
 
 struct DecodeArgs {
@@ -116,6 +118,10 @@ struct TcFwdArgs {
   const void *target;
   void *dmse;
   float *loss;
+  // Key/value prefix of the anchor window: [B*H][P][128] bf16, the P <= window
+  // tokens before token 0 (P = 0: none).
+  const void *k_prefix, *v_prefix;
+  int P;
 };
 
 struct TcSwaBwdArgs {
@@ -156,6 +162,18 @@ cudaError_t launch_prep(const PrepArgs &a, int BH, int D, bool bf16, cudaStream_
 cudaError_t launch_gla_fwd_simt(const GlaFwdArgs &a, int BH, int D, bool bf16, cudaStream_t s);
 cudaError_t launch_swa_mix_simt(const SwaMixArgs &a, int BH, int D, bool bf16, cudaStream_t s);
 bool tc_fwd_supported(int dk, int dv, int window, int M, bool bf16);
+// Sequence-parallel pieces.  Tensor-core segment summary: the state pass over
+// whole sequences from a zero start, writing U [BH][D][D] and the summed
+// log-decay R [BH][D]; its scratch (the gate factors) is
+// tc_segment_state_workspace_bytes() bytes.
+size_t tc_segment_state_workspace_bytes(int BH, int L);
+cudaError_t launch_tc_segment_state(const TcFwdArgs &a, float *U, float *R, void *scratch, cudaStream_t s);
+// R [BH][D] = sum over the L tokens of the log-decay a [BH][L][D] (portable).
+cudaError_t launch_decay_sum(const float *a, float *R, int BH, int L, int D, cudaStream_t s);
+// out = S_rank with S_0 = state_in (or 0), S_{j+1} = diag(exp R_j) S_j + U_j;
+// U [nseg][BH][D][D], R [nseg][BH][D].
+cudaError_t launch_chain_states(const float *U, const float *R, const float *state_in, float *out, int BH, int D,
+                                int rank, cudaStream_t s);
 size_t tc_fwd_workspace_bytes(int BH, int L);
 int tc_fwd_stage_count(int BH, int L);
 // stage 3: gate factors of every tile (first, when the GLA branch is on);

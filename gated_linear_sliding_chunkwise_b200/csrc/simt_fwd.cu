@@ -256,7 +256,8 @@ __global__ void __launch_bounds__(256) gla_fwd_simt(GlaFwdArgs p) {
 // ------------------------------------------------------- anchor + mix -----
 // Online softmax over blocks of 64 keys; the meta tokens form the first
 // block.  Thread (ty, tx) owns query rows ty*4..+3 and value columns
-// tx*VT..+VT-1 of the accumulator.
+// tx*VT..+VT-1 of the accumulator.  Keys j < 0 come from the prefix (row
+// P + j of k_prefix / v_prefix), when there is one.
 template <typename T, int D>
 __global__ void __launch_bounds__(256) swa_mix_simt(SwaMixArgs p) {
   constexpr int VT = D / 16;
@@ -276,6 +277,8 @@ __global__ void __launch_bounds__(256) swa_mix_simt(SwaMixArgs p) {
   const T* qs = static_cast<const T*>(p.q);
   const T* ks = static_cast<const T*>(p.k);
   const T* vs = static_cast<const T*>(p.v);
+  const T* kps = static_cast<const T*>(p.k_prefix);
+  const T* vps = static_cast<const T*>(p.v_prefix);
   T* os = static_cast<T*>(p.o);
   const size_t base = (size_t)bh * p.L * D;
   const float alpha = p.alpha ? p.alpha[h] : 1.f;
@@ -293,7 +296,7 @@ __global__ void __launch_bounds__(256) swa_mix_simt(SwaMixArgs p) {
       Q[e] = t < nq ? to_f32(qs[base + (size_t)t0 * D + e]) : 0.f;
     }
     if (tid < kSwaQ) { mrow[tid] = kNegBig; lrow[tid] = 0.f; }
-    const int kstart = max(0, t0 - p.window + 1);
+    const int kstart = max(-p.P, t0 - p.window + 1);
     const int kend = min(p.L, t0 + nq);   // exclusive
     const int nblk = (kend - kstart + kSwaK - 1) / kSwaK + (p.M > 0 ? 1 : 0);
     for (int blk = 0; blk < nblk; ++blk) {
@@ -310,9 +313,13 @@ __global__ void __launch_bounds__(256) swa_mix_simt(SwaMixArgs p) {
           }
         } else {
           const int j = ks0 + jj;
-          if (j < kend) {
+          if (j < kend && j >= 0) {
             kv = to_f32(ks[base + (size_t)j * D + i]);
             vv = to_f32(vs[base + (size_t)j * D + i]);
+          } else if (j < kend) {   // -P <= j < 0
+            const size_t pr = ((size_t)bh * p.P + (p.P + j)) * D + i;
+            kv = to_f32(kps[pr]);
+            vv = to_f32(vps[pr]);
           }
         }
         Kb[e] = kv;

@@ -82,6 +82,7 @@ constexpr uint32_t ST_TIMEOUT = 1u, ST_RANGE = 2u;
 
 struct Params {
   CUtensorMap mq, mk, mv, mg;
+  CUtensorMap mkp, mvp;     // key / value prefix [BH][P][D] (P > 0 only)
   const float *wq, *wk, *meta_k, *meta_v, *alpha, *state_in;
   __nv_bfloat16 *o;
   float *state_out, *lse;
@@ -96,6 +97,7 @@ struct Params {
   int H, L, M, window, branch;
   int mode;                 // 0: full forward, 1: state pass
   int nseg, tiles_per_seg;
+  int P;                    // prefix tokens before token 0 (0: none)
   float inv_tau, scale;
   // stage-1 loss (target null: off): dmse = mse_grad (o - target), *loss += mse_loss sum (o - target)^2
   const __nv_bfloat16 *target;
@@ -112,7 +114,12 @@ __device__ __forceinline__ void issue_tile_loads(const Params &p, unsigned char 
   for (int r = 0; r < 2; ++r) {
     if (full) {
       tma_load_3d(sm + R_XQ + r * REG, &p.mq, bar, 64 * r, t0, bh);
-      tma_load_3d(sm + R_KP + r * REG, &p.mk, bar, 64 * r, t0 - T, bh);
+      // keys of the previous tile; before token 0, the prefix (its rows
+      // before the first prefix token read as zero)
+      if (t0 == 0 && p.P > 0)
+        tma_load_3d(sm + R_KP + r * REG, &p.mkp, bar, 64 * r, p.P - T, bh);
+      else
+        tma_load_3d(sm + R_KP + r * REG, &p.mk, bar, 64 * r, t0 - T, bh);
       tma_load_3d(sm + R_G + r * REG, &p.mg, bar, 64 * r, t0, bh);
     }
     tma_load_3d(sm + R_XK + r * REG, &p.mk, bar, 64 * r, t0, bh);
@@ -323,14 +330,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       if (wg == 1 && gla) s_dec[row] = __expf(p.gate_r[((size_t)bh * ntiles_all + c) * D + row]);   // exp(r)
       float lsum = 1.f, mx = 0.f;                 // row normaliser and max (scaled logits)
       // Logit column cl holds key t0 - T + cl.  Row r sees columns
-      // [r + T + 1 - window, r + T] (and keys >= 0), so warp w4 only visits
-      // 32-column chunks w4 + (T + 1 - window) / 32 .. w4 + 4, and only the
-      // first and last of those need the band mask.
+      // [r + T + 1 - window, r + T] (and keys >= -P, P the prefix length),
+      // so warp w4 only visits 32-column chunks w4 + (T + 1 - window) / 32
+      // .. w4 + 4, and only the first and last of those need the band mask.
       const int w4 = warp & 3;
       const int cbase = t0 - T;
-      const int lo_c = max(tq - p.window + 1, 0) - cbase, hi_c = tq - cbase;
+      const int lo_c = max(tq - p.window + 1, -p.P) - cbase, hi_c = tq - cbase;
       int ch_lo = (32 * w4 + T + 1 - p.window) >> 5;
-      if (cbase < 0) ch_lo = max(ch_lo, 4);
+      if (cbase < 0) ch_lo = max(ch_lo, (T - p.P) >> 5);
       const int ch_hi = w4 + 4;
       const int in_lo = 32 * w4 + 31 + T + 1 - p.window;   // interior chunk: 32 ch >= in_lo
       const int ch_first = ch_lo + 1 - wg;                 // this group's first chunk
@@ -366,7 +373,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
           float v[32];
           tmem_ld32(tl + C_L + ch * 32, v);
           float m4[4] = {kNegBig, kNegBig, kNegBig, kNegBig};
-          if (32 * ch >= in_lo && 32 * ch + 31 <= 32 * w4 + T && 32 * ch + cbase >= 0) {
+          if (32 * ch >= in_lo && 32 * ch + 31 <= 32 * w4 + T && 32 * ch + cbase >= -p.P) {
 #pragma unroll
             for (int u = 0; u < 32; ++u) m4[u & 3] = fmaxf(m4[u & 3], v[u]);
           } else {
@@ -393,7 +400,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
           if (ch > ch_hi) continue;
           float v[32];
           tmem_ld32(tl + C_L + ch * 32, v);
-          const bool inner = 32 * ch >= in_lo && 32 * ch + 31 <= 32 * w4 + T && 32 * ch + cbase >= 0;
+          const bool inner = 32 * ch >= in_lo && 32 * ch + 31 <= 32 * w4 + T && 32 * ch + cbase >= -p.P;
 #pragma unroll
           for (int u = 0; u < 32; u += 2) {
             float e0 = __expf(fmaf(v[u], p.scale, -mx));
@@ -484,7 +491,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       mma_commit(&bar_m2);
       // V of the previous tile into the G region (E has been consumed)
       mbar_expect_tx(&bar_vp, swa ? TILE : 0);
-      if (swa) {
+      if (swa && t0 == 0 && p.P > 0) {
+        tma_load_3d(sm + R_G, &p.mvp, &bar_vp, 0, p.P - T, bh);
+        tma_load_3d(sm + R_G + REG, &p.mvp, &bar_vp, 64, p.P - T, bh);
+      } else if (swa) {
         tma_load_3d(sm + R_G, &p.mv, &bar_vp, 0, t0 - T, bh);
         tma_load_3d(sm + R_G + REG, &p.mv, &bar_vp, 64, t0 - T, bh);
       }
@@ -912,6 +922,47 @@ cudaError_t launch_tc_state_snapshots(const TcFwdArgs &a, void *snap, const floa
   return cudaGetLastError();
 }
 
+// Scratch of the segment summary: the fp32 decay factors E32 [BH][L][D], then
+// the tiles' log-decays r [BH][ntiles][D].
+size_t tc_segment_state_workspace_bytes(int BH, int L) {
+  return up256((size_t)BH * L * D * 4) + up256((size_t)BH * ((L + T - 1) / T) * D * 4);
+}
+
+// Segment summary for sequence parallelism: the state pass (mode 1) over
+// whole sequences from a zero start, U = its end state, R = the summed
+// log-decay of every key dimension.
+cudaError_t launch_tc_segment_state(const TcFwdArgs &a, float *U, float *R, void *scratch, cudaStream_t s) {
+  float *e32 = static_cast<float *>(scratch);
+  float *r = reinterpret_cast<float *>(static_cast<unsigned char *>(scratch) + up256((size_t)a.BH * a.L * D * 4));
+  cudaError_t e = launch_gate_prep(a.g, nullptr, e32, r, a.status, a.BH, a.L, a.inv_tau, a.scalar_gate != 0, s);
+  if (e != cudaSuccess) return e;
+  Params p;
+  memset(&p, 0, sizeof(p));
+  const uint64_t rows = (uint64_t)a.L;
+  // the state pass reads keys and values only (its query map is never loaded)
+  if (!make_map_bf16_3d(&p.mq, a.k, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mk, a.k, D, rows, a.BH, T) ||
+      !make_map_bf16_3d(&p.mv, a.v, D, rows, a.BH, T))
+    return cudaErrorInvalidValue;
+  p.gate_e32 = e32;
+  p.gate_r = r;
+  p.wk = a.wk;
+  p.status = a.status;
+  p.seg_state = U;
+  p.seg_decay = R;
+  p.H = a.H;
+  p.L = a.L;
+  p.window = a.window;
+  p.mode = 1;
+  p.nseg = 1;
+  p.tiles_per_seg = (a.L + T - 1) / T;
+  p.inv_tau = a.inv_tau;
+  p.scale = a.scale;
+  e = cudaFuncSetAttribute(tc_fwd_kernel<K_STATE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  tc_fwd_kernel<K_STATE><<<dim3(a.BH, 1), NTHREADS, SMEM_BYTES, s>>>(p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_tc_fwd(const TcFwdArgs &a, int stage, cudaStream_t s) {
   int nseg, tps;
   tc_fwd_segments(a.BH, a.L, &nseg, &tps);
@@ -955,6 +1006,12 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, int stage, cudaStream_t s) {
   p.state_out = a.state_out;
   p.lse = a.lse;
   p.status = a.status;
+  if (a.P > 0 && a.branch != 1) {
+    if (!make_map_bf16_3d(&p.mkp, a.k_prefix, D, (uint64_t)a.P, a.BH, T) ||
+        !make_map_bf16_3d(&p.mvp, a.v_prefix, D, (uint64_t)a.P, a.BH, T))
+      return cudaErrorInvalidValue;
+    p.P = a.P;
+  }
   p.seg_start = w.seg_start;
   p.seg_state = w.seg_state;
   p.seg_decay = w.seg_decay;

@@ -44,7 +44,8 @@ class FwdArgs(ctypes.Structure):
                 ("fmap_wq", _vp), ("fmap_wk", _vp), ("meta_k", _vp), ("meta_v", _vp),
                 ("alpha", _vp), ("state_in", _vp), ("o", _vp), ("state_out", _vp),
                 ("lse", _vp), ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t),
-                ("launch_events", ctypes.POINTER(_vp)), ("n_launch_events", _i32)]
+                ("launch_events", ctypes.POINTER(_vp)), ("n_launch_events", _i32),
+                ("k_prefix", _vp), ("v_prefix", _vp), ("prefix_len", _i32)]
 
 
 class BwdArgs(ctypes.Structure):
@@ -95,6 +96,17 @@ class CacheArgs(ctypes.Structure):
                 ("pos", _vp)]
 
 
+class ChainArgs(ctypes.Structure):
+    _fields_ = [("B", _i32), ("H", _i32), ("dk", _i32), ("dv", _i32), ("nseg", _i32), ("rank", _i32),
+                ("seg_state", _vp), ("seg_log_decay", _vp), ("state_in", _vp), ("state_out", _vp)]
+
+
+_lib.lizard_segment_state_workspace_size.argtypes = [ctypes.POINTER(FwdArgs)]
+_lib.lizard_segment_state_workspace_size.restype = ctypes.c_size_t
+_lib.lizard_segment_state.argtypes = [ctypes.POINTER(FwdArgs), _vp, _vp]
+_lib.lizard_segment_state.restype = ctypes.c_int
+_lib.lizard_chain_states.argtypes = [ctypes.POINTER(ChainArgs), _vp]
+_lib.lizard_chain_states.restype = ctypes.c_int
 _lib.lizard_prefill_cache.argtypes = [ctypes.POINTER(CacheArgs), _vp]
 _lib.lizard_prefill_cache.restype = ctypes.c_int
 _lib.lizard_decode_status.argtypes = []
@@ -229,15 +241,20 @@ def attn_fwd(q, k, v, g, *, window, chunk=64, gate_temp=16.0, softmax_scale=0.0,
              fmap_wq=None, fmap_wk=None, meta_k=None, meta_v=None, alpha=None,
              state_in=None, want_state=False, want_lse=False,
              branch=BRANCH_BOTH, impl=IMPL_AUTO, out=None, workspace=None, stream=None,
-             events=None, plan_only=False):
+             events=None, plan_only=False, k_prefix=None, v_prefix=None):
     """Forward of the hybrid layer (lizard_attn_fwd).  Tensors on one CUDA
     device, contiguous; returns a dict with o, state_out, lse.  `events`
     (torch.cuda.Event list) are recorded around each kernel; plan_only returns
-    the kernel names without launching."""
+    the kernel names without launching.  k_prefix, v_prefix [B, H, P, d]: the
+    P <= window tokens before token 0, seen by the anchor window."""
     a = _fwd_struct(q, k, v, g, window=window, chunk=chunk, gate_temp=gate_temp,
                     softmax_scale=softmax_scale, fmap_wq=fmap_wq, fmap_wk=fmap_wk,
                     meta_k=meta_k, meta_v=meta_v, alpha=alpha, state_in=state_in,
                     branch=branch, impl=impl)
+    if (k_prefix is None) != (v_prefix is None):
+        raise ValueError("k_prefix and v_prefix go together")
+    if k_prefix is not None:
+        a.k_prefix, a.v_prefix, a.prefix_len = _ptr(k_prefix), _ptr(v_prefix), k_prefix.shape[2]
     B, H, L, dk = q.shape
     dv = v.shape[-1]
     o = torch.empty(B, H, L, dv, dtype=q.dtype, device=q.device) if out is None else out
@@ -382,3 +399,34 @@ def prefill_cache(k, v, k_cache, v_cache, pos, stream=None):
     a.k, a.v = _ptr(k), _ptr(v)
     a.k_cache, a.v_cache, a.pos = _ptr(k_cache), _ptr(v_cache), _ptr(pos)
     _check(_lib.lizard_prefill_cache(ctypes.byref(a), _stream(stream)), "lizard_prefill_cache")
+
+
+# ------------------------------------------------- sequence parallelism ---
+def segment_state(k, v, g, *, window, chunk=64, gate_temp=16.0, fmap_wk=None, impl=IMPL_AUTO,
+                  workspace=None, stream=None):
+    """(U, R) of one segment (lizard_segment_state): U [B, H, dk, dv] fp32 the
+    GLA state after the segment's tokens from a zero start, R [B, H, dk] fp32
+    the summed log-decay; a start state S ends the segment as
+    diag(exp R) S + U."""
+    a = _fwd_struct(k, k, v, g, window=window, chunk=chunk, gate_temp=gate_temp,
+                    softmax_scale=0.0, fmap_wq=None, fmap_wk=fmap_wk, meta_k=None, meta_v=None,
+                    alpha=None, state_in=None, branch=BRANCH_GLA_ONLY, impl=impl)
+    a.q = None
+    B, H, _, dk = k.shape
+    U = torch.empty(B, H, dk, v.shape[-1], dtype=torch.float32, device=k.device)
+    R = torch.empty(B, H, dk, dtype=torch.float32, device=k.device)
+    a.state_out = _ptr(U)
+    ws = _workspace(int(_lib.lizard_segment_state_workspace_size(ctypes.byref(a))), k.device, workspace)
+    a.workspace, a.workspace_bytes = ws.data_ptr(), ws.numel() * ws.element_size()
+    _check(_lib.lizard_segment_state(ctypes.byref(a), _ptr(R), _stream(stream)), "lizard_segment_state")
+    return U, R, ws
+
+
+def chain_states(seg_state, seg_log_decay, rank, *, state_in=None, out=None, stream=None):
+    """Start state of segment `rank` (lizard_chain_states) from the gathered
+    summaries seg_state [nseg, B, H, dk, dv] and seg_log_decay [nseg, B, H, dk]."""
+    nseg, B, H, dk, dv = seg_state.shape
+    S = torch.empty(B, H, dk, dv, dtype=torch.float32, device=seg_state.device) if out is None else out
+    a = ChainArgs(B, H, dk, dv, nseg, rank, _ptr(seg_state), _ptr(seg_log_decay), _ptr(state_in), _ptr(S))
+    _check(_lib.lizard_chain_states(ctypes.byref(a), _stream(stream)), "lizard_chain_states")
+    return S

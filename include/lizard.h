@@ -121,6 +121,17 @@ enum {
  *              anchor branch runs)
  * gate_temp is tau (> 0); softmax_scale 0 means 1/sqrt(dk).
  * chunk is the GLA chunk length (64); it changes the schedule, not the result.
+ *
+ * Key/value prefix (a segment of a longer sequence, e.g. one rank's share
+ * under sequence parallelism): with prefix_len = P > 0, the P tokens just
+ * before token 0 are visible to the anchor window of the first tokens, as if
+ * the call's sequence continued them (the GLA branch takes that history
+ * through state_in instead).
+ *   k_prefix   [B, H, P, dk] dtype, v_prefix [B, H, P, dv] dtype: row P - 1
+ *              is token -1, row 0 token -P
+ *   0 <= P <= window; the pointers are NULL iff P == 0.  Forward only:
+ *   lizard_attn_bwd and lizard_stage1_step return LIZARD_ERR_UNSUPPORTED for
+ *   a nonzero prefix_len.
  */
 typedef struct {
   int32_t B, H, L, dk, dv, chunk, window, M;
@@ -146,6 +157,8 @@ typedef struct {
    * `stream`.  lizard_fwd_launch_plan() names the kernels in order. */
   void *const *launch_events;
   int32_t n_launch_events;
+  const void *k_prefix, *v_prefix;   /* see "Key/value prefix" above */
+  int32_t prefix_len;
 } lizard_fwd_args;
 
 /* Bytes of device workspace the forward needs for these arguments (pointer
@@ -190,6 +203,50 @@ typedef struct {
 
 size_t lizard_bwd_workspace_size(const lizard_bwd_args *args);
 lizard_status lizard_attn_bwd(const lizard_bwd_args *args, lizard_stream_t stream);
+
+/*
+ * Sequence parallelism: one long sequence split into consecutive segments,
+ * one per process (GPU).  The GLA recurrence is affine in its start state:
+ * over a segment with summed log-decay R (per key dimension) and end state U
+ * from a zero start, a start state S ends as diag(exp R) S + U (English
+ * summary, section 2.A "State Update", applied over a run of tokens).  So
+ * every segment computes (U, R) at once, the segments exchange them, and
+ * each chains the (U, R) of the segments before it into its own start state;
+ * then every segment runs lizard_attn_fwd with that state_in and the last
+ * `window` keys and values of the previous segment as its prefix.
+ *
+ * lizard_segment_state: (U, R) of the segment in args.
+ *   args       as for lizard_attn_fwd over the segment's L tokens; read are
+ *              the sizes, dtype, impl, gate, gate_temp, k, v, g, fmap_wk and
+ *              the workspace (q, o, meta tokens, alpha and lse are ignored;
+ *              state_in and the prefix must be NULL / 0; branch must not be
+ *              LIZARD_BRANCH_SWA_ONLY)
+ *   args->state_out  [B, H, dk, dv] fp32, written: U
+ *   log_decay  [B, H, dk] fp32, written: R = sum over the segment's tokens of
+ *              logsigmoid(g) / gate_temp
+ * Workspace: lizard_segment_state_workspace_size() bytes.  Errors as
+ * lizard_attn_fwd (the status word in the workspace included).
+ *
+ * lizard_chain_states: the start state of segment `rank` from the gathered
+ * (U, R) of every segment.
+ *   seg_state  [nseg, B, H, dk, dv] fp32, seg_log_decay [nseg, B, H, dk] fp32
+ *              (segment j's U and R at index j; only j < rank are read)
+ *   state_in   [B, H, dk, dv] fp32 state before segment 0, or NULL for zeros
+ *   state_out  [B, H, dk, dv] fp32, written:
+ *              S_0 = state_in, S_{j+1} = diag(exp R_j) S_j + U_j, out = S_rank
+ *   0 <= rank <= nseg.  No workspace.
+ */
+size_t lizard_segment_state_workspace_size(const lizard_fwd_args *args);
+lizard_status lizard_segment_state(const lizard_fwd_args *args, float *log_decay, lizard_stream_t stream);
+
+typedef struct {
+  int32_t B, H, dk, dv, nseg, rank;
+  const float *seg_state, *seg_log_decay;
+  const float *state_in;
+  float *state_out;
+} lizard_chain_args;
+
+lizard_status lizard_chain_states(const lizard_chain_args *args, lizard_stream_t stream);
 
 /*
  * One stage-1 training step (attention approximation: the layer learns to

@@ -19,6 +19,8 @@ from .lizard_ref import (  # noqa: F401
     lizard_decode_step,
     attention_mse,
     lizard_stage1_step,
+    gla_segment_state,
+    chain_states,
     BRANCH_BOTH,
     BRANCH_GLA_ONLY,
     BRANCH_SWA_ONLY,

@@ -51,6 +51,11 @@ What the pages fix, and the reading taken where they are silent:
   cache): one token updates S and writes (k, v) into slot pos mod window of a
   ring buffer; the softmax runs over the min(pos + 1, window) filled slots
   plus the meta tokens.
+* Sequence parallelism (a reading; the pages split no sequence): a segment
+  of a longer sequence receives the GLA history as its start state and the
+  keys and values just before it as a prefix of the anchor window.  The
+  start states chain segment summaries (U, R) through the affine form of
+  the state update (gla_segment_state, chain_states).
 
 Parity status: every public function here is pinned by the CPU tests against
 closed forms, library routines (causal softmax attention, autograd) and
@@ -229,7 +234,8 @@ def _window_probs(q, k, meta_k, t, window, scale):
     return j0, p[..., :n], p_meta, lse
 
 
-def swa_forward(q, k, v, meta_k, meta_v, window, scale=None):
+def swa_forward(q, k, v, meta_k, meta_v, window, scale=None,
+                k_prefix=None, v_prefix=None):
     """Sliding-window softmax attention with meta-token sinks.
 
     [EN] 2.A "Anchor Window Attention": the meta tokens sit in the softmax
@@ -237,18 +243,28 @@ def swa_forward(q, k, v, meta_k, meta_v, window, scale=None):
     q, k: [B,H,L,dk]; v: [B,H,L,dv]; meta_k: [H,M,dk] or None;
     meta_v: [H,M,dv] or None.  Returns (o_swa [B,H,L,dv], lse [B,H,L]),
     lse the natural-log normaliser over window and meta logits.
+
+    k_prefix, v_prefix [B,H,P,d] (a reading for a segment of a longer
+    sequence): the P keys and values just before token 0, which the window
+    of the first tokens reaches as if the sequence started P tokens earlier.
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
     meta_k, meta_v = _f64(meta_k), _f64(meta_v)
     B, H, L, dk = q.shape
     if scale is None:
         scale = 1.0 / np.sqrt(dk)
-    o = np.zeros(v.shape)
+    P = 0 if k_prefix is None else _f64(k_prefix).shape[2]
+    if P:
+        # the queries of the prefix positions are never used
+        q = np.concatenate([np.zeros((B, H, P, dk)), q], axis=2)
+        k = np.concatenate([_f64(k_prefix), k], axis=2)
+        v = np.concatenate([_f64(v_prefix), v], axis=2)
+    o = np.zeros((B, H, L, v.shape[-1]))
     lse = np.zeros((B, H, L))
     for t in range(L):
-        j0, p_win, p_meta, lse[:, :, t] = _window_probs(q, k, meta_k, t,
+        j0, p_win, p_meta, lse[:, :, t] = _window_probs(q, k, meta_k, P + t,
                                                         window, scale)
-        o[:, :, t] = np.einsum("bhj,bhjd->bhd", p_win, v[:, :, j0:t + 1])
+        o[:, :, t] = np.einsum("bhj,bhjd->bhd", p_win, v[:, :, j0:P + t + 1])
         if p_meta is not None and meta_v is not None:
             o[:, :, t] += np.einsum("bhm,hmd->bhd", p_meta, meta_v)
     return o, lse
@@ -316,12 +332,14 @@ def _defaults(q, alpha, scale, meta_k):
 def lizard_forward(q, k, v, g, *, window, tau=16.0, scale=None,
                    fmap_wq=None, fmap_wk=None, meta_k=None, meta_v=None,
                    alpha=None, state_in=None, branch=BRANCH_BOTH,
-                   gate=GATE_PER_DIM):
+                   gate=GATE_PER_DIM, k_prefix=None, v_prefix=None):
     """Hybrid layer forward: o = o_gla + alpha_h * o_swa.
 
     Mixing rule: [FR] 2.A last line, [EN] 2.A "Final Output".  `branch`
     keeps only one term of the sum (test hook): GLA_ONLY gives o_gla,
-    SWA_ONLY gives alpha_h * o_swa.
+    SWA_ONLY gives alpha_h * o_swa.  k_prefix / v_prefix: keys and values
+    before token 0 for the anchor window (see swa_forward); the GLA branch
+    takes the earlier history through state_in.
     Returns a dict with o, state_out (S_L, GLA run only), lse (anchor run
     only), o_gla and o_swa.
     """
@@ -338,10 +356,46 @@ def lizard_forward(q, k, v, g, *, window, tau=16.0, scale=None,
         out["o"] += o_gla
         out["o_gla"], out["state_out"] = o_gla, S_L
     if branch != BRANCH_GLA_ONLY:
-        o_swa, lse = swa_forward(q, k, v, meta_k, meta_v, window, scale)
+        o_swa, lse = swa_forward(q, k, v, meta_k, meta_v, window, scale,
+                                 k_prefix, v_prefix)
         out["o"] += alpha[None, :, None, None] * o_swa
         out["o_swa"], out["lse"] = o_swa, lse
     return out
+
+
+# ---------------------------------------------------------------------------
+# Sequence parallelism: segment summaries of the GLA recurrence
+# ---------------------------------------------------------------------------
+
+def gla_segment_state(k, v, g, *, tau=16.0, fmap_wk=None, gate=GATE_PER_DIM):
+    """Summary (U, R) of one segment of a sequence.
+
+    Reading of [EN] 2.A "State Update" over a run of tokens: the recurrence
+    S_t = diag(exp a_t) S_{t-1} + phi(k_t) v_t^T is affine in the state it
+    starts from, so over the segment a start state S ends as
+    diag(exp R) S + U, with R = sum_t a_t (per key dimension) and U the
+    state reached from S = 0.  U is that recurrence run from zero; R the
+    plain sum.  Returns (U [B,H,dk,dv], R [B,H,dk]).
+    """
+    k, v, g = _f64(k), _f64(v), _f64(g)
+    dk = k.shape[-1]
+    a = layer_log_decay(g, tau, gate, dk)
+    phk = feature_map(k, fmap_wk)
+    B, H, L, _ = k.shape
+    U = np.zeros((B, H, dk, v.shape[-1]))
+    for t in range(L):
+        U = np.exp(a[:, :, t])[..., None] * U + np.einsum("bhi,bhj->bhij", phk[:, :, t], v[:, :, t])
+    return U, a.sum(axis=2)
+
+
+def chain_states(seg_states, seg_log_decays, rank, state_in=None):
+    """Start state of segment `rank`: S_0 = state_in (or 0),
+    S_{j+1} = diag(exp R_j) S_j + U_j over the segments before it."""
+    U0 = _f64(seg_states[0])
+    S = np.zeros(U0.shape) if state_in is None else _f64(state_in).copy()
+    for j in range(rank):
+        S = np.exp(_f64(seg_log_decays[j]))[..., None] * S + _f64(seg_states[j])
+    return S
 
 
 def lizard_backward(q, k, v, g, dout, *, window, tau=16.0, scale=None,

@@ -49,7 +49,7 @@ def test_struct_layouts_match_c(lz, tmp_path):
     fields = {
         "lizard_fwd_args": lz.FwdArgs, "lizard_bwd_args": lz.BwdArgs,
         "lizard_decode_args": lz.DecodeArgs, "lizard_cache_args": lz.CacheArgs,
-        "lizard_stage1_args": lz.Stage1Args,
+        "lizard_stage1_args": lz.Stage1Args, "lizard_chain_args": lz.ChainArgs,
     }
     lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "lizard.h"',
              "int main(void) {"]
@@ -111,6 +111,11 @@ def _fwd(lz, **over):
     ({"meta_k": None}, 1),            # M > 0 needs meta keys
     ({"M": 0}, 1),                    # meta keys given but M == 0
     ({"q": 0x10004}, 1),              # not 16-byte aligned
+    ({"prefix_len": 17, "k_prefix": 0x10000, "v_prefix": 0x10000}, 1),   # prefix longer than the window
+    ({"prefix_len": -1}, 1),
+    ({"prefix_len": 4}, 1),           # prefix pointers missing
+    ({"k_prefix": 0x10000}, 1),       # prefix pointers without a length
+    ({"prefix_len": 4, "k_prefix": 0x10000, "v_prefix": 0x10008}, 1),   # misaligned prefix
 ])
 def test_forward_rejects_bad_arguments_on_host(lz, over, code):
     a = _fwd(lz, **over)
@@ -230,3 +235,78 @@ def test_stage1_launch_plan_fuses_the_loss_on_tensor_cores(lz):
         got = [names[i].decode() for i in range(n)]
         assert ("mse_kernel" in got) != fused, got
         assert "gate_grad_kernel" in got or "finish_bwd" in got, got
+
+
+# ------------------------------------------------- sequence parallelism ---
+def test_prefix_does_not_change_the_workspace_and_is_forward_only(lz):
+    a = _fwd(lz)
+    b = _fwd(lz, prefix_len=16, k_prefix=0x10000, v_prefix=0x10000)
+    assert lz.fwd_workspace_bytes(b) == lz.fwd_workspace_bytes(a) > 0
+    bw = lz.BwdArgs()
+    bw.fwd = b
+    fake = 0x10000
+    bw.dout = bw.dq = bw.dk = bw.dv = bw.dg = fake
+    need = lz.bwd_workspace_bytes(bw)
+    assert need > 0
+    bw.workspace, bw.workspace_bytes = 0x20000, need
+    assert lz.lib().lizard_attn_bwd(ctypes.byref(bw), None) == lz.ERR_UNSUPPORTED
+    s1 = lz.Stage1Args()
+    s1.bwd = bw
+    s1.target, s1.loss = fake, fake
+    s1.bwd.workspace_bytes = 1 << 40
+    assert lz.lib().lizard_stage1_step(ctypes.byref(s1), None) == lz.ERR_UNSUPPORTED
+
+
+def _seg(lz, **over):
+    a = _fwd(lz, M=0, meta_k=None)
+    a.q = a.o = None            # not read by the summary
+    a.state_out = 0x30000
+    for k_, v_ in over.items():
+        setattr(a, k_, v_)
+    return a
+
+
+@pytest.mark.parametrize("over,code", [
+    ({"state_out": None}, 1),
+    ({"branch": 2}, 1),                   # the summary is of the GLA branch
+    ({"state_in": 0x30000}, 1),           # summaries start from zero
+    ({"prefix_len": 4, "k_prefix": 0x10000, "v_prefix": 0x10000}, 1),
+    ({"k": None}, 1),
+    ({"dk": 96, "dv": 96}, 2),
+    ({"impl": 2}, 2),                     # tensor cores need bf16, d = 128 and W_k
+])
+def test_segment_state_rejects_bad_arguments_on_host(lz, over, code):
+    a = _seg(lz, **over)
+    a.workspace, a.workspace_bytes = 0x20000, 1 << 40
+    assert lz.lib().lizard_segment_state(ctypes.byref(a), 0x40000, None) == code
+
+
+def test_segment_state_needs_its_outputs_and_workspace(lz):
+    a = _seg(lz)
+    assert lz.lib().lizard_segment_state(ctypes.byref(a), None, None) == lz.ERR_INVALID_ARG
+    assert lz.lib().lizard_segment_state(ctypes.byref(a), 0x40004, None) == lz.ERR_INVALID_ARG
+    need = lz.lib().lizard_segment_state_workspace_size(ctypes.byref(a))
+    assert need > 0
+    a.workspace, a.workspace_bytes = 0x20000, need - 1
+    assert lz.lib().lizard_segment_state(ctypes.byref(a), 0x40000, None) == lz.ERR_WORKSPACE
+    # the tensor-core summary (bf16, d = 128, W_k) needs only the gate factors
+    tc = _seg(lz, dk=128, dv=128, fmap_wk=0x50000)
+    simt = _seg(lz, dk=128, dv=128)
+    assert 0 < lz.lib().lizard_segment_state_workspace_size(ctypes.byref(tc)) < \
+        lz.lib().lizard_segment_state_workspace_size(ctypes.byref(simt))
+
+
+@pytest.mark.parametrize("over,code", [
+    ({"rank": 3}, 1),                     # rank > nseg
+    ({"rank": -1}, 1),
+    ({"B": 0}, 1),
+    ({"seg_state": None}, 1),             # needed for rank > 0
+    ({"state_out": None}, 1),
+    ({"dk": 96, "dv": 96}, 2),
+    ({"seg_log_decay": 0x10004}, 1),
+])
+def test_chain_rejects_bad_arguments_on_host(lz, over, code):
+    a = lz.ChainArgs(1, 2, 64, 64, 2, 1, 0x10000, 0x20000, None, 0x30000)
+    for k_, v_ in over.items():
+        setattr(a, k_, v_)
+    assert lz.lib().lizard_chain_states(ctypes.byref(a), None) == code
