@@ -283,7 +283,7 @@ void fwd_plan(const lizard_fwd_args *a, void *ws, cudaStream_t s, Plan &plan, co
                     a->branch, 1.f / a->gate_temp, scale_of(a), scalar_gate(a), target, dmse, loss,
                     a->k_prefix, a->v_prefix, a->prefix_len};
     if (gla_on(a)) plan.add("gate_prep_kernel", [=](cudaStream_t s) { return lz::launch_tc_fwd(t, 3, s); });
-    if (lz::tc_fwd_stage_count(BH, a->L) > 1) {
+    if (gla_on(a) && lz::tc_fwd_stage_count(BH, a->L) > 1) {   // segment start states (GLA only)
       plan.add("tc_fwd_kernel(state pass)", [=](cudaStream_t s) { return lz::launch_tc_fwd(t, 0, s); });
       plan.add("seg_combine_kernel", [=](cudaStream_t s) { return lz::launch_tc_fwd(t, 1, s); });
     }

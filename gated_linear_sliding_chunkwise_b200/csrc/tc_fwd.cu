@@ -265,7 +265,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
   // group writes one half of the columns
   {
     const float *src = nullptr;
-    if (full && p.nseg > 1) src = p.seg_start + (((size_t)bh * p.nseg + seg) * D + row) * D;
+    if (full && p.nseg > 1 && gla) src = p.seg_start + (((size_t)bh * p.nseg + seg) * D + row) * D;
     else if (full && p.state_in) src = p.state_in + ((size_t)bh * D + row) * D;
     else if (p.snap && p.state_in) src = p.state_in + ((size_t)bh * D + row) * D;
 #pragma unroll
@@ -305,6 +305,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
     if (LOSS && full && qvalid)               // the epilogue's target half-row, toward L2 early
       asm volatile("prefetch.global.L2 [%0];" ::"l"(p.target + ((size_t)bh * p.L + tq) * D + 64 * wg));
 
+    // the tile's log-decay r of dimension `row` (group 1 in the full pass,
+    // group 0 in the state pass), in flight during the wait
+    const float r_dim = (gla && wg == (full ? 1 : 0)) ? p.gate_r[((size_t)bh * ntiles_all + c) * D + row] : 0.f;
+
     // ---------------------------------------------------------- MMA 1 ---
     bool ok = mbar_wait(&bar_tma, par, err, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) { s_fail = 1; break; }
@@ -327,7 +331,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       //      the meta logits), then one half of phi_q, phi_k per group
       ok &= mbar_wait(&bar_m1, par, err, ST_TIMEOUT);
       tc_fence_after();
-      if (wg == 1 && gla) s_dec[row] = __expf(p.gate_r[((size_t)bh * ntiles_all + c) * D + row]);   // exp(r)
+      if (wg == 1 && gla) s_dec[row] = __expf(r_dim);   // exp(r)
       float lsum = 1.f, mx = 0.f;                 // row normaliser and max (scaled logits)
       // Logit column cl holds key t0 - T + cl.  Row r sees columns
       // [r + T + 1 - window, r + T] (and keys >= -P, P the prefix length),
@@ -468,9 +472,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         }
         if (c + 1 < cend) e_load(c + 1);
         if (wg == 0) {   // thread row = key dimension: the tile's decay
-          const float r = p.gate_r[((size_t)bh * ntiles_all + c) * D + row];
-          s_dec[row] = __expf(r);
-          tot_decay += r;
+          s_dec[row] = __expf(r_dim);
+          tot_decay += r_dim;
         }
       }
       tmem_st_wait();
@@ -972,6 +975,7 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, int stage, cudaStream_t s) {
     if (!gla) return cudaSuccess;
     return launch_gate_prep(a.g, w.e16, w.e32, w.r, a.status, a.BH, a.L, a.inv_tau, a.scalar_gate != 0, s);
   }
+  if (nseg > 1 && (stage == 0 || stage == 1) && !gla) return cudaSuccess;   // no state to carry
   if (nseg > 1 && stage == 1) {
     seg_combine_kernel<<<dim3(a.BH, D * D / 256), 256, 0, s>>>(w.seg_state, w.seg_decay, a.state_in, w.seg_start,
                                                                nseg);

@@ -160,6 +160,8 @@ __global__ void __launch_bounds__(NT_DS, 1) tc_gla_dstates_kernel(const __grid_c
   for (int c = ntiles - 1; c >= 0; --c) {
     const uint32_t par = (ntiles - 1 - c) & 1;
     const int t0 = c * T;
+    // the tile's log-decay r of this row's dimension, in flight during the wait
+    const float r_dim = wg == 0 ? p.gate_r[((size_t)bh * ntiles + c) * D + row] : 0.f;
     bool ok = mbar_wait(&bar_tma, par, p.status, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) { fail = true; break; }
     if (tid == 0) {
@@ -196,7 +198,7 @@ __global__ void __launch_bounds__(NT_DS, 1) tc_gla_dstates_kernel(const __grid_c
     // E in fp32 (dimensions 64 wg ..) into TMEM; the tile's decay exp(r)
     e_half_store(epre, tl + C_E + 64 * wg);
     if (c > 0) e_load(c - 1);
-    if (wg == 0) s_dec[row] = __expf(p.gate_r[((size_t)bh * ntiles + c) * D + row]);
+    if (wg == 0) s_dec[row] = __expf(r_dim);
     tmem_st_wait();
     ok = mbar_wait(&bar_m1, par, p.status, ST_TIMEOUT);
     tc_fence_after();
@@ -276,8 +278,12 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
   __shared__ uint64_t bars[8];
   __shared__ uint32_t s_tmem;
   // Per row: dO . S'[0], V . dS[0], sum_i Kt[i] -- the rank-one parts of GQ,
-  // GK and dv that the copies (S' - 1 S'[0], dS - 1 dS[0]) leave out
-  __shared__ float s_r1[3][T];
+  // GK and dv that the copies (S' - 1 S'[0], dS - 1 dS[0]) leave out.  Before
+  // the sums are formed, and again once they are read, the same storage holds
+  // the row-0 vectors S'[0] (floats 0..127) and dS[0] (128..255), which every
+  // row reads.
+  __shared__ __align__(16) float s_r1[3][T];
+  float *s_row0 = &s_r1[0][0];
   // X_q -> Qt (hi), X_k -> Kt (hi), V, dO, Qt (lo), [W_q | W_k] -> S' -> dS, Kt (lo)
   constexpr uint32_t R_XQ = 0, R_XK = TILE, R_V = 2 * TILE, R_O = 3 * TILE, R_QL = 4 * TILE, R_W = 5 * TILE,
                      R_KL = 6 * TILE;
@@ -315,6 +321,10 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
   const uint32_t id_mn = idesc_bf16(128, 128, 0, 1);
   const uint32_t id_z = idesc_bf16(128, 64, 0, 1);
   float r1[3];   // this half's dO . S'[0], V . dS[0], sum Kt
+  if (tid < 64) {   // the row-0 vectors, while the tile arrives
+    const float *src = tid < 32 ? p.sp_r0 + (size_t)snap_idx * D + 4 * tid : p.ds_r0 + (size_t)snap_idx * D + 4 * (tid - 32);
+    *reinterpret_cast<float4 *>(s_row0 + 4 * tid) = __ldg(reinterpret_cast<const float4 *>(src));
+  }
   float4 epre[16];   // this row's fp32 decay factors (its dimension half), loaded while the tile arrives
   e_half_load(p.e32, ((size_t)bh * p.L + (valid ? tq : 0)) * D, valid, wg, epre);
   bool ok = mbar_wait(&bars[0], 0, p.status, ST_TIMEOUT);
@@ -365,16 +375,16 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
   tmem_st_wait();
   r1[0] = r1[1] = r1[2] = 0.f;
   {
-    const float *ms = p.sp_r0 + (size_t)snap_idx * D + 64 * wg, *md = p.ds_r0 + (size_t)snap_idx * D + 64 * wg;
+    const float *ms = s_row0 + 64 * wg, *md = s_row0 + D + 64 * wg;
 #pragma unroll 2
     for (int ch = 0; ch < 8; ++ch) {
       float o8[8], v8[8];
       unpack8(*chunk_ptr(sm, R_O, row, 8 * wg + ch), o8);
       unpack8(*chunk_ptr(sm, R_V, row, 8 * wg + ch), v8);
-      const float4 a0 = __ldg(reinterpret_cast<const float4 *>(ms + 8 * ch)),
-                   a1 = __ldg(reinterpret_cast<const float4 *>(ms + 8 * ch + 4));
-      const float4 b0 = __ldg(reinterpret_cast<const float4 *>(md + 8 * ch)),
-                   b1 = __ldg(reinterpret_cast<const float4 *>(md + 8 * ch + 4));
+      const float4 a0 = *reinterpret_cast<const float4 *>(ms + 8 * ch),
+                   a1 = *reinterpret_cast<const float4 *>(ms + 8 * ch + 4);
+      const float4 b0 = *reinterpret_cast<const float4 *>(md + 8 * ch),
+                   b1 = *reinterpret_cast<const float4 *>(md + 8 * ch + 4);
       r1[0] += o8[0] * a0.x + o8[1] * a0.y + o8[2] * a0.z + o8[3] * a0.w + o8[4] * a1.x + o8[5] * a1.y +
                o8[6] * a1.z + o8[7] * a1.w;
       r1[1] += v8[0] * b0.x + v8[1] * b0.y + v8[2] * b0.z + v8[3] * b0.w + v8[4] * b1.x + v8[5] * b1.y +
@@ -405,15 +415,12 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
       }
     }
   }
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();   // every row is done with the row-0 vectors: s_r1 takes the sums
   if (wg == 1)
 #pragma unroll
     for (int k = 0; k < 3; ++k) s_r1[k][row] = r1[k];
-  fence_proxy_async();
-  tc_fence_before();
-  __syncthreads();
-  if (wg == 0)   // the two halves' sums meet; read after the next barrier
-#pragma unroll
-    for (int k = 0; k < 3; ++k) s_r1[k][row] += r1[k];
   // 3. A^T = Kt Qt^T (rows = keys)
   if (tid == 0) {
     tc_fence_after();
@@ -422,6 +429,9 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
   }
   ok = mbar_wait(&bars[3], 0, p.status, ST_TIMEOUT);
   if (__syncthreads_or(!ok)) goto done;
+  if (wg == 0)   // the two halves' sums meet; read after the next barrier
+#pragma unroll
+    for (int k = 0; k < 3; ++k) s_r1[k][row] += r1[k];
   tc_fence_after();
   //    A^T^ = A^T masked to queries j >= key row, packed bf16 into TMEM over
   //    the spent E columns, 64 query columns per group
@@ -482,6 +492,9 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
 #pragma unroll
     for (int u = 0; u < 16; ++u)
       e4[u] = valid ? *reinterpret_cast<const float4 *>(er + 4 * u) : make_float4(1.f, 1.f, 1.f, 1.f);
+    // dS[0] for the dv pass, back into shared memory once the sums are read
+    const float4 ds0 = tid < 32 ? __ldg(reinterpret_cast<const float4 *>(p.ds_r0 + (size_t)snap_idx * D + 4 * tid))
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
     ok = mbar_wait(&bars[7], 0, p.status, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) goto done;
     tc_fence_after();
@@ -521,6 +534,7 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
       for (int bx = 0; bx < 4; ++bx) tma_store_3d(&p.mdb, st0 + bx * 16384, 32 * bx, t0, bh);
       bulk_commit();
     }
+    if (tid < 32) *reinterpret_cast<float4 *>(s_row0 + D + 4 * tid) = ds0;   // read after two barriers
 #pragma unroll
     for (int k4 = 0; k4 < 4; ++k4) {
       const int c16 = 4 * wg + k4;
@@ -553,13 +567,13 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
       bulk_wait_read_but_last();   // the dB tile has been read out of V | dO
     }
     __syncthreads();
-    const float *md = p.ds_r0 + (size_t)snap_idx * D;
+    const float *md = s_row0 + D;
     for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
       float dv[32];
       tmem_ld32(tl + C_DV + ch * 32, dv);
 #pragma unroll
       for (int u = 0; u < 32; u += 4) {   // + (sum_i Kt[i]) dS[0]
-        const float4 m4 = __ldg(reinterpret_cast<const float4 *>(md + ch * 32 + u));
+        const float4 m4 = *reinterpret_cast<const float4 *>(md + ch * 32 + u);
         *f32_stage_ptr(st0, row, ch * 32 + u) = make_float4(fmaf(kap, m4.x, dv[u]), fmaf(kap, m4.y, dv[u + 1]),
                                                             fmaf(kap, m4.z, dv[u + 2]), fmaf(kap, m4.w, dv[u + 3]));
       }

@@ -91,10 +91,11 @@ def test_forward_sweep(lz, impl, dtype, d, L, window, M, with_mv, with_state, ra
 
 
 @pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("L", [150, 1100])          # 1100: few sequences, segmented forward
 @pytest.mark.parametrize("branch", [ref.BRANCH_GLA_ONLY, ref.BRANCH_SWA_ONLY])
-def test_branch_hooks(lz, impl, branch):
+def test_branch_hooks(lz, impl, branch, L):
     dtype, d = ("fp32", 64) if impl == "simt" else ("bf16", 128)
-    w = Workload("branch", B=1, H=2, L=150, d=d, window=20, M=4, dtype=dtype, seed=3)
+    w = Workload("branch", B=1, H=2, L=L, d=d, window=20, M=4, dtype=dtype, seed=3)
     inp = make_inputs(w)
     inp["alpha"] = random_alpha(2, seed=9)
     got = _run(lz, to_device(inp), w, _impl(lz, impl), branch=branch)
