@@ -305,10 +305,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
     if (LOSS && full && qvalid)               // the epilogue's target half-row, toward L2 early
       asm volatile("prefetch.global.L2 [%0];" ::"l"(p.target + ((size_t)bh * p.L + tq) * D + 64 * wg));
 
-    // the tile's log-decay r of dimension `row` (group 1 in the full pass,
-    // group 0 in the state pass), in flight during the wait
-    const float r_dim = (gla && wg == (full ? 1 : 0)) ? p.gate_r[((size_t)bh * ntiles_all + c) * D + row] : 0.f;
-
     // ---------------------------------------------------------- MMA 1 ---
     bool ok = mbar_wait(&bar_tma, par, err, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) { s_fail = 1; break; }
@@ -331,7 +327,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       //      the meta logits), then one half of phi_q, phi_k per group
       ok &= mbar_wait(&bar_m1, par, err, ST_TIMEOUT);
       tc_fence_after();
-      if (wg == 1 && gla) s_dec[row] = __expf(r_dim);   // exp(r)
+      if (wg == 1 && gla) s_dec[row] = __expf(p.gate_r[((size_t)bh * ntiles_all + c) * D + row]);   // exp(r)
       float lsum = 1.f, mx = 0.f;                 // row normaliser and max (scaled logits)
       // Logit column cl holds key t0 - T + cl.  Row r sees columns
       // [r + T + 1 - window, r + T] (and keys >= -P, P the prefix length),
@@ -472,8 +468,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         }
         if (c + 1 < cend) e_load(c + 1);
         if (wg == 0) {   // thread row = key dimension: the tile's decay
-          s_dec[row] = __expf(r_dim);
-          tot_decay += r_dim;
+          const float r = p.gate_r[((size_t)bh * ntiles_all + c) * D + row];
+          s_dec[row] = __expf(r);
+          tot_decay += r;
         }
       }
       tmem_st_wait();

@@ -160,8 +160,6 @@ __global__ void __launch_bounds__(NT_DS, 1) tc_gla_dstates_kernel(const __grid_c
   for (int c = ntiles - 1; c >= 0; --c) {
     const uint32_t par = (ntiles - 1 - c) & 1;
     const int t0 = c * T;
-    // the tile's log-decay r of this row's dimension, in flight during the wait
-    const float r_dim = wg == 0 ? p.gate_r[((size_t)bh * ntiles + c) * D + row] : 0.f;
     bool ok = mbar_wait(&bar_tma, par, p.status, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) { fail = true; break; }
     if (tid == 0) {
@@ -198,7 +196,7 @@ __global__ void __launch_bounds__(NT_DS, 1) tc_gla_dstates_kernel(const __grid_c
     // E in fp32 (dimensions 64 wg ..) into TMEM; the tile's decay exp(r)
     e_half_store(epre, tl + C_E + 64 * wg);
     if (c > 0) e_load(c - 1);
-    if (wg == 0) s_dec[row] = __expf(r_dim);
+    if (wg == 0) s_dec[row] = __expf(p.gate_r[((size_t)bh * ntiles + c) * D + row]);
     tmem_st_wait();
     ok = mbar_wait(&bar_m1, par, p.status, ST_TIMEOUT);
     tc_fence_after();
