@@ -26,8 +26,9 @@
 //
 // tc_gla_dstates_kernel  reverse pass per sequence: dS of every tile (bf16
 //                        copies) and the gradient of the initial state.
-// tc_gla_bwd_tile_kernel one CTA per (tile, sequence): the formulas above,
-//                        given the S' and dS copies.
+// tc_gla_bwd_tile_kernel the formulas above per 128-token tile, given the
+//                        S' and dS copies; one persistent CTA per SM walks a
+//                        contiguous run of (sequence, tile) items.
 // gate_grad_kernel       reverse cumulative sum of dB -> gate-logit gradient.
 #include "common.cuh"
 #include "lizard_internal.h"
@@ -66,7 +67,7 @@ struct TileParams {
   const float *sp_r0, *ds_r0;  // [BH*ntiles][D] row 0 of S' and of dS (the copies hold the rest)
   float *dphq, *dphk, *dB, *dv;
   uint32_t *status;
-  int H, L, ntiles;
+  int H, L, ntiles, BH;
   float inv_tau;
 };
 
@@ -159,7 +160,6 @@ __global__ void __launch_bounds__(NT_DS, 1) tc_gla_dstates_kernel(const __grid_c
   bool fail = false;
   for (int c = ntiles - 1; c >= 0; --c) {
     const uint32_t par = (ntiles - 1 - c) & 1;
-    const int t0 = c * T;
     bool ok = mbar_wait(&bar_tma, par, p.status, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) { fail = true; break; }
     if (tid == 0) {
@@ -282,8 +282,8 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
   // row reads.
   __shared__ __align__(16) float s_r1[3][T];
   float *s_row0 = &s_r1[0][0];
-  // X_q -> Qt (hi), X_k -> Kt (hi), V, dO, Qt (lo), [W_q | W_k] -> S' -> dS, Kt (lo)
-  constexpr uint32_t R_XQ = 0, R_XK = TILE, R_V = 2 * TILE, R_O = 3 * TILE, R_QL = 4 * TILE, R_W = 5 * TILE,
+  // X_q -> Qt (hi), X_k -> Kt (hi), V, dO, [W_q | W_k] -> S' -> dS, Qt (lo), Kt (lo)
+  constexpr uint32_t R_XQ = 0, R_XK = TILE, R_V = 2 * TILE, R_O = 3 * TILE, R_W = 4 * TILE, R_QL = 5 * TILE,
                      R_KL = 6 * TILE;
   // TMEM, in order of use:
   //   dA [128,256) dA^T [256,384) Zq [384,448) Zk [448,512)
@@ -293,40 +293,73 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
                      C_AT = 256, C_GQ = 256, C_ZQ = 384, C_ZK = 448, C_GK = 384;
   const int tid = threadIdx.x, warp = tid >> 5, wg = tid >> 7, row = tid & 127;
   const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-  const int c = blockIdx.x, bh = blockIdx.y, h = bh % p.H, t0 = c * T, tq = t0 + row;
-  const bool valid = tq < p.L;
   const uint32_t sbase = smem_u32(sm);
+  // Persistent: CTA b walks the contiguous run [w0, w1) of (sequence, tile)
+  // items, item w = tile w % ntiles of sequence w / ntiles.  The next item's
+  // inputs go out as this item frees their places: the weights once the last
+  // products are done, the decay factors during the dv pass, X_q and X_k once
+  // the dphi stores have read their staging, V and dO after the dv store.
+  const int nwork = p.ntiles * p.BH;
+  const int w0 = (int)((long long)blockIdx.x * nwork / gridDim.x);
+  const int w1 = (int)((long long)(blockIdx.x + 1) * nwork / gridDim.x);
+  auto item_loads = [&](int w, int part) {   // part 0: weights (arms the barrier), 1: X_q, X_k, 2: V, dO
+    const int lbh = w / p.ntiles, lt0 = (w % p.ntiles) * T;
+    if (part == 0) mbar_expect_tx(&bars[0], 5 * TILE);
+    for (int r = 0; r < 2; ++r) {
+      if (part == 0) tma_load_3d(sm + R_W + r * REG, &p.mw, &bars[0], 0, 0, 2 * (lbh % p.H) + r);
+      if (part == 1) {
+        tma_load_3d(sm + R_XQ + r * REG, &p.mq, &bars[0], 64 * r, lt0, lbh);
+        tma_load_3d(sm + R_XK + r * REG, &p.mk, &bars[0], 64 * r, lt0, lbh);
+      }
+      if (part == 2) {
+        tma_load_3d(sm + R_V + r * REG, &p.mv, &bars[0], 64 * r, lt0, lbh);
+        tma_load_3d(sm + R_O + r * REG, &p.mo, &bars[0], 64 * r, lt0, lbh);
+      }
+    }
+  };
+  auto e_load = [&](int w, float4 *e) {   // this row's fp32 decay factors (its dimension half) of item w
+    const int lbh = w / p.ntiles, ltq = (w % p.ntiles) * T + row;
+    e_half_load(p.e32, ((size_t)lbh * p.L + (ltq < p.L ? ltq : 0)) * D, ltq < p.L, wg, e);
+  };
   if (warp == 0) { tmem_alloc(&s_tmem, 512); tmem_relinquish(); }
   if (tid == 0) {
     for (int i = 0; i < 8; ++i) mbar_init(&bars[i], 1);
     fence_barrier_init();
-    // the tile and this head's bf16 feature-map weights (converted once per call)
-    mbar_expect_tx(&bars[0], 5 * TILE);
-    for (int r = 0; r < 2; ++r) {
-      tma_load_3d(sm + R_XQ + r * REG, &p.mq, &bars[0], 64 * r, t0, bh);
-      tma_load_3d(sm + R_XK + r * REG, &p.mk, &bars[0], 64 * r, t0, bh);
-      tma_load_3d(sm + R_V + r * REG, &p.mv, &bars[0], 64 * r, t0, bh);
-      tma_load_3d(sm + R_O + r * REG, &p.mo, &bars[0], 64 * r, t0, bh);
-      tma_load_3d(sm + R_W + r * REG, &p.mw, &bars[0], 0, 0, 2 * h + r);
+    if (w0 < w1) {
+      item_loads(w0, 0);
+      item_loads(w0, 1);
+      item_loads(w0, 2);
     }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = s_tmem, tl = tb + lane_off;
-  const int snap_idx = bh * p.ntiles + c;
   const uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
   const uint32_t id_mn = idesc_bf16(128, 128, 0, 1);
   const uint32_t id_z = idesc_bf16(128, 64, 0, 1);
+  float4 epre[16];   // this row's decay factors of the item to come
+  if (w0 < w1) e_load(w0, epre);
+  // copies in flight when a wait gives up (tid 0's view): the parity of an
+  // armed phase of bars[0], and whether the S' / dS loads of this item are out
+  int pend0 = w0 < w1 ? 0 : -1;
+  bool pend_sp = false, pend_ds = false;
+  bool ok = true;
+  uint32_t par = 0;
+  for (int w = w0, itn = 0; w < w1; ++w, ++itn) {
+  par = (uint32_t)itn & 1u;
+  const int bh = w / p.ntiles, c = w % p.ntiles, t0 = c * T, tq = t0 + row;
+  const bool valid = tq < p.L;
+  const int snap_idx = w;   // == bh * ntiles + c
+  const bool more = w + 1 < w1;
   float r1[3];   // this half's dO . S'[0], V . dS[0], sum Kt
   if (tid < 64) {   // the row-0 vectors, while the tile arrives
     const float *src = tid < 32 ? p.sp_r0 + (size_t)snap_idx * D + 4 * tid : p.ds_r0 + (size_t)snap_idx * D + 4 * (tid - 32);
     *reinterpret_cast<float4 *>(s_row0 + 4 * tid) = __ldg(reinterpret_cast<const float4 *>(src));
   }
-  float4 epre[16];   // this row's fp32 decay factors (its dimension half), loaded while the tile arrives
-  e_half_load(p.e32, ((size_t)bh * p.L + (valid ? tq : 0)) * D, valid, wg, epre);
-  bool ok = mbar_wait(&bars[0], 0, p.status, ST_TIMEOUT);
-  if (__syncthreads_or(!ok)) goto done;
+  ok = mbar_wait(&bars[0], par, p.status, ST_TIMEOUT);
+  if (__syncthreads_or(!ok)) { ok = false; goto done; }
+  pend0 = -1;
   // 1. dA = dO V^T, dA^T = V dO^T, Zq = X_q W_q, Zk = X_k W_k
   if (tid == 0) {
     tc_fence_after();
@@ -336,10 +369,11 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
     for (int s = 0; s < 8; ++s) mma_ss(tb + C_ZK, desc_k(sbase + R_XK, s), desc_mn(sbase + R_W + REG, s), id_z, s > 0);
     mma_commit(&bars[1]);
   }
-  ok = mbar_wait(&bars[1], 0, p.status, ST_TIMEOUT);
-  if (__syncthreads_or(!ok)) goto done;
+  ok = mbar_wait(&bars[1], par, p.status, ST_TIMEOUT);
+  if (__syncthreads_or(!ok)) { ok = false; goto done; }
   tc_fence_after();
   if (tid == 0) {   // the weights are consumed: S' goes into their place
+    pend_sp = true;
     mbar_expect_tx(&bars[2], TILE);
     tma_load_3d(sm + R_W, &p.msp, &bars[2], 0, 0, snap_idx);
     tma_load_3d(sm + R_W + REG, &p.msp, &bars[2], 64, 0, snap_idx);
@@ -425,8 +459,8 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
     for (int s = 0; s < 8; ++s) mma_ss(tb + C_AT, desc_k(sbase + R_XK, s), desc_k(sbase + R_XQ, s), id_kk, s > 0);
     mma_commit(&bars[3]);
   }
-  ok = mbar_wait(&bars[3], 0, p.status, ST_TIMEOUT);
-  if (__syncthreads_or(!ok)) goto done;
+  ok = mbar_wait(&bars[3], par, p.status, ST_TIMEOUT);
+  if (__syncthreads_or(!ok)) { ok = false; goto done; }
   if (wg == 0)   // the two halves' sums meet; read after the next barrier
 #pragma unroll
     for (int k = 0; k < 3; ++k) s_r1[k][row] += r1[k];
@@ -447,8 +481,9 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
   }
   tmem_st_wait();
   tc_fence_before();
-  ok = mbar_wait(&bars[2], 0, p.status, ST_TIMEOUT);
-  if (__syncthreads_or(!ok)) goto done;
+  ok = mbar_wait(&bars[2], par, p.status, ST_TIMEOUT);
+  if (__syncthreads_or(!ok)) { ok = false; goto done; }
+  pend_sp = false;
   // 4a. GQ = dO S'^T + dA^ (Kt hi + lo) ;  GK = dA^T^ (Qt hi + lo) ; dS
   //     replaces S' once its product is done
   if (tid == 0) {
@@ -460,15 +495,17 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
     for (int s = 0; s < 8; ++s) mma_ts(tb + C_GK, tb + C_DATH + s * 8, desc_mn(sbase + R_XQ, s), id_mn, s > 0);
     for (int s = 0; s < 8; ++s) mma_ts(tb + C_GK, tb + C_DATH + s * 8, desc_mn(sbase + R_QL, s), id_mn, 1);
     mma_commit(&bars[5]);
-    if (mbar_wait(&bars[4], 0, p.status, ST_TIMEOUT)) {
+    if (mbar_wait(&bars[4], par, p.status, ST_TIMEOUT)) {
+      pend_ds = true;
       mbar_expect_tx(&bars[6], TILE);
       tma_load_3d(sm + R_W, &p.mds, &bars[6], 0, 0, snap_idx);
       tma_load_3d(sm + R_W + REG, &p.mds, &bars[6], 64, 0, snap_idx);
     }
   }
-  ok = mbar_wait(&bars[5], 0, p.status, ST_TIMEOUT);
-  ok &= mbar_wait(&bars[6], 0, p.status, ST_TIMEOUT);
-  if (__syncthreads_or(!ok)) goto done;
+  ok = mbar_wait(&bars[5], par, p.status, ST_TIMEOUT);
+  ok &= mbar_wait(&bars[6], par, p.status, ST_TIMEOUT);
+  if (__syncthreads_or(!ok)) { ok = false; goto done; }
+  pend_ds = false;
   // 4b. GK += V dS^T ;  DV = A^T^ dO + Kt dS
   if (tid == 0) {
     tc_fence_after();
@@ -481,7 +518,7 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
     // 5. rows, dimension half per group, staged as fp32 tiles in the spent
     //    regions and written with TMA stores (rows past L are clipped by the
     //    maps): dB = Qt GQ - Kt GK (Qt, Kt as hi + lo, so that dB matches the
-    //    products) over V | dO; then dphi_q = E GQ over Qt lo | dS and
+    //    products) over V | dO; then dphi_q = E GQ over Qt lo | Kt lo and
     //    dphi_k = GK / E over Qt hi | Kt hi; then dv over V | dO again.  E
     //    (fp32) is read again from global memory, its loads in flight while
     //    the last products run.
@@ -493,9 +530,13 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
     // dS[0] for the dv pass, back into shared memory once the sums are read
     const float4 ds0 = tid < 32 ? __ldg(reinterpret_cast<const float4 *>(p.ds_r0 + (size_t)snap_idx * D + 4 * tid))
                                 : make_float4(0.f, 0.f, 0.f, 0.f);
-    ok = mbar_wait(&bars[7], 0, p.status, ST_TIMEOUT);
-    if (__syncthreads_or(!ok)) goto done;
+    ok = mbar_wait(&bars[7], par, p.status, ST_TIMEOUT);
+    if (__syncthreads_or(!ok)) { ok = false; goto done; }
     tc_fence_after();
+    if (tid == 0 && more) {   // the products are done with the weights' place: the next item's weights
+      pend0 = (int)(par ^ 1u);
+      item_loads(w + 1, 0);
+    }
     unsigned char *st0 = sm + R_V, *st1 = sm + R_QL, *st2 = sm + R_XQ;
     // rank-one parts of GQ and GK left out of the S' and dS copies
     const float cq = s_r1[0][row], ck = s_r1[1][row], kap = s_r1[2][row];
@@ -554,6 +595,7 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
                         __fdividef(gk[4 * u + 2], E.z), __fdividef(gk[4 * u + 3], E.w));
       }
     }
+    if (more) e_load(w + 1, epre);   // the next item's decay factors, in flight during the dv pass
     fence_proxy_async();
     __syncthreads();
     if (tid == 0) {
@@ -581,10 +623,26 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
     if (tid == 0) {
       for (int bx = 0; bx < 4; ++bx) tma_store_3d(&p.mdv, st0 + bx * 16384, 32 * bx, t0, bh);
       bulk_commit();
-      bulk_wait_all();
+      if (more) {
+        bulk_wait_read_but_last();   // the dphi tiles have been read out of Qt | Kt
+        item_loads(w + 1, 1);
+        bulk_wait_read();            // and the dv tile out of V | dO
+        item_loads(w + 1, 2);
+      }
     }
   }
+  tc_fence_before();
+  __syncthreads();   // this item's TMEM and shared-memory reads are done
+  }
 done:
+  if (tid == 0) {
+    bulk_wait_all();   // this CTA's stores are complete (and have read their staging)
+    if (!ok) {         // a wait gave up: let the copies still in flight land first
+      if (pend0 >= 0) mbar_wait(&bars[0], (uint32_t)pend0, nullptr, 0, 1u << 16);
+      if (pend_sp) mbar_wait(&bars[2], par, nullptr, 0, 1u << 16);
+      if (pend_ds) mbar_wait(&bars[6], par, nullptr, 0, 1u << 16);
+    }
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(s_tmem, 512);
@@ -775,10 +833,17 @@ cudaError_t launch_tc_gla_bwd(const TcGlaBwdArgs &a, int stage, cudaStream_t s) 
     p.H = a.H;
     p.L = a.L;
     p.ntiles = ntiles;
+    p.BH = a.BH;
     p.inv_tau = a.inv_tau;
     cudaError_t e = cudaFuncSetAttribute(tc_gla_bwd_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TILE_SMEM);
     if (e != cudaSuccess) return e;
-    tc_gla_bwd_tile_kernel<<<dim3(ntiles, a.BH), NT_TILE, TILE_SMEM, s>>>(p);
+    int dev = 0, sms = 148;
+    e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const int nwork = ntiles * a.BH;   // one persistent CTA per SM over contiguous runs of tiles
+    tc_gla_bwd_tile_kernel<<<nwork < sms ? nwork : sms, NT_TILE, TILE_SMEM, s>>>(p);
     return cudaGetLastError();
   }
   if (a.scalar_gate)
