@@ -158,6 +158,23 @@ def test_train_step_full_size_sampled_heads(lz, impl):
             check(f"{name}[{b},{h}]", got[name][b:b + 1, h:h + 1], r[name], "bf16")
 
 
+def test_persistent_kernels_walk_ragged_tiles_across_sequences(lz):
+    """256 sequences of a ragged length (three 128-token tiles, the last one
+    44 tokens): the persistent backward kernels give every CTA a run of
+    tiles or key blocks that crosses sequence boundaries; sampled sequences
+    at the start, middle and end of the runs against the oracle."""
+    w = Workload("ragged_many", B=8, H=32, L=300, d=128, window=128, M=4, dtype="bf16", seed=31,
+                 kind="train")
+    inp = make_inputs(w)
+    got = _run(lz, to_device(inp), w, lz.IMPL_TC)
+    torch.cuda.synchronize()
+    pairs = [(0, 0), (3, 17), (7, 31)]
+    want = oracle_backward(inp, window=w.window, tau=w.gate_temp, pairs=pairs)
+    for (b, h), r in want.items():
+        for name in ("dq", "dk", "dv", "dg", "dstate_in"):
+            check(f"{name}[{b},{h}]", got[name][b:b + 1, h:h + 1], r[name], "bf16")
+
+
 @pytest.mark.parametrize("case", ["swa_portable", "no_fmap_weights"])
 def test_backward_mixed_paths(lz, case):
     """bf16, d = 128 combinations outside the fused tensor-core configuration:
