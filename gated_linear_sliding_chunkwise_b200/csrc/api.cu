@@ -363,10 +363,7 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan) {
                        w ? at<float>(ws, lay.dv_swa) : nullptr,
                        b->dq, b->dk, b->dv, b->dg, b->dfmap_wq, b->dfmap_wk, a->H, a->L, inv_tau,
                        gla_tc ? 0 : 1, static_cast<uint32_t *>(ws), nullptr, nullptr, scalar_gate(a)};
-  if (gla_tc) {
-    fa.da = nullptr;   // the gate gradient comes from gate_grad_kernel
-    fa.w16 = at<void>(ws, lay.w16);   // bf16 weights from weights_bf16_kernel, earlier in the plan
-  }
+  if (gla_tc) fa.da = nullptr;   // the gate gradient comes from gate_grad_kernel
   lz::TcGlaBwdArgs tg{a->q, a->k, a->v, a->g, b->dout, a->fmap_wq, a->fmap_wk, nullptr, nullptr, nullptr,
                       nullptr, at<float>(ws, lay.da), nullptr, b->dg, nullptr, static_cast<uint32_t *>(ws),
                       a->H, BH, a->L, inv_tau, nullptr, nullptr, scalar_gate(a)};

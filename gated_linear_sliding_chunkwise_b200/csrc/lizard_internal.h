@@ -100,7 +100,6 @@ struct FinishBwdArgs {
   // dq, dk, dv to them.
   void *xq_part, *xk_part;
   int scalar_gate;   // g and dg hold one value per (token, head): [B*H][L]
-  const void *w16;   // tensor-core finish: bf16 [H][2][128][64] feature-map weights (launch_weights_bf16)
 };
 
 struct TcFwdArgs {

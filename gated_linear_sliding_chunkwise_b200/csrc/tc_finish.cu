@@ -6,10 +6,8 @@
 // n = softmax(-z), z = x W and dphi = [dp, dn]:
 //   dz = p (dp - <dp, p>) - n (dn - <dn, n>)
 //   dx = dz W^T,   dW += x^T dz
-// Persistent: one CTA per SM walks a contiguous run of (sequence, 128-token
-// tile) items; dW_q and dW_k accumulate in TMEM over the run's tiles of one
-// head and are added to the output when the head changes.  The bf16 weights
-// (converted once per call) arrive by TMA with the tiles.  dz is
+// One CTA per sequence walks its 128-token tiles; dW_q and dW_k accumulate
+// in TMEM across the tiles and are added to the output once per CTA.  dz is
 // formed in fp32 (the subtraction above cancels) and only then rounded to
 // bf16 as an MMA operand.
 #include "common.cuh"
@@ -31,7 +29,6 @@ constexpr uint32_t ST_TIMEOUT = 1u;
 
 struct Params {
   CUtensorMap mq, mk;
-  CUtensorMap mw;                          // bf16 weights [H*2][D][F] (W_q, W_k per head)
   CUtensorMap mxq, mxk;                    // bf16 dx_q, dx_k parts (fused mode)
   const float *wq, *wk;
   const float *dphq, *dphk, *dv_gla;       // GLA parts (fp32), null when the branch is off
@@ -39,7 +36,7 @@ struct Params {
   __nv_bfloat16 *dq, *dk, *dv;
   float *dwq, *dwk;
   uint32_t *status;
-  int H, L, BH;
+  int H, L;
   int fused;                               // write dx_q, dx_k parts; the anchor kernels finish dq, dk, dv
 };
 
@@ -59,6 +56,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
   constexpr uint32_t C_WQ = 0, C_WK = 64, C_ZQ = 128, C_ZK = 192, C_XQ = 256, C_XK = 384;
   const int tid = threadIdx.x, warp = tid >> 5, wg = tid >> 7, row = tid & 127;
   const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+  const int bh = blockIdx.x, h = bh % p.H;
   const uint32_t sbase = smem_u32(sm);
   const bool gla = p.dphq != nullptr;
   if (warp == 0) { tmem_alloc(&s_tmem, 512); tmem_relinquish(); }
@@ -69,21 +67,27 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
     fence_barrier_init();
   }
   const int ntiles = (p.L + T - 1) / T;
-  const int nwork = ntiles * p.BH;
-  const int w0 = (int)((long long)blockIdx.x * nwork / gridDim.x);
-  const int w1 = (int)((long long)(blockIdx.x + 1) * nwork / gridDim.x);
-  // X_q, X_k of item w, and the weights ([dk row][feature], MN-major for
-  // z = x W, K-major for dz W^T) when its head differs from the last item's
-  auto loads = [&](int w, bool weights) {
-    const int lbh = w / ntiles, lt0 = (w % ntiles) * T;
-    mbar_expect_tx(&bar_tma, (weights ? 3 : 2) * TILE);
+  auto loads = [&](int c) {
+    mbar_expect_tx(&bar_tma, 2 * TILE);
     for (int r = 0; r < 2; ++r) {
-      tma_load_3d(sm + R_XQ + r * REG, &p.mq, &bar_tma, 64 * r, lt0, lbh);
-      tma_load_3d(sm + R_XK + r * REG, &p.mk, &bar_tma, 64 * r, lt0, lbh);
-      if (weights) tma_load_3d(sm + R_WQ + r * REG, &p.mw, &bar_tma, 0, 0, 2 * (lbh % p.H) + r);
+      tma_load_3d(sm + R_XQ + r * REG, &p.mq, &bar_tma, 64 * r, c * T, bh);
+      tma_load_3d(sm + R_XK + r * REG, &p.mk, &bar_tma, 64 * r, c * T, bh);
     }
   };
-  if (tid == 0 && w0 < w1 && gla) loads(w0, true);
+  if (tid == 0 && ntiles > 0 && gla) loads(0);   // in flight while the weights are staged
+  // weights -> bf16 [dk row][feature] (MN-major for z = x W, K-major for dz W^T);
+  // group 0 W_q, group 1 W_k
+  {
+    const float *W = wg == 0 ? p.wq : p.wk;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      float f[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) f[u] = W[((size_t)h * D + row) * F + c * 8 + u];
+      *reinterpret_cast<uint4 *>(sm + (wg == 0 ? R_WQ : R_WK) + sw128_offset(row, c * 8)) = pack8(f);
+    }
+  }
+  fence_proxy_async();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -93,44 +97,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
   const uint32_t id_dw = idesc_bf16(128, 64, 1, 1);    // X^T (MN-major) x dZ (MN-major, N = 64)
   bool fail = false;
   // this row's dphi values (its group's half) of one map, loaded ahead: map 0
-  // of the next item while this item finishes, map 1 while map 0 is used
+  // of the next tile while this tile finishes, map 1 while map 0 is used
   float4 dpre[16];
-  auto dphi_load = [&](int m, int w) {
-    const int lbh = w / ntiles, t = (w % ntiles) * T + row;
-    const float *src = (m == 0 ? p.dphq : p.dphk) + ((size_t)lbh * p.L + (t < p.L ? t : 0)) * D + wg * F;
+  auto dphi_load = [&](int m, int c) {
+    const int t = c * T + row;
+    const float *src = (m == 0 ? p.dphq : p.dphk) + ((size_t)bh * p.L + (t < p.L ? t : 0)) * D + wg * F;
 #pragma unroll
     for (int u = 0; u < 16; ++u)
       dpre[u] = t < p.L ? *reinterpret_cast<const float4 *>(src + 4 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
   };
-  // dW of the head the accumulators hold, added to the output (group 0 dW_q,
-  // group 1 dW_k; lane = dk index, 64 feature columns per map)
-  auto flush_dw = [&](int hh) {
-    float *dW = wg == 0 ? p.dwq : p.dwk;
-    if (!dW) return;
-    float v[32];
-    for (int ch = 0; ch < 2; ++ch) {
-      tmem_ld32(tl + (wg == 0 ? C_WQ : C_WK) + ch * 32, v);
-#pragma unroll
-      for (int u = 0; u < 32; ++u) atomicAdd(dW + ((size_t)hh * D + row) * F + ch * 32 + u, v[u]);
-    }
-  };
-  if (gla && w0 < w1) dphi_load(0, w0);
-  int cur_h = -1;           // head whose dW the TMEM accumulators hold
-  for (int w = w0, itn = 0; w < w1; ++w, ++itn) {
-    const uint32_t par = (uint32_t)itn & 1u;
-    const int bh = w / ntiles, c = w % ntiles, h = bh % p.H;
+  if (gla && ntiles > 0) dphi_load(0, 0);
+  for (int c = 0; c < ntiles; ++c) {
+    const uint32_t par = c & 1;
     const int tq = c * T + row;
     const bool valid = tq < p.L;
     const size_t off = ((size_t)bh * p.L + (valid ? tq : 0)) * D;
-    const bool first = h != cur_h;   // first item of this head in the run: dW starts afresh
-    if (gla && first && cur_h >= 0) {
-      // the last item's products are done (its bar_d wait): its head's dW out
-      tc_fence_after();
-      flush_dw(cur_h);
-      tmem_ld_wait();
-      tc_fence_before();
-    }
-    if (gla) cur_h = h;
     if (gla) {
       bool ok = mbar_wait(&bar_tma, par, p.status, ST_TIMEOUT);
       if (__syncthreads_or(!ok)) { fail = true; break; }
@@ -172,8 +153,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
           ph[4 * u + 2] *= d[u].z - dot;
           ph[4 * u + 3] *= d[u].w - dot;
         }
-        if (m == 0) dphi_load(1, w);   // the k map's values, in flight while this map finishes
-        else if (w + 1 < w1) dphi_load(0, w + 1);
+        if (m == 0) dphi_load(1, c);   // the k map's values, in flight while this map finishes
+        else if (c + 1 < ntiles) dphi_load(0, c + 1);
         // send the half-terms of the other group's features
         unsigned char *mine = sm + R_STG + (2 * m + wg) * 16384;
         const unsigned char *theirs = sm + R_STG + (2 * m + 1 - wg) * 16384;
@@ -214,15 +195,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
         tc_fence_after();
         for (int s = 0; s < 4; ++s) mma_ss(tb + C_XQ, desc_k(sbase + R_ZQ, s), desc_k(sbase + R_WQ, s), id_dx, s > 0);
         for (int s = 0; s < 4; ++s) mma_ss(tb + C_XK, desc_k(sbase + R_ZK, s), desc_k(sbase + R_WK, s), id_dx, s > 0);
-        for (int s = 0; s < 8; ++s) mma_ss(tb + C_WQ, desc_mn(sbase + R_XQ, s), desc_mn(sbase + R_ZQ, s), id_dw, !first || s > 0);
-        for (int s = 0; s < 8; ++s) mma_ss(tb + C_WK, desc_mn(sbase + R_XK, s), desc_mn(sbase + R_ZK, s), id_dw, !first || s > 0);
+        for (int s = 0; s < 8; ++s) mma_ss(tb + C_WQ, desc_mn(sbase + R_XQ, s), desc_mn(sbase + R_ZQ, s), id_dw, c > 0 || s > 0);
+        for (int s = 0; s < 8; ++s) mma_ss(tb + C_WK, desc_mn(sbase + R_XK, s), desc_mn(sbase + R_ZK, s), id_dw, c > 0 || s > 0);
         mma_commit(&bar_d);
       }
       ok = mbar_wait(&bar_d, par, p.status, ST_TIMEOUT);
       if (__syncthreads_or(!ok)) { fail = true; break; }
       tc_fence_after();
-      // X tiles and weights consumed by the products: the next item's
-      if (tid == 0 && w + 1 < w1) loads(w + 1, (w + 1) / ntiles % p.H != h);
+      if (tid == 0 && c + 1 < ntiles) loads(c + 1);   // X tiles consumed by the dW products
     }
     if (p.fused) {
       // dx of this group's map, bf16, staged over R_STG and written with TMA
@@ -284,9 +264,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
     tc_fence_before();
     __syncthreads();
   }
-  if (gla && !fail && cur_h >= 0) {
+  if (gla && !fail) {
     tc_fence_after();
-    flush_dw(cur_h);
+    // dW rows: lane = dk index, 64 feature columns per map; group 0 dW_q, group 1 dW_k
+    float *dW = wg == 0 ? p.dwq : p.dwk;
+    if (dW) {
+      float v[32];
+      for (int ch = 0; ch < 2; ++ch) {
+        tmem_ld32(tl + (wg == 0 ? C_WQ : C_WK) + ch * 32, v);
+#pragma unroll
+        for (int u = 0; u < 32; ++u) atomicAdd(dW + ((size_t)h * D + row) * F + ch * 32 + u, v[u]);
+      }
+    }
   }
   if (p.fused && tid == 0) bulk_wait_all();
   tc_fence_before();
@@ -308,7 +297,6 @@ cudaError_t launch_tc_finish(const FinishBwdArgs &a, int BH, cudaStream_t s) {
   if (p.fused && (!make_map_bf16_3d(&p.mxq, a.xq_part, D, rows, BH, T) ||
                   !make_map_bf16_3d(&p.mxk, a.xk_part, D, rows, BH, T)))
     return cudaErrorInvalidValue;
-  if (a.dphq && (!a.w16 || !make_map_bf16_3d(&p.mw, a.w16, F, D, (uint64_t)a.H * 2, T))) return cudaErrorInvalidValue;
   p.wq = a.wq;
   p.wk = a.wk;
   p.dphq = a.dphq;
@@ -325,17 +313,9 @@ cudaError_t launch_tc_finish(const FinishBwdArgs &a, int BH, cudaStream_t s) {
   p.status = a.status;
   p.H = a.H;
   p.L = a.L;
-  p.BH = BH;
   cudaError_t e = cudaFuncSetAttribute(tc_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148;
-  e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess) return e;
-  const int nwork = (a.L + T - 1) / T * BH;   // one persistent CTA per SM over contiguous runs of tiles
-  if (nwork == 0) return cudaSuccess;
-  tc_finish_kernel<<<nwork < sms ? nwork : sms, NTHREADS, SMEM_BYTES, s>>>(p);
+  tc_finish_kernel<<<BH, NTHREADS, SMEM_BYTES, s>>>(p);
   return cudaGetLastError();
 }
 
