@@ -177,10 +177,12 @@ def gla_forward(phq, phk, v, a, S0=None, keep_states=False):
     return o, S, states
 
 
-def gla_backward(phq, phk, v, a, S0, do):
+def gla_backward(phq, phk, v, a, S0, do, dS_L=None):
     """Reverse-mode derivative of :func:`gla_forward`, from the recurrence.
 
-    With dS the gradient flowing into S_t from tokens >= t:
+    dS_L: gradient flowing into the final state S_{L-1} from outside the
+    sequence (None: the final state is unused).  With dS the gradient
+    flowing into S_t from tokens >= t (and from dS_L):
       dS   += phq_t do_t^T
       dphq_t = S_t do_t,  dphk_t = dS v_t,  dv_t = dS^T phk_t
       da_t   = exp(a_t) * rowsum(dS * S_{t-1})
@@ -196,7 +198,7 @@ def gla_backward(phq, phk, v, a, S0, do):
     dphk = np.zeros_like(phk)
     dv = np.zeros_like(v)
     da = np.zeros_like(a)
-    dS = np.zeros((B, H, dk, dv_))
+    dS = np.zeros((B, H, dk, dv_)) if dS_L is None else _f64(dS_L).copy()
     for t in range(L - 1, -1, -1):
         dS += phq[:, :, t, :, None] * do[:, :, t, None, :]
         St = states[t]
@@ -401,8 +403,13 @@ def chain_states(seg_states, seg_log_decays, rank, state_in=None):
 def lizard_backward(q, k, v, g, dout, *, window, tau=16.0, scale=None,
                     fmap_wq=None, fmap_wk=None, meta_k=None, meta_v=None,
                     alpha=None, state_in=None, branch=BRANCH_BOTH,
-                    gate=GATE_PER_DIM):
+                    gate=GATE_PER_DIM, dstate_out=None):
     """Gradients of sum(dout * lizard_forward(...)['o']) w.r.t. every input.
+
+    dstate_out [B,H,dk,dv]: gradient of the loss with respect to the final
+    state (the loss then is sum(dout * o) + sum(dstate_out * state_out), the
+    form a caller that chains sequences through their states has); None for
+    an unused final state.
 
     Returns a dict: dq, dk, dv, dg (the shape of g: [B,H,L,dk], or [B,H,L]
     for gate="scalar"), dmeta_k, dmeta_v, dfmap_wq,
@@ -425,7 +432,8 @@ def lizard_backward(q, k, v, g, dout, *, window, tau=16.0, scale=None,
         a = layer_log_decay(g, tau, gate, dk)
         phq = feature_map(q, fmap_wq)
         phk = feature_map(k, fmap_wk)
-        dphq, dphk, dv_g, da, dS0 = gla_backward(phq, phk, v, a, state_in, dout)
+        dphq, dphk, dv_g, da, dS0 = gla_backward(phq, phk, v, a, state_in, dout,
+                                                 dstate_out)
         dq_g, dWq = feature_map_backward(q, fmap_wq, dphq)
         dk_g, dWk = feature_map_backward(k, fmap_wk, dphk)
         res["dq"] += dq_g
