@@ -331,7 +331,8 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan) {
     lz::TcGlaBwdArgs t{a->q, a->k, a->v, a->g, b->dout, a->fmap_wq, a->fmap_wk, snap_s,
                        at<void>(ws, lay.snap_ds), at<float>(ws, lay.dphq), at<float>(ws, lay.dphk),
                        at<float>(ws, lay.da), at<float>(ws, lay.dv_gla), b->dg, b->dstate_in,
-                       status, a->H, BH, a->L, inv_tau, e32, gr, scalar_gate(a), at<void>(ws, lay.w16)};
+                       status, a->H, BH, a->L, inv_tau, e32, gr, scalar_gate(a), at<void>(ws, lay.w16),
+                       b->dstate_out};
     void *w16 = at<void>(ws, lay.w16);
     plan.add("weights_bf16_kernel", [=](cudaStream_t s) { return lz::launch_weights_bf16(a->fmap_wq, a->fmap_wk, w16, a->H, s); });
     plan.add("tc_gla_dstates_kernel", [=](cudaStream_t s) { return lz::launch_tc_gla_bwd(t, 0, s); });
@@ -345,7 +346,7 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan) {
     plan.add("gla_states_simt", [=](cudaStream_t s) { return lz::launch_gla_states(sa, BH, D, bf16, s); });
     lz::GlaBwdArgs ga{at<float>(ws, lay.phq), at<float>(ws, lay.phk), at<float>(ws, lay.a), a->v, b->dout,
                       at<float>(ws, lay.sprev), at<float>(ws, lay.dphq), at<float>(ws, lay.dphk),
-                      at<float>(ws, lay.da), at<float>(ws, lay.dv_gla), b->dstate_in, a->L};
+                      at<float>(ws, lay.da), at<float>(ws, lay.dv_gla), b->dstate_in, a->L, b->dstate_out};
     plan.add("gla_bwd_simt", [=](cudaStream_t s) { return lz::launch_gla_bwd_simt(ga, BH, D, bf16, s); });
   }
   const bool swa_tc = w && bwd_swa_uses_tc(a, b->impl);
@@ -480,8 +481,9 @@ static lizard_status check_bwd(const lizard_bwd_args *b) {
   if ((b->dmeta_k && !f.meta_k) || (b->dmeta_v && !f.meta_v) || (b->dfmap_wq && !f.fmap_wq) ||
       (b->dfmap_wk && !f.fmap_wk))
     return LIZARD_ERR_INVALID_ARG;
+  if (b->dstate_out && !gla_on(&f)) return LIZARD_ERR_INVALID_ARG;   // no final state without the GLA branch
   const void *ptrs[] = {b->dout, b->dq, b->dk, b->dv, b->dg, b->dmeta_k, b->dmeta_v,
-                        b->dfmap_wq, b->dfmap_wk, b->dalpha, b->dstate_in};
+                        b->dfmap_wq, b->dfmap_wk, b->dalpha, b->dstate_in, b->dstate_out};
   for (const void *p : ptrs)
     if (!ok_ptr(p)) return LIZARD_ERR_INVALID_ARG;
   return LIZARD_OK;

@@ -65,6 +65,7 @@ struct GlaBwdArgs {
   float *dphq, *dphk, *da, *dv_gla;
   float *dstate_in;  // may be null
   int L;
+  const float *dstate_out;   // [BH][D][D] gradient into the final state, or null (zero)
 };
 
 struct SwaBwdQArgs {
@@ -154,6 +155,7 @@ struct TcGlaBwdArgs {
   const float *gate_r;          // fp32 [B*H][L/128][128] log-decay of every tile
   int scalar_gate;              // g and dg hold one value per (token, head): [B*H][L]
   const void *w16;              // bf16 [H][2][128][64] feature-map weights (launch_weights_bf16)
+  const float *dstate_out;      // [BH][D][D] gradient into the final state, or null (zero)
 };
 
 constexpr int kBwdC = 32;   // GLA chunk used by the portable backward

@@ -106,7 +106,9 @@ __global__ void __launch_bounds__(256) gla_bwd_simt(GlaBwdArgs p) {
   const T *vsrc = static_cast<const T *>(p.v);
   const T *osrc = static_cast<const T *>(p.dout);
   const int nch = (p.L + C - 1) / C;
-  for (int i = tid; i < D * SP; i += 256) dS[i] = 0.f;
+  // dS starts as the gradient flowing into the final state (zero when unused)
+  for (int i = tid; i < D * SP; i += 256)
+    dS[i] = (p.dstate_out && i % SP < D) ? p.dstate_out[(size_t)bh * D * D + (i / SP) * D + i % SP] : 0.f;
   float carry = 0.f;                   // reverse running sum of dB (thread i < D)
   __syncthreads();
   for (int c = nch - 1; c >= 0; --c) {

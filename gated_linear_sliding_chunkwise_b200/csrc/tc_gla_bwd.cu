@@ -54,6 +54,7 @@ struct DsParams {
   __nv_bfloat16 *snap;      // [BH][ntiles][D][D] dS - 1 dS[0] at each tile's end (bf16)
   float *snap_r0;           // [BH][ntiles][D] row 0 of that dS (fp32)
   float *dstate_in;         // [BH][D][D] or null
+  const float *dstate_out;  // [BH][D][D] gradient into the final state, or null (zero)
   uint32_t *status;
   int H, L;
   float inv_tau;
@@ -134,9 +135,15 @@ __global__ void __launch_bounds__(NT_DS, 1) tc_gla_dstates_kernel(const __grid_c
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = s_tmem, tl = tb + lane_off;
-  {   // dS starts at zero: nothing flows into the last tile's end state
-    uint32_t z[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int c = 64 * wg; c < 64 * wg + 64; c += 8) tmem_st8(tl + C_S + c, z);
+  {   // dS starts as the gradient flowing into the last tile's end state (the
+      // final state): dstate_out, or zero; lane = key dimension, column half per group
+    const float *src = p.dstate_out ? p.dstate_out + ((size_t)bh * D + row) * D : nullptr;
+    for (int c = 64 * wg; c < 64 * wg + 64; c += 8) {
+      uint32_t z[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) z[u] = __float_as_uint(src ? src[c + u] : 0.f);
+      tmem_st8(tl + C_S + c, z);
+    }
     tmem_st_wait();
   }
   const uint32_t id_z = idesc_bf16(128, 64, 0, 1);
@@ -802,6 +809,7 @@ cudaError_t launch_tc_gla_bwd(const TcGlaBwdArgs &a, int stage, cudaStream_t s) 
     p.snap = static_cast<__nv_bfloat16 *>(a.snap_ds);
     p.snap_r0 = const_cast<float *>(snapshot_row0(a.snap_ds, a.BH, a.L));
     p.dstate_in = a.dstate_in;
+    p.dstate_out = a.dstate_out;
     p.status = a.status;
     p.H = a.H;
     p.L = a.L;

@@ -53,7 +53,8 @@ class BwdArgs(ctypes.Structure):
                 ("dg", _vp), ("dmeta_k", _vp), ("dmeta_v", _vp), ("dfmap_wq", _vp),
                 ("dfmap_wk", _vp), ("dalpha", _vp), ("dstate_in", _vp), ("impl", _i32),
                 ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t),
-                ("launch_events", ctypes.POINTER(_vp)), ("n_launch_events", _i32)]
+                ("launch_events", ctypes.POINTER(_vp)), ("n_launch_events", _i32),
+                ("dstate_out", _vp)]
 
 
 class DecodeArgs(ctypes.Structure):
@@ -301,14 +302,17 @@ def _bwd_struct(f, q, k, v, g, dout, *, meta_k, meta_v, fmap_wq, fmap_wk, impl, 
 def attn_bwd(q, k, v, g, dout, *, window, chunk=64, gate_temp=16.0, softmax_scale=0.0,
              fmap_wq=None, fmap_wk=None, meta_k=None, meta_v=None, alpha=None,
              state_in=None, branch=BRANCH_BOTH, impl=IMPL_AUTO, want_dstate=True,
-             workspace=None, stream=None, events=None, plan_only=False):
-    """Backward of the hybrid layer (lizard_attn_bwd); returns every gradient."""
+             workspace=None, stream=None, events=None, plan_only=False, dstate_out=None):
+    """Backward of the hybrid layer (lizard_attn_bwd); returns every gradient.
+    dstate_out [B, H, dk, dv] fp32: gradient flowing into the final state
+    (None: the final state is unused)."""
     f = _fwd_struct(q, k, v, g, window=window, chunk=chunk, gate_temp=gate_temp,
                     softmax_scale=softmax_scale, fmap_wq=fmap_wq, fmap_wk=fmap_wk,
                     meta_k=meta_k, meta_v=meta_v, alpha=alpha, state_in=state_in,
                     branch=branch, impl=impl)
     b, res = _bwd_struct(f, q, k, v, g, dout, meta_k=meta_k, meta_v=meta_v, fmap_wq=fmap_wq,
                          fmap_wk=fmap_wk, impl=impl, want_dstate=want_dstate)
+    b.dstate_out = _ptr(dstate_out)
     dev = q.device
     nbytes = bwd_workspace_bytes(b)
     ws = _workspace(nbytes, dev, workspace)

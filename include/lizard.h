@@ -183,7 +183,12 @@ lizard_status lizard_attn_fwd(const lizard_fwd_args *args, lizard_stream_t strea
  *            shapes as the inputs, written (overwritten, not accumulated);
  *            each may be NULL when not wanted (and must be NULL when the
  *            matching input is NULL).
- * The final state S_{L-1} is treated as unused (zero incoming gradient).
+ *   dstate_out [B, H, dk, dv] fp32 gradient flowing into the final state
+ *            S_{L-1} from outside the call (a later chunk's dstate_in, when a
+ *            long sequence is trained chunk by chunk through state_in /
+ *            state_out), or NULL for an unused final state.  The gradients
+ *            are then those of sum(dout * o) + sum(dstate_out * S_{L-1}).
+ *            Needs the GLA branch.
  */
 typedef struct {
   lizard_fwd_args fwd;
@@ -199,6 +204,7 @@ typedef struct {
   size_t workspace_bytes;
   void *const *launch_events;   /* as in lizard_fwd_args */
   int32_t n_launch_events;
+  const float *dstate_out;      /* see above; NULL = zero */
 } lizard_bwd_args;
 
 size_t lizard_bwd_workspace_size(const lizard_bwd_args *args);

@@ -310,3 +310,15 @@ def test_chain_rejects_bad_arguments_on_host(lz, over, code):
     for k_, v_ in over.items():
         setattr(a, k_, v_)
     assert lz.lib().lizard_chain_states(ctypes.byref(a), None) == code
+
+
+def test_backward_checks_the_incoming_state_gradient(lz):
+    fake = 0x10000
+    for branch, ds, code in [(lz.BRANCH_SWA_ONLY, 0x30000, lz.ERR_INVALID_ARG),   # no final state
+                             (lz.BRANCH_BOTH, 0x30004, lz.ERR_INVALID_ARG)]:     # misaligned
+        b = lz.BwdArgs()
+        b.fwd = _fwd(lz, branch=branch)
+        b.dout = b.dq = b.dk = b.dv = b.dg = fake
+        b.dstate_out = ds
+        b.workspace, b.workspace_bytes = 0x20000, 1 << 40
+        assert lz.lib().lizard_attn_bwd(ctypes.byref(b), None) == code

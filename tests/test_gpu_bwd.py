@@ -5,7 +5,7 @@ import pytest
 import torch
 
 from gated_linear_sliding_chunkwise_b200.synth import WORKLOADS, Workload, make_inputs, random_alpha
-from lizard_testutil import check, oracle_backward, to_device
+from lizard_testutil import check, oracle_backward, to64, to_device
 from oracle import lizard_ref as ref
 
 pytestmark = pytest.mark.gpu
@@ -173,6 +173,60 @@ def test_persistent_kernels_walk_ragged_tiles_across_sequences(lz):
     for (b, h), r in want.items():
         for name in ("dq", "dk", "dv", "dg", "dstate_in"):
             check(f"{name}[{b},{h}]", got[name][b:b + 1, h:h + 1], r[name], "bf16")
+
+
+DSTATE_CASES = [
+    # impl, dtype, d, L, window, M
+    ("simt", "fp32", 64, 97, 16, 4),
+    ("tc", "bf16", 128, 300, 128, 4),
+]
+
+
+@pytest.mark.parametrize("impl,dtype,d,L,window,M", DSTATE_CASES)
+def test_backward_with_incoming_state_gradient(lz, impl, dtype, d, L, window, M):
+    """dstate_out: the gradients of sum(dout * o) + sum(G * state_out)."""
+    w = Workload("dstate", B=2, H=2, L=L, d=d, window=window, M=M, dtype=dtype, seed=700 + L,
+                 kind="train")
+    inp = make_inputs(w)
+    inp["state_in"] = torch.randn(2, 2, d, d, generator=torch.Generator().manual_seed(9)) * 0.1
+    G = torch.randn(2, 2, d, d, generator=torch.Generator().manual_seed(10))
+    x = to_device(inp)
+    got = _run(lz, x, w, _impl(lz, impl), dstate_out=G.cuda())
+    assert lz.workspace_status(got["workspace"]) == lz.OK
+    y = {k_: to64(v_) for k_, v_ in inp.items() if v_ is not None}
+    want = ref.lizard_backward(y["q"], y["k"], y["v"], y["g"], y["dout"], window=window, tau=w.gate_temp,
+                               fmap_wq=y["fmap_wq"], fmap_wk=y["fmap_wk"], meta_k=y["meta_k"],
+                               meta_v=y["meta_v"], alpha=y["alpha"], state_in=y["state_in"],
+                               dstate_out=to64(G))
+    for name in GRADS:
+        check(name, got[name], want[name], dtype)
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_chunks_chained_through_states_give_the_whole_backward(lz, impl):
+    """A sequence trained in two chunks (the GLA branch, which carries all of
+    the history in its state): forward of chunk 1 gives chunk 2 its
+    state_in; backward of chunk 2 gives chunk 1 its dstate_out."""
+    dtype, d = ("fp32", 64) if impl == "simt" else ("bf16", 128)
+    L, cut = 400, 256
+    w = Workload("chunks", B=2, H=2, L=L, d=d, window=64, M=0, dtype=dtype, seed=77, kind="train")
+    inp = make_inputs(w)
+    inp["meta_k"] = inp["meta_v"] = None
+    x = to_device(inp)
+    kw = dict(window=w.window, gate_temp=w.gate_temp, fmap_wq=x["fmap_wq"], fmap_wk=x["fmap_wk"],
+              branch=lz.BRANCH_GLA_ONLY, impl=_impl(lz, impl))
+    part = lambda a, b: {k_: x[k_][:, :, a:b].contiguous() for k_ in ("q", "k", "v", "g", "dout")}
+    c1, c2 = part(0, cut), part(cut, L)
+    S_cut = lz.attn_fwd(c1["q"], c1["k"], c1["v"], c1["g"], want_state=True, **kw)["state_out"]
+    b2 = lz.attn_bwd(c2["q"], c2["k"], c2["v"], c2["g"], c2["dout"], state_in=S_cut, **kw)
+    b1 = lz.attn_bwd(c1["q"], c1["k"], c1["v"], c1["g"], c1["dout"], dstate_out=b2["dstate_in"], **kw)
+    torch.cuda.synchronize()
+    want = oracle_backward(inp, window=w.window, tau=w.gate_temp, branch=ref.BRANCH_GLA_ONLY)
+    for name in ("dq", "dk", "dv", "dg"):
+        check(name, torch.cat([b1[name], b2[name]], dim=2), want[name], dtype)
+    check("dstate_in", b1["dstate_in"], want["dstate_in"], dtype)
+    for name in ("dfmap_wq", "dfmap_wk"):
+        check(name, b1[name] + b2[name], want[name], dtype)
 
 
 @pytest.mark.parametrize("case", ["swa_portable", "no_fmap_weights"])
