@@ -111,7 +111,7 @@ bool bwd_gla_uses_tc(const lizard_fwd_args *a, int impl) {
 
 struct BwdLayout {
   size_t phq, phk, a, sprev, dphq, dphk, da, dv_gla, dq_swa, dk_swa, dv_swa, lse, Dterm, dsm, pm, snap_s,
-      snap_ds, e32, gr, w16, total;
+      snap_ds, e32, gr, w16, kap, total;
 };
 BwdLayout bwd_layout(const lizard_fwd_args *a, int impl) {
   const size_t BH = (size_t)a->B * a->H;
@@ -132,6 +132,7 @@ BwdLayout bwd_layout(const lizard_fwd_args *a, int impl) {
     l.e32 = off; off += nd;      // fp32 decay factors E of every tile
     l.gr = off; off += up(BH * ((a->L + 127) / 128) * a->dk * sizeof(float));   // tiles' log-decays
     l.w16 = off; off += up(lz::tc_gla_bwd_weights_bytes(a->H));                  // bf16 W_q, W_k
+    l.kap = off; off += up(BH * 2 * a->dk * sizeof(float));   // final-state share of the decay gradient
   } else if (gla_on(a)) {
     l.phq = off; off += nd;
     l.phk = off; off += nd;
@@ -141,6 +142,7 @@ BwdLayout bwd_layout(const lizard_fwd_args *a, int impl) {
     l.dphk = off; off += nd;
     l.da = off; off += nd;
     l.dv_gla = off; off += nv;
+    l.kap = off; off += up(BH * a->dk * sizeof(float));       // final-state share of the decay gradient
   }
   if (swa_on(a)) {
     l.dq_swa = off; off += nd;
@@ -318,6 +320,8 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan) {
     lz::TcFwdArgs f{a->q, a->k, a->v, a->g, a->fmap_wq, a->fmap_wk, a->meta_k, a->meta_v, a->alpha,
                     a->state_in, nullptr, nullptr, nullptr, static_cast<uint32_t *>(ws), nullptr, BH, a->H,
                     a->L, a->M, a->window, 0, inv_tau, scale_of(a), scalar_gate(a)};
+    f.dstate_out = b->dstate_out;   // the state copies also form the final state's share of dg
+    f.kap = at<float>(ws, lay.kap);
     void *snap_s = at<void>(ws, lay.snap_s);
     float *e32 = at<float>(ws, lay.e32), *gr = at<float>(ws, lay.gr);
     uint32_t *status = static_cast<uint32_t *>(ws);
@@ -342,11 +346,13 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan) {
     lz::PrepArgs pa{a->q, a->k, a->g, a->fmap_wq, a->fmap_wk, at<float>(ws, lay.phq), at<float>(ws, lay.phk),
                     at<float>(ws, lay.a), a->H, a->L, inv_tau, scalar_gate(a)};
     plan.add("prep_kernel", [=](cudaStream_t s) { return lz::launch_prep(pa, BH, D, bf16, s); });
-    lz::GlaStatesArgs sa{at<float>(ws, lay.phk), at<float>(ws, lay.a), a->v, a->state_in, at<float>(ws, lay.sprev), a->L};
+    float *kap = b->dstate_out ? at<float>(ws, lay.kap) : nullptr;
+    lz::GlaStatesArgs sa{at<float>(ws, lay.phk), at<float>(ws, lay.a), a->v, a->state_in, at<float>(ws, lay.sprev), a->L,
+                         b->dstate_out, kap};
     plan.add("gla_states_simt", [=](cudaStream_t s) { return lz::launch_gla_states(sa, BH, D, bf16, s); });
     lz::GlaBwdArgs ga{at<float>(ws, lay.phq), at<float>(ws, lay.phk), at<float>(ws, lay.a), a->v, b->dout,
                       at<float>(ws, lay.sprev), at<float>(ws, lay.dphq), at<float>(ws, lay.dphk),
-                      at<float>(ws, lay.da), at<float>(ws, lay.dv_gla), b->dstate_in, a->L, b->dstate_out};
+                      at<float>(ws, lay.da), at<float>(ws, lay.dv_gla), b->dstate_in, a->L, b->dstate_out, kap};
     plan.add("gla_bwd_simt", [=](cudaStream_t s) { return lz::launch_gla_bwd_simt(ga, BH, D, bf16, s); });
   }
   const bool swa_tc = w && bwd_swa_uses_tc(a, b->impl);
@@ -368,6 +374,7 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan) {
   lz::TcGlaBwdArgs tg{a->q, a->k, a->v, a->g, b->dout, a->fmap_wq, a->fmap_wk, nullptr, nullptr, nullptr,
                       nullptr, at<float>(ws, lay.da), nullptr, b->dg, nullptr, static_cast<uint32_t *>(ws),
                       a->H, BH, a->L, inv_tau, nullptr, nullptr, scalar_gate(a)};
+  if (gla_tc && b->dstate_out) tg.kap = at<float>(ws, lay.kap);
   if (fused) {
     // the gate-logit gradient (from dB) beside the feature-map and anchor passes
     plan.fork();

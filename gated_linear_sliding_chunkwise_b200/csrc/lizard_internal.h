@@ -56,6 +56,10 @@ struct GlaStatesArgs {
   const float *state_in;
   float *sprev;     // [BH][nchunk][D][D] state at the start of each chunk
   int L;
+  // With an incoming final-state gradient G: kap[bh][i] = sum_v G[i][v] S_L[i][v],
+  // the final state's share of every token's log-decay gradient (null: none)
+  const float *dstate_out;
+  float *kap;
 };
 
 struct GlaBwdArgs {
@@ -66,6 +70,7 @@ struct GlaBwdArgs {
   float *dstate_in;  // may be null
   int L;
   const float *dstate_out;   // [BH][D][D] gradient into the final state, or null (zero)
+  const float *kap;          // [BH][D] from gla_states_simt when dstate_out is set: the reverse sum's start
 };
 
 struct SwaBwdQArgs {
@@ -123,6 +128,11 @@ struct TcFwdArgs {
   // tokens before token 0 (P = 0: none).
   const void *k_prefix, *v_prefix;
   int P;
+  // State pass that writes the backward's copies, with an incoming final-state
+  // gradient G = dstate_out: kap [BH][2][128], the two column halves of
+  // sum_v G[i][v] S_L[i][v] (null: none)
+  const float *dstate_out;
+  float *kap;
 };
 
 struct TcSwaBwdArgs {
@@ -156,6 +166,7 @@ struct TcGlaBwdArgs {
   int scalar_gate;              // g and dg hold one value per (token, head): [B*H][L]
   const void *w16;              // bf16 [H][2][128][64] feature-map weights (launch_weights_bf16)
   const float *dstate_out;      // [BH][D][D] gradient into the final state, or null (zero)
+  const float *kap;             // [BH][2][128] final-state share of the log-decay gradient, or null
 };
 
 constexpr int kBwdC = 32;   // GLA chunk used by the portable backward

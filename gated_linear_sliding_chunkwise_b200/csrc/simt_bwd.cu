@@ -82,6 +82,15 @@ __global__ void __launch_bounds__(256) gla_states_simt(GlaStatesArgs p) {
       for (int c_ = 0; c_ < ST; ++c_) S[(ty * ST + a_) * D + tx * ST + c_] = acc[a_][c_];
     __syncthreads();
   }
+  // S = S_L: with an incoming final-state gradient G, every token's log-decay
+  // gradient also carries sum_v G[i][v] S_L[i][v] (S_L scales with the total
+  // log-decay of dimension i)
+  if (p.kap && tid < D) {
+    const float *G = p.dstate_out + ((size_t)bh * D + tid) * D;
+    float s = 0.f;
+    for (int v = 0; v < D; ++v) s = fmaf(G[v], S[tid * D + v], s);
+    p.kap[(size_t)bh * D + tid] = s;
+  }
 }
 
 // ------------------------------------------------------ GLA reverse scan --
@@ -109,7 +118,8 @@ __global__ void __launch_bounds__(256) gla_bwd_simt(GlaBwdArgs p) {
   // dS starts as the gradient flowing into the final state (zero when unused)
   for (int i = tid; i < D * SP; i += 256)
     dS[i] = (p.dstate_out && i % SP < D) ? p.dstate_out[(size_t)bh * D * D + (i / SP) * D + i % SP] : 0.f;
-  float carry = 0.f;                   // reverse running sum of dB (thread i < D)
+  // reverse running sum of dB (thread i < D), from the final state's share
+  float carry = (p.kap && tid < D) ? p.kap[(size_t)bh * D + tid] : 0.f;
   __syncthreads();
   for (int c = nch - 1; c >= 0; --c) {
     const int c0 = c * C, n = min(C, p.L - c0);

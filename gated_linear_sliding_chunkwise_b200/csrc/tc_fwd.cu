@@ -94,6 +94,8 @@ struct Params {
   float *snap_r0;           // ... and [BH][ntiles][D] fp32 row 0 of S' (the part taken out of every row)
   const float *gate_r;      // [BH][ntiles][D] log-decay r of every tile (gate_prep_kernel)
   const float *gate_e32;    // mode 1: [BH][L][D] fp32 decay factors E (mode 0 loads bf16 E as the G tiles)
+  const float *kap_g;       // mode 1 with copies: incoming final-state gradient G [BH][D][D], or null
+  float *kap;               // ... and [BH][2][D]: the column halves of sum_v G[i][v] S_L[i][v]
   int H, L, M, window, branch;
   int mode;                 // 0: full forward, 1: state pass
   int nseg, tiles_per_seg;
@@ -669,6 +671,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
     sdst = p.seg_state + (((size_t)bh * p.nseg + seg) * D + row) * D;
     if (wg == 0) p.seg_decay[((size_t)bh * p.nseg + seg) * D + row] = tot_decay;
   }
+  if (!s_fail && p.kap) {   // thread row = key dimension i, column half per group
+    tc_fence_after();
+    const float *G = p.kap_g + ((size_t)bh * D + row) * D;
+    float part = 0.f;
+    for (int c16 = 4 * wg; c16 < 4 * wg + 4; ++c16) {
+      float v[16];
+      tmem_ld16(tl + C_S + c16 * 16, v);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) part = fmaf(G[c16 * 16 + u], v[u], part);
+    }
+    p.kap[((size_t)bh * 2 + wg) * D + row] = part;
+  }
   if (!s_fail && sdst) {
     tc_fence_after();
     for (int c16 = 4 * wg; c16 < 4 * wg + 4; ++c16) {
@@ -915,6 +929,8 @@ cudaError_t launch_tc_state_snapshots(const TcFwdArgs &a, void *snap, const floa
   p.seg_start = a.state_in;
   p.seg_state = nullptr;
   p.seg_decay = nullptr;
+  p.kap_g = a.dstate_out;
+  p.kap = a.dstate_out ? a.kap : nullptr;
   cudaError_t e =
       cudaFuncSetAttribute(tc_fwd_kernel<K_STATE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;

@@ -663,7 +663,7 @@ done:
 // give its carry, and a second pass walks it backwards writing dg.
 constexpr int kGateSeg = 8;
 __global__ void __launch_bounds__(256) gate_grad_kernel(const float *dB, const __nv_bfloat16 *g, float *dg, int L,
-                                                       float inv_tau) {
+                                                       float inv_tau, const float *kap) {
   __shared__ float s_tot[kGateSeg][32];
   const int bh = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int i = blockIdx.y * 32 + lane;
@@ -679,7 +679,8 @@ __global__ void __launch_bounds__(256) gate_grad_kernel(const float *dB, const _
   for (; t < tz; ++t) part[0] += dB[base + (size_t)t * D];
   s_tot[warp][lane] = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
   __syncthreads();
-  float carry = 0.f;
+  // the sum starts with the final state's share (an incoming final-state gradient)
+  float carry = kap ? kap[(size_t)bh * 2 * D + i] + kap[((size_t)bh * 2 + 1) * D + i] : 0.f;
   for (int w = warp + 1; w < kGateSeg; ++w) carry += s_tot[w][lane];
   t = tz - 1;
   for (; t - 7 >= ta; t -= 8) {
@@ -709,7 +710,7 @@ __global__ void __launch_bounds__(256) gate_grad_kernel(const float *dB, const _
 // backwards 32 rows at a time with a warp-wide suffix scan, starting from
 // the later segments' totals.
 __global__ void __launch_bounds__(256) gate_grad_scalar_kernel(const float *dB, const __nv_bfloat16 *g, float *dg,
-                                                              int L, float inv_tau) {
+                                                              int L, float inv_tau, const float *kap) {
   __shared__ float s_tot[kGateSeg];
   const int bh = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int seg = (L + kGateSeg - 1) / kGateSeg;
@@ -742,7 +743,14 @@ __global__ void __launch_bounds__(256) gate_grad_scalar_kernel(const float *dB, 
   }
   if (lane == 0) s_tot[warp] = total;
   __syncthreads();   // also orders each warp's parked row sums before pass 2
-  float carry = 0.f;
+  float carry = 0.f;   // starts with the final state's share, summed over the dimensions
+  if (kap) {
+    const float *k2 = kap + (size_t)bh * 2 * D;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) carry += k2[lane * 8 + u];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) carry += __shfl_xor_sync(0xffffffffu, carry, o);
+  }
   for (int w = warp + 1; w < kGateSeg; ++w) carry += s_tot[w];
   for (int hi = tz - 1; hi >= ta; hi -= 32) {
     const int t = hi - lane;                   // lane 0 takes the latest row
@@ -856,10 +864,10 @@ cudaError_t launch_tc_gla_bwd(const TcGlaBwdArgs &a, int stage, cudaStream_t s) 
   }
   if (a.scalar_gate)
     gate_grad_scalar_kernel<<<a.BH, 256, 0, s>>>(a.dB, static_cast<const __nv_bfloat16 *>(a.g), a.dg, a.L,
-                                                 a.inv_tau);
+                                                 a.inv_tau, a.kap);
   else
     gate_grad_kernel<<<dim3(a.BH, D / 32), 256, 0, s>>>(a.dB, static_cast<const __nv_bfloat16 *>(a.g), a.dg, a.L,
-                                                        a.inv_tau);
+                                                        a.inv_tau, a.kap);
   return cudaGetLastError();
 }
 
