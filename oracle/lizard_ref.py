@@ -318,6 +318,23 @@ def swa_backward(q, k, v, meta_k, meta_v, window, scale, do):
     return dq, dk_, dv, dmk, dmv
 
 
+def swa_backward_prefix(q, k, v, meta_k, meta_v, window, scale, do, k_prefix, v_prefix):
+    """:func:`swa_backward` for a segment whose window reaches P keys and
+    values before token 0 (see :func:`swa_forward`).  The prefix tokens are
+    the first P positions of one longer sequence whose own outputs carry no
+    gradient (their queries are never used).  Returns (dq, dk, dv, dmeta_k,
+    dmeta_v, dk_prefix, dv_prefix)."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    kp, vp = _f64(k_prefix), _f64(v_prefix)
+    B, H, _, dk = q.shape
+    P = kp.shape[2]
+    dq, dk_, dv, dmk, dmv = swa_backward(
+        np.concatenate([np.zeros((B, H, P, dk)), q], axis=2), np.concatenate([kp, k], axis=2),
+        np.concatenate([vp, v], axis=2), meta_k, meta_v, window, scale,
+        np.concatenate([np.zeros((B, H, P, do.shape[-1])), do], axis=2))
+    return dq[:, :, P:], dk_[:, :, P:], dv[:, :, P:], dmk, dmv, dk_[:, :, :P], dv[:, :, :P]
+
+
 # ---------------------------------------------------------------------------
 # The hybrid layer
 # ---------------------------------------------------------------------------
@@ -403,13 +420,15 @@ def chain_states(seg_states, seg_log_decays, rank, state_in=None):
 def lizard_backward(q, k, v, g, dout, *, window, tau=16.0, scale=None,
                     fmap_wq=None, fmap_wk=None, meta_k=None, meta_v=None,
                     alpha=None, state_in=None, branch=BRANCH_BOTH,
-                    gate=GATE_PER_DIM, dstate_out=None):
+                    gate=GATE_PER_DIM, dstate_out=None, k_prefix=None, v_prefix=None):
     """Gradients of sum(dout * lizard_forward(...)['o']) w.r.t. every input.
 
     dstate_out [B,H,dk,dv]: gradient of the loss with respect to the final
     state (the loss then is sum(dout * o) + sum(dstate_out * state_out), the
     form a caller that chains sequences through their states has); None for
-    an unused final state.
+    an unused final state.  k_prefix / v_prefix: the anchor window's prefix,
+    as in lizard_forward; their gradients come back as dk_prefix, dv_prefix
+    (None without a prefix).
 
     Returns a dict: dq, dk, dv, dg (the shape of g: [B,H,L,dk], or [B,H,L]
     for gate="scalar"), dmeta_k, dmeta_v, dfmap_wq,
@@ -427,7 +446,9 @@ def lizard_backward(q, k, v, g, dout, *, window, tau=16.0, scale=None,
            "dmeta_v": None if meta_v is None else np.zeros(_f64(meta_v).shape),
            "dfmap_wq": None if fmap_wq is None else np.zeros(_f64(fmap_wq).shape),
            "dfmap_wk": None if fmap_wk is None else np.zeros(_f64(fmap_wk).shape),
-           "dalpha": np.zeros(H), "dstate_in": np.zeros((B, H, dk, dv_))}
+           "dalpha": np.zeros(H), "dstate_in": np.zeros((B, H, dk, dv_)),
+           "dk_prefix": None if k_prefix is None else np.zeros(_f64(k_prefix).shape),
+           "dv_prefix": None if v_prefix is None else np.zeros(_f64(v_prefix).shape)}
     if branch != BRANCH_SWA_ONLY:
         a = layer_log_decay(g, tau, gate, dk)
         phq = feature_map(q, fmap_wq)
@@ -450,11 +471,15 @@ def lizard_backward(q, k, v, g, dout, *, window, tau=16.0, scale=None,
         if fmap_wk is not None:
             res["dfmap_wk"] = dWk
     if branch != BRANCH_GLA_ONLY:
-        o_swa, _ = swa_forward(q, k, v, meta_k, meta_v, window, scale)
+        o_swa, _ = swa_forward(q, k, v, meta_k, meta_v, window, scale, k_prefix, v_prefix)
         res["dalpha"] = np.einsum("bhld,bhld->h", dout, o_swa)
         dsw = alpha[None, :, None, None] * dout
-        dq_s, dk_s, dv_s, dmk, dmv = swa_backward(q, k, v, meta_k, meta_v,
-                                                  window, scale, dsw)
+        if k_prefix is None:
+            dq_s, dk_s, dv_s, dmk, dmv = swa_backward(q, k, v, meta_k, meta_v,
+                                                      window, scale, dsw)
+        else:
+            dq_s, dk_s, dv_s, dmk, dmv, res["dk_prefix"], res["dv_prefix"] = swa_backward_prefix(
+                q, k, v, meta_k, meta_v, window, scale, dsw, k_prefix, v_prefix)
         res["dq"] += dq_s
         res["dk"] += dk_s
         res["dv"] += dv_s
