@@ -773,6 +773,8 @@ const char *lizard_status_string(lizard_status s) {
 
 const char *lizard_version(void) { return "0.1.0"; }
 
+void lizard_debug_inject_wait_timeout(int32_t count) { lz::g_inject_wait = count > 0 ? count : 0; }
+
 }  // extern "C"
 
 // ------------------------------------------------- sequence parallelism ---

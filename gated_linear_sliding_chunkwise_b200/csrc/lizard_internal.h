@@ -174,6 +174,7 @@ constexpr int kBwdC = 32;   // GLA chunk used by the portable backward
 cudaError_t launch_prep(const PrepArgs &a, int BH, int D, bool bf16, cudaStream_t s);
 cudaError_t launch_gla_fwd_simt(const GlaFwdArgs &a, int BH, int D, bool bf16, cudaStream_t s);
 cudaError_t launch_swa_mix_simt(const SwaMixArgs &a, int BH, int D, bool bf16, cudaStream_t s);
+extern int g_inject_wait;   // test hook (lizard_debug_inject_wait_timeout)
 bool tc_fwd_supported(int dk, int dv, int window, int M, bool bf16);
 // Sequence-parallel pieces.  Tensor-core segment summary: the state pass over
 // whole sequences from a zero start, writing U [BH][D][D] and the summed

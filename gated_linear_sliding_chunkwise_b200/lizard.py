@@ -116,6 +116,8 @@ _lib.lizard_workspace_status.argtypes = [_vp, _vp]
 _lib.lizard_workspace_status.restype = ctypes.c_int
 _lib.lizard_status_string.argtypes = [ctypes.c_int]
 _lib.lizard_status_string.restype = ctypes.c_char_p
+_lib.lizard_debug_inject_wait_timeout.argtypes = [_i32]
+_lib.lizard_debug_inject_wait_timeout.restype = None
 _lib.lizard_version.argtypes = []
 _lib.lizard_version.restype = ctypes.c_char_p
 
@@ -132,6 +134,12 @@ def status_string(code: int) -> str:
 
 def version() -> str:
     return _lib.lizard_version().decode()
+
+
+def debug_inject_wait_timeout(count: int) -> None:
+    """Test hook: the next `count` tensor-core forward full passes wait on a
+    barrier that nothing completes and report LIZARD_ERR_TIMEOUT."""
+    _lib.lizard_debug_inject_wait_timeout(int(count))
 
 
 def lib() -> ctypes.CDLL:

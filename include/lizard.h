@@ -366,6 +366,17 @@ lizard_status lizard_prefill_cache(const lizard_cache_args *args, lizard_stream_
 lizard_status lizard_decode_status(void);
 
 /*
+ * Test hook for failure detection: the next `count` launches of the
+ * tensor-core forward's full pass (lizard_attn_fwd on the tensor-core path)
+ * first wait on a barrier that nothing completes.  The wait gives up after
+ * its iteration limit, the kernel records LIZARD_ERR_TIMEOUT in the
+ * workspace status word, frees its TMEM and returns without computing, as a
+ * real timed-out wait would.  count <= 0 clears it.  Host only; meant for
+ * one test thread.
+ */
+void lizard_debug_inject_wait_timeout(int32_t count);
+
+/*
  * Forward for callers that cannot allocate device memory.
  *
  * Some callers have no way to obtain a device workspace: a plug-in living

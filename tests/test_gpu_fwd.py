@@ -29,6 +29,24 @@ def _run(lz, x, w, impl, **kw):
 IMPLS = ["simt", "tc"]
 
 
+def test_a_wait_that_runs_out_is_reported_and_the_context_stays_usable(lz):
+    """Failure detection without a fault: the test hook makes the forward's
+    first wait run out; the call reports LIZARD_ERR_TIMEOUT through the
+    workspace status, and the next call on the same context computes."""
+    w = Workload("inject", B=1, H=2, L=256, d=128, window=128, M=4, dtype="bf16", seed=5)
+    inp = make_inputs(w)
+    x = to_device(inp)
+    lz.debug_inject_wait_timeout(1)
+    try:
+        got = _run(lz, x, w, lz.IMPL_TC)
+        assert lz.workspace_status(got["workspace"]) == lz.ERR_TIMEOUT
+    finally:
+        lz.debug_inject_wait_timeout(0)
+    got = _run(lz, x, w, lz.IMPL_TC)
+    assert lz.workspace_status(got["workspace"]) == lz.OK
+    check("o", got["o"], oracle_forward(inp, window=w.window, tau=w.gate_temp)["o"], "bf16")
+
+
 def _impl(lz, name):
     return {"simt": lz.IMPL_SIMT, "tc": lz.IMPL_TC, "auto": lz.IMPL_AUTO}[name]
 
