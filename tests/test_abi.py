@@ -322,3 +322,42 @@ def test_backward_checks_the_incoming_state_gradient(lz):
         b.dstate_out = ds
         b.workspace, b.workspace_bytes = 0x20000, 1 << 40
         assert lz.lib().lizard_attn_bwd(ctypes.byref(b), None) == code
+
+
+def test_a_plain_c_program_links_and_calls_the_host_entry_points(lz, tmp_path):
+    """The boundary is plain C: a C11 program built with gcc against
+    include/lizard.h and linked with liblizard.so calls the size queries,
+    the launch plan and the argument checks (none of which needs a GPU)."""
+    src = tmp_path / "client.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include <string.h>
+#include "lizard.h"
+int main(void) {
+  lizard_fwd_args a;
+  memset(&a, 0, sizeof a);
+  a.B = 1; a.H = 2; a.L = 300; a.dk = 128; a.dv = 128; a.chunk = 64; a.window = 128; a.M = 0;
+  a.dtype = LIZARD_BF16; a.branch = LIZARD_BRANCH_BOTH; a.impl = LIZARD_IMPL_AUTO;
+  a.gate = LIZARD_GATE_PER_DIM; a.gate_temp = 16.f;
+  size_t ws = lizard_fwd_workspace_size(&a);
+  const char *names[16];
+  a.q = a.k = a.v = a.g = (const void *)0x10000; a.o = (void *)0x10000;
+  a.fmap_wq = a.fmap_wk = (const float *)0x10000;
+  int n = lizard_fwd_launch_plan(&a, names, 16);
+  lizard_fwd_args bad = a;
+  bad.dk = bad.dv = 96;
+  lizard_status st = lizard_attn_fwd(&bad, NULL);
+  printf("%zu %d %s %d %s %s\n", ws, n, n > 0 ? names[n - 1] : "-", (int)st,
+         lizard_status_string(st), lizard_version());
+  return 0;
+}
+""")
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(lz.LIB_PATH)
+    subprocess.run(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                    "-L", libdir, "-llizard", "-Wl,-rpath," + libdir], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
+    assert int(out[0]) > 0                       # workspace bytes
+    assert int(out[1]) >= 1 and out[2] == "tc_fwd_kernel"   # the tensor-core plan ends with the full pass
+    assert int(out[3]) == lz.ERR_UNSUPPORTED     # d = 96 is refused on the host
+    assert out[-1] == lz.version()
