@@ -99,3 +99,40 @@ def test_prefix_gradients_match_central_differences():
         assert err < 1e-6, f"{gname}: rel err {err:.2e}"
     # only the last window - 1 prefix tokens are in any query's window
     assert np.all(grads["dk_prefix"][:, :, 0] == 0) and np.any(grads["dk_prefix"][:, :, 1:] != 0)
+
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=25, deadline=None)
+@given(L=st.integers(2, 14), window=st.integers(1, 6), cut_frac=st.floats(0.05, 0.95),
+       gate=st.sampled_from(["dim", "scalar"]), with_G=st.booleans(), seed=st.integers(0, 2 ** 16))
+def test_random_splits_reproduce_the_whole_forward_and_backward(L, window, cut_frac, gate, with_G, seed):
+    """Any cut of any short sequence, with a prefix of min(window, cut) tokens:
+    the two halves' outputs and chained gradients equal the whole's."""
+    cut = min(L - 1, max(1, int(round(cut_frac * L))))
+    x, kw = _inputs(B=1, H=2, L=L, d=4, seed=seed, gate=gate)
+    rng = np.random.default_rng(seed + 1)
+    dout = rng.standard_normal(x["v"].shape)
+    G = rng.standard_normal(kw["state_in"].shape) if with_G else None
+    whole_f = ref.lizard_forward(**x, window=window, gate=gate, **kw)
+    whole_b = ref.lizard_backward(**x, dout=dout, window=window, gate=gate, dstate_out=G, **kw)
+    P = min(window, cut)
+    x1, x2 = _part(x, 0, cut), _part(x, cut, None)
+    S_cut = ref.lizard_forward(**x1, window=window, gate=gate, **kw)["state_out"]
+    pre = {"k_prefix": x["k"][:, :, cut - P:cut], "v_prefix": x["v"][:, :, cut - P:cut]}
+    kw2 = dict(kw, state_in=S_cut)
+    f2 = ref.lizard_forward(**x2, window=window, gate=gate, **pre, **kw2)
+    np.testing.assert_allclose(f2["o"], whole_f["o"][:, :, cut:], rtol=1e-10, atol=1e-11)
+    b2 = ref.lizard_backward(**x2, dout=dout[:, :, cut:], window=window, gate=gate, dstate_out=G, **pre, **kw2)
+    b1 = ref.lizard_backward(**x1, dout=dout[:, :, :cut], window=window, gate=gate,
+                             dstate_out=b2["dstate_in"], **kw)
+    dk1, dv1 = b1["dk"].copy(), b1["dv"].copy()
+    dk1[:, :, cut - P:] += b2["dk_prefix"]
+    dv1[:, :, cut - P:] += b2["dv_prefix"]
+    np.testing.assert_allclose(np.concatenate([dk1, b2["dk"]], axis=2), whole_b["dk"], rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(np.concatenate([dv1, b2["dv"]], axis=2), whole_b["dv"], rtol=1e-10, atol=1e-11)
+    for key in ("dq", "dg"):
+        np.testing.assert_allclose(np.concatenate([b1[key], b2[key]], axis=2), whole_b[key], rtol=1e-10,
+                                   atol=1e-11, err_msg=key)
+    np.testing.assert_allclose(b1["dstate_in"], whole_b["dstate_in"], rtol=1e-10, atol=1e-11)
