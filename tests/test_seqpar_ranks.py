@@ -114,6 +114,7 @@ def _run(world, cuts, gate):
     (2, [0, 13, L], "dim"),
     (3, [0, 9, 18, L], "dim"),
     (3, [0, 4, 20, L], "scalar"),     # a segment exactly one window long
+    (4, [0, 5, 12, 22, L], "dim"),    # four uneven segments
 ])
 def test_split_forward_equals_the_whole_forward(world, cuts, gate):
     got = _run(world, cuts, gate)
