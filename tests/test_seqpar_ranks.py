@@ -1,5 +1,5 @@
 """The sequence-parallel forward's exchange logic on the CPU: one process per
-rank over gloo, world sizes 2 and 3.  The compute steps are the oracle's
+rank over gloo, world sizes 2, 3 and 4.  The compute steps are the oracle's
 (a test stand-in passed as `ops`; the product's default ops are the CUDA
 library); what is tested is the driver: halo send/receive, the all-gather
 of segment summaries, each rank's chain, and that the segments' outputs put
