@@ -1,7 +1,5 @@
 // Forward with its scratch in a static device array, for callers that
 // cannot allocate device memory (see lizard_attn_fwd_noalloc in lizard.h).
-#include <mutex>
-
 #include "../../include/lizard.h"
 
 namespace {
@@ -11,22 +9,13 @@ namespace {
 // the device address comes from cudaGetSymbolAddress below.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[LIZARD_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void *g_addr[kMaxDevices] = {};
-
-// Device address of the scratch on the current device, looked up once per
-// device with that device current.  Null on failure.
+// Device address of the scratch on the current device, looked up on every
+// call with that device current (so a context that was torn down and made
+// again never sees a stale address).  Null on failure.
 void *scratch_address() {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_addr[dev]) {
-    void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
-    g_addr[dev] = p;
-  }
-  return g_addr[dev];
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+  return p;
 }
 
 }  // namespace
@@ -44,12 +33,17 @@ extern "C" lizard_status lizard_attn_fwd_noalloc(const lizard_fwd_args *args, li
   if (need > LIZARD_NOALLOC_SCRATCH_BYTES) return LIZARD_ERR_UNSUPPORTED;
   void *scratch = scratch_address();
   if (!scratch) return LIZARD_ERR_CUDA;
-  // The status word at the start of a workspace must start at zero; the
-  // rest of the scratch is written before it is read by every kernel.
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(scratch, 0, 256, s) != cudaSuccess) return LIZARD_ERR_CUDA;
+  // lizard_attn_fwd clears the status word at the start of the scratch
+  // itself before its first kernel; every other byte of the scratch is
+  // written before it is read.
   lizard_fwd_args a = *args;
   a.workspace = scratch;
   a.workspace_bytes = LIZARD_NOALLOC_SCRATCH_BYTES;
   return lizard_attn_fwd(&a, stream);
+}
+
+extern "C" lizard_status lizard_noalloc_status(lizard_stream_t stream) {
+  void *scratch = scratch_address();
+  if (!scratch) return LIZARD_ERR_CUDA;
+  return lizard_workspace_status(scratch, stream);
 }

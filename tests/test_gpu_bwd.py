@@ -158,6 +158,23 @@ def test_train_step_full_size_sampled_heads(lz, impl):
             check(f"{name}[{b},{h}]", got[name][b:b + 1, h:h + 1], r[name], "bf16")
 
 
+@pytest.mark.parametrize("gate", ["dim", "scalar"])
+def test_parameter_grads_full_length_every_sequence(lz, gate):
+    """The per-head parameter gradients at the training step's full length and
+    batch (B=8, L=2048, d=128; two heads keep the oracle to seconds): they sum
+    fp32 atomics over 8 x 2048 tokens, so they are compared with the oracle
+    over every (b, h), with the per-token gradients, on the tensor-core path."""
+    w = Workload("params_full", B=8, H=2, L=2048, d=128, dtype="bf16", seed=17, kind="train",
+                 gate=gate)
+    inp = make_inputs(w)
+    got = _run(lz, to_device(inp), w, lz.IMPL_TC)
+    assert lz.workspace_status(got["workspace"]) == lz.OK
+    want = oracle_backward(inp, window=w.window, tau=w.gate_temp)
+    for name in ("dmeta_k", "dmeta_v", "dfmap_wq", "dfmap_wk", "dalpha", "dg", "dq", "dk", "dv",
+                 "dstate_in"):
+        check(f"{name} ({gate} gate)", got[name], want[name], "bf16")
+
+
 def test_persistent_kernels_walk_ragged_tiles_across_sequences(lz):
     """256 sequences of a ragged length (three 128-token tiles, the last one
     44 tokens): the persistent backward kernels give every CTA a run of

@@ -7,7 +7,7 @@ import pytest
 import torch
 
 from gated_linear_sliding_chunkwise_b200.synth import WORKLOADS, Workload, make_inputs, random_alpha
-from lizard_testutil import check, oracle_backward, oracle_forward, to64, to_device
+from lizard_testutil import check, oracle_backward, oracle_forward, report, to64, to_device
 from oracle import lizard_ref as ref
 
 pytestmark = pytest.mark.gpu
@@ -146,4 +146,5 @@ def test_feature_map_weight_gradients_keep_their_cancellation(lz, gate):
     for name in ("dfmap_wq", "dfmap_wk", "dg", "dstate_in"):
         g_, r_ = to64(got[name]), want[name]
         rel = float(np.max(np.abs(g_ - r_)) / np.max(np.abs(r_)))
+        report(f"PARITY guard {name} ({gate} gate) normwise={rel:.3e}")
         assert rel <= 8e-3, f"{name}: {rel:.2e}"
