@@ -118,6 +118,22 @@ def kernel_model(name, w, N, BH):
     return table.get(name, (0, 0))
 
 
+def kernel_io(dom, per, w, N, BH, peaks, args):
+    """The dominant kernel's own input/output rate: every array it reads or
+    writes (workspace intermediates included, each counted once) over its
+    launch time.  These are the bytes of this decomposition into kernels,
+    not the step's algorithmic bytes, so they are reported apart from the
+    step-level roofline."""
+    iob, iofl = kernel_model(dom, w, N, BH)
+    dt = per[dom] / 1e3
+    out = {"kernel": dom, "ms_per_launch": per[dom], "io_bytes": iob,
+           "io_gbs": iob / dt / 1e9, "io_frac_of_hbm": iob / dt / 1e9 / peaks["hbm_gbs"],
+           "tflops": iofl / dt / 1e12, "tflops_frac_of_bf16": iofl / dt / 1e12 / peaks["bf16_tflops"],
+           "traffic": MEASURED_TRAFFIC.get(dom) if args.kernels in ("auto", "tc") else None,
+           "modeled_step_io_bytes": sum(kernel_model(n, w, N, BH)[0] for n in per)}
+    return out
+
+
 # ------------------------------------------------------------- clocks -----
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples during the timed region."""
@@ -178,9 +194,9 @@ class ClockSampler:
 # -------------------------------------------------------------- helpers ----
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch on the
 # train_step workload (B=8, H=32, L=2048), from an ncu capture of the current
-# kernel build.
+# kernel build ("step" = the sum over every kernel of one training step).
+# Kernels changed since their capture are left out.
 MEASURED_TRAFFIC = {
-    "tc_gla_bwd_tile_kernel": 1.121389e9 + 1.023010e9,
 }
 
 
@@ -216,6 +232,19 @@ def barrier(world):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
+
+
+DATA = "synthetic (seeded N(0,1)/8 q,k,v; N(0,1) gate logits and dout)"
+
+
+def train_config(w, world, kernels):
+    """The headline workload's config, shared by both arms."""
+    return {"workload": "train_step: lizard_attn_fwd + lizard_attn_bwd",
+            "B": w.B, "H": w.H, "L": w.L, "d": w.d, "chunk": w.chunk,
+            "window": w.window, "M": w.M, "global_batch": w.B * world,
+            "seq_len": w.L, "parallelism": f"dp{world} (independent replicas)",
+            "kernels": kernels,
+            "l2": "inputs larger than L2 (q,k,v,g,dout = 5 x 134 MB per step)"}
 
 
 # ------------------------------------------------------------ our arm -----
@@ -292,36 +321,24 @@ def run_ours(args, rank, world, local):
             t = statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
             per[n] = per.get(n, 0.0) + t
     dom = max(per, key=per.get)
-    dbytes, dflops = kernel_model(dom, w, N, BH)
-    dt = per[dom] / 1e3
-    ai = dflops / max(dbytes, 1)
-    if dom.endswith("_simt") or dom in ("prep_kernel", "swa_bwd_q", "swa_bwd_kv", "finish_bwd",
-                                         "meta_grad_kernel", "gate_grad_kernel", "gate_prep_kernel"):
-        # CUDA-core kernels: fp32 FMA peak from unit counts and clock
-        alu_peak = SM_COUNT * FP32_LANES_PER_SM * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
-        ridge = alu_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
-        if ai >= ridge:
-            roof = {"bound": "alu", "achieved": dflops / dt / 1e12, "peak": alu_peak,
-                    "unit": "TFLOP/s"}
-        else:
-            roof = {"bound": "hbm", "achieved": dbytes / dt / 1e9, "peak": peaks["hbm_gbs"],
-                    "unit": "GB/s"}
-    else:
-        ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
-        if ai >= ridge:
-            roof = {"bound": "tensor", "achieved": dflops / dt / 1e12,
-                    "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
-        else:
-            roof = {"bound": "hbm", "achieved": dbytes / dt / 1e9, "peak": peaks["hbm_gbs"],
-                    "unit": "GB/s"}
+    kio = kernel_io(dom, per, w, N, BH, peaks, args)
+    # Step-level roofline: the training step's algorithmic bytes (q, k, v, g
+    # and dout in, o, dq, dk, dv and dg out, q, k, v, g read again: 3840 B per
+    # token-head at d = 128) over the measured step time, against the HBM
+    # peak (the step's arithmetic intensity, 126 FLOP/B, is below the bf16
+    # ridge of about 249 FLOP/B).
+    step_bytes = N * by["train"]
+    roof = {"bound": "hbm", "achieved": step_bytes / (ms_max / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
+            "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    # DRAM bytes (read + write) of one ncu capture of the kernel on this
-    # workload, per launch; kernels changed since their capture are left out
-    roof["traffic"] = MEASURED_TRAFFIC.get(dom) if args.kernels in ("auto", "tc") else None
-    roof["kernel"] = dom
-    roof["ms_per_launch"] = per[dom]
+    roof["traffic"] = MEASURED_TRAFFIC.get("step") if args.kernels in ("auto", "tc") else None
+    roof["scope"] = ("one training step (every kernel of lizard_attn_fwd + lizard_attn_bwd); "
+                     "achieved = 3840 B per token-head x B*H*L / ms_per_step")
+    roof["algorithmic_bytes"] = step_bytes
+    roof["floor_ms"] = step_bytes / (peaks["hbm_gbs"] * 1e9) * 1e3
     roof["peak_source"] = peaks["source"]
     kernels = {n: round(t, 4) for n, t in per.items()}
+
 
     # end to end: pinned host inputs in, gradients out, every step.  Three
     # streams: the inputs of step i + 1 go up and the gradients of step i come
@@ -405,6 +422,8 @@ def run_ours(args, rank, world, local):
     decode = None if args.no_decode else run_decode(args, lz, dev, rank, world, peaks)
     fwd_long = None if args.no_fwd_long else run_forward(args, lz, dev, rank, world, peaks,
                                                          "long_fwd_16k", max(K, 5))
+    fwd_layer = None if args.no_fwd_layer else run_forward(args, lz, dev, rank, world, peaks,
+                                                           "llama8b_layer_fwd", max(K, 5))
     variants = None if args.no_variants else run_variants(args, lz, dev, rank, world, peaks,
                                                           max(min(K, 30), 5))
 
@@ -412,25 +431,21 @@ def run_ours(args, rank, world, local):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded N(0,1)/8 q,k,v; N(0,1) gate logits and dout)",
-        "config": {"workload": "train_step: lizard_attn_fwd + lizard_attn_bwd",
-                   "B": w.B, "H": w.H, "L": w.L, "d": w.d, "chunk": w.chunk,
-                   "window": w.window, "M": w.M, "global_batch": w.B * world,
-                   "seq_len": w.L, "parallelism": f"dp{world} (independent replicas)",
-                   "kernels": args.kernels,
-                   "l2": "inputs larger than L2 (q,k,v,g,dout = 5 x 134 MB per step)"},
+        "data": DATA,
+        "config": train_config(w, world, args.kernels),
         "tflops": tflops, "tflops_frac_of_bf16_peak": tflops / peaks["bf16_tflops"],
         "hbm_floor_ms": (N * by["train"]) / (peaks["hbm_gbs"] * 1e9) * 1e3,
-        "roofline": roof, "kernel_ms": kernels,
+        "roofline": roof, "kernel_io": kio, "kernel_ms": kernels,
         "kernel_timing": "per-kernel CUDA events on the launching stream, in a second pass of the same steps "
                          "with every kernel in order (the timed steps run independent backward kernels "
                          "side by side)",
         "gpu_launches": K * (len(fwd_names) + len(bwd_names)),
         "clocks": clk, "e2e": e2e, "decode": decode, "fwd_long_16k": fwd_long,
+        "fwd_llama8b_layer": fwd_layer,
         "variants": variants,
     }
     if rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(inp, w, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget, seed=w.seed + rank)
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -472,11 +487,13 @@ def run_forward(args, lz, dev, rank, world, peaks, name, steps):
            "tflops_frac_of_bf16_peak": tfl / peaks["bf16_tflops"],
            "hbm_gbs": gbs, "hbm_frac": gbs / (world * peaks["hbm_gbs"]),
            "kernel_ms": {n: round(t, 4) for n, t in per.items()}, "launches": len(names)}
-    if len(names) == 1:
-        out["roofline"] = {"bound": "hbm", "achieved": by / (per[names[0]] / 1e3) / 1e9,
-                           "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                           "frac": by / (per[names[0]] / 1e3) / 1e9 / peaks["hbm_gbs"],
-                           "kernel": names[0]}
+    # the forward's algorithmic bytes (q, k, v, g in, o out: 1280 B per
+    # token-head) over the whole call's time; arithmetic intensity 117 FLOP/B,
+    # below the bf16 ridge, so HBM bounds it
+    out["roofline"] = {"bound": "hbm", "achieved": gbs / world, "peak": peaks["hbm_gbs"],
+                       "unit": "GB/s", "frac": gbs / (world * peaks["hbm_gbs"]),
+                       "floor_ms": by / (peaks["hbm_gbs"] * 1e9) * 1e3,
+                       "scope": "one lizard_attn_fwd call (all its kernels)"}
     return out
 
 
@@ -632,70 +649,52 @@ def run_decode(args, lz, dev, rank, world, peaks):
 
 
 # ---------------------------------------------------------- CPU oracle ----
-def cpu_baseline(inp, w, budget_s=15.0, pairs=None):
-    """Time the fp64 oracle's forward + backward on whole sampled sequences
-    of the same workload, on this host; report layer tokens/s."""
-    import numpy as np
-    from oracle import lizard_ref as ref
+def _oracle_timer(*opts):
+    """Run the oracle timing harness (oracle/cpu_time.py) in a fresh process
+    that never touches a GPU and forks one worker per host core; returns its
+    JSON result."""
+    cmd = [sys.executable, "-m", "oracle.cpu_time", *map(str, opts)]
+    r = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=900)
+    if r.returncode != 0:
+        raise RuntimeError("oracle timing failed: " + r.stderr[-2000:])
+    return json.loads(r.stdout.strip().splitlines()[-1])
 
-    pairs = pairs or [(0, 0), (1, 1), (2, 2), (3, 3), (4, 4), (5, 5), (6, 6), (7, 7)]
-    done = 0
-    t0 = time.perf_counter()
-    for (b, h) in pairs:
-        f = {k: inp[k][b:b + 1, h:h + 1].double().numpy() for k in ("q", "k", "v", "g", "dout")}
-        p = {k: inp[k][h:h + 1].double().numpy() for k in ("fmap_wq", "fmap_wk", "meta_k", "meta_v", "alpha")}
-        kw = dict(window=w.window, tau=w.gate_temp, **p)
-        ref.lizard_forward(f["q"], f["k"], f["v"], f["g"], **kw)
-        ref.lizard_backward(f["q"], f["k"], f["v"], f["g"], f["dout"], **kw)
-        done += 1
-        if time.perf_counter() - t0 > budget_s:
-            break
-    dt = time.perf_counter() - t0
-    token_heads = done * w.L
-    return {"value": token_heads / w.H / dt, "unit": "tokens/s", "cores": 1,
-            "host_cores_available": len(os.sched_getaffinity(0)), "kind": "oracle",
-            "sample": f"{done} whole (batch, head) sequences of L={w.L} (fp64 NumPy "
-                      f"forward + backward), {dt:.1f} s; tokens/s counts a token of all "
-                      f"H={w.H} heads, i.e. token-heads / {w.H}"}
+
+def cpu_baseline(w, budget_s=15.0, seed=None):
+    """Time the fp64 oracle's forward + backward on whole sequences of the
+    same workload, on every host core; report layer tokens/s."""
+    r = _oracle_timer("--workload", w.name, "--budget", budget_s,
+                      *(("--seed", seed) if seed is not None else ()))
+    return {"value": r["token_heads_per_s"] / w.H, "unit": "tokens/s", "cores": r["cores"],
+            "host_cores_available": r["host_cores_available"], "kind": "oracle",
+            "sample": f"{r['sequences']} whole (batch, head) sequences of L={w.L} (fp64 NumPy "
+                      f"forward + backward, one process per core), {r['seconds']:.1f} s; tokens/s "
+                      f"counts a token of all H={w.H} heads, i.e. token-heads / {w.H}"}
 
 
 # ------------------------------------------------------ reference arm -----
 def run_reference(args, rank, world):
     """The oracle as it stands, timed on the host cores over bounded samples
-    of the same workload (rank 0 only)."""
+    of the same workload (rank 0 only): every step runs one (batch, head)
+    sequence's first 256 tokens on each core."""
     if rank != 0:
         return
-    from gated_linear_sliding_chunkwise_b200.synth import WORKLOADS, make_inputs
-    from oracle import lizard_ref as ref
+    from gated_linear_sliding_chunkwise_b200.synth import WORKLOADS
 
     w = WORKLOADS["train_step"]
-    inp = make_inputs(w, B=1, H=1)            # one whole sequence per step
-    L = 256                                   # bounded sample: the first 256 tokens
-    f = {k: inp[k][:, :, :L].double().numpy() for k in ("q", "k", "v", "g", "dout")}
-    p = {k: inp[k].double().numpy() for k in ("fmap_wq", "fmap_wk", "meta_k", "meta_v", "alpha")}
-    kw = dict(window=w.window, tau=w.gate_temp, **p)
-
-    def step():
-        ref.lizard_forward(f["q"], f["k"], f["v"], f["g"], **kw)
-        ref.lizard_backward(f["q"], f["k"], f["v"], f["g"], f["dout"], **kw)
-
-    for _ in range(args.warmup):
-        step()
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        step()
-    dt = (time.perf_counter() - t0) / args.steps
-    value = L / w.H / dt
-    sample = (f"one (batch, head) sequence, first {L} tokens of the train_step workload, "
-              f"fp64 NumPy forward + backward per step; tokens/s counts a token of all "
-              f"H={w.H} heads")
+    L = 256
+    r = _oracle_timer("--workload", w.name, "--tokens", L, "--steps", args.steps,
+                      "--warmup", args.warmup)
+    value = r["token_heads_per_s"] / w.H
+    sample = (f"each step: {r['cores']} (batch, head) sequences of the train_step workload, one per "
+              f"host core, first {L} tokens each, fp64 NumPy forward + backward; tokens/s counts a "
+              f"token of all H={w.H} heads")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "train_step (oracle sample)", "B": w.B, "H": w.H,
-                       "L": w.L, "d": w.d, "chunk": w.chunk, "window": w.window, "M": w.M},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1,
+            "ms_per_step": r["sec_per_step"] * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": DATA,
+            "config": train_config(w, world, args.kernels),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": r["cores"],
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -716,6 +715,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-fwd-long", action="store_true")
+    ap.add_argument("--no-fwd-layer", action="store_true",
+                    help="skip the Llama-3-8B-shaped layer forward (B=4 H=32 L=2048)")
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the stage-1 step and scalar-gate timings")
     ap.add_argument("--only", choices=["train", "fwd", "bwd", "decode"], default="train",
