@@ -645,7 +645,7 @@ def run_decode(args, lz, dev, rank, world, peaks):
     return {"value": gbs, "unit": "GB/s", "frac_of_hbm": gbs / (world * peaks["hbm_gbs"]),
             "us_per_step": us, "steps": n, "bytes_per_step": step_bytes,
             "workload": f"decode: B={w.B} H={w.H} d={w.d} window {w.window} M={w.M}, pos {w.decode_pos}",
-            "launches_per_step": 2}
+            "launches_per_step": 1}
 
 
 # ---------------------------------------------------------- CPU oracle ----

@@ -68,6 +68,8 @@ bool swa_on(const lizard_fwd_args *a) { return a->branch != LIZARD_BRANCH_GLA_ON
 // them (the identity map) the GLA branch takes the portable kernels.
 bool fmap_weights(const lizard_fwd_args *a) { return a->fmap_wq != nullptr && a->fmap_wk != nullptr; }
 
+size_t nch32(const lizard_fwd_args *a) { return (a->L + lz::kBwdC - 1) / lz::kBwdC; }
+
 bool fwd_uses_tc(const lizard_fwd_args *a) {
   const bool ok = lz::tc_fwd_supported(a->dk, a->dv, a->window, a->M, a->dtype == LIZARD_BF16) &&
                   (fmap_weights(a) || a->branch == LIZARD_BRANCH_SWA_ONLY);
@@ -75,16 +77,53 @@ bool fwd_uses_tc(const lizard_fwd_args *a) {
   return a->impl == LIZARD_IMPL_AUTO && ok;
 }
 
+// Exact fallback of the tensor-core GLA branch: the per-sequence marks
+// (right after the status header, so that the call's first memset clears
+// both), each sequence's slot, each slot's sequence, then per slot the
+// portable kernels' scratch: `per_slot` bytes.
+struct FallbackLayout {
+  size_t flags, slot_of, seq_of_slot, scratch, per_slot, end;
+};
+FallbackLayout fallback_layout(size_t off, const lizard_fwd_args *a, size_t per_slot) {
+  const size_t BH = (size_t)a->B * a->H;
+  FallbackLayout f{};
+  f.flags = off; off += up(BH * sizeof(uint32_t));
+  f.slot_of = off; off += up(BH * sizeof(int));
+  f.seq_of_slot = off; off += up(lz::kFallbackSlots * sizeof(int));
+  f.per_slot = per_slot;
+  f.scratch = off; off += lz::kFallbackSlots * per_slot;
+  f.end = off;
+  return f;
+}
+int fallback_slots(const lizard_fwd_args *a) {
+  const int BH = a->B * a->H;
+  return BH < lz::kFallbackSlots ? BH : lz::kFallbackSlots;
+}
+// bytes the call's first memset clears: the status header and, with the
+// exact fallback, the per-sequence marks that follow it
+size_t cleared_bytes(const lizard_fwd_args *a, bool fallback) {
+  return fallback ? kHeader + up((size_t)a->B * a->H * sizeof(uint32_t)) : sizeof(uint32_t);
+}
+
 // Forward workspace: the status header, plus fp32 scratch for the portable path.
 struct FwdLayout {
   size_t phq, phk, a, o_gla, total;
+  bool fallback;
+  FallbackLayout fb;
 };
-FwdLayout fwd_layout(const lizard_fwd_args *a) {
+FwdLayout fwd_layout(const lizard_fwd_args *a, bool stage1 = false) {
   const size_t N = (size_t)a->B * a->H * a->L;
   const size_t nd = up(N * a->dk * sizeof(float));
   FwdLayout l{};
   size_t off = kHeader;
   if (fwd_uses_tc(a)) {
+    // the stage-1 step keeps its loss in the tensor-core epilogue: no fallback
+    l.fallback = gla_on(a) && !stage1;
+    if (l.fallback) {
+      const size_t Ld = up((size_t)a->L * a->dk * sizeof(float));
+      l.fb = fallback_layout(off, a, 3 * Ld);   // phi_q, phi_k and a of one sequence
+      off = l.fb.end;
+    }
     l.phq = off;   // segment states of the tensor-core path
     off += up(lz::tc_fwd_workspace_bytes(a->B * a->H, a->L));
   } else if (gla_on(a)) {
@@ -112,8 +151,10 @@ bool bwd_gla_uses_tc(const lizard_fwd_args *a, int impl) {
 struct BwdLayout {
   size_t phq, phk, a, sprev, dphq, dphk, da, dv_gla, dq_swa, dk_swa, dv_swa, lse, Dterm, dsm, pm, snap_s,
       snap_ds, e32, gr, w16, kap, total;
+  bool fallback;
+  FallbackLayout fb;
 };
-BwdLayout bwd_layout(const lizard_fwd_args *a, int impl) {
+BwdLayout bwd_layout(const lizard_fwd_args *a, int impl, bool stage1 = false) {
   const size_t BH = (size_t)a->B * a->H;
   const size_t N = BH * a->L;
   const size_t nd = up(N * a->dk * sizeof(float));
@@ -121,6 +162,15 @@ BwdLayout bwd_layout(const lizard_fwd_args *a, int impl) {
   const size_t nch = (a->L + lz::kBwdC - 1) / lz::kBwdC;
   BwdLayout l{};
   size_t off = kHeader;
+  if (gla_on(a) && bwd_gla_uses_tc(a, impl) && !stage1) {
+    // exact fallback: per slot phi_q, phi_k, a, the chunk states and kap of
+    // the portable backward
+    const size_t Ld = up((size_t)a->L * a->dk * sizeof(float));
+    const size_t per = 3 * Ld + up(nch * a->dk * a->dv * sizeof(float)) + up(a->dk * sizeof(float));
+    l.fallback = true;
+    l.fb = fallback_layout(off, a, per);
+    off = l.fb.end;
+  }
   if (gla_on(a) && bwd_gla_uses_tc(a, impl)) {
     const size_t snap = up(lz::tc_gla_bwd_snapshot_bytes((int)BH, a->L));
     l.snap_s = off; off += snap;
@@ -275,7 +325,7 @@ lizard_status Plan::run(cudaStream_t s, void *const *events, int nev) const {
 // forms in its epilogue (null otherwise).
 void fwd_plan(const lizard_fwd_args *a, void *ws, cudaStream_t s, Plan &plan, const void *target = nullptr,
               void *dmse = nullptr, float *loss = nullptr) {
-  const FwdLayout lay = fwd_layout(a);
+  const FwdLayout lay = fwd_layout(a, target != nullptr);
   const int BH = a->B * a->H, D = a->dk;
   const bool bf16 = a->dtype == LIZARD_BF16;
   if (fwd_uses_tc(a)) {
@@ -284,12 +334,39 @@ void fwd_plan(const lizard_fwd_args *a, void *ws, cudaStream_t s, Plan &plan, co
                     static_cast<uint32_t *>(ws), at<void>(ws, lay.phq), BH, a->H, a->L, a->M, a->window,
                     a->branch, 1.f / a->gate_temp, scale_of(a), scalar_gate(a), target, dmse, loss,
                     a->k_prefix, a->v_prefix, a->prefix_len};
+    const FallbackLayout fb = lay.fb;
+    const int K = fallback_slots(a);
+    uint32_t *status = static_cast<uint32_t *>(ws);
+    if (lay.fallback) {
+      t.seqflag = at<uint32_t>(ws, fb.flags);
+      t.slot_of = at<int>(ws, fb.slot_of);
+    }
     if (gla_on(a)) plan.add("gate_prep_kernel", [=](cudaStream_t s) { return lz::launch_tc_fwd(t, 3, s); });
+    if (lay.fallback)
+      plan.add("assign_slots_kernel", [=](cudaStream_t s) {
+        return lz::launch_assign_slots(at<uint32_t>(ws, fb.flags), at<int>(ws, fb.slot_of), at<int>(ws, fb.seq_of_slot),
+                                       BH, K, status, s);
+      });
     if (gla_on(a) && lz::tc_fwd_stage_count(BH, a->L) > 1) {   // segment start states (GLA only)
       plan.add("tc_fwd_kernel(state pass)", [=](cudaStream_t s) { return lz::launch_tc_fwd(t, 0, s); });
       plan.add("seg_combine_kernel", [=](cudaStream_t s) { return lz::launch_tc_fwd(t, 1, s); });
     }
     plan.add("tc_fwd_kernel", [=](cudaStream_t s) { return lz::launch_tc_fwd(t, 2, s); });
+    if (lay.fallback) {
+      // the GLA branch of the marked sequences, exactly, on the portable
+      // kernels (one grid slot each; a slot with no sequence exits at once)
+      // scratch: phi_q, phi_k, a, each [K][L][D] fp32; the GLA kernel adds
+      // its output to o in place
+      const size_t arr = (size_t)K * (fb.per_slot / 3);
+      const int *seq = at<int>(ws, fb.seq_of_slot);
+      lz::PrepArgs pa{a->q, a->k, a->g, a->fmap_wq, a->fmap_wk, at<float>(ws, fb.scratch),
+                      at<float>(ws, fb.scratch + arr), at<float>(ws, fb.scratch + 2 * arr),
+                      a->H, a->L, 1.f / a->gate_temp, scalar_gate(a), seq};
+      plan.add("prep_kernel(exact fallback)", [=](cudaStream_t s) { return lz::launch_prep(pa, K, D, bf16, s); });
+      lz::GlaFwdArgs ga{pa.phq, pa.phk, pa.a, a->v, a->state_in, nullptr, a->state_out, a->L, seq, a->o};
+      plan.add("gla_fwd_simt(exact fallback)",
+               [=](cudaStream_t s) { return lz::launch_gla_fwd_simt(ga, K, D, bf16, s); });
+    }
     return;
   }
   float *o_gla = nullptr;
@@ -308,9 +385,9 @@ void fwd_plan(const lizard_fwd_args *a, void *ws, cudaStream_t s, Plan &plan, co
   plan.add("swa_mix_simt", [=](cudaStream_t s) { return lz::launch_swa_mix_simt(sa, BH, D, bf16, s); });
 }
 
-void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan) {
+void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan, bool stage1 = false) {
   const lizard_fwd_args *a = &b->fwd;
-  const BwdLayout lay = bwd_layout(a, b->impl);
+  const BwdLayout lay = bwd_layout(a, b->impl, stage1);
   const int BH = a->B * a->H, D = a->dk;
   const bool bf16 = a->dtype == LIZARD_BF16;
   const float inv_tau = 1.f / a->gate_temp;
@@ -325,9 +402,17 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan) {
     void *snap_s = at<void>(ws, lay.snap_s);
     float *e32 = at<float>(ws, lay.e32), *gr = at<float>(ws, lay.gr);
     uint32_t *status = static_cast<uint32_t *>(ws);
+    uint32_t *flags = lay.fallback ? at<uint32_t>(ws, lay.fb.flags) : nullptr;
     plan.add("gate_prep_kernel",
              [=](cudaStream_t s) { return lz::launch_gate_prep(a->g, nullptr, e32, gr, status, BH, a->L, inv_tau, f.scalar_gate != 0,
-                                               s); });
+                                               s, flags); });
+    if (lay.fallback) {
+      const FallbackLayout fb = lay.fb;
+      const int K = fallback_slots(a);
+      plan.add("assign_slots_kernel", [=](cudaStream_t s) {
+        return lz::launch_assign_slots(flags, at<int>(ws, fb.slot_of), at<int>(ws, fb.seq_of_slot), BH, K, status, s);
+      });
+    }
     // the state copies beside the weight conversion and the reverse dS pass
     plan.fork();
     plan.add("tc_fwd_kernel(state copies)",
@@ -342,6 +427,30 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan) {
     plan.add("tc_gla_dstates_kernel", [=](cudaStream_t s) { return lz::launch_tc_gla_bwd(t, 0, s); });
     plan.join();
     plan.add("tc_gla_bwd_tile_kernel", [=](cudaStream_t s) { return lz::launch_tc_gla_bwd(t, 1, s); });
+    if (lay.fallback) {
+      // the GLA backward of the marked sequences, exactly, on the portable
+      // kernels: their dphi_q, dphi_k, dv and dstate_in replace what the
+      // tensor-core kernels wrote, and their per-token da goes to the dB
+      // array (the marked sequences' dg is formed from it at the end)
+      const FallbackLayout fb = lay.fb;
+      const int K = fallback_slots(a);
+      const int *seq = at<int>(ws, fb.seq_of_slot);
+      const size_t Ld = up((size_t)a->L * a->dk * sizeof(float));
+      const size_t o_phq = fb.scratch, o_phk = o_phq + K * Ld, o_a = o_phk + K * Ld, o_sp = o_a + K * Ld;
+      const size_t o_kap = o_sp + K * up(nch32(a) * a->dk * a->dv * sizeof(float));
+      lz::PrepArgs pa{a->q, a->k, a->g, a->fmap_wq, a->fmap_wk, at<float>(ws, o_phq), at<float>(ws, o_phk),
+                      at<float>(ws, o_a), a->H, a->L, inv_tau, scalar_gate(a), seq};
+      plan.add("prep_kernel(exact fallback)", [=](cudaStream_t s) { return lz::launch_prep(pa, K, D, bf16, s); });
+      float *kap = b->dstate_out ? at<float>(ws, o_kap) : nullptr;
+      lz::GlaStatesArgs sa{pa.phk, pa.a, a->v, a->state_in, at<float>(ws, o_sp), a->L, b->dstate_out, kap, seq};
+      plan.add("gla_states_simt(exact fallback)",
+               [=](cudaStream_t s) { return lz::launch_gla_states(sa, K, D, bf16, s); });
+      lz::GlaBwdArgs ga{pa.phq, pa.phk, pa.a, a->v, b->dout, at<float>(ws, o_sp), at<float>(ws, lay.dphq),
+                        at<float>(ws, lay.dphk), at<float>(ws, lay.da), at<float>(ws, lay.dv_gla), b->dstate_in,
+                        a->L, b->dstate_out, kap, seq};
+      plan.add("gla_bwd_simt(exact fallback)",
+               [=](cudaStream_t s) { return lz::launch_gla_bwd_simt(ga, K, D, bf16, s); });
+    }
   } else if (g) {
     lz::PrepArgs pa{a->q, a->k, a->g, a->fmap_wq, a->fmap_wk, at<float>(ws, lay.phq), at<float>(ws, lay.phk),
                     at<float>(ws, lay.a), a->H, a->L, inv_tau, scalar_gate(a)};
@@ -399,6 +508,11 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan) {
       t.dk_out = b->dk;
       t.dv_out = b->dv;
     }
+    t.k_prefix = a->k_prefix;
+    t.v_prefix = a->v_prefix;
+    t.dk_prefix = b->dk_prefix;
+    t.dv_prefix = b->dv_prefix;
+    t.P = a->prefix_len;
     plan.add("tc_swa_bwd_q_kernel", [=](cudaStream_t s) { return lz::launch_tc_swa_bwd(t, 0, s); });
     if (a->M > 0 && (b->dmeta_k || b->dmeta_v)) {   // beside the dk / dv pass, after the dq pass's terms
       plan.fork();
@@ -409,10 +523,12 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan) {
   } else if (w) {
     lz::SwaBwdQArgs qa{a->q, a->k, a->v, b->dout, a->meta_k, a->meta_v, a->alpha,
                        at<float>(ws, lay.dq_swa), at<float>(ws, lay.lse), at<float>(ws, lay.Dterm),
-                       b->dmeta_k, b->dmeta_v, b->dalpha, a->H, a->L, a->window, a->M, scale_of(a)};
+                       b->dmeta_k, b->dmeta_v, b->dalpha, a->H, a->L, a->window, a->M, scale_of(a),
+                       a->k_prefix, a->v_prefix, a->prefix_len};
     plan.add("swa_bwd_q", [=](cudaStream_t s) { return lz::launch_swa_bwd_q(qa, BH, D, bf16, s); });
     lz::SwaBwdKVArgs ka{a->q, a->k, a->v, b->dout, a->alpha, at<float>(ws, lay.lse), at<float>(ws, lay.Dterm),
-                        at<float>(ws, lay.dk_swa), at<float>(ws, lay.dv_swa), a->H, a->L, a->window, scale_of(a)};
+                        at<float>(ws, lay.dk_swa), at<float>(ws, lay.dv_swa), a->H, a->L, a->window, scale_of(a),
+                        a->k_prefix, a->v_prefix, b->dk_prefix, b->dv_prefix, a->prefix_len};
     plan.add("swa_bwd_kv", [=](cudaStream_t s) { return lz::launch_swa_bwd_kv(ka, BH, D, bf16, s); });
   }
   if (!fused) {
@@ -423,6 +539,14 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan) {
   }
   if (gla_tc && !fused)
     plan.add("gate_grad_kernel", [=](cudaStream_t s) { return lz::launch_tc_gla_bwd(tg, 2, s); });
+  if (lay.fallback) {   // dg of the marked sequences from the exact da (after the gate-gradient pass)
+    const int K = fallback_slots(a);
+    const int *seq = at<int>(ws, lay.fb.seq_of_slot);
+    const float *da = at<float>(ws, lay.da);
+    plan.add("slot_dg_kernel", [=](cudaStream_t s) {
+      return lz::launch_slot_dg(b->dg, da, a->g, seq, K, a->L, D, inv_tau, scalar_gate(a) != 0, bf16, s);
+    });
+  }
 }
 
 }  // namespace
@@ -468,7 +592,7 @@ lizard_status lizard_attn_fwd(const lizard_fwd_args *a, lizard_stream_t stream) 
     }
     return LIZARD_OK;
   }
-  if (cudaMemsetAsync(a->workspace, 0, sizeof(uint32_t), s) != cudaSuccess) return LIZARD_ERR_CUDA;
+  if (cudaMemsetAsync(a->workspace, 0, cleared_bytes(a, lay.fallback), s) != cudaSuccess) return LIZARD_ERR_CUDA;
   Plan plan;
   fwd_plan(a, a->workspace, s, plan);
   return plan.run(s, a->launch_events, a->n_launch_events);
@@ -489,8 +613,10 @@ static lizard_status check_bwd(const lizard_bwd_args *b) {
       (b->dfmap_wk && !f.fmap_wk))
     return LIZARD_ERR_INVALID_ARG;
   if (b->dstate_out && !gla_on(&f)) return LIZARD_ERR_INVALID_ARG;   // no final state without the GLA branch
+  if (f.prefix_len == 0 && (b->dk_prefix || b->dv_prefix)) return LIZARD_ERR_INVALID_ARG;
   const void *ptrs[] = {b->dout, b->dq, b->dk, b->dv, b->dg, b->dmeta_k, b->dmeta_v,
-                        b->dfmap_wq, b->dfmap_wk, b->dalpha, b->dstate_in, b->dstate_out};
+                        b->dfmap_wq, b->dfmap_wk, b->dalpha, b->dstate_in, b->dstate_out,
+                        b->dk_prefix, b->dv_prefix};
   for (const void *p : ptrs)
     if (!ok_ptr(p)) return LIZARD_ERR_INVALID_ARG;
   return LIZARD_OK;
@@ -530,6 +656,15 @@ static cudaError_t bwd_zero_outputs(const lizard_bwd_args *b, cudaStream_t s) {
     if (z.p && z.n && (e = cudaMemsetAsync(z.p, 0, z.n, s)) != cudaSuccess) return e;
   const size_t BHdd = (size_t)BH * a->dk * a->dv * sizeof(float);
   if ((a->L == 0 || !gla_on(a)) && b->dstate_in) e = cudaMemsetAsync(b->dstate_in, 0, BHdd, s);
+  if (e != cudaSuccess) return e;
+  // the prefix is read only by the anchor branch: without it (or without
+  // queries) its gradients are zero
+  if (a->prefix_len > 0 && (a->L == 0 || !swa_on(a)) && b->dk_prefix && b->dv_prefix) {
+    const size_t esz = a->dtype == LIZARD_BF16 ? 2 : 4;
+    const size_t n = (size_t)BH * a->prefix_len * a->dk * esz;
+    if ((e = cudaMemsetAsync(b->dk_prefix, 0, n, s)) != cudaSuccess) return e;
+    e = cudaMemsetAsync(b->dv_prefix, 0, n, s);
+  }
   return e;
 }
 
@@ -539,14 +674,15 @@ lizard_status lizard_attn_bwd(const lizard_bwd_args *b, lizard_stream_t stream) 
   const lizard_fwd_args *a = &b->fwd;
   if (b->impl == LIZARD_IMPL_TC && swa_on(a) && !bwd_swa_uses_tc(a, b->impl)) return LIZARD_ERR_UNSUPPORTED;
   if (b->impl == LIZARD_IMPL_TC && gla_on(a) && !bwd_gla_uses_tc(a, b->impl)) return LIZARD_ERR_UNSUPPORTED;
-  if (a->prefix_len != 0) return LIZARD_ERR_UNSUPPORTED;   // forward only
+  // with a prefix, its key and value gradients are outputs of the call
+  if (a->prefix_len > 0 && (!b->dk_prefix || !b->dv_prefix)) return LIZARD_ERR_INVALID_ARG;
   const BwdLayout lay = bwd_layout(a, b->impl);
   if (!b->workspace || b->workspace_bytes < lay.total) return LIZARD_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (bwd_zero_outputs(b, s) != cudaSuccess) return LIZARD_ERR_CUDA;
   if (a->L == 0) return LIZARD_OK;
   void *ws = b->workspace;
-  if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), s) != cudaSuccess) return LIZARD_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, cleared_bytes(a, lay.fallback), s) != cudaSuccess) return LIZARD_ERR_CUDA;
   Plan plan;
   bwd_plan(b, ws, s, plan);
   return plan.run(s, b->launch_events, b->n_launch_events);
@@ -567,7 +703,7 @@ struct S1Layout {
 S1Layout s1_layout(const lizard_stage1_args *a) {
   const lizard_bwd_args *b = &a->bwd;
   const lizard_fwd_args *f = &b->fwd;
-  const size_t fw = fwd_layout(f).total, bw = bwd_layout(f, b->impl).total;
+  const size_t fw = fwd_layout(f, true).total, bw = bwd_layout(f, b->impl, true).total;
   const size_t nel = (size_t)f->B * f->H * f->L * f->dv, esz = f->dtype == LIZARD_BF16 ? 2 : 4;
   S1Layout l{};
   size_t off = up(fw > bw ? fw : bw);
@@ -618,7 +754,7 @@ void stage1_plan(const lizard_stage1_args *a, S1Views &v, void *ws, cudaStream_t
     plan.add("mse_kernel", [=](cudaStream_t s) { return lz::launch_mse(f->o, target, dmse, loss, nel, bf16, s); });
   }
   v.b.dout = dmse;
-  bwd_plan(&v.b, ws, s, plan);
+  bwd_plan(&v.b, ws, s, plan, true);
 }
 
 }  // namespace
@@ -655,7 +791,7 @@ lizard_status lizard_stage1_step(const lizard_stage1_args *a, lizard_stream_t st
   if (f->impl == LIZARD_IMPL_TC && !fwd_uses_tc(f)) return LIZARD_ERR_UNSUPPORTED;
   if (b->impl == LIZARD_IMPL_TC && swa_on(f) && !bwd_swa_uses_tc(f, b->impl)) return LIZARD_ERR_UNSUPPORTED;
   if (b->impl == LIZARD_IMPL_TC && gla_on(f) && !bwd_gla_uses_tc(f, b->impl)) return LIZARD_ERR_UNSUPPORTED;
-  if (f->prefix_len != 0) return LIZARD_ERR_UNSUPPORTED;   // forward only
+  if (f->prefix_len != 0) return LIZARD_ERR_UNSUPPORTED;   // whole sequences only
   const S1Layout lay = s1_layout(a);
   if (!b->workspace || b->workspace_bytes < lay.total) return LIZARD_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

@@ -14,6 +14,8 @@
 //     as 16-byte vectors, all in flight together.
 // The state update S <- diag(gamma) S + phi_k v^T and the read-out
 // o = S^T phi_q happen in the same pass over the registers.
+#include <atomic>
+
 #include "common.cuh"
 #include "lizard_internal.h"
 
@@ -24,6 +26,29 @@ constexpr int kDecWB = 128;   // window slots staged in shared memory per block
 __global__ void advance_pos_kernel(int64_t *pos, int B) {
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b < B) pos[b] += 1;
+}
+
+// The pos increment folded into the step: every CTA arrives on a counter
+// once it has read all the pos values it uses (one thread per CTA, after a
+// barrier behind those reads); the last to arrive adds 1 to every pos and
+// resets the counter.  Launches take their counter from a ring of
+// kPosSlots, so steps in flight on different streams do not share one.
+constexpr int kPosSlots = 64;
+__device__ unsigned int g_pos_arrivals[kPosSlots];
+
+LZ_DEV void pos_arrive(const DecodeArgs &p) {
+  if (!p.pos_inc) return;
+  __threadfence();
+  const unsigned int ctas = gridDim.x * gridDim.y * gridDim.z;
+  if (atomicAdd(&g_pos_arrivals[p.pos_slot], 1u) == ctas - 1) {
+    g_pos_arrivals[p.pos_slot] = 0u;
+    for (int b = 0; b < p.pos_B; ++b) p.pos_inc[b] += 1;
+  }
+}
+
+int next_pos_slot() {
+  static std::atomic<unsigned int> ctr{0};
+  return (int)(ctr.fetch_add(1u) % kPosSlots);
 }
 
 LZ_DEV void cp_async16(void *smem, const void *gmem) {
@@ -94,6 +119,10 @@ __global__ void __launch_bounds__(256, 2) decode_kernel(DecodeArgs p) {
   const T *gs = static_cast<const T *>(p.g) + (size_t)bh * (p.scalar_gate ? 1 : D);
   float *S = p.state + (size_t)bh * D * D;
   const long long pos = p.pos[b];
+  if (p.pos_inc) {   // every thread has read pos: this CTA arrives
+    __syncthreads();
+    if (tid == 0) pos_arrive(p);
+  }
   const int W = p.window;
   const int slot = (int)(pos % W);
   const int n = (int)(pos + 1 < (long long)W ? pos + 1 : W);
@@ -489,6 +518,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_stream_kernel(const __g
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
   __syncthreads();
+  // with the increment folded in, every pair's (n, slot) was read above
+  if (tid == 0) pos_arrive(p);
 
   if (warp == kConsumers / 32) {
     // ------------------------------------------------------- producer ---
@@ -834,9 +865,16 @@ cudaError_t launch_decode_stream(const DecodeArgs &a, int B, int64_t *pos, cudaS
   const int BH = B * a.H;
   const int run = (BH + sms[dev] - 1) / sms[dev];   // pairs per CTA
   const int grid = (BH + run - 1) / run;
-  decode_stream_kernel<<<grid, kDecThreads, smem, s>>>(a, B, run);
+  // The increment rides on the step when every CTA reads its pos values at
+  // its start (runs of at most kMaxRunPairs pairs); else a second kernel.
+  DecodeArgs d = a;
+  const bool fold = run <= kMaxRunPairs;
+  d.pos_inc = fold ? pos : nullptr;
+  d.pos_slot = fold ? next_pos_slot() : 0;
+  d.pos_B = B;
+  decode_stream_kernel<<<grid, kDecThreads, smem, s>>>(d, B, run);
   e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  if (e != cudaSuccess || fold) return e;
   advance_pos_kernel<<<(B + 127) / 128, 128, 0, s>>>(pos, B);
   return cudaGetLastError();
 }
@@ -891,10 +929,11 @@ static cudaError_t launch_decode_t(const DecodeArgs &a, int B, int64_t *pos, cud
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) configured[dev] = smem;
   }
-  k<<<B * a.H, 256, smem, s>>>(a);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  advance_pos_kernel<<<(B + 127) / 128, 128, 0, s>>>(pos, B);
+  DecodeArgs d = a;   // the pos increment rides on the step
+  d.pos_inc = pos;
+  d.pos_slot = next_pos_slot();
+  d.pos_B = B;
+  k<<<B * a.H, 256, smem, s>>>(d);
   return cudaGetLastError();
 }
 

@@ -7,6 +7,12 @@
 
 namespace lz {
 
+// Exact fallback of the tensor-core path (sequences whose in-tile decay
+// spread leaves the tensor-core range): when seq_of_slot is set, the portable
+// GLA kernels below run one grid slot k per entry, on sequence
+// bh = seq_of_slot[k] (nothing when it is negative); their scratch arrays
+// (phi, a, o_gla, chunk states, kap) are indexed by the slot k, their inputs
+// and outputs by bh.
 struct PrepArgs {
   const void *q, *k, *g;
   const float *wq, *wk;
@@ -14,6 +20,7 @@ struct PrepArgs {
   int H, L;
   float inv_tau;
   int scalar_gate;   // g holds one logit per (token, head): [B*H][L]
+  const int *seq_of_slot;
 };
 
 struct GlaFwdArgs {
@@ -23,6 +30,8 @@ struct GlaFwdArgs {
   float *o_gla;
   float *state_out;
   int L;
+  const int *seq_of_slot;
+  void *o_add;   // when set (with seq_of_slot): o[bh] += o_gla in the activation dtype, o_gla not written
 };
 
 struct SwaMixArgs {
@@ -47,6 +56,11 @@ struct DecodeArgs {
   int H, window, M;
   float inv_tau, scale;
   int scalar_gate;   // g holds one logit per (batch, head): [B*H]
+  // Set by the launcher: when pos_inc is set, the last CTA to have read pos
+  // adds 1 to pos[0 .. B) (arrival counter pos_slot of the library's ring),
+  // so no second kernel is needed.
+  int64_t *pos_inc;
+  int pos_slot, pos_B;
 };
 
 // Backward (portable fp32 kernels).
@@ -60,6 +74,7 @@ struct GlaStatesArgs {
   // the final state's share of every token's log-decay gradient (null: none)
   const float *dstate_out;
   float *kap;
+  const int *seq_of_slot;
 };
 
 struct GlaBwdArgs {
@@ -71,6 +86,7 @@ struct GlaBwdArgs {
   int L;
   const float *dstate_out;   // [BH][D][D] gradient into the final state, or null (zero)
   const float *kap;          // [BH][D] from gla_states_simt when dstate_out is set: the reverse sum's start
+  const int *seq_of_slot;
 };
 
 struct SwaBwdQArgs {
@@ -80,6 +96,8 @@ struct SwaBwdQArgs {
   float *dmeta_k, *dmeta_v, *dalpha;   // accumulated atomically; may be null
   int H, L, window, M;
   float scale;
+  const void *k_prefix, *v_prefix;     // [B*H][P][D]: the P tokens before token 0 (P = 0: none)
+  int P;
 };
 
 struct SwaBwdKVArgs {
@@ -88,6 +106,11 @@ struct SwaBwdKVArgs {
   float *dk_swa, *dv_swa;
   int H, L, window;
   float scale;
+  // Key/value prefix (P = 0: none) and the gradients of its keys and values,
+  // [B*H][P][D] in the activation dtype (the anchor branch's part only).
+  const void *k_prefix, *v_prefix;
+  void *dk_prefix, *dv_prefix;
+  int P;
 };
 
 struct FinishBwdArgs {
@@ -133,6 +156,12 @@ struct TcFwdArgs {
   // sum_v G[i][v] S_L[i][v] (null: none)
   const float *dstate_out;
   float *kap;
+  // Exact fallback (exact_fallback.cu): the gate prep marks sequences whose
+  // in-tile decay spread leaves the tensor-core range in seqflag [BH] (zeroed
+  // by the caller; null: it sets the status word's RANGE bit instead), and
+  // the passes leave the GLA branch out for sequences with slot_of[bh] >= 0.
+  uint32_t *seqflag;
+  const int *slot_of;
 };
 
 struct TcSwaBwdArgs {
@@ -150,6 +179,11 @@ struct TcSwaBwdArgs {
   const void *xq_part, *xk_part;   // bf16 [B*H*L][128] feature-map parts dx_q, dx_k
   const float *dv_gla;             // fp32 [B*H*L][128] value part
   void *dq_out, *dk_out, *dv_out;  // bf16 dq, dk, dv
+  // Key/value prefix of the anchor window ([B*H][P][128] bf16, P <= window;
+  // P = 0: none) and the gradients of its keys and values (bf16, same shape).
+  const void *k_prefix, *v_prefix;
+  void *dk_prefix, *dv_prefix;
+  int P;
 };
 
 struct TcGlaBwdArgs {
@@ -225,7 +259,15 @@ cudaError_t launch_tc_state_snapshots(const TcFwdArgs &a, void *snap, const floa
 cudaError_t launch_mse(const void *o, const void *target, void *dout, float *loss, size_t n, bool bf16,
                        cudaStream_t s);
 cudaError_t launch_gate_prep(const void *g, void *E16, float *E32, float *r, uint32_t *status, int BH, int L,
-                             float inv_tau, bool scalar_gate, cudaStream_t s);
+                             float inv_tau, bool scalar_gate, cudaStream_t s, uint32_t *seqflag = nullptr);
+// Exact fallback for sequences outside the tensor-core decay range
+// (exact_fallback.cu): up to kFallbackSlots marked sequences per call get a
+// slot (slot_of [BH], seq_of_slot [K]); the others set the RANGE bit.
+constexpr int kFallbackSlots = 4;
+cudaError_t launch_assign_slots(const uint32_t *flags, int *slot_of, int *seq_of_slot, int BH, int K,
+                                uint32_t *status, cudaStream_t s);
+cudaError_t launch_slot_dg(float *dg, const float *da, const void *g, const int *seq_of_slot, int K, int L, int D,
+                           float inv_tau, bool scalar_gate, bool bf16, cudaStream_t s);
 // stage 0: reverse dS pass, 1: per-tile gradients, 2: gate-logit gradient
 cudaError_t launch_tc_gla_bwd(const TcGlaBwdArgs &a, int stage, cudaStream_t s);
 // tensor-core finish: bf16, d = 128, both feature maps present

@@ -36,21 +36,28 @@ __global__ void __launch_bounds__(256) gla_states_simt(GlaStatesArgs p) {
   float *Bb = Kb + C * D;         // [C][D]
   float *Vb = Bb + C * D;         // [C][D]
   float *dec = Vb + C * D;        // [D]
-  const int bh = blockIdx.x, tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  int bh = blockIdx.x;
+  const int sb = blockIdx.x;   // scratch row: the grid slot
+  if (p.seq_of_slot) {
+    bh = p.seq_of_slot[sb];
+    if (bh < 0) return;
+  }
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   const T *vsrc = static_cast<const T *>(p.v);
   const int nch = (p.L + C - 1) / C;
   for (int i = tid; i < D * D; i += 256) S[i] = p.state_in ? p.state_in[(size_t)bh * D * D + i] : 0.f;
   __syncthreads();
   for (int c = 0; c < nch; ++c) {
     const int c0 = c * C, n = min(C, p.L - c0);
-    float *dst = p.sprev + ((size_t)bh * nch + c) * D * D;
+    float *dst = p.sprev + ((size_t)sb * nch + c) * D * D;
     for (int i = tid; i < D * D; i += 256) dst[i] = S[i];
-    const size_t base = ((size_t)bh * p.L + c0) * D;
+    const size_t base = ((size_t)sb * p.L + c0) * D;    // scratch
+    const size_t ibase = ((size_t)bh * p.L + c0) * D;   // inputs
     for (int e = tid; e < C * D; e += 256) {
       const bool ok = e / D < n;
       Kb[e] = ok ? p.phk[base + e] : 0.f;
       Bb[e] = ok ? p.a[base + e] : 0.f;
-      Vb[e] = ok ? to_f32(vsrc[base + e]) : 0.f;
+      Vb[e] = ok ? to_f32(vsrc[ibase + e]) : 0.f;
     }
     __syncthreads();
     if (tid < D) {
@@ -89,7 +96,7 @@ __global__ void __launch_bounds__(256) gla_states_simt(GlaStatesArgs p) {
     const float *G = p.dstate_out + ((size_t)bh * D + tid) * D;
     float s = 0.f;
     for (int v = 0; v < D; ++v) s = fmaf(G[v], S[tid * D + v], s);
-    p.kap[(size_t)bh * D + tid] = s;
+    p.kap[(size_t)sb * D + tid] = s;
   }
 }
 
@@ -111,7 +118,13 @@ __global__ void __launch_bounds__(256) gla_bwd_simt(GlaBwdArgs p) {
   float *A = Ob + C * D;               // [C][C]
   float *dA = A + C * C;               // [C][C]
   float *dec = dA + C * C;             // [D]
-  const int bh = blockIdx.x, tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  int bh = blockIdx.x;
+  const int sb = blockIdx.x;   // scratch row: the grid slot
+  if (p.seq_of_slot) {
+    bh = p.seq_of_slot[sb];
+    if (bh < 0) return;
+  }
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   const T *vsrc = static_cast<const T *>(p.v);
   const T *osrc = static_cast<const T *>(p.dout);
   const int nch = (p.L + C - 1) / C;
@@ -119,18 +132,19 @@ __global__ void __launch_bounds__(256) gla_bwd_simt(GlaBwdArgs p) {
   for (int i = tid; i < D * SP; i += 256)
     dS[i] = (p.dstate_out && i % SP < D) ? p.dstate_out[(size_t)bh * D * D + (i / SP) * D + i % SP] : 0.f;
   // reverse running sum of dB (thread i < D), from the final state's share
-  float carry = (p.kap && tid < D) ? p.kap[(size_t)bh * D + tid] : 0.f;
+  float carry = (p.kap && tid < D) ? p.kap[(size_t)sb * D + tid] : 0.f;
   __syncthreads();
   for (int c = nch - 1; c >= 0; --c) {
     const int c0 = c * C, n = min(C, p.L - c0);
-    const size_t base = ((size_t)bh * p.L + c0) * D;
-    const float *sp_src = p.sprev + ((size_t)bh * nch + c) * D * D;
+    const size_t sbase = ((size_t)sb * p.L + c0) * D;   // scratch
+    const size_t base = ((size_t)bh * p.L + c0) * D;    // inputs and outputs
+    const float *sp_src = p.sprev + ((size_t)sb * nch + c) * D * D;
     for (int e = tid; e < D * D; e += 256) Sp[(e / D) * SP + e % D] = sp_src[e];
     for (int e = tid; e < C * D; e += 256) {
       const bool ok = e / D < n;
-      Qb[e] = ok ? p.phq[base + e] : 0.f;
-      Kb[e] = ok ? p.phk[base + e] : 0.f;
-      Bb[e] = ok ? p.a[base + e] : 0.f;
+      Qb[e] = ok ? p.phq[sbase + e] : 0.f;
+      Kb[e] = ok ? p.phk[sbase + e] : 0.f;
+      Bb[e] = ok ? p.a[sbase + e] : 0.f;
       Vb[e] = ok ? to_f32(vsrc[base + e]) : 0.f;
       Ob[e] = ok ? to_f32(osrc[base + e]) : 0.f;
     }
@@ -324,10 +338,13 @@ __global__ void __launch_bounds__(256) swa_bwd_q(SwaBwdQArgs p) {
     G[e] = ok ? to_f32(gs[base + (size_t)t0 * D + e]) : 0.f;   // raw dout
   }
   if (tid < kSwaT) { mrow[tid] = kNegBig; lrow[tid] = 0.f; }
-  const int kstart = max(0, t0 - p.window + 1);
+  // keys j < 0 come from the prefix (row P + j of k_prefix / v_prefix)
+  const int kstart = max(-p.P, t0 - p.window + 1);
   const int kend = t0 + nq;
   const int hasm = p.M > 0 ? 1 : 0;
   const int nblk = (kend - kstart + kSwaT - 1) / kSwaT + hasm;
+  const T *kps = static_cast<const T *>(p.k_prefix);
+  const T *vps = static_cast<const T *>(p.v_prefix);
 
   auto load_block = [&](int blk, bool &meta, int &ks0) {
     meta = hasm && blk == 0;
@@ -340,9 +357,13 @@ __global__ void __launch_bounds__(256) swa_bwd_q(SwaBwdQArgs p) {
           kv = p.meta_k[((size_t)h * p.M + jj) * D + i];
           vv = p.meta_v ? p.meta_v[((size_t)h * p.M + jj) * D + i] : 0.f;
         }
-      } else if (ks0 + jj < kend) {
+      } else if (ks0 + jj < kend && ks0 + jj >= 0) {
         kv = to_f32(ks[base + (size_t)(ks0 + jj) * D + i]);
         vv = to_f32(vs[base + (size_t)(ks0 + jj) * D + i]);
+      } else if (ks0 + jj < kend) {   // -P <= j < 0
+        const size_t pr = ((size_t)bh * p.P + (p.P + ks0 + jj)) * D + i;
+        kv = to_f32(kps[pr]);
+        vv = to_f32(vps[pr]);
       }
       Kb[e] = kv;
       Vb[e] = vv;
@@ -537,6 +558,8 @@ __global__ void __launch_bounds__(256) swa_bwd_q(SwaBwdQArgs p) {
 
 // --------------------------------------------- anchor branch: dk, dv -----
 // Key tile [j0, j0+64); the queries that see it are [j0, j0+63+window).
+// With a key/value prefix of P tokens, the first ceil(P/64) tiles cover the
+// prefix keys -P .. -1 (j0 < 0; their gradients go to dk_prefix / dv_prefix).
 template <typename T, int D>
 __global__ void __launch_bounds__(256) swa_bwd_kv(SwaBwdKVArgs p) {
   constexpr int VT = D / 16;
@@ -550,19 +573,32 @@ __global__ void __launch_bounds__(256) swa_bwd_kv(SwaBwdKVArgs p) {
   float *dSm = P + kSwaT * KP;         // [64 q][KP]
   float *lse = dSm + kSwaT * KP;       // [64]
   float *Dq = lse + kSwaT;             // [64]
-  const int bh = blockIdx.y, h = bh % p.H, j0 = blockIdx.x * kSwaT;
+  const int npre = (p.P + kSwaT - 1) / kSwaT;
+  const int bh = blockIdx.y, h = bh % p.H, j0 = ((int)blockIdx.x - npre) * kSwaT;
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   const T *qs = static_cast<const T *>(p.q);
   const T *ks = static_cast<const T *>(p.k);
   const T *vs = static_cast<const T *>(p.v);
   const T *gs = static_cast<const T *>(p.dout);
+  const T *kps = static_cast<const T *>(p.k_prefix);
+  const T *vps = static_cast<const T *>(p.v_prefix);
   const size_t base = (size_t)bh * p.L * D;
   const float alpha = p.alpha ? p.alpha[h] : 1.f;
   const int nk = min(kSwaT, p.L - j0);
+  const int jlo = -p.P;                 // the first key there is
   for (int e = tid; e < kSwaT * D; e += 256) {
-    const bool ok = e / D < nk;
-    Kt[e] = ok ? to_f32(ks[base + (size_t)j0 * D + e]) : 0.f;
-    Vt[e] = ok ? to_f32(vs[base + (size_t)j0 * D + e]) : 0.f;
+    const int j = j0 + e / D, i = e % D;
+    float kv = 0.f, vv = 0.f;
+    if (j >= 0 && e / D < nk) {
+      kv = to_f32(ks[base + (size_t)j * D + i]);
+      vv = to_f32(vs[base + (size_t)j * D + i]);
+    } else if (j < 0 && j >= jlo) {
+      const size_t pr = ((size_t)bh * p.P + (p.P + j)) * D + i;
+      kv = to_f32(kps[pr]);
+      vv = to_f32(vps[pr]);
+    }
+    Kt[e] = kv;
+    Vt[e] = vv;
   }
   float dk[4][VT], dv[4][VT];
 #pragma unroll
@@ -570,7 +606,7 @@ __global__ void __launch_bounds__(256) swa_bwd_kv(SwaBwdKVArgs p) {
 #pragma unroll
     for (int c = 0; c < VT; ++c) { dk[a_][c] = 0.f; dv[a_][c] = 0.f; }
   const int qend = min(p.L, j0 + nk - 1 + p.window);   // exclusive
-  for (int q0 = j0; q0 < qend; q0 += kSwaT) {
+  for (int q0 = max(j0, 0); q0 < qend; q0 += kSwaT) {
     const int nq = min(kSwaT, qend - q0);
     __syncthreads();
     for (int e = tid; e < kSwaT * D; e += 256) {
@@ -610,7 +646,7 @@ __global__ void __launch_bounds__(256) swa_bwd_kv(SwaBwdKVArgs p) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const int jj = tx * 4 + c, j = j0 + jj;
-          const bool ok = tq < nq && jj < nk && j <= t && j > t - p.window;
+          const bool ok = tq < nq && jj < nk && j >= jlo && j <= t && j > t - p.window;
           const float pr = ok ? expf(s[a_][c] * p.scale - lse[tq]) : 0.f;
           P[tq * KP + jj] = pr;
           dSm[tq * KP + jj] = pr * (dp[a_][c] - Dq[tq]);
@@ -634,13 +670,22 @@ __global__ void __launch_bounds__(256) swa_bwd_kv(SwaBwdKVArgs p) {
   }
 #pragma unroll
   for (int a_ = 0; a_ < 4; ++a_) {
-    const int jj = ty * 4 + a_;
-    if (jj < nk)
+    const int jj = ty * 4 + a_, j = j0 + jj;
+    if (j >= 0 && jj < nk) {
 #pragma unroll
       for (int c = 0; c < VT; ++c) {
-        p.dk_swa[base + (size_t)(j0 + jj) * D + tx * VT + c] = dk[a_][c] * p.scale;
-        p.dv_swa[base + (size_t)(j0 + jj) * D + tx * VT + c] = dv[a_][c];
+        p.dk_swa[base + (size_t)j * D + tx * VT + c] = dk[a_][c] * p.scale;
+        p.dv_swa[base + (size_t)j * D + tx * VT + c] = dv[a_][c];
       }
+    } else if (j < 0 && j >= jlo) {   // a prefix key: its final gradient (anchor part only)
+      T *dkp = static_cast<T *>(p.dk_prefix), *dvp = static_cast<T *>(p.dv_prefix);
+      const size_t pr = ((size_t)bh * p.P + (p.P + j)) * D;
+#pragma unroll
+      for (int c = 0; c < VT; ++c) {
+        dkp[pr + tx * VT + c] = from_f32<T>(dk[a_][c] * p.scale);
+        dvp[pr + tx * VT + c] = from_f32<T>(dv[a_][c]);
+      }
+    }
   }
 }
 
@@ -868,7 +913,7 @@ static cudaError_t swakv_t(const SwaBwdKVArgs &a, int BH, cudaStream_t s) {
   const size_t smem = (4 * (size_t)kSwaT * D + 2 * kSwaT * (kSwaT + 1) + 2 * kSwaT) * sizeof(float);
   cudaError_t e = prep_launch(swa_bwd_kv<T, D>, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((a.L + kSwaT - 1) / kSwaT, BH);
+  dim3 grid((a.P + kSwaT - 1) / kSwaT + (a.L + kSwaT - 1) / kSwaT, BH);
   swa_bwd_kv<T, D><<<grid, 256, smem, s>>>(a);
   return cudaGetLastError();
 }

@@ -35,7 +35,13 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepArgs p) {
   extern __shared__ float sm[];
   float* Wq = sm;              // [D][F]
   float* Wk = sm + D * F;      // [D][F]
-  const int bh = blockIdx.y, h = bh % p.H;
+  int bh = blockIdx.y;
+  const int sb = blockIdx.y;          // scratch row: the grid slot
+  if (p.seq_of_slot) {
+    bh = p.seq_of_slot[sb];
+    if (bh < 0) return;
+  }
+  const int h = bh % p.H;
   const int t0 = blockIdx.x * kPrepTok;
   const bool has_wq = p.wq != nullptr, has_wk = p.wk != nullptr;
   if (has_wq)
@@ -50,13 +56,14 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepArgs p) {
   for (int tt = warp; tt < kPrepTok; tt += 8) {
     const int t = t0 + tt;
     if (t >= p.L) break;
-    const size_t row = ((size_t)bh * p.L + t) * D;
+    const size_t row = ((size_t)bh * p.L + t) * D;    // inputs
+    const size_t srow = ((size_t)sb * p.L + t) * D;   // scratch outputs
     // scalar gate: one logit per token and head, the same decay for every dimension
     const float a_tok = p.scalar_gate ? log_decay(to_f32(gs[(size_t)bh * p.L + t]), p.inv_tau) : 0.f;
 #pragma unroll
     for (int j = 0; j < XJ; ++j) {
       const int i = lane + 32 * j;
-      p.a[row + i] = p.scalar_gate ? a_tok : log_decay(to_f32(gs[row + i]), p.inv_tau);
+      p.a[srow + i] = p.scalar_gate ? a_tok : log_decay(to_f32(gs[row + i]), p.inv_tau);
     }
 #pragma unroll
     for (int which = 0; which < 2; ++which) {
@@ -69,7 +76,7 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepArgs p) {
       for (int j = 0; j < XJ; ++j) xr[j] = to_f32(xs[row + lane + 32 * j]);
       if (!has_w) {
 #pragma unroll
-        for (int j = 0; j < XJ; ++j) out[row + lane + 32 * j] = xr[j];
+        for (int j = 0; j < XJ; ++j) out[srow + lane + 32 * j] = xr[j];
         continue;
       }
       float z[ZJ];
@@ -103,8 +110,8 @@ __global__ void __launch_bounds__(256) prep_kernel(PrepArgs p) {
       const float ip = 1.f / sp, in_ = 1.f / sn;
 #pragma unroll
       for (int jj = 0; jj < ZJ; ++jj) {
-        out[row + lane + 32 * jj] = ep[jj] * ip;
-        out[row + F + lane + 32 * jj] = en[jj] * in_;
+        out[srow + lane + 32 * jj] = ep[jj] * ip;
+        out[srow + F + lane + 32 * jj] = en[jj] * in_;
       }
     }
   }
@@ -125,7 +132,12 @@ __global__ void __launch_bounds__(256) gla_fwd_simt(GlaFwdArgs p) {
   float* A = Vs + C * D;              // [C][C]
   float* dec = A + C * C;             // [D] exp(r): state decay over the chunk
   float* eq = dec + D;                // [D] multiplier turning P1 into phi_q exp(b)
-  const int bh = blockIdx.x;
+  int bh = blockIdx.x;
+  const int sb = blockIdx.x;          // scratch row: the grid slot
+  if (p.seq_of_slot) {
+    bh = p.seq_of_slot[sb];
+    if (bh < 0) return;
+  }
   const int tid = threadIdx.x;
   const int tx = tid & 15, ty = tid >> 4;
   const T* vsrc = static_cast<const T*>(p.v);
@@ -134,14 +146,15 @@ __global__ void __launch_bounds__(256) gla_fwd_simt(GlaFwdArgs p) {
   __syncthreads();
   for (int c0 = 0; c0 < p.L; c0 += C) {
     const int n = min(C, p.L - c0);
-    const size_t base = ((size_t)bh * p.L + c0) * D;
+    const size_t base = ((size_t)sb * p.L + c0) * D;    // scratch
+    const size_t ibase = ((size_t)bh * p.L + c0) * D;   // inputs
     for (int e = tid; e < C * D; e += 256) {
       const int t = e / D;
       const bool ok = t < n;
       P1[e] = ok ? p.phq[base + e] : 0.f;
       P2[e] = ok ? p.phk[base + e] : 0.f;
       P3[e] = ok ? p.a[base + e] : 0.f;
-      Vs[e] = ok ? to_f32(vsrc[base + e]) : 0.f;
+      Vs[e] = ok ? to_f32(vsrc[ibase + e]) : 0.f;
     }
     __syncthreads();
     float spread = 0.f;
@@ -217,9 +230,16 @@ __global__ void __launch_bounds__(256) gla_fwd_simt(GlaFwdArgs p) {
 #pragma unroll
       for (int a_ = 0; a_ < 4; ++a_) {
         const int t = ty * 4 + a_;
-        if (t < n)
+        if (t < n) {
+          if (p.o_add) {   // exact fallback: add to the output the anchor pass wrote
+            T *o = static_cast<T*>(p.o_add) + ibase + t * D + tx * VT;
 #pragma unroll
-          for (int c = 0; c < VT; ++c) p.o_gla[base + t * D + tx * VT + c] = acc[a_][c];
+            for (int c = 0; c < VT; ++c) o[c] = from_f32<T>(to_f32(o[c]) + acc[a_][c]);
+          } else {
+#pragma unroll
+            for (int c = 0; c < VT; ++c) p.o_gla[base + t * D + tx * VT + c] = acc[a_][c];
+          }
+        }
       }
     }
     __syncthreads();

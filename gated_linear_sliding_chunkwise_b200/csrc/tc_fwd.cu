@@ -101,6 +101,7 @@ struct Params {
   int nseg, tiles_per_seg;
   int P;                    // prefix tokens before token 0 (0: none)
   int inject;               // test hook: first wait on a barrier nothing completes
+  const int *slot_of;       // exact fallback: sequences with slot_of[bh] >= 0 leave the GLA branch out
   float inv_tau, scale;
   // stage-1 loss (target null: off): dmse = mse_grad (o - target), *loss += mse_loss sum (o - target)^2
   const __nv_bfloat16 *target;
@@ -215,7 +216,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
   const int bh = blockIdx.x, h = bh % p.H, seg = blockIdx.y;
   const float alpha = p.alpha ? p.alpha[h] : 1.f;
   constexpr bool full = KIND != K_STATE;
-  const bool gla = p.branch != 2, swa = full && p.branch != 1;
+  // a sequence taken by the exact fallback runs the anchor branch only here
+  const bool gla = p.branch != 2 && !(p.slot_of && p.slot_of[bh] >= 0), swa = full && p.branch != 1;
   const uint32_t sbase = smem_u32(sm);
   const int ntiles_all = (p.L + T - 1) / T;
   const int cbeg = seg * p.tiles_per_seg;
@@ -333,10 +335,38 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
     if (full) {
       // ---- full pass: the anchor softmax split between the groups (group 1
       //      the band chunks ch_lo, ch_lo + 2, ..., group 0 the others and
-      //      the meta logits), then one half of phi_q, phi_k per group
+      //      the meta logits), then one half of phi_q, phi_k per group.
+      //      The meta logits (CUDA cores, from X_q in shared memory) and the
+      //      tile's decay exp(r) are formed while MMA 1 runs.
+      float pmeta = kNegBig;
+      if (swa && wg == 0) {
+        // meta logits q . mk_m (scaled) into s_ml, four meta tokens per pass
+        for (int m0 = 0; m0 < p.M; m0 += 4) {
+          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+          for (int ch = 0; ch < 16; ++ch) {
+            float q8[8];
+            unpack8(*chunk_ptr(sm, R_XQ, row, ch), q8);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float4 a = *reinterpret_cast<const float4 *>(&s_mk[m0 + k][ch * 8]);
+              const float4 b = *reinterpret_cast<const float4 *>(&s_mk[m0 + k][ch * 8 + 4]);
+              acc[2 * k] = fmaf(q8[0], a.x, fmaf(q8[1], a.y, fmaf(q8[2], a.z, fmaf(q8[3], a.w, acc[2 * k]))));
+              acc[2 * k + 1] = fmaf(q8[4], b.x, fmaf(q8[5], b.y, fmaf(q8[6], b.z, fmaf(q8[7], b.w, acc[2 * k + 1]))));
+            }
+          }
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            if (m0 + k < p.M) {
+              const float l = (acc[2 * k] + acc[2 * k + 1]) * p.scale;
+              s_ml[m0 + k][row] = l;
+              pmeta = fmaxf(pmeta, l);
+            }
+        }
+      }
+      if (wg == 1 && gla) s_dec[row] = __expf(p.gate_r[((size_t)bh * ntiles_all + c) * D + row]);   // exp(r)
       ok &= mbar_wait(&bar_m1, par, err, ST_TIMEOUT);
       tc_fence_after();
-      if (wg == 1 && gla) s_dec[row] = __expf(p.gate_r[((size_t)bh * ntiles_all + c) * D + row]);   // exp(r)
       float lsum = 1.f, mx = 0.f;                 // row normaliser and max (scaled logits)
       // Logit column cl holds key t0 - T + cl.  Row r sees columns
       // [r + T + 1 - window, r + T] (and keys >= -P, P the prefix length),
@@ -351,35 +381,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       const int in_lo = 32 * w4 + 31 + T + 1 - p.window;   // interior chunk: 32 ch >= in_lo
       const int ch_first = ch_lo + 1 - wg;                 // this group's first chunk
       uint32_t pk[3][16];
+      // this group's logit chunks, read from TMEM once (the stage-1 instance,
+      // short of registers, reads them again for the exponentials)
+      constexpr int KEPT = LOSS ? 1 : 3;
+      float lv[KEPT][32];
       if (swa) {
-        float pmax = kNegBig;
-        if (wg == 0) {
-          // meta logits q . mk_m (scaled) into s_ml, four meta tokens per pass
-          for (int m0 = 0; m0 < p.M; m0 += 4) {
-            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-            for (int ch = 0; ch < 16; ++ch) {
-              float q8[8];
-              unpack8(*chunk_ptr(sm, R_XQ, row, ch), q8);
+        float pmax = pmeta;
 #pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const float4 a = *reinterpret_cast<const float4 *>(&s_mk[m0 + k][ch * 8]);
-                const float4 b = *reinterpret_cast<const float4 *>(&s_mk[m0 + k][ch * 8 + 4]);
-                acc[2 * k] = fmaf(q8[0], a.x, fmaf(q8[1], a.y, fmaf(q8[2], a.z, fmaf(q8[3], a.w, acc[2 * k]))));
-                acc[2 * k + 1] = fmaf(q8[4], b.x, fmaf(q8[5], b.y, fmaf(q8[6], b.z, fmaf(q8[7], b.w, acc[2 * k + 1]))));
-              }
-            }
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              if (m0 + k < p.M) {
-                const float l = (acc[2 * k] + acc[2 * k + 1]) * p.scale;
-                s_ml[m0 + k][row] = l;
-                pmax = fmaxf(pmax, l);
-              }
-          }
-        }
-        for (int ch = ch_first; ch <= ch_hi; ch += 2) {
-          float v[32];
+        for (int k = 0; k < 3; ++k) {
+          const int ch = ch_first + 2 * k;
+          if (ch > ch_hi) continue;
+          float *v = lv[LOSS ? 0 : k];
           tmem_ld32(tl + C_L + ch * 32, v);
           float m4[4] = {kNegBig, kNegBig, kNegBig, kNegBig};
           if (32 * ch >= in_lo && 32 * ch + 31 <= 32 * w4 + T && 32 * ch + cbase >= -p.P) {
@@ -407,8 +419,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         for (int k = 0; k < 3; ++k) {
           const int ch = ch_first + 2 * k;
           if (ch > ch_hi) continue;
-          float v[32];
-          tmem_ld32(tl + C_L + ch * 32, v);
+          const float *v = lv[LOSS ? 0 : k];
+          if (LOSS) tmem_ld32(tl + C_L + ch * 32, lv[0]);
           const bool inner = 32 * ch >= in_lo && 32 * ch + 31 <= 32 * w4 + T && 32 * ch + cbase >= -p.P;
 #pragma unroll
           for (int u = 0; u < 32; u += 2) {
@@ -728,7 +740,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
 template <bool SCALAR>
 __global__ void __launch_bounds__(256) gate_prep_kernel(const __nv_bfloat16 *g, __nv_bfloat16 *E16, float *E32,
                                                         float *rr, uint32_t *status, int L, int ntiles,
-                                                        float inv_tau) {
+                                                        float inv_tau, uint32_t *seqflag) {
   __shared__ float2 s_tot[8][32];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int i = blockIdx.x * 64 + 2 * lane, c = blockIdx.y, bh = blockIdx.z;
@@ -776,21 +788,24 @@ __global__ void __launch_bounds__(256) gate_prep_kernel(const __nv_bfloat16 *g, 
   if (w == 0) {   // carry = -r: the whole tile
     *reinterpret_cast<float2 *>(rr + ((size_t)bh * ntiles + c) * 128 + i) = make_float2(-carry.x, -carry.y);
     const float spread = fmaxf(carry.x - a[0].x, carry.y - a[0].y);   // sum over s > 0
-    if (spread > kMaxSpread) atomicOr(status, 2u);
+    if (spread > kMaxSpread) {
+      if (seqflag) seqflag[bh] = 1u;   // the exact fallback takes this sequence
+      else atomicOr(status, 2u);
+    }
   }
 }
 
 cudaError_t launch_gate_prep(const void *g, void *E16, float *E32, float *r, uint32_t *status, int BH, int L,
-                             float inv_tau, bool scalar_gate, cudaStream_t s) {
+                             float inv_tau, bool scalar_gate, cudaStream_t s, uint32_t *seqflag) {
   if (L == 0) return cudaSuccess;
   const int ntiles = (L + tc::kTileRows - 1) / tc::kTileRows;
   const dim3 grid(2, ntiles, BH);
   const __nv_bfloat16 *gp = static_cast<const __nv_bfloat16 *>(g);
   __nv_bfloat16 *e16 = static_cast<__nv_bfloat16 *>(E16);
   if (scalar_gate)
-    gate_prep_kernel<true><<<grid, 256, 0, s>>>(gp, e16, E32, r, status, L, ntiles, inv_tau);
+    gate_prep_kernel<true><<<grid, 256, 0, s>>>(gp, e16, E32, r, status, L, ntiles, inv_tau, seqflag);
   else
-    gate_prep_kernel<false><<<grid, 256, 0, s>>>(gp, e16, E32, r, status, L, ntiles, inv_tau);
+    gate_prep_kernel<false><<<grid, 256, 0, s>>>(gp, e16, E32, r, status, L, ntiles, inv_tau, seqflag);
   return cudaGetLastError();
 }
 
@@ -995,7 +1010,8 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, int stage, cudaStream_t s) {
   const bool gla = a.branch != 2 && a.g != nullptr;
   if (stage == 3) {
     if (!gla) return cudaSuccess;
-    return launch_gate_prep(a.g, w.e16, w.e32, w.r, a.status, a.BH, a.L, a.inv_tau, a.scalar_gate != 0, s);
+    return launch_gate_prep(a.g, w.e16, w.e32, w.r, a.status, a.BH, a.L, a.inv_tau, a.scalar_gate != 0, s,
+                            a.seqflag);
   }
   if (nseg > 1 && (stage == 0 || stage == 1) && !gla) return cudaSuccess;   // no state to carry
   if (nseg > 1 && stage == 1) {
@@ -1041,6 +1057,7 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, int stage, cudaStream_t s) {
   p.seg_start = w.seg_start;
   p.seg_state = w.seg_state;
   p.seg_decay = w.seg_decay;
+  p.slot_of = a.slot_of;
   p.H = a.H;
   p.L = a.L;
   p.M = a.M;

@@ -12,6 +12,11 @@
 //                       dq, the log-normaliser, D and the per-row meta terms.
 // tc_swa_bwd_kv_kernel  one CTA per (sequence, 128-key block): the two query
 //                       tiles that see the block; dK and dV accumulate in TMEM.
+//
+// A key/value prefix of P <= window tokens before token 0 (a segment of a
+// longer sequence) enters the first query tile's band as its previous keys
+// and values, and adds one key block per sequence (keys -128 .. -1, of which
+// -P .. -1 exist) whose gradients go to dk_prefix / dv_prefix.
 // meta_grad_kernel      meta-token gradients: per head, sums over tokens.
 //
 // Every mbarrier wait is bounded; a wait that gives up sets the TIMEOUT bit
@@ -35,6 +40,7 @@ constexpr uint32_t ST_TIMEOUT = 1u;
 
 struct QParams {
   CUtensorMap mq, mk, mv, mo;
+  CUtensorMap mkp, mvp;       // key / value prefix [BH][P][D] (P > 0 only)
   CUtensorMap mdq;            // fp32 dq output (TMA stores)
   CUtensorMap mxq, mdqo;      // fused: bf16 GLA part dx_q (load), bf16 final dq (store)
   const float *meta_k, *meta_v, *alpha;
@@ -44,20 +50,24 @@ struct QParams {
   float scale;
   int fused;
   int BH;
+  int P;
 };
 
 struct KVParams {
   CUtensorMap mq, mk, mv, mo;
+  CUtensorMap mkp, mvp;       // key / value prefix [BH][P][D] (P > 0 only)
   CUtensorMap mdk, mdv;       // fp32 dk, dv outputs (TMA stores)
   CUtensorMap mxk, mdvg;      // fused: bf16 GLA part dx_k, fp32 GLA dv (loads)
   CUtensorMap mdko, mdvo;     // fused: bf16 final dk, dv (stores)
   const float *alpha, *lse, *Dterm;
   float *dk, *dv;
+  __nv_bfloat16 *dk_prefix, *dv_prefix;   // [BH][P][D] (P > 0 only)
   uint32_t *status;
   int H, L, window;
   float scale;
   int fused;
   int BH;
+  int P;
 };
 
 __device__ __forceinline__ void setup_cta(uint32_t *tmem_slot, uint64_t *bars, int nbars, int tid) {
@@ -118,9 +128,16 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
         tma_load_3d(sm + R_O + r * kReg, &p.mo, bar_tma, 64 * r, lt0, lbh);
       }
       if (early) {
-        tma_load_3d(sm + R_KP + r * kReg, &p.mk, bar_tma, 64 * r, lt0 - T, lbh);
+        // keys and values of the previous tile; before token 0, the prefix
+        // (its rows before the first prefix token read as zero)
+        if (lt0 == 0 && p.P > 0) {
+          tma_load_3d(sm + R_KP + r * kReg, &p.mkp, bar_tma, 64 * r, p.P - T, lbh);
+          tma_load_3d(sm + R_VP + r * kReg, &p.mvp, bar_tma, 64 * r, p.P - T, lbh);
+        } else {
+          tma_load_3d(sm + R_KP + r * kReg, &p.mk, bar_tma, 64 * r, lt0 - T, lbh);
+          tma_load_3d(sm + R_VP + r * kReg, &p.mv, bar_tma, 64 * r, lt0 - T, lbh);
+        }
         tma_load_3d(sm + R_K + r * kReg, &p.mk, bar_tma, 64 * r, lt0, lbh);
-        tma_load_3d(sm + R_VP + r * kReg, &p.mv, bar_tma, 64 * r, lt0 - T, lbh);
       }
       if (v_early ? early : late) tma_load_3d(sm + R_V + r * kReg, &p.mv, bar_tma, 64 * r, lt0, lbh);
     }
@@ -211,17 +228,18 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
     // 2. softmax over the band (see the forward): logit column cl holds key
     //    t0 - T + cl; warp w4 visits chunks ch_lo .. ch_hi, group wg the
     //    chunks ch_lo + wg, ch_lo + wg + 2, ...
+    //    (keys >= -P, P the prefix length)
     const int w4 = warp & 3, cbase = t0 - T;
-    const int lo_c = max(tq - p.window + 1, 0) - cbase, hi_c = tq - cbase;
+    const int lo_c = max(tq - p.window + 1, -p.P) - cbase, hi_c = tq - cbase;
     int ch_lo = (32 * w4 + T + 1 - p.window) >> 5;
-    if (cbase < 0) ch_lo = max(ch_lo, 4);
+    if (cbase < 0) ch_lo = max(ch_lo, (T - p.P) >> 5);
     const int ch_hi = w4 + 4;
     const int in_lo = 32 * w4 + 31 + T + 1 - p.window;
     for (int ch = ch_lo + wg; ch <= ch_hi; ch += 2) {
       float v[32];
       tmem_ld32(tl + C_L + ch * 32, v);
       float m4[4] = {kNegBig, kNegBig, kNegBig, kNegBig};
-      if (32 * ch >= in_lo && 32 * ch + 31 <= 32 * w4 + T && 32 * ch + cbase >= 0) {
+      if (32 * ch >= in_lo && 32 * ch + 31 <= 32 * w4 + T && 32 * ch + cbase >= -p.P) {
 #pragma unroll
         for (int u = 0; u < 32; ++u) m4[u & 3] = fmaxf(m4[u & 3], v[u]);
       } else {
@@ -247,7 +265,7 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
       if (ch > ch_hi) continue;
       float v[32];
       tmem_ld32(tl + C_L + ch * 32, v);
-      const bool inner = 32 * ch >= in_lo && 32 * ch + 31 <= 32 * w4 + T && 32 * ch + cbase >= 0;
+      const bool inner = 32 * ch >= in_lo && 32 * ch + 31 <= 32 * w4 + T && 32 * ch + cbase >= -p.P;
 #pragma unroll
       for (int u = 0; u < 32; u += 2) {
         float e0 = __expf(fmaf(v[u], p.scale, -mx));
@@ -509,16 +527,26 @@ __global__ void __launch_bounds__(NT_KV, 1) tc_swa_bwd_kv_kernel(const __grid_co
   // Persistent: CTA b walks the contiguous run [w0, w1) of (sequence, key
   // block) items; the next item's query tile b is loaded once this item's
   // products are done with it, the rest after its store.
-  const int nblk = (p.L + T - 1) / T, nwork = nblk * p.BH;
+  // With a prefix, block 0 of every sequence holds keys -128 .. -1 (the
+  // prefix in its last P rows, zeros before) and block b > 0 keys
+  // 128 (b - 1) ..; the query tiles of block 0 are then tokens -128 .. -1
+  // (none: read as zeros and masked) and 0 .. 127.
+  const int npre = p.P > 0 ? 1 : 0;
+  const int nblk = (p.L + T - 1) / T + npre, nwork = nblk * p.BH;
   const int w0 = (int)((long long)blockIdx.x * nwork / gridDim.x);
   const int w1 = (int)((long long)(blockIdx.x + 1) * nwork / gridDim.x);
   auto tile_loads = [&](int w, bool early, bool late) {
-    const int lbh = w / nblk, lj0 = (w % nblk) * T;
+    const int lbh = w / nblk, lj0 = (w % nblk - npre) * T;
     if (early) mbar_expect_tx(&bars[0], 6 * TILE);
     for (int r = 0; r < 2; ++r) {
-      if (late) {
+      if (late && lj0 < 0) {
+        tma_load_3d(sm + R_K + r * kReg, &p.mkp, &bars[0], 64 * r, p.P - T, lbh);
+        tma_load_3d(sm + R_V + r * kReg, &p.mvp, &bars[0], 64 * r, p.P - T, lbh);
+      } else if (late) {
         tma_load_3d(sm + R_K + r * kReg, &p.mk, &bars[0], 64 * r, lj0, lbh);
         tma_load_3d(sm + R_V + r * kReg, &p.mv, &bars[0], 64 * r, lj0, lbh);
+      }
+      if (late) {
         tma_load_3d(sm + R_Q0 + r * kReg, &p.mq, &bars[0], 64 * r, lj0, lbh);
         tma_load_3d(sm + R_O0 + r * kReg, &p.mo, &bars[0], 64 * r, lj0, lbh);
       }
@@ -539,12 +567,13 @@ __global__ void __launch_bounds__(NT_KV, 1) tc_swa_bwd_kv_kernel(const __grid_co
   bool ok = true;
   for (int w = w0, itn = 0; w < w1; ++w, ++itn) {
   const uint32_t par = (uint32_t)itn & 1u;
-  const int bh = w / nblk, h = bh % p.H, j0 = (w % nblk) * T, tk = j0 + row;
+  const int bh = w / nblk, h = bh % p.H, j0 = (w % nblk - npre) * T, tk = j0 + row;
+  const bool pre = j0 < 0;                     // the prefix block
   const float alpha = p.alpha ? p.alpha[h] : 1.f;
   for (int e = tid; e < 2 * T; e += NT_KV) {   // the softmax statistics of the two query tiles
     const int t = j0 + e;
-    s_lse[e] = t < p.L ? p.lse[(size_t)bh * p.L + t] : 0.f;
-    s_D[e] = t < p.L ? p.Dterm[(size_t)bh * p.L + t] : 0.f;
+    s_lse[e] = (t >= 0 && t < p.L) ? p.lse[(size_t)bh * p.L + t] : 0.f;
+    s_D[e] = (t >= 0 && t < p.L) ? p.Dterm[(size_t)bh * p.L + t] : 0.f;
   }
   ok = mbar_wait(&bars[0], par, p.status, ST_TIMEOUT);
   if (__syncthreads_or(!ok)) goto done;
@@ -591,7 +620,7 @@ __global__ void __launch_bounds__(NT_KV, 1) tc_swa_bwd_kv_kernel(const __grid_co
           for (int w = 0; w < 2; ++w) {
             const int qi = it * T + ch * 32 + u + w;       // query row within the two tiles
             const int t = j0 + qi;
-            const bool valid = t < p.L && tk < p.L && t >= tk && t - tk < p.window;
+            const bool valid = t >= 0 && t < p.L && tk >= -p.P && tk < p.L && t >= tk && t - tk < p.window;
             pr[w] = valid ? __expf(sv[u + w] * p.scale - s_lse[qi]) : 0.f;
             ds[w] = pr[w] * (alpha * dv[u + w] - s_D[qi]);
           }
@@ -652,13 +681,21 @@ __global__ void __launch_bounds__(NT_KV, 1) tc_swa_bwd_kv_kernel(const __grid_co
           g8[u] = fmaf(a[8 * k8 + u], p.scale, g8[u]);
           v8[u] = fmaf(b[8 * k8 + u], alpha, dg[u]);
         }
-        *cp = pack8(g8);
-        *chunk_ptr(sm, R_V, row, 4 * ch + k8) = pack8(v8);
+        if (pre) {   // prefix keys (no GLA part: the loads read zeros)
+          if (tk >= -p.P) {
+            const size_t o = ((size_t)bh * p.P + (p.P + tk)) * D + 32 * ch + 8 * k8;
+            *reinterpret_cast<uint4 *>(p.dk_prefix + o) = pack8(g8);
+            *reinterpret_cast<uint4 *>(p.dv_prefix + o) = pack8(v8);
+          }
+        } else {
+          *cp = pack8(g8);
+          *chunk_ptr(sm, R_V, row, 4 * ch + k8) = pack8(v8);
+        }
       }
     }
     fence_proxy_async();
     __syncthreads();
-    if (tid == 0) {
+    if (tid == 0 && !pre) {
       tma_store_3d(&p.mdko, sm + R_K, 0, j0, bh);
       tma_store_3d(&p.mdko, sm + R_K + kReg, 64, j0, bh);
       tma_store_3d(&p.mdvo, sm + R_V, 0, j0, bh);
@@ -674,6 +711,19 @@ __global__ void __launch_bounds__(NT_KV, 1) tc_swa_bwd_kv_kernel(const __grid_co
       float a[32], b[32];
       tmem_ld32(tl + C_DK + ch * 32, a);
       tmem_ld32(tl + C_DV + ch * 32, b);
+      if (pre) {   // prefix keys: their final bf16 gradients
+        if (tk >= -p.P) {
+          const size_t o = ((size_t)bh * p.P + (p.P + tk)) * D + 32 * ch;
+#pragma unroll
+          for (int u = 0; u < 32; ++u) { a[u] *= p.scale; b[u] *= alpha; }
+#pragma unroll
+          for (int k8 = 0; k8 < 4; ++k8) {
+            *reinterpret_cast<uint4 *>(p.dk_prefix + o + 8 * k8) = pack8(a + 8 * k8);
+            *reinterpret_cast<uint4 *>(p.dv_prefix + o + 8 * k8) = pack8(b + 8 * k8);
+          }
+        }
+        continue;
+      }
 #pragma unroll
       for (int u = 0; u < 32; u += 4) {
         *f32_stage_ptr(st0, row, ch * 32 + u) =
@@ -684,7 +734,7 @@ __global__ void __launch_bounds__(NT_KV, 1) tc_swa_bwd_kv_kernel(const __grid_co
     }
     fence_proxy_async();
     __syncthreads();
-    if (tid == 0) {
+    if (tid == 0 && !pre) {
       for (int bx = 0; bx < 4; ++bx) {
         tma_store_3d(&p.mdk, st0 + bx * 16384, 32 * bx, j0, bh);
         tma_store_3d(&p.mdv, st1 + bx * 16384, 32 * bx, j0, bh);
@@ -822,6 +872,12 @@ cudaError_t launch_tc_swa_bwd(const TcSwaBwdArgs &a, int stage, cudaStream_t s) 
     if (p.fused && (!make_map_bf16_3d(&p.mxq, a.xq_part, D, rows, a.BH, T) ||
                     !make_map_bf16_3d(&p.mdqo, a.dq_out, D, rows, a.BH, T)))
       return cudaErrorInvalidValue;
+    if (a.P > 0) {
+      if (!make_map_bf16_3d(&p.mkp, a.k_prefix, D, (uint64_t)a.P, a.BH, T) ||
+          !make_map_bf16_3d(&p.mvp, a.v_prefix, D, (uint64_t)a.P, a.BH, T))
+        return cudaErrorInvalidValue;
+      p.P = a.P;
+    }
     p.meta_k = a.meta_k;
     p.meta_v = a.meta_v;
     p.alpha = a.alpha;
@@ -860,6 +916,14 @@ cudaError_t launch_tc_swa_bwd(const TcSwaBwdArgs &a, int stage, cudaStream_t s) 
                   !make_map_bf16_3d(&p.mdko, a.dk_out, D, rows, a.BH, T) ||
                   !make_map_bf16_3d(&p.mdvo, a.dv_out, D, rows, a.BH, T)))
     return cudaErrorInvalidValue;
+  if (a.P > 0) {
+    if (!make_map_bf16_3d(&p.mkp, a.k_prefix, D, (uint64_t)a.P, a.BH, T) ||
+        !make_map_bf16_3d(&p.mvp, a.v_prefix, D, (uint64_t)a.P, a.BH, T))
+      return cudaErrorInvalidValue;
+    p.P = a.P;
+    p.dk_prefix = static_cast<__nv_bfloat16 *>(a.dk_prefix);
+    p.dv_prefix = static_cast<__nv_bfloat16 *>(a.dv_prefix);
+  }
   p.alpha = a.alpha;
   p.lse = a.lse;
   p.Dterm = a.Dterm;
@@ -877,7 +941,7 @@ cudaError_t launch_tc_swa_bwd(const TcSwaBwdArgs &a, int stage, cudaStream_t s) 
     int sms = 148;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    const int nwork = ntiles * a.BH;
+    const int nwork = (ntiles + (a.P > 0 ? 1 : 0)) * a.BH;
     tc_swa_bwd_kv_kernel<<<nwork < sms ? nwork : sms, NT_KV, SMEM_BYTES, s>>>(p);
   }
   return cudaGetLastError();

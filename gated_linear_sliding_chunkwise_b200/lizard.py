@@ -54,7 +54,7 @@ class BwdArgs(ctypes.Structure):
                 ("dfmap_wk", _vp), ("dalpha", _vp), ("dstate_in", _vp), ("impl", _i32),
                 ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t),
                 ("launch_events", ctypes.POINTER(_vp)), ("n_launch_events", _i32),
-                ("dstate_out", _vp)]
+                ("dstate_out", _vp), ("dk_prefix", _vp), ("dv_prefix", _vp)]
 
 
 class DecodeArgs(ctypes.Structure):
@@ -114,6 +114,10 @@ _lib.lizard_decode_status.argtypes = []
 _lib.lizard_decode_status.restype = ctypes.c_int
 _lib.lizard_workspace_status.argtypes = [_vp, _vp]
 _lib.lizard_workspace_status.restype = ctypes.c_int
+_lib.lizard_attn_fwd_noalloc.argtypes = [ctypes.POINTER(FwdArgs), _vp]
+_lib.lizard_attn_fwd_noalloc.restype = ctypes.c_int
+_lib.lizard_noalloc_status.argtypes = [_vp]
+_lib.lizard_noalloc_status.restype = ctypes.c_int
 _lib.lizard_status_string.argtypes = [ctypes.c_int]
 _lib.lizard_status_string.restype = ctypes.c_char_p
 _lib.lizard_debug_inject_wait_timeout.argtypes = [_i32]
@@ -310,17 +314,29 @@ def _bwd_struct(f, q, k, v, g, dout, *, meta_k, meta_v, fmap_wq, fmap_wk, impl, 
 def attn_bwd(q, k, v, g, dout, *, window, chunk=64, gate_temp=16.0, softmax_scale=0.0,
              fmap_wq=None, fmap_wk=None, meta_k=None, meta_v=None, alpha=None,
              state_in=None, branch=BRANCH_BOTH, impl=IMPL_AUTO, want_dstate=True,
-             workspace=None, stream=None, events=None, plan_only=False, dstate_out=None):
+             workspace=None, stream=None, events=None, plan_only=False, dstate_out=None,
+             k_prefix=None, v_prefix=None):
     """Backward of the hybrid layer (lizard_attn_bwd); returns every gradient.
     dstate_out [B, H, dk, dv] fp32: gradient flowing into the final state
-    (None: the final state is unused)."""
+    (None: the final state is unused).  k_prefix, v_prefix [B, H, P, d]: the
+    anchor window's prefix, as in attn_fwd; their gradients come back as
+    dk_prefix, dv_prefix."""
     f = _fwd_struct(q, k, v, g, window=window, chunk=chunk, gate_temp=gate_temp,
                     softmax_scale=softmax_scale, fmap_wq=fmap_wq, fmap_wk=fmap_wk,
                     meta_k=meta_k, meta_v=meta_v, alpha=alpha, state_in=state_in,
                     branch=branch, impl=impl)
+    if (k_prefix is None) != (v_prefix is None):
+        raise ValueError("k_prefix and v_prefix go together")
     b, res = _bwd_struct(f, q, k, v, g, dout, meta_k=meta_k, meta_v=meta_v, fmap_wq=fmap_wq,
                          fmap_wk=fmap_wk, impl=impl, want_dstate=want_dstate)
     b.dstate_out = _ptr(dstate_out)
+    res["dk_prefix"] = res["dv_prefix"] = None
+    if k_prefix is not None:
+        b.fwd.k_prefix, b.fwd.v_prefix = _ptr(k_prefix), _ptr(v_prefix)
+        b.fwd.prefix_len = k_prefix.shape[2]
+        res["dk_prefix"] = torch.empty_like(k_prefix)
+        res["dv_prefix"] = torch.empty_like(v_prefix)
+        b.dk_prefix, b.dv_prefix = _ptr(res["dk_prefix"]), _ptr(res["dv_prefix"])
     dev = q.device
     nbytes = bwd_workspace_bytes(b)
     ws = _workspace(nbytes, dev, workspace)
@@ -392,6 +408,12 @@ def decode_step(q, k, v, g, state, k_cache, v_cache, pos, *, gate_temp=16.0,
 def workspace_status(workspace, stream=None) -> int:
     """Status word left in a workspace by kernels with bounded waits."""
     return int(_lib.lizard_workspace_status(workspace.data_ptr(), _stream(stream)))
+
+
+def noalloc_status(stream=None) -> int:
+    """Status word of the last lizard_attn_fwd_noalloc call on the current
+    device (it lives in the library's built-in scratch); reading clears it."""
+    return int(_lib.lizard_noalloc_status(_stream(stream)))
 
 
 def decode_status() -> int:

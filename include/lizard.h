@@ -49,11 +49,16 @@
  *     recorded in a status word at the start of the workspace, cleared at the
  *     start of every forward or backward call and read back by
  *     lizard_workspace_status(): a kernel that gives up on a bounded wait
- *     records LIZARD_ERR_TIMEOUT; the tensor-core forward records
- *     LIZARD_ERR_RANGE when, inside one 128-token tile, the cumulative
- *     log-decay of some key dimension spans more than 64 (gate logits below
- *     about -8 per token at gate_temp 16); such inputs need LIZARD_IMPL_SIMT,
- *     which computes them exactly.
+ *     records LIZARD_ERR_TIMEOUT.
+ *   - Wide decay on the tensor-core path: when, inside one 128-token tile, the
+ *     cumulative log-decay of some key dimension spans more than 64 (gate
+ *     logits below about -8 per token at gate_temp 16), the tensor-core
+ *     kernels' log-space factors leave their exponent range.  Such sequences
+ *     get the GLA branch from the portable kernels instead (exact for any
+ *     decay), up to 4 of them per call; a fifth and later one in the same call
+ *     keeps the tensor-core result, and the call records LIZARD_ERR_RANGE.
+ *     lizard_stage1_step has no such fallback: it records LIZARD_ERR_RANGE
+ *     for any of them.
  */
 #ifndef LIZARD_H_
 #define LIZARD_H_
@@ -74,7 +79,7 @@ typedef enum {
   LIZARD_ERR_CUDA = 3,        /* a launch or CUDA runtime call failed */
   LIZARD_ERR_TIMEOUT = 4,     /* a kernel gave up on a bounded wait */
   LIZARD_ERR_WORKSPACE = 5,   /* workspace NULL or smaller than the queried size */
-  LIZARD_ERR_RANGE = 6        /* the tensor-core forward met a gate decay outside its range */
+  LIZARD_ERR_RANGE = 6        /* tensor-core path: more wide-decay sequences than its exact fallback takes */
 } lizard_status;
 
 typedef enum { LIZARD_BF16 = 0, LIZARD_FP32 = 1 } lizard_dtype;
@@ -129,9 +134,10 @@ enum {
  * through state_in instead).
  *   k_prefix   [B, H, P, dk] dtype, v_prefix [B, H, P, dv] dtype: row P - 1
  *              is token -1, row 0 token -P
- *   0 <= P <= window; the pointers are NULL iff P == 0.  Forward only:
- *   lizard_attn_bwd and lizard_stage1_step return LIZARD_ERR_UNSUPPORTED for
- *   a nonzero prefix_len.
+ *   0 <= P <= window; the pointers are NULL iff P == 0.  lizard_attn_bwd
+ *   returns the prefix's key and value gradients (lizard_bwd_args.dk_prefix,
+ *   dv_prefix); lizard_stage1_step, which trains whole sequences, returns
+ *   LIZARD_ERR_UNSUPPORTED for a nonzero prefix_len.
  */
 typedef struct {
   int32_t B, H, L, dk, dv, chunk, window, M;
@@ -189,6 +195,12 @@ lizard_status lizard_attn_fwd(const lizard_fwd_args *args, lizard_stream_t strea
  *            state_out), or NULL for an unused final state.  The gradients
  *            are then those of sum(dout * o) + sum(dstate_out * S_{L-1}).
  *            Needs the GLA branch.
+ *   dk_prefix, dv_prefix [B, H, P, dk|dv] dtype, written: with a key/value
+ *            prefix (fwd.prefix_len = P > 0), the gradients with respect to
+ *            fwd.k_prefix and fwd.v_prefix -- the anchor window's reach into
+ *            the previous segment, to be added to that segment's last P key
+ *            and value gradients (the GLA history's gradient is dstate_in).
+ *            Required when P > 0, NULL when P == 0.
  */
 typedef struct {
   lizard_fwd_args fwd;
@@ -205,6 +217,7 @@ typedef struct {
   void *const *launch_events;   /* as in lizard_fwd_args */
   int32_t n_launch_events;
   const float *dstate_out;      /* see above; NULL = zero */
+  void *dk_prefix, *dv_prefix;  /* see above */
 } lizard_bwd_args;
 
 size_t lizard_bwd_workspace_size(const lizard_bwd_args *args);
@@ -309,9 +322,12 @@ int32_t lizard_stage1_launch_plan(const lizard_stage1_args *args, const char **n
  *   o          [B, H, dv] dtype, written: o = S^T phi_q(q) + alpha_h o^swa,
  *              the softmax covering the min(pos+1, window) filled slots and
  *              the M meta tokens
- * Parameters as in lizard_fwd_args.  Needs no workspace.  Two kernels are
- * enqueued (the step, then the pos increment), so concurrent heads of one
- * sequence all see the same pos.
+ * Parameters as in lizard_fwd_args.  Needs no workspace.  One kernel is
+ * enqueued: every head of a sequence reads pos before any CTA increments it
+ * (the last CTA to have read its pos values adds 1 to every pos[b]; only
+ * with more than 64 x SM-count (batch, head) pairs in a bf16, d = 128 step
+ * does a second, increment kernel follow).  Steps on the same pos array
+ * must be ordered (one stream).
  */
 typedef struct {
   int32_t B, H, dk, dv, window, M;
@@ -395,9 +411,9 @@ void lizard_debug_inject_wait_timeout(int32_t count);
  *     lizard_fwd_workspace_size) return LIZARD_ERR_UNSUPPORTED and launch
  *     nothing.  With dk = dv = 128 that is above roughly 16K token-heads
  *     (B * H * L) for the portable kernels.
- *   - The first call on each device looks up the array's device address
- *     (with that device current).  Make that first call before any stream
- *     capture.
+ *   - Every call looks up the array's device address on the current device
+ *     (the first lookup on a device loads the library's device code there).
+ *     Make the first call on each device before any stream capture.
  *   - No cudaMalloc, cudaFree or other allocating routine is called.
  *   - All calls share the one array and it keeps the last call's contents.
  *     Calls that overlap on the GPU (different streams, or different host
@@ -406,6 +422,14 @@ void lizard_debug_inject_wait_timeout(int32_t count);
  */
 #define LIZARD_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
 lizard_status lizard_attn_fwd_noalloc(const lizard_fwd_args *args, lizard_stream_t stream);
+
+/* The device status of the last lizard_attn_fwd_noalloc call on the current
+ * device: waits for `stream`, then reads and clears the status word at the
+ * start of the built-in scratch, exactly as lizard_workspace_status does for
+ * a caller's workspace (LIZARD_OK, LIZARD_ERR_TIMEOUT or LIZARD_ERR_RANGE;
+ * LIZARD_ERR_CUDA if the copy fails).  Allocates nothing.  The word belongs
+ * to the shared scratch: read it before the next noalloc call. */
+lizard_status lizard_noalloc_status(lizard_stream_t stream);
 
 /* Waits for `stream`, then reads and clears the status word that the last
  * forward or backward call left at the start of `workspace` (a device

@@ -238,7 +238,10 @@ def test_stage1_launch_plan_fuses_the_loss_on_tensor_cores(lz):
 
 
 # ------------------------------------------------- sequence parallelism ---
-def test_prefix_does_not_change_the_workspace_and_is_forward_only(lz):
+def test_prefix_does_not_change_the_workspaces_and_its_gradients_are_outputs(lz):
+    """A prefix needs no extra workspace in either direction; the backward
+    requires the prefix's gradient outputs with a prefix and refuses them
+    without one; the stage-1 step (whole sequences) refuses a prefix."""
     a = _fwd(lz)
     b = _fwd(lz, prefix_len=16, k_prefix=0x10000, v_prefix=0x10000)
     assert lz.fwd_workspace_bytes(b) == lz.fwd_workspace_bytes(a) > 0
@@ -248,8 +251,21 @@ def test_prefix_does_not_change_the_workspace_and_is_forward_only(lz):
     bw.dout = bw.dq = bw.dk = bw.dv = bw.dg = fake
     need = lz.bwd_workspace_bytes(bw)
     assert need > 0
+    bw0 = lz.BwdArgs()
+    bw0.fwd = a
+    bw0.dout = bw0.dq = bw0.dk = bw0.dv = bw0.dg = fake
+    assert lz.bwd_workspace_bytes(bw0) == need
     bw.workspace, bw.workspace_bytes = 0x20000, need
-    assert lz.lib().lizard_attn_bwd(ctypes.byref(bw), None) == lz.ERR_UNSUPPORTED
+    # no prefix gradient outputs: refused before anything runs
+    assert lz.lib().lizard_attn_bwd(ctypes.byref(bw), None) == lz.ERR_INVALID_ARG
+    bw.dk_prefix = fake
+    assert lz.lib().lizard_attn_bwd(ctypes.byref(bw), None) == lz.ERR_INVALID_ARG
+    bw.dv_prefix = 0x10008          # misaligned
+    assert lz.lib().lizard_attn_bwd(ctypes.byref(bw), None) == lz.ERR_INVALID_ARG
+    bw0.workspace, bw0.workspace_bytes = 0x20000, need
+    bw0.dk_prefix = bw0.dv_prefix = fake   # gradients of a prefix that is not there
+    assert lz.lib().lizard_attn_bwd(ctypes.byref(bw0), None) == lz.ERR_INVALID_ARG
+    bw.dk_prefix = bw.dv_prefix = None
     s1 = lz.Stage1Args()
     s1.bwd = bw
     s1.target, s1.loss = fake, fake
@@ -347,7 +363,9 @@ int main(void) {
   lizard_fwd_args bad = a;
   bad.dk = bad.dv = 96;
   lizard_status st = lizard_attn_fwd(&bad, NULL);
-  printf("%zu %d %s %d %s %s\n", ws, n, n > 0 ? names[n - 1] : "-", (int)st,
+  int tc = 0;
+  for (int i = 0; i < n && i < 16; ++i) tc |= strcmp(names[i], "tc_fwd_kernel") == 0;
+  printf("%zu %d %s %d %s %s\n", ws, n, tc ? "tc_fwd_kernel" : "-", (int)st,
          lizard_status_string(st), lizard_version());
   return 0;
 }
@@ -358,6 +376,6 @@ int main(void) {
                     "-L", libdir, "-llizard", "-Wl,-rpath," + libdir], check=True)
     out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
     assert int(out[0]) > 0                       # workspace bytes
-    assert int(out[1]) >= 1 and out[2] == "tc_fwd_kernel"   # the tensor-core plan ends with the full pass
+    assert int(out[1]) >= 1 and out[2] == "tc_fwd_kernel"   # the tensor-core plan has the full pass
     assert int(out[3]) == lz.ERR_UNSUPPORTED     # d = 96 is refused on the host
     assert out[-1] == lz.version()

@@ -129,6 +129,40 @@ def test_backward_extreme_decay(lz, impl):
         check(name, got[name], want[name], "fp32")
 
 
+@pytest.mark.parametrize("impl", ["tc", "auto"])
+@pytest.mark.parametrize("gate", ["dim", "scalar"])
+@pytest.mark.parametrize("with_g", [False, True])
+def test_tc_backward_computes_wide_decay_exactly(lz, impl, gate, with_g):
+    """The backward's exact fallback: sequences whose in-tile decay spread
+    leaves the tensor-core range get their GLA gradients from the portable
+    kernels (dphi, dv, dstate_in, da and dg), the rest of the call from the
+    tensor-core kernels; every gradient matches the oracle, with and without
+    an incoming final-state gradient."""
+    w = Workload("brange", B=2, H=2, L=300, d=128, window=128, M=4, dtype="bf16", seed=9, kind="train",
+                 gate=gate)
+    inp = make_inputs(w)
+    g = inp["g"].clone()
+    if gate == "dim":
+        g[0, 1, 130:200, :3] = -300.0
+        g[1, 0, 20:21, :] = -2000.0
+    else:
+        g[0, 1, 130:200] = -300.0
+        g[1, 0, 20:21] = -2000.0
+    inp["g"] = g
+    inp["state_in"] = torch.randn(2, 2, 128, 128, generator=torch.Generator().manual_seed(4)) * 0.1
+    G = torch.randn(2, 2, 128, 128, generator=torch.Generator().manual_seed(5)) if with_g else None
+    got = _run(lz, to_device(inp), w, _impl(lz, impl), dstate_out=None if G is None else G.cuda())
+    assert lz.workspace_status(got["workspace"]) == lz.OK
+    y = {k_: to64(v_) for k_, v_ in inp.items() if v_ is not None}
+    want = ref.lizard_backward(y["q"], y["k"], y["v"], y["g"], y["dout"], window=w.window, tau=w.gate_temp,
+                               fmap_wq=y["fmap_wq"], fmap_wk=y["fmap_wk"], meta_k=y["meta_k"],
+                               meta_v=y["meta_v"], alpha=y["alpha"], state_in=y["state_in"],
+                               dstate_out=None if G is None else to64(G),
+                               gate=ref.GATE_SCALAR if gate == "scalar" else ref.GATE_PER_DIM)
+    for name in GRADS:
+        check(f"{name} ({gate} gate)", got[name], want[name], "bf16")
+
+
 @pytest.mark.parametrize("impl", IMPLS)
 def test_parameter_grads_bf16_full_reduction(lz, impl):
     """Gradients of the per-head parameters reduce over batch and tokens:

@@ -132,14 +132,59 @@ def test_alpha_zero_drops_anchor_branch(lz, impl):
     check("o", got["o"], want["o"], dtype)
 
 
-def test_tc_flags_decay_outside_its_range(lz):
-    """Gate logits of -300 make one tile's cumulative decay span far more than
-    the tensor-core forward's range: it must say so in the status word."""
-    w = Workload("range", B=1, H=1, L=256, d=128, window=128, M=4, dtype="bf16", seed=2)
-    inp = make_inputs(w)
+def _wide_decay(inp, heads):
+    """Gate logits of -300 over part of a tile (log-decay -18.75 per token on
+    a few key dimensions) and one token of -2000 (it wipes the state): the
+    in-tile spread leaves the tensor-core absorption's range."""
     g = inp["g"].clone()
-    g[:, :, 130:200, :3] = -300.0
+    scalar = g.dim() == inp["q"].dim() - 1
+    for b, h in heads:
+        if scalar:
+            g[b, h, 130:200] = -300.0
+            g[b, h, 20:21] = -2000.0
+        else:
+            g[b, h, 130:200, :3] = -300.0
+            g[b, h, 20:21, :] = -2000.0
     inp["g"] = g
+    return inp
+
+
+@pytest.mark.parametrize("impl", ["tc", "auto"])
+@pytest.mark.parametrize("gate", ["dim", "scalar"])
+def test_tc_path_computes_wide_decay_exactly(lz, impl, gate):
+    """Sequences whose in-tile decay spread leaves the tensor-core range go
+    to the exact fallback (their GLA branch on the portable kernels): the
+    output, final state and normaliser match the oracle, the status is OK,
+    and the other sequences of the call stay on the tensor cores."""
+    w = Workload("range", B=2, H=3, L=300, d=128, window=128, M=4, dtype="bf16", seed=2, gate=gate)
+    inp = _wide_decay(make_inputs(w), [(0, 1), (1, 2)])
+    inp["state_in"] = torch.randn(2, 3, 128, 128, generator=torch.Generator().manual_seed(3)) * 0.1
+    got = _run(lz, to_device(inp), w, _impl(lz, impl), want_state=True, want_lse=True)
+    assert lz.workspace_status(got["workspace"]) == lz.OK
+    want = oracle_forward(inp, window=w.window, tau=w.gate_temp)
+    for name in ("o", "state_out", "lse"):
+        check(name, got[name], want[name], "bf16")
+
+
+def test_tc_wide_decay_in_a_segmented_forward(lz):
+    """Few sequences and a long one (the forward splits sequences into
+    segments with a state pass): a marked sequence's GLA branch still comes
+    whole from the exact fallback."""
+    w = Workload("range_seg", B=1, H=2, L=1100, d=128, window=128, M=4, dtype="bf16", seed=5)
+    inp = _wide_decay(make_inputs(w), [(0, 0)])
+    got = _run(lz, to_device(inp), w, lz.IMPL_TC, want_state=True)
+    assert lz.workspace_status(got["workspace"]) == lz.OK
+    want = oracle_forward(inp, window=w.window, tau=w.gate_temp)
+    check("o", got["o"], want["o"], "bf16")
+    check("state_out", got["state_out"], want["state_out"], "bf16")
+
+
+def test_tc_flags_wide_decay_beyond_its_fallback_slots(lz):
+    """More marked sequences in one call than the exact fallback has slots
+    (four): the ones beyond keep the tensor-core result and the status word
+    says RANGE; a call without such gates reads OK again."""
+    w = Workload("range_many", B=3, H=2, L=256, d=128, window=128, M=4, dtype="bf16", seed=2)
+    inp = _wide_decay(make_inputs(w), [(b, h) for b in range(3) for h in range(2)])
     got = _run(lz, to_device(inp), w, lz.IMPL_TC)
     assert lz.workspace_status(got["workspace"]) == lz.ERR_RANGE
     ok = _run(lz, to_device(make_inputs(w)), w, lz.IMPL_TC)

@@ -1,8 +1,8 @@
 """GPU parity of the sequence-parallel pieces against the oracle, through
-the C ABI: the forward with a key/value prefix, the segment summary (U, R),
-the chain of summaries, and a sequence split into segments run one after
-another on one GPU (each segment the work of one rank) against the
-whole-sequence forward."""
+the C ABI: the forward and the backward with a key/value prefix, the segment
+summary (U, R), the chain of summaries, and a sequence split into segments
+run one after another on one GPU (each segment the work of one rank)
+against the whole-sequence forward and backward."""
 
 import os
 
@@ -74,6 +74,34 @@ def test_forward_with_prefix_matches_oracle(lz, impl, dtype, d, B, H, L, window,
                               tau=w.gate_temp, state_in=to64(S_in), k_prefix=y["k"][:, :, :P],
                               v_prefix=y["v"][:, :, :P], gate=gate_of(y), **_params(y))
     for name in ("o", "state_out", "lse"):
+        check(name, got[name], want[name], dtype)
+
+
+BWD_GRADS = ("dq", "dk", "dv", "dg", "dmeta_k", "dmeta_v", "dfmap_wq", "dfmap_wk", "dalpha",
+             "dstate_in", "dk_prefix", "dv_prefix")
+
+
+@pytest.mark.parametrize("impl,dtype,d,B,H,L,window,M,P,gate", PREFIX_CASES)
+def test_backward_with_prefix_matches_oracle(lz, impl, dtype, d, B, H, L, window, M, P, gate):
+    """lizard_attn_bwd of a segment with a key/value prefix: every gradient,
+    the prefix's own key and value gradients included, against the oracle."""
+    w, inp = _whole(dtype, d, B, H, P + L, window, M, gate, seed=650 + L)
+    S_in = torch.randn(B, H, d, d, generator=torch.Generator().manual_seed(7)) * 0.1
+    dout = torch.randn(B, H, L, d, generator=torch.Generator().manual_seed(11)).to(inp["q"].dtype)
+    x = to_device(inp)
+    t = _span(x, P, P + L)
+    kp, vp = x["k"][:, :, :P].contiguous(), x["v"][:, :, :P].contiguous()
+    got = lz.attn_bwd(t["q"], t["k"], t["v"], t["g"], dout.cuda(), window=window, gate_temp=w.gate_temp,
+                      state_in=S_in.cuda(), impl=_impl(lz, impl), k_prefix=kp, v_prefix=vp, **_params(x))
+    assert lz.workspace_status(got["workspace"]) == lz.OK
+    y = {k_: to64(v_) for k_, v_ in inp.items() if v_ is not None}
+    want = ref.lizard_backward(*(y[k_][:, :, P:] for k_ in ("q", "k", "v", "g")), to64(dout), window=window,
+                               tau=w.gate_temp, state_in=to64(S_in), k_prefix=y["k"][:, :, :P],
+                               v_prefix=y["v"][:, :, :P], gate=gate_of(y), **_params(y))
+    for name in BWD_GRADS:
+        if want[name] is None:
+            assert got[name] is None, name
+            continue
         check(name, got[name], want[name], dtype)
 
 
@@ -158,6 +186,68 @@ def test_segments_one_after_another_reproduce_the_whole_forward(lz, impl, dtype,
                               state_in=to64(S_in), gate=gate_of(y), **_params(y))
     check("o", torch.cat(outs, dim=2), want["o"], dtype)
     check("state_out", last, want["state_out"], dtype)
+
+
+BWD_SPLIT_CASES = [
+    # impl, dtype, d, B, H, cuts, window, M, gate
+    ("tc", "bf16", 128, 2, 2, [0, 256, 400, 650], 128, 4, "dim"),
+    ("tc", "bf16", 128, 2, 2, [0, 300, 517], 100, 4, "scalar"),
+    ("simt", "fp32", 64, 2, 2, [0, 40, 97, 150], 16, 4, "dim"),
+]
+
+
+@pytest.mark.parametrize("impl,dtype,d,B,H,cuts,window,M,gate", BWD_SPLIT_CASES)
+def test_segments_one_after_another_reproduce_the_whole_backward(lz, impl, dtype, d, B, H, cuts, window,
+                                                                  M, gate):
+    """The split backward as the ranks run it, one segment after another on
+    one GPU (the gathers are stacks here; the collectives are tested on the
+    CPU): each segment's backward from its start state and prefix, the
+    end-state gradients chained from the last segment down, the GLA-only
+    correction with that gradient, the prefix gradients added to the
+    previous segment's last keys and values, parameter gradients summed."""
+    w, inp = _whole(dtype, d, B, H, cuts[-1], window, M, gate, seed=850 + cuts[-1])
+    S_in = torch.randn(B, H, d, d, generator=torch.Generator().manual_seed(9)) * 0.1
+    G = torch.randn(B, H, d, d, generator=torch.Generator().manual_seed(10)) * 0.1
+    dout = torch.randn(B, H, cuts[-1], d, generator=torch.Generator().manual_seed(12)).to(inp["q"].dtype)
+    x = to_device(inp)
+    x["dout"] = dout.cuda()
+    im = _impl(lz, impl)
+    n = len(cuts) - 1
+    kw = dict(window=window, gate_temp=w.gate_temp, impl=im, **_params(x))
+    seg = [dict(_span(x, cuts[r], cuts[r + 1]), dout=x["dout"][:, :, cuts[r]:cuts[r + 1]].contiguous())
+           for r in range(n)]
+    sums = [lz.segment_state(s["k"], s["v"], s["g"], window=window, gate_temp=w.gate_temp,
+                             fmap_wk=x["fmap_wk"], impl=im) for s in seg]
+    U_all = torch.stack([u for u, _, _ in sums])
+    R_all = torch.stack([r_ for _, r_, _ in sums])
+    S0 = [lz.chain_states(U_all, R_all, r, state_in=S_in.cuda()) for r in range(n)]
+    pre = [{}] + [{"k_prefix": x["k"][:, :, cuts[r] - window:cuts[r]].contiguous(),
+                   "v_prefix": x["v"][:, :, cuts[r] - window:cuts[r]].contiguous()} for r in range(1, n)]
+    gr = [lz.attn_bwd(s["q"], s["k"], s["v"], s["g"], s["dout"], state_in=S0[r],
+                      dstate_out=G.cuda() if r == n - 1 else None, **pre[r], **kw)
+          for r, s in enumerate(seg)]
+    D_all = torch.stack([gr[r]["dstate_in"] for r in range(n)])
+    for r in range(n - 1):
+        X = lz.chain_states(torch.flip(D_all, dims=[0]).contiguous(), torch.flip(R_all, dims=[0]).contiguous(),
+                            n - 1 - r)
+        s = seg[r]
+        c = lz.attn_bwd(s["q"], s["k"], s["v"], s["g"], torch.zeros_like(s["dout"]), state_in=S0[r],
+                        dstate_out=X, branch=lz.BRANCH_GLA_ONLY, **kw)
+        for name in ("dq", "dk", "dv", "dg", "dfmap_wq", "dfmap_wk", "dstate_in"):
+            gr[r][name] = gr[r][name] + c[name]
+    for r in range(1, n):
+        gr[r - 1]["dk"][:, :, -window:] += gr[r]["dk_prefix"]
+        gr[r - 1]["dv"][:, :, -window:] += gr[r]["dv_prefix"]
+    for r in range(n):
+        assert lz.workspace_status(gr[r]["workspace"]) == lz.OK
+    y = {k_: to64(v_) for k_, v_ in inp.items() if v_ is not None}
+    want = ref.lizard_backward(y["q"], y["k"], y["v"], y["g"], to64(dout), window=window, tau=w.gate_temp,
+                               state_in=to64(S_in), dstate_out=to64(G), gate=gate_of(y), **_params(y))
+    for name in ("dq", "dk", "dv", "dg"):
+        check(name, torch.cat([g_[name] for g_ in gr], dim=2), want[name], dtype)
+    for name in ("dmeta_k", "dmeta_v", "dfmap_wq", "dfmap_wk", "dalpha"):
+        check(name, sum(g_[name] for g_ in gr), want[name], dtype)
+    check("dstate_in", gr[0]["dstate_in"], want["dstate_in"], dtype)
 
 
 @pytest.mark.timeout(300)
