@@ -107,9 +107,9 @@ def kernel_model(name, w, N, BH):
         "seg_combine_kernel": (3 * seg_states, 0),
         "tc_fwd_kernel(state copies)": (2 * Nd * esz + Nd * 4 + snaps, N * (2 * d * d + phi / 2)),
         "tc_gla_dstates_kernel": (2 * Nd * esz + Nd * 4 + snaps + BH * d * d * 4, N * (2 * d * d + phi / 2)),
-        "tc_gla_bwd_tile_kernel": (4 * Nd * esz + 2 * snaps + Nd * 4 + 4 * Nd * 4,
+        "tc_gla_bwd_tile_kernel": (4 * Nd * esz + 2 * snaps + Nd * 4 + 2 * Nd * 4 + 2 * Nd * 2,
                                    N * (2 * fl["gla_fwd"] + phi)),
-        "tc_finish_kernel": (4 * Nd * esz + 2 * Nd * 4, N * 3 * phi),
+        "tc_finish_kernel": (4 * Nd * esz + 2 * Nd * 2, N * 3 * phi),
         "tc_swa_bwd_q_kernel": (6 * Nd * esz + 2 * N * 4 + 2 * N * mw * 4, N * 1.5 * fl["swa_fwd"]),
         "tc_swa_bwd_kv_kernel": (7 * Nd * esz + Nd * 4 + 2 * N * 4, N * 2.0 * fl["swa_fwd"]),
         "meta_grad_kernel": (2 * Nd * esz + 2 * N * mw * 4, N * 4 * d * w.M),

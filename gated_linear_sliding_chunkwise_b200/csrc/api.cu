@@ -84,6 +84,10 @@ bool fwd_uses_tc(const lizard_fwd_args *a) {
 struct FallbackLayout {
   size_t flags, slot_of, seq_of_slot, scratch, per_slot, end;
 };
+int fallback_slots(const lizard_fwd_args *a) {
+  const int BH = a->B * a->H;
+  return BH < lz::kFallbackSlots ? BH : lz::kFallbackSlots;
+}
 FallbackLayout fallback_layout(size_t off, const lizard_fwd_args *a, size_t per_slot) {
   const size_t BH = (size_t)a->B * a->H;
   FallbackLayout f{};
@@ -91,13 +95,9 @@ FallbackLayout fallback_layout(size_t off, const lizard_fwd_args *a, size_t per_
   f.slot_of = off; off += up(BH * sizeof(int));
   f.seq_of_slot = off; off += up(lz::kFallbackSlots * sizeof(int));
   f.per_slot = per_slot;
-  f.scratch = off; off += lz::kFallbackSlots * per_slot;
+  f.scratch = off; off += (size_t)fallback_slots(a) * per_slot;
   f.end = off;
   return f;
-}
-int fallback_slots(const lizard_fwd_args *a) {
-  const int BH = a->B * a->H;
-  return BH < lz::kFallbackSlots ? BH : lz::kFallbackSlots;
 }
 // bytes the call's first memset clears: the status header and, with the
 // exact fallback, the per-sequence marks that follow it
@@ -108,8 +108,8 @@ size_t cleared_bytes(const lizard_fwd_args *a, bool fallback) {
 // Forward workspace: the status header, plus fp32 scratch for the portable path.
 struct FwdLayout {
   size_t phq, phk, a, o_gla, total;
-  bool fallback;
-  FallbackLayout fb;
+  bool fallback;   // wide-decay marks (tensor-core GLA branch)
+  size_t flags;
 };
 FwdLayout fwd_layout(const lizard_fwd_args *a, bool stage1 = false) {
   const size_t N = (size_t)a->B * a->H * a->L;
@@ -119,10 +119,9 @@ FwdLayout fwd_layout(const lizard_fwd_args *a, bool stage1 = false) {
   if (fwd_uses_tc(a)) {
     // the stage-1 step keeps its loss in the tensor-core epilogue: no fallback
     l.fallback = gla_on(a) && !stage1;
-    if (l.fallback) {
-      const size_t Ld = up((size_t)a->L * a->dk * sizeof(float));
-      l.fb = fallback_layout(off, a, 3 * Ld);   // phi_q, phi_k and a of one sequence
-      off = l.fb.end;
+    if (l.fallback) {   // one mark per sequence, right after the header
+      l.flags = off;
+      off += up((size_t)a->B * a->H * sizeof(uint32_t));
     }
     l.phq = off;   // segment states of the tensor-core path
     off += up(lz::tc_fwd_workspace_bytes(a->B * a->H, a->L));
@@ -164,9 +163,9 @@ BwdLayout bwd_layout(const lizard_fwd_args *a, int impl, bool stage1 = false) {
   size_t off = kHeader;
   if (gla_on(a) && bwd_gla_uses_tc(a, impl) && !stage1) {
     // exact fallback: per slot phi_q, phi_k, a, the chunk states and kap of
-    // the portable backward
+    // the portable backward, then its fp32 dphi_q, dphi_k
     const size_t Ld = up((size_t)a->L * a->dk * sizeof(float));
-    const size_t per = 3 * Ld + up(nch * a->dk * a->dv * sizeof(float)) + up(a->dk * sizeof(float));
+    const size_t per = 5 * Ld + up(nch * a->dk * a->dv * sizeof(float)) + up(a->dk * sizeof(float));
     l.fallback = true;
     l.fb = fallback_layout(off, a, per);
     off = l.fb.end;
@@ -175,8 +174,8 @@ BwdLayout bwd_layout(const lizard_fwd_args *a, int impl, bool stage1 = false) {
     const size_t snap = up(lz::tc_gla_bwd_snapshot_bytes((int)BH, a->L));
     l.snap_s = off; off += snap;
     l.snap_ds = off; off += snap;
-    l.dphq = off; off += nd;
-    l.dphk = off; off += nd;
+    l.dphq = off; off += up(N * a->dk * 2);   // bf16, row halves centred
+    l.dphk = off; off += up(N * a->dk * 2);
     l.da = off; off += nd;       // dB: gradient of the in-tile cumulative log-decay
     l.dv_gla = off; off += nv;
     l.e32 = off; off += nd;      // fp32 decay factors E of every tile
@@ -334,39 +333,15 @@ void fwd_plan(const lizard_fwd_args *a, void *ws, cudaStream_t s, Plan &plan, co
                     static_cast<uint32_t *>(ws), at<void>(ws, lay.phq), BH, a->H, a->L, a->M, a->window,
                     a->branch, 1.f / a->gate_temp, scale_of(a), scalar_gate(a), target, dmse, loss,
                     a->k_prefix, a->v_prefix, a->prefix_len};
-    const FallbackLayout fb = lay.fb;
-    const int K = fallback_slots(a);
-    uint32_t *status = static_cast<uint32_t *>(ws);
-    if (lay.fallback) {
-      t.seqflag = at<uint32_t>(ws, fb.flags);
-      t.slot_of = at<int>(ws, fb.slot_of);
-    }
+    // wide decay: the gate prep marks the sequences, whose GLA branch the
+    // full pass then runs as the exact recurrence
+    if (lay.fallback) t.seqflag = at<uint32_t>(ws, lay.flags);
     if (gla_on(a)) plan.add("gate_prep_kernel", [=](cudaStream_t s) { return lz::launch_tc_fwd(t, 3, s); });
-    if (lay.fallback)
-      plan.add("assign_slots_kernel", [=](cudaStream_t s) {
-        return lz::launch_assign_slots(at<uint32_t>(ws, fb.flags), at<int>(ws, fb.slot_of), at<int>(ws, fb.seq_of_slot),
-                                       BH, K, status, s);
-      });
     if (gla_on(a) && lz::tc_fwd_stage_count(BH, a->L) > 1) {   // segment start states (GLA only)
       plan.add("tc_fwd_kernel(state pass)", [=](cudaStream_t s) { return lz::launch_tc_fwd(t, 0, s); });
       plan.add("seg_combine_kernel", [=](cudaStream_t s) { return lz::launch_tc_fwd(t, 1, s); });
     }
     plan.add("tc_fwd_kernel", [=](cudaStream_t s) { return lz::launch_tc_fwd(t, 2, s); });
-    if (lay.fallback) {
-      // the GLA branch of the marked sequences, exactly, on the portable
-      // kernels (one grid slot each; a slot with no sequence exits at once)
-      // scratch: phi_q, phi_k, a, each [K][L][D] fp32; the GLA kernel adds
-      // its output to o in place
-      const size_t arr = (size_t)K * (fb.per_slot / 3);
-      const int *seq = at<int>(ws, fb.seq_of_slot);
-      lz::PrepArgs pa{a->q, a->k, a->g, a->fmap_wq, a->fmap_wk, at<float>(ws, fb.scratch),
-                      at<float>(ws, fb.scratch + arr), at<float>(ws, fb.scratch + 2 * arr),
-                      a->H, a->L, 1.f / a->gate_temp, scalar_gate(a), seq};
-      plan.add("prep_kernel(exact fallback)", [=](cudaStream_t s) { return lz::launch_prep(pa, K, D, bf16, s); });
-      lz::GlaFwdArgs ga{pa.phq, pa.phk, pa.a, a->v, a->state_in, nullptr, a->state_out, a->L, seq, a->o};
-      plan.add("gla_fwd_simt(exact fallback)",
-               [=](cudaStream_t s) { return lz::launch_gla_fwd_simt(ga, K, D, bf16, s); });
-    }
     return;
   }
   float *o_gla = nullptr;
@@ -438,6 +413,7 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan, bo
       const size_t Ld = up((size_t)a->L * a->dk * sizeof(float));
       const size_t o_phq = fb.scratch, o_phk = o_phq + K * Ld, o_a = o_phk + K * Ld, o_sp = o_a + K * Ld;
       const size_t o_kap = o_sp + K * up(nch32(a) * a->dk * a->dv * sizeof(float));
+      const size_t o_dpq = o_kap + K * up(a->dk * sizeof(float)), o_dpk = o_dpq + K * Ld;
       lz::PrepArgs pa{a->q, a->k, a->g, a->fmap_wq, a->fmap_wk, at<float>(ws, o_phq), at<float>(ws, o_phk),
                       at<float>(ws, o_a), a->H, a->L, inv_tau, scalar_gate(a), seq};
       plan.add("prep_kernel(exact fallback)", [=](cudaStream_t s) { return lz::launch_prep(pa, K, D, bf16, s); });
@@ -445,8 +421,8 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan, bo
       lz::GlaStatesArgs sa{pa.phk, pa.a, a->v, a->state_in, at<float>(ws, o_sp), a->L, b->dstate_out, kap, seq};
       plan.add("gla_states_simt(exact fallback)",
                [=](cudaStream_t s) { return lz::launch_gla_states(sa, K, D, bf16, s); });
-      lz::GlaBwdArgs ga{pa.phq, pa.phk, pa.a, a->v, b->dout, at<float>(ws, o_sp), at<float>(ws, lay.dphq),
-                        at<float>(ws, lay.dphk), at<float>(ws, lay.da), at<float>(ws, lay.dv_gla), b->dstate_in,
+      lz::GlaBwdArgs ga{pa.phq, pa.phk, pa.a, a->v, b->dout, at<float>(ws, o_sp), at<float>(ws, o_dpq),
+                        at<float>(ws, o_dpk), at<float>(ws, lay.da), at<float>(ws, lay.dv_gla), b->dstate_in,
                         a->L, b->dstate_out, kap, seq};
       plan.add("gla_bwd_simt(exact fallback)",
                [=](cudaStream_t s) { return lz::launch_gla_bwd_simt(ga, K, D, bf16, s); });
@@ -480,6 +456,20 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan, bo
                        b->dq, b->dk, b->dv, b->dg, b->dfmap_wq, b->dfmap_wk, a->H, a->L, inv_tau,
                        gla_tc ? 0 : 1, static_cast<uint32_t *>(ws), nullptr, nullptr, scalar_gate(a)};
   if (gla_tc) fa.da = nullptr;   // the gate gradient comes from gate_grad_kernel
+  if (finish_tc) {   // the tensor-core GLA backward's dphi: bf16, row halves centred
+    fa.dphq16 = at<void>(ws, lay.dphq);
+    fa.dphk16 = at<void>(ws, lay.dphk);
+    fa.dphq = fa.dphk = nullptr;
+    if (lay.fallback) {
+      const int K = fallback_slots(a);
+      const size_t Ld = up((size_t)a->L * a->dk * sizeof(float));
+      const size_t o_kap = lay.fb.scratch + 3 * K * Ld + K * up(nch32(a) * a->dk * a->dv * sizeof(float));
+      const size_t o_dpq = o_kap + K * up(a->dk * sizeof(float));
+      fa.slot_of = at<int>(ws, lay.fb.slot_of);
+      fa.fb_dphq = at<float>(ws, o_dpq);
+      fa.fb_dphk = at<float>(ws, o_dpq + K * Ld);
+    }
+  }
   lz::TcGlaBwdArgs tg{a->q, a->k, a->v, a->g, b->dout, a->fmap_wq, a->fmap_wk, nullptr, nullptr, nullptr,
                       nullptr, at<float>(ws, lay.da), nullptr, b->dg, nullptr, static_cast<uint32_t *>(ws),
                       a->H, BH, a->L, inv_tau, nullptr, nullptr, scalar_gate(a)};
@@ -560,7 +550,10 @@ size_t lizard_fwd_workspace_size(const lizard_fwd_args *args) {
   a.q = a.k = a.v = a.g = nullptr;
   a.o = nullptr;
   a.workspace = nullptr;
-  a.fmap_wq = a.fmap_wk = a.alpha = a.state_in = nullptr;
+  a.alpha = a.state_in = nullptr;
+  // whether feature-map weights are given selects the kernels (and so the layout)
+  a.fmap_wq = args->fmap_wq ? reinterpret_cast<const float *>(16) : nullptr;
+  a.fmap_wk = args->fmap_wk ? reinterpret_cast<const float *>(16) : nullptr;
   a.state_out = a.lse = nullptr;
   const bool meta = a.M > 0;
   a.meta_k = meta ? reinterpret_cast<const float *>(16) : nullptr;
@@ -629,7 +622,10 @@ size_t lizard_bwd_workspace_size(const lizard_bwd_args *args) {
   a.q = a.k = a.v = a.g = nullptr;
   a.o = nullptr;
   a.workspace = nullptr;
-  a.fmap_wq = a.fmap_wk = a.alpha = a.state_in = nullptr;
+  a.alpha = a.state_in = nullptr;
+  // whether feature-map weights are given selects the kernels (and so the layout)
+  a.fmap_wq = args->fwd.fmap_wq ? reinterpret_cast<const float *>(16) : nullptr;
+  a.fmap_wk = args->fwd.fmap_wk ? reinterpret_cast<const float *>(16) : nullptr;
   a.state_out = a.lse = nullptr;
   a.meta_k = a.M > 0 ? reinterpret_cast<const float *>(16) : nullptr;
   a.meta_v = nullptr;
@@ -769,7 +765,10 @@ size_t lizard_stage1_workspace_size(const lizard_stage1_args *args) {
   const bool keep_o = f.o != nullptr;
   f.q = f.k = f.v = f.g = nullptr;
   f.o = nullptr;
-  f.fmap_wq = f.fmap_wk = f.alpha = f.state_in = nullptr;
+  f.alpha = f.state_in = nullptr;
+  // whether feature-map weights are given selects the kernels (and so the layout)
+  f.fmap_wq = args->bwd.fwd.fmap_wq ? reinterpret_cast<const float *>(16) : nullptr;
+  f.fmap_wk = args->bwd.fwd.fmap_wk ? reinterpret_cast<const float *>(16) : nullptr;
   f.state_out = f.lse = nullptr;
   f.meta_k = f.M > 0 ? reinterpret_cast<const float *>(16) : nullptr;
   f.meta_v = nullptr;

@@ -1,23 +1,22 @@
-// Exact fallback of the tensor-core path for sequences whose cumulative
+// Exact fallback of the tensor-core backward for sequences whose cumulative
 // log-decay spans more than the tensor-core kernels' exponent range inside
 // one 128-token tile (the low-precision underflow that the log-space gate
 // absorption is about: Chinese gist.science summary, section 2.3; English
-// summary, section 2.C).
+// summary, section 2.C).  (The forward handles such sequences inside its
+// own kernel: tc_fwd.cu, exact_gla_sequence.)
 //
 // The tensor-core kernels absorb the decay of a tile as exp(b - r) and
 // exp(r - b) around one reference point r per tile.  When, in some key
 // dimension, the tile's log-decay spread exceeds kMaxSpread, those factors
 // leave the bf16 / fp32 exponent range.  The gate prep marks such sequences;
-// here they get slots (up to kFallbackSlots per call), the tensor-core
-// kernels leave out their GLA branch, and the portable kernels -- whose
-// chunked products use the element-wise exp(b_t - b_j), exact for any decay
-// -- compute it, one grid slot per marked sequence:
-//   forward:  o += o_gla (the tensor-core pass wrote alpha o_swa; the GLA
-//             kernel adds in place), state_out;
-//   backward: dphi_q, dphi_k, dv_gla, da and dstate_in into the same arrays
-//             the tensor-core kernels use, then dg from da at the end.
-// A marked sequence beyond the last slot keeps the tensor-core result and
-// sets the RANGE bit of the status word.
+// here they get slots (up to kFallbackSlots per call), and the portable
+// kernels -- whose chunked products use the element-wise exp(b_t - b_j),
+// exact for any decay -- rerun their GLA backward, one grid slot per marked
+// sequence: dphi_q, dphi_k (fp32, in the slot's arrays, which the feature-map
+// pass reads for these sequences), dv_gla, da and dstate_in into the arrays
+// the tensor-core kernels use, then dg from da at the end.  A marked
+// sequence beyond the last slot keeps the tensor-core result and sets the
+// RANGE bit of the status word.
 #include "common.cuh"
 #include "lizard_internal.h"
 

@@ -7,11 +7,11 @@
 
 namespace lz {
 
-// Exact fallback of the tensor-core path (sequences whose in-tile decay
+// Exact fallback of the tensor-core backward (sequences whose in-tile decay
 // spread leaves the tensor-core range): when seq_of_slot is set, the portable
-// GLA kernels below run one grid slot k per entry, on sequence
+// prep and GLA backward kernels run one grid slot k per entry, on sequence
 // bh = seq_of_slot[k] (nothing when it is negative); their scratch arrays
-// (phi, a, o_gla, chunk states, kap) are indexed by the slot k, their inputs
+// (phi, a, chunk states, kap, dphi) are indexed by the slot k, their inputs
 // and outputs by bh.
 struct PrepArgs {
   const void *q, *k, *g;
@@ -30,8 +30,6 @@ struct GlaFwdArgs {
   float *o_gla;
   float *state_out;
   int L;
-  const int *seq_of_slot;
-  void *o_add;   // when set (with seq_of_slot): o[bh] += o_gla in the activation dtype, o_gla not written
 };
 
 struct SwaMixArgs {
@@ -81,7 +79,7 @@ struct GlaBwdArgs {
   const float *phq, *phk, *a;
   const void *v, *dout;
   const float *sprev;
-  float *dphq, *dphk, *da, *dv_gla;
+  float *dphq, *dphk, *da, *dv_gla;   // in slot mode dphq, dphk are slot arrays too
   float *dstate_in;  // may be null
   int L;
   const float *dstate_out;   // [BH][D][D] gradient into the final state, or null (zero)
@@ -129,6 +127,14 @@ struct FinishBwdArgs {
   // dq, dk, dv to them.
   void *xq_part, *xk_part;
   int scalar_gate;   // g and dg hold one value per (token, head): [B*H][L]
+  // Tensor-core finish: the tensor-core GLA backward's dphi_q, dphi_k come as
+  // bf16 with each row's half centred (dphq16, dphk16, [B*H*L][128]; dphq,
+  // dphk then null), except for the sequences of the exact fallback
+  // (slot_of[bh] >= 0), whose fp32 dphi are in the fallback's slot arrays
+  // fb_dphq, fb_dphk ([K][L][128]).
+  const void *dphq16, *dphk16;
+  const int *slot_of;
+  const float *fb_dphq, *fb_dphk;
 };
 
 struct TcFwdArgs {
@@ -156,12 +162,11 @@ struct TcFwdArgs {
   // sum_v G[i][v] S_L[i][v] (null: none)
   const float *dstate_out;
   float *kap;
-  // Exact fallback (exact_fallback.cu): the gate prep marks sequences whose
-  // in-tile decay spread leaves the tensor-core range in seqflag [BH] (zeroed
-  // by the caller; null: it sets the status word's RANGE bit instead), and
-  // the passes leave the GLA branch out for sequences with slot_of[bh] >= 0.
+  // Wide decay: the gate prep marks sequences whose in-tile decay spread
+  // leaves the tensor-core range in seqflag [BH] (zeroed by the caller;
+  // null: it sets the status word's RANGE bit instead); the full pass then
+  // runs their GLA branch as the exact recurrence.
   uint32_t *seqflag;
-  const int *slot_of;
 };
 
 struct TcSwaBwdArgs {
@@ -190,7 +195,11 @@ struct TcGlaBwdArgs {
   const void *q, *k, *v, *g, *dout;
   const float *wq, *wk;
   void *snap_s, *snap_ds;       // bf16 [B*H][L/128][128][128]: S' and dS of every tile
-  float *dphq, *dphk, *dB, *dv; // fp32 [B*H*L][128]
+  // dphi_q, dphi_k: bf16 [B*H*L][128], each row's two halves centred (the
+  // feature map's softmax backward ignores a constant added to one half);
+  // dB, dv: fp32 [B*H*L][128]
+  void *dphq, *dphk;
+  float *dB, *dv;
   float *dg, *dstate_in;
   uint32_t *status;
   int H, BH, L;

@@ -246,9 +246,10 @@ __global__ void __launch_bounds__(256) gla_bwd_simt(GlaBwdArgs p) {
         const float ek = expf(r - bt);
         const float dk_ = Xk[a_][u] + ek * W;
         dB[a_][u] = Yq[a_][u] + Qb[t * D + i] * U - Yk[a_][u] - Kb[t * D + i] * W;
-        if (t < n) {
-          p.dphq[base + t * D + i] = dq_;
-          p.dphk[base + t * D + i] = dk_;
+        if (t < n) {   // in slot mode (exact fallback) dphi go to the slot's fp32 arrays
+          const size_t o = (p.seq_of_slot ? sbase : base) + t * D + i;
+          p.dphq[o] = dq_;
+          p.dphk[o] = dk_;
         }
       }
     }

@@ -132,12 +132,7 @@ __global__ void __launch_bounds__(256) gla_fwd_simt(GlaFwdArgs p) {
   float* A = Vs + C * D;              // [C][C]
   float* dec = A + C * C;             // [D] exp(r): state decay over the chunk
   float* eq = dec + D;                // [D] multiplier turning P1 into phi_q exp(b)
-  int bh = blockIdx.x;
-  const int sb = blockIdx.x;          // scratch row: the grid slot
-  if (p.seq_of_slot) {
-    bh = p.seq_of_slot[sb];
-    if (bh < 0) return;
-  }
+  const int bh = blockIdx.x;
   const int tid = threadIdx.x;
   const int tx = tid & 15, ty = tid >> 4;
   const T* vsrc = static_cast<const T*>(p.v);
@@ -146,15 +141,14 @@ __global__ void __launch_bounds__(256) gla_fwd_simt(GlaFwdArgs p) {
   __syncthreads();
   for (int c0 = 0; c0 < p.L; c0 += C) {
     const int n = min(C, p.L - c0);
-    const size_t base = ((size_t)sb * p.L + c0) * D;    // scratch
-    const size_t ibase = ((size_t)bh * p.L + c0) * D;   // inputs
+    const size_t base = ((size_t)bh * p.L + c0) * D;
     for (int e = tid; e < C * D; e += 256) {
       const int t = e / D;
       const bool ok = t < n;
       P1[e] = ok ? p.phq[base + e] : 0.f;
       P2[e] = ok ? p.phk[base + e] : 0.f;
       P3[e] = ok ? p.a[base + e] : 0.f;
-      Vs[e] = ok ? to_f32(vsrc[ibase + e]) : 0.f;
+      Vs[e] = ok ? to_f32(vsrc[base + e]) : 0.f;
     }
     __syncthreads();
     float spread = 0.f;
@@ -230,16 +224,9 @@ __global__ void __launch_bounds__(256) gla_fwd_simt(GlaFwdArgs p) {
 #pragma unroll
       for (int a_ = 0; a_ < 4; ++a_) {
         const int t = ty * 4 + a_;
-        if (t < n) {
-          if (p.o_add) {   // exact fallback: add to the output the anchor pass wrote
-            T *o = static_cast<T*>(p.o_add) + ibase + t * D + tx * VT;
+        if (t < n)
 #pragma unroll
-            for (int c = 0; c < VT; ++c) o[c] = from_f32<T>(to_f32(o[c]) + acc[a_][c]);
-          } else {
-#pragma unroll
-            for (int c = 0; c < VT; ++c) p.o_gla[base + t * D + tx * VT + c] = acc[a_][c];
-          }
-        }
+          for (int c = 0; c < VT; ++c) p.o_gla[base + t * D + tx * VT + c] = acc[a_][c];
       }
     }
     __syncthreads();

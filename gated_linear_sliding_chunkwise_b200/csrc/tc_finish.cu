@@ -31,7 +31,14 @@ struct Params {
   CUtensorMap mq, mk;
   CUtensorMap mxq, mxk;                    // bf16 dx_q, dx_k parts (fused mode)
   const float *wq, *wk;
-  const float *dphq, *dphk, *dv_gla;       // GLA parts (fp32), null when the branch is off
+  // GLA parts, null when the branch is off: dphi_q, dphi_k in bf16 with each
+  // row's halves centred (the softmax backward below ignores a constant added
+  // to a half), dv in fp32; the exact fallback's sequences (slot_of[bh] >= 0)
+  // have fp32 dphi in its slot arrays fb_dphq, fb_dphk [slot][L][D]
+  const __nv_bfloat16 *dphq, *dphk;
+  const float *dv_gla;
+  const int *slot_of;
+  const float *fb_dphq, *fb_dphk;
   const float *dq_swa, *dk_swa, *dv_swa;   // anchor parts (fp32), null when the branch is off
   __nv_bfloat16 *dq, *dk, *dv;
   float *dwq, *dwk;
@@ -99,12 +106,29 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
   // this row's dphi values (its group's half) of one map, loaded ahead: map 0
   // of the next tile while this tile finishes, map 1 while map 0 is used
   float4 dpre[16];
+  const int fb_slot = (gla && p.slot_of) ? p.slot_of[bh] : -1;
   auto dphi_load = [&](int m, int c) {
     const int t = c * T + row;
-    const float *src = (m == 0 ? p.dphq : p.dphk) + ((size_t)bh * p.L + (t < p.L ? t : 0)) * D + wg * F;
+    if (fb_slot >= 0) {   // the exact fallback's fp32 dphi
+      const float *src = (m == 0 ? p.fb_dphq : p.fb_dphk) + ((size_t)fb_slot * p.L + (t < p.L ? t : 0)) * D + wg * F;
 #pragma unroll
-    for (int u = 0; u < 16; ++u)
-      dpre[u] = t < p.L ? *reinterpret_cast<const float4 *>(src + 4 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int u = 0; u < 16; ++u)
+        dpre[u] = t < p.L ? *reinterpret_cast<const float4 *>(src + 4 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+      return;
+    }
+    const __nv_bfloat16 *src = (m == 0 ? p.dphq : p.dphk) + ((size_t)bh * p.L + (t < p.L ? t : 0)) * D + wg * F;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      float f[8];
+      if (t < p.L) {
+        unpack8(*reinterpret_cast<const uint4 *>(src + 8 * u), f);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) f[i] = 0.f;
+      }
+      dpre[2 * u] = make_float4(f[0], f[1], f[2], f[3]);
+      dpre[2 * u + 1] = make_float4(f[4], f[5], f[6], f[7]);
+    }
   };
   if (gla && ntiles > 0) dphi_load(0, 0);
   for (int c = 0; c < ntiles; ++c) {
@@ -299,9 +323,12 @@ cudaError_t launch_tc_finish(const FinishBwdArgs &a, int BH, cudaStream_t s) {
     return cudaErrorInvalidValue;
   p.wq = a.wq;
   p.wk = a.wk;
-  p.dphq = a.dphq;
-  p.dphk = a.dphk;
+  p.dphq = static_cast<const __nv_bfloat16 *>(a.dphq16);
+  p.dphk = static_cast<const __nv_bfloat16 *>(a.dphk16);
   p.dv_gla = a.dv_gla;
+  p.slot_of = a.slot_of;
+  p.fb_dphq = a.fb_dphq;
+  p.fb_dphk = a.fb_dphk;
   p.dq_swa = a.dq_swa;
   p.dk_swa = a.dk_swa;
   p.dv_swa = a.dv_swa;

@@ -40,11 +40,15 @@
 // state and total log-decay, a combine kernel chains them into each
 // segment's start state, and the full pass runs all segments in parallel.
 //
-// A tile whose in-tile log-decay spread exceeds kMaxSpread in some key
-// dimension sets the RANGE bit of the workspace status word (the portable
-// path computes such inputs exactly).  Every mbarrier wait is bounded; a
-// wait that gives up sets the TIMEOUT bit and the CTA stops, frees its TMEM
-// and returns.
+// A sequence with a tile whose in-tile log-decay spread exceeds kMaxSpread
+// in some key dimension (the gate prep marks it) cannot go through the
+// log-space absorption: its E = exp(b - r) leaves the exponent range.  The
+// CTA of its first segment then walks every tile for the anchor branch alone
+// and afterwards runs the GLA recurrence token by token in fp32 over the
+// whole sequence (exact for any decay), adding it to o (exact_gla_sequence);
+// the sequence's other CTAs return at once.  Every mbarrier wait is
+// bounded; a wait that gives up sets the TIMEOUT bit and the CTA stops,
+// frees its TMEM and returns.
 #include "common.cuh"
 #include "lizard_internal.h"
 #include "tc_common.cuh"
@@ -101,7 +105,12 @@ struct Params {
   int nseg, tiles_per_seg;
   int P;                    // prefix tokens before token 0 (0: none)
   int inject;               // test hook: first wait on a barrier nothing completes
-  const int *slot_of;       // exact fallback: sequences with slot_of[bh] >= 0 leave the GLA branch out
+  // Wide decay: seqflag[bh] != 0 marks a sequence whose GLA branch runs as
+  // the exact recurrence (exact_gla_sequence) instead; null: none.  Its
+  // inputs: the activations themselves.
+  const uint32_t *seqflag;
+  const __nv_bfloat16 *xq, *xk, *xv, *xg;
+  int scalar_gate;
   float inv_tau, scale;
   // stage-1 loss (target null: off): dmse = mse_grad (o - target), *loss += mse_loss sum (o - target)^2
   const __nv_bfloat16 *target;
@@ -184,6 +193,102 @@ __device__ __forceinline__ void kt_half(unsigned char *sm, uint32_t tl, int row,
   }
 }
 
+// The GLA branch of one whole sequence as the plain recurrence, for a
+// sequence whose decay is too wide for the tile absorption:
+//   S_t = diag(exp a_t) S_{t-1} + phi_k(k_t) v_t^T,   o_t += S_t^T phi_q(q_t)
+// in fp32 (the English summary's state update, section 2.A), exact for any
+// decay.  Thread (v = tid / 2, half = tid % 2) updates S[64 half .. 64 half +
+// 63][v] (fp32, in shared memory); the tokens go in chunks of 32, whose feature maps (from
+// the bf16 weights already staged at wq_s / wk_s), decays and values are
+// formed into shared memory first (warp per token).  o gets the GLA part
+// added (add: the anchor pass of this CTA wrote it) or written (the anchor
+// branch is off); state_out is written.
+constexpr int XC = 32;   // tokens per chunk of the exact recurrence
+__device__ __forceinline__ void exact_gla_sequence(const Params &p, unsigned char *buf, const unsigned char *wq_s,
+                                                const unsigned char *wk_s, int bh, bool add) {
+  float *PQ = reinterpret_cast<float *>(buf);          // [XC][D] phi_q
+  float *PK = PQ + XC * D;                             // [XC][D] phi_k
+  float *DEC = PK + XC * D;                            // [XC][D] exp(a)
+  float *VV = DEC + XC * D;                            // [XC][D] v
+  float *OB = VV + XC * D;                             // [XC][D] this chunk's GLA output
+  float *S = OB + XC * D;                              // [D][D] the state, row = key dimension
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int v = tid >> 1, half = tid & 1;
+  for (int e = tid; e < D * D; e += NTHREADS) S[e] = p.state_in ? p.state_in[(size_t)bh * D * D + e] : 0.f;
+  float *Sc = S + 64 * half * D + v;                   // this thread's column: Sc[ii * D]
+  for (int c0 = 0; c0 < p.L; c0 += XC) {
+    const int n = min(XC, p.L - c0);
+    // feature maps, decays and values of the chunk's tokens
+    for (int tt = warp; tt < n; tt += NTHREADS / 32) {
+      const size_t rowoff = ((size_t)bh * p.L + c0 + tt) * D;
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        const __nv_bfloat16 *x = (m == 0 ? p.xq : p.xk) + rowoff;
+        const unsigned char *W = m == 0 ? wq_s : wk_s;
+        float xr[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) xr[j] = __bfloat162float(x[lane + 32 * j]);
+        float z0 = 0.f, z1 = 0.f;   // z_f = sum_i x_i W[i][f], f = lane, lane + 32
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          for (int il = 0; il < 32; ++il) {
+            const float xi = __shfl_sync(0xffffffffu, xr[j], il);
+            const int i = 32 * j + il;
+            z0 = fmaf(xi, __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(W + sw128_offset(i, lane))), z0);
+            z1 = fmaf(xi, __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(W + sw128_offset(i, lane + 32))),
+                      z1);
+          }
+        const float mx = warp_max(fmaxf(z0, z1)), mn = -warp_max(-fminf(z0, z1));
+        const float p0 = expf(z0 - mx), p1 = expf(z1 - mx), n0 = expf(mn - z0), n1 = expf(mn - z1);
+        const float ip = 1.f / warp_sum(p0 + p1), in_ = 1.f / warp_sum(n0 + n1);
+        float *dst = (m == 0 ? PQ : PK) + tt * D;
+        dst[lane] = p0 * ip;
+        dst[lane + 32] = p1 * ip;
+        dst[64 + lane] = n0 * in_;
+        dst[96 + lane] = n1 * in_;
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = lane + 32 * j;
+        const float g = __bfloat162float(p.scalar_gate ? p.xg[(size_t)bh * p.L + c0 + tt] : p.xg[rowoff + i]);
+        const float a = (fminf(g, 0.f) - log1pf(expf(-fabsf(g)))) * p.inv_tau;   // logsigmoid(g) / tau
+        DEC[tt * D + i] = expf(a);
+        VV[tt * D + i] = __bfloat162float(p.xv[rowoff + i]);
+      }
+    }
+    __syncthreads();
+    for (int tt = 0; tt < n; ++tt) {
+      const float vt = VV[tt * D + v];
+      const float4 *dec = reinterpret_cast<const float4 *>(DEC + tt * D + 64 * half);
+      const float4 *pk = reinterpret_cast<const float4 *>(PK + tt * D + 64 * half);
+      const float4 *pq = reinterpret_cast<const float4 *>(PQ + tt * D + 64 * half);
+      float o = 0.f;
+#pragma unroll 4
+      for (int q4 = 0; q4 < 16; ++q4) {
+        const float4 d4 = dec[q4], k4 = pk[q4], f4 = pq[q4];
+        float *sc = Sc + 4 * q4 * D;
+        const float s0 = fmaf(d4.x, sc[0], k4.x * vt), s1 = fmaf(d4.y, sc[D], k4.y * vt);
+        const float s2 = fmaf(d4.z, sc[2 * D], k4.z * vt), s3 = fmaf(d4.w, sc[3 * D], k4.w * vt);
+        sc[0] = s0;
+        sc[D] = s1;
+        sc[2 * D] = s2;
+        sc[3 * D] = s3;
+        o = fmaf(s0, f4.x, fmaf(s1, f4.y, fmaf(s2, f4.z, fmaf(s3, f4.w, o))));
+      }
+      o += __shfl_xor_sync(0xffffffffu, o, 1);
+      if (half == 0) OB[tt * D + v] = o;
+    }
+    __syncthreads();
+    for (int e = tid; e < n * D; e += NTHREADS) {
+      __nv_bfloat16 *dst = p.o + ((size_t)bh * p.L + c0) * D + e;
+      *dst = __float2bfloat16_rn((add ? __bfloat162float(*dst) : 0.f) + OB[e]);
+    }
+    __syncthreads();
+  }
+  if (p.state_out)
+    for (int e = tid; e < D * D; e += NTHREADS) p.state_out[(size_t)bh * D * D + e] = S[e];
+}
+
 // Named barriers (id 0 is __syncthreads).
 constexpr int BAR_A = 1;       // both groups' row maxima written
 constexpr int BAR_B = 2;       // both groups' row sums written, all logits read
@@ -216,12 +321,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
   const int bh = blockIdx.x, h = bh % p.H, seg = blockIdx.y;
   const float alpha = p.alpha ? p.alpha[h] : 1.f;
   constexpr bool full = KIND != K_STATE;
-  // a sequence taken by the exact fallback runs the anchor branch only here
-  const bool gla = p.branch != 2 && !(p.slot_of && p.slot_of[bh] >= 0), swa = full && p.branch != 1;
+  // A sequence marked for the exact recurrence: its first segment's CTA of
+  // the full pass walks every tile for the anchor branch, then runs the GLA
+  // branch exactly; its other CTAs (and state passes) have nothing to do.
+  const bool marked = p.seqflag && p.seqflag[bh] != 0u;
+  if (marked && (!full || seg > 0)) return;
+  const bool gla = p.branch != 2 && !marked, swa = full && p.branch != 1;
   const uint32_t sbase = smem_u32(sm);
   const int ntiles_all = (p.L + T - 1) / T;
-  const int cbeg = seg * p.tiles_per_seg;
-  const int cend = min(ntiles_all, cbeg + p.tiles_per_seg);
+  const int cbeg = marked ? 0 : seg * p.tiles_per_seg;
+  const int cend = marked ? ntiles_all : min(ntiles_all, cbeg + p.tiles_per_seg);
 
   if (warp == 0) {
     tmem_alloc(&s_tmem, 512);
@@ -339,27 +448,28 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       //      The meta logits (CUDA cores, from X_q in shared memory) and the
       //      tile's decay exp(r) are formed while MMA 1 runs.
       float pmeta = kNegBig;
-      if (swa && wg == 0) {
-        // meta logits q . mk_m (scaled) into s_ml, four meta tokens per pass
-        for (int m0 = 0; m0 < p.M; m0 += 4) {
-          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (swa) {
+        // meta logits q . mk_m (scaled) into s_ml: group wg takes the meta
+        // tokens wg, wg + 2, ..., two per pass
+        for (int m0 = wg; m0 < p.M; m0 += 4) {
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 4
           for (int ch = 0; ch < 16; ++ch) {
             float q8[8];
             unpack8(*chunk_ptr(sm, R_XQ, row, ch), q8);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const float4 a = *reinterpret_cast<const float4 *>(&s_mk[m0 + k][ch * 8]);
-              const float4 b = *reinterpret_cast<const float4 *>(&s_mk[m0 + k][ch * 8 + 4]);
+            for (int k = 0; k < 2; ++k) {
+              const float4 a = *reinterpret_cast<const float4 *>(&s_mk[m0 + 2 * k][ch * 8]);
+              const float4 b = *reinterpret_cast<const float4 *>(&s_mk[m0 + 2 * k][ch * 8 + 4]);
               acc[2 * k] = fmaf(q8[0], a.x, fmaf(q8[1], a.y, fmaf(q8[2], a.z, fmaf(q8[3], a.w, acc[2 * k]))));
               acc[2 * k + 1] = fmaf(q8[4], b.x, fmaf(q8[5], b.y, fmaf(q8[6], b.z, fmaf(q8[7], b.w, acc[2 * k + 1]))));
             }
           }
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            if (m0 + k < p.M) {
+          for (int k = 0; k < 2; ++k)
+            if (m0 + 2 * k < p.M) {
               const float l = (acc[2 * k] + acc[2 * k + 1]) * p.scale;
-              s_ml[m0 + k][row] = l;
+              s_ml[m0 + 2 * k][row] = l;
               pmeta = fmaxf(pmeta, l);
             }
         }
@@ -370,37 +480,42 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       float lsum = 1.f, mx = 0.f;                 // row normaliser and max (scaled logits)
       // Logit column cl holds key t0 - T + cl.  Row r sees columns
       // [r + T + 1 - window, r + T] (and keys >= -P, P the prefix length),
-      // so warp w4 only visits 32-column chunks w4 + (T + 1 - window) / 32
-      // .. w4 + 4, and only the first and last of those need the band mask.
+      // so warp w4 only visits the 16-column half-chunks from
+      // (32 w4 + T + 1 - window) / 16 to 2 w4 + 9 (ten at window 128, five
+      // per group: group wg the ones hc_lo + wg, hc_lo + wg + 2, ...), and
+      // only those at the band's edges need the mask.
       const int w4 = warp & 3;
       const int cbase = t0 - T;
       const int lo_c = max(tq - p.window + 1, -p.P) - cbase, hi_c = tq - cbase;
-      int ch_lo = (32 * w4 + T + 1 - p.window) >> 5;
-      if (cbase < 0) ch_lo = max(ch_lo, (T - p.P) >> 5);
-      const int ch_hi = w4 + 4;
-      const int in_lo = 32 * w4 + 31 + T + 1 - p.window;   // interior chunk: 32 ch >= in_lo
-      const int ch_first = ch_lo + 1 - wg;                 // this group's first chunk
-      uint32_t pk[3][16];
-      // this group's logit chunks, read from TMEM once (the stage-1 instance,
-      // short of registers, reads them again for the exponentials)
-      constexpr int KEPT = LOSS ? 1 : 3;
-      float lv[KEPT][32];
+      int hc_lo = (32 * w4 + T + 1 - p.window) >> 4;
+      if (cbase < 0) hc_lo = max(hc_lo, (T - p.P) >> 4);
+      const int hc_hi = 2 * w4 + 9;
+      const int in_lo = 32 * w4 + 31 + T + 1 - p.window;   // interior half-chunk: 16 hc >= in_lo
+      const int hc_first = hc_lo + wg;                     // this group's first half-chunk
+      constexpr int NH = 5;                                // half-chunks per group, at most
+      uint32_t pk[NH][8];
+      // this group's logit half-chunks, all five loads in flight together
+      // (a half-chunk past the band reloads the last one and is skipped)
+      uint32_t la[NH];
+#pragma unroll
+      for (int k = 0; k < NH; ++k) la[k] = tl + C_L + 16 * min(hc_first + 2 * k, hc_hi);
+      float lv[NH][16];
       if (swa) {
         float pmax = pmeta;
+        tmem_ld16x5(la, lv);
 #pragma unroll
-        for (int k = 0; k < 3; ++k) {
-          const int ch = ch_first + 2 * k;
-          if (ch > ch_hi) continue;
-          float *v = lv[LOSS ? 0 : k];
-          tmem_ld32(tl + C_L + ch * 32, v);
+        for (int k = 0; k < NH; ++k) {
+          const int hc = hc_first + 2 * k;
+          if (hc > hc_hi) continue;
+          float *v = lv[k];
           float m4[4] = {kNegBig, kNegBig, kNegBig, kNegBig};
-          if (32 * ch >= in_lo && 32 * ch + 31 <= 32 * w4 + T && 32 * ch + cbase >= -p.P) {
+          if (16 * hc >= in_lo && 16 * hc + 15 <= 32 * w4 + T && 16 * hc + cbase >= -p.P) {
 #pragma unroll
-            for (int u = 0; u < 32; ++u) m4[u & 3] = fmaxf(m4[u & 3], v[u]);
+            for (int u = 0; u < 16; ++u) m4[u & 3] = fmaxf(m4[u & 3], v[u]);
           } else {
 #pragma unroll
-            for (int u = 0; u < 32; ++u) {
-              const int cl = 32 * ch + u;
+            for (int u = 0; u < 16; ++u) {
+              const int cl = 16 * hc + u;
               if (cl >= lo_c && cl <= hi_c) m4[u & 3] = fmaxf(m4[u & 3], v[u]);
             }
           }
@@ -413,21 +528,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       if (swa) {
         mx = fmaxf(s_pmax[0][row], s_pmax[1][row]);
         // P^ = exp(l - max), packed and held until both groups have read
-        // their logits (P^ column 16 ch overlays logit chunk ch / 2)
+        // their logits (P^ column 8 hc overlays logit half-chunk hc / 2)
         float s4[4] = {0.f, 0.f, 0.f, 0.f};
+        tmem_ld16x5(la, lv);   // again: the registers are needed in between
 #pragma unroll
-        for (int k = 0; k < 3; ++k) {
-          const int ch = ch_first + 2 * k;
-          if (ch > ch_hi) continue;
-          const float *v = lv[LOSS ? 0 : k];
-          if (LOSS) tmem_ld32(tl + C_L + ch * 32, lv[0]);
-          const bool inner = 32 * ch >= in_lo && 32 * ch + 31 <= 32 * w4 + T && 32 * ch + cbase >= -p.P;
+        for (int k = 0; k < NH; ++k) {
+          const int hc = hc_first + 2 * k;
+          if (hc > hc_hi) continue;
+          const float *v = lv[k];
+          const bool inner = 16 * hc >= in_lo && 16 * hc + 15 <= 32 * w4 + T && 16 * hc + cbase >= -p.P;
 #pragma unroll
-          for (int u = 0; u < 32; u += 2) {
+          for (int u = 0; u < 16; u += 2) {
             float e0 = __expf(fmaf(v[u], p.scale, -mx));
             float e1 = __expf(fmaf(v[u + 1], p.scale, -mx));
             if (!inner) {
-              const int cl = 32 * ch + u;
+              const int cl = 16 * hc + u;
               e0 = (cl >= lo_c && cl <= hi_c) ? e0 : 0.f;
               e1 = (cl + 1 >= lo_c && cl + 1 <= hi_c) ? e1 : 0.f;
             }
@@ -436,12 +551,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
           }
         }
         float psum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-        if (wg == 0)
-          for (int m = 0; m < p.M; ++m) {
-            const float e = __expf(s_ml[m][row] - mx);
-            psum += e;
-            s_ml[m][row] = e;
-          }
+        for (int m = wg; m < p.M; m += 2) {   // this group's meta tokens
+          const float e = __expf(s_ml[m][row] - mx);
+          psum += e;
+          s_ml[m][row] = e;
+        }
         s_psum[wg][row] = psum;
       }
       bar_sync(BAR_B, NTHREADS);
@@ -449,17 +563,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         lsum = s_psum[0][row] + s_psum[1][row];
         if (!qvalid) lsum = 1.f;
 #pragma unroll
-        for (int k = 0; k < 3; ++k) {
-          const int ch = ch_first + 2 * k;
-          if (ch > ch_hi) continue;
-          tmem_st8(tl + C_P + ch * 16, pk[k]);
-          tmem_st8(tl + C_P + ch * 16 + 8, pk[k] + 8);
+        for (int k = 0; k < NH; ++k) {
+          const int hc = hc_first + 2 * k;
+          if (hc > hc_hi) continue;
+          tmem_st8(tl + C_P + hc * 8, pk[k]);
         }
         uint32_t zero[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-        for (int ch = wg; ch < 8; ch += 2) {   // chunks outside the band: P = 0
-          if (ch >= ch_lo && ch <= ch_hi) continue;
-          tmem_st8(tl + C_P + ch * 16, zero);
-          tmem_st8(tl + C_P + ch * 16 + 8, zero);
+        for (int hc = wg; hc < 16; hc += 2) {   // half-chunks outside the band: P = 0
+          if (hc >= hc_lo && hc <= hc_hi) continue;
+          tmem_st8(tl + C_P + hc * 8, zero);
         }
         if (wg == 0 && qvalid && p.lse) p.lse[(size_t)bh * p.L + tq] = mx + logf(lsum);
       }
@@ -526,9 +638,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       tc_fence_after();
       const int i = row;
       const float dec = s_dec[i];
-      for (int c16 = 4 * wg; c16 < 4 * wg + 4; ++c16) {
-        float v[16];
-        tmem_ld16(tl + C_S + c16 * 16, v);
+#pragma unroll 1
+      for (int c32 = 2 * wg; c32 < 2 * wg + 2; ++c32) {   // two 16-column loads in flight together
+        float vv[2][16];
+        tmem_ld16x2(tl + C_S + c32 * 32, tl + C_S + c32 * 32 + 16, vv[0], vv[1]);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+        const int c16 = 2 * c32 + hh;
+        float *v = vv[hh];
         uint32_t r[8];
 #pragma unroll
         for (int u = 0; u < 16; ++u) v[u] *= dec;
@@ -544,6 +661,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         } else if (p.snap && i == 0) {
 #pragma unroll
           for (int u = 0; u < 16; ++u) s_row0[c16 * 16 + u] = v[u];
+        }
         }
       }
       if (!full && p.snap) {
@@ -571,9 +689,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
 
     // ---------------------- masked intra A (column half per group) ---
     if (gla && full) {
-      for (int c16 = 4 * wg; c16 < 4 * wg + 4; ++c16) {
-        float v[16];
-        tmem_ld16(tl + C_A + c16 * 16, v);
+#pragma unroll 1
+      for (int c32 = 2 * wg; c32 < 2 * wg + 2; ++c32) {
+        float vv[2][16];
+        tmem_ld16x2(tl + C_A + c32 * 32, tl + C_A + c32 * 32 + 16, vv[0], vv[1]);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+        const int c16 = 2 * c32 + hh;
+        const float *v = vv[hh];
         uint32_t r[8];
 #pragma unroll
         for (int u = 0; u < 16; u += 2) {
@@ -584,6 +707,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
           r[u / 2] = pack_bf16(a0, a1);
         }
         tmem_st8(tl + C_AH + c16 * 8, r);
+        }
       }
     }
     tmem_st_wait();
@@ -628,11 +752,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       // tcgen05.ld is warp-collective: every lane loads, valid rows store
       const size_t roff = ((size_t)bh * p.L + (qvalid ? tq : 0)) * D;
       const float oscale = s_oscale[row];
-#pragma unroll(LOSS ? 4 : 1)
+      float vall[64];   // this group's 64 columns of O, all four loads in flight together
+      tmem_ld32x2(tl + C_O + 64 * wg, tl + C_O + 64 * wg + 32, vall, vall + 32);
+#pragma unroll
       for (int k4 = 0; k4 < 4; ++k4) {
         const int c16 = 4 * wg + k4;
-        float v[16];
-        tmem_ld16(tl + C_O + c16 * 16, v);
+        float *v = vall + 16 * k4;
 #pragma unroll
         for (int u = 0; u < 16; ++u) v[u] *= oscale;
         if (swa && p.meta_v) {
@@ -719,6 +844,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tb, 512);
+  // every tile's loads and MMAs are done: the tile regions hold the exact
+  // recurrence's buffers, the staged weights stay in place
+  if (marked && !s_fail && p.branch != 2) exact_gla_sequence(p, sm, sm + R_WQ, sm + R_WK, bh, p.branch != 1);
 }
 
 }  // namespace
@@ -1057,7 +1185,12 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, int stage, cudaStream_t s) {
   p.seg_start = w.seg_start;
   p.seg_state = w.seg_state;
   p.seg_decay = w.seg_decay;
-  p.slot_of = a.slot_of;
+  p.seqflag = a.seqflag;
+  p.xq = static_cast<const __nv_bfloat16 *>(a.q);
+  p.xk = static_cast<const __nv_bfloat16 *>(a.k);
+  p.xv = static_cast<const __nv_bfloat16 *>(a.v);
+  p.xg = static_cast<const __nv_bfloat16 *>(a.g);
+  p.scalar_gate = a.scalar_gate;
   p.H = a.H;
   p.L = a.L;
   p.M = a.M;

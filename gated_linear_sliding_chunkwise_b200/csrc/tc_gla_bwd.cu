@@ -28,7 +28,11 @@
 //                        copies) and the gradient of the initial state.
 // tc_gla_bwd_tile_kernel the formulas above per 128-token tile, given the
 //                        S' and dS copies; one persistent CTA per SM walks a
-//                        contiguous run of (sequence, tile) items.
+//                        contiguous run of (sequence, tile) items.  dB and dv
+//                        go out in fp32; dphi_q and dphi_k in bf16, each
+//                        half-row shifted by its first value (the feature
+//                        map's softmax backward ignores a constant per half,
+//                        and the shift takes out the part all features share).
 // gate_grad_kernel       reverse cumulative sum of dB -> gate-logit gradient.
 #include "common.cuh"
 #include "lizard_internal.h"
@@ -63,10 +67,10 @@ struct DsParams {
 struct TileParams {
   CUtensorMap mq, mk, mv, mo, msp, mds;       // msp / mds: [BH*ntiles][D][D] snapshots
   CUtensorMap mw;                             // [H*2][D][F] bf16 feature-map weights (W_q, W_k per head)
-  CUtensorMap mdq, mdk, mdb, mdv;             // fp32 outputs dphi_q, dphi_k, dB, dv (TMA stores)
+  CUtensorMap mdq, mdk;                       // bf16 outputs dphi_q, dphi_k, row halves centred (TMA stores)
+  CUtensorMap mdb, mdv;                       // fp32 outputs dB, dv (TMA stores)
   const float *e32;            // fp32 decay factors [BH*L][D]
   const float *sp_r0, *ds_r0;  // [BH*ntiles][D] row 0 of S' and of dS (the copies hold the rest)
-  float *dphq, *dphk, *dB, *dv;
   uint32_t *status;
   int H, L, ntiles, BH;
   float inv_tau;
@@ -544,7 +548,7 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
       pend0 = (int)(par ^ 1u);
       item_loads(w + 1, 0);
     }
-    unsigned char *st0 = sm + R_V, *st1 = sm + R_QL, *st2 = sm + R_XQ;
+    unsigned char *st0 = sm + R_V;
     // rank-one parts of GQ and GK left out of the S' and dS copies
     const float cq = s_r1[0][row], ck = s_r1[1][row], kap = s_r1[2][row];
     for (int c16 = 4 * wg; c16 < 4 * wg + 4; ++c16) {
@@ -556,6 +560,7 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
         gq[u] += cq;
         gk[u] += ck;
       }
+
       unpack8(*chunk_ptr(sm, R_XQ, row, 2 * c16), q16);
       unpack8(*chunk_ptr(sm, R_XQ, row, 2 * c16 + 1), q16 + 8);
       unpack8(*chunk_ptr(sm, R_QL, row, 2 * c16), lo);
@@ -581,6 +586,13 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
       bulk_commit();
     }
     if (tid < 32) *reinterpret_cast<float4 *>(s_row0 + D + 4 * tid) = ds0;   // read after two barriers
+    // dphi_q - c_q (bf16) over Qt lo, dphi_k - c_k over Qt hi, one 32 KB
+    // swizzled bf16 tile each, c the half-row's first value: a constant added
+    // to one half of a row leaves the feature map's softmax backward
+    // unchanged, so the finish pass reads them as they are, and taking out
+    // the part all features share keeps the per-feature differences that the
+    // backward uses at full bf16 precision
+    float mq = 0.f, mk = 0.f;
 #pragma unroll
     for (int k4 = 0; k4 < 4; ++k4) {
       const int c16 = 4 * wg + k4;
@@ -592,23 +604,34 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
         gq[u] += cq;
         gk[u] += ck;
       }
+      if (k4 == 0) {
+        mq = e4[0].x * gq[0];
+        mk = __fdividef(gk[0], e4[0].x);
+      }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const float4 E = e4[4 * k4 + u];
-        *f32_stage_ptr(st1, row, c16 * 16 + 4 * u) =
-            make_float4(E.x * gq[4 * u], E.y * gq[4 * u + 1], E.z * gq[4 * u + 2], E.w * gq[4 * u + 3]);
-        *f32_stage_ptr(st2, row, c16 * 16 + 4 * u) =
-            make_float4(__fdividef(gk[4 * u], E.x), __fdividef(gk[4 * u + 1], E.y),
-                        __fdividef(gk[4 * u + 2], E.z), __fdividef(gk[4 * u + 3], E.w));
+        gq[4 * u] = E.x * gq[4 * u] - mq;
+        gq[4 * u + 1] = E.y * gq[4 * u + 1] - mq;
+        gq[4 * u + 2] = E.z * gq[4 * u + 2] - mq;
+        gq[4 * u + 3] = E.w * gq[4 * u + 3] - mq;
+        gk[4 * u] = __fdividef(gk[4 * u], E.x) - mk;
+        gk[4 * u + 1] = __fdividef(gk[4 * u + 1], E.y) - mk;
+        gk[4 * u + 2] = __fdividef(gk[4 * u + 2], E.z) - mk;
+        gk[4 * u + 3] = __fdividef(gk[4 * u + 3], E.w) - mk;
       }
+      *chunk_ptr(sm, R_QL, row, 2 * c16) = pack8(gq);
+      *chunk_ptr(sm, R_QL, row, 2 * c16 + 1) = pack8(gq + 8);
+      *chunk_ptr(sm, R_XQ, row, 2 * c16) = pack8(gk);
+      *chunk_ptr(sm, R_XQ, row, 2 * c16 + 1) = pack8(gk + 8);
     }
     if (more) e_load(w + 1, epre);   // the next item's decay factors, in flight during the dv pass
     fence_proxy_async();
     __syncthreads();
     if (tid == 0) {
-      for (int bx = 0; bx < 4; ++bx) {
-        tma_store_3d(&p.mdq, st1 + bx * 16384, 32 * bx, t0, bh);
-        tma_store_3d(&p.mdk, st2 + bx * 16384, 32 * bx, t0, bh);
+      for (int r = 0; r < 2; ++r) {
+        tma_store_3d(&p.mdq, sm + R_QL + r * REG, 64 * r, t0, bh);
+        tma_store_3d(&p.mdk, sm + R_XQ + r * REG, 64 * r, t0, bh);
       }
       bulk_commit();
       bulk_wait_read_but_last();   // the dB tile has been read out of V | dO
@@ -835,16 +858,13 @@ cudaError_t launch_tc_gla_bwd(const TcGlaBwdArgs &a, int stage, cudaStream_t s) 
         !make_map_bf16_3d(&p.msp, a.snap_s, D, D, (uint64_t)a.BH * ntiles, T) ||
         !make_map_bf16_3d(&p.mw, a.w16, F, D, (uint64_t)a.H * 2, T) ||
         !make_map_bf16_3d(&p.mds, a.snap_ds, D, D, (uint64_t)a.BH * ntiles, T) ||
-        !make_map_f32_3d(&p.mdq, a.dphq, D, rows, a.BH, T) || !make_map_f32_3d(&p.mdk, a.dphk, D, rows, a.BH, T) ||
+        !make_map_bf16_3d(&p.mdq, a.dphq, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mdk, a.dphk, D, rows, a.BH, T) ||
         !make_map_f32_3d(&p.mdb, a.dB, D, rows, a.BH, T) || !make_map_f32_3d(&p.mdv, a.dv, D, rows, a.BH, T))
       return cudaErrorInvalidValue;
     p.e32 = a.e32;
     p.sp_r0 = snapshot_row0(a.snap_s, a.BH, a.L);
     p.ds_r0 = snapshot_row0(a.snap_ds, a.BH, a.L);
-    p.dphq = a.dphq;
-    p.dphk = a.dphk;
-    p.dB = a.dB;
-    p.dv = a.dv;
+
     p.status = a.status;
     p.H = a.H;
     p.L = a.L;

@@ -54,11 +54,11 @@
  *     cumulative log-decay of some key dimension spans more than 64 (gate
  *     logits below about -8 per token at gate_temp 16), the tensor-core
  *     kernels' log-space factors leave their exponent range.  Such sequences
- *     get the GLA branch from the portable kernels instead (exact for any
- *     decay), up to 4 of them per call; a fifth and later one in the same call
- *     keeps the tensor-core result, and the call records LIZARD_ERR_RANGE.
- *     lizard_stage1_step has no such fallback: it records LIZARD_ERR_RANGE
- *     for any of them.
+ *     get their GLA branch computed exactly instead: in lizard_attn_fwd, any
+ *     number of them; in lizard_attn_bwd, up to 4 of them per call (a fifth
+ *     and later one keeps the tensor-core result, and the call records
+ *     LIZARD_ERR_RANGE).  lizard_stage1_step has no such fallback: it records
+ *     LIZARD_ERR_RANGE for any of them.
  */
 #ifndef LIZARD_H_
 #define LIZARD_H_
@@ -79,7 +79,7 @@ typedef enum {
   LIZARD_ERR_CUDA = 3,        /* a launch or CUDA runtime call failed */
   LIZARD_ERR_TIMEOUT = 4,     /* a kernel gave up on a bounded wait */
   LIZARD_ERR_WORKSPACE = 5,   /* workspace NULL or smaller than the queried size */
-  LIZARD_ERR_RANGE = 6        /* tensor-core path: more wide-decay sequences than its exact fallback takes */
+  LIZARD_ERR_RANGE = 6        /* tensor-core backward: more wide-decay sequences than its exact fallback takes */
 } lizard_status;
 
 typedef enum { LIZARD_BF16 = 0, LIZARD_FP32 = 1 } lizard_dtype;
@@ -167,8 +167,9 @@ typedef struct {
   int32_t prefix_len;
 } lizard_fwd_args;
 
-/* Bytes of device workspace the forward needs for these arguments (pointer
- * fields are ignored).  Returns 0 when the sizes are invalid. */
+/* Bytes of device workspace the forward needs for these arguments.  Pointer
+ * fields are ignored, except whether fmap_wq / fmap_wk are given (that
+ * selects the kernels).  Returns 0 when the sizes are invalid. */
 size_t lizard_fwd_workspace_size(const lizard_fwd_args *args);
 
 /* Enqueue the forward.  See the conventions above for errors. */

@@ -163,6 +163,21 @@ def test_tc_backward_computes_wide_decay_exactly(lz, impl, gate, with_g):
         check(f"{name} ({gate} gate)", got[name], want[name], "bf16")
 
 
+def test_tc_backward_flags_wide_decay_beyond_its_fallback_slots(lz):
+    """More sequences with wide decay in one backward call than its exact
+    fallback has slots (four): the status word says RANGE; a call without
+    such gates reads OK again."""
+    w = Workload("brange_many", B=3, H=2, L=256, d=128, window=128, M=4, dtype="bf16", seed=2, kind="train")
+    inp = make_inputs(w)
+    g = inp["g"].clone()
+    g[:, :, 130:200, :3] = -300.0
+    inp["g"] = g
+    got = _run(lz, to_device(inp), w, lz.IMPL_TC)
+    assert lz.workspace_status(got["workspace"]) == lz.ERR_RANGE
+    ok = _run(lz, to_device(make_inputs(w)), w, lz.IMPL_TC)
+    assert lz.workspace_status(ok["workspace"]) == lz.OK
+
+
 @pytest.mark.parametrize("impl", IMPLS)
 def test_parameter_grads_bf16_full_reduction(lz, impl):
     """Gradients of the per-head parameters reduce over batch and tokens:

@@ -152,10 +152,11 @@ def _wide_decay(inp, heads):
 @pytest.mark.parametrize("impl", ["tc", "auto"])
 @pytest.mark.parametrize("gate", ["dim", "scalar"])
 def test_tc_path_computes_wide_decay_exactly(lz, impl, gate):
-    """Sequences whose in-tile decay spread leaves the tensor-core range go
-    to the exact fallback (their GLA branch on the portable kernels): the
-    output, final state and normaliser match the oracle, the status is OK,
-    and the other sequences of the call stay on the tensor cores."""
+    """Sequences whose in-tile decay spread leaves the tensor-core range get
+    their GLA branch from the exact token-by-token recurrence inside the
+    forward kernel: the output, final state and normaliser match the oracle,
+    the status is OK, and the other sequences of the call stay on the tensor
+    cores."""
     w = Workload("range", B=2, H=3, L=300, d=128, window=128, M=4, dtype="bf16", seed=2, gate=gate)
     inp = _wide_decay(make_inputs(w), [(0, 1), (1, 2)])
     inp["state_in"] = torch.randn(2, 3, 128, 128, generator=torch.Generator().manual_seed(3)) * 0.1
@@ -179,16 +180,18 @@ def test_tc_wide_decay_in_a_segmented_forward(lz):
     check("state_out", got["state_out"], want["state_out"], "bf16")
 
 
-def test_tc_flags_wide_decay_beyond_its_fallback_slots(lz):
-    """More marked sequences in one call than the exact fallback has slots
-    (four): the ones beyond keep the tensor-core result and the status word
-    says RANGE; a call without such gates reads OK again."""
+@pytest.mark.parametrize("branch", [ref.BRANCH_BOTH, ref.BRANCH_GLA_ONLY])
+def test_tc_forward_computes_every_marked_sequence_exactly(lz, branch):
+    """Every sequence of a call marked for wide decay (the forward has no
+    limit on how many): all of them match the oracle, also with the anchor
+    branch off (the exact recurrence then writes o rather than adds to it)."""
     w = Workload("range_many", B=3, H=2, L=256, d=128, window=128, M=4, dtype="bf16", seed=2)
     inp = _wide_decay(make_inputs(w), [(b, h) for b in range(3) for h in range(2)])
-    got = _run(lz, to_device(inp), w, lz.IMPL_TC)
-    assert lz.workspace_status(got["workspace"]) == lz.ERR_RANGE
-    ok = _run(lz, to_device(make_inputs(w)), w, lz.IMPL_TC)
-    assert lz.workspace_status(ok["workspace"]) == lz.OK
+    got = _run(lz, to_device(inp), w, lz.IMPL_TC, want_state=True, branch=branch)
+    assert lz.workspace_status(got["workspace"]) == lz.OK
+    want = oracle_forward(inp, window=w.window, tau=w.gate_temp, branch=branch)
+    check("o", got["o"], want["o"], "bf16")
+    check("state_out", got["state_out"], want["state_out"], "bf16")
 
 
 @pytest.mark.parametrize("impl", ["simt"])
