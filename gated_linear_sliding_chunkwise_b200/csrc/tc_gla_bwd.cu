@@ -393,18 +393,24 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
   //    (row = key, query j >= row); packed bf16 into [0,128)
   {
     const uint32_t src = wg == 0 ? C_DA : C_DAT, dst = wg == 0 ? C_DAH : C_DATH;
-    for (int ch = 0; ch < 4; ++ch) {
-      float v[32];
-      tmem_ld32(tl + src + ch * 32, v);
-      uint32_t a[16];
+#pragma unroll 1
+    for (int c2 = 0; c2 < 2; ++c2) {
+      float dav[2][32];
+      tmem_ld32x2(tl + src + c2 * 64, tl + src + c2 * 64 + 32, dav[0], dav[1]);
 #pragma unroll
-      for (int u = 0; u < 32; u += 2) {
-        const int j = ch * 32 + u;
-        const bool k0 = wg == 0 ? j <= row : j >= row, k1 = wg == 0 ? j + 1 <= row : j + 1 >= row;
-        a[u / 2] = pack_bf16(k0 ? v[u] : 0.f, k1 ? v[u + 1] : 0.f);
+      for (int h = 0; h < 2; ++h) {
+        const int ch = 2 * c2 + h;
+        const float *v = dav[h];
+        uint32_t a[16];
+#pragma unroll
+        for (int u = 0; u < 32; u += 2) {
+          const int j = ch * 32 + u;
+          const bool k0 = wg == 0 ? j <= row : j >= row, k1 = wg == 0 ? j + 1 <= row : j + 1 >= row;
+          a[u / 2] = pack_bf16(k0 ? v[u] : 0.f, k1 ? v[u + 1] : 0.f);
+        }
+        tmem_st8(tl + dst + ch * 16, a);
+        tmem_st8(tl + dst + ch * 16 + 8, a + 8);
       }
-      tmem_st8(tl + dst + ch * 16, a);
-      tmem_st8(tl + dst + ch * 16 + 8, a + 8);
     }
   }
   tmem_st_wait();
@@ -478,9 +484,12 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
   tc_fence_after();
   //    A^T^ = A^T masked to queries j >= key row, packed bf16 into TMEM over
   //    the spent E columns, 64 query columns per group
-  for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
-    float v[32];
-    tmem_ld32(tl + C_AT + ch * 32, v);
+  float atv[2][32];
+  tmem_ld32x2(tl + C_AT + 64 * wg, tl + C_AT + 64 * wg + 32, atv[0], atv[1]);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int ch = 2 * wg + h;
+    const float *v = atv[h];
     uint32_t a[16];
 #pragma unroll
     for (int u = 0; u < 32; u += 2) {
@@ -553,8 +562,7 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
     const float cq = s_r1[0][row], ck = s_r1[1][row], kap = s_r1[2][row];
     for (int c16 = 4 * wg; c16 < 4 * wg + 4; ++c16) {
       float gq[16], gk[16], q16[16], k16[16], lo[16];
-      tmem_ld16(tl + C_GQ + c16 * 16, gq);
-      tmem_ld16(tl + C_GK + c16 * 16, gk);
+      tmem_ld16x2(tl + C_GQ + c16 * 16, tl + C_GK + c16 * 16, gq, gk);
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
         gq[u] += cq;
@@ -597,8 +605,7 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
     for (int k4 = 0; k4 < 4; ++k4) {
       const int c16 = 4 * wg + k4;
       float gq[16], gk[16];
-      tmem_ld16(tl + C_GQ + c16 * 16, gq);
-      tmem_ld16(tl + C_GK + c16 * 16, gk);
+      tmem_ld16x2(tl + C_GQ + c16 * 16, tl + C_GK + c16 * 16, gq, gk);
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
         gq[u] += cq;
@@ -638,9 +645,12 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
     }
     __syncthreads();
     const float *md = s_row0 + D;
-    for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
-      float dv[32];
-      tmem_ld32(tl + C_DV + ch * 32, dv);
+    float dvv[2][32];
+    tmem_ld32x2(tl + C_DV + 64 * wg, tl + C_DV + 64 * wg + 32, dvv[0], dvv[1]);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int ch = 2 * wg + h;
+      const float *dv = dvv[h];
 #pragma unroll
       for (int u = 0; u < 32; u += 4) {   // + (sum_i Kt[i]) dS[0]
         const float4 m4 = *reinterpret_cast<const float4 *>(md + ch * 32 + u);
