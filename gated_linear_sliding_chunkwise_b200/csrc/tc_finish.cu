@@ -104,31 +104,32 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
   const uint32_t id_dw = idesc_bf16(128, 64, 1, 1);    // X^T (MN-major) x dZ (MN-major, N = 64)
   bool fail = false;
   // this row's dphi values (its group's half) of one map, loaded ahead: map 0
-  // of the next tile while this tile finishes, map 1 while map 0 is used
-  float4 dpre[16];
+  // of the next tile while this tile finishes, map 1 while map 0 is used.
+  // They stay packed (bf16) until used, so that the loads are still in flight
+  // when the call returns.
+  uint4 dpre[8];
   const int fb_slot = (gla && p.slot_of) ? p.slot_of[bh] : -1;
   auto dphi_load = [&](int m, int c) {
     const int t = c * T + row;
-    if (fb_slot >= 0) {   // the exact fallback's fp32 dphi
+    if (fb_slot >= 0) {
+      // the exact fallback's fp32 dphi, centred on the half row's first value
+      // like the tensor-core kernel's (the softmax backward does not see a
+      // constant added to one half)
       const float *src = (m == 0 ? p.fb_dphq : p.fb_dphk) + ((size_t)fb_slot * p.L + (t < p.L ? t : 0)) * D + wg * F;
+      const float c0 = t < p.L ? src[0] : 0.f;
 #pragma unroll
-      for (int u = 0; u < 16; ++u)
-        dpre[u] = t < p.L ? *reinterpret_cast<const float4 *>(src + 4 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int u = 0; u < 8; ++u) {
+        float f[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) f[i] = t < p.L ? src[8 * u + i] - c0 : 0.f;
+        dpre[u] = pack8(f);
+      }
       return;
     }
     const __nv_bfloat16 *src = (m == 0 ? p.dphq : p.dphk) + ((size_t)bh * p.L + (t < p.L ? t : 0)) * D + wg * F;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      float f[8];
-      if (t < p.L) {
-        unpack8(*reinterpret_cast<const uint4 *>(src + 8 * u), f);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) f[i] = 0.f;
-      }
-      dpre[2 * u] = make_float4(f[0], f[1], f[2], f[3]);
-      dpre[2 * u + 1] = make_float4(f[4], f[5], f[6], f[7]);
-    }
+    for (int u = 0; u < 8; ++u)
+      dpre[u] = t < p.L ? *reinterpret_cast<const uint4 *>(src + 8 * u) : make_uint4(0u, 0u, 0u, 0u);
   };
   if (gla && ntiles > 0) dphi_load(0, 0);
   for (int c = 0; c < ntiles; ++c) {
@@ -159,23 +160,24 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
       for (int m = 0; m < 2; ++m) {
         float ph[F];
         const float sc = feature_half(tl + (m == 0 ? C_ZQ : C_ZK), wg, ph);
-        const float4 *d = dpre;
         float dot4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          ph[4 * u] *= sc;
-          ph[4 * u + 1] *= sc;
-          ph[4 * u + 2] *= sc;
-          ph[4 * u + 3] *= sc;
-          dot4[u & 3] += d[u].x * ph[4 * u] + d[u].y * ph[4 * u + 1] + d[u].z * ph[4 * u + 2] + d[u].w * ph[4 * u + 3];
+        for (int u = 0; u < 8; ++u) {
+          float d[8];
+          unpack8(dpre[u], d);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            ph[8 * u + i] *= sc;
+            dot4[i & 3] += d[i] * ph[8 * u + i];
+          }
         }
         const float dot = (dot4[0] + dot4[1]) + (dot4[2] + dot4[3]);
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {   // ph <- this group's half-term
-          ph[4 * u] *= d[u].x - dot;
-          ph[4 * u + 1] *= d[u].y - dot;
-          ph[4 * u + 2] *= d[u].z - dot;
-          ph[4 * u + 3] *= d[u].w - dot;
+        for (int u = 0; u < 8; ++u) {   // ph <- this group's half-term
+          float d[8];
+          unpack8(dpre[u], d);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) ph[8 * u + i] *= d[i] - dot;
         }
         if (m == 0) dphi_load(1, c);   // the k map's values, in flight while this map finishes
         else if (c + 1 < ntiles) dphi_load(0, c + 1);

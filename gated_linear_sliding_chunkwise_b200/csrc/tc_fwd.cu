@@ -448,28 +448,27 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       //      The meta logits (CUDA cores, from X_q in shared memory) and the
       //      tile's decay exp(r) are formed while MMA 1 runs.
       float pmeta = kNegBig;
-      if (swa) {
-        // meta logits q . mk_m (scaled) into s_ml: group wg takes the meta
-        // tokens wg, wg + 2, ..., two per pass
-        for (int m0 = wg; m0 < p.M; m0 += 4) {
-          float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      if (swa && wg == 0) {
+        // meta logits q . mk_m (scaled) into s_ml, four meta tokens per pass
+        for (int m0 = 0; m0 < p.M; m0 += 4) {
+          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll 4
           for (int ch = 0; ch < 16; ++ch) {
             float q8[8];
             unpack8(*chunk_ptr(sm, R_XQ, row, ch), q8);
 #pragma unroll
-            for (int k = 0; k < 2; ++k) {
-              const float4 a = *reinterpret_cast<const float4 *>(&s_mk[m0 + 2 * k][ch * 8]);
-              const float4 b = *reinterpret_cast<const float4 *>(&s_mk[m0 + 2 * k][ch * 8 + 4]);
+            for (int k = 0; k < 4; ++k) {
+              const float4 a = *reinterpret_cast<const float4 *>(&s_mk[m0 + k][ch * 8]);
+              const float4 b = *reinterpret_cast<const float4 *>(&s_mk[m0 + k][ch * 8 + 4]);
               acc[2 * k] = fmaf(q8[0], a.x, fmaf(q8[1], a.y, fmaf(q8[2], a.z, fmaf(q8[3], a.w, acc[2 * k]))));
               acc[2 * k + 1] = fmaf(q8[4], b.x, fmaf(q8[5], b.y, fmaf(q8[6], b.z, fmaf(q8[7], b.w, acc[2 * k + 1]))));
             }
           }
 #pragma unroll
-          for (int k = 0; k < 2; ++k)
-            if (m0 + 2 * k < p.M) {
+          for (int k = 0; k < 4; ++k)
+            if (m0 + k < p.M) {
               const float l = (acc[2 * k] + acc[2 * k + 1]) * p.scale;
-              s_ml[m0 + 2 * k][row] = l;
+              s_ml[m0 + k][row] = l;
               pmeta = fmaxf(pmeta, l);
             }
         }
@@ -480,42 +479,42 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       float lsum = 1.f, mx = 0.f;                 // row normaliser and max (scaled logits)
       // Logit column cl holds key t0 - T + cl.  Row r sees columns
       // [r + T + 1 - window, r + T] (and keys >= -P, P the prefix length),
-      // so warp w4 only visits the 16-column half-chunks from
-      // (32 w4 + T + 1 - window) / 16 to 2 w4 + 9 (ten at window 128, five
-      // per group: group wg the ones hc_lo + wg, hc_lo + wg + 2, ...), and
-      // only those at the band's edges need the mask.
+      // so warp w4 only visits 32-column chunks w4 + (T + 1 - window) / 32
+      // .. w4 + 4, and only the first and last of those need the band mask.
       const int w4 = warp & 3;
       const int cbase = t0 - T;
       const int lo_c = max(tq - p.window + 1, -p.P) - cbase, hi_c = tq - cbase;
-      int hc_lo = (32 * w4 + T + 1 - p.window) >> 4;
-      if (cbase < 0) hc_lo = max(hc_lo, (T - p.P) >> 4);
-      const int hc_hi = 2 * w4 + 9;
-      const int in_lo = 32 * w4 + 31 + T + 1 - p.window;   // interior half-chunk: 16 hc >= in_lo
-      const int hc_first = hc_lo + wg;                     // this group's first half-chunk
-      constexpr int NH = 5;                                // half-chunks per group, at most
-      uint32_t pk[NH][8];
-      // this group's logit half-chunks, all five loads in flight together
-      // (a half-chunk past the band reloads the last one and is skipped)
-      uint32_t la[NH];
-#pragma unroll
-      for (int k = 0; k < NH; ++k) la[k] = tl + C_L + 16 * min(hc_first + 2 * k, hc_hi);
-      float lv[NH][16];
+      int ch_lo = (32 * w4 + T + 1 - p.window) >> 5;
+      if (cbase < 0) ch_lo = max(ch_lo, (T - p.P) >> 5);
+      const int ch_hi = w4 + 4;
+      const int in_lo = 32 * w4 + 31 + T + 1 - p.window;   // interior chunk: 32 ch >= in_lo
+      const int ch_first = ch_lo + 1 - wg;                 // this group's first chunk
+      uint32_t pk[3][16];
+      // this group's logit chunks, read from TMEM once (the stage-1 instance,
+      // short of registers, reads them again for the exponentials)
+      constexpr int KEPT = LOSS ? 1 : 3;
+      float lv[KEPT][32];
       if (swa) {
         float pmax = pmeta;
-        tmem_ld16x5(la, lv);
+        if constexpr (!LOSS) {   // the three chunks' loads in flight together (one past the band reloads the last)
+          const uint32_t la[3] = {tl + C_L + 32 * min(ch_first, ch_hi), tl + C_L + 32 * min(ch_first + 2, ch_hi),
+                                  tl + C_L + 32 * min(ch_first + 4, ch_hi)};
+          tmem_ld32x3(la, lv);
+        }
 #pragma unroll
-        for (int k = 0; k < NH; ++k) {
-          const int hc = hc_first + 2 * k;
-          if (hc > hc_hi) continue;
-          float *v = lv[k];
+        for (int k = 0; k < 3; ++k) {
+          const int ch = ch_first + 2 * k;
+          if (ch > ch_hi) continue;
+          float *v = lv[LOSS ? 0 : k];
+          if (LOSS) tmem_ld32(tl + C_L + ch * 32, v);
           float m4[4] = {kNegBig, kNegBig, kNegBig, kNegBig};
-          if (16 * hc >= in_lo && 16 * hc + 15 <= 32 * w4 + T && 16 * hc + cbase >= -p.P) {
+          if (32 * ch >= in_lo && 32 * ch + 31 <= 32 * w4 + T && 32 * ch + cbase >= -p.P) {
 #pragma unroll
-            for (int u = 0; u < 16; ++u) m4[u & 3] = fmaxf(m4[u & 3], v[u]);
+            for (int u = 0; u < 32; ++u) m4[u & 3] = fmaxf(m4[u & 3], v[u]);
           } else {
 #pragma unroll
-            for (int u = 0; u < 16; ++u) {
-              const int cl = 16 * hc + u;
+            for (int u = 0; u < 32; ++u) {
+              const int cl = 32 * ch + u;
               if (cl >= lo_c && cl <= hi_c) m4[u & 3] = fmaxf(m4[u & 3], v[u]);
             }
           }
@@ -528,21 +527,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       if (swa) {
         mx = fmaxf(s_pmax[0][row], s_pmax[1][row]);
         // P^ = exp(l - max), packed and held until both groups have read
-        // their logits (P^ column 8 hc overlays logit half-chunk hc / 2)
+        // their logits (P^ column 16 ch overlays logit chunk ch / 2)
         float s4[4] = {0.f, 0.f, 0.f, 0.f};
-        tmem_ld16x5(la, lv);   // again: the registers are needed in between
 #pragma unroll
-        for (int k = 0; k < NH; ++k) {
-          const int hc = hc_first + 2 * k;
-          if (hc > hc_hi) continue;
-          const float *v = lv[k];
-          const bool inner = 16 * hc >= in_lo && 16 * hc + 15 <= 32 * w4 + T && 16 * hc + cbase >= -p.P;
+        for (int k = 0; k < 3; ++k) {
+          const int ch = ch_first + 2 * k;
+          if (ch > ch_hi) continue;
+          const float *v = lv[LOSS ? 0 : k];
+          if (LOSS) tmem_ld32(tl + C_L + ch * 32, lv[0]);
+          const bool inner = 32 * ch >= in_lo && 32 * ch + 31 <= 32 * w4 + T && 32 * ch + cbase >= -p.P;
 #pragma unroll
-          for (int u = 0; u < 16; u += 2) {
+          for (int u = 0; u < 32; u += 2) {
             float e0 = __expf(fmaf(v[u], p.scale, -mx));
             float e1 = __expf(fmaf(v[u + 1], p.scale, -mx));
             if (!inner) {
-              const int cl = 16 * hc + u;
+              const int cl = 32 * ch + u;
               e0 = (cl >= lo_c && cl <= hi_c) ? e0 : 0.f;
               e1 = (cl + 1 >= lo_c && cl + 1 <= hi_c) ? e1 : 0.f;
             }
@@ -551,11 +550,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
           }
         }
         float psum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-        for (int m = wg; m < p.M; m += 2) {   // this group's meta tokens
-          const float e = __expf(s_ml[m][row] - mx);
-          psum += e;
-          s_ml[m][row] = e;
-        }
+        if (wg == 0)
+          for (int m = 0; m < p.M; ++m) {
+            const float e = __expf(s_ml[m][row] - mx);
+            psum += e;
+            s_ml[m][row] = e;
+          }
         s_psum[wg][row] = psum;
       }
       bar_sync(BAR_B, NTHREADS);
@@ -563,15 +563,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         lsum = s_psum[0][row] + s_psum[1][row];
         if (!qvalid) lsum = 1.f;
 #pragma unroll
-        for (int k = 0; k < NH; ++k) {
-          const int hc = hc_first + 2 * k;
-          if (hc > hc_hi) continue;
-          tmem_st8(tl + C_P + hc * 8, pk[k]);
+        for (int k = 0; k < 3; ++k) {
+          const int ch = ch_first + 2 * k;
+          if (ch > ch_hi) continue;
+          tmem_st8(tl + C_P + ch * 16, pk[k]);
+          tmem_st8(tl + C_P + ch * 16 + 8, pk[k] + 8);
         }
         uint32_t zero[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-        for (int hc = wg; hc < 16; hc += 2) {   // half-chunks outside the band: P = 0
-          if (hc >= hc_lo && hc <= hc_hi) continue;
-          tmem_st8(tl + C_P + hc * 8, zero);
+        for (int ch = wg; ch < 8; ch += 2) {   // chunks outside the band: P = 0
+          if (ch >= ch_lo && ch <= ch_hi) continue;
+          tmem_st8(tl + C_P + ch * 16, zero);
+          tmem_st8(tl + C_P + ch * 16 + 8, zero);
         }
         if (wg == 0 && qvalid && p.lse) p.lse[(size_t)bh * p.L + tq] = mx + logf(lsum);
       }
