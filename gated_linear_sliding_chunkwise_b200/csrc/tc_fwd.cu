@@ -444,38 +444,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
     if (full) {
       // ---- full pass: the anchor softmax split between the groups (group 1
       //      the band chunks ch_lo, ch_lo + 2, ..., group 0 the others and
-      //      the meta logits), then one half of phi_q, phi_k per group.
-      //      The meta logits (CUDA cores, from X_q in shared memory) and the
-      //      tile's decay exp(r) are formed while MMA 1 runs.
-      float pmeta = kNegBig;
-      if (swa && wg == 0) {
-        // meta logits q . mk_m (scaled) into s_ml, four meta tokens per pass
-        for (int m0 = 0; m0 < p.M; m0 += 4) {
-          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-          for (int ch = 0; ch < 16; ++ch) {
-            float q8[8];
-            unpack8(*chunk_ptr(sm, R_XQ, row, ch), q8);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const float4 a = *reinterpret_cast<const float4 *>(&s_mk[m0 + k][ch * 8]);
-              const float4 b = *reinterpret_cast<const float4 *>(&s_mk[m0 + k][ch * 8 + 4]);
-              acc[2 * k] = fmaf(q8[0], a.x, fmaf(q8[1], a.y, fmaf(q8[2], a.z, fmaf(q8[3], a.w, acc[2 * k]))));
-              acc[2 * k + 1] = fmaf(q8[4], b.x, fmaf(q8[5], b.y, fmaf(q8[6], b.z, fmaf(q8[7], b.w, acc[2 * k + 1]))));
-            }
-          }
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            if (m0 + k < p.M) {
-              const float l = (acc[2 * k] + acc[2 * k + 1]) * p.scale;
-              s_ml[m0 + k][row] = l;
-              pmeta = fmaxf(pmeta, l);
-            }
-        }
-      }
-      if (wg == 1 && gla) s_dec[row] = __expf(p.gate_r[((size_t)bh * ntiles_all + c) * D + row]);   // exp(r)
+      //      the meta logits), then one half of phi_q, phi_k per group
       ok &= mbar_wait(&bar_m1, par, err, ST_TIMEOUT);
       tc_fence_after();
+      if (wg == 1 && gla) s_dec[row] = __expf(p.gate_r[((size_t)bh * ntiles_all + c) * D + row]);   // exp(r)
       float lsum = 1.f, mx = 0.f;                 // row normaliser and max (scaled logits)
       // Logit column cl holds key t0 - T + cl.  Row r sees columns
       // [r + T + 1 - window, r + T] (and keys >= -P, P the prefix length),
@@ -490,23 +462,36 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       const int in_lo = 32 * w4 + 31 + T + 1 - p.window;   // interior chunk: 32 ch >= in_lo
       const int ch_first = ch_lo + 1 - wg;                 // this group's first chunk
       uint32_t pk[3][16];
-      // this group's logit chunks, read from TMEM once (the stage-1 instance,
-      // short of registers, reads them again for the exponentials)
-      constexpr int KEPT = LOSS ? 1 : 3;
-      float lv[KEPT][32];
       if (swa) {
-        float pmax = pmeta;
-        if constexpr (!LOSS) {   // the three chunks' loads in flight together (one past the band reloads the last)
-          const uint32_t la[3] = {tl + C_L + 32 * min(ch_first, ch_hi), tl + C_L + 32 * min(ch_first + 2, ch_hi),
-                                  tl + C_L + 32 * min(ch_first + 4, ch_hi)};
-          tmem_ld32x3(la, lv);
-        }
+        float pmax = kNegBig;
+        if (wg == 0) {
+          // meta logits q . mk_m (scaled) into s_ml, four meta tokens per pass
+          for (int m0 = 0; m0 < p.M; m0 += 4) {
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+            for (int ch = 0; ch < 16; ++ch) {
+              float q8[8];
+              unpack8(*chunk_ptr(sm, R_XQ, row, ch), q8);
 #pragma unroll
-        for (int k = 0; k < 3; ++k) {
-          const int ch = ch_first + 2 * k;
-          if (ch > ch_hi) continue;
-          float *v = lv[LOSS ? 0 : k];
-          if (LOSS) tmem_ld32(tl + C_L + ch * 32, v);
+              for (int k = 0; k < 4; ++k) {
+                const float4 a = *reinterpret_cast<const float4 *>(&s_mk[m0 + k][ch * 8]);
+                const float4 b = *reinterpret_cast<const float4 *>(&s_mk[m0 + k][ch * 8 + 4]);
+                acc[2 * k] = fmaf(q8[0], a.x, fmaf(q8[1], a.y, fmaf(q8[2], a.z, fmaf(q8[3], a.w, acc[2 * k]))));
+                acc[2 * k + 1] = fmaf(q8[4], b.x, fmaf(q8[5], b.y, fmaf(q8[6], b.z, fmaf(q8[7], b.w, acc[2 * k + 1]))));
+              }
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              if (m0 + k < p.M) {
+                const float l = (acc[2 * k] + acc[2 * k + 1]) * p.scale;
+                s_ml[m0 + k][row] = l;
+                pmax = fmaxf(pmax, l);
+              }
+          }
+        }
+        for (int ch = ch_first; ch <= ch_hi; ch += 2) {
+          float v[32];
+          tmem_ld32(tl + C_L + ch * 32, v);
           float m4[4] = {kNegBig, kNegBig, kNegBig, kNegBig};
           if (32 * ch >= in_lo && 32 * ch + 31 <= 32 * w4 + T && 32 * ch + cbase >= -p.P) {
 #pragma unroll
@@ -533,8 +518,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         for (int k = 0; k < 3; ++k) {
           const int ch = ch_first + 2 * k;
           if (ch > ch_hi) continue;
-          const float *v = lv[LOSS ? 0 : k];
-          if (LOSS) tmem_ld32(tl + C_L + ch * 32, lv[0]);
+          float v[32];
+          tmem_ld32(tl + C_L + ch * 32, v);
           const bool inner = 32 * ch >= in_lo && 32 * ch + 31 <= 32 * w4 + T && 32 * ch + cbase >= -p.P;
 #pragma unroll
           for (int u = 0; u < 32; u += 2) {
@@ -640,14 +625,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       tc_fence_after();
       const int i = row;
       const float dec = s_dec[i];
-#pragma unroll 1
-      for (int c32 = 2 * wg; c32 < 2 * wg + 2; ++c32) {   // two 16-column loads in flight together
-        float vv[2][16];
-        tmem_ld16x2(tl + C_S + c32 * 32, tl + C_S + c32 * 32 + 16, vv[0], vv[1]);
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-        const int c16 = 2 * c32 + hh;
-        float *v = vv[hh];
+      for (int c16 = 4 * wg; c16 < 4 * wg + 4; ++c16) {
+        float v[16];
+        tmem_ld16(tl + C_S + c16 * 16, v);
         uint32_t r[8];
 #pragma unroll
         for (int u = 0; u < 16; ++u) v[u] *= dec;
@@ -663,7 +643,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         } else if (p.snap && i == 0) {
 #pragma unroll
           for (int u = 0; u < 16; ++u) s_row0[c16 * 16 + u] = v[u];
-        }
         }
       }
       if (!full && p.snap) {
@@ -691,14 +670,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
 
     // ---------------------- masked intra A (column half per group) ---
     if (gla && full) {
-#pragma unroll 1
-      for (int c32 = 2 * wg; c32 < 2 * wg + 2; ++c32) {
-        float vv[2][16];
-        tmem_ld16x2(tl + C_A + c32 * 32, tl + C_A + c32 * 32 + 16, vv[0], vv[1]);
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-        const int c16 = 2 * c32 + hh;
-        const float *v = vv[hh];
+      for (int c16 = 4 * wg; c16 < 4 * wg + 4; ++c16) {
+        float v[16];
+        tmem_ld16(tl + C_A + c16 * 16, v);
         uint32_t r[8];
 #pragma unroll
         for (int u = 0; u < 16; u += 2) {
@@ -709,7 +683,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
           r[u / 2] = pack_bf16(a0, a1);
         }
         tmem_st8(tl + C_AH + c16 * 8, r);
-        }
       }
     }
     tmem_st_wait();
@@ -754,12 +727,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       // tcgen05.ld is warp-collective: every lane loads, valid rows store
       const size_t roff = ((size_t)bh * p.L + (qvalid ? tq : 0)) * D;
       const float oscale = s_oscale[row];
-      float vall[64];   // this group's 64 columns of O, all four loads in flight together
-      tmem_ld32x2(tl + C_O + 64 * wg, tl + C_O + 64 * wg + 32, vall, vall + 32);
-#pragma unroll
+#pragma unroll(LOSS ? 4 : 1)
       for (int k4 = 0; k4 < 4; ++k4) {
         const int c16 = 4 * wg + k4;
-        float *v = vall + 16 * k4;
+        float v[16];
+        tmem_ld16(tl + C_O + c16 * 16, v);
 #pragma unroll
         for (int u = 0; u < 16; ++u) v[u] *= oscale;
         if (swa && p.meta_v) {

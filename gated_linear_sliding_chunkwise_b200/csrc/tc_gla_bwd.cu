@@ -298,30 +298,31 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
                      R_KL = 6 * TILE;
   // TMEM, in order of use:
   //   dA [128,256) dA^T [256,384) Zq [384,448) Zk [448,512)
-  //   dA^ [0,64) dA^T^ [64,128) ; E (fp32, while Qt and Kt are formed) [128,256)
-  //   A^T [256,384) ; A^T^ (bf16) [128,192) ; GQ [256,384) GK [384,512) ; DV [0,128)
+  //   dA^ [0,64) dA^T^ [64,128) ; GQ [256,384) (its dO S'^T part while the
+  //   rows form Qt and Kt) ; E (fp32, while Qt and Kt are formed) [128,256)
+  //   A^T [384,512) ; A^T^ (bf16) [128,192) ; GK [384,512) ; DV [0,128)
   constexpr uint32_t C_DAH = 0, C_DATH = 64, C_DV = 0, C_DA = 128, C_E = 128, C_ATH = 128, C_DAT = 256,
-                     C_AT = 256, C_GQ = 256, C_ZQ = 384, C_ZK = 448, C_GK = 384;
+                     C_AT = 384, C_GQ = 256, C_ZQ = 384, C_ZK = 448, C_GK = 384;
   const int tid = threadIdx.x, warp = tid >> 5, wg = tid >> 7, row = tid & 127;
   const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
   const uint32_t sbase = smem_u32(sm);
   // Persistent: CTA b walks the contiguous run [w0, w1) of (sequence, tile)
   // items, item w = tile w % ntiles of sequence w / ntiles.  The next item's
   // inputs go out as this item frees their places: the weights once the last
-  // products are done, the decay factors during the dv pass, X_q and X_k once
-  // the dphi stores have read their staging, V and dO after the dv store.
+  // products are done, the decay factors during the dphi pass, V and dO once
+  // the dB store has read its staging, X_q after the dphi stores, X_k after
+  // the dv store.
   const int nwork = p.ntiles * p.BH;
   const int w0 = (int)((long long)blockIdx.x * nwork / gridDim.x);
   const int w1 = (int)((long long)(blockIdx.x + 1) * nwork / gridDim.x);
-  auto item_loads = [&](int w, int part) {   // part 0: weights (arms the barrier), 1: X_q, X_k, 2: V, dO
+  // part 0: weights (arms the barrier), 1: X_q, 2: V, dO, 3: X_k
+  auto item_loads = [&](int w, int part) {
     const int lbh = w / p.ntiles, lt0 = (w % p.ntiles) * T;
     if (part == 0) mbar_expect_tx(&bars[0], 5 * TILE);
     for (int r = 0; r < 2; ++r) {
       if (part == 0) tma_load_3d(sm + R_W + r * REG, &p.mw, &bars[0], 0, 0, 2 * (lbh % p.H) + r);
-      if (part == 1) {
-        tma_load_3d(sm + R_XQ + r * REG, &p.mq, &bars[0], 64 * r, lt0, lbh);
-        tma_load_3d(sm + R_XK + r * REG, &p.mk, &bars[0], 64 * r, lt0, lbh);
-      }
+      if (part == 1) tma_load_3d(sm + R_XQ + r * REG, &p.mq, &bars[0], 64 * r, lt0, lbh);
+      if (part == 3) tma_load_3d(sm + R_XK + r * REG, &p.mk, &bars[0], 64 * r, lt0, lbh);
       if (part == 2) {
         tma_load_3d(sm + R_V + r * REG, &p.mv, &bars[0], 64 * r, lt0, lbh);
         tma_load_3d(sm + R_O + r * REG, &p.mo, &bars[0], 64 * r, lt0, lbh);
@@ -340,6 +341,7 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
       item_loads(w0, 0);
       item_loads(w0, 1);
       item_loads(w0, 2);
+      item_loads(w0, 3);
     }
   }
   tc_fence_before();
@@ -417,6 +419,18 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
   tc_fence_before();
   __syncthreads();   // dA read out before E overwrites its columns
   tc_fence_after();
+  // 3a. GQ = dO S'^T (the columns of dA^T are spent): it runs while the rows
+  //     form Qt and Kt, and once it is done the dS copy can take S's place
+  bool t0ok = true;   // tid 0: its own waits below succeeded
+  if (tid == 0) {
+    t0ok = mbar_wait(&bars[2], par, p.status, ST_TIMEOUT);
+    if (t0ok) {
+      pend_sp = false;
+      tc_fence_after();
+      for (int s = 0; s < 8; ++s) mma_ss(tb + C_GQ, desc_k(sbase + R_O, s), desc_k(sbase + R_W, s), id_kk, s > 0);
+      mma_commit(&bars[4]);
+    }
+  }
   //    E in fp32 (dimensions 64 wg ..) into TMEM, then Qt = phi_q E and
   //    Kt = phi_k / E for the same dimensions (rows past L: Kt = 0), each as
   //    a bf16 pair hi + lo
@@ -466,18 +480,26 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
   }
   fence_proxy_async();
   tc_fence_before();
-  __syncthreads();   // every row is done with the row-0 vectors: s_r1 takes the sums
+  // every row is done with the row-0 vectors (s_r1 takes the sums) and with Zq, Zk
+  if (__syncthreads_or(!t0ok)) { ok = false; goto done; }
   if (wg == 1)
 #pragma unroll
     for (int k = 0; k < 3; ++k) s_r1[k][row] = r1[k];
-  // 3. A^T = Kt Qt^T (rows = keys)
+  // 3b. A^T = Kt Qt^T (rows = keys) over Zq, Zk; the dS copy replaces S'
   if (tid == 0) {
     tc_fence_after();
     for (int s = 0; s < 8; ++s) mma_ss(tb + C_AT, desc_k(sbase + R_XK, s), desc_k(sbase + R_XQ, s), id_kk, s > 0);
     mma_commit(&bars[3]);
+    t0ok = mbar_wait(&bars[4], par, p.status, ST_TIMEOUT);
+    if (t0ok) {
+      pend_ds = true;
+      mbar_expect_tx(&bars[6], TILE);
+      tma_load_3d(sm + R_W, &p.mds, &bars[6], 0, 0, snap_idx);
+      tma_load_3d(sm + R_W + REG, &p.mds, &bars[6], 64, 0, snap_idx);
+    }
   }
   ok = mbar_wait(&bars[3], par, p.status, ST_TIMEOUT);
-  if (__syncthreads_or(!ok)) { ok = false; goto done; }
+  if (__syncthreads_or(!ok || !t0ok)) { ok = false; goto done; }
   if (wg == 0)   // the two halves' sums meet; read after the next barrier
 #pragma unroll
     for (int k = 0; k < 3; ++k) s_r1[k][row] += r1[k];
@@ -501,26 +523,15 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
   }
   tmem_st_wait();
   tc_fence_before();
-  ok = mbar_wait(&bars[2], par, p.status, ST_TIMEOUT);
-  if (__syncthreads_or(!ok)) { ok = false; goto done; }
-  pend_sp = false;
-  // 4a. GQ = dO S'^T + dA^ (Kt hi + lo) ;  GK = dA^T^ (Qt hi + lo) ; dS
-  //     replaces S' once its product is done
+  __syncthreads();   // A^T read out before GK overwrites its columns
+  // 4a. GQ += dA^ (Kt hi + lo) ;  GK = dA^T^ (Qt hi + lo)
   if (tid == 0) {
     tc_fence_after();
-    for (int s = 0; s < 8; ++s) mma_ss(tb + C_GQ, desc_k(sbase + R_O, s), desc_k(sbase + R_W, s), id_kk, s > 0);
-    mma_commit(&bars[4]);
     for (int s = 0; s < 8; ++s) mma_ts(tb + C_GQ, tb + C_DAH + s * 8, desc_mn(sbase + R_XK, s), id_mn, 1);
     for (int s = 0; s < 8; ++s) mma_ts(tb + C_GQ, tb + C_DAH + s * 8, desc_mn(sbase + R_KL, s), id_mn, 1);
     for (int s = 0; s < 8; ++s) mma_ts(tb + C_GK, tb + C_DATH + s * 8, desc_mn(sbase + R_XQ, s), id_mn, s > 0);
     for (int s = 0; s < 8; ++s) mma_ts(tb + C_GK, tb + C_DATH + s * 8, desc_mn(sbase + R_QL, s), id_mn, 1);
     mma_commit(&bars[5]);
-    if (mbar_wait(&bars[4], par, p.status, ST_TIMEOUT)) {
-      pend_ds = true;
-      mbar_expect_tx(&bars[6], TILE);
-      tma_load_3d(sm + R_W, &p.mds, &bars[6], 0, 0, snap_idx);
-      tma_load_3d(sm + R_W + REG, &p.mds, &bars[6], 64, 0, snap_idx);
-    }
   }
   ok = mbar_wait(&bars[5], par, p.status, ST_TIMEOUT);
   ok &= mbar_wait(&bars[6], par, p.status, ST_TIMEOUT);
@@ -538,10 +549,10 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
     // 5. rows, dimension half per group, staged as fp32 tiles in the spent
     //    regions and written with TMA stores (rows past L are clipped by the
     //    maps): dB = Qt GQ - Kt GK (Qt, Kt as hi + lo, so that dB matches the
-    //    products) over V | dO; then dphi_q = E GQ over Qt lo | Kt lo and
-    //    dphi_k = GK / E over Qt hi | Kt hi; then dv over V | dO again.  E
-    //    (fp32) is read again from global memory, its loads in flight while
-    //    the last products run.
+    //    products) over V | dO; then dphi_q = E GQ (bf16) over Qt lo and
+    //    dphi_k = GK / E over Qt hi; then dv over Kt hi | Kt lo.  E (fp32) is
+    //    read again from global memory, its loads in flight while the last
+    //    products run.
     float4 e4[16];
     const float *er = p.e32 + ((size_t)bh * p.L + (valid ? tq : 0)) * D + 64 * wg;
 #pragma unroll
@@ -641,10 +652,11 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
         tma_store_3d(&p.mdk, sm + R_XQ + r * REG, 64 * r, t0, bh);
       }
       bulk_commit();
-      bulk_wait_read_but_last();   // the dB tile has been read out of V | dO
     }
-    __syncthreads();
+    // dv, staged in the spent Kt hi | Kt lo regions (group wg's two 32-column
+    // boxes in one of them), so that it need not wait for the dB store
     const float *md = s_row0 + D;
+    unsigned char *st_dv = sm + (wg == 0 ? R_XK : R_KL);
     float dvv[2][32];
     tmem_ld32x2(tl + C_DV + 64 * wg, tl + C_DV + 64 * wg + 32, dvv[0], dvv[1]);
 #pragma unroll
@@ -654,20 +666,23 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
 #pragma unroll
       for (int u = 0; u < 32; u += 4) {   // + (sum_i Kt[i]) dS[0]
         const float4 m4 = *reinterpret_cast<const float4 *>(md + ch * 32 + u);
-        *f32_stage_ptr(st0, row, ch * 32 + u) = make_float4(fmaf(kap, m4.x, dv[u]), fmaf(kap, m4.y, dv[u + 1]),
-                                                            fmaf(kap, m4.z, dv[u + 2]), fmaf(kap, m4.w, dv[u + 3]));
+        *f32_stage_ptr(st_dv, row, h * 32 + u) = make_float4(fmaf(kap, m4.x, dv[u]), fmaf(kap, m4.y, dv[u + 1]),
+                                                             fmaf(kap, m4.z, dv[u + 2]), fmaf(kap, m4.w, dv[u + 3]));
       }
     }
     fence_proxy_async();
     __syncthreads();
     if (tid == 0) {
-      for (int bx = 0; bx < 4; ++bx) tma_store_3d(&p.mdv, st0 + bx * 16384, 32 * bx, t0, bh);
+      for (int bx = 0; bx < 4; ++bx)
+        tma_store_3d(&p.mdv, sm + (bx < 2 ? R_XK : R_KL) + (bx & 1) * 16384, 32 * bx, t0, bh);
       bulk_commit();
-      if (more) {
-        bulk_wait_read_but_last();   // the dphi tiles have been read out of Qt | Kt
-        item_loads(w + 1, 1);
-        bulk_wait_read();            // and the dv tile out of V | dO
+      if (more) {   // the next item's tiles, each as soon as its place has been read out
+        bulk_wait_read_n<2>();   // dB out of V | dO
         item_loads(w + 1, 2);
+        bulk_wait_read_n<1>();   // dphi out of Qt lo | Qt hi
+        item_loads(w + 1, 1);
+        bulk_wait_read();        // dv out of Kt hi | Kt lo
+        item_loads(w + 1, 3);
       }
     }
   }

@@ -235,18 +235,9 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
     if (cbase < 0) ch_lo = max(ch_lo, (T - p.P) >> 5);
     const int ch_hi = w4 + 4;
     const int in_lo = 32 * w4 + 31 + T + 1 - p.window;
-    // this group's (up to) three band chunks, loaded together (a chunk past
-    // the band reloads the last one and is skipped)
-    uint32_t la[3];
-#pragma unroll
-    for (int k = 0; k < 3; ++k) la[k] = tl + C_L + 32 * min(ch_lo + wg + 2 * k, ch_hi);
-    float lv[3][32];
-    tmem_ld32x3(la, lv);
-#pragma unroll
-    for (int k = 0; k < 3; ++k) {
-      const int ch = ch_lo + wg + 2 * k;
-      if (ch > ch_hi) continue;
-      const float *v = lv[k];
+    for (int ch = ch_lo + wg; ch <= ch_hi; ch += 2) {
+      float v[32];
+      tmem_ld32(tl + C_L + ch * 32, v);
       float m4[4] = {kNegBig, kNegBig, kNegBig, kNegBig};
       if (32 * ch >= in_lo && 32 * ch + 31 <= 32 * w4 + T && 32 * ch + cbase >= -p.P) {
 #pragma unroll
@@ -272,7 +263,8 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
     for (int k = 0; k < 3; ++k) {
       const int ch = ch_lo + wg + 2 * k;
       if (ch > ch_hi) continue;
-      const float *v = lv[k];
+      float v[32];
+      tmem_ld32(tl + C_L + ch * 32, v);
       const bool inner = 32 * ch >= in_lo && 32 * ch + 31 <= 32 * w4 + T && 32 * ch + cbase >= -p.P;
 #pragma unroll
       for (int u = 0; u < 32; u += 2) {
@@ -328,11 +320,9 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
     if (__syncthreads_or(!ok)) goto done;
     tc_fence_after();
     float dpart = 0.f;                    // dout . o_swa for this row, column half per group
-    float ov[2][32];
-    tmem_ld32x2(tl + C_O + 64 * wg, tl + C_O + 64 * wg + 32, ov[0], ov[1]);
-#pragma unroll
     for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
-      const float *v = ov[ch - 2 * wg];
+      float v[32];
+      tmem_ld32(tl + C_O + ch * 32, v);
 #pragma unroll
       for (int c8 = 0; c8 < 4; ++c8) {
         float o8[8];
@@ -383,7 +373,8 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
       uint32_t ds[16];
       if (ch >= ch_lo && ch <= ch_hi) {
         float dp[32], pp[32], pk16[16];
-        tmem_ld32_16(tl + C_DP + ch * 32, tl + C_P + ch * 16, dp, pk16);
+        tmem_ld32(tl + C_DP + ch * 32, dp);
+        tmem_ld16(tl + C_P + ch * 16, pk16);
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
           const uint32_t w = __float_as_uint(pk16[u]);
@@ -436,11 +427,9 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
       // part in the V region and stored with TMA (rows past L are clipped)
       ok = mbar_wait(&bars[5], par, p.status, ST_TIMEOUT);
       if (__syncthreads_or(!ok)) goto done;
-      float qv[2][32];
-      tmem_ld32x2(tl + C_DQ + 64 * wg, tl + C_DQ + 64 * wg + 32, qv[0], qv[1]);
-#pragma unroll
       for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
-        float *v = qv[ch - 2 * wg];
+        float v[32];
+        tmem_ld32(tl + C_DQ + ch * 32, v);
         for (int m = 0; m < p.M; ++m) {
           const float w = s_x[m][row];
           const float4 *mk = reinterpret_cast<const float4 *>(&s_mk[m][ch * 32]);
@@ -469,17 +458,15 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
         tma_store_3d(&p.mdqo, sm + R_V, 0, t0, bh);
         tma_store_3d(&p.mdqo, sm + R_V + kReg, 64, t0, bh);
         bulk_commit();
-        bulk_wait_all();
+        bulk_wait_read();   // the staging is free once read (the writes need not have landed)
       }
     } else {
     // dq, staged as an fp32 tile over the free Q | dO regions and written
     // with TMA stores (rows past L are clipped by the map)
     unsigned char *st = sm + R_Q;
-    float qv[2][32];
-    tmem_ld32x2(tl + C_DQ + 64 * wg, tl + C_DQ + 64 * wg + 32, qv[0], qv[1]);
-#pragma unroll
     for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
-      float *v = qv[ch - 2 * wg];
+      float v[32];
+      tmem_ld32(tl + C_DQ + ch * 32, v);
       for (int m = 0; m < p.M; ++m) {
         const float w = s_x[m][row];
         const float4 *mk = reinterpret_cast<const float4 *>(&s_mk[m][ch * 32]);
@@ -502,7 +489,7 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
     if (tid == 0) {
       for (int bx = 0; bx < 4; ++bx) tma_store_3d(&p.mdq, st + bx * 16384, 32 * bx, t0, bh);
       bulk_commit();
-      bulk_wait_all();
+      bulk_wait_read();   // the staging is free once read (the writes need not have landed)
     }
     }
   }
@@ -624,7 +611,8 @@ __global__ void __launch_bounds__(NT_KV, 1) tc_swa_bwd_kv_kernel(const __grid_co
           continue;
         }
         float sv[32], dv[32];
-        tmem_ld32x2(tl + C_S + ch * 32, tl + C_DP + ch * 32, sv, dv);
+        tmem_ld32(tl + C_S + ch * 32, sv);
+        tmem_ld32(tl + C_DP + ch * 32, dv);
 #pragma unroll
         for (int u = 0; u < 32; u += 2) {
           float pr[2], ds[2];
@@ -678,7 +666,8 @@ __global__ void __launch_bounds__(NT_KV, 1) tc_swa_bwd_kv_kernel(const __grid_co
     if (__syncthreads_or(!ok)) goto done;
     for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
       float a[32], b[32];
-      tmem_ld32x2(tl + C_DK + ch * 32, tl + C_DV + ch * 32, a, b);
+      tmem_ld32(tl + C_DK + ch * 32, a);
+      tmem_ld32(tl + C_DV + ch * 32, b);
 #pragma unroll
       for (int k8 = 0; k8 < 4; ++k8) {
         uint4 *cp = chunk_ptr(sm, R_K, row, 4 * ch + k8);
@@ -712,7 +701,7 @@ __global__ void __launch_bounds__(NT_KV, 1) tc_swa_bwd_kv_kernel(const __grid_co
       tma_store_3d(&p.mdvo, sm + R_V, 0, j0, bh);
       tma_store_3d(&p.mdvo, sm + R_V + kReg, 64, j0, bh);
       bulk_commit();
-      bulk_wait_all();
+      bulk_wait_read();   // the staging is free once read (the writes need not have landed)
     }
   } else {
     // dK, dV, staged as fp32 tiles over the free K | V and Q_a | dO_a regions
@@ -720,7 +709,8 @@ __global__ void __launch_bounds__(NT_KV, 1) tc_swa_bwd_kv_kernel(const __grid_co
     unsigned char *st0 = sm + R_K, *st1 = sm + R_Q0;
     for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
       float a[32], b[32];
-      tmem_ld32x2(tl + C_DK + ch * 32, tl + C_DV + ch * 32, a, b);
+      tmem_ld32(tl + C_DK + ch * 32, a);
+      tmem_ld32(tl + C_DV + ch * 32, b);
       if (pre) {   // prefix keys: their final bf16 gradients
         if (tk >= -p.P) {
           const size_t o = ((size_t)bh * p.P + (p.P + tk)) * D + 32 * ch;
@@ -750,7 +740,7 @@ __global__ void __launch_bounds__(NT_KV, 1) tc_swa_bwd_kv_kernel(const __grid_co
         tma_store_3d(&p.mdv, st1 + bx * 16384, 32 * bx, j0, bh);
       }
       bulk_commit();
-      bulk_wait_all();
+      bulk_wait_read();   // the staging is free once read (the writes need not have landed)
     }
   }
   // the store has read this item's staging: the rest of the next item's tiles
