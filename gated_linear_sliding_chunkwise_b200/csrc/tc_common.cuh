@@ -368,7 +368,8 @@ __device__ __forceinline__ float log_decay_fast(float g, float inv_tau) {
 // projections z in TMEM: half 0 is softmax(z), half 1 is softmax(-z).  ph
 // gets the unnormalised terms exp(+-z_f - max); the result is 1 / their sum.
 __device__ __forceinline__ float feature_half(uint32_t taddr, int half, float *ph) {
-  tmem_ld32x2(taddr, taddr + 32, ph, ph + 32);
+  tmem_ld32(taddr, ph);
+  tmem_ld32(taddr + 32, ph + 32);
   const float sg = half ? -1.f : 1.f;
   float m[4];
 #pragma unroll

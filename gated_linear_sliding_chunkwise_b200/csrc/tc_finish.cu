@@ -104,7 +104,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
   const uint32_t id_dw = idesc_bf16(128, 64, 1, 1);    // X^T (MN-major) x dZ (MN-major, N = 64)
   bool fail = false;
   // this row's dphi values (its group's half) of one map, loaded ahead: map 0
-  // of the next tile while this tile finishes, map 1 while map 0 is used.
+  // of the next tile at the end of this one, map 1 while map 0 is used.
   // They stay packed (bf16) until used, so that the loads are still in flight
   // when the call returns.
   uint4 dpre[8];
@@ -180,7 +180,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
           for (int i = 0; i < 8; ++i) ph[8 * u + i] *= d[i] - dot;
         }
         if (m == 0) dphi_load(1, c);   // the k map's values, in flight while this map finishes
-        else if (c + 1 < ntiles) dphi_load(0, c + 1);
         // send the half-terms of the other group's features
         unsigned char *mine = sm + R_STG + (2 * m + wg) * 16384;
         const unsigned char *theirs = sm + R_STG + (2 * m + 1 - wg) * 16384;
@@ -287,6 +286,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
         }
       }
     }
+    // the next tile's q-map values, in flight until they are used (issued
+    // past this tile's proxy fences, which would wait for them)
+    if (gla && c + 1 < ntiles) dphi_load(0, c + 1);
     tc_fence_before();
     __syncthreads();
   }

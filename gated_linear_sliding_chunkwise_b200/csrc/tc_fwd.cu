@@ -586,7 +586,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
                                   __float_as_uint(e[2 * u + 1].z), __float_as_uint(e[2 * u + 1].w)};
           tmem_st8(tl + C_L + 64 * wg + 8 * u, r8);
         }
-        if (c + 1 < cend) e_load(c + 1);
         if (wg == 0) {   // thread row = key dimension: the tile's decay
           const float r = p.gate_r[((size_t)bh * ntiles_all + c) * D + row];
           s_dec[row] = __expf(r);
@@ -710,6 +709,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         for (int s = 0; s < 8; ++s) mma_ss(tb + C_S, desc_mn(sbase + R_KP, s), desc_mn(v, s), id_st, 1);
       mma_commit(&bar_m3);
     }
+    // state pass: the next tile's decay factors, in flight until its rows
+    // need them (issued past this tile's proxy fences, which would wait for them)
+    if (!full && c + 1 < cend) e_load(c + 1);
     // stage-1 loss: this thread's half-row of the target, in flight during MMA 3
     uint4 ytgt[8];
     if (LOSS && full && qvalid) {

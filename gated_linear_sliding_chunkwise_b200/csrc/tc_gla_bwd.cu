@@ -643,7 +643,10 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
       *chunk_ptr(sm, R_XQ, row, 2 * c16) = pack8(gk);
       *chunk_ptr(sm, R_XQ, row, 2 * c16 + 1) = pack8(gk + 8);
     }
-    if (more) e_load(w + 1, epre);   // the next item's decay factors, in flight during the dv pass
+    // the next item's decay factors (the proxy fence below waits for them;
+    // issued at the item's end instead, they were measured to arrive too
+    // late for the next item's rows)
+    if (more) e_load(w + 1, epre);
     fence_proxy_async();
     __syncthreads();
     if (tid == 0) {
