@@ -69,6 +69,7 @@ struct TileParams {
   CUtensorMap mw;                             // [H*2][D][F] bf16 feature-map weights (W_q, W_k per head)
   CUtensorMap mdq, mdk;                       // bf16 outputs dphi_q, dphi_k, row halves centred (TMA stores)
   CUtensorMap mdb, mdv;                       // fp32 outputs dB, dv (TMA stores)
+  CUtensorMap me;                             // fp32 decay factors (loads)
   const float *e32;            // fp32 decay factors [BH*L][D]
   const float *sp_r0, *ds_r0;  // [BH*ntiles][D] row 0 of S' and of dS (the copies hold the rest)
   uint32_t *status;
@@ -206,6 +207,9 @@ __global__ void __launch_bounds__(NT_DS, 1) tc_gla_dstates_kernel(const __grid_c
     }
     // E in fp32 (dimensions 64 wg ..) into TMEM; the tile's decay exp(r)
     e_half_store(epre, tl + C_E + 64 * wg);
+    // the previous tile's factors: in flight through the proxy fence below,
+    // which waits for them (issued past it, they were measured to arrive too
+    // late for that tile's rows)
     if (c > 0) e_load(c - 1);
     if (wg == 0) s_dec[row] = __expf(p.gate_r[((size_t)bh * ntiles + c) * D + row]);
     tmem_st_wait();
@@ -284,7 +288,7 @@ constexpr int NT_TILE = 256;
 __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __grid_constant__ TileParams p) {
   extern __shared__ unsigned char smraw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
-  __shared__ uint64_t bars[8];
+  __shared__ uint64_t bars[9];
   __shared__ uint32_t s_tmem;
   // Per row: dO . S'[0], V . dS[0], sum_i Kt[i] -- the rank-one parts of GQ,
   // GK and dv that the copies (S' - 1 S'[0], dS - 1 dS[0]) leave out.  Before
@@ -309,9 +313,8 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
   // Persistent: CTA b walks the contiguous run [w0, w1) of (sequence, tile)
   // items, item w = tile w % ntiles of sequence w / ntiles.  The next item's
   // inputs go out as this item frees their places: the weights once the last
-  // products are done, the decay factors during the dphi pass, V and dO once
-  // the dB store has read its staging, X_q after the dphi stores, X_k after
-  // the dv store.
+  // products are done, V and dO once the dB store has read its staging, X_q
+  // after the dphi stores, X_k and the decay factors after the dv store.
   const int nwork = p.ntiles * p.BH;
   const int w0 = (int)((long long)blockIdx.x * nwork / gridDim.x);
   const int w1 = (int)((long long)(blockIdx.x + 1) * nwork / gridDim.x);
@@ -329,19 +332,25 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
       }
     }
   };
-  auto e_load = [&](int w, float4 *e) {   // this row's fp32 decay factors (its dimension half) of item w
-    const int lbh = w / p.ntiles, ltq = (w % p.ntiles) * T + row;
-    e_half_load(p.e32, ((size_t)lbh * p.L + (ltq < p.L ? ltq : 0)) * D, ltq < p.L, wg, e);
+  // the fp32 decay factors of item w, four 32-column boxes: dimensions 0..63
+  // over Qt lo, 64..127 over Kt lo (free from the item's end until its
+  // rows have moved them to TMEM); rows past L read as zero
+  auto e_tma = [&](int w) {
+    const int lbh = w / p.ntiles, lt0 = (w % p.ntiles) * T;
+    mbar_expect_tx(&bars[8], 2 * TILE);
+    for (int bx = 0; bx < 4; ++bx)
+      tma_load_3d(sm + (bx < 2 ? R_QL : R_KL) + (bx & 1) * 16384, &p.me, &bars[8], 32 * bx, lt0, lbh);
   };
   if (warp == 0) { tmem_alloc(&s_tmem, 512); tmem_relinquish(); }
   if (tid == 0) {
-    for (int i = 0; i < 8; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < 9; ++i) mbar_init(&bars[i], 1);
     fence_barrier_init();
     if (w0 < w1) {
       item_loads(w0, 0);
       item_loads(w0, 1);
       item_loads(w0, 2);
       item_loads(w0, 3);
+      e_tma(w0);
     }
   }
   tc_fence_before();
@@ -351,11 +360,10 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
   const uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
   const uint32_t id_mn = idesc_bf16(128, 128, 0, 1);
   const uint32_t id_z = idesc_bf16(128, 64, 0, 1);
-  float4 epre[16];   // this row's decay factors of the item to come
-  if (w0 < w1) e_load(w0, epre);
   // copies in flight when a wait gives up (tid 0's view): the parity of an
-  // armed phase of bars[0], and whether the S' / dS loads of this item are out
-  int pend0 = w0 < w1 ? 0 : -1;
+  // armed phase of bars[0] and of bars[8], and whether the S' / dS loads of
+  // this item are out
+  int pend0 = w0 < w1 ? 0 : -1, pend_e = w0 < w1 ? 0 : -1;
   bool pend_sp = false, pend_ds = false;
   bool ok = true;
   uint32_t par = 0;
@@ -431,11 +439,25 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
       mma_commit(&bars[4]);
     }
   }
-  //    E in fp32 (dimensions 64 wg ..) into TMEM, then Qt = phi_q E and
-  //    Kt = phi_k / E for the same dimensions (rows past L: Kt = 0), each as
-  //    a bf16 pair hi + lo
-  e_half_store(epre, tl + C_E + 64 * wg);
+  //    E in fp32 (dimensions 64 wg .., from shared memory) into TMEM, then
+  //    Qt = phi_q E and Kt = phi_k / E for the same dimensions (rows past L:
+  //    Kt = 0), each as a bf16 pair hi + lo
+  ok = mbar_wait(&bars[8], par, p.status, ST_TIMEOUT);
+  if (__syncthreads_or(!ok)) { ok = false; goto done; }
+  pend_e = -1;
+  {
+    const unsigned char *es = sm + (wg == 0 ? R_QL : R_KL);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float4 a = *f32_stage_ptr(const_cast<unsigned char *>(es), row, 8 * u);
+      const float4 b = *f32_stage_ptr(const_cast<unsigned char *>(es), row, 8 * u + 4);
+      const uint32_t r8[8] = {__float_as_uint(a.x), __float_as_uint(a.y), __float_as_uint(a.z), __float_as_uint(a.w),
+                              __float_as_uint(b.x), __float_as_uint(b.y), __float_as_uint(b.z), __float_as_uint(b.w)};
+      tmem_st8(tl + C_E + 64 * wg + 8 * u, r8);
+    }
+  }
   tmem_st_wait();
+  __syncthreads();   // E read out of Qt lo | Kt lo before they are written
   r1[0] = r1[1] = r1[2] = 0.f;
   {
     const float *ms = s_row0 + 64 * wg, *md = s_row0 + D + 64 * wg;
@@ -643,10 +665,6 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
       *chunk_ptr(sm, R_XQ, row, 2 * c16) = pack8(gk);
       *chunk_ptr(sm, R_XQ, row, 2 * c16 + 1) = pack8(gk + 8);
     }
-    // the next item's decay factors (the proxy fence below waits for them;
-    // issued at the item's end instead, they were measured to arrive too
-    // late for the next item's rows)
-    if (more) e_load(w + 1, epre);
     fence_proxy_async();
     __syncthreads();
     if (tid == 0) {
@@ -686,6 +704,8 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
         item_loads(w + 1, 1);
         bulk_wait_read();        // dv out of Kt hi | Kt lo
         item_loads(w + 1, 3);
+        pend_e = (int)(par ^ 1u);
+        e_tma(w + 1);            // over Qt lo | Kt lo, both read out by now
       }
     }
   }
@@ -697,6 +717,7 @@ done:
     bulk_wait_all();   // this CTA's stores are complete (and have read their staging)
     if (!ok) {         // a wait gave up: let the copies still in flight land first
       if (pend0 >= 0) mbar_wait(&bars[0], (uint32_t)pend0, nullptr, 0, 1u << 16);
+      if (pend_e >= 0) mbar_wait(&bars[8], (uint32_t)pend_e, nullptr, 0, 1u << 16);
       if (pend_sp) mbar_wait(&bars[2], par, nullptr, 0, 1u << 16);
       if (pend_ds) mbar_wait(&bars[6], par, nullptr, 0, 1u << 16);
     }
@@ -887,7 +908,8 @@ cudaError_t launch_tc_gla_bwd(const TcGlaBwdArgs &a, int stage, cudaStream_t s) 
         !make_map_bf16_3d(&p.mw, a.w16, F, D, (uint64_t)a.H * 2, T) ||
         !make_map_bf16_3d(&p.mds, a.snap_ds, D, D, (uint64_t)a.BH * ntiles, T) ||
         !make_map_bf16_3d(&p.mdq, a.dphq, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mdk, a.dphk, D, rows, a.BH, T) ||
-        !make_map_f32_3d(&p.mdb, a.dB, D, rows, a.BH, T) || !make_map_f32_3d(&p.mdv, a.dv, D, rows, a.BH, T))
+        !make_map_f32_3d(&p.mdb, a.dB, D, rows, a.BH, T) || !make_map_f32_3d(&p.mdv, a.dv, D, rows, a.BH, T) ||
+        !make_map_f32_3d(&p.me, a.e32, D, rows, a.BH, T))
       return cudaErrorInvalidValue;
     p.e32 = a.e32;
     p.sp_r0 = snapshot_row0(a.snap_s, a.BH, a.L);
