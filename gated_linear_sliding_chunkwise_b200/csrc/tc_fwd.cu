@@ -87,6 +87,7 @@ constexpr uint32_t ST_TIMEOUT = 1u, ST_RANGE = 2u;
 struct Params {
   CUtensorMap mq, mk, mv, mg;
   CUtensorMap mkp, mvp;     // key / value prefix [BH][P][D] (P > 0 only)
+  CUtensorMap me;           // mode 1: fp32 decay factors E [BH][L][D] (loads)
   const float *wq, *wk, *meta_k, *meta_v, *alpha, *state_in;
   __nv_bfloat16 *o;
   float *state_out, *lse;
@@ -97,7 +98,7 @@ struct Params {
   __nv_bfloat16 *snap;      // mode 1 with nseg == 1: [BH][ntiles][D][D] bf16 S' - 1 S'[0] of every tile
   float *snap_r0;           // ... and [BH][ntiles][D] fp32 row 0 of S' (the part taken out of every row)
   const float *gate_r;      // [BH][ntiles][D] log-decay r of every tile (gate_prep_kernel)
-  const float *gate_e32;    // mode 1: [BH][L][D] fp32 decay factors E (mode 0 loads bf16 E as the G tiles)
+  const float *gate_e32;    // mode 1: [BH][L][D] fp32 decay factors E, loaded through `me` (mode 0 loads bf16 E as the G tiles)
   const float *kap_g;       // mode 1 with copies: incoming final-state gradient G [BH][D][D], or null
   float *kap;               // ... and [BH][2][D]: the column halves of sum_v G[i][v] S_L[i][v]
   int H, L, M, window, branch;
@@ -122,7 +123,7 @@ struct Params {
 
 __device__ __forceinline__ void issue_tile_loads(const Params &p, unsigned char *sm, uint64_t *bar, int bh,
                                                  int t0, bool full) {
-  mbar_expect_tx(bar, (full ? 5 : 2) * TILE);
+  mbar_expect_tx(bar, (full ? 5 : 4) * TILE);
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
     if (full) {
@@ -138,6 +139,9 @@ __device__ __forceinline__ void issue_tile_loads(const Params &p, unsigned char 
     tma_load_3d(sm + R_XK + r * REG, &p.mk, bar, 64 * r, t0, bh);
     tma_load_3d(sm + R_V + r * REG, &p.mv, bar, 64 * r, t0, bh);
   }
+  if (!full)   // state pass: the fp32 decay factors, dimensions 0..63 over X_q, 64..127 over G (unused there)
+    for (int bx = 0; bx < 4; ++bx)
+      tma_load_3d(sm + (bx < 2 ? R_XQ : R_G) + (bx & 1) * 16384, &p.me, bar, 32 * bx, t0, bh);
 }
 
 // Qt for dimensions 64 h .. 64 h + 63: phi_q E gscale, bf16 pairs into TMEM.
@@ -159,26 +163,33 @@ __device__ __forceinline__ void qt_half(unsigned char *sm, uint32_t tl, int row,
 
 // Kt for dimensions 64 h .. 64 h + 63: phi_k / E, bf16 into shared memory
 // over X_k.  E comes as bf16 from the gate region (full pass) or as fp32
-// from TMEM (state pass, which also writes the rounding remainder Kt - bf16(Kt)
-// over the K_prev region, so that its state update runs on hi + lo).  Rows
-// past L (where the full pass's E is zero) get Kt = 0.
-__device__ __forceinline__ void kt_half(unsigned char *sm, uint32_t tl, int row, int h, bool e_in_tmem,
-                                        bool valid) {
+// tiles over X_q | G (state pass, which also writes the rounding remainder
+// Kt - bf16(Kt) over the K_prev region, so that its state update runs on
+// hi + lo).  Rows past L (where E is zero) get Kt = 0.
+__device__ __forceinline__ void kt_half(unsigned char *sm, uint32_t tl, int row, int h, bool e_fp32, bool valid) {
   float ph[F];
   float s = feature_half(tl + C_ZK, h, ph);   // warp-collective TMEM loads: every lane
   if (!valid) s = 0.f;
 #pragma unroll
   for (int c16 = 0; c16 < 4; ++c16) {
     float e16[16], k16[16];
-    if (e_in_tmem) {
-      tmem_ld16(tl + C_L + 64 * h + 16 * c16, e16);
+    if (e_fp32) {
+      unsigned char *es = sm + (h == 0 ? R_XQ : R_G);
+#pragma unroll
+      for (int u = 0; u < 16; u += 4) {
+        const float4 e4 = *f32_stage_ptr(es, row, 16 * c16 + u);
+        e16[u] = e4.x;
+        e16[u + 1] = e4.y;
+        e16[u + 2] = e4.z;
+        e16[u + 3] = e4.w;
+      }
     } else {
       unpack8(*chunk_ptr(sm, R_G, row, 8 * h + 2 * c16), e16);
       unpack8(*chunk_ptr(sm, R_G, row, 8 * h + 2 * c16 + 1), e16 + 8);
     }
 #pragma unroll
     for (int u = 0; u < 16; ++u) k16[u] = valid ? __fdividef(ph[16 * c16 + u] * s, e16[u]) : 0.f;
-    if (e_in_tmem) {
+    if (e_fp32) {
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         uint4 hi, lo;
@@ -405,17 +416,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
   const uint32_t id_st = idesc_bf16(128, 128, 1, 1);
 
   float mse_acc = 0.f;                        // this thread's share of sum (o - target)^2
-  // state pass: this row's fp32 decay factors (its dimension half) of the
-  // next tile, loaded one tile ahead
-  float4 epre[16];
-  auto e_load = [&](int c) {
-    const int t = c * T + row;
-    const float *er = p.gate_e32 + ((size_t)bh * p.L + (t < p.L ? t : 0)) * D + 64 * wg;
-#pragma unroll
-    for (int u = 0; u < 16; ++u)
-      epre[u] = t < p.L ? *reinterpret_cast<const float4 *>(er + 4 * u) : make_float4(1.f, 1.f, 1.f, 1.f);
-  };
-  if (!full && cbeg < cend) e_load(cbeg);
   const int cstop = s_fail ? cbeg : cend;
   for (int c = cbeg; c < cstop; ++c) {
     const uint32_t par = (c - cbeg) & 1;
@@ -575,24 +575,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       qt_half(sm, tl, row, wg, gscale);
       kt_half(sm, tl, row, wg, false, qvalid);
     } else {
-      // ------ state pass: fp32 decay factors of this row's dimension half
-      //        (from gate_prep_kernel) into TMEM, phi_k half per group ---
-      {
-        const float4 *e = epre;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const uint32_t r8[8] = {__float_as_uint(e[2 * u].x), __float_as_uint(e[2 * u].y), __float_as_uint(e[2 * u].z),
-                                  __float_as_uint(e[2 * u].w), __float_as_uint(e[2 * u + 1].x), __float_as_uint(e[2 * u + 1].y),
-                                  __float_as_uint(e[2 * u + 1].z), __float_as_uint(e[2 * u + 1].w)};
-          tmem_st8(tl + C_L + 64 * wg + 8 * u, r8);
-        }
-        if (wg == 0) {   // thread row = key dimension: the tile's decay
-          const float r = p.gate_r[((size_t)bh * ntiles_all + c) * D + row];
-          s_dec[row] = __expf(r);
-          tot_decay += r;
-        }
+      // ------ state pass: phi_k half per group, with the fp32 decay factors
+      //        (from gate_prep_kernel) that came with the tile's loads ---
+      if (wg == 0) {   // thread row = key dimension: the tile's decay
+        const float r = p.gate_r[((size_t)bh * ntiles_all + c) * D + row];
+        s_dec[row] = __expf(r);
+        tot_decay += r;
       }
-      tmem_st_wait();
       ok &= mbar_wait(&bar_m1, par, err, ST_TIMEOUT);
       tc_fence_after();
       kt_half(sm, tl, row, wg, true, qvalid);
@@ -709,9 +698,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         for (int s = 0; s < 8; ++s) mma_ss(tb + C_S, desc_mn(sbase + R_KP, s), desc_mn(v, s), id_st, 1);
       mma_commit(&bar_m3);
     }
-    // state pass: the next tile's decay factors, in flight until its rows
-    // need them (issued past this tile's proxy fences, which would wait for them)
-    if (!full && c + 1 < cend) e_load(c + 1);
     // stage-1 loss: this thread's half-row of the target, in flight during MMA 3
     uint4 ytgt[8];
     if (LOSS && full && qvalid) {
@@ -1030,7 +1016,8 @@ cudaError_t launch_tc_state_snapshots(const TcFwdArgs &a, void *snap, const floa
   if (!make_map_bf16_3d(&p.mq, a.q, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mk, a.k, D, rows, a.BH, T) ||
       !make_map_bf16_3d(&p.mv, a.v, D, rows, a.BH, T))
     return cudaErrorInvalidValue;
-  p.gate_e32 = e32;   // the state pass loads no gate tiles (p.mg stays unset)
+  p.gate_e32 = e32;   // the state pass loads fp32 factors, no gate tiles (p.mg stays unset)
+  if (!make_map_f32_3d(&p.me, e32, D, rows, a.BH, T)) return cudaErrorInvalidValue;
   p.gate_r = r;
   p.wq = a.wq;
   p.wk = a.wk;
@@ -1086,6 +1073,7 @@ cudaError_t launch_tc_segment_state(const TcFwdArgs &a, float *U, float *R, void
       !make_map_bf16_3d(&p.mv, a.v, D, rows, a.BH, T))
     return cudaErrorInvalidValue;
   p.gate_e32 = e32;
+  if (!make_map_f32_3d(&p.me, e32, D, rows, a.BH, T)) return cudaErrorInvalidValue;
   p.gate_r = r;
   p.wk = a.wk;
   p.status = a.status;
@@ -1134,6 +1122,7 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, int stage, cudaStream_t s) {
     return cudaErrorInvalidValue;
   p.gate_r = gla ? w.r : nullptr;
   p.gate_e32 = gla ? w.e32 : nullptr;
+  if (gla && nseg > 1 && !make_map_f32_3d(&p.me, w.e32, D, rows, a.BH, T)) return cudaErrorInvalidValue;
   p.wq = a.wq;
   p.wk = a.wk;
   p.meta_k = a.meta_k;

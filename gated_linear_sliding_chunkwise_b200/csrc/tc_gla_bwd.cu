@@ -53,6 +53,7 @@ constexpr uint32_t ST_TIMEOUT = 1u, ST_RANGE = 2u;
 
 struct DsParams {
   CUtensorMap mq, mo;
+  CUtensorMap me;              // fp32 decay factors (loads)
   const float *wq;
   const float *e32, *gate_r;   // fp32 decay factors [BH*L][D] and tile log-decays [BH][ntiles][D]
   __nv_bfloat16 *snap;      // [BH][ntiles][D][D] dS - 1 dS[0] at each tile's end (bf16)
@@ -88,25 +89,6 @@ __device__ __forceinline__ void stage_weights(unsigned char *dst, const float *W
   }
 }
 
-// fp32 decay factors of tile row `t` (< L, else 1), dimensions 64 h ..
-// 64 h + 63, from the precomputed array into TMEM columns col .. col + 63,
-// in two halves: the loads (in flight early) and the TMEM stores.
-__device__ __forceinline__ void e_half_load(const float *e32, size_t row_off, bool valid, int h, float4 *e) {
-  const float *er = e32 + row_off + 64 * h;
-#pragma unroll
-  for (int u = 0; u < 16; ++u)
-    e[u] = valid ? *reinterpret_cast<const float4 *>(er + 4 * u) : make_float4(1.f, 1.f, 1.f, 1.f);
-}
-__device__ __forceinline__ void e_half_store(const float4 *e, uint32_t taddr) {
-#pragma unroll
-  for (int u = 0; u < 8; ++u) {
-    const uint32_t r8[8] = {__float_as_uint(e[2 * u].x), __float_as_uint(e[2 * u].y), __float_as_uint(e[2 * u].z),
-                            __float_as_uint(e[2 * u].w), __float_as_uint(e[2 * u + 1].x), __float_as_uint(e[2 * u + 1].y),
-                            __float_as_uint(e[2 * u + 1].z), __float_as_uint(e[2 * u + 1].w)};
-    tmem_st8(taddr + 8 * u, r8);
-  }
-}
-
 // ------------------------------------------------------ reverse dS pass ---
 // Two warpgroups (256 threads): thread = tile row / state row `row` of its
 // group; the groups take halves of the key dimensions (E, phi_q) and of the
@@ -119,9 +101,10 @@ __global__ void __launch_bounds__(NT_DS, 1) tc_gla_dstates_kernel(const __grid_c
   __shared__ __align__(16) float s_row0[D];   // row 0 of dS, taken out of the bf16 copy
   __shared__ uint64_t bar_tma, bar_m1, bar_m2;
   __shared__ uint32_t s_tmem;
-  // Qt (hi) over X_q, the remainder Qt - bf16(Qt) in R_QL, dO, W_q
-  constexpr uint32_t R_XQ = 0, R_QL = TILE, R_O = 2 * TILE, R_W = 3 * TILE;
-  constexpr uint32_t C_S = 0, C_Z = 128, C_E = 256;
+  // Qt (hi) over X_q, the remainder Qt - bf16(Qt) in R_QL, dO, W_q, the
+  // tile's fp32 decay factors E (four 32-column boxes)
+  constexpr uint32_t R_XQ = 0, R_QL = TILE, R_O = 2 * TILE, R_W = 3 * TILE, R_E = 3 * TILE + TILE / 2;
+  constexpr uint32_t C_S = 0, C_Z = 128;
   const int tid = threadIdx.x, warp = tid >> 5, wg = tid >> 7, row = tid & 127;
   const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
   const int bh = blockIdx.x, h = bh % p.H;
@@ -154,21 +137,14 @@ __global__ void __launch_bounds__(NT_DS, 1) tc_gla_dstates_kernel(const __grid_c
   const uint32_t id_z = idesc_bf16(128, 64, 0, 1);
   const uint32_t id_st = idesc_bf16(128, 128, 1, 1);
   auto loads = [&](int c) {
-    mbar_expect_tx(&bar_tma, 2 * TILE);
+    mbar_expect_tx(&bar_tma, 4 * TILE);
     for (int r = 0; r < 2; ++r) {
       tma_load_3d(sm + R_XQ + r * REG, &p.mq, &bar_tma, 64 * r, c * T, bh);
       tma_load_3d(sm + R_O + r * REG, &p.mo, &bar_tma, 64 * r, c * T, bh);
     }
+    for (int bx = 0; bx < 4; ++bx) tma_load_3d(sm + R_E + bx * 16384, &p.me, &bar_tma, 32 * bx, c * T, bh);
   };
   if (tid == 0 && ntiles > 0) loads(ntiles - 1);
-  // this row's fp32 decay factors (its dimension half) of the tile to come:
-  // loaded one tile ahead, so that they are in flight during the previous one
-  float4 epre[16];
-  auto e_load = [&](int c) {
-    const int t = c * T + row;
-    e_half_load(p.e32, ((size_t)bh * p.L + (t < p.L ? t : 0)) * D, t < p.L, wg, epre);
-  };
-  if (ntiles > 0) e_load(ntiles - 1);
   bool fail = false;
   for (int c = ntiles - 1; c >= 0; --c) {
     const uint32_t par = (ntiles - 1 - c) & 1;
@@ -205,14 +181,8 @@ __global__ void __launch_bounds__(NT_DS, 1) tc_gla_dstates_kernel(const __grid_c
       }
       if (tid < D) p.snap_r0[tile * D + tid] = s_row0[tid];
     }
-    // E in fp32 (dimensions 64 wg ..) into TMEM; the tile's decay exp(r)
-    e_half_store(epre, tl + C_E + 64 * wg);
-    // the previous tile's factors: in flight through the proxy fence below,
-    // which waits for them (issued past it, they were measured to arrive too
-    // late for that tile's rows)
-    if (c > 0) e_load(c - 1);
+    // the tile's decay exp(r)
     if (wg == 0) s_dec[row] = __expf(p.gate_r[((size_t)bh * ntiles + c) * D + row]);
-    tmem_st_wait();
     ok = mbar_wait(&bar_m1, par, p.status, ST_TIMEOUT);
     tc_fence_after();
     {   // Qt = phi_q E into shared memory over X_q (row = token), dimension half per group
@@ -220,10 +190,15 @@ __global__ void __launch_bounds__(NT_DS, 1) tc_gla_dstates_kernel(const __grid_c
       const float sc = feature_half(tl + C_Z, wg, ph);
 #pragma unroll
       for (int c16 = 0; c16 < 4; ++c16) {
-        float E[16], q16[16];
-        tmem_ld16(tl + C_E + 64 * wg + 16 * c16, E);
+        float q16[16];
 #pragma unroll
-        for (int u = 0; u < 16; ++u) q16[u] = ph[16 * c16 + u] * sc * E[u];
+        for (int u = 0; u < 16; u += 4) {   // E of dimensions 64 wg + 16 c16 + u .. (zero past L)
+          const float4 E = *f32_stage_ptr(sm + R_E, row, 64 * wg + 16 * c16 + u);
+          q16[u] = ph[16 * c16 + u] * sc * E.x;
+          q16[u + 1] = ph[16 * c16 + u + 1] * sc * E.y;
+          q16[u + 2] = ph[16 * c16 + u + 2] * sc * E.z;
+          q16[u + 3] = ph[16 * c16 + u + 3] * sc * E.w;
+        }
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           uint4 hi, lo;
@@ -852,7 +827,7 @@ __global__ void __launch_bounds__(256) weights_bf16_kernel(const float *wq, cons
   }
 }
 
-constexpr size_t DS_SMEM = 3 * TILE + TILE / 2 + 1024;
+constexpr size_t DS_SMEM = 5 * TILE + TILE / 2 + 1024;
 constexpr size_t TILE_SMEM = 7 * TILE + 1024;
 
 }  // namespace
@@ -881,7 +856,8 @@ cudaError_t launch_tc_gla_bwd(const TcGlaBwdArgs &a, int stage, cudaStream_t s) 
   if (stage == 0) {   // reverse dS pass
     DsParams p;
     memset(&p, 0, sizeof(p));
-    if (!make_map_bf16_3d(&p.mq, a.q, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mo, a.dout, D, rows, a.BH, T))
+    if (!make_map_bf16_3d(&p.mq, a.q, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mo, a.dout, D, rows, a.BH, T) ||
+        !make_map_f32_3d(&p.me, a.e32, D, rows, a.BH, T))
       return cudaErrorInvalidValue;
     p.wq = a.wq;
     p.e32 = a.e32;
