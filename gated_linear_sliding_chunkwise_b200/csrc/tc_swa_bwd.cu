@@ -93,15 +93,15 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
   __shared__ __align__(16) float s_mk[MAXM][D];
   __shared__ __align__(16) float s_mv[MAXM][D];
   __shared__ float s_x[MAXM][T];        // dO . mv_m per row, later the meta dS per row
-  __shared__ float s_pmax[2][T], s_psum[2][T];
+  __shared__ float s_pmax[2][T], s_psum[2][T], s_dpart[2][T];
   __shared__ float s_red[4];
   __shared__ uint64_t bars[6];
   __shared__ uint32_t s_tmem;
   // regions: Q, dO, K_prev, K, V_prev, V
   constexpr uint32_t R_Q = 0, R_O = TILE, R_KP = 2 * TILE, R_K = 3 * TILE, R_VP = 4 * TILE, R_V = 5 * TILE;
-  // TMEM: P^ [0,128) (over the logits [0,256)), O' [256,384), dP' [128,384),
-  // dS [384,512), dq' [128,256)
-  constexpr uint32_t C_L = 0, C_P = 0, C_O = 256, C_DP = 128, C_DS = 384, C_DQ = 128;
+  // TMEM: logits [0,256) then P^ [0,128), dP' [256,512) (issued with the
+  // logits), dS [128,256), dq' [0,128)
+  constexpr uint32_t C_L = 0, C_P = 0, C_DP = 256, C_DS = 128, C_DQ = 0;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wg = tid >> 7, row = tid & 127;
   const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
@@ -169,11 +169,13 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
   ok = mbar_wait(bar_tma, par, p.status, ST_TIMEOUT);
   if (__syncthreads_or(!ok)) goto done;
 
-  // 1. logits L = Q [K_prev ; K]^T
+  // 1. logits L = Q [K_prev ; K]^T and dP' = dO [V_prev ; V]^T
   if (tid == 0) {
     tc_fence_after();
     for (int s = 0; s < 8; ++s) mma_ss(tb + C_L, desc_k(sbase + R_Q, s), desc_k(sbase + R_KP, s), id_kk, s > 0);
     for (int s = 0; s < 8; ++s) mma_ss(tb + C_L + 128, desc_k(sbase + R_Q, s), desc_k(sbase + R_K, s), id_kk, s > 0);
+    for (int s = 0; s < 8; ++s) mma_ss(tb + C_DP, desc_k(sbase + R_O, s), desc_k(sbase + R_VP, s), id_kk, s > 0);
+    for (int s = 0; s < 8; ++s) mma_ss(tb + C_DP + 128, desc_k(sbase + R_O, s), desc_k(sbase + R_V, s), id_kk, s > 0);
     mma_commit(bar_m);
   }
   {
@@ -214,6 +216,11 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
     ok = mbar_wait(bar_m, par, p.status, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) goto done;
     tc_fence_after();
+    if (p.fused && tid == 0) {   // the GLA part of dq into the V region (only dP' read V)
+      mbar_expect_tx(&bars[5], TILE);
+      tma_load_3d(sm + R_V, &p.mxq, &bars[5], 0, t0, bh);
+      tma_load_3d(sm + R_V + kReg, &p.mxq, &bars[5], 64, t0, bh);
+    }
     float mx = kNegBig;
     if (wg == 0) {
 #pragma unroll
@@ -257,14 +264,17 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
     mx = fmaxf(s_pmax[0][row], s_pmax[1][row]);
     //    P^ = exp(l - max) of this group's chunks, held in registers until
     //    both groups have read their logits (P^ overlays logit chunks 0 .. 3)
+    //    and, for D = dO_swa . o_swa = alpha (sum_j P^_j dP'_j + sum_m e_m
+    //    dO . mv_m) / l, the sums of P^ dP' over the same chunks
     uint32_t pk[3][16];
-    float s4[4] = {0.f, 0.f, 0.f, 0.f};
+    float s4[4] = {0.f, 0.f, 0.f, 0.f}, d4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int k = 0; k < 3; ++k) {
       const int ch = ch_lo + wg + 2 * k;
       if (ch > ch_hi) continue;
-      float v[32];
+      float v[32], dp[32];
       tmem_ld32(tl + C_L + ch * 32, v);
+      tmem_ld32(tl + C_DP + ch * 32, dp);
       const bool inner = 32 * ch >= in_lo && 32 * ch + 31 <= 32 * w4 + T && 32 * ch + cbase >= -p.P;
 #pragma unroll
       for (int u = 0; u < 32; u += 2) {
@@ -276,16 +286,23 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
           e1 = (cl + 1 >= lo_c && cl + 1 <= hi_c) ? e1 : 0.f;
         }
         s4[(u >> 1) & 3] += e0 + e1;
+        d4[(u >> 1) & 3] = fmaf(e0, dp[u], fmaf(e1, dp[u + 1], d4[(u >> 1) & 3]));
         pk[k][u / 2] = pack_bf16(e0, e1);
       }
     }
     float psum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+    float dpart = (d4[0] + d4[1]) + (d4[2] + d4[3]);
     if (wg == 0) {
 #pragma unroll
       for (int m = 0; m < MAXM; ++m)
-        if (m < p.M) { em[m] = __expf(ml[m] - mx); psum += em[m]; }
+        if (m < p.M) {
+          em[m] = __expf(ml[m] - mx);
+          psum += em[m];
+          dpart = fmaf(em[m], dom[m], dpart);
+        }
     }
     s_psum[wg][row] = psum;
+    s_dpart[wg][row] = dpart;
     bar_sync(2, NT_Q);
     const float lsum = s_psum[0][row] + s_psum[1][row];
     const float inv_l = 1.f / lsum;
@@ -306,38 +323,8 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
     }
     if (wg == 0 && qvalid) p.lse[(size_t)bh * p.L + tq] = mx + logf(lsum);
     tmem_st_wait();
-    tc_fence_before();
-    __syncthreads();
-
-    // 3. O' = P^ [V_prev ; V]   (o_swa = (O' + sum_m em_m mv_m) / l)
-    if (tid == 0) {
-      tc_fence_after();
-      for (int s = 0; s < 8; ++s) mma_ts(tb + C_O, tb + C_P + s * 8, desc_mn(sbase + R_VP, s), id_mn, s > 0);
-      for (int s = 0; s < 8; ++s) mma_ts(tb + C_O, tb + C_P + 64 + s * 8, desc_mn(sbase + R_V, s), id_mn, 1);
-      mma_commit(&bars[2]);
-    }
-    ok = mbar_wait(&bars[2], par, p.status, ST_TIMEOUT);
-    if (__syncthreads_or(!ok)) goto done;
-    tc_fence_after();
-    float dpart = 0.f;                    // dout . o_swa for this row, column half per group
-    for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
-      float v[32];
-      tmem_ld32(tl + C_O + ch * 32, v);
-#pragma unroll
-      for (int c8 = 0; c8 < 4; ++c8) {
-        float o8[8];
-        unpack8(*chunk_ptr(sm, R_O, row, ch * 4 + c8), o8);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) dpart = fmaf(o8[u], v[c8 * 8 + u], dpart);
-      }
-    }
-    if (wg == 0) {
-#pragma unroll
-      for (int m = 0; m < MAXM; ++m) dpart = fmaf(em[m], dom[m], dpart);
-    }
-    s_pmax[wg][row] = dpart;
-    bar_sync(3, NT_Q);
-    float dal = (s_pmax[0][row] + s_pmax[1][row]) * inv_l;
+    // 3. D (dO_swa . o_swa) from the two groups' sums
+    float dal = (s_dpart[0][row] + s_dpart[1][row]) * inv_l;
     if (!qvalid) dal = 0.f;
     const float Dt = alpha * dal;
     if (wg == 0) {
@@ -348,26 +335,11 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
       }
     }
     tc_fence_before();
-    __syncthreads();
+    __syncthreads();   // also: every group's P^ stores are in before the other reads them
+    tc_fence_after();
     if (tid == 0 && p.dalpha) atomicAdd(p.dalpha + h, s_red[0] + s_red[1] + s_red[2] + s_red[3]);
 
-    // 4. dP' = dO [V_prev ; V]^T
-    if (tid == 0) {
-      tc_fence_after();
-      for (int s = 0; s < 8; ++s) mma_ss(tb + C_DP, desc_k(sbase + R_O, s), desc_k(sbase + R_VP, s), id_kk, s > 0);
-      for (int s = 0; s < 8; ++s) mma_ss(tb + C_DP + 128, desc_k(sbase + R_O, s), desc_k(sbase + R_V, s), id_kk, s > 0);
-      mma_commit(&bars[3]);
-    }
-    ok = mbar_wait(&bars[3], par, p.status, ST_TIMEOUT);
-    if (__syncthreads_or(!ok)) goto done;
-    tc_fence_after();
-    if (p.fused && tid == 0) {   // the GLA part of dq into the free V region
-      mbar_expect_tx(&bars[5], TILE);
-      tma_load_3d(sm + R_V, &p.mxq, &bars[5], 0, t0, bh);
-      tma_load_3d(sm + R_V + kReg, &p.mxq, &bars[5], 64, t0, bh);
-    }
-
-    // 5. dS = P (alpha dP' - D), P = P^ / l, on the band (zero elsewhere,
+    // 4. dS = P (alpha dP' - D), P = P^ / l, on the band (zero elsewhere,
     //    as P^ is); alternate chunks per group; the meta terms go to memory
     for (int ch = wg; ch < 8; ch += 2) {
       uint32_t ds[16];
@@ -409,7 +381,7 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
     tc_fence_before();
     __syncthreads();
 
-    // 6. dq' = dS [K_prev ; K]
+    // 5. dq' = dS [K_prev ; K]
     if (tid == 0) {
       tc_fence_after();
       for (int s = 0; s < 8; ++s) mma_ts(tb + C_DQ, tb + C_DS + s * 8, desc_mn(sbase + R_KP, s), id_mn, s > 0);
