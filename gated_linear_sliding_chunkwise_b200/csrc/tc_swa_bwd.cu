@@ -484,7 +484,8 @@ constexpr int NT_KV = 256;
 __global__ void __launch_bounds__(NT_KV, 1) tc_swa_bwd_kv_kernel(const __grid_constant__ KVParams p) {
   extern __shared__ unsigned char smraw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
-  __shared__ float s_lse[2 * T], s_D[2 * T];
+  __shared__ __align__(16) float s_lse[2 * T];
+  __shared__ __align__(16) float s_D[2 * T];
   __shared__ uint64_t bars[7];
   __shared__ uint32_t s_tmem;
   // regions: K, V, Q_a, dO_a, Q_b, dO_b  (query tiles kb and kb + 1)
@@ -573,6 +574,11 @@ __global__ void __launch_bounds__(NT_KV, 1) tc_swa_bwd_kv_kernel(const __grid_co
     // (P and dS overlay the logit columns of the lower chunks).
     {
       const int qlo = max(0, r0 - it * T), qhi = min(T - 1, r0 + 31 + p.window - 1 - it * T);
+      // this thread's key tk sees the query rows qi (t = j0 + qi) with
+      // tk <= t < tk + window and 0 <= t < L: qi in [vlo, vhi] (none when tk
+      // is outside [-P, L))
+      const bool kvalid = tk >= -p.P && tk < p.L;
+      const int vlo = max(tk - j0, -j0), vhi = min(tk - j0 + p.window - 1, p.L - 1 - j0);
       uint32_t pk[2][16], dk[2][16];
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
@@ -585,19 +591,25 @@ __global__ void __launch_bounds__(NT_KV, 1) tc_swa_bwd_kv_kernel(const __grid_co
         float sv[32], dv[32];
         tmem_ld32(tl + C_S + ch * 32, sv);
         tmem_ld32(tl + C_DP + ch * 32, dv);
+        const int qb = it * T + ch * 32;                   // the chunk's first query row within the two tiles
+        const int lo = kvalid ? vlo - qb : 32, hi = vhi - qb;
+        const bool all = lo <= 0 && hi >= 31;              // every query of the chunk sees this key
 #pragma unroll
-        for (int u = 0; u < 32; u += 2) {
-          float pr[2], ds[2];
+        for (int u = 0; u < 32; u += 4) {
+          const float4 l4 = *reinterpret_cast<const float4 *>(&s_lse[qb + u]);
+          const float4 d4 = *reinterpret_cast<const float4 *>(&s_D[qb + u]);
+          const float lq[4] = {l4.x, l4.y, l4.z, l4.w}, dq[4] = {d4.x, d4.y, d4.z, d4.w};
+          float pr[4], ds[4];
 #pragma unroll
-          for (int w = 0; w < 2; ++w) {
-            const int qi = it * T + ch * 32 + u + w;       // query row within the two tiles
-            const int t = j0 + qi;
-            const bool valid = t >= 0 && t < p.L && tk >= -p.P && tk < p.L && t >= tk && t - tk < p.window;
-            pr[w] = valid ? __expf(sv[u + w] * p.scale - s_lse[qi]) : 0.f;
-            ds[w] = pr[w] * (alpha * dv[u + w] - s_D[qi]);
+          for (int w = 0; w < 4; ++w) {
+            pr[w] = __expf(fmaf(sv[u + w], p.scale, -lq[w]));
+            if (!all) pr[w] = (u + w >= lo && u + w <= hi) ? pr[w] : 0.f;
+            ds[w] = pr[w] * (alpha * dv[u + w] - dq[w]);
           }
           pk[k][u / 2] = pack_bf16(pr[0], pr[1]);
+          pk[k][u / 2 + 1] = pack_bf16(pr[2], pr[3]);
           dk[k][u / 2] = pack_bf16(ds[0], ds[1]);
+          dk[k][u / 2 + 1] = pack_bf16(ds[2], ds[3]);
         }
       }
       bar_sync(1, NT_KV);
