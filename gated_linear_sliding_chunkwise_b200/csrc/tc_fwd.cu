@@ -121,9 +121,11 @@ struct Params {
 };
 
 
-__device__ __forceinline__ void issue_tile_loads(const Params &p, unsigned char *sm, uint64_t *bar, int bh,
-                                                 int t0, bool full) {
-  mbar_expect_tx(bar, (full ? 5 : 4) * TILE);
+__device__ __forceinline__ void issue_tile_loads(const Params &p, unsigned char *sm, float *s_rt, uint64_t *bar,
+                                                 int bh, int t0, bool full) {
+  mbar_expect_tx(bar, (full ? 5 : 4) * TILE + (p.gate_r ? D * 4 : 0));
+  if (p.gate_r)   // the tile's log-decays r (one 512-byte row)
+    bulk_load_1d(s_rt, p.gate_r + ((size_t)bh * ((p.L + T - 1) / T) + t0 / T) * D, D * 4, bar);
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
     if (full) {
@@ -324,6 +326,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
   __shared__ int s_fail;
   __shared__ float s_mse[NTHREADS / 32];
   __shared__ __align__(16) float s_row0[D];   // state pass: row 0 of S' (taken out of the copies)
+  __shared__ __align__(16) float s_rt[D];     // the tile's log-decays r (arrive with its loads)
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const int wg = tid >> 7;                             // warpgroup
@@ -357,7 +360,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
     s_fail = 0;
   }
   // the first tile's loads go out before the weights and meta tokens are staged
-  if (tid == 0 && cbeg < cend && !p.inject) issue_tile_loads(p, sm, &bar_tma, bh, cbeg * T, full);
+  if (tid == 0 && cbeg < cend && !p.inject) issue_tile_loads(p, sm, s_rt, &bar_tma, bh, cbeg * T, full);
   // feature-map weights -> bf16, MN-major [dk row][feature]; group 0 W_q, group 1 W_k
   {
     const int i = row;
@@ -447,7 +450,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       //      the meta logits), then one half of phi_q, phi_k per group
       ok &= mbar_wait(&bar_m1, par, err, ST_TIMEOUT);
       tc_fence_after();
-      if (wg == 1 && gla) s_dec[row] = __expf(p.gate_r[((size_t)bh * ntiles_all + c) * D + row]);   // exp(r)
+      if (wg == 1 && gla) s_dec[row] = __expf(s_rt[row]);   // exp(r)
       float lsum = 1.f, mx = 0.f;                 // row normaliser and max (scaled logits)
       // Logit column cl holds key t0 - T + cl.  Row r sees columns
       // [r + T + 1 - window, r + T] (and keys >= -P, P the prefix length),
@@ -578,7 +581,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       // ------ state pass: phi_k half per group, with the fp32 decay factors
       //        (from gate_prep_kernel) that came with the tile's loads ---
       if (wg == 0) {   // thread row = key dimension: the tile's decay
-        const float r = p.gate_r[((size_t)bh * ntiles_all + c) * D + row];
+        const float r = s_rt[row];
         s_dec[row] = __expf(r);
         tot_decay += r;
       }
@@ -708,7 +711,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
     ok = mbar_wait(&bar_m3, par, err, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) { s_fail = 1; break; }
     tc_fence_after();
-    if (tid == 0 && c + 1 < cend) issue_tile_loads(p, sm, &bar_tma, bh, t0 + T, full);
+    if (tid == 0 && c + 1 < cend) issue_tile_loads(p, sm, s_rt, &bar_tma, bh, t0 + T, full);
 
     // ---------------------------- epilogue (column half per group) ---
     if (full) {

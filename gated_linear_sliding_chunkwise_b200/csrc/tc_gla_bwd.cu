@@ -99,6 +99,7 @@ __global__ void __launch_bounds__(NT_DS, 1) tc_gla_dstates_kernel(const __grid_c
   unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
   __shared__ float s_dec[D];
   __shared__ __align__(16) float s_row0[D];   // row 0 of dS, taken out of the bf16 copy
+  __shared__ __align__(16) float s_rt[D];     // the tile's log-decays r (arrive with its loads)
   __shared__ uint64_t bar_tma, bar_m1, bar_m2;
   __shared__ uint32_t s_tmem;
   // Qt (hi) over X_q, the remainder Qt - bf16(Qt) in R_QL, dO, W_q, the
@@ -137,7 +138,8 @@ __global__ void __launch_bounds__(NT_DS, 1) tc_gla_dstates_kernel(const __grid_c
   const uint32_t id_z = idesc_bf16(128, 64, 0, 1);
   const uint32_t id_st = idesc_bf16(128, 128, 1, 1);
   auto loads = [&](int c) {
-    mbar_expect_tx(&bar_tma, 4 * TILE);
+    mbar_expect_tx(&bar_tma, 4 * TILE + D * 4);
+    bulk_load_1d(s_rt, p.gate_r + ((size_t)bh * ntiles + c) * D, D * 4, &bar_tma);
     for (int r = 0; r < 2; ++r) {
       tma_load_3d(sm + R_XQ + r * REG, &p.mq, &bar_tma, 64 * r, c * T, bh);
       tma_load_3d(sm + R_O + r * REG, &p.mo, &bar_tma, 64 * r, c * T, bh);
@@ -182,7 +184,7 @@ __global__ void __launch_bounds__(NT_DS, 1) tc_gla_dstates_kernel(const __grid_c
       if (tid < D) p.snap_r0[tile * D + tid] = s_row0[tid];
     }
     // the tile's decay exp(r)
-    if (wg == 0) s_dec[row] = __expf(p.gate_r[((size_t)bh * ntiles + c) * D + row]);
+    if (wg == 0) s_dec[row] = __expf(s_rt[row]);
     ok = mbar_wait(&bar_m1, par, p.status, ST_TIMEOUT);
     tc_fence_after();
     {   // Qt = phi_q E into shared memory over X_q (row = token), dimension half per group
