@@ -291,7 +291,7 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
   // items, item w = tile w % ntiles of sequence w / ntiles.  The next item's
   // inputs go out as this item frees their places: the weights once the last
   // products are done, V and dO once the dB store has read its staging, X_q
-  // after the dphi stores, X_k and the decay factors after the dv store.
+  // and X_k after the dphi stores, the decay factors after the dv store.
   const int nwork = p.ntiles * p.BH;
   const int w0 = (int)((long long)blockIdx.x * nwork / gridDim.x);
   const int w1 = (int)((long long)(blockIdx.x + 1) * nwork / gridDim.x);
@@ -548,8 +548,8 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
     // 5. rows, dimension half per group, staged as fp32 tiles in the spent
     //    regions and written with TMA stores (rows past L are clipped by the
     //    maps): dB = Qt GQ - Kt GK (Qt, Kt as hi + lo, so that dB matches the
-    //    products) over V | dO; then dphi_q = E GQ (bf16) over Qt lo and
-    //    dphi_k = GK / E over Qt hi; then dv over Kt hi | Kt lo.  E (fp32) is
+    //    products) over V | dO; then dphi_q = E GQ (bf16) over Qt hi and
+    //    dphi_k = GK / E over Kt hi; then dv over Qt lo | Kt lo.  E (fp32) is
     //    read again from global memory, its loads in flight while the last
     //    products run.
     float4 e4[16];
@@ -604,7 +604,7 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
       bulk_commit();
     }
     if (tid < 32) *reinterpret_cast<float4 *>(s_row0 + D + 4 * tid) = ds0;   // read after two barriers
-    // dphi_q - c_q (bf16) over Qt lo, dphi_k - c_k over Qt hi, one 32 KB
+    // dphi_q - c_q (bf16) over Qt hi, dphi_k - c_k over Kt hi, one 32 KB
     // swizzled bf16 tile each, c the half-row's first value: a constant added
     // to one half of a row leaves the feature map's softmax backward
     // unchanged, so the finish pass reads them as they are, and taking out
@@ -637,24 +637,24 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
         gk[4 * u + 2] = __fdividef(gk[4 * u + 2], E.z) - mk;
         gk[4 * u + 3] = __fdividef(gk[4 * u + 3], E.w) - mk;
       }
-      *chunk_ptr(sm, R_QL, row, 2 * c16) = pack8(gq);
-      *chunk_ptr(sm, R_QL, row, 2 * c16 + 1) = pack8(gq + 8);
-      *chunk_ptr(sm, R_XQ, row, 2 * c16) = pack8(gk);
-      *chunk_ptr(sm, R_XQ, row, 2 * c16 + 1) = pack8(gk + 8);
+      *chunk_ptr(sm, R_XQ, row, 2 * c16) = pack8(gq);
+      *chunk_ptr(sm, R_XQ, row, 2 * c16 + 1) = pack8(gq + 8);
+      *chunk_ptr(sm, R_XK, row, 2 * c16) = pack8(gk);
+      *chunk_ptr(sm, R_XK, row, 2 * c16 + 1) = pack8(gk + 8);
     }
     fence_proxy_async();
     __syncthreads();
     if (tid == 0) {
       for (int r = 0; r < 2; ++r) {
-        tma_store_3d(&p.mdq, sm + R_QL + r * REG, 64 * r, t0, bh);
-        tma_store_3d(&p.mdk, sm + R_XQ + r * REG, 64 * r, t0, bh);
+        tma_store_3d(&p.mdq, sm + R_XQ + r * REG, 64 * r, t0, bh);
+        tma_store_3d(&p.mdk, sm + R_XK + r * REG, 64 * r, t0, bh);
       }
       bulk_commit();
     }
-    // dv, staged in the spent Kt hi | Kt lo regions (group wg's two 32-column
+    // dv, staged in the spent Qt lo | Kt lo regions (group wg's two 32-column
     // boxes in one of them), so that it need not wait for the dB store
     const float *md = s_row0 + D;
-    unsigned char *st_dv = sm + (wg == 0 ? R_XK : R_KL);
+    unsigned char *st_dv = sm + (wg == 0 ? R_QL : R_KL);
     float dvv[2][32];
     tmem_ld32x2(tl + C_DV + 64 * wg, tl + C_DV + 64 * wg + 32, dvv[0], dvv[1]);
 #pragma unroll
@@ -672,15 +672,15 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
     __syncthreads();
     if (tid == 0) {
       for (int bx = 0; bx < 4; ++bx)
-        tma_store_3d(&p.mdv, sm + (bx < 2 ? R_XK : R_KL) + (bx & 1) * 16384, 32 * bx, t0, bh);
+        tma_store_3d(&p.mdv, sm + (bx < 2 ? R_QL : R_KL) + (bx & 1) * 16384, 32 * bx, t0, bh);
       bulk_commit();
       if (more) {   // the next item's tiles, each as soon as its place has been read out
         bulk_wait_read_n<2>();   // dB out of V | dO
         item_loads(w + 1, 2);
-        bulk_wait_read_n<1>();   // dphi out of Qt lo | Qt hi
+        bulk_wait_read_n<1>();   // dphi out of Qt hi | Kt hi
         item_loads(w + 1, 1);
-        bulk_wait_read();        // dv out of Kt hi | Kt lo
         item_loads(w + 1, 3);
+        bulk_wait_read();        // dv out of Qt lo | Kt lo
         pend_e = (int)(par ^ 1u);
         e_tma(w + 1);            // over Qt lo | Kt lo, both read out by now
       }
