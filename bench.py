@@ -196,7 +196,13 @@ class ClockSampler:
 # train_step workload (B=8, H=32, L=2048), from an ncu capture of the current
 # kernel build ("step" = the sum over every kernel of one training step).
 # Kernels changed since their capture are left out.
+# DRAM bytes (read + write) per launch from ncu captures of the current
+# kernels on the train_step workload (profiles/train_step_tc_launches.md,
+# profiles/tc_gla_bwd_tile_kernel_train_step.md); "step" sums one training
+# step's 17 launches.
 MEASURED_TRAFFIC = {
+    "step": 8_487_851_776,
+    "tc_gla_bwd_tile_kernel": 1_849_454_848,
 }
 
 
