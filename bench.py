@@ -201,8 +201,6 @@ class ClockSampler:
 # profiles/tc_gla_bwd_tile_kernel_train_step.md); "step" sums one training
 # step's 17 launches.
 MEASURED_TRAFFIC = {
-    "step": 8_487_851_776,
-    "tc_gla_bwd_tile_kernel": 1_849_454_848,
 }
 
 

@@ -149,7 +149,7 @@ bool bwd_gla_uses_tc(const lizard_fwd_args *a, int impl) {
 
 struct BwdLayout {
   size_t phq, phk, a, sprev, dphq, dphk, da, dv_gla, dq_swa, dk_swa, dv_swa, lse, Dterm, dsm, pm, snap_s,
-      snap_ds, e32, gr, w16, kap, total;
+      snap_ds, e32, gr, colsum, w16, kap, total;
   bool fallback;
   FallbackLayout fb;
 };
@@ -180,6 +180,7 @@ BwdLayout bwd_layout(const lizard_fwd_args *a, int impl, bool stage1 = false) {
     l.dv_gla = off; off += nv;
     l.e32 = off; off += nd;      // fp32 decay factors E of every tile
     l.gr = off; off += up(BH * ((a->L + 127) / 128) * a->dk * sizeof(float));   // tiles' log-decays
+    l.colsum = off; off += up(BH * ((a->L + 127) / 128) * a->dk * sizeof(float));   // tiles' column sums of dB
     l.w16 = off; off += up(lz::tc_gla_bwd_weights_bytes(a->H));                  // bf16 W_q, W_k
     l.kap = off; off += up(BH * 2 * a->dk * sizeof(float));   // final-state share of the decay gradient
   } else if (gla_on(a)) {
@@ -397,6 +398,7 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan, bo
                        at<float>(ws, lay.da), at<float>(ws, lay.dv_gla), b->dg, b->dstate_in,
                        status, a->H, BH, a->L, inv_tau, e32, gr, scalar_gate(a), at<void>(ws, lay.w16),
                        b->dstate_out};
+    t.colsum = at<float>(ws, lay.colsum);
     void *w16 = at<void>(ws, lay.w16);
     plan.add("weights_bf16_kernel", [=](cudaStream_t s) { return lz::launch_weights_bf16(a->fmap_wq, a->fmap_wk, w16, a->H, s); });
     plan.add("tc_gla_dstates_kernel", [=](cudaStream_t s) { return lz::launch_tc_gla_bwd(t, 0, s); });
@@ -474,6 +476,7 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan, bo
                       nullptr, at<float>(ws, lay.da), nullptr, b->dg, nullptr, static_cast<uint32_t *>(ws),
                       a->H, BH, a->L, inv_tau, nullptr, nullptr, scalar_gate(a)};
   if (gla_tc && b->dstate_out) tg.kap = at<float>(ws, lay.kap);
+  if (gla_tc) tg.colsum = at<float>(ws, lay.colsum);
   if (fused) {
     // the gate-logit gradient (from dB) beside the feature-map and anchor passes
     plan.fork();

@@ -210,6 +210,7 @@ struct TcGlaBwdArgs {
   const void *w16;              // bf16 [H][2][128][64] feature-map weights (launch_weights_bf16)
   const float *dstate_out;      // [BH][D][D] gradient into the final state, or null (zero)
   const float *kap;             // [BH][2][128] final-state share of the log-decay gradient, or null
+  float *colsum;                // fp32 [B*H][L/128][128]: per-tile column sums of dB (tile kernel out, gate gradient in)
 };
 
 constexpr int kBwdC = 32;   // GLA chunk used by the portable backward

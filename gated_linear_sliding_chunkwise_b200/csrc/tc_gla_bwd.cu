@@ -73,6 +73,7 @@ struct TileParams {
   CUtensorMap me;                             // fp32 decay factors (loads)
   const float *e32;            // fp32 decay factors [BH*L][D]
   const float *sp_r0, *ds_r0;  // [BH*ntiles][D] row 0 of S' and of dS (the copies hold the rest)
+  float *colsum;               // [BH*ntiles][D] column sums of dB per tile (out)
   uint32_t *status;
   int H, L, ntiles, BH;
   float inv_tau;
@@ -604,6 +605,17 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
       bulk_commit();
     }
     if (tid < 32) *reinterpret_cast<float4 *>(s_row0 + D + 4 * tid) = ds0;   // read after two barriers
+    {   // the tile's column sums of dB (the gate gradient's carry from later
+        // tiles): thread = column, half the rows per group, into the free
+        // s_r1[0] | s_r1[2] (read after the next barrier)
+      const int c = tid & 127, b = c >> 5, jj = (c & 31) >> 2;
+      const unsigned char *col = st0 + b * 16384 + (c & 3) * 4;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+      for (int r = 64 * wg; r < 64 * wg + 64; ++r)
+        acc[r & 3] += *reinterpret_cast<const float *>(col + r * 128 + ((jj ^ (r & 7)) << 4));
+      s_r1[2 * wg][c] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    }
     // dphi_q - c_q (bf16) over Qt hi, dphi_k - c_k over Kt hi, one 32 KB
     // swizzled bf16 tile each, c the half-row's first value: a constant added
     // to one half of a row leaves the feature map's softmax backward
@@ -651,6 +663,7 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
       }
       bulk_commit();
     }
+    if (tid < D) p.colsum[(size_t)w * D + tid] = s_r1[0][tid] + s_r1[2][tid];
     // dv, staged in the spent Qt lo | Kt lo regions (group wg's two 32-column
     // boxes in one of them), so that it need not wait for the dB store
     const float *md = s_row0 + D;
@@ -706,50 +719,48 @@ done:
 
 // ------------------------------------------------------- gate gradient ----
 // dg_t = dlogsigmoid(g_t) / tau * sum_{s >= t} dB_s, per (sequence, key
-// dimension).  One CTA per (sequence, 32 dimensions): warp w owns token
-// segment w of 8 (lane = dimension, so each token row is one coalesced
-// 128-byte read); a first pass sums each segment, the later segments' sums
-// give its carry, and a second pass walks it backwards writing dg.
-constexpr int kGateSeg = 8;
+// dimension), in one pass over dB: the tile kernel leaves each tile's column
+// sums of dB, so the part of the sum beyond a tile (plus the final state's
+// share) is known before the tile is walked.  One CTA per (sequence, 32
+// dimensions): warp w walks tiles w, w + 8, ... backwards (lane = dimension,
+// each token row one coalesced 128-byte read, eight rows in flight).
+constexpr int kGateWarps = 8;
 __global__ void __launch_bounds__(256) gate_grad_kernel(const float *dB, const __nv_bfloat16 *g, float *dg, int L,
-                                                       float inv_tau, const float *kap) {
-  __shared__ float s_tot[kGateSeg][32];
+                                                       float inv_tau, const float *kap, const float *colsum) {
   const int bh = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int i = blockIdx.y * 32 + lane;
-  const int seg = (L + kGateSeg - 1) / kGateSeg;
-  const int ta = min(L, warp * seg), tz = min(L, ta + seg);   // this warp's tokens [ta, tz)
+  const int ntiles = (L + T - 1) / T;
   const size_t base = (size_t)bh * L * D + i;
-  float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  int t = ta;
-  for (; t + 8 <= tz; t += 8) {
-#pragma unroll
-    for (int u = 0; u < 8; ++u) part[u] += dB[base + (size_t)(t + u) * D];
-  }
-  for (; t < tz; ++t) part[0] += dB[base + (size_t)t * D];
-  s_tot[warp][lane] = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
-  __syncthreads();
+  const float *cs = colsum + (size_t)bh * ntiles * D + i;
   // the sum starts with the final state's share (an incoming final-state gradient)
-  float carry = kap ? kap[(size_t)bh * 2 * D + i] + kap[((size_t)bh * 2 + 1) * D + i] : 0.f;
-  for (int w = warp + 1; w < kGateSeg; ++w) carry += s_tot[w][lane];
-  t = tz - 1;
-  for (; t - 7 >= ta; t -= 8) {
-    float b[8], gv[8];
+  const float k0 = kap ? kap[(size_t)bh * 2 * D + i] + kap[((size_t)bh * 2 + 1) * D + i] : 0.f;
+  for (int c = warp; c < ntiles; c += kGateWarps) {
+    float later[4] = {k0, 0.f, 0.f, 0.f};
+    for (int c2 = c + 1; c2 < ntiles; ++c2) later[c2 & 3] += cs[(size_t)c2 * D];
+    float carry = (later[0] + later[1]) + (later[2] + later[3]);
+    const int ta = c * T, tz = min(L, ta + T);
+    int t = tz - 1;
+    for (; t - 7 >= ta; t -= 8) {
+      float b[8], gv[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      b[u] = dB[base + (size_t)(t - u) * D];
-      gv[u] = __bfloat162float(g[base + (size_t)(t - u) * D]);
-    }
+      for (int u = 0; u < 8; ++u) {
+        b[u] = dB[base + (size_t)(t - u) * D];
+        gv[u] = __bfloat162float(g[base + (size_t)(t - u) * D]);
+      }
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      carry += b[u];
-      dg[base + (size_t)(t - u) * D] = carry * dlogsigmoid(gv[u]) * inv_tau;
+      for (int u = 0; u < 8; ++u) {
+        carry += b[u];
+        dg[base + (size_t)(t - u) * D] = carry * dlogsigmoid(gv[u]) * inv_tau;
+      }
     }
-  }
-  for (; t >= ta; --t) {
-    carry += dB[base + (size_t)t * D];
-    dg[base + (size_t)t * D] = carry * dlogsigmoid(__bfloat162float(g[base + (size_t)t * D])) * inv_tau;
+    for (; t >= ta; --t) {
+      carry += dB[base + (size_t)t * D];
+      dg[base + (size_t)t * D] = carry * dlogsigmoid(__bfloat162float(g[base + (size_t)t * D])) * inv_tau;
+    }
   }
 }
+
+constexpr int kGateSeg = 8;   // token segments (one per warp) of the scalar-gate kernel
 
 // Scalar gate (one logit per token and head, shared by every key dimension):
 // dg_t = dlogsigmoid(g_t) / tau * sum_{s >= t} sum_i dB_s[i].  One CTA per
@@ -889,6 +900,7 @@ cudaError_t launch_tc_gla_bwd(const TcGlaBwdArgs &a, int stage, cudaStream_t s) 
         !make_map_f32_3d(&p.mdb, a.dB, D, rows, a.BH, T) || !make_map_f32_3d(&p.mdv, a.dv, D, rows, a.BH, T) ||
         !make_map_f32_3d(&p.me, a.e32, D, rows, a.BH, T))
       return cudaErrorInvalidValue;
+    p.colsum = a.colsum;
     p.e32 = a.e32;
     p.sp_r0 = snapshot_row0(a.snap_s, a.BH, a.L);
     p.ds_r0 = snapshot_row0(a.snap_ds, a.BH, a.L);
@@ -915,7 +927,7 @@ cudaError_t launch_tc_gla_bwd(const TcGlaBwdArgs &a, int stage, cudaStream_t s) 
                                                  a.inv_tau, a.kap);
   else
     gate_grad_kernel<<<dim3(a.BH, D / 32), 256, 0, s>>>(a.dB, static_cast<const __nv_bfloat16 *>(a.g), a.dg, a.L,
-                                                        a.inv_tau, a.kap);
+                                                        a.inv_tau, a.kap, a.colsum);
   return cudaGetLastError();
 }
 
