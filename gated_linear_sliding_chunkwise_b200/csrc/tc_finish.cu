@@ -30,6 +30,7 @@ constexpr uint32_t ST_TIMEOUT = 1u;
 struct Params {
   CUtensorMap mq, mk;
   CUtensorMap mxq, mxk;                    // bf16 dx_q, dx_k parts (fused mode)
+  CUtensorMap mphq, mphk;                  // bf16 dphi_q, dphi_k (TMA loads)
   const float *wq, *wk;
   // GLA parts, null when the branch is off: dphi_q, dphi_k in bf16 with each
   // row's halves centred (the softmax backward below ignores a constant added
@@ -54,7 +55,7 @@ constexpr int NTHREADS = 256;
 __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_constant__ Params p) {
   extern __shared__ unsigned char smraw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
-  __shared__ uint64_t bar_tma, bar_z, bar_d;
+  __shared__ uint64_t bar_tma, bar_z, bar_d, bar_ph;
   __shared__ uint32_t s_tmem;
   // X_q, X_k, W_q | W_k (64-column tiles), dZ_q | dZ_k (64-column tiles)
   constexpr uint32_t R_XQ = 0, R_XK = TILE, R_WQ = 2 * TILE, R_WK = 2 * TILE + REG, R_ZQ = 3 * TILE,
@@ -71,6 +72,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
     mbar_init(&bar_tma, 1);
     mbar_init(&bar_z, 1);
     mbar_init(&bar_d, 1);
+    mbar_init(&bar_ph, 1);
     fence_barrier_init();
   }
   const int ntiles = (p.L + T - 1) / T;
@@ -103,12 +105,24 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
   const uint32_t id_dx = idesc_bf16(128, 128, 0, 0);   // dZ (K-major) x W^T (K-major, N = 128)
   const uint32_t id_dw = idesc_bf16(128, 64, 1, 1);    // X^T (MN-major) x dZ (MN-major, N = 64)
   bool fail = false;
-  // this row's dphi values (its group's half) of one map, loaded ahead: map 0
-  // of the next tile at the end of this one, map 1 while map 0 is used.
-  // They stay packed (bf16) until used, so that the loads are still in flight
-  // when the call returns.
+  // this row's dphi values (its group's half) of one map, packed bf16.  They
+  // come by TMA into R_STG (dphi_q over its first half, dphi_k over its
+  // second, from the end of the previous tile; the exchange of each map's
+  // half-terms reuses the map's half once every row has read it), except for
+  // a sequence of the exact fallback, whose fp32 values are loaded into
+  // registers ahead (map 0 of the next tile at the end of this one, map 1
+  // while map 0 is used) and centred there.
   uint4 dpre[8];
   const int fb_slot = (gla && p.slot_of) ? p.slot_of[bh] : -1;
+  const bool ph_tma = gla && fb_slot < 0;
+  int pend_ph = -1;   // tid 0: the parity of a dphi load in flight
+  auto ph_loads = [&](int c) {
+    mbar_expect_tx(&bar_ph, 2 * TILE);
+    for (int r = 0; r < 2; ++r) {
+      tma_load_3d(sm + R_STG + r * REG, &p.mphq, &bar_ph, 64 * r, c * T, bh);
+      tma_load_3d(sm + R_STG + TILE + r * REG, &p.mphk, &bar_ph, 64 * r, c * T, bh);
+    }
+  };
   auto dphi_load = [&](int m, int c) {
     const int t = c * T + row;
     if (fb_slot >= 0) {
@@ -131,7 +145,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
     for (int u = 0; u < 8; ++u)
       dpre[u] = t < p.L ? *reinterpret_cast<const uint4 *>(src + 8 * u) : make_uint4(0u, 0u, 0u, 0u);
   };
-  if (gla && ntiles > 0) dphi_load(0, 0);
+  if (ph_tma && ntiles > 0) {
+    if (tid == 0) {
+      pend_ph = 0;
+      ph_loads(0);
+    }
+  } else if (gla && ntiles > 0) {
+    dphi_load(0, 0);
+  }
   for (int c = 0; c < ntiles; ++c) {
     const uint32_t par = c & 1;
     const int tq = c * T + row;
@@ -147,7 +168,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
         mma_commit(&bar_z);
       }
       ok = mbar_wait(&bar_z, par, p.status, ST_TIMEOUT);
+      if (ph_tma) ok &= mbar_wait(&bar_ph, par, p.status, ST_TIMEOUT);
       if (__syncthreads_or(!ok)) { fail = true; break; }
+      if (tid == 0) pend_ph = -1;
       tc_fence_after();
       // dz of both maps, one map at a time (fp32 math, bf16 dZ tiles): group
       // 0 owns the softmax(z) half (p, dp), group 1 the softmax(-z) half
@@ -158,6 +181,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
       // f < 32, group 1 for f >= 32.
 #pragma unroll 1
       for (int m = 0; m < 2; ++m) {
+        if (ph_tma)
+#pragma unroll
+          for (int u = 0; u < 8; ++u) dpre[u] = *chunk_ptr(sm, R_STG + m * TILE, row, 8 * wg + u);
         float ph[F];
         const float sc = feature_half(tl + (m == 0 ? C_ZQ : C_ZK), wg, ph);
         float dot4[4] = {0.f, 0.f, 0.f, 0.f};
@@ -179,7 +205,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
 #pragma unroll
           for (int i = 0; i < 8; ++i) ph[8 * u + i] *= d[i] - dot;
         }
-        if (m == 0) dphi_load(1, c);   // the k map's values, in flight while this map finishes
+        if (!ph_tma && m == 0) dphi_load(1, c);   // the k map's values, in flight while this map finishes
+        if (ph_tma) bar_sync(2, NTHREADS);   // every row has read this map's dphi: its half takes the exchange
         // send the half-terms of the other group's features
         unsigned char *mine = sm + R_STG + (2 * m + wg) * 16384;
         const unsigned char *theirs = sm + R_STG + (2 * m + 1 - wg) * 16384;
@@ -288,9 +315,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
     }
     // the next tile's q-map values, in flight until they are used (issued
     // past this tile's proxy fences, which would wait for them)
-    if (gla && c + 1 < ntiles) dphi_load(0, c + 1);
+    if (!ph_tma && gla && c + 1 < ntiles) dphi_load(0, c + 1);
     tc_fence_before();
     __syncthreads();
+    if (ph_tma && tid == 0 && c + 1 < ntiles) {   // R_STG is read out: the next tile's dphi
+      pend_ph = (int)((c + 1) & 1);
+      ph_loads(c + 1);
+    }
   }
   if (gla && !fail) {
     tc_fence_after();
@@ -305,6 +336,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
       }
     }
   }
+  if (tid == 0 && pend_ph >= 0) mbar_wait(&bar_ph, (uint32_t)pend_ph, nullptr, 0, 1u << 16);   // after a failed wait
   if (p.fused && tid == 0) bulk_wait_all();
   tc_fence_before();
   __syncthreads();
@@ -329,6 +361,9 @@ cudaError_t launch_tc_finish(const FinishBwdArgs &a, int BH, cudaStream_t s) {
   p.wk = a.wk;
   p.dphq = static_cast<const __nv_bfloat16 *>(a.dphq16);
   p.dphk = static_cast<const __nv_bfloat16 *>(a.dphk16);
+  if (p.dphq && (!make_map_bf16_3d(&p.mphq, a.dphq16, D, rows, BH, T) ||
+                 !make_map_bf16_3d(&p.mphk, a.dphk16, D, rows, BH, T)))
+    return cudaErrorInvalidValue;
   p.dv_gla = a.dv_gla;
   p.slot_of = a.slot_of;
   p.fb_dphq = a.fb_dphq;
