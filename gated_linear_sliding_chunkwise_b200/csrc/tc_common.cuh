@@ -373,6 +373,79 @@ __device__ __forceinline__ float log_decay_fast(float g, float inv_tau) {
   return (fminf(g, 0.f) - __logf(1.f + __expf(-fabsf(g)))) * inv_tau;
 }
 
+// ------------------------------------- small row dots on mma.sync ------
+// Dot products of the 32 rows of one warp (rows row0 .. row0 + 31 of a
+// 128-row tile of 128 bf16 columns, K-major and 128-byte swizzled at
+// sm + region) with up to 16 fp32 vectors W[m][0 .. 127] (m < M): the meta
+// tokens' logits and value products, which are too narrow for a tcgen05 tile
+// and too long for the CUDA cores.  Warp-level mma.sync m16n8k16 (bf16 in,
+// fp32 accumulate) with W split into bf16 hi + lo, so the result carries
+// fp32-level precision in W; A fragments come from the swizzled tile by
+// ldmatrix.  Writes out[m][row] for the warp's rows and m < M (a warp-local
+// result: __syncwarp() before another lane reads it).
+__device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t *>(&v);
+}
+__device__ __forceinline__ void rowdots_mma(const unsigned char *sm, uint32_t region, int row0, const float (*W)[128],
+                                            int M, float (*out)[128], int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  for (int n0 = 0; n0 < M; n0 += 8) {          // eight vectors per pass
+    float acc[2][4];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[mt][j] = 0.f;
+    const int n = n0 + g;                      // this lane's B column
+#pragma unroll 2
+    for (int ks = 0; ks < 8; ++ks) {           // 16 columns per step
+      // B = W^T (k x n, "col" layout): b0 holds k = 2t, 2t + 1, b1 k = 2t + 8, 2t + 9
+      uint32_t bh[2], bl[2];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        float w0 = 0.f, w1 = 0.f;
+        if (n < M) {
+          const float2 w = *reinterpret_cast<const float2 *>(&W[n][16 * ks + 2 * t + 8 * hh]);
+          w0 = w.x;
+          w1 = w.y;
+        }
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(w0, w1);
+        const float2 hf = __bfloat1622float2(hi);
+        bh[hh] = *reinterpret_cast<const uint32_t *>(&hi);
+        bl[hh] = pack_bf16x2_rn(w0 - hf.x, w1 - hf.y);
+      }
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        // A: rows row0 + 16 mt .. + 15, columns 16 ks .. + 15 as four 8 x 8 matrices
+        const int r = row0 + 16 * mt + (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int c = 2 * ks + (lane >> 4);    // 16-byte chunk (8 columns)
+        const uint32_t addr = smem_u32(sm + region + (c >> 3) * kReg + sw128_offset(r, (c & 7) * 8));
+        uint32_t a0, a1, a2, a3;
+        asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];\n"
+                     : "=r"(a0), "=r"(a1), "=r"(a2), "=r"(a3)
+                     : "r"(addr));
+#pragma unroll
+        for (int hl = 0; hl < 2; ++hl) {
+          const uint32_t b0 = hl ? bl[0] : bh[0], b1 = hl ? bl[1] : bh[1];
+          asm volatile(
+              "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+              "{%0, %1, %2, %3};\n"
+              : "+f"(acc[mt][0]), "+f"(acc[mt][1]), "+f"(acc[mt][2]), "+f"(acc[mt][3])
+              : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+        }
+      }
+    }
+    // C: acc[mt][0..1] row g, columns 2t, 2t + 1; acc[mt][2..3] row g + 8
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int m = n0 + 2 * t + (j & 1), rr = row0 + 16 * mt + g + 8 * (j >> 1);
+        if (m < M) out[m][rr] = acc[mt][j];
+      }
+  }
+}
+
 // One half of the feature map of this thread's row, from the 64
 // projections z in TMEM: half 0 is softmax(z), half 1 is softmax(-z).  ph
 // gets the unnormalised terms exp(+-z_f - max); the result is 1 / their sum.

@@ -467,29 +467,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       uint32_t pk[3][16];
       if (swa) {
         float pmax = kNegBig;
-        if (wg == 0) {
-          // meta logits q . mk_m (scaled) into s_ml, four meta tokens per pass
-          for (int m0 = 0; m0 < p.M; m0 += 4) {
-            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-            for (int ch = 0; ch < 16; ++ch) {
-              float q8[8];
-              unpack8(*chunk_ptr(sm, R_XQ, row, ch), q8);
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const float4 a = *reinterpret_cast<const float4 *>(&s_mk[m0 + k][ch * 8]);
-                const float4 b = *reinterpret_cast<const float4 *>(&s_mk[m0 + k][ch * 8 + 4]);
-                acc[2 * k] = fmaf(q8[0], a.x, fmaf(q8[1], a.y, fmaf(q8[2], a.z, fmaf(q8[3], a.w, acc[2 * k]))));
-                acc[2 * k + 1] = fmaf(q8[4], b.x, fmaf(q8[5], b.y, fmaf(q8[6], b.z, fmaf(q8[7], b.w, acc[2 * k + 1]))));
-              }
-            }
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              if (m0 + k < p.M) {
-                const float l = (acc[2 * k] + acc[2 * k + 1]) * p.scale;
-                s_ml[m0 + k][row] = l;
-                pmax = fmaxf(pmax, l);
-              }
+        if (wg == 0 && p.M > 0) {
+          // meta logits q . mk_m (scaled) into s_ml: this warp's 32 rows by mma.sync
+          rowdots_mma(sm, R_XQ, 32 * w4, s_mk, p.M, s_ml, threadIdx.x & 31);
+          __syncwarp();
+          for (int m = 0; m < p.M; ++m) {
+            const float l = s_ml[m][row] * p.scale;
+            s_ml[m][row] = l;
+            pmax = fmaxf(pmax, l);
           }
         }
         for (int ch = ch_first; ch <= ch_hi; ch += 2) {

@@ -179,39 +179,23 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
     mma_commit(bar_m);
   }
   {
-    // meta dot products on the CUDA cores while the MMAs run: group 0
-    // q . mk_m (kept in registers), group 1 dO . mv_m (to shared memory);
-    // four meta tokens per pass, passes beyond M skipped
+    // meta dot products while the MMAs run, by mma.sync over each warp's 32
+    // rows: group 0 q . mk_m (through s_x into registers), then group 1
+    // dO . mv_m (into s_x, read after the barrier below)
     float ml[MAXM], em[MAXM], dom[MAXM];
 #pragma unroll
     for (int m = 0; m < MAXM; ++m) { ml[m] = 0.f; em[m] = 0.f; dom[m] = 0.f; }
-    {
-      const uint32_t reg = wg == 0 ? R_Q : R_O;
-      const float(*W)[D] = wg == 0 ? s_mk : s_mv;
-#pragma unroll
-      for (int g = 0; g < MAXM / 4; ++g) {
-        if (4 * g < p.M) {
-          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-          for (int ch = 0; ch < 16; ++ch) {
-            float x8[8];
-            unpack8(*chunk_ptr(sm, reg, row, ch), x8);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const float4 a = *reinterpret_cast<const float4 *>(&W[4 * g + k][ch * 8]);
-              const float4 b = *reinterpret_cast<const float4 *>(&W[4 * g + k][ch * 8 + 4]);
-              acc[2 * k] = fmaf(x8[0], a.x, fmaf(x8[1], a.y, fmaf(x8[2], a.z, fmaf(x8[3], a.w, acc[2 * k]))));
-              acc[2 * k + 1] = fmaf(x8[4], b.x, fmaf(x8[5], b.y, fmaf(x8[6], b.z, fmaf(x8[7], b.w, acc[2 * k + 1]))));
-            }
-          }
-#pragma unroll
-          for (int k = 0; k < 4; ++k) ml[4 * g + k] = acc[2 * k] + acc[2 * k + 1];
-        }
-      }
-      if (wg == 1)
+    if (p.M > 0) {
+      const int wrow = 32 * (warp & 3);
+      if (wg == 0) {
+        rowdots_mma(sm, R_Q, wrow, s_mk, p.M, s_x, lane);
+        __syncwarp();
 #pragma unroll
         for (int m = 0; m < MAXM; ++m)
-          if (m < p.M) s_x[m][row] = ml[m];
+          if (m < p.M) ml[m] = s_x[m][row];
+      }
+      bar_sync(3, NT_Q);   // group 0 has read its logits out of s_x
+      if (wg == 1) rowdots_mma(sm, R_O, wrow, s_mv, p.M, s_x, lane);
     }
     ok = mbar_wait(bar_m, par, p.status, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) goto done;
