@@ -382,15 +382,20 @@ __device__ __forceinline__ float log_decay_fast(float g, float inv_tau) {
 // fp32 accumulate) with W split into bf16 hi + lo, so the result carries
 // fp32-level precision in W; A fragments come from the swizzled tile by
 // ldmatrix.  Writes out[m][row] for the warp's rows and m < M (a warp-local
-// result: __syncwarp() before another lane reads it).
+// result: __syncwarp() before another lane reads it).  M <= 16.
 __device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t *>(&v);
 }
+// OWN: instead of out, every lane gets its own row's (row0 + lane) products in
+// own[m] (gathered from the accumulator fragments by warp shuffles).
+template <bool OWN = false>
 __device__ __forceinline__ void rowdots_mma(const unsigned char *sm, uint32_t region, int row0, const float (*W)[128],
-                                            int M, float (*out)[128], int lane) {
+                                            int M, float (*out)[128], int lane, float *own = nullptr) {
   const int g = lane >> 2, t = lane & 3;
-  for (int n0 = 0; n0 < M; n0 += 8) {          // eight vectors per pass
+#pragma unroll
+  for (int n0 = 0; n0 < 16; n0 += 8) {         // eight vectors per pass
+    if (n0 >= M) break;
     float acc[2][4];
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt)
@@ -436,13 +441,27 @@ __device__ __forceinline__ void rowdots_mma(const unsigned char *sm, uint32_t re
       }
     }
     // C: acc[mt][0..1] row g, columns 2t, 2t + 1; acc[mt][2..3] row g + 8
+    if (OWN) {
+      // row r = lane of this warp: fragment mt = r / 16, half = (r / 8) % 2, held by lane 4 (r % 8) + (m - n0) / 2
+      const int mt = lane >> 4, half = (lane >> 3) & 1;
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int m = n0 + 2 * t + (j & 1), rr = row0 + 16 * mt + g + 8 * (j >> 1);
-        if (m < M) out[m][rr] = acc[mt][j];
+      for (int mm = 0; mm < 8; ++mm) {
+        const int src = 4 * (lane & 7) + (mm >> 1);
+        const float v00 = __shfl_sync(0xffffffffu, acc[0][mm & 1], src);
+        const float v01 = __shfl_sync(0xffffffffu, acc[0][2 + (mm & 1)], src);
+        const float v10 = __shfl_sync(0xffffffffu, acc[1][mm & 1], src);
+        const float v11 = __shfl_sync(0xffffffffu, acc[1][2 + (mm & 1)], src);
+        own[n0 + mm] = mt == 0 ? (half == 0 ? v00 : v01) : (half == 0 ? v10 : v11);
       }
+    } else {
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int m = n0 + 2 * t + (j & 1), rr = row0 + 16 * mt + g + 8 * (j >> 1);
+          if (m < M) out[m][rr] = acc[mt][j];
+        }
+    }
   }
 }
 

@@ -180,22 +180,17 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
   }
   {
     // meta dot products while the MMAs run, by mma.sync over each warp's 32
-    // rows: group 0 q . mk_m (through s_x into registers), then group 1
-    // dO . mv_m (into s_x, read after the barrier below)
+    // rows, every lane getting its own row's: group 0 q . mk_m (kept in
+    // registers), group 1 dO . mv_m (to shared memory)
     float ml[MAXM], em[MAXM], dom[MAXM];
 #pragma unroll
     for (int m = 0; m < MAXM; ++m) { ml[m] = 0.f; em[m] = 0.f; dom[m] = 0.f; }
     if (p.M > 0) {
-      const int wrow = 32 * (warp & 3);
-      if (wg == 0) {
-        rowdots_mma(sm, R_Q, wrow, s_mk, p.M, s_x, lane);
-        __syncwarp();
+      rowdots_mma<true>(sm, wg == 0 ? R_Q : R_O, 32 * (warp & 3), wg == 0 ? s_mk : s_mv, p.M, nullptr, lane, ml);
+      if (wg == 1)
 #pragma unroll
         for (int m = 0; m < MAXM; ++m)
-          if (m < p.M) ml[m] = s_x[m][row];
-      }
-      bar_sync(3, NT_Q);   // group 0 has read its logits out of s_x
-      if (wg == 1) rowdots_mma(sm, R_O, wrow, s_mv, p.M, s_x, lane);
+          if (m < p.M) s_x[m][row] = ml[m];
     }
     ok = mbar_wait(bar_m, par, p.status, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) goto done;
