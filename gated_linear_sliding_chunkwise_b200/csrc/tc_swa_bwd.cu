@@ -212,8 +212,9 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
     }
 
     // 2. softmax over the band (see the forward): logit column cl holds key
-    //    t0 - T + cl; warp w4 visits chunks ch_lo .. ch_hi, group wg the
-    //    chunks ch_lo + wg, ch_lo + wg + 2, ...
+    //    t0 - T + cl; warp w4 visits chunks ch_lo .. ch_hi, group 1 the
+    //    chunks ch_lo, ch_lo + 2, ... and group 0 (which also has the meta
+    //    terms) the others
     //    (keys >= -P, P the prefix length)
     const int w4 = warp & 3, cbase = t0 - T;
     const int lo_c = max(tq - p.window + 1, -p.P) - cbase, hi_c = tq - cbase;
@@ -221,7 +222,7 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
     if (cbase < 0) ch_lo = max(ch_lo, (T - p.P) >> 5);
     const int ch_hi = w4 + 4;
     const int in_lo = 32 * w4 + 31 + T + 1 - p.window;
-    for (int ch = ch_lo + wg; ch <= ch_hi; ch += 2) {
+    for (int ch = ch_lo + 1 - wg; ch <= ch_hi; ch += 2) {
       float v[32];
       tmem_ld32(tl + C_L + ch * 32, v);
       float m4[4] = {kNegBig, kNegBig, kNegBig, kNegBig};
@@ -249,7 +250,7 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
     float s4[4] = {0.f, 0.f, 0.f, 0.f}, d4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int k = 0; k < 3; ++k) {
-      const int ch = ch_lo + wg + 2 * k;
+      const int ch = ch_lo + 1 - wg + 2 * k;
       if (ch > ch_hi) continue;
       float v[32], dp[32];
       tmem_ld32(tl + C_L + ch * 32, v);
@@ -287,7 +288,7 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
     const float inv_l = 1.f / lsum;
 #pragma unroll
     for (int k = 0; k < 3; ++k) {
-      const int ch = ch_lo + wg + 2 * k;
+      const int ch = ch_lo + 1 - wg + 2 * k;
       if (ch > ch_hi) continue;
       tmem_st8(tl + C_P + ch * 16, pk[k]);
       tmem_st8(tl + C_P + ch * 16 + 8, pk[k] + 8);
