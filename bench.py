@@ -201,6 +201,8 @@ class ClockSampler:
 # profiles/tc_gla_bwd_tile_kernel_train_step.md); "step" sums one training
 # step's 17 launches.
 MEASURED_TRAFFIC = {
+    "step": 8_281_418_496,
+    "tc_gla_bwd_tile_kernel": 1_852_018_912,
 }
 
 
