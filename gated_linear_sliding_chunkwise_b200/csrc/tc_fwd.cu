@@ -464,7 +464,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       const int ch_hi = w4 + 4;
       const int in_lo = 32 * w4 + 31 + T + 1 - p.window;   // interior chunk: 32 ch >= in_lo
       const int ch_first = ch_lo + 1 - wg;                 // this group's first chunk
-      uint32_t pk[3][16];
+      // The band's chunks alternate between the groups (group 1 from ch_lo);
+      // an odd count's last chunk is halved: group 1 takes its first 16
+      // columns, group 0 (which also has the meta logits) the other 16.
+      const bool split = ((ch_hi - ch_lo) & 1) == 0;
+      const int full_hi = split ? ch_hi - 1 : ch_hi;       // last chunk taken whole
+      const int hcol = 32 * ch_hi + 16 * (1 - wg);          // this group's half of a split chunk
+      const bool hinner = hcol >= in_lo && hcol + 15 <= 32 * w4 + T && hcol + cbase >= -p.P;
+      uint32_t pk[2][16], pkh[8];
       if (swa) {
         float pmax = kNegBig;
         if (wg == 0 && p.M > 0) {
@@ -477,7 +484,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
             pmax = fmaxf(pmax, l);
           }
         }
-        for (int ch = ch_first; ch <= ch_hi; ch += 2) {
+        if (split) {
+          float v[16];
+          tmem_ld16(tl + C_L + hcol, v);
+          float m4[4] = {kNegBig, kNegBig, kNegBig, kNegBig};
+#pragma unroll
+          for (int u = 0; u < 16; ++u)
+            if (hinner || (hcol + u >= lo_c && hcol + u <= hi_c)) m4[u & 3] = fmaxf(m4[u & 3], v[u]);
+          const float cm = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+          if (cm > kNegBig) pmax = fmaxf(pmax, cm * p.scale);
+        }
+        for (int ch = ch_first; ch <= full_hi; ch += 2) {
           float v[32];
           tmem_ld32(tl + C_L + ch * 32, v);
           float m4[4] = {kNegBig, kNegBig, kNegBig, kNegBig};
@@ -502,10 +519,26 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         // P^ = exp(l - max), packed and held until both groups have read
         // their logits (P^ column 16 ch overlays logit chunk ch / 2)
         float s4[4] = {0.f, 0.f, 0.f, 0.f};
+        if (split) {
+          float v[16];
+          tmem_ld16(tl + C_L + hcol, v);
 #pragma unroll
-        for (int k = 0; k < 3; ++k) {
+          for (int u = 0; u < 16; u += 2) {
+            float e0 = __expf(fmaf(v[u], p.scale, -mx));
+            float e1 = __expf(fmaf(v[u + 1], p.scale, -mx));
+            if (!hinner) {
+              const int cl = hcol + u;
+              e0 = (cl >= lo_c && cl <= hi_c) ? e0 : 0.f;
+              e1 = (cl + 1 >= lo_c && cl + 1 <= hi_c) ? e1 : 0.f;
+            }
+            s4[(u >> 1) & 3] += e0 + e1;
+            pkh[u / 2] = alpha != 0.f ? pack_bf16(e0, e1) : 0u;
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
           const int ch = ch_first + 2 * k;
-          if (ch > ch_hi) continue;
+          if (ch > full_hi) continue;
           float v[32];
           tmem_ld32(tl + C_L + ch * 32, v);
           const bool inner = 32 * ch >= in_lo && 32 * ch + 31 <= 32 * w4 + T && 32 * ch + cbase >= -p.P;
@@ -536,12 +569,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         lsum = s_psum[0][row] + s_psum[1][row];
         if (!qvalid) lsum = 1.f;
 #pragma unroll
-        for (int k = 0; k < 3; ++k) {
+        for (int k = 0; k < 2; ++k) {
           const int ch = ch_first + 2 * k;
-          if (ch > ch_hi) continue;
+          if (ch > full_hi) continue;
           tmem_st8(tl + C_P + ch * 16, pk[k]);
           tmem_st8(tl + C_P + ch * 16 + 8, pk[k] + 8);
         }
+        if (split) tmem_st8(tl + C_P + ch_hi * 16 + 8 * (1 - wg), pkh);
         uint32_t zero[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
         for (int ch = wg; ch < 8; ch += 2) {   // chunks outside the band: P = 0
           if (ch >= ch_lo && ch <= ch_hi) continue;
