@@ -222,7 +222,23 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
     if (cbase < 0) ch_lo = max(ch_lo, (T - p.P) >> 5);
     const int ch_hi = w4 + 4;
     const int in_lo = 32 * w4 + 31 + T + 1 - p.window;
-    for (int ch = ch_lo + 1 - wg; ch <= ch_hi; ch += 2) {
+    // an odd band's last chunk is halved: group 1 its first 16 columns,
+    // group 0 the other 16 (as in the forward)
+    const bool split = ((ch_hi - ch_lo) & 1) == 0;
+    const int full_hi = split ? ch_hi - 1 : ch_hi;
+    const int hcol = 32 * ch_hi + 16 * (1 - wg);
+    const bool hinner = hcol >= in_lo && hcol + 15 <= 32 * w4 + T && hcol + cbase >= -p.P;
+    if (split) {
+      float v[16];
+      tmem_ld16(tl + C_L + hcol, v);
+      float m4[4] = {kNegBig, kNegBig, kNegBig, kNegBig};
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+        if (hinner || (hcol + u >= lo_c && hcol + u <= hi_c)) m4[u & 3] = fmaxf(m4[u & 3], v[u]);
+      const float cm = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      if (cm > kNegBig) mx = fmaxf(mx, cm * p.scale);
+    }
+    for (int ch = ch_lo + 1 - wg; ch <= full_hi; ch += 2) {
       float v[32];
       tmem_ld32(tl + C_L + ch * 32, v);
       float m4[4] = {kNegBig, kNegBig, kNegBig, kNegBig};
@@ -246,12 +262,30 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
     //    both groups have read their logits (P^ overlays logit chunks 0 .. 3)
     //    and, for D = dO_swa . o_swa = alpha (sum_j P^_j dP'_j + sum_m e_m
     //    dO . mv_m) / l, the sums of P^ dP' over the same chunks
-    uint32_t pk[3][16];
+    uint32_t pk[2][16], pkh[8];
     float s4[4] = {0.f, 0.f, 0.f, 0.f}, d4[4] = {0.f, 0.f, 0.f, 0.f};
+    if (split) {
+      float v[16], dp[16];
+      tmem_ld16(tl + C_L + hcol, v);
+      tmem_ld16(tl + C_DP + hcol, dp);
 #pragma unroll
-    for (int k = 0; k < 3; ++k) {
+      for (int u = 0; u < 16; u += 2) {
+        float e0 = __expf(fmaf(v[u], p.scale, -mx));
+        float e1 = __expf(fmaf(v[u + 1], p.scale, -mx));
+        if (!hinner) {
+          const int cl = hcol + u;
+          e0 = (cl >= lo_c && cl <= hi_c) ? e0 : 0.f;
+          e1 = (cl + 1 >= lo_c && cl + 1 <= hi_c) ? e1 : 0.f;
+        }
+        s4[(u >> 1) & 3] += e0 + e1;
+        d4[(u >> 1) & 3] = fmaf(e0, dp[u], fmaf(e1, dp[u + 1], d4[(u >> 1) & 3]));
+        pkh[u / 2] = pack_bf16(e0, e1);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
       const int ch = ch_lo + 1 - wg + 2 * k;
-      if (ch > ch_hi) continue;
+      if (ch > full_hi) continue;
       float v[32], dp[32];
       tmem_ld32(tl + C_L + ch * 32, v);
       tmem_ld32(tl + C_DP + ch * 32, dp);
@@ -287,12 +321,13 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
     const float lsum = s_psum[0][row] + s_psum[1][row];
     const float inv_l = 1.f / lsum;
 #pragma unroll
-    for (int k = 0; k < 3; ++k) {
+    for (int k = 0; k < 2; ++k) {
       const int ch = ch_lo + 1 - wg + 2 * k;
-      if (ch > ch_hi) continue;
+      if (ch > full_hi) continue;
       tmem_st8(tl + C_P + ch * 16, pk[k]);
       tmem_st8(tl + C_P + ch * 16 + 8, pk[k] + 8);
     }
+    if (split) tmem_st8(tl + C_P + ch_hi * 16 + 8 * (1 - wg), pkh);
     {
       uint32_t zero[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
       for (int ch = wg; ch < 8; ch += 2) {
