@@ -70,11 +70,12 @@ def tc_segments(BH, L, T=128):
     return math.ceil(nt / tps)
 
 
-def kernel_model(name, w, N, BH):
+def kernel_model(name, w, N, BH, train=False):
     """(algorithmic bytes, algorithmic flops) of one launch of a kernel of the
     library over N token-heads (BH sequences): every input and output of the
     kernel counted once (workspace arrays at their stored width), and the
-    dense contractions it exists to perform."""
+    dense contractions it exists to perform.  train: the forward of a
+    training step, which also writes the backward's saved tensors."""
     d, esz = w.d, 2 if w.dtype == "bf16" else 4
     Nd = N * d
     fl = flops_per_token_head(d, w.chunk, w.window, w.M)
@@ -99,8 +100,9 @@ def kernel_model(name, w, N, BH):
         # tensor-core kernels (the configuration the bench runs: both branches
         # on the tensor cores, so the branch sums are fused into the anchor
         # kernels and the GLA feature-map parts travel in bf16)
-        "gate_prep_kernel": (Nd * esz * 2 + BH * nt * d * 4, 0),
-        "tc_fwd_kernel": (5 * Nd * esz + N * 4 + BH * nt * d * 4 + (seg_states if nseg > 1 else 0),
+        "gate_prep_kernel": (Nd * esz * 2 + BH * nt * d * 4 + (Nd * 4 if train else 0), 0),
+        "tc_fwd_kernel": (5 * Nd * esz + N * 4 + BH * nt * d * 4 + (seg_states if nseg > 1 else 0)
+                          + (snaps + BH * nt * d * 4 + BH * d * d * 4 if train else 0),
                           N * (fl["fwd"] + phi)),
         "tc_fwd_kernel(state pass)": ((2 * Nd * esz + Nd * 4) * (nseg - 1) / nseg + seg_states,
                                       N * (nseg - 1) / nseg * (2 * d * d + phi / 2)),
@@ -124,13 +126,13 @@ def kernel_io(dom, per, w, N, BH, peaks, args):
     launch time.  These are the bytes of this decomposition into kernels,
     not the step's algorithmic bytes, so they are reported apart from the
     step-level roofline."""
-    iob, iofl = kernel_model(dom, w, N, BH)
+    iob, iofl = kernel_model(dom, w, N, BH, train=True)
     dt = per[dom] / 1e3
     out = {"kernel": dom, "ms_per_launch": per[dom], "io_bytes": iob,
            "io_gbs": iob / dt / 1e9, "io_frac_of_hbm": iob / dt / 1e9 / peaks["hbm_gbs"],
            "tflops": iofl / dt / 1e12, "tflops_frac_of_bf16": iofl / dt / 1e12 / peaks["bf16_tflops"],
            "traffic": MEASURED_TRAFFIC.get(dom) if args.kernels in ("auto", "tc") else None,
-           "modeled_step_io_bytes": sum(kernel_model(n, w, N, BH)[0] for n in per)}
+           "modeled_step_io_bytes": sum(kernel_model(n, w, N, BH, train=True)[0] for n in per)}
     return out
 
 
@@ -201,7 +203,6 @@ class ClockSampler:
 # profiles/tc_gla_bwd_tile_kernel_train_step.md); "step" sums one training
 # step's 17 launches.
 MEASURED_TRAFFIC = {
-    "step": 8_281_418_496,
     "tc_gla_bwd_tile_kernel": 1_852_018_912,
 }
 
@@ -267,21 +268,23 @@ def run_ours(args, rank, world, local):
     kw = dict(window=w.window, chunk=w.chunk, gate_temp=w.gate_temp, fmap_wq=x["fmap_wq"],
               fmap_wk=x["fmap_wk"], meta_k=x["meta_k"], meta_v=x["meta_v"], alpha=x["alpha"],
               impl=impl)
-    fwd_names = lz.attn_fwd(x["q"], x["k"], x["v"], x["g"], plan_only=True, **kw)
-    bwd_names = lz.attn_bwd(x["q"], x["k"], x["v"], x["g"], x["dout"], plan_only=True, **kw)
-    # persistent outputs/workspaces so the timed loop allocates nothing
+    # persistent outputs/workspaces so the timed loop allocates nothing; the
+    # forward keeps its saved-for-backward tensors in `sv` (None on paths
+    # that keep nothing), which the backward reads
     o = torch.empty_like(x["q"])
-    r0 = lz.attn_fwd(x["q"], x["k"], x["v"], x["g"], out=o, **kw)
-    fws = r0["workspace"]
-    g0 = lz.attn_bwd(x["q"], x["k"], x["v"], x["g"], x["dout"], **kw)
+    r0 = lz.attn_fwd(x["q"], x["k"], x["v"], x["g"], out=o, saved=True, **kw)
+    fws, sv = r0["workspace"], r0["saved"]
+    g0 = lz.attn_bwd(x["q"], x["k"], x["v"], x["g"], x["dout"], saved=sv, **kw)
     bws = g0["workspace"]
     del g0
+    fwd_names = lz.attn_fwd(x["q"], x["k"], x["v"], x["g"], plan_only=True, saved=sv, **kw)
+    bwd_names = lz.attn_bwd(x["q"], x["k"], x["v"], x["g"], x["dout"], plan_only=True, saved=sv, **kw)
     torch.cuda.synchronize()
 
     def step(evf=None, evb=None):
-        lz.attn_fwd(x["q"], x["k"], x["v"], x["g"], out=o, workspace=fws, events=evf, **kw)
+        lz.attn_fwd(x["q"], x["k"], x["v"], x["g"], out=o, workspace=fws, events=evf, saved=sv, **kw)
         return lz.attn_bwd(x["q"], x["k"], x["v"], x["g"], x["dout"], workspace=bws,
-                           events=evb, **kw)
+                           events=evb, saved=sv, **kw)
 
     for _ in range(args.warmup):
         step()
@@ -384,8 +387,8 @@ def run_ours(args, rank, world, local):
             d = dbuf[j]
             with torch.cuda.stream(s_comp):
                 s_comp.wait_event(ev_in[j])
-                lz.attn_fwd(d["q"], d["k"], d["v"], d["g"], out=o, workspace=fws, **kw)
-                gr = lz.attn_bwd(d["q"], d["k"], d["v"], d["g"], d["dout"], workspace=bws, **kw)
+                lz.attn_fwd(d["q"], d["k"], d["v"], d["g"], out=o, workspace=fws, saved=sv, **kw)
+                gr = lz.attn_bwd(d["q"], d["k"], d["v"], d["g"], d["dout"], workspace=bws, saved=sv, **kw)
                 ev_used[j].record(s_comp)
                 ev_out[j].record(s_comp)
             grads[j] = gr
@@ -597,15 +600,18 @@ def run_variants(args, lz, dev, rank, world, peaks, steps):
     kw = dict(window=w.window, chunk=w.chunk, gate_temp=w.gate_temp, fmap_wq=x["fmap_wq"],
               fmap_wk=x["fmap_wk"], meta_k=x["meta_k"], meta_v=x["meta_v"], alpha=x["alpha"],
               impl=impl)
-    fn = lz.attn_fwd(x["q"], x["k"], x["v"], x["g"], plan_only=True, **kw)
-    bn = lz.attn_bwd(x["q"], x["k"], x["v"], x["g"], x["dout"], plan_only=True, **kw)
     o = torch.empty_like(x["q"])
-    fws = lz.attn_fwd(x["q"], x["k"], x["v"], x["g"], out=o, **kw)["workspace"]
-    bws = lz.attn_bwd(x["q"], x["k"], x["v"], x["g"], x["dout"], **kw)["workspace"]
+    r0 = lz.attn_fwd(x["q"], x["k"], x["v"], x["g"], out=o, saved=True, **kw)
+    fws, sv = r0["workspace"], r0["saved"]
+    bws = lz.attn_bwd(x["q"], x["k"], x["v"], x["g"], x["dout"], saved=sv, **kw)["workspace"]
+    fn = lz.attn_fwd(x["q"], x["k"], x["v"], x["g"], plan_only=True, saved=sv, **kw)
+    bn = lz.attn_bwd(x["q"], x["k"], x["v"], x["g"], x["dout"], plan_only=True, saved=sv, **kw)
     msf, perf = _time_steps(lambda ev: lz.attn_fwd(x["q"], x["k"], x["v"], x["g"], out=o, workspace=fws,
-                                                   events=ev, **kw), fn, lz, world, dev, args.warmup, steps)
+                                                   events=ev, saved=sv, **kw), fn, lz, world, dev, args.warmup,
+                            steps)
     msb, perb = _time_steps(lambda ev: lz.attn_bwd(x["q"], x["k"], x["v"], x["g"], x["dout"], workspace=bws,
-                                                   events=ev, **kw), bn, lz, world, dev, args.warmup, steps)
+                                                   events=ev, saved=sv, **kw), bn, lz, world, dev, args.warmup,
+                            steps)
     out["scalar_gate_train_step"] = {
         "workload": f"train_step shape, scalar per-head gate g [B,H,L]: B={w.B} H={w.H} L={w.L}",
         "ms": msf + msb, "fwd_ms": msf, "bwd_ms": msb,

@@ -47,7 +47,7 @@ lizard_status check_fwd(const lizard_fwd_args *a) {
     return LIZARD_ERR_INVALID_ARG;
   const void *ptrs[] = {a->q, a->k, a->v, a->g, a->fmap_wq, a->fmap_wk, a->meta_k, a->meta_v,
                         a->alpha, a->state_in, a->o, a->state_out, a->lse, a->workspace,
-                        a->k_prefix, a->v_prefix};
+                        a->k_prefix, a->v_prefix, a->saved};
   for (const void *p : ptrs)
     if (!ok_ptr(p)) return LIZARD_ERR_INVALID_ARG;
   return LIZARD_OK;
@@ -69,6 +69,12 @@ bool swa_on(const lizard_fwd_args *a) { return a->branch != LIZARD_BRANCH_GLA_ON
 bool fmap_weights(const lizard_fwd_args *a) { return a->fmap_wq != nullptr && a->fmap_wk != nullptr; }
 
 size_t nch32(const lizard_fwd_args *a) { return (a->L + lz::kBwdC - 1) / lz::kBwdC; }
+
+// Whether the backward's GLA branch runs on the tensor-core kernels.
+bool bwd_gla_uses_tc_impl(const lizard_fwd_args *a, int impl) {
+  const bool ok = a->dtype == LIZARD_BF16 && a->dk == 128 && a->dv == 128 && fmap_weights(a);
+  return (impl == LIZARD_IMPL_AUTO || impl == LIZARD_IMPL_TC) && ok;
+}
 
 bool fwd_uses_tc(const lizard_fwd_args *a) {
   const bool ok = lz::tc_fwd_supported(a->dk, a->dv, a->window, a->M, a->dtype == LIZARD_BF16) &&
@@ -103,6 +109,43 @@ FallbackLayout fallback_layout(size_t off, const lizard_fwd_args *a, size_t per_
 // exact fallback, the per-sequence marks that follow it
 size_t cleared_bytes(const lizard_fwd_args *a, bool fallback) {
   return fallback ? kHeader + up((size_t)a->B * a->H * sizeof(uint32_t)) : sizeof(uint32_t);
+}
+
+// Whether a training forward keeps tensors for the backward: the forward's
+// GLA branch on the tensor cores with the backward's tensor-core GLA kernels
+// applicable (bf16, d = 128, feature-map weights).
+bool fwd_keeps(const lizard_fwd_args *a) {
+  return gla_on(a) && fwd_uses_tc(a) && a->dtype == LIZARD_BF16 && a->dk == 128 && a->dv == 128 &&
+         fmap_weights(a);
+}
+
+// The saved-for-backward buffer of a training forward: the wide-decay marks
+// [BH] (cleared by the forward), the tiles' log-decays r [BH][ntiles][d] and
+// fp32 decay factors E [BH][L][d] (the gate prep), the state copies of every
+// tile (bf16 S' - 1 S'[0], then the fp32 rows S'[0]), the final state
+// [BH][d][d] and, with the anchor branch, the softmax normalisers [BH][L]
+// (the full pass).
+struct SavedLayout {
+  size_t flags, r, e32, snap, state, lse, total;
+};
+SavedLayout saved_layout(const lizard_fwd_args *a) {
+  SavedLayout l{};
+  if (!fwd_keeps(a)) return l;
+  const size_t BH = (size_t)a->B * a->H, nt = (a->L + 127) / 128;
+  size_t off = 0;
+  l.flags = off; off += up(BH * sizeof(uint32_t));
+  l.r = off; off += up(BH * nt * a->dk * sizeof(float));
+  l.e32 = off; off += up(BH * a->L * a->dk * sizeof(float));
+  l.snap = off; off += up(lz::tc_gla_bwd_snapshot_bytes((int)BH, a->L));
+  l.state = off; off += up(BH * a->dk * a->dv * sizeof(float));
+  if (swa_on(a)) { l.lse = off; off += up(BH * a->L * sizeof(float)); }   // the anchor softmax normalisers
+  l.total = off;
+  return l;
+}
+
+// Whether the backward reads a training forward's saved tensors.
+bool bwd_reads_saved(const lizard_fwd_args *a, int impl, bool stage1) {
+  return !stage1 && a->saved != nullptr && fwd_keeps(a) && bwd_gla_uses_tc_impl(a, impl);
 }
 
 // Forward workspace: the status header, plus fp32 scratch for the portable path.
@@ -141,11 +184,7 @@ bool bwd_swa_uses_tc(const lizard_fwd_args *a, int impl) {
   return (impl == LIZARD_IMPL_AUTO || impl == LIZARD_IMPL_TC) && ok;
 }
 
-// Whether the backward's GLA branch runs on the tensor-core kernels.
-bool bwd_gla_uses_tc(const lizard_fwd_args *a, int impl) {
-  const bool ok = a->dtype == LIZARD_BF16 && a->dk == 128 && a->dv == 128 && fmap_weights(a);
-  return (impl == LIZARD_IMPL_AUTO || impl == LIZARD_IMPL_TC) && ok;
-}
+bool bwd_gla_uses_tc(const lizard_fwd_args *a, int impl) { return bwd_gla_uses_tc_impl(a, impl); }
 
 struct BwdLayout {
   size_t phq, phk, a, sprev, dphq, dphk, da, dv_gla, dq_swa, dk_swa, dv_swa, lse, Dterm, dsm, pm, snap_s,
@@ -171,15 +210,20 @@ BwdLayout bwd_layout(const lizard_fwd_args *a, int impl, bool stage1 = false) {
     off = l.fb.end;
   }
   if (gla_on(a) && bwd_gla_uses_tc(a, impl)) {
+    // with a training forward's saved tensors, the state copies S', the
+    // fp32 factors E and the tile decays come from there
+    const bool saved = bwd_reads_saved(a, impl, stage1);
     const size_t snap = up(lz::tc_gla_bwd_snapshot_bytes((int)BH, a->L));
-    l.snap_s = off; off += snap;
+    if (!saved) { l.snap_s = off; off += snap; }
     l.snap_ds = off; off += snap;
     l.dphq = off; off += up(N * a->dk * 2);   // bf16, row halves centred
     l.dphk = off; off += up(N * a->dk * 2);
     l.da = off; off += nd;       // dB: gradient of the in-tile cumulative log-decay
     l.dv_gla = off; off += nv;
-    l.e32 = off; off += nd;      // fp32 decay factors E of every tile
-    l.gr = off; off += up(BH * ((a->L + 127) / 128) * a->dk * sizeof(float));   // tiles' log-decays
+    if (!saved) {
+      l.e32 = off; off += nd;      // fp32 decay factors E of every tile
+      l.gr = off; off += up(BH * ((a->L + 127) / 128) * a->dk * sizeof(float));   // tiles' log-decays
+    }
     l.colsum = off; off += up(BH * ((a->L + 127) / 128) * a->dk * sizeof(float));   // tiles' column sums of dB
     l.w16 = off; off += up(lz::tc_gla_bwd_weights_bytes(a->H));                  // bf16 W_q, W_k
     l.kap = off; off += up(BH * 2 * a->dk * sizeof(float));   // final-state share of the decay gradient
@@ -337,6 +381,15 @@ void fwd_plan(const lizard_fwd_args *a, void *ws, cudaStream_t s, Plan &plan, co
     // wide decay: the gate prep marks the sequences, whose GLA branch the
     // full pass then runs as the exact recurrence
     if (lay.fallback) t.seqflag = at<uint32_t>(ws, lay.flags);
+    if (a->saved && !target && fwd_keeps(a)) {   // training: keep what the backward would recompute
+      const SavedLayout sv = saved_layout(a);
+      t.seqflag = at<uint32_t>(a->saved, sv.flags);
+      t.keep_r = at<float>(a->saved, sv.r);
+      t.keep_e32 = at<float>(a->saved, sv.e32);
+      t.snap = at<void>(a->saved, sv.snap);
+      t.state_keep = at<float>(a->saved, sv.state);
+      if (swa_on(a)) t.lse_keep = at<float>(a->saved, sv.lse);
+    }
     if (gla_on(a)) plan.add("gate_prep_kernel", [=](cudaStream_t s) { return lz::launch_tc_fwd(t, 3, s); });
     if (gla_on(a) && lz::tc_fwd_stage_count(BH, a->L) > 1) {   // segment start states (GLA only)
       plan.add("tc_fwd_kernel(state pass)", [=](cudaStream_t s) { return lz::launch_tc_fwd(t, 0, s); });
@@ -375,13 +428,17 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan, bo
                     a->L, a->M, a->window, 0, inv_tau, scale_of(a), scalar_gate(a)};
     f.dstate_out = b->dstate_out;   // the state copies also form the final state's share of dg
     f.kap = at<float>(ws, lay.kap);
-    void *snap_s = at<void>(ws, lay.snap_s);
-    float *e32 = at<float>(ws, lay.e32), *gr = at<float>(ws, lay.gr);
+    const bool saved = bwd_reads_saved(a, b->impl, stage1);
+    const SavedLayout sv = saved_layout(a);
+    void *snap_s = saved ? at<void>(a->saved, sv.snap) : at<void>(ws, lay.snap_s);
+    float *e32 = saved ? at<float>(a->saved, sv.e32) : at<float>(ws, lay.e32);
+    float *gr = saved ? at<float>(a->saved, sv.r) : at<float>(ws, lay.gr);
     uint32_t *status = static_cast<uint32_t *>(ws);
-    uint32_t *flags = lay.fallback ? at<uint32_t>(ws, lay.fb.flags) : nullptr;
-    plan.add("gate_prep_kernel",
-             [=](cudaStream_t s) { return lz::launch_gate_prep(a->g, nullptr, e32, gr, status, BH, a->L, inv_tau, f.scalar_gate != 0,
-                                               s, flags); });
+    uint32_t *flags = !lay.fallback ? nullptr : saved ? at<uint32_t>(a->saved, sv.flags) : at<uint32_t>(ws, lay.fb.flags);
+    if (!saved)
+      plan.add("gate_prep_kernel", [=](cudaStream_t s) {
+        return lz::launch_gate_prep(a->g, nullptr, e32, gr, status, BH, a->L, inv_tau, f.scalar_gate != 0, s, flags);
+      });
     if (lay.fallback) {
       const FallbackLayout fb = lay.fb;
       const int K = fallback_slots(a);
@@ -389,10 +446,20 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan, bo
         return lz::launch_assign_slots(flags, at<int>(ws, fb.slot_of), at<int>(ws, fb.seq_of_slot), BH, K, status, s);
       });
     }
-    // the state copies beside the weight conversion and the reverse dS pass
-    plan.fork();
-    plan.add("tc_fwd_kernel(state copies)",
-             [=](cudaStream_t s) { return lz::launch_tc_state_snapshots(f, snap_s, e32, gr, s); }, 1);
+    if (saved) {
+      // the forward kept the state copies; the final state's share of dg
+      // comes from its kept final state
+      if (b->dstate_out) {
+        const float *sl = at<float>(a->saved, sv.state);
+        float *kap = f.kap;
+        plan.add("state_share_kernel", [=](cudaStream_t s) { return lz::launch_state_share(sl, b->dstate_out, kap, BH, s); });
+      }
+    } else {
+      // the state copies beside the weight conversion and the reverse dS pass
+      plan.fork();
+      plan.add("tc_fwd_kernel(state copies)",
+               [=](cudaStream_t s) { return lz::launch_tc_state_snapshots(f, snap_s, e32, gr, s); }, 1);
+    }
     lz::TcGlaBwdArgs t{a->q, a->k, a->v, a->g, b->dout, a->fmap_wq, a->fmap_wk, snap_s,
                        at<void>(ws, lay.snap_ds), at<float>(ws, lay.dphq), at<float>(ws, lay.dphk),
                        at<float>(ws, lay.da), at<float>(ws, lay.dv_gla), b->dg, b->dstate_in,
@@ -506,6 +573,8 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan, bo
     t.dk_prefix = b->dk_prefix;
     t.dv_prefix = b->dv_prefix;
     t.P = a->prefix_len;
+    // the training forward's softmax normalisers spare the dq pass its max pass
+    if (bwd_reads_saved(a, b->impl, stage1)) t.lse_in = at<float>(a->saved, saved_layout(a).lse);
     plan.add("tc_swa_bwd_q_kernel", [=](cudaStream_t s) { return lz::launch_tc_swa_bwd(t, 0, s); });
     if (a->M > 0 && (b->dmeta_k || b->dmeta_v)) {   // beside the dk / dv pass, after the dq pass's terms
       plan.fork();
@@ -571,6 +640,21 @@ size_t lizard_fwd_workspace_size(const lizard_fwd_args *args) {
   return fwd_layout(&a).total;
 }
 
+size_t lizard_fwd_saved_size(const lizard_fwd_args *args) {
+  if (!args) return 0;
+  lizard_fwd_args a = *args;
+  a.fmap_wq = args->fmap_wq ? reinterpret_cast<const float *>(16) : nullptr;
+  a.fmap_wk = args->fmap_wk ? reinterpret_cast<const float *>(16) : nullptr;
+  a.q = a.k = a.v = a.g = reinterpret_cast<const void *>(16);
+  a.o = reinterpret_cast<void *>(16);
+  a.meta_k = a.M > 0 ? reinterpret_cast<const float *>(16) : nullptr;
+  a.meta_v = a.alpha = a.state_in = a.state_out = a.lse = nullptr;
+  a.workspace = a.saved = nullptr;
+  prefix_standin(a);
+  if (check_fwd(&a) != LIZARD_OK || a.L == 0) return 0;
+  return saved_layout(&a).total;
+}
+
 lizard_status lizard_attn_fwd(const lizard_fwd_args *a, lizard_stream_t stream) {
   lizard_status st = check_fwd(a);
   if (st != LIZARD_OK) return st;
@@ -588,7 +672,13 @@ lizard_status lizard_attn_fwd(const lizard_fwd_args *a, lizard_stream_t stream) 
     }
     return LIZARD_OK;
   }
+  const bool keep = a->saved && fwd_keeps(a);
+  const SavedLayout sv = saved_layout(a);
+  if (keep && a->saved_bytes < sv.total) return LIZARD_ERR_WORKSPACE;
   if (cudaMemsetAsync(a->workspace, 0, cleared_bytes(a, lay.fallback), s) != cudaSuccess) return LIZARD_ERR_CUDA;
+  // a training forward's wide-decay marks start cleared
+  if (keep && cudaMemsetAsync(at<void>(a->saved, sv.flags), 0, (size_t)BH * sizeof(uint32_t), s) != cudaSuccess)
+    return LIZARD_ERR_CUDA;
   Plan plan;
   fwd_plan(a, a->workspace, s, plan);
   return plan.run(s, a->launch_events, a->n_launch_events);
@@ -677,6 +767,7 @@ lizard_status lizard_attn_bwd(const lizard_bwd_args *b, lizard_stream_t stream) 
   if (a->prefix_len > 0 && (!b->dk_prefix || !b->dv_prefix)) return LIZARD_ERR_INVALID_ARG;
   const BwdLayout lay = bwd_layout(a, b->impl);
   if (!b->workspace || b->workspace_bytes < lay.total) return LIZARD_ERR_WORKSPACE;
+  if (bwd_reads_saved(a, b->impl, false) && a->saved_bytes < saved_layout(a).total) return LIZARD_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (bwd_zero_outputs(b, s) != cudaSuccess) return LIZARD_ERR_CUDA;
   if (a->L == 0) return LIZARD_OK;

@@ -167,6 +167,15 @@ struct TcFwdArgs {
   // null: it sets the status word's RANGE bit instead); the full pass then
   // runs their GLA branch as the exact recurrence.
   uint32_t *seqflag;
+  // Training forward (all null: off): the gate prep writes the fp32 decay
+  // factors and tile decays to keep_e32 [BH*L][128] and keep_r
+  // [BH][ntiles][128] (instead of the workspace), and the full pass writes
+  // the backward's state copies `snap` (tc_gla_bwd_snapshot_bytes() bytes)
+  // and the fp32 final state state_keep [BH][128][128].
+  float *keep_e32, *keep_r;
+  void *snap;
+  float *state_keep;
+  float *lse_keep;    // [BH][L] copy of the anchor softmax normalisers (beside lse), or null
 };
 
 struct TcSwaBwdArgs {
@@ -189,6 +198,7 @@ struct TcSwaBwdArgs {
   const void *k_prefix, *v_prefix;
   void *dk_prefix, *dv_prefix;
   int P;
+  const float *lse_in;          // [B*H*L] the forward's softmax normalisers, or null (formed into lse)
 };
 
 struct TcGlaBwdArgs {
@@ -255,6 +265,10 @@ bool tc_swa_bwd_supported(int dk, int dv, int window, int M, bool bf16);
 // stage 0: dq pass, 1: dk/dv pass, 2: meta-token gradients
 cudaError_t launch_tc_swa_bwd(const TcSwaBwdArgs &a, int stage, cudaStream_t s);
 size_t tc_gla_bwd_snapshot_bytes(int BH, int L);
+// kap [BH][2][128] from a kept final state S [BH][128][128] and the incoming
+// final-state gradient G (same layout): the two column halves of
+// sum_v G[i][v] S[i][v].
+cudaError_t launch_state_share(const float *S, const float *G, float *kap, int BH, cudaStream_t s);
 // bf16 copies of W_q, W_k ([H][2][128][64]) for the per-tile backward's TMA loads
 size_t tc_gla_bwd_weights_bytes(int H);
 cudaError_t launch_weights_bf16(const float *wq, const float *wk, void *out, int H, cudaStream_t s);

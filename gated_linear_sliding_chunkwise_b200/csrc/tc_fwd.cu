@@ -95,8 +95,11 @@ struct Params {
   const float *seg_start;   // [BH][nseg][D][D] start state of each segment (nseg > 1)
   float *seg_state;         // mode 1: [BH][nseg][D][D] local end state (zero start)
   float *seg_decay;         // mode 1: [BH][nseg][D] summed log-decay of the segment
-  __nv_bfloat16 *snap;      // mode 1 with nseg == 1: [BH][ntiles][D][D] bf16 S' - 1 S'[0] of every tile
+  __nv_bfloat16 *snap;      // mode 1 with nseg == 1, or a training full pass: [BH][ntiles][D][D]
+                            // bf16 S' - 1 S'[0] of every tile (the backward's copies)
   float *snap_r0;           // ... and [BH][ntiles][D] fp32 row 0 of S' (the part taken out of every row)
+  float *state_keep;        // training full pass: [BH][D][D] fp32 final state for the backward, or null
+  float *lse_keep;          // training full pass: [BH][L] copy of lse for the backward, or null
   const float *gate_r;      // [BH][ntiles][D] log-decay r of every tile (gate_prep_kernel)
   const float *gate_e32;    // mode 1: [BH][L][D] fp32 decay factors E, loaded through `me` (mode 0 loads bf16 E as the G tiles)
   const float *kap_g;       // mode 1 with copies: incoming final-state gradient G [BH][D][D], or null
@@ -300,6 +303,8 @@ __device__ __forceinline__ void exact_gla_sequence(const Params &p, unsigned cha
   }
   if (p.state_out)
     for (int e = tid; e < D * D; e += NTHREADS) p.state_out[(size_t)bh * D * D + e] = S[e];
+  if (p.state_keep)
+    for (int e = tid; e < D * D; e += NTHREADS) p.state_keep[(size_t)bh * D * D + e] = S[e];
 }
 
 // Named barriers (id 0 is __syncthreads).
@@ -325,7 +330,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
   __shared__ uint32_t s_tmem;
   __shared__ int s_fail;
   __shared__ float s_mse[NTHREADS / 32];
-  __shared__ __align__(16) float s_row0[D];   // state pass: row 0 of S' (taken out of the copies)
+  __shared__ __align__(16) float s_row0[D];   // row 0 of S' (state pass) or of S (full pass), taken out of the copies
   __shared__ __align__(16) float s_rt[D];     // the tile's log-decays r (arrive with its loads)
 
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -407,6 +412,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
 #pragma unroll
       for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(src ? src[c + u] : 0.f);
       tmem_st8(tl + C_S + c, r);
+      if (full && p.snap && row == 0)   // the first tile's centre for the backward's copies
+#pragma unroll
+        for (int u = 0; u < 8; ++u) s_row0[c + u] = __uint_as_float(r[u]);
     }
     tmem_st_wait();
   }
@@ -582,7 +590,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
           tmem_st8(tl + C_P + ch * 16, zero);
           tmem_st8(tl + C_P + ch * 16 + 8, zero);
         }
-        if (wg == 0 && qvalid && p.lse) p.lse[(size_t)bh * p.L + tq] = mx + logf(lsum);
+        if (wg == 0 && qvalid && (p.lse || p.lse_keep)) {
+          const float lse = mx + logf(lsum);
+          if (p.lse) p.lse[(size_t)bh * p.L + tq] = lse;
+          if (p.lse_keep) p.lse_keep[(size_t)bh * p.L + tq] = lse;
+        }
       }
       // GLA operands carry l/alpha so that one accumulator holds both terms
       const bool mixed = swa && alpha != 0.f;
@@ -650,6 +662,32 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         if (full) {   // bf16 copy S'[i][v], MN-major: rows = i (K of the O = Qt S' product)
           *chunk_ptr(sm, R_XQ, i, 2 * c16) = pack8(v);
           *chunk_ptr(sm, R_XQ, i, 2 * c16 + 1) = pack8(v + 8);
+          if (p.snap) {
+            // training: the backward's copy S' - 1 S'[0] (as the state pass
+            // below writes it), S'[0] = exp(r_0) S[0] with S[0] staged at the
+            // end of the previous tile; row 0 itself goes out in fp32
+            const size_t tile = (size_t)bh * ntiles_all + c;
+            const float d0 = s_dec[0];
+            const float4 *r0 = reinterpret_cast<const float4 *>(s_row0 + c16 * 16);
+            float w[16];
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              const float4 x = r0[q4];
+              w[4 * q4] = v[4 * q4] - __fmul_rn(x.x, d0);
+              w[4 * q4 + 1] = v[4 * q4 + 1] - __fmul_rn(x.y, d0);
+              w[4 * q4 + 2] = v[4 * q4 + 2] - __fmul_rn(x.z, d0);
+              w[4 * q4 + 3] = v[4 * q4 + 3] - __fmul_rn(x.w, d0);
+            }
+            uint4 *dst = reinterpret_cast<uint4 *>(p.snap + (tile * D + i) * D + c16 * 16);
+            dst[0] = pack8(w);
+            dst[1] = pack8(w + 8);
+            if (i == 0) {
+              float4 *d4 = reinterpret_cast<float4 *>(p.snap_r0 + tile * D + c16 * 16);
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4)
+                d4[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+            }
+          }
         } else if (p.snap && i == 0) {
 #pragma unroll
           for (int u = 0; u < 16; ++u) s_row0[c16 * 16 + u] = v[u];
@@ -779,6 +817,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         }
       }
     }
+    if (full && gla && p.snap && (warp & 3) == 0 && c + 1 < cend) {
+      // row 0 of the state this tile leaves: the next tile's centre
+      for (int c16 = 4 * wg; c16 < 4 * wg + 4; ++c16) {
+        float v[16];
+        tmem_ld16(tl + C_S + c16 * 16, v);
+        if (row == 0) {
+          float4 *d4 = reinterpret_cast<float4 *>(s_row0 + c16 * 16);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) d4[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+        }
+      }
+    }
     tc_fence_before();
     __syncthreads();
   }
@@ -793,8 +843,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       atomicAdd(p.loss, tot * p.mse_loss);
     }
   }
-  float *sdst = nullptr;
+  float *sdst = nullptr, *skeep = nullptr;
   if (full && p.state_out && gla && seg == p.nseg - 1) sdst = p.state_out + ((size_t)bh * D + row) * D;
+  if (full && p.state_keep && gla && seg == p.nseg - 1) skeep = p.state_keep + ((size_t)bh * D + row) * D;
   if (!full && p.seg_state) {
     sdst = p.seg_state + (((size_t)bh * p.nseg + seg) * D + row) * D;
     if (wg == 0) p.seg_decay[((size_t)bh * p.nseg + seg) * D + row] = tot_decay;
@@ -811,14 +862,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
     }
     p.kap[((size_t)bh * 2 + wg) * D + row] = part;
   }
-  if (!s_fail && sdst) {
+  if (!s_fail && (sdst || skeep)) {
     tc_fence_after();
     for (int c16 = 4 * wg; c16 < 4 * wg + 4; ++c16) {
       float v[16];
       tmem_ld16(tl + C_S + c16 * 16, v);
 #pragma unroll
-      for (int u = 0; u < 16; u += 4)
-        *reinterpret_cast<float4 *>(sdst + c16 * 16 + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
+      for (int u = 0; u < 16; u += 4) {
+        const float4 x = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
+        if (sdst) *reinterpret_cast<float4 *>(sdst + c16 * 16 + u) = x;
+        if (skeep) *reinterpret_cast<float4 *>(skeep + c16 * 16 + u) = x;
+      }
     }
   }
   if (s_fail && tid == 0) {
@@ -1122,9 +1176,13 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, int stage, cudaStream_t s) {
   tc_fwd_segments(a.BH, a.L, &nseg, &tps);
   const FwdWs w = fwd_ws(a.seg_ws, a.BH, a.L);
   const bool gla = a.branch != 2 && a.g != nullptr;
+  // a training forward keeps the fp32 factors and the tile decays for the
+  // backward (in the caller's arrays instead of the workspace)
+  float *e32 = a.keep_e32 ? a.keep_e32 : w.e32;
+  float *rr = a.keep_r ? a.keep_r : w.r;
   if (stage == 3) {
     if (!gla) return cudaSuccess;
-    return launch_gate_prep(a.g, w.e16, w.e32, w.r, a.status, a.BH, a.L, a.inv_tau, a.scalar_gate != 0, s,
+    return launch_gate_prep(a.g, w.e16, e32, rr, a.status, a.BH, a.L, a.inv_tau, a.scalar_gate != 0, s,
                             a.seqflag);
   }
   if (nseg > 1 && (stage == 0 || stage == 1) && !gla) return cudaSuccess;   // no state to carry
@@ -1142,9 +1200,15 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, int stage, cudaStream_t s) {
   if (!make_map_bf16_3d(&p.mq, a.q, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mk, a.k, D, rows, a.BH, T) ||
       !make_map_bf16_3d(&p.mv, a.v, D, rows, a.BH, T) || !make_map_bf16_3d(&p.mg, gsrc, D, rows, a.BH, T))
     return cudaErrorInvalidValue;
-  p.gate_r = gla ? w.r : nullptr;
-  p.gate_e32 = gla ? w.e32 : nullptr;
-  if (gla && nseg > 1 && !make_map_f32_3d(&p.me, w.e32, D, rows, a.BH, T)) return cudaErrorInvalidValue;
+  p.gate_r = gla ? rr : nullptr;
+  p.gate_e32 = gla ? e32 : nullptr;
+  if (gla && nseg > 1 && !make_map_f32_3d(&p.me, e32, D, rows, a.BH, T)) return cudaErrorInvalidValue;
+  if (gla && a.snap && stage == 2) {   // training: the backward's state copies and final state
+    p.snap = static_cast<__nv_bfloat16 *>(a.snap);
+    p.snap_r0 = reinterpret_cast<float *>(p.snap + (size_t)a.BH * ((a.L + T - 1) / T) * D * D);
+    p.state_keep = a.state_keep;
+  }
+  if (a.branch != 1 && stage == 2) p.lse_keep = a.lse_keep;
   p.wq = a.wq;
   p.wk = a.wk;
   p.meta_k = a.meta_k;

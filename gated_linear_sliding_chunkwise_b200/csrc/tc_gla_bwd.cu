@@ -854,6 +854,32 @@ cudaError_t launch_weights_bf16(const float *wq, const float *wk, void *out, int
   return cudaGetLastError();
 }
 
+namespace {
+// The final state's share of the log-decay gradient from a final state the
+// forward kept: kap[bh][h][i] = sum over column half h of G[i][v] S_L[i][v]
+// (G the incoming final-state gradient); thread = (half, key dimension).
+__global__ void __launch_bounds__(256) state_share_kernel(const float *S, const float *G, float *kap) {
+  const int bh = blockIdx.x, i = threadIdx.x & 127, h = threadIdx.x >> 7;
+  const float4 *s4 = reinterpret_cast<const float4 *>(S + ((size_t)bh * D + i) * D + 64 * h);
+  const float4 *g4 = reinterpret_cast<const float4 *>(G + ((size_t)bh * D + i) * D + 64 * h);
+  float part = 0.f;
+#pragma unroll 4
+  for (int u = 0; u < 16; ++u) {
+    const float4 a = s4[u], b = g4[u];
+    part = fmaf(b.x, a.x, part);
+    part = fmaf(b.y, a.y, part);
+    part = fmaf(b.z, a.z, part);
+    part = fmaf(b.w, a.w, part);
+  }
+  kap[((size_t)bh * 2 + h) * D + i] = part;
+}
+}  // namespace
+
+cudaError_t launch_state_share(const float *S, const float *G, float *kap, int BH, cudaStream_t s) {
+  state_share_kernel<<<BH, 256, 0, s>>>(S, G, kap);
+  return cudaGetLastError();
+}
+
 size_t tc_gla_bwd_snapshot_bytes(int BH, int L) {
   const size_t n = (size_t)BH * ((L + T - 1) / T);
   return n * D * D * sizeof(__nv_bfloat16) + n * D * sizeof(float);

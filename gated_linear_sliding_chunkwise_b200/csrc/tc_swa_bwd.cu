@@ -45,6 +45,7 @@ struct QParams {
   CUtensorMap mxq, mdqo;      // fused: bf16 GLA part dx_q (load), bf16 final dq (store)
   const float *meta_k, *meta_v, *alpha;
   float *dq, *lse, *Dterm, *dsm, *pm, *dalpha;
+  const float *lse_in;        // the forward's softmax normalisers (null: formed here, into lse)
   uint32_t *status;
   int H, L, M, window;
   float scale;
@@ -179,6 +180,7 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
     mma_commit(bar_m);
   }
   {
+    const float lse_row = (p.lse_in && qvalid) ? p.lse_in[(size_t)bh * p.L + tq] : 0.f;
     // meta dot products while the MMAs run, by mma.sync over each warp's 32
     // rows, every lane getting its own row's: group 0 q . mk_m (kept in
     // registers), group 1 dO . mv_m (to shared memory)
@@ -210,6 +212,9 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
           mx = fmaxf(mx, ml[m]);
         }
     }
+    // With the forward's normaliser lse = log sum exp of the row's scaled
+    // logits, P = exp(l - lse) directly: no max pass, and P^ below is P.
+    const bool given = p.lse_in != nullptr;
 
     // 2. softmax over the band (see the forward): logit column cl holds key
     //    t0 - T + cl; warp w4 visits chunks ch_lo .. ch_hi, group 1 the
@@ -228,6 +233,9 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
     const int full_hi = split ? ch_hi - 1 : ch_hi;
     const int hcol = 32 * ch_hi + 16 * (1 - wg);
     const bool hinner = hcol >= in_lo && hcol + 15 <= 32 * w4 + T && hcol + cbase >= -p.P;
+    if (given) {
+      mx = lse_row;
+    } else {
     if (split) {
       float v[16];
       tmem_ld16(tl + C_L + hcol, v);
@@ -258,6 +266,7 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
     s_pmax[wg][row] = mx;
     bar_sync(1, NT_Q);
     mx = fmaxf(s_pmax[0][row], s_pmax[1][row]);
+    }
     //    P^ = exp(l - max) of this group's chunks, held in registers until
     //    both groups have read their logits (P^ overlays logit chunks 0 .. 3)
     //    and, for D = dO_swa . o_swa = alpha (sum_j P^_j dP'_j + sum_m e_m
@@ -319,7 +328,7 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
     s_dpart[wg][row] = dpart;
     bar_sync(2, NT_Q);
     const float lsum = s_psum[0][row] + s_psum[1][row];
-    const float inv_l = 1.f / lsum;
+    const float inv_l = given ? 1.f : 1.f / lsum;
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       const int ch = ch_lo + 1 - wg + 2 * k;
@@ -336,7 +345,7 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
         tmem_st8(tl + C_P + ch * 16 + 8, zero);
       }
     }
-    if (wg == 0 && qvalid) p.lse[(size_t)bh * p.L + tq] = mx + logf(lsum);
+    if (wg == 0 && qvalid && !given) p.lse[(size_t)bh * p.L + tq] = mx + logf(lsum);
     tmem_st_wait();
     // 3. D (dO_swa . o_swa) from the two groups' sums
     float dal = (s_dpart[0][row] + s_dpart[1][row]) * inv_l;
@@ -882,6 +891,7 @@ cudaError_t launch_tc_swa_bwd(const TcSwaBwdArgs &a, int stage, cudaStream_t s) 
     p.alpha = a.alpha;
     p.dq = a.dq;
     p.lse = a.lse;
+    p.lse_in = a.lse_in;
     p.Dterm = a.Dterm;
     p.dsm = a.dsm;
     p.pm = a.pm;
@@ -924,7 +934,7 @@ cudaError_t launch_tc_swa_bwd(const TcSwaBwdArgs &a, int stage, cudaStream_t s) 
     p.dv_prefix = static_cast<__nv_bfloat16 *>(a.dv_prefix);
   }
   p.alpha = a.alpha;
-  p.lse = a.lse;
+  p.lse = a.lse_in ? a.lse_in : a.lse;
   p.Dterm = a.Dterm;
   p.dk = a.dk;
   p.dv = a.dv;

@@ -45,7 +45,8 @@ class FwdArgs(ctypes.Structure):
                 ("alpha", _vp), ("state_in", _vp), ("o", _vp), ("state_out", _vp),
                 ("lse", _vp), ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t),
                 ("launch_events", ctypes.POINTER(_vp)), ("n_launch_events", _i32),
-                ("k_prefix", _vp), ("v_prefix", _vp), ("prefix_len", _i32)]
+                ("k_prefix", _vp), ("v_prefix", _vp), ("prefix_len", _i32),
+                ("saved", _vp), ("saved_bytes", ctypes.c_size_t)]
 
 
 class BwdArgs(ctypes.Structure):
@@ -75,6 +76,8 @@ _lib.lizard_fwd_workspace_size.argtypes = [ctypes.POINTER(FwdArgs)]
 _lib.lizard_fwd_workspace_size.restype = ctypes.c_size_t
 _lib.lizard_attn_fwd.argtypes = [ctypes.POINTER(FwdArgs), _vp]
 _lib.lizard_attn_fwd.restype = ctypes.c_int
+_lib.lizard_fwd_saved_size.argtypes = [ctypes.POINTER(FwdArgs)]
+_lib.lizard_fwd_saved_size.restype = ctypes.c_size_t
 _lib.lizard_bwd_workspace_size.argtypes = [ctypes.POINTER(BwdArgs)]
 _lib.lizard_bwd_workspace_size.restype = ctypes.c_size_t
 _lib.lizard_attn_bwd.argtypes = [ctypes.POINTER(BwdArgs), _vp]
@@ -208,6 +211,19 @@ def fwd_workspace_bytes(args: FwdArgs) -> int:
     return int(_lib.lizard_fwd_workspace_size(ctypes.byref(args)))
 
 
+def fwd_saved_bytes(args: FwdArgs) -> int:
+    """Bytes of the training forward's saved-for-backward buffer (0: none)."""
+    return int(_lib.lizard_fwd_saved_size(ctypes.byref(args)))
+
+
+def _attach_saved(args: FwdArgs, saved):
+    """Point the struct at a saved-for-backward buffer (a uint8 tensor)."""
+    if saved is None:
+        args.saved, args.saved_bytes = None, 0
+    else:
+        args.saved, args.saved_bytes = saved.data_ptr(), saved.numel() * saved.element_size()
+
+
 def bwd_workspace_bytes(args: BwdArgs) -> int:
     return int(_lib.lizard_bwd_workspace_size(ctypes.byref(args)))
 
@@ -254,12 +270,16 @@ def attn_fwd(q, k, v, g, *, window, chunk=64, gate_temp=16.0, softmax_scale=0.0,
              fmap_wq=None, fmap_wk=None, meta_k=None, meta_v=None, alpha=None,
              state_in=None, want_state=False, want_lse=False,
              branch=BRANCH_BOTH, impl=IMPL_AUTO, out=None, workspace=None, stream=None,
-             events=None, plan_only=False, k_prefix=None, v_prefix=None):
+             events=None, plan_only=False, k_prefix=None, v_prefix=None, saved=None):
     """Forward of the hybrid layer (lizard_attn_fwd).  Tensors on one CUDA
     device, contiguous; returns a dict with o, state_out, lse.  `events`
     (torch.cuda.Event list) are recorded around each kernel; plan_only returns
     the kernel names without launching.  k_prefix, v_prefix [B, H, P, d]: the
-    P <= window tokens before token 0, seen by the anchor window."""
+    P <= window tokens before token 0, seen by the anchor window.  saved: a
+    uint8 device tensor of at least fwd_saved_bytes() bytes, or True to
+    allocate one, into which a training forward writes what attn_bwd(...,
+    saved=) reads instead of recomputing (returned as "saved"; None when the
+    forward keeps nothing for these arguments)."""
     a = _fwd_struct(q, k, v, g, window=window, chunk=chunk, gate_temp=gate_temp,
                     softmax_scale=softmax_scale, fmap_wq=fmap_wq, fmap_wk=fmap_wk,
                     meta_k=meta_k, meta_v=meta_v, alpha=alpha, state_in=state_in,
@@ -277,12 +297,16 @@ def attn_fwd(q, k, v, g, *, window, chunk=64, gate_temp=16.0, softmax_scale=0.0,
     nbytes = fwd_workspace_bytes(a)
     ws = _workspace(nbytes, q.device, workspace)
     a.workspace, a.workspace_bytes = ws.data_ptr(), ws.numel() * ws.element_size()
+    if saved is True:
+        n = fwd_saved_bytes(a)
+        saved = torch.empty(n, dtype=torch.uint8, device=q.device) if n > 0 else None
+    _attach_saved(a, saved)
     if plan_only:
         return _plan(_lib.lizard_fwd_launch_plan, a)
     keep = _attach_events(a, events)
     _check(_lib.lizard_attn_fwd(ctypes.byref(a), _stream(stream)), "lizard_attn_fwd")
     del keep
-    return {"o": o, "state_out": S, "lse": lse, "workspace": ws}
+    return {"o": o, "state_out": S, "lse": lse, "workspace": ws, "saved": saved}
 
 
 def _bwd_struct(f, q, k, v, g, dout, *, meta_k, meta_v, fmap_wq, fmap_wk, impl, want_dstate):
@@ -315,12 +339,13 @@ def attn_bwd(q, k, v, g, dout, *, window, chunk=64, gate_temp=16.0, softmax_scal
              fmap_wq=None, fmap_wk=None, meta_k=None, meta_v=None, alpha=None,
              state_in=None, branch=BRANCH_BOTH, impl=IMPL_AUTO, want_dstate=True,
              workspace=None, stream=None, events=None, plan_only=False, dstate_out=None,
-             k_prefix=None, v_prefix=None):
+             k_prefix=None, v_prefix=None, saved=None):
     """Backward of the hybrid layer (lizard_attn_bwd); returns every gradient.
     dstate_out [B, H, dk, dv] fp32: gradient flowing into the final state
     (None: the final state is unused).  k_prefix, v_prefix [B, H, P, d]: the
     anchor window's prefix, as in attn_fwd; their gradients come back as
-    dk_prefix, dv_prefix."""
+    dk_prefix, dv_prefix.  saved: the buffer attn_fwd(..., saved=) filled for
+    the same inputs (None: recompute)."""
     f = _fwd_struct(q, k, v, g, window=window, chunk=chunk, gate_temp=gate_temp,
                     softmax_scale=softmax_scale, fmap_wq=fmap_wq, fmap_wk=fmap_wk,
                     meta_k=meta_k, meta_v=meta_v, alpha=alpha, state_in=state_in,
@@ -330,6 +355,7 @@ def attn_bwd(q, k, v, g, dout, *, window, chunk=64, gate_temp=16.0, softmax_scal
     b, res = _bwd_struct(f, q, k, v, g, dout, meta_k=meta_k, meta_v=meta_v, fmap_wq=fmap_wq,
                          fmap_wk=fmap_wk, impl=impl, want_dstate=want_dstate)
     b.dstate_out = _ptr(dstate_out)
+    _attach_saved(b.fwd, saved)
     res["dk_prefix"] = res["dv_prefix"] = None
     if k_prefix is not None:
         b.fwd.k_prefix, b.fwd.v_prefix = _ptr(k_prefix), _ptr(v_prefix)

@@ -165,6 +165,11 @@ typedef struct {
   int32_t n_launch_events;
   const void *k_prefix, *v_prefix;   /* see "Key/value prefix" above */
   int32_t prefix_len;
+  /* Training forward: device buffer of >= lizard_fwd_saved_size() bytes (16-byte
+   * aligned) into which the forward writes what lizard_attn_bwd would
+   * otherwise recompute, or NULL.  See "Saved for the backward" below. */
+  void *saved;
+  size_t saved_bytes;
 } lizard_fwd_args;
 
 /* Bytes of device workspace the forward needs for these arguments.  Pointer
@@ -176,11 +181,41 @@ size_t lizard_fwd_workspace_size(const lizard_fwd_args *args);
 lizard_status lizard_attn_fwd(const lizard_fwd_args *args, lizard_stream_t stream);
 
 /*
+ * Saved for the backward (training).  The backward of the GLA branch needs,
+ * per 128-token tile, the state at the tile's start decayed by the tile's
+ * gates (S' = diag(exp r) S, the state-update recurrence of the English
+ * gist.science summary, section 2.A) and the tile's decay factors in fp32
+ * (the log-space gate absorption of the Chinese summary, section 2.3), and
+ * its anchor softmax needs each row's normaliser (section 2.A, anchor window
+ * attention).  The forward has all three at hand; without a saved buffer the
+ * backward recomputes them (a gate pass, a state pass over the sequence and
+ * a max pass over the window logits).
+ *
+ * With args->saved set, lizard_attn_fwd also writes, into that buffer: the
+ * wide-decay marks, the tiles' log-decays and fp32 decay factors, a bf16
+ * copy of every tile's S' (rows less row 0, which is kept in fp32), the
+ * fp32 final state and, with the anchor branch, the normalisers (lse).  A backward whose fwd.saved points at that buffer (same
+ * inputs, enqueued after the forward) reads them instead of recomputing; its
+ * results agree with the recomputing backward's to bf16 rounding of S'.
+ * lizard_bwd_workspace_size() is smaller when fwd.saved is set.
+ *
+ * Returns the bytes the buffer needs for these arguments (pointer fields
+ * are ignored, except whether fmap_wq / fmap_wk are given), or 0 when the
+ * forward keeps nothing for these arguments (GLA branch off, not on the
+ * tensor-core path, no feature-map weights); saved is then ignored by the
+ * forward and the backward.  A saved buffer smaller than this size is
+ * LIZARD_ERR_WORKSPACE in both calls.
+ */
+size_t lizard_fwd_saved_size(const lizard_fwd_args *args);
+
+/*
  * Backward of the hybrid layer: gradients of sum(dout * o) with respect to
  * every input of lizard_attn_fwd.
  *
  *   fwd      the forward's inputs (fwd.o, fwd.state_out, fwd.lse and the
- *            forward workspace are ignored)
+ *            forward workspace are ignored); fwd.saved, when not NULL, is a
+ *            buffer lizard_attn_fwd filled for these inputs (see "Saved for
+ *            the backward"), which the call reads but does not change
  *   dout     [B, H, L, dv] dtype
  *   dq, dk   [B, H, L, dk] dtype, written
  *   dv       [B, H, L, dv] dtype, written
@@ -280,7 +315,7 @@ lizard_status lizard_chain_states(const lizard_chain_args *args, lizard_stream_t
  *            and bwd.fwd.o may be NULL (the output is then not kept) or
  *            receives o.  bwd.fwd.impl selects the forward's kernels,
  *            bwd.impl the backward's.  bwd.workspace and bwd.launch_events
- *            serve the whole step.
+ *            serve the whole step; bwd.fwd.saved is ignored.
  *   target   [B, H, L, dv] dtype: the teacher's attention output y
  *   loss     one fp32, written: sum over every element of (o - y)^2 divided
  *            by the element count B H L dv; dL/do = 2 (o - y) / (B H L dv)

@@ -140,6 +140,43 @@ def test_workspace_size_rejects_bad_sizes(lz):
     assert lz.lib().lizard_fwd_workspace_size(None) == 0
 
 
+def test_saved_size_and_refusals_on_host(lz):
+    """The training forward's saved buffer: its size follows the tensor-core
+    GLA path (0 without it), it shrinks the backward's workspace, a buffer
+    one byte short is refused by both calls before anything is enqueued, and
+    a misaligned one is an invalid argument."""
+    w = dict(dk=128, dv=128, window=128, fmap_wq=0x10000, fmap_wk=0x10000)
+    a = _fwd(lz, **w)
+    need = lz.fwd_saved_bytes(a)
+    BH, L, nt = 2, 128, 1
+    # marks, tile decays, fp32 factors, bf16 copies + their fp32 row 0, final state, softmax
+    # normalisers (256-byte aligned each); the GLA branch alone keeps no normalisers
+    up = lambda x: (x + 255) // 256 * 256
+    gla = (up(BH * 4) + up(BH * nt * 128 * 4) + up(BH * L * 128 * 4)
+           + up(BH * nt * 128 * 128 * 2 + BH * nt * 128 * 4) + up(BH * 128 * 128 * 4))
+    assert need == gla + up(BH * L * 4)
+    assert lz.fwd_saved_bytes(_fwd(lz, **w, branch=lz.BRANCH_GLA_ONLY)) == gla
+    for over in ({"branch": lz.BRANCH_SWA_ONLY}, {"fmap_wq": None, "fmap_wk": None},
+                 {"impl": lz.IMPL_SIMT}, {"dk": 64, "dv": 64}, {"L": 0}):
+        assert lz.fwd_saved_bytes(_fwd(lz, **{**w, **over})) == 0, over
+    assert lz.lib().lizard_fwd_saved_size(None) == 0
+    a.workspace, a.workspace_bytes = 0x20000, lz.fwd_workspace_bytes(a)
+    a.saved, a.saved_bytes = 0x30000, need - 1
+    assert lz.lib().lizard_attn_fwd(ctypes.byref(a), None) == lz.ERR_WORKSPACE
+    a.saved = 0x30008
+    assert lz.lib().lizard_attn_fwd(ctypes.byref(a), None) == lz.ERR_INVALID_ARG
+    b = lz.BwdArgs()
+    b.fwd = _fwd(lz, **w)
+    fake = 0x10000
+    b.dout = b.dq = b.dk = b.dv = b.dg = fake
+    plain = lz.bwd_workspace_bytes(b)
+    b.fwd.saved, b.fwd.saved_bytes = 0x30000, need - 1
+    lean = lz.bwd_workspace_bytes(b)
+    assert 0 < lean < plain
+    b.workspace, b.workspace_bytes = 0x20000, lean
+    assert lz.lib().lizard_attn_bwd(ctypes.byref(b), None) == lz.ERR_WORKSPACE
+
+
 def test_backward_rejects_bad_arguments_on_host(lz):
     b = lz.BwdArgs()
     b.fwd = _fwd(lz)
