@@ -88,6 +88,7 @@ struct Params {
   CUtensorMap mq, mk, mv, mg;
   CUtensorMap mkp, mvp;     // key / value prefix [BH][P][D] (P > 0 only)
   CUtensorMap me;           // mode 1: fp32 decay factors E [BH][L][D] (loads)
+  CUtensorMap msnap;        // training full pass: the state copies [BH*ntiles][D][D] bf16 (stores)
   const float *wq, *wk, *meta_k, *meta_v, *alpha, *state_in;
   __nv_bfloat16 *o;
   float *state_out, *lse;
@@ -150,9 +151,11 @@ __device__ __forceinline__ void issue_tile_loads(const Params &p, unsigned char 
 }
 
 // Qt for dimensions 64 h .. 64 h + 63: phi_q E gscale, bf16 pairs into TMEM.
-__device__ __forceinline__ void qt_half(unsigned char *sm, uint32_t tl, int row, int h, float gscale) {
+// With `sum`, returns the sum of the stored (bf16-rounded) values.
+__device__ __forceinline__ float qt_half(unsigned char *sm, uint32_t tl, int row, int h, float gscale, bool sum) {
   float ph[F];
   const float s = feature_half(tl + C_ZQ, h, ph) * gscale;
+  float acc[2] = {0.f, 0.f};
 #pragma unroll
   for (int c16 = 0; c16 < 4; ++c16) {     // 16 dims = 8 TMEM columns
     float e16[16];
@@ -160,10 +163,16 @@ __device__ __forceinline__ void qt_half(unsigned char *sm, uint32_t tl, int row,
     unpack8(*chunk_ptr(sm, R_G, row, 8 * h + 2 * c16 + 1), e16 + 8);
     uint32_t r8[8];
 #pragma unroll
-    for (int u = 0; u < 16; u += 2)
+    for (int u = 0; u < 16; u += 2) {
       r8[u / 2] = pack_bf16(ph[16 * c16 + u] * e16[u] * s, ph[16 * c16 + u + 1] * e16[u + 1] * s);
+      if (sum) {
+        acc[0] += __uint_as_float(r8[u / 2] << 16);
+        acc[1] += __uint_as_float(r8[u / 2] & 0xffff0000u);
+      }
+    }
     tmem_st8(tl + C_QT + 32 * h + 8 * c16, r8);
   }
+  return acc[0] + acc[1];
 }
 
 // Kt for dimensions 64 h .. 64 h + 63: phi_k / E, bf16 into shared memory
@@ -331,6 +340,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
   __shared__ int s_fail;
   __shared__ float s_mse[NTHREADS / 32];
   __shared__ __align__(16) float s_row0[D];   // row 0 of S' (state pass) or of S (full pass), taken out of the copies
+  __shared__ __align__(16) float s_r0v[D];    // full pass, centred: row 0 of this tile's S'
+  __shared__ float s_qsum[2][T];              // full pass, centred: each group's sum of its Qt dimensions
   __shared__ __align__(16) float s_rt[D];     // the tile's log-decays r (arrive with its loads)
 
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -346,6 +357,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
   const bool marked = p.seqflag && p.seqflag[bh] != 0u;
   if (marked && (!full || seg > 0)) return;
   const bool gla = p.branch != 2 && !marked, swa = full && p.branch != 1;
+  // Training: MMA 3 reads S' as the bf16 copy of S' - 1 S'[0] (rows less
+  // their first; the epilogue adds back (sum_i Qt[i]) S'[0] in fp32), and
+  // that copy goes to the backward as is, with one TMA store per tile.
+  const bool centre = full && gla && p.snap != nullptr;
   const uint32_t sbase = smem_u32(sm);
   const int ntiles_all = (p.L + T - 1) / T;
   const int cbeg = marked ? 0 : seg * p.tiles_per_seg;
@@ -412,7 +427,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
 #pragma unroll
       for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(src ? src[c + u] : 0.f);
       tmem_st8(tl + C_S + c, r);
-      if (full && p.snap && row == 0)   // the first tile's centre for the backward's copies
+      if (centre && row == 0)   // row 0 of the start state: the first tile's centre
 #pragma unroll
         for (int u = 0; u < 8; ++u) s_row0[c + u] = __uint_as_float(r[u]);
     }
@@ -606,7 +621,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
           for (int m = 0; m < p.M; ++m) s_ml[m][row] *= mscale;
         }
       }
-      qt_half(sm, tl, row, wg, gscale);
+      const float qs = qt_half(sm, tl, row, wg, gscale, centre);
+      if (centre) s_qsum[wg][row] = qs;
       kt_half(sm, tl, row, wg, false, qvalid);
     } else {
       // ------ state pass: phi_k half per group, with the fp32 decay factors
@@ -660,13 +676,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         for (int u = 0; u < 8; ++u) r[u] = __float_as_uint(v[8 + u]);
         tmem_st8(tl + C_S + c16 * 16 + 8, r);
         if (full) {   // bf16 copy S'[i][v], MN-major: rows = i (K of the O = Qt S' product)
-          *chunk_ptr(sm, R_XQ, i, 2 * c16) = pack8(v);
-          *chunk_ptr(sm, R_XQ, i, 2 * c16 + 1) = pack8(v + 8);
-          if (p.snap) {
-            // training: the backward's copy S' - 1 S'[0] (as the state pass
-            // below writes it), S'[0] = exp(r_0) S[0] with S[0] staged at the
-            // end of the previous tile; row 0 itself goes out in fp32
-            const size_t tile = (size_t)bh * ntiles_all + c;
+          if (centre) {
+            // S'[0] = exp(r_0) S[0], S[0] staged at the end of the previous
+            // tile (row 0 itself comes out exactly zero); row 0 in fp32 to
+            // the epilogue and to the backward
             const float d0 = s_dec[0];
             const float4 *r0 = reinterpret_cast<const float4 *>(s_row0 + c16 * 16);
             float w[16];
@@ -678,15 +691,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
               w[4 * q4 + 2] = v[4 * q4 + 2] - __fmul_rn(x.z, d0);
               w[4 * q4 + 3] = v[4 * q4 + 3] - __fmul_rn(x.w, d0);
             }
-            uint4 *dst = reinterpret_cast<uint4 *>(p.snap + (tile * D + i) * D + c16 * 16);
-            dst[0] = pack8(w);
-            dst[1] = pack8(w + 8);
+            *chunk_ptr(sm, R_XQ, i, 2 * c16) = pack8(w);
+            *chunk_ptr(sm, R_XQ, i, 2 * c16 + 1) = pack8(w + 8);
             if (i == 0) {
+              const size_t tile = (size_t)bh * ntiles_all + c;
               float4 *d4 = reinterpret_cast<float4 *>(p.snap_r0 + tile * D + c16 * 16);
+              float4 *s4 = reinterpret_cast<float4 *>(s_r0v + c16 * 16);
 #pragma unroll
-              for (int q4 = 0; q4 < 4; ++q4)
-                d4[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+              for (int q4 = 0; q4 < 4; ++q4) {
+                const float4 x = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+                d4[q4] = x;
+                s4[q4] = x;
+              }
             }
+          } else {
+            *chunk_ptr(sm, R_XQ, i, 2 * c16) = pack8(v);
+            *chunk_ptr(sm, R_XQ, i, 2 * c16 + 1) = pack8(v + 8);
           }
         } else if (p.snap && i == 0) {
 #pragma unroll
@@ -757,6 +777,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
       if (gla && !full)   // the state pass's Kt remainder
         for (int s = 0; s < 8; ++s) mma_ss(tb + C_S, desc_mn(sbase + R_KP, s), desc_mn(v, s), id_st, 1);
       mma_commit(&bar_m3);
+      if (centre) {   // the backward's copy of S' - 1 S'[0]: the swizzled tile as it stands
+        const int tile = bh * ntiles_all + c;
+        tma_store_3d(&p.msnap, sm + R_XQ, 0, 0, tile);
+        tma_store_3d(&p.msnap, sm + R_XQ + REG, 64, 0, tile);
+        bulk_commit();
+      }
     }
     // stage-1 loss: this thread's half-row of the target, in flight during MMA 3
     uint4 ytgt[8];
@@ -768,18 +794,33 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
     ok = mbar_wait(&bar_m3, par, err, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) { s_fail = 1; break; }
     tc_fence_after();
-    if (tid == 0 && c + 1 < cend) issue_tile_loads(p, sm, s_rt, &bar_tma, bh, t0 + T, full);
+    if (tid == 0 && c + 1 < cend) {
+      if (centre) bulk_wait_read();   // the copy's store has read X_q's place
+      issue_tile_loads(p, sm, s_rt, &bar_tma, bh, t0 + T, full);
+    }
 
     // ---------------------------- epilogue (column half per group) ---
     if (full) {
       // tcgen05.ld is warp-collective: every lane loads, valid rows store
       const size_t roff = ((size_t)bh * p.L + (qvalid ? tq : 0)) * D;
       const float oscale = s_oscale[row];
+      const float qs = centre ? s_qsum[0][row] + s_qsum[1][row] : 0.f;   // (sum_i Qt[i]) S'[0] left out of MMA 3
 #pragma unroll(LOSS ? 4 : 1)
       for (int k4 = 0; k4 < 4; ++k4) {
         const int c16 = 4 * wg + k4;
         float v[16];
         tmem_ld16(tl + C_O + c16 * 16, v);
+        if (centre) {
+          const float4 *r4 = reinterpret_cast<const float4 *>(s_r0v + c16 * 16);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const float4 x = r4[q4];
+            v[4 * q4] = fmaf(qs, x.x, v[4 * q4]);
+            v[4 * q4 + 1] = fmaf(qs, x.y, v[4 * q4 + 1]);
+            v[4 * q4 + 2] = fmaf(qs, x.z, v[4 * q4 + 2]);
+            v[4 * q4 + 3] = fmaf(qs, x.w, v[4 * q4 + 3]);
+          }
+        }
 #pragma unroll
         for (int u = 0; u < 16; ++u) v[u] *= oscale;
         if (swa && p.meta_v) {
@@ -817,7 +858,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
         }
       }
     }
-    if (full && gla && p.snap && (warp & 3) == 0 && c + 1 < cend) {
+    if (centre && (warp & 3) == 0 && c + 1 < cend) {
       // row 0 of the state this tile leaves: the next tile's centre
       for (int c16 = 4 * wg; c16 < 4 * wg + 4; ++c16) {
         float v[16];
@@ -879,6 +920,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
     // let whatever was issued drain before the shared memory is released
     mbar_wait(&bar_tma, 0, nullptr, 0, 1u << 16);
   }
+  if (centre && tid == 0) bulk_wait_all();   // the state copies' stores are complete
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tb, 512);
@@ -1206,6 +1248,8 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, int stage, cudaStream_t s) {
   if (gla && a.snap && stage == 2) {   // training: the backward's state copies and final state
     p.snap = static_cast<__nv_bfloat16 *>(a.snap);
     p.snap_r0 = reinterpret_cast<float *>(p.snap + (size_t)a.BH * ((a.L + T - 1) / T) * D * D);
+    if (!make_map_bf16_3d(&p.msnap, a.snap, D, D, (uint64_t)a.BH * ((a.L + T - 1) / T), T))
+      return cudaErrorInvalidValue;
     p.state_keep = a.state_keep;
   }
   if (a.branch != 1 && stage == 2) p.lse_keep = a.lse_keep;

@@ -454,7 +454,7 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
                v8[6] * b1.z + v8[7] * b1.w;
     }
   }
-#pragma unroll
+#pragma unroll 1
   for (int m = 0; m < 2; ++m) {
     float ph[F];
     const float s = feature_half(tl + (m == 0 ? C_ZQ : C_ZK), wg, ph);
@@ -571,6 +571,7 @@ __global__ void __launch_bounds__(NT_TILE, 1) tc_gla_bwd_tile_kernel(const __gri
     unsigned char *st0 = sm + R_V;
     // rank-one parts of GQ and GK left out of the S' and dS copies
     const float cq = s_r1[0][row], ck = s_r1[1][row], kap = s_r1[2][row];
+#pragma unroll 1
     for (int c16 = 4 * wg; c16 < 4 * wg + 4; ++c16) {
       float gq[16], gk[16], q16[16], k16[16], lo[16];
       tmem_ld16x2(tl + C_GQ + c16 * 16, tl + C_GK + c16 * 16, gq, gk);
