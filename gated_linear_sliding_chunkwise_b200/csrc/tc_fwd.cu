@@ -151,7 +151,8 @@ __device__ __forceinline__ void issue_tile_loads(const Params &p, unsigned char 
 }
 
 // Qt for dimensions 64 h .. 64 h + 63: phi_q E gscale, bf16 pairs into TMEM.
-// With `sum`, returns the sum of the stored (bf16-rounded) values.
+// With `sum`, returns the sum of the values (before their bf16 rounding,
+// whose share of the sum is of the order of the MMAs' own rounding).
 __device__ __forceinline__ float qt_half(unsigned char *sm, uint32_t tl, int row, int h, float gscale, bool sum) {
   float ph[F];
   const float s = feature_half(tl + C_ZQ, h, ph) * gscale;
@@ -164,10 +165,11 @@ __device__ __forceinline__ float qt_half(unsigned char *sm, uint32_t tl, int row
     uint32_t r8[8];
 #pragma unroll
     for (int u = 0; u < 16; u += 2) {
-      r8[u / 2] = pack_bf16(ph[16 * c16 + u] * e16[u] * s, ph[16 * c16 + u + 1] * e16[u + 1] * s);
+      const float a = ph[16 * c16 + u] * e16[u] * s, b = ph[16 * c16 + u + 1] * e16[u + 1] * s;
+      r8[u / 2] = pack_bf16(a, b);
       if (sum) {
-        acc[0] += __uint_as_float(r8[u / 2] << 16);
-        acc[1] += __uint_as_float(r8[u / 2] & 0xffff0000u);
+        acc[0] += a;
+        acc[1] += b;
       }
     }
     tmem_st8(tl + C_QT + 32 * h + 8 * c16, r8);
@@ -323,7 +325,7 @@ constexpr int BAR_B = 2;       // both groups' row sums written, all logits read
 // Kernel instances: the full pass, the full pass that also forms the
 // stage-1 loss (p.target set), and the state pass.  Each keeps its own
 // register budget.
-constexpr int K_FULL = 0, K_LOSS = 1, K_STATE = 2;
+constexpr int K_FULL = 0, K_LOSS = 1, K_STATE = 2, K_TRAIN = 3;   // K_TRAIN: full pass + the backward's copies
 template <int KIND>
 __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_constant__ Params p) {
   constexpr bool LOSS = KIND == K_LOSS;
@@ -360,7 +362,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
   // Training: MMA 3 reads S' as the bf16 copy of S' - 1 S'[0] (rows less
   // their first; the epilogue adds back (sum_i Qt[i]) S'[0] in fp32), and
   // that copy goes to the backward as is, with one TMA store per tile.
-  const bool centre = full && gla && p.snap != nullptr;
+  const bool centre = KIND == K_TRAIN && gla;
   const uint32_t sbase = smem_u32(sm);
   const int ntiles_all = (p.L + T - 1) / T;
   const int cbeg = marked ? 0 : seg * p.tiles_per_seg;
@@ -605,10 +607,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
           tmem_st8(tl + C_P + ch * 16, zero);
           tmem_st8(tl + C_P + ch * 16 + 8, zero);
         }
-        if (wg == 0 && qvalid && (p.lse || p.lse_keep)) {
+        float *lse_keep = KIND == K_TRAIN ? p.lse_keep : nullptr;
+        if (wg == 0 && qvalid && (p.lse || lse_keep)) {
           const float lse = mx + logf(lsum);
           if (p.lse) p.lse[(size_t)bh * p.L + tq] = lse;
-          if (p.lse_keep) p.lse_keep[(size_t)bh * p.L + tq] = lse;
+          if (lse_keep) lse_keep[(size_t)bh * p.L + tq] = lse;
         }
       }
       // GLA operands carry l/alpha so that one accumulator holds both terms
@@ -1304,6 +1307,8 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, int stage, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(tc_fwd_kernel<K_LOSS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(tc_fwd_kernel<K_TRAIN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(tc_fwd_kernel<K_STATE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) configured[dev] = SMEM_BYTES;
@@ -1319,6 +1324,8 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, int stage, cudaStream_t s) {
     }
     if (p.target)
       tc_fwd_kernel<K_LOSS><<<dim3(a.BH, nseg), NTHREADS, SMEM_BYTES, s>>>(p);
+    else if (p.snap)
+      tc_fwd_kernel<K_TRAIN><<<dim3(a.BH, nseg), NTHREADS, SMEM_BYTES, s>>>(p);
     else
       tc_fwd_kernel<K_FULL><<<dim3(a.BH, nseg), NTHREADS, SMEM_BYTES, s>>>(p);
   }
