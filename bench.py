@@ -201,9 +201,10 @@ class ClockSampler:
 # DRAM bytes (read + write) per launch from ncu captures of the current
 # kernels on the train_step workload (profiles/train_step_tc_launches.md,
 # profiles/tc_gla_bwd_tile_kernel_train_step.md); "step" sums one training
-# step's 17 launches.
+# step's 15 launches (forward with the saved buffer, backward reading it).
 MEASURED_TRAFFIC = {
-    "tc_gla_bwd_tile_kernel": 1_852_018_912,
+    "step": 7_671_755_776,
+    "tc_gla_bwd_tile_kernel": 1_852_190_208,
 }
 
 
