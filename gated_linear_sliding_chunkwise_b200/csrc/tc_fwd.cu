@@ -567,15 +567,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
           float v[32];
           tmem_ld32(tl + C_L + ch * 32, v);
           const bool inner = 32 * ch >= in_lo && 32 * ch + 31 <= 32 * w4 + T && 32 * ch + cbase >= -p.P;
+          // one masked copy of the loop (interior chunks: bounds that pass every column)
+          const int lo_e = inner ? -1 : lo_c - 32 * ch, hi_e = inner ? 32 : hi_c - 32 * ch;
 #pragma unroll
           for (int u = 0; u < 32; u += 2) {
             float e0 = __expf(fmaf(v[u], p.scale, -mx));
             float e1 = __expf(fmaf(v[u + 1], p.scale, -mx));
-            if (!inner) {
-              const int cl = 32 * ch + u;
-              e0 = (cl >= lo_c && cl <= hi_c) ? e0 : 0.f;
-              e1 = (cl + 1 >= lo_c && cl + 1 <= hi_c) ? e1 : 0.f;
-            }
+            e0 = (u >= lo_e && u <= hi_e) ? e0 : 0.f;
+            e1 = (u + 1 >= lo_e && u + 1 <= hi_e) ? e1 : 0.f;
             s4[(u >> 1) & 3] += e0 + e1;
             pk[k][u / 2] = alpha != 0.f ? pack_bf16(e0, e1) : 0u;
           }
