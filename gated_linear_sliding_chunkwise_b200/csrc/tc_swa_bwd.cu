@@ -233,6 +233,7 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
     const int full_hi = split ? ch_hi - 1 : ch_hi;
     const int hcol = 32 * ch_hi + 16 * (1 - wg);
     const bool hinner = hcol >= in_lo && hcol + 15 <= 32 * w4 + T && hcol + cbase >= -p.P;
+    const int lo_h = hinner ? -1 : lo_c - hcol, hi_h = hinner ? 16 : hi_c - hcol;   // the half's exponent mask
     if (given) {
       mx = lse_row;
     } else {
@@ -281,11 +282,8 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
       for (int u = 0; u < 16; u += 2) {
         float e0 = __expf(fmaf(v[u], p.scale, -mx));
         float e1 = __expf(fmaf(v[u + 1], p.scale, -mx));
-        if (!hinner) {
-          const int cl = hcol + u;
-          e0 = (cl >= lo_c && cl <= hi_c) ? e0 : 0.f;
-          e1 = (cl + 1 >= lo_c && cl + 1 <= hi_c) ? e1 : 0.f;
-        }
+        e0 = (u >= lo_h && u <= hi_h) ? e0 : 0.f;
+        e1 = (u + 1 >= lo_h && u + 1 <= hi_h) ? e1 : 0.f;
         s4[(u >> 1) & 3] += e0 + e1;
         d4[(u >> 1) & 3] = fmaf(e0, dp[u], fmaf(e1, dp[u + 1], d4[(u >> 1) & 3]));
         pkh[u / 2] = pack_bf16(e0, e1);
