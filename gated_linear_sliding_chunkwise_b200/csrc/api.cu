@@ -143,9 +143,10 @@ SavedLayout saved_layout(const lizard_fwd_args *a) {
   return l;
 }
 
-// Whether the backward reads a training forward's saved tensors.
-bool bwd_reads_saved(const lizard_fwd_args *a, int impl, bool stage1) {
-  return !stage1 && a->saved != nullptr && fwd_keeps(a) && bwd_gla_uses_tc_impl(a, impl);
+// Whether the backward reads a training forward's saved tensors (the
+// stage-1 step points fwd.saved at a region of its own workspace).
+bool bwd_reads_saved(const lizard_fwd_args *a, int impl) {
+  return a->saved != nullptr && fwd_keeps(a) && bwd_gla_uses_tc_impl(a, impl);
 }
 
 // Forward workspace: the status header, plus fp32 scratch for the portable path.
@@ -212,7 +213,7 @@ BwdLayout bwd_layout(const lizard_fwd_args *a, int impl, bool stage1 = false) {
   if (gla_on(a) && bwd_gla_uses_tc(a, impl)) {
     // with a training forward's saved tensors, the state copies S', the
     // fp32 factors E and the tile decays come from there
-    const bool saved = bwd_reads_saved(a, impl, stage1);
+    const bool saved = bwd_reads_saved(a, impl);
     const size_t snap = up(lz::tc_gla_bwd_snapshot_bytes((int)BH, a->L));
     if (!saved) { l.snap_s = off; off += snap; }
     l.snap_ds = off; off += snap;
@@ -381,9 +382,11 @@ void fwd_plan(const lizard_fwd_args *a, void *ws, cudaStream_t s, Plan &plan, co
     // wide decay: the gate prep marks the sequences, whose GLA branch the
     // full pass then runs as the exact recurrence
     if (lay.fallback) t.seqflag = at<uint32_t>(ws, lay.flags);
-    if (a->saved && !target && fwd_keeps(a)) {   // training: keep what the backward would recompute
+    if (a->saved && fwd_keeps(a)) {   // training: keep what the backward would recompute
       const SavedLayout sv = saved_layout(a);
-      t.seqflag = at<uint32_t>(a->saved, sv.flags);
+      // the stage-1 step (target set) forms its loss in the epilogue, so it
+      // marks no sequence for the exact recurrence
+      if (!target) t.seqflag = at<uint32_t>(a->saved, sv.flags);
       t.keep_r = at<float>(a->saved, sv.r);
       t.keep_e32 = at<float>(a->saved, sv.e32);
       t.snap = at<void>(a->saved, sv.snap);
@@ -428,7 +431,7 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan, bo
                     a->L, a->M, a->window, 0, inv_tau, scale_of(a), scalar_gate(a)};
     f.dstate_out = b->dstate_out;   // the state copies also form the final state's share of dg
     f.kap = at<float>(ws, lay.kap);
-    const bool saved = bwd_reads_saved(a, b->impl, stage1);
+    const bool saved = bwd_reads_saved(a, b->impl);
     const SavedLayout sv = saved_layout(a);
     void *snap_s = saved ? at<void>(a->saved, sv.snap) : at<void>(ws, lay.snap_s);
     float *e32 = saved ? at<float>(a->saved, sv.e32) : at<float>(ws, lay.e32);
@@ -574,7 +577,7 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan, bo
     t.dv_prefix = b->dv_prefix;
     t.P = a->prefix_len;
     // the training forward's softmax normalisers spare the dq pass its max pass
-    if (bwd_reads_saved(a, b->impl, stage1)) t.lse_in = at<float>(a->saved, saved_layout(a).lse);
+    if (bwd_reads_saved(a, b->impl)) t.lse_in = at<float>(a->saved, saved_layout(a).lse);
     plan.add("tc_swa_bwd_q_kernel", [=](cudaStream_t s) { return lz::launch_tc_swa_bwd(t, 0, s); });
     if (a->M > 0 && (b->dmeta_k || b->dmeta_v)) {   // beside the dk / dv pass, after the dq pass's terms
       plan.fork();
@@ -767,7 +770,7 @@ lizard_status lizard_attn_bwd(const lizard_bwd_args *b, lizard_stream_t stream) 
   if (a->prefix_len > 0 && (!b->dk_prefix || !b->dv_prefix)) return LIZARD_ERR_INVALID_ARG;
   const BwdLayout lay = bwd_layout(a, b->impl);
   if (!b->workspace || b->workspace_bytes < lay.total) return LIZARD_ERR_WORKSPACE;
-  if (bwd_reads_saved(a, b->impl, false) && a->saved_bytes < saved_layout(a).total) return LIZARD_ERR_WORKSPACE;
+  if (bwd_reads_saved(a, b->impl) && a->saved_bytes < saved_layout(a).total) return LIZARD_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (bwd_zero_outputs(b, s) != cudaSuccess) return LIZARD_ERR_CUDA;
   if (a->L == 0) return LIZARD_OK;
@@ -781,25 +784,39 @@ lizard_status lizard_attn_bwd(const lizard_bwd_args *b, lizard_stream_t stream) 
 // ---------------------------------------------------------- stage 1 ----
 // One workspace for the whole step: the forward's and the backward's scratch
 // share its start (the backward begins after the forward's last kernel, and
-// both keep the status word at offset 0), then dL/do, then the output when
-// the portable forward needs one and the caller gave none.
+// both keep the status word at offset 0), then dL/do, then the forward's
+// saved-for-backward tensors when both GLA halves run on the tensor cores,
+// then the output when the portable forward needs one and the caller gave
+// none.
 }  // extern "C"
 
 namespace {
 
+// Whether the step's forward keeps the backward's tensors (the forward's
+// GLA branch on the tensor cores and the backward's GLA kernels too).
+bool s1_keeps(const lizard_stage1_args *a) {
+  return fwd_keeps(&a->bwd.fwd) && bwd_gla_uses_tc_impl(&a->bwd.fwd, a->bwd.impl);
+}
+
 struct S1Layout {
-  size_t dmse, o, total;
+  size_t dmse, saved, saved_bytes, o, total;
 };
 S1Layout s1_layout(const lizard_stage1_args *a) {
   const lizard_bwd_args *b = &a->bwd;
-  const lizard_fwd_args *f = &b->fwd;
-  const size_t fw = fwd_layout(f, true).total, bw = bwd_layout(f, b->impl, true).total;
-  const size_t nel = (size_t)f->B * f->H * f->L * f->dv, esz = f->dtype == LIZARD_BF16 ? 2 : 4;
+  lizard_fwd_args f = b->fwd;   // the caller's fwd.saved is not used: the step keeps its own
+  f.saved = s1_keeps(a) ? reinterpret_cast<void *>(16) : nullptr;
+  const size_t fw = fwd_layout(&f, true).total, bw = bwd_layout(&f, b->impl, true).total;
+  const size_t nel = (size_t)f.B * f.H * f.L * f.dv, esz = f.dtype == LIZARD_BF16 ? 2 : 4;
   S1Layout l{};
   size_t off = up(fw > bw ? fw : bw);
   l.dmse = off;
   off += up(nel * esz);
-  if (!f->o && !fwd_uses_tc(f)) {
+  if (f.saved) {
+    l.saved = off;
+    l.saved_bytes = saved_layout(&f).total;
+    off += up(l.saved_bytes);
+  }
+  if (!f.o && !fwd_uses_tc(&f)) {
     l.o = off;
     off += up(nel * esz);
   }
@@ -828,7 +845,9 @@ struct S1Views {
 void stage1_plan(const lizard_stage1_args *a, S1Views &v, void *ws, cudaStream_t s, Plan &plan) {
   const S1Layout lay = s1_layout(a);
   v.b = a->bwd;
-  v.f = a->bwd.fwd;
+  v.b.fwd.saved = lay.saved_bytes ? at<void>(ws, lay.saved) : nullptr;
+  v.b.fwd.saved_bytes = lay.saved_bytes;
+  v.f = v.b.fwd;
   v.f.workspace = ws;
   void *dmse = at<void>(ws, lay.dmse);
   const lizard_fwd_args *f = &v.f;

@@ -323,12 +323,14 @@ constexpr int BAR_A = 1;       // both groups' row maxima written
 constexpr int BAR_B = 2;       // both groups' row sums written, all logits read
 
 // Kernel instances: the full pass, the full pass that also forms the
-// stage-1 loss (p.target set), and the state pass.  Each keeps its own
-// register budget.
-constexpr int K_FULL = 0, K_LOSS = 1, K_STATE = 2, K_TRAIN = 3;   // K_TRAIN: full pass + the backward's copies
+// stage-1 loss (p.target set), the state pass, and the two full passes that
+// also keep the backward's tensors (p.snap set: K_TRAIN, and K_TRAIN_LOSS
+// for the stage-1 step).  Each keeps its own register budget.
+constexpr int K_FULL = 0, K_LOSS = 1, K_STATE = 2, K_TRAIN = 3, K_TRAIN_LOSS = 4;
 template <int KIND>
 __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_constant__ Params p) {
-  constexpr bool LOSS = KIND == K_LOSS;
+  constexpr bool LOSS = KIND == K_LOSS || KIND == K_TRAIN_LOSS;
+  constexpr bool TRAIN = KIND == K_TRAIN || KIND == K_TRAIN_LOSS;
   extern __shared__ unsigned char smraw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
   __shared__ __align__(16) float s_mk[MAXM][D];
@@ -362,7 +364,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
   // Training: MMA 3 reads S' as the bf16 copy of S' - 1 S'[0] (rows less
   // their first; the epilogue adds back (sum_i Qt[i]) S'[0] in fp32), and
   // that copy goes to the backward as is, with one TMA store per tile.
-  const bool centre = KIND == K_TRAIN && gla;
+  const bool centre = TRAIN && gla;
   const uint32_t sbase = smem_u32(sm);
   const int ntiles_all = (p.L + T - 1) / T;
   const int cbeg = marked ? 0 : seg * p.tiles_per_seg;
@@ -604,7 +606,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
           tmem_st8(tl + C_P + ch * 16, zero);
           tmem_st8(tl + C_P + ch * 16 + 8, zero);
         }
-        float *lse_keep = KIND == K_TRAIN ? p.lse_keep : nullptr;
+        float *lse_keep = TRAIN ? p.lse_keep : nullptr;
         if (wg == 0 && qvalid && (p.lse || lse_keep)) {
           const float lse = mx + logf(lsum);
           if (p.lse) p.lse[(size_t)bh * p.L + tq] = lse;
@@ -1306,6 +1308,9 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, int stage, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(tc_fwd_kernel<K_TRAIN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(tc_fwd_kernel<K_TRAIN_LOSS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(tc_fwd_kernel<K_STATE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) configured[dev] = SMEM_BYTES;
@@ -1319,7 +1324,9 @@ cudaError_t launch_tc_fwd(const TcFwdArgs &a, int stage, cudaStream_t s) {
       --g_inject_wait;
       p.inject = 1;
     }
-    if (p.target)
+    if (p.target && p.snap)
+      tc_fwd_kernel<K_TRAIN_LOSS><<<dim3(a.BH, nseg), NTHREADS, SMEM_BYTES, s>>>(p);
+    else if (p.target)
       tc_fwd_kernel<K_LOSS><<<dim3(a.BH, nseg), NTHREADS, SMEM_BYTES, s>>>(p);
     else if (p.snap)
       tc_fwd_kernel<K_TRAIN><<<dim3(a.BH, nseg), NTHREADS, SMEM_BYTES, s>>>(p);

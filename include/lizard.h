@@ -315,7 +315,10 @@ lizard_status lizard_chain_states(const lizard_chain_args *args, lizard_stream_t
  *            and bwd.fwd.o may be NULL (the output is then not kept) or
  *            receives o.  bwd.fwd.impl selects the forward's kernels,
  *            bwd.impl the backward's.  bwd.workspace and bwd.launch_events
- *            serve the whole step; bwd.fwd.saved is ignored.
+ *            serve the whole step; bwd.fwd.saved is ignored: when both
+ *            halves run the GLA branch on the tensor cores, the step keeps
+ *            the forward's saved-for-backward tensors (see "Saved for the
+ *            backward") in its own workspace, and its backward reads them.
  *   target   [B, H, L, dv] dtype: the teacher's attention output y
  *   loss     one fp32, written: sum over every element of (o - y)^2 divided
  *            by the element count B H L dv; dL/do = 2 (o - y) / (B H L dv)

@@ -260,8 +260,9 @@ def test_stage1_rejects_bad_arguments_on_host(lz):
 
 
 def test_stage1_launch_plan_fuses_the_loss_on_tensor_cores(lz):
-    """The tensor-core forward forms the loss in its epilogue; the portable
-    forward adds one elementwise kernel before the backward."""
+    """The tensor-core forward forms the loss in its epilogue and keeps the
+    backward's tensors; the portable forward adds one elementwise kernel
+    before the backward."""
     import ctypes as ct
     for impl, fused in ((lz.IMPL_TC, True), (lz.IMPL_SIMT, False)):
         a = _stage1(lz)
@@ -272,6 +273,9 @@ def test_stage1_launch_plan_fuses_the_loss_on_tensor_cores(lz):
         got = [names[i].decode() for i in range(n)]
         assert ("mse_kernel" in got) != fused, got
         assert "gate_grad_kernel" in got or "finish_bwd" in got, got
+        if fused:   # the backward reads the forward's saved tensors: no second gate or state pass
+            assert got.count("gate_prep_kernel") == 1, got
+            assert "tc_fwd_kernel(state copies)" not in got, got
 
 
 # ------------------------------------------------- sequence parallelism ---
