@@ -85,7 +85,6 @@ def kernel_model(name, w, N, BH, train=False):
     snaps = BH * nt * d * d * 2          # one bf16 d x d state per 128-token tile
     nseg = tc_segments(BH, w.L)
     seg_states = BH * nseg * d * d * 4
-    mw = 16                               # per-row meta buffers [N][16] fp32
     table = {
         # portable kernels
         "prep_kernel": (3 * Nd * esz + 3 * Nd * 4, N * phi),
@@ -112,9 +111,8 @@ def kernel_model(name, w, N, BH, train=False):
         "tc_gla_bwd_tile_kernel": (4 * Nd * esz + 2 * snaps + Nd * 4 + 2 * Nd * 4 + 2 * Nd * 2,
                                    N * (2 * fl["gla_fwd"] + phi)),
         "tc_finish_kernel": (4 * Nd * esz + 2 * Nd * 2, N * 3 * phi),
-        "tc_swa_bwd_q_kernel": (6 * Nd * esz + 2 * N * 4 + 2 * N * mw * 4, N * 1.5 * fl["swa_fwd"]),
+        "tc_swa_bwd_q_kernel": (6 * Nd * esz + 2 * N * 4, N * (1.5 * fl["swa_fwd"] + 4 * d * w.M)),
         "tc_swa_bwd_kv_kernel": (7 * Nd * esz + Nd * 4 + 2 * N * 4, N * 2.0 * fl["swa_fwd"]),
-        "meta_grad_kernel": (2 * Nd * esz + 2 * N * mw * 4, N * 4 * d * w.M),
         "gate_grad_kernel": (Nd * 4 + Nd * esz + Nd * 4, 0),
     }
     return table.get(name, (0, 0))

@@ -188,7 +188,7 @@ bool bwd_swa_uses_tc(const lizard_fwd_args *a, int impl) {
 bool bwd_gla_uses_tc(const lizard_fwd_args *a, int impl) { return bwd_gla_uses_tc_impl(a, impl); }
 
 struct BwdLayout {
-  size_t phq, phk, a, sprev, dphq, dphk, da, dv_gla, dq_swa, dk_swa, dv_swa, lse, Dterm, dsm, pm, snap_s,
+  size_t phq, phk, a, sprev, dphq, dphk, da, dv_gla, dq_swa, dk_swa, dv_swa, lse, Dterm, snap_s,
       snap_ds, e32, gr, colsum, w16, kap, total;
   bool fallback;
   FallbackLayout fb;
@@ -245,10 +245,6 @@ BwdLayout bwd_layout(const lizard_fwd_args *a, int impl, bool stage1 = false) {
     l.dv_swa = off; off += nv;
     l.lse = off; off += up(N * sizeof(float));
     l.Dterm = off; off += up(N * sizeof(float));
-    if (bwd_swa_uses_tc(a, impl)) {
-      l.dsm = off; off += up(N * 16 * sizeof(float));
-      l.pm = off; off += up(N * 16 * sizeof(float));
-    }
   }
   l.total = off;
   return l;
@@ -559,8 +555,8 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan, bo
   if (swa_tc) {
     lz::TcSwaBwdArgs t{a->q, a->k, a->v, b->dout, a->meta_k, a->meta_v, a->alpha,
                        at<float>(ws, lay.dq_swa), at<float>(ws, lay.dk_swa), at<float>(ws, lay.dv_swa),
-                       at<float>(ws, lay.lse), at<float>(ws, lay.Dterm), at<float>(ws, lay.dsm),
-                       at<float>(ws, lay.pm), b->dmeta_k, b->dmeta_v, b->dalpha, static_cast<uint32_t *>(ws),
+                       at<float>(ws, lay.lse), at<float>(ws, lay.Dterm), b->dmeta_k, b->dmeta_v, b->dalpha,
+                       static_cast<uint32_t *>(ws),
                        a->B, a->H, BH, a->L, a->M, a->window, scale_of(a)};
     if (fused) {
       t.dq = t.dk = t.dv = nullptr;
@@ -579,10 +575,6 @@ void bwd_plan(const lizard_bwd_args *b, void *ws, cudaStream_t s, Plan &plan, bo
     // the training forward's softmax normalisers spare the dq pass its max pass
     if (bwd_reads_saved(a, b->impl)) t.lse_in = at<float>(a->saved, saved_layout(a).lse);
     plan.add("tc_swa_bwd_q_kernel", [=](cudaStream_t s) { return lz::launch_tc_swa_bwd(t, 0, s); });
-    if (a->M > 0 && (b->dmeta_k || b->dmeta_v)) {   // beside the dk / dv pass, after the dq pass's terms
-      plan.fork();
-      plan.add("meta_grad_kernel", [=](cudaStream_t s) { return lz::launch_tc_swa_bwd(t, 2, s); }, 1);
-    }
     plan.add("tc_swa_bwd_kv_kernel", [=](cudaStream_t s) { return lz::launch_tc_swa_bwd(t, 1, s); });
     plan.join();
   } else if (w) {

@@ -183,8 +183,7 @@ struct TcSwaBwdArgs {
   const float *meta_k, *meta_v, *alpha;
   float *dq, *dk, *dv;          // anchor-branch parts, fp32 [B*H*L][128]
   float *lse, *Dterm;           // [B*H*L]
-  float *dsm, *pm;              // per-row meta-token terms, [B*H*L][16]
-  float *dmeta_k, *dmeta_v, *dalpha;
+  float *dmeta_k, *dmeta_v, *dalpha;   // accumulated by the dq pass
   uint32_t *status;
   int B, H, BH, L, M, window;
   float scale;

@@ -9,7 +9,10 @@
 //
 // tc_swa_bwd_q_kernel   one CTA per (sequence, 128-query tile): logits and
 //                       softmax again, o_swa = P V for D, dP, dS, dq; writes
-//                       dq, the log-normaliser, D and the per-row meta terms.
+//                       dq, the log-normaliser and D, and adds the tile's
+//                       terms of the meta-token gradients
+//                       (dmeta_k += scale sum_t dS_meta[t] q_t,
+//                       dmeta_v += alpha sum_t p_meta[t] dout_t).
 // tc_swa_bwd_kv_kernel  one CTA per (sequence, 128-key block): the two query
 //                       tiles that see the block; dK and dV accumulate in TMEM.
 //
@@ -17,7 +20,6 @@
 // longer sequence) enters the first query tile's band as its previous keys
 // and values, and adds one key block per sequence (keys -128 .. -1, of which
 // -P .. -1 exist) whose gradients go to dk_prefix / dv_prefix.
-// meta_grad_kernel      meta-token gradients: per head, sums over tokens.
 //
 // Every mbarrier wait is bounded; a wait that gives up sets the TIMEOUT bit
 // of the status word and the CTA leaves after freeing its TMEM.
@@ -44,7 +46,8 @@ struct QParams {
   CUtensorMap mdq;            // fp32 dq output (TMA stores)
   CUtensorMap mxq, mdqo;      // fused: bf16 GLA part dx_q (load), bf16 final dq (store)
   const float *meta_k, *meta_v, *alpha;
-  float *dq, *lse, *Dterm, *dsm, *pm, *dalpha;
+  float *dq, *lse, *Dterm, *dalpha;
+  float *dmeta_k, *dmeta_v;   // meta-token gradients [H][M][D], accumulated (null: not wanted)
   const float *lse_in;        // the forward's softmax normalisers (null: formed here, into lse)
   uint32_t *status;
   int H, L, M, window;
@@ -88,6 +91,62 @@ __device__ __forceinline__ void setup_cta(uint32_t *tmem_slot, uint64_t *bars, i
 // and dq', and the meta dot products (group 0 q . mk, group 1 dO . mv);
 // row sums and maxima meet in shared memory.
 constexpr int NT_Q = 256;
+
+// Meta-token gradient terms of one 128-row tile, for this warp's 32 columns
+// n0 .. n0 + 31: acc[m][n] += sum_r W[m][r] X[r][n] over the tile's rows r
+// (tokens), X the swizzled bf16 tile at region xreg, W the per-row meta
+// weights as bf16 hi + lo planes [MAXM][ld] (rows m >= M read as zero).
+// Warp-level mma.sync m16n8k16: A = W (16 meta rows x 16 tokens per step),
+// B = X (16 tokens x 8 columns, read transposed by ldmatrix.trans), four
+// n-tiles of 8 columns; acc[j] is n-tile j's C fragment (rows g and g + 8,
+// columns 2t, 2t + 1 with g = lane / 4, t = lane % 4).  W enters as hi + lo,
+// so the sums keep about 16 bits of each weight.
+__device__ __forceinline__ void meta_grad_mma(const unsigned char *sm, uint32_t xreg, const __nv_bfloat16 *whi,
+                                              const __nv_bfloat16 *wlo, int ld, int n0, int M, int lane,
+                                              float (&acc)[4][4]) {
+  const int g = lane >> 2, t = lane & 3;
+  const bool r0 = g < M, r1 = g + 8 < M;
+#pragma unroll 2
+  for (int ks = 0; ks < 8; ++ks) {
+    const int k0 = 16 * ks;
+    uint32_t ah[4], al[4];
+    const int e0 = g * ld + k0 + 2 * t, e1 = (g + 8) * ld + k0 + 2 * t;
+    ah[0] = r0 ? *reinterpret_cast<const uint32_t *>(whi + e0) : 0u;
+    ah[1] = r1 ? *reinterpret_cast<const uint32_t *>(whi + e1) : 0u;
+    ah[2] = r0 ? *reinterpret_cast<const uint32_t *>(whi + e0 + 8) : 0u;
+    ah[3] = r1 ? *reinterpret_cast<const uint32_t *>(whi + e1 + 8) : 0u;
+    al[0] = r0 ? *reinterpret_cast<const uint32_t *>(wlo + e0) : 0u;
+    al[1] = r1 ? *reinterpret_cast<const uint32_t *>(wlo + e1) : 0u;
+    al[2] = r0 ? *reinterpret_cast<const uint32_t *>(wlo + e0 + 8) : 0u;
+    al[3] = r1 ? *reinterpret_cast<const uint32_t *>(wlo + e1 + 8) : 0u;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      // matrices: rows k0 .. k0 + 7 | k0 + 8 .. k0 + 15 of columns c .. c + 7,
+      // then the same of columns c + 8 .. c + 15 (c = n0 + 16 j)
+      const int r = k0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+      const int col = n0 + 16 * j + ((lane >> 4) & 1) * 8;
+      const uint32_t addr = smem_u32(sm + xreg + (col >> 6) * kReg + sw128_offset(r, col & 63));
+      uint32_t b[4];
+      asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];\n"
+                   : "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3])
+                   : "r"(addr));
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        float *c = acc[2 * j + u];
+#pragma unroll
+        for (int hl = 0; hl < 2; ++hl) {
+          const uint32_t *a = hl ? al : ah;
+          asm volatile(
+              "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+              "{%0, %1, %2, %3};\n"
+              : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+              : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[2 * u]), "r"(b[2 * u + 1]));
+        }
+      }
+    }
+  }
+}
+
 __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_constant__ QParams p) {
   extern __shared__ unsigned char smraw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
@@ -103,6 +162,12 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
   // TMEM: logits [0,256) then P^ [0,128), dP' [256,512) (issued with the
   // logits), dS [128,256), dq' [0,128)
   constexpr uint32_t C_L = 0, C_P = 0, C_DP = 256, C_DS = 128, C_DQ = 0;
+  // The meta weights of the meta-token gradients (per row: the meta dS for
+  // dmeta_k, the meta probabilities for dmeta_v), bf16 hi + lo planes
+  // [2][2][MAXM][MW_LD], in the V_prev region: only dP' reads V_prev, and
+  // the next item's tiles arrive there after the dq' product.
+  constexpr uint32_t R_MW = R_VP;
+  constexpr int MW_LD = T + 8;   // padded rows: conflict-free fragment loads
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wg = tid >> 7, row = tid & 127;
   const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
@@ -151,6 +216,16 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
   const uint32_t id_kk = idesc_bf16(128, 128, 0, 0);
   const uint32_t id_mn = idesc_bf16(128, 128, 0, 1);
   const int m_rows = (p.M + 3) / 4 * 4;   // meta rows read (groups of four; zero past M)
+  // meta-token gradients: group 0 dmeta_k (rows of Q), group 1 dmeta_v (rows
+  // of dO), each warp 32 columns; summed over the CTA's items of one head in
+  // registers, added to memory when the head changes
+  const bool mgrad = p.M > 0 && (wg == 0 ? p.dmeta_k != nullptr : p.dmeta_v != nullptr);
+  const bool mw_write = p.M > 0 && (p.dmeta_k != nullptr || p.dmeta_v != nullptr);
+  float macc[4][4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) macc[j][u] = 0.f;
   int cur_h = -1;
   bool ok = true;
   for (int w = w0, it = 0; w < w1; ++w, ++it) {
@@ -385,18 +460,27 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
       tmem_st8(tl + C_DS + ch * 16 + 8, ds + 8);
     }
     if (wg == 0) {
+      __nv_bfloat16 *mw = reinterpret_cast<__nv_bfloat16 *>(sm + R_MW);
 #pragma unroll
       for (int m = 0; m < MAXM; ++m) {
         if (m < p.M) {
           const float pm = em[m] * inv_l;
           const float dsm = pm * (alpha * dom[m] - Dt);
           s_x[m][row] = dsm;
-          if (qvalid) {
-            p.dsm[((size_t)bh * p.L + tq) * MAXM + m] = dsm;
-            p.pm[((size_t)bh * p.L + tq) * MAXM + m] = pm;
+          if (mw_write) {   // plane (which, hi | lo): ((which * 2 + hl) * MAXM + m) * MW_LD + row
+            const float wv[2] = {qvalid ? dsm : 0.f, qvalid ? pm : 0.f};
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+              const __nv_bfloat16 hi = __float2bfloat16_rn(wv[which]);
+              const __nv_bfloat16 lo = __float2bfloat16_rn(wv[which] - __bfloat162float(hi));
+              mw[((which * 2 + 0) * MAXM + m) * MW_LD + row] = hi;
+              mw[((which * 2 + 1) * MAXM + m) * MW_LD + row] = lo;
+            }
           }
         }
       }
+      // the next item's tiles overwrite the weights by TMA
+      if (mw_write) fence_proxy_async();
     }
     tmem_st_wait();
     tc_fence_before();
@@ -408,6 +492,12 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
       for (int s = 0; s < 8; ++s) mma_ts(tb + C_DQ, tb + C_DS + s * 8, desc_mn(sbase + R_KP, s), id_mn, s > 0);
       for (int s = 0; s < 8; ++s) mma_ts(tb + C_DQ, tb + C_DS + 64 + s * 8, desc_mn(sbase + R_K, s), id_mn, 1);
       mma_commit(&bars[4]);
+    }
+    // the meta-token gradient terms of this tile while dq' runs (Q and dO
+    // stay in place until the product is done)
+    if (mgrad) {
+      const __nv_bfloat16 *mw = reinterpret_cast<const __nv_bfloat16 *>(sm + R_MW) + (size_t)wg * 2 * MAXM * MW_LD;
+      meta_grad_mma(sm, wg == 0 ? R_Q : R_O, mw, mw + MAXM * MW_LD, MW_LD, 32 * (warp & 3), p.M, lane, macc);
     }
     ok = mbar_wait(&bars[4], par, p.status, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) goto done;
@@ -484,6 +574,24 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
       bulk_commit();
       bulk_wait_read();   // the staging is free once read (the writes need not have landed)
     }
+    }
+  }
+  // this CTA's share of the head's meta-token gradients, once its last item
+  // of the head is done: C rows g and g + 8 (meta tokens), columns 2t, 2t + 1
+  // of each n-tile
+  if (mgrad && (w + 1 >= w1 || ((w + 1) / ntiles) % p.H != h)) {
+    float *out = wg == 0 ? p.dmeta_k : p.dmeta_v;
+    const float f = wg == 0 ? p.scale : alpha;
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = 32 * (warp & 3) + 8 * j + 2 * t;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int m = g + 8 * (u >> 1);
+        if (m < p.M) atomicAdd(out + ((size_t)h * p.M + m) * D + n + (u & 1), f * macc[j][u]);
+        macc[j][u] = 0.f;
+      }
     }
   }
   // the store has read this item's staging: the rest of the next item's tiles
@@ -759,84 +867,6 @@ done:
   if (warp == 0) tmem_dealloc(s_tmem, 512);
 }
 
-// ------------------------------------------------------- meta gradients ---
-// dmeta_k[h][m] += scale sum_t dSm[t][m] q_t ; dmeta_v[h][m] += alpha sum_t pm[t][m] dout_t
-//
-// A streaming reduction over the tokens of one head: each warp walks every
-// 8th token of the CTA's range reading whole 256-byte rows of q and dout
-// (lane = 4 dimensions); the per-row meta terms are broadcast loads.  MM is
-// the meta-token count rounded up to 4, 8 or 16; U tokens are in flight per
-// warp.  Warps combine in shared memory, then one global add per element.
-constexpr int kMetaTok = 256;   // tokens per CTA: enough CTAs that the last wave is a small share
-template <int MM, int U>
-__global__ void __launch_bounds__(256) meta_grad_kernel(const __nv_bfloat16 *q, const __nv_bfloat16 *dout,
-                                                         const float *dsm, const float *pm, const float *alpha,
-                                                         float *dmk, float *dmv, int B, int H, int L, int M,
-                                                         float scale) {
-  __shared__ float s_red[2][MM][D];
-  const int h = blockIdx.y, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int n0 = blockIdx.x * kMetaTok;
-  const int n1 = min(B * L, n0 + kMetaTok);
-  for (int e = threadIdx.x; e < 2 * MM * D; e += 256) (&s_red[0][0][0])[e] = 0.f;
-  float ak[MM][4], av[MM][4];
-#pragma unroll
-  for (int m = 0; m < MM; ++m)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) { ak[m][j] = 0.f; av[m][j] = 0.f; }
-  for (int nb = n0 + warp; nb < n1; nb += 8 * U) {
-    uint2 qv[U], ov[U];
-    float4 ds[U][MM / 4], pw[U][MM / 4];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {       // all loads of U tokens in flight together
-      const int n = nb + 8 * u;
-      const bool in = n < n1;
-      const size_t tok = ((size_t)((in ? n : n0) / L) * H + h) * L + (in ? n : n0) % L;
-      qv[u] = in ? *reinterpret_cast<const uint2 *>(q + tok * D + lane * 4) : make_uint2(0u, 0u);
-      ov[u] = in ? *reinterpret_cast<const uint2 *>(dout + tok * D + lane * 4) : make_uint2(0u, 0u);
-#pragma unroll
-      for (int k = 0; k < MM / 4; ++k) {
-        ds[u][k] = in ? *reinterpret_cast<const float4 *>(dsm + tok * MAXM + 4 * k) : make_float4(0.f, 0.f, 0.f, 0.f);
-        pw[u][k] = in ? *reinterpret_cast<const float4 *>(pm + tok * MAXM + 4 * k) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const float2 q01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&qv[u].x));
-      const float2 q23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&qv[u].y));
-      const float2 o01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ov[u].x));
-      const float2 o23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ov[u].y));
-      const float qf[4] = {q01.x, q01.y, q23.x, q23.y}, of[4] = {o01.x, o01.y, o23.x, o23.y};
-#pragma unroll
-      for (int k = 0; k < MM / 4; ++k) {
-        const float dk4[4] = {ds[u][k].x, ds[u][k].y, ds[u][k].z, ds[u][k].w};
-        const float pv4[4] = {pw[u][k].x, pw[u][k].y, pw[u][k].z, pw[u][k].w};
-#pragma unroll
-        for (int r = 0; r < 4; ++r)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            ak[4 * k + r][j] = fmaf(dk4[r], qf[j], ak[4 * k + r][j]);
-            av[4 * k + r][j] = fmaf(pv4[r], of[j], av[4 * k + r][j]);
-          }
-      }
-    }
-  }
-  __syncthreads();
-#pragma unroll
-  for (int m = 0; m < MM; ++m)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      atomicAdd(&s_red[0][m][lane * 4 + j], ak[m][j]);
-      atomicAdd(&s_red[1][m][lane * 4 + j], av[m][j]);
-    }
-  __syncthreads();
-  const float a = alpha ? alpha[h] : 1.f;
-  for (int e = threadIdx.x; e < M * D; e += 256) {
-    const int m = e / D, i = e % D;
-    if (dmk) atomicAdd(dmk + ((size_t)h * M + m) * D + i, s_red[0][m][i] * scale);
-    if (dmv) atomicAdd(dmv + ((size_t)h * M + m) * D + i, s_red[1][m][i] * a);
-  }
-}
-
 }  // namespace
 
 bool tc_swa_bwd_supported(int dk, int dv, int window, int M, bool bf16) {
@@ -846,22 +876,6 @@ bool tc_swa_bwd_supported(int dk, int dv, int window, int M, bool bf16) {
 cudaError_t launch_tc_swa_bwd(const TcSwaBwdArgs &a, int stage, cudaStream_t s) {
   const int ntiles = (a.L + T - 1) / T;
   const uint64_t rows = (uint64_t)a.L;
-  if (stage == 2) {
-    if (a.M == 0 || (!a.dmeta_k && !a.dmeta_v)) return cudaSuccess;
-    dim3 grid((a.B * a.L + kMetaTok - 1) / kMetaTok, a.H);
-    const auto *qp = static_cast<const __nv_bfloat16 *>(a.q);
-    const auto *op = static_cast<const __nv_bfloat16 *>(a.dout);
-    if (a.M <= 4)
-      meta_grad_kernel<4, 8><<<grid, 256, 0, s>>>(qp, op, a.dsm, a.pm, a.alpha, a.dmeta_k, a.dmeta_v, a.B, a.H,
-                                                  a.L, a.M, a.scale);
-    else if (a.M <= 8)
-      meta_grad_kernel<8, 2><<<grid, 256, 0, s>>>(qp, op, a.dsm, a.pm, a.alpha, a.dmeta_k, a.dmeta_v, a.B, a.H,
-                                                  a.L, a.M, a.scale);
-    else
-      meta_grad_kernel<16, 1><<<grid, 256, 0, s>>>(qp, op, a.dsm, a.pm, a.alpha, a.dmeta_k, a.dmeta_v, a.B, a.H,
-                                                   a.L, a.M, a.scale);
-    return cudaGetLastError();
-  }
   // the attribute is per device: set it every launch on devices not yet seen
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -890,8 +904,8 @@ cudaError_t launch_tc_swa_bwd(const TcSwaBwdArgs &a, int stage, cudaStream_t s) 
     p.lse = a.lse;
     p.lse_in = a.lse_in;
     p.Dterm = a.Dterm;
-    p.dsm = a.dsm;
-    p.pm = a.pm;
+    p.dmeta_k = a.dmeta_k;
+    p.dmeta_v = a.dmeta_v;
     p.dalpha = a.dalpha;
     p.status = a.status;
     p.H = a.H;
