@@ -55,6 +55,10 @@ SWEEP = [
     ("fp32", 64, 150, 1, 0, False, True, False),
     ("bf16", 128, 260, 128, 4, True, True, True),
     ("bf16", 64, 129, 33, 16, True, False, True),
+    # the tensor-core dq pass's meta-token gradients past eight meta tokens
+    # (a second fragment of meta columns), with and without meta values
+    ("bf16", 128, 300, 100, 16, True, False, True),
+    ("bf16", 128, 200, 128, 9, False, True, False),
 ]
 
 
