@@ -106,7 +106,7 @@ __device__ __forceinline__ void meta_grad_mma(const unsigned char *sm, uint32_t 
                                               float (&acc)[4][4]) {
   const int g = lane >> 2, t = lane & 3;
   const bool r0 = g < M, r1 = g + 8 < M;
-#pragma unroll 2
+#pragma unroll
   for (int ks = 0; ks < 8; ++ks) {
     const int k0 = 16 * ks;
     uint32_t ah[4], al[4];
