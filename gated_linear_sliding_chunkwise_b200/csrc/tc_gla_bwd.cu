@@ -722,41 +722,60 @@ done:
 // dg_t = dlogsigmoid(g_t) / tau * sum_{s >= t} dB_s, per (sequence, key
 // dimension), in one pass over dB: the tile kernel leaves each tile's column
 // sums of dB, so the part of the sum beyond a tile (plus the final state's
-// share) is known before the tile is walked.  One CTA per (sequence, 32
-// dimensions): warp w walks tiles w, w + 8, ... backwards (lane = dimension,
-// each token row one coalesced 128-byte read, eight rows in flight).
+// share) is known before the tile is walked.  One CTA per (sequence, 64
+// dimensions): warp w walks tiles w, w + 8, ... backwards (lane = two
+// dimensions, eight token rows in flight).
 constexpr int kGateWarps = 8;
-__global__ void __launch_bounds__(256) gate_grad_kernel(const float *dB, const __nv_bfloat16 *g, float *dg, int L,
-                                                       float inv_tau, const float *kap, const float *colsum) {
+__global__ void __launch_bounds__(256) gate_grad_kernel(const float *__restrict__ dB,
+                                                       const __nv_bfloat16 *__restrict__ g, float *__restrict__ dg,
+                                                       int L, float inv_tau, const float *kap, const float *colsum) {
+  // lane = two adjacent dimensions: a warp reads whole 128-byte lines of g
+  // (32 dimensions per lane left half lines) and 256-byte rows of dB and dg
   const int bh = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int i = blockIdx.y * 32 + lane;
+  const int i = blockIdx.y * 64 + 2 * lane;
   const int ntiles = (L + T - 1) / T;
   const size_t base = (size_t)bh * L * D + i;
   const float *cs = colsum + (size_t)bh * ntiles * D + i;
   // the sum starts with the final state's share (an incoming final-state gradient)
-  const float k0 = kap ? kap[(size_t)bh * 2 * D + i] + kap[((size_t)bh * 2 + 1) * D + i] : 0.f;
+  float2 k0 = make_float2(0.f, 0.f);
+  if (kap) {
+    const float2 a = *reinterpret_cast<const float2 *>(kap + (size_t)bh * 2 * D + i);
+    const float2 b = *reinterpret_cast<const float2 *>(kap + ((size_t)bh * 2 + 1) * D + i);
+    k0 = make_float2(a.x + b.x, a.y + b.y);
+  }
   for (int c = warp; c < ntiles; c += kGateWarps) {
-    float later[4] = {k0, 0.f, 0.f, 0.f};
-    for (int c2 = c + 1; c2 < ntiles; ++c2) later[c2 & 3] += cs[(size_t)c2 * D];
-    float carry = (later[0] + later[1]) + (later[2] + later[3]);
+    float2 later[4] = {k0, make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+    for (int c2 = c + 1; c2 < ntiles; ++c2) {
+      const float2 v = *reinterpret_cast<const float2 *>(cs + (size_t)c2 * D);
+      later[c2 & 3].x += v.x;
+      later[c2 & 3].y += v.y;
+    }
+    float cx = (later[0].x + later[1].x) + (later[2].x + later[3].x);
+    float cy = (later[0].y + later[1].y) + (later[2].y + later[3].y);
     const int ta = c * T, tz = min(L, ta + T);
     int t = tz - 1;
     for (; t - 7 >= ta; t -= 8) {
-      float b[8], gv[8];
+      float2 b[8], gv[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        b[u] = dB[base + (size_t)(t - u) * D];
-        gv[u] = __bfloat162float(g[base + (size_t)(t - u) * D]);
+        b[u] = *reinterpret_cast<const float2 *>(dB + base + (size_t)(t - u) * D);
+        gv[u] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(g + base + (size_t)(t - u) * D));
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        carry += b[u];
-        dg[base + (size_t)(t - u) * D] = carry * dlogsigmoid(gv[u]) * inv_tau;
+        cx += b[u].x;
+        cy += b[u].y;
+        *reinterpret_cast<float2 *>(dg + base + (size_t)(t - u) * D) =
+            make_float2(cx * dlogsigmoid(gv[u].x) * inv_tau, cy * dlogsigmoid(gv[u].y) * inv_tau);
       }
     }
     for (; t >= ta; --t) {
-      carry += dB[base + (size_t)t * D];
-      dg[base + (size_t)t * D] = carry * dlogsigmoid(__bfloat162float(g[base + (size_t)t * D])) * inv_tau;
+      const float2 b = *reinterpret_cast<const float2 *>(dB + base + (size_t)t * D);
+      const float2 gv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(g + base + (size_t)t * D));
+      cx += b.x;
+      cy += b.y;
+      *reinterpret_cast<float2 *>(dg + base + (size_t)t * D) =
+          make_float2(cx * dlogsigmoid(gv.x) * inv_tau, cy * dlogsigmoid(gv.y) * inv_tau);
     }
   }
 }
@@ -953,7 +972,7 @@ cudaError_t launch_tc_gla_bwd(const TcGlaBwdArgs &a, int stage, cudaStream_t s) 
     gate_grad_scalar_kernel<<<a.BH, 256, 0, s>>>(a.dB, static_cast<const __nv_bfloat16 *>(a.g), a.dg, a.L,
                                                  a.inv_tau, a.kap);
   else
-    gate_grad_kernel<<<dim3(a.BH, D / 32), 256, 0, s>>>(a.dB, static_cast<const __nv_bfloat16 *>(a.g), a.dg, a.L,
+    gate_grad_kernel<<<dim3(a.BH, D / 64), 256, 0, s>>>(a.dB, static_cast<const __nv_bfloat16 *>(a.g), a.dg, a.L,
                                                         a.inv_tau, a.kap, a.colsum);
   return cudaGetLastError();
 }
