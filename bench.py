@@ -192,16 +192,14 @@ class ClockSampler:
 
 
 # -------------------------------------------------------------- helpers ----
-# dram__bytes_read.sum + dram__bytes_write.sum of one launch on the
-# train_step workload (B=8, H=32, L=2048), from an ncu capture of the current
-# kernel build ("step" = the sum over every kernel of one training step).
-# Kernels changed since their capture are left out.
-# DRAM bytes (read + write) per launch from ncu captures of the current
-# kernels on the train_step workload (profiles/train_step_tc_launches.md,
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch from
+# ncu captures of the current kernels on the train_step workload (B=8, H=32,
+# L=2048; profiles/train_step_tc_launches.md,
 # profiles/tc_gla_bwd_tile_kernel_train_step.md); "step" sums one training
-# step's 15 launches (forward with the saved buffer, backward reading it).
+# step's 14 launches (forward with the saved buffer, backward reading it).
+# Kernels changed since their capture are left out.
 MEASURED_TRAFFIC = {
-    "step": 7_671_755_776,
+    "step": 7_241_132_032,
     "tc_gla_bwd_tile_kernel": 1_852_190_208,
 }
 
