@@ -261,7 +261,7 @@ cudaError_t launch_gla_bwd_simt(const GlaBwdArgs &a, int BH, int D, bool bf16, c
 cudaError_t launch_swa_bwd_q(const SwaBwdQArgs &a, int BH, int D, bool bf16, cudaStream_t s);
 cudaError_t launch_swa_bwd_kv(const SwaBwdKVArgs &a, int BH, int D, bool bf16, cudaStream_t s);
 bool tc_swa_bwd_supported(int dk, int dv, int window, int M, bool bf16);
-// stage 0: dq pass, 1: dk/dv pass, 2: meta-token gradients
+// stage 0: dq pass (with the meta-token gradients), 1: dk/dv pass
 cudaError_t launch_tc_swa_bwd(const TcSwaBwdArgs &a, int stage, cudaStream_t s);
 size_t tc_gla_bwd_snapshot_bytes(int BH, int L);
 // kap [BH][2][128] from a kept final state S [BH][128][128] and the incoming

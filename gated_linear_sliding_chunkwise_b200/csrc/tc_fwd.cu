@@ -125,15 +125,17 @@ struct Params {
 };
 
 
+// defer_xq: leave X_q's two loads to issue_xq_loads (its region is still being
+// read by a store); the barrier expects their bytes all the same.
 __device__ __forceinline__ void issue_tile_loads(const Params &p, unsigned char *sm, float *s_rt, uint64_t *bar,
-                                                 int bh, int t0, bool full) {
+                                                 int bh, int t0, bool full, bool defer_xq = false) {
   mbar_expect_tx(bar, (full ? 5 : 4) * TILE + (p.gate_r ? D * 4 : 0));
   if (p.gate_r)   // the tile's log-decays r (one 512-byte row)
     bulk_load_1d(s_rt, p.gate_r + ((size_t)bh * ((p.L + T - 1) / T) + t0 / T) * D, D * 4, bar);
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
     if (full) {
-      tma_load_3d(sm + R_XQ + r * REG, &p.mq, bar, 64 * r, t0, bh);
+      if (!defer_xq) tma_load_3d(sm + R_XQ + r * REG, &p.mq, bar, 64 * r, t0, bh);
       // keys of the previous tile; before token 0, the prefix (its rows
       // before the first prefix token read as zero)
       if (t0 == 0 && p.P > 0)
@@ -148,6 +150,11 @@ __device__ __forceinline__ void issue_tile_loads(const Params &p, unsigned char 
   if (!full)   // state pass: the fp32 decay factors, dimensions 0..63 over X_q, 64..127 over G (unused there)
     for (int bx = 0; bx < 4; ++bx)
       tma_load_3d(sm + (bx < 2 ? R_XQ : R_G) + (bx & 1) * 16384, &p.me, bar, 32 * bx, t0, bh);
+}
+
+__device__ __forceinline__ void issue_xq_loads(const Params &p, unsigned char *sm, uint64_t *bar, int bh, int t0) {
+#pragma unroll
+  for (int r = 0; r < 2; ++r) tma_load_3d(sm + R_XQ + r * REG, &p.mq, bar, 64 * r, t0, bh);
 }
 
 // Qt for dimensions 64 h .. 64 h + 63: phi_q E gscale, bf16 pairs into TMEM.
@@ -797,8 +804,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_fwd_kernel(const __grid_consta
     if (__syncthreads_or(!ok)) { s_fail = 1; break; }
     tc_fence_after();
     if (tid == 0 && c + 1 < cend) {
-      if (centre) bulk_wait_read();   // the copy's store has read X_q's place
-      issue_tile_loads(p, sm, s_rt, &bar_tma, bh, t0 + T, full);
+      issue_tile_loads(p, sm, s_rt, &bar_tma, bh, t0 + T, full, centre);
+      if (centre) {
+        bulk_wait_read();   // the copy's store has read X_q's place
+        issue_xq_loads(p, sm, &bar_tma, bh, t0 + T);
+      }
     }
 
     // ---------------------------- epilogue (column half per group) ---

@@ -59,6 +59,7 @@ SWEEP = [
     # (a second fragment of meta columns), with and without meta values
     ("bf16", 128, 300, 100, 16, True, False, True),
     ("bf16", 128, 200, 128, 9, False, True, False),
+    ("bf16", 128, 150, 64, 2, True, True, False),
 ]
 
 
