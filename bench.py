@@ -300,6 +300,12 @@ def run_ours(args, rank, world, local):
     barrier(world)
     ms = start.elapsed_time(end) / K
     ms_max = max_over_ranks(ms, world, dev)
+    # the device status of every call so far (range, timeout): a step whose
+    # kernels gave up or left their range is not a measurement
+    for ws_ in (fws, bws):
+        st = lz.workspace_status(ws_)
+        if st != lz.OK:
+            raise RuntimeError(f"training step: device status {st} ({lz.status_string(st)})")
     # Per-kernel device times: the same steps with the library's launch events,
     # which run every kernel in order on the call's stream (the timed steps
     # above let independent backward kernels share the GPU).
