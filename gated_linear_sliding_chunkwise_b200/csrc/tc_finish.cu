@@ -59,7 +59,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
   __shared__ uint32_t s_tmem;
   // X_q, X_k, W_q | W_k (64-column tiles), dZ_q | dZ_k (64-column tiles)
   constexpr uint32_t R_XQ = 0, R_XK = TILE, R_WQ = 2 * TILE, R_WK = 2 * TILE + REG, R_ZQ = 3 * TILE,
-                     R_ZK = 3 * TILE + REG, R_STG = 4 * TILE;   // R_STG: dx_q | dx_k staging (fused mode)
+                     R_ZK = 3 * TILE + REG, R_STG = 4 * TILE;   // R_STG: dphi_q | dphi_k, then the half-terms
   // TMEM: dWq [0,64) dWk [64,128) Zq [128,192) Zk [192,256) dXq [256,384) dXk [384,512)
   constexpr uint32_t C_WQ = 0, C_WK = 64, C_ZQ = 128, C_ZK = 192, C_XQ = 256, C_XK = 384;
   const int tid = threadIdx.x, warp = tid >> 5, wg = tid >> 7, row = tid & 127;
@@ -107,7 +107,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
   bool fail = false;
   // this row's dphi values (its group's half) of one map, packed bf16.  They
   // come by TMA into R_STG (dphi_q over its first half, dphi_k over its
-  // second, from the end of the previous tile; the exchange of each map's
+  // second, issued with the previous tile's last products; the exchange of each map's
   // half-terms reuses the map's half once every row has read it), except for
   // a sequence of the exact fallback, whose fp32 values are loaded into
   // registers ahead (map 0 of the next tile at the end of this one, map 1
@@ -250,6 +250,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
         for (int s = 0; s < 8; ++s) mma_ss(tb + C_WQ, desc_mn(sbase + R_XQ, s), desc_mn(sbase + R_ZQ, s), id_dw, c > 0 || s > 0);
         for (int s = 0; s < 8; ++s) mma_ss(tb + C_WK, desc_mn(sbase + R_XK, s), desc_mn(sbase + R_ZK, s), id_dw, c > 0 || s > 0);
         mma_commit(&bar_d);
+        if (ph_tma && c + 1 < ntiles) {   // this tile's dphi and half-terms are read: the next tile's dphi
+          pend_ph = (int)((c + 1) & 1);
+          ph_loads(c + 1);
+        }
       }
       ok = mbar_wait(&bar_d, par, p.status, ST_TIMEOUT);
       if (__syncthreads_or(!ok)) { fail = true; break; }
@@ -257,24 +261,29 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
       if (tid == 0 && c + 1 < ntiles) loads(c + 1);   // X tiles consumed by the dW products
     }
     if (p.fused) {
-      // dx of this group's map, bf16, staged over R_STG and written with TMA
-      // stores (rows past L are clipped by the map)
-      unsigned char *st = sm + R_STG + wg * TILE;
-      for (int ch = 0; ch < 4; ++ch) {
-        float v[32];
-        tmem_ld32(tl + (wg == 0 ? C_XQ : C_XK) + ch * 32, v);
+      // dx, bf16, one map at a time (64 columns per group) staged over the
+      // spent dZ tiles (R_ZQ | R_ZK, one 32 KB tile) and written with TMA
+      // stores (rows past L are clipped by the map); the next tile's dphi
+      // is arriving in R_STG meanwhile
+      unsigned char *st = sm + R_ZQ;
+#pragma unroll 1
+      for (int m = 0; m < 2; ++m) {
+        for (int ch = 2 * wg; ch < 2 * wg + 2; ++ch) {
+          float v[32];
+          tmem_ld32(tl + (m == 0 ? C_XQ : C_XK) + ch * 32, v);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) *chunk_ptr(st, 0, row, 4 * ch + k) = pack8(v + 8 * k);
-      }
-      fence_proxy_async();
-      __syncthreads();
-      if (tid == 0) {
-        tma_store_3d(&p.mxq, sm + R_STG, 0, c * T, bh);
-        tma_store_3d(&p.mxq, sm + R_STG + REG, 64, c * T, bh);
-        tma_store_3d(&p.mxk, sm + R_STG + TILE, 0, c * T, bh);
-        tma_store_3d(&p.mxk, sm + R_STG + TILE + REG, 64, c * T, bh);
-        bulk_commit();
-        bulk_wait_read();
+          for (int k = 0; k < 4; ++k) *chunk_ptr(st, 0, row, 4 * ch + k) = pack8(v + 8 * k);
+        }
+        fence_proxy_async();
+        __syncthreads();
+        if (tid == 0) {
+          const CUtensorMap *mx = m == 0 ? &p.mxq : &p.mxk;
+          tma_store_3d(mx, st, 0, c * T, bh);
+          tma_store_3d(mx, st + REG, 64, c * T, bh);
+          bulk_commit();
+          bulk_wait_read();   // the staging is free once read
+        }
+        if (m == 0) __syncthreads();
       }
     }
     // dq (group 0), dk (group 1) = GLA (dz W^T) + anchor parts; dv = both
@@ -318,10 +327,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_finish_kernel(const __grid_con
     if (!ph_tma && gla && c + 1 < ntiles) dphi_load(0, c + 1);
     tc_fence_before();
     __syncthreads();
-    if (ph_tma && tid == 0 && c + 1 < ntiles) {   // R_STG is read out: the next tile's dphi
-      pend_ph = (int)((c + 1) & 1);
-      ph_loads(c + 1);
-    }
   }
   if (gla && !fail) {
     tc_fence_after();
