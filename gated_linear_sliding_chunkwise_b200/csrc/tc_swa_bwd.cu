@@ -155,7 +155,7 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
   __shared__ float s_x[MAXM][T];        // dO . mv_m per row, later the meta dS per row
   __shared__ float s_pmax[2][T], s_psum[2][T], s_dpart[2][T];
   __shared__ float s_red[4];
-  __shared__ uint64_t bars[6];
+  __shared__ uint64_t bars[7];
   __shared__ uint32_t s_tmem;
   // regions: Q, dO, K_prev, K, V_prev, V
   constexpr uint32_t R_Q = 0, R_O = TILE, R_KP = 2 * TILE, R_K = 3 * TILE, R_VP = 4 * TILE, R_V = 5 * TILE;
@@ -172,8 +172,8 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wg = tid >> 7, row = tid & 127;
   const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
   const uint32_t sbase = smem_u32(sm);
-  uint64_t *bar_tma = &bars[0], *bar_m = &bars[1];
-  setup_cta(&s_tmem, bars, 6, tid);
+  uint64_t *bar_tma = &bars[0], *bar_m = &bars[1], *bar_late = &bars[6];
+  setup_cta(&s_tmem, bars, 7, tid);
   // Persistent: CTA b walks the contiguous run [w0, w1) of (sequence, tile)
   // items, the tiles of a sequence in order; the meta tokens are staged again
   // only when the head changes, and the next item's tiles are loaded as soon
@@ -183,15 +183,19 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
   const int w1 = (int)((long long)(blockIdx.x + 1) * nwork / gridDim.x);
   // Tile loads of item w, in two parts: `early` = the regions free once the
   // dq' product has run (all but V when the GLA part arrives in V, all but
-  // Q | dO when dq is staged there), `late` = the rest, after the store.
+  // Q | dO when dq is staged there), on bar_tma; `late` = the rest, after
+  // the store, on bar_late.  With the GLA part in V, only the last product
+  // (dO V^T) waits for the late tile.
   auto tile_loads = [&](int w, bool early, bool late) {
     const int lbh = w / ntiles, lt0 = (w % ntiles) * T;
-    if (early) mbar_expect_tx(bar_tma, 6 * TILE);
+    if (early) mbar_expect_tx(bar_tma, (p.fused ? 5 : 4) * TILE);
+    if (late) mbar_expect_tx(bar_late, (p.fused ? 1 : 2) * TILE);
     const bool qo_early = p.fused != 0, v_early = p.fused == 0;
     for (int r = 0; r < 2; ++r) {
       if (qo_early ? early : late) {
-        tma_load_3d(sm + R_Q + r * kReg, &p.mq, bar_tma, 64 * r, lt0, lbh);
-        tma_load_3d(sm + R_O + r * kReg, &p.mo, bar_tma, 64 * r, lt0, lbh);
+        uint64_t *b = qo_early ? bar_tma : bar_late;
+        tma_load_3d(sm + R_Q + r * kReg, &p.mq, b, 64 * r, lt0, lbh);
+        tma_load_3d(sm + R_O + r * kReg, &p.mo, b, 64 * r, lt0, lbh);
       }
       if (early) {
         // keys and values of the previous tile; before token 0, the prefix
@@ -205,7 +209,7 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
         }
         tma_load_3d(sm + R_K + r * kReg, &p.mk, bar_tma, 64 * r, lt0, lbh);
       }
-      if (v_early ? early : late) tma_load_3d(sm + R_V + r * kReg, &p.mv, bar_tma, 64 * r, lt0, lbh);
+      if (v_early ? early : late) tma_load_3d(sm + R_V + r * kReg, &p.mv, v_early ? bar_tma : bar_late, 64 * r, lt0, lbh);
     }
   };
   if (tid == 0 && w0 < w1) tile_loads(w0, true, true);
@@ -243,16 +247,21 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
     __syncthreads();
   }
   ok = mbar_wait(bar_tma, par, p.status, ST_TIMEOUT);
+  if (!p.fused) ok = ok && mbar_wait(bar_late, par, p.status, ST_TIMEOUT);   // Q and dO come late
   if (__syncthreads_or(!ok)) goto done;
 
-  // 1. logits L = Q [K_prev ; K]^T and dP' = dO [V_prev ; V]^T
+  // 1. logits L = Q [K_prev ; K]^T and dP' = dO [V_prev ; V]^T (with the GLA
+  //    part in V, dO V^T once V has arrived, after the meta dot products)
+  bool v_ok = true;
   if (tid == 0) {
     tc_fence_after();
     for (int s = 0; s < 8; ++s) mma_ss(tb + C_L, desc_k(sbase + R_Q, s), desc_k(sbase + R_KP, s), id_kk, s > 0);
     for (int s = 0; s < 8; ++s) mma_ss(tb + C_L + 128, desc_k(sbase + R_Q, s), desc_k(sbase + R_K, s), id_kk, s > 0);
     for (int s = 0; s < 8; ++s) mma_ss(tb + C_DP, desc_k(sbase + R_O, s), desc_k(sbase + R_VP, s), id_kk, s > 0);
-    for (int s = 0; s < 8; ++s) mma_ss(tb + C_DP + 128, desc_k(sbase + R_O, s), desc_k(sbase + R_V, s), id_kk, s > 0);
-    mma_commit(bar_m);
+    if (!p.fused) {
+      for (int s = 0; s < 8; ++s) mma_ss(tb + C_DP + 128, desc_k(sbase + R_O, s), desc_k(sbase + R_V, s), id_kk, s > 0);
+      mma_commit(bar_m);
+    }
   }
   {
     const float lse_row = (p.lse_in && qvalid) ? p.lse_in[(size_t)bh * p.L + tq] : 0.f;
@@ -269,7 +278,14 @@ __global__ void __launch_bounds__(NT_Q, 1) tc_swa_bwd_q_kernel(const __grid_cons
         for (int m = 0; m < MAXM; ++m)
           if (m < p.M) s_x[m][row] = ml[m];
     }
-    ok = mbar_wait(bar_m, par, p.status, ST_TIMEOUT);
+    if (p.fused && tid == 0) {
+      v_ok = mbar_wait(bar_late, par, p.status, ST_TIMEOUT);
+      tc_fence_after();
+      if (v_ok)
+        for (int s = 0; s < 8; ++s) mma_ss(tb + C_DP + 128, desc_k(sbase + R_O, s), desc_k(sbase + R_V, s), id_kk, s > 0);
+      mma_commit(bar_m);   // also when V never came: the products issued above complete
+    }
+    ok = mbar_wait(bar_m, par, p.status, ST_TIMEOUT) && v_ok;
     if (__syncthreads_or(!ok)) goto done;
     tc_fence_after();
     if (p.fused && tid == 0) {   // the GLA part of dq into the V region (only dP' read V)
