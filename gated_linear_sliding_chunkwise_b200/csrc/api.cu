@@ -362,6 +362,20 @@ lizard_status Plan::run(cudaStream_t s, void *const *events, int nev) const {
   return LIZARD_OK;
 }
 
+// Once per device, before the first kernel of a call: the GLA tile kernel's
+// code goes in first (its placement then does not depend on the kernels that
+// run before it).  False when the runtime refuses.
+bool preload_once() {
+  constexpr int kDev = 64;
+  static bool done[kDev] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (dev < 0 || dev >= kDev || done[dev]) return true;
+  if (lz::tc_gla_bwd_preload() != cudaSuccess) return false;
+  done[dev] = true;
+  return true;
+}
+
 // `target`, `dmse`, `loss`: the stage-1 loss, which the tensor-core forward
 // forms in its epilogue (null otherwise).
 void fwd_plan(const lizard_fwd_args *a, void *ws, cudaStream_t s, Plan &plan, const void *target = nullptr,
@@ -674,6 +688,7 @@ lizard_status lizard_attn_fwd(const lizard_fwd_args *a, lizard_stream_t stream) 
   // a training forward's wide-decay marks start cleared
   if (keep && cudaMemsetAsync(at<void>(a->saved, sv.flags), 0, (size_t)BH * sizeof(uint32_t), s) != cudaSuccess)
     return LIZARD_ERR_CUDA;
+  if (!preload_once()) return LIZARD_ERR_CUDA;
   Plan plan;
   fwd_plan(a, a->workspace, s, plan);
   return plan.run(s, a->launch_events, a->n_launch_events);
@@ -768,6 +783,7 @@ lizard_status lizard_attn_bwd(const lizard_bwd_args *b, lizard_stream_t stream) 
   if (a->L == 0) return LIZARD_OK;
   void *ws = b->workspace;
   if (cudaMemsetAsync(ws, 0, cleared_bytes(a, lay.fallback), s) != cudaSuccess) return LIZARD_ERR_CUDA;
+  if (!preload_once()) return LIZARD_ERR_CUDA;
   Plan plan;
   bwd_plan(b, ws, s, plan);
   return plan.run(s, b->launch_events, b->n_launch_events);
@@ -905,6 +921,7 @@ lizard_status lizard_stage1_step(const lizard_stage1_args *a, lizard_stream_t st
   void *ws = b->workspace;
   if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), s) != cudaSuccess) return LIZARD_ERR_CUDA;
   S1Views views;
+  if (!preload_once()) return LIZARD_ERR_CUDA;
   Plan plan;
   stage1_plan(a, views, ws, s, plan);
   return plan.run(s, b->launch_events, b->n_launch_events);

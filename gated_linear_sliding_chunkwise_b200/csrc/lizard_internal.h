@@ -293,6 +293,8 @@ cudaError_t launch_slot_dg(float *dg, const float *da, const void *g, const int 
                            float inv_tau, bool scalar_gate, bool bf16, cudaStream_t s);
 // stage 0: reverse dS pass, 1: per-tile gradients, 2: gate-logit gradient
 cudaError_t launch_tc_gla_bwd(const TcGlaBwdArgs &a, int stage, cudaStream_t s);
+// Loads the GLA tile kernel before the library's other kernels (see tc_gla_bwd.cu).
+cudaError_t tc_gla_bwd_preload();
 // tensor-core finish: bf16, d = 128, both feature maps present
 cudaError_t launch_tc_finish(const FinishBwdArgs &a, int BH, cudaStream_t s);
 cudaError_t launch_finish_bwd(const FinishBwdArgs &a, int BH, int D, bool bf16, cudaStream_t s);

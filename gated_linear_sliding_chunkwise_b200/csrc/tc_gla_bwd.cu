@@ -909,6 +909,14 @@ static const float *snapshot_row0(const void *snap, int BH, int L) {
                                          (size_t)BH * ((L + T - 1) / T) * D * D);
 }
 
+// The GLA tile kernel's speed depends on where the driver places its code,
+// which follows the order in which kernels are first touched: setting its
+// attribute before any other kernel of the library is used puts it first,
+// whatever the sizes of the kernels that run before it.
+cudaError_t tc_gla_bwd_preload() {
+  return cudaFuncSetAttribute(tc_gla_bwd_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TILE_SMEM);
+}
+
 cudaError_t launch_tc_gla_bwd(const TcGlaBwdArgs &a, int stage, cudaStream_t s) {
   const int ntiles = (a.L + T - 1) / T;
   const uint64_t rows = (uint64_t)a.L;
