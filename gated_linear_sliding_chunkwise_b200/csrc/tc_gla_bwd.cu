@@ -138,21 +138,35 @@ __global__ void __launch_bounds__(NT_DS, 1) tc_gla_dstates_kernel(const __grid_c
   }
   const uint32_t id_z = idesc_bf16(128, 64, 0, 1);
   const uint32_t id_st = idesc_bf16(128, 128, 1, 1);
-  auto loads = [&](int c) {
-    mbar_expect_tx(&bar_tma, 4 * TILE + D * 4);
-    bulk_load_1d(s_rt, p.gate_r + ((size_t)bh * ntiles + c) * D, D * 4, &bar_tma);
-    for (int r = 0; r < 2; ++r) {
-      tma_load_3d(sm + R_XQ + r * REG, &p.mq, &bar_tma, 64 * r, c * T, bh);
-      tma_load_3d(sm + R_O + r * REG, &p.mo, &bar_tma, 64 * r, c * T, bh);
+  // Tile c's loads in two parts: E and r (their places are free once Qt is
+  // formed, so they go out before the dS product), then X_q and dO (free
+  // once the product is done).  The barrier expects all of them at once.
+  auto loads = [&](int c, bool e_r, bool xq_o) {
+    if (e_r) {
+      mbar_expect_tx(&bar_tma, 4 * TILE + D * 4);
+      bulk_load_1d(s_rt, p.gate_r + ((size_t)bh * ntiles + c) * D, D * 4, &bar_tma);
+      for (int bx = 0; bx < 4; ++bx) tma_load_3d(sm + R_E + bx * 16384, &p.me, &bar_tma, 32 * bx, c * T, bh);
     }
-    for (int bx = 0; bx < 4; ++bx) tma_load_3d(sm + R_E + bx * 16384, &p.me, &bar_tma, 32 * bx, c * T, bh);
+    if (xq_o)
+      for (int r = 0; r < 2; ++r) {
+        tma_load_3d(sm + R_XQ + r * REG, &p.mq, &bar_tma, 64 * r, c * T, bh);
+        tma_load_3d(sm + R_O + r * REG, &p.mo, &bar_tma, 64 * r, c * T, bh);
+      }
   };
-  if (tid == 0 && ntiles > 0) loads(ntiles - 1);
+  // thread 0: parity and tile of a load batch issued and not yet waited for
+  // (pend -1: none), and whether its X_q / dO half is still to be issued
+  int pend = -1, pend_c = 0;
+  bool half = false;
+  if (tid == 0 && ntiles > 0) {
+    loads(ntiles - 1, true, true);
+    pend = 0;
+  }
   bool fail = false;
   for (int c = ntiles - 1; c >= 0; --c) {
     const uint32_t par = (ntiles - 1 - c) & 1;
     bool ok = mbar_wait(&bar_tma, par, p.status, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) { fail = true; break; }
+    pend = -1;
     if (tid == 0) {
       tc_fence_after();
       for (int s = 0; s < 8; ++s) mma_ss(tb + C_Z, desc_k(sbase + R_XQ, s), desc_mn(sbase + R_W, s), id_z, s > 0);
@@ -219,11 +233,20 @@ __global__ void __launch_bounds__(NT_DS, 1) tc_gla_dstates_kernel(const __grid_c
       for (int s = 0; s < 8; ++s) mma_ss(tb + C_S, desc_mn(sbase + R_XQ, s), desc_mn(sbase + R_O, s), id_st, 1);
       for (int s = 0; s < 8; ++s) mma_ss(tb + C_S, desc_mn(sbase + R_QL, s), desc_mn(sbase + R_O, s), id_st, 1);
       mma_commit(&bar_m2);
+      if (c > 0) {   // E and r were read before the barrier above
+        loads(c - 1, true, false);
+        pend = (int)(par ^ 1u);
+        pend_c = c - 1;
+        half = true;
+      }
     }
     ok = mbar_wait(&bar_m2, par, p.status, ST_TIMEOUT);
     if (__syncthreads_or(!ok)) { fail = true; break; }
     tc_fence_after();
-    if (tid == 0 && c > 0) loads(c - 1);
+    if (tid == 0 && c > 0) {
+      loads(c - 1, false, true);
+      half = false;
+    }
     {   // dS_prev = diag(exp r) (dS + Qt^T dO), column half per group
       const float dec = s_dec[row];
       for (int ch = 4 * wg; ch < 4 * wg + 4; ++ch) {
@@ -241,6 +264,12 @@ __global__ void __launch_bounds__(NT_DS, 1) tc_gla_dstates_kernel(const __grid_c
     }
     tc_fence_before();
     __syncthreads();
+  }
+  if (fail && tid == 0 && pend >= 0) {
+    // let the loads already issued land before the shared memory is released
+    // (a half-issued batch is completed first, so the barrier's wait can end)
+    if (half) loads(pend_c, false, true);
+    mbar_wait(&bar_tma, (uint32_t)pend, nullptr, 0, 1u << 16);
   }
   if (!fail && p.dstate_in) {
     tc_fence_after();
